@@ -1,0 +1,250 @@
+"""Python face of the float64 CPU oracle (test infrastructure only).
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
+leg may import this module. It loads ``liboracle.so`` built from
+``gs_oracle.cpp`` (see ``build.py``) and adds the two steps whose definitions
+are one line each -- the view-space gradient statistics and Adam -- written in
+numpy float64.
+
+Every array crossing this interface is float64 (inputs are the float32 scene
+arrays widened exactly), except the float32 depth keys and the int32 flags.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+from . import build as _build
+
+_LIB = None
+
+_D = ctypes.POINTER(ctypes.c_double)
+_F = ctypes.POINTER(ctypes.c_float)
+_I32 = ctypes.POINTER(ctypes.c_int32)
+_I64 = ctypes.POINTER(ctypes.c_int64)
+_U64 = ctypes.POINTER(ctypes.c_uint64)
+
+
+def lib():
+    """Load (building first if needed) the oracle shared library."""
+    global _LIB
+    if _LIB is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        L.orc_sh_basis.argtypes = [ctypes.c_int64, _D, ctypes.c_int, _D]
+        L.orc_project.argtypes = [ctypes.c_int64, _D, _D, _D, _D, _D, ctypes.c_int, _D,
+                                  ctypes.c_double, _D, _I32, _F]
+        L.orc_tile_lists.argtypes = [ctypes.c_int, ctypes.c_int64, _I32, _F, _I32, _I32,
+                                     ctypes.c_int64, _I32, _I64, _I32]
+        L.orc_render.argtypes = [ctypes.c_int, ctypes.c_int64, _D, _F, _I32, _I32, ctypes.c_int64,
+                                 _I32, _D, ctypes.c_double, ctypes.c_double, _D, _D, _I32, _I32,
+                                 _I64, _I32, _U64]
+        L.orc_render_bwd.argtypes = [ctypes.c_int, ctypes.c_int64, _D, _F, _I32, _I32,
+                                     ctypes.c_int64, _I32, _D, _D, _D]
+        L.orc_project_bwd.argtypes = [ctypes.c_int64, _D, _D, _D, _D, _D, ctypes.c_int,
+                                      ctypes.c_int, _D, _I32, _D, _D, _D, _D, _D, _D]
+        L.orc_num_threads.restype = ctypes.c_int
+        _LIB = L
+    return _LIB
+
+
+def num_threads() -> int:
+    return int(lib().orc_num_threads())
+
+
+def _p(a: np.ndarray, t):
+    return a.ctypes.data_as(t)
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def pack_camera(cam) -> np.ndarray:
+    """22 doubles: viewmat (3x4 row-major), fx, fy, cx, cy, W, H, campos, 0."""
+    c = cam if isinstance(cam, dict) else cam.as_dict()
+    out = np.zeros(22, np.float64)
+    out[:12] = np.asarray(c["viewmat"], np.float32).astype(np.float64).reshape(12)
+    out[12:16] = [np.float32(c["fx"]), np.float32(c["fy"]), np.float32(c["cx"]), np.float32(c["cy"])]
+    out[16:18] = [c["width"], c["height"]]
+    out[18:21] = np.asarray(c["campos"], np.float32).astype(np.float64)
+    return out
+
+
+def sh_basis(dirs: np.ndarray, deg: int) -> np.ndarray:
+    """Real SH basis [n, 16] (Legendre recursion) for unit directions [n, 3]."""
+    d = _f64(dirs)
+    n = d.shape[0]
+    out = np.zeros((n, 16), np.float64)
+    lib().orc_sh_basis(n, _p(d, _D), int(deg), _p(out, _D))
+    return out
+
+
+def _raw(scene):
+    n = scene.n
+    k = (scene.sh_degree + 1) ** 2
+    return (_f64(scene.means[:, :3]), _f64(scene.log_scales[:, :3]), _f64(scene.quats),
+            _f64(scene.opacity_logit), _f64(scene.sh.reshape(n, k, 3)))
+
+
+def project(scene, cam, tol: float = 1e-9) -> Dict[str, np.ndarray]:
+    """Project every Gaussian of ``scene`` into ``cam`` (float64)."""
+    m, s, q, lg, sh = _raw(scene)
+    n = scene.n
+    geom = np.zeros((n, 16), np.float64)
+    ints = np.zeros((n, 8), np.int32)
+    key = np.zeros(n, np.float32)
+    lib().orc_project(n, _p(m, _D), _p(s, _D), _p(q, _D), _p(lg, _D), _p(sh, _D),
+                      int(scene.sh_degree), _p(pack_camera(cam), _D), float(tol),
+                      _p(geom, _D), _p(ints, _I32), _p(key, _F))
+    return dict(
+        xy=geom[:, 0:2].copy(), depth=geom[:, 2].copy(), cov=geom[:, 3:6].copy(),
+        conic=geom[:, 6:9].copy(), opacity=geom[:, 9].copy(), rgb=geom[:, 10:13].copy(),
+        lam=geom[:, 13].copy(), radius_arg=geom[:, 14].copy(),
+        valid=ints[:, 0].copy(), radius=ints[:, 1].copy(), rect=ints[:, 2:6].copy(),
+        clamp=ints[:, 6].copy(), ambiguous=ints[:, 7].copy(), key=key)
+
+
+def project_views(scene, tol: float = 1e-9) -> List[Dict[str, np.ndarray]]:
+    return [project(scene, c, tol) for c in scene.cameras]
+
+
+def _stack_views(projs: Sequence[dict]):
+    g2d = np.ascontiguousarray(np.stack([np.concatenate(
+        [p["xy"], p["conic"], p["opacity"][:, None], p["rgb"]], axis=1) for p in projs]))
+    keys = np.ascontiguousarray(np.stack([p["key"] for p in projs]).astype(np.float32))
+    rects = np.ascontiguousarray(np.stack([p["rect"] for p in projs]).astype(np.int32))
+    return g2d, keys, rects
+
+
+def _dims(cams) -> np.ndarray:
+    out = []
+    for c in cams:
+        c = c if isinstance(c, dict) else c.as_dict()
+        out.append([c["width"], c["height"]])
+    return np.ascontiguousarray(np.asarray(out, np.int32))
+
+
+def tile_lists(rects: np.ndarray, keys: np.ndarray, tiles_xy: Sequence, requests: np.ndarray):
+    """Sorted Gaussian ids of the requested (view, tile) pairs.
+
+    ``rects`` int32 [V, n, 4]; ``keys`` float32 [V, n]; ``tiles_xy`` [(tx, ty)]
+    per view; ``requests`` int32 [R, 2]. Returns (counts [R], ids concatenated).
+    """
+    rects = np.ascontiguousarray(rects, np.int32)
+    keys = np.ascontiguousarray(keys, np.float32)
+    V, n = keys.shape
+    tx = np.ascontiguousarray([t[0] for t in tiles_xy], np.int32)
+    ty = np.ascontiguousarray([t[1] for t in tiles_xy], np.int32)
+    req = np.ascontiguousarray(requests, np.int32)
+    R = req.shape[0]
+    counts = np.zeros(R, np.int64)
+    lib().orc_tile_lists(V, n, _p(rects, _I32), _p(keys, _F), _p(tx, _I32), _p(ty, _I32), R,
+                         _p(req, _I32), _p(counts, _I64), None)
+    ids = np.zeros(max(int(counts.sum()), 1), np.int32)
+    lib().orc_tile_lists(V, n, _p(rects, _I32), _p(keys, _F), _p(tx, _I32), _p(ty, _I32), R,
+                         _p(req, _I32), _p(counts, _I64), _p(ids, _I32))
+    return counts, ids[: int(counts.sum())]
+
+
+def render(projs: Sequence[dict], cams, bg, pixels: np.ndarray,
+           win_alpha: float = 0.0, win_T: float = 0.0) -> Dict[str, np.ndarray]:
+    """Render the listed pixels ``[(view, x, y)]`` from projected Gaussians."""
+    g2d, keys, rects = _stack_views(projs)
+    V, n = keys.shape
+    pix = np.ascontiguousarray(pixels, np.int32).reshape(-1, 3)
+    P = pix.shape[0]
+    color = np.zeros((P, 3)); T = np.zeros(P); nc = np.zeros(P, np.int32)
+    flags = np.zeros(P, np.int32); nexp = np.zeros(P, np.int64); used = np.zeros(P, np.int32)
+    sig = np.zeros(P, np.uint64)
+    bgd = _f64(bg)
+    lib().orc_render(V, n, _p(g2d, _D), _p(keys, _F), _p(rects, _I32), _p(_dims(cams), _I32),
+                     P, _p(pix, _I32), _p(bgd, _D), float(win_alpha), float(win_T),
+                     _p(color, _D), _p(T, _D), _p(nc, _I32), _p(flags, _I32), _p(nexp, _I64),
+                     _p(used, _I32), _p(sig, _U64))
+    return dict(color=color, T=T, n_contrib=nc, flags=flags, n_exp=nexp, n_used=used, sig=sig)
+
+
+def render_bwd(projs: Sequence[dict], cams, bg, pixels: np.ndarray, dL_dC: np.ndarray) -> np.ndarray:
+    """Screen-space gradients [V, n, 10] for the listed pixels and upstream dL/dC [P, 3]."""
+    g2d, keys, rects = _stack_views(projs)
+    V, n = keys.shape
+    pix = np.ascontiguousarray(pixels, np.int32).reshape(-1, 3)
+    P = pix.shape[0]
+    gC = _f64(dL_dC).reshape(P, 3)
+    out = np.zeros((V, n, 10), np.float64)
+    lib().orc_render_bwd(V, n, _p(g2d, _D), _p(keys, _F), _p(rects, _I32), _p(_dims(cams), _I32),
+                         P, _p(pix, _I32), _p(_f64(bg), _D), _p(gC, _D), _p(out, _D))
+    return out
+
+
+def project_bwd(scene, projs: Sequence[dict], grad2d: np.ndarray) -> Dict[str, np.ndarray]:
+    """Gradients of the raw parameters from screen-space gradients [V, n, 10]."""
+    m, s, q, lg, sh = _raw(scene)
+    n = scene.n
+    V = len(scene.cameras)
+    K = (scene.sh_degree + 1) ** 2
+    cams = np.ascontiguousarray(np.stack([pack_camera(c) for c in scene.cameras]))
+    valid = np.ascontiguousarray(np.stack([p["valid"] for p in projs]).astype(np.int32))
+    g = _f64(grad2d)
+    gm = np.zeros((n, 3)); gs = np.zeros((n, 3)); gq = np.zeros((n, 4)); gl = np.zeros(n)
+    gsh = np.zeros((n, K, 3))
+    lib().orc_project_bwd(n, _p(m, _D), _p(s, _D), _p(q, _D), _p(lg, _D), _p(sh, _D),
+                          int(scene.sh_degree), V, _p(cams, _D), _p(valid, _I32), _p(g, _D),
+                          _p(gm, _D), _p(gs, _D), _p(gq, _D), _p(gl, _D), _p(gsh, _D))
+    return dict(means=gm, log_scales=gs, quats=gq, opacity_logit=gl, sh=gsh)
+
+
+def densify_stats(grad2d: np.ndarray, valid: np.ndarray, accum_plain=None, accum_abs=None,
+                  denom=None):
+    """View-space gradient statistics for densification, summed over views.
+
+    Per view v and visible Gaussian i (the "plain" and "absolute" gradients of
+    the absolute-gradient densification page, sec. 2 table):
+      plain_i += || sum_p g_{i,p} ||_2   (the view's dL/dmean2D)
+      abs_i   += sum_p || g_{i,p} ||_2
+      denom_i += 1
+    """
+    g = np.asarray(grad2d, np.float64)
+    vis = np.asarray(valid) != 0
+    n = g.shape[1]
+    plain = np.zeros(n) if accum_plain is None else np.array(accum_plain, np.float64)
+    absg = np.zeros(n) if accum_abs is None else np.array(accum_abs, np.float64)
+    den = np.zeros(n, np.int64) if denom is None else np.array(denom, np.int64)
+    for v in range(g.shape[0]):
+        plain += np.where(vis[v], np.hypot(g[v, :, 0], g[v, :, 1]), 0.0)
+        absg += np.where(vis[v], g[v, :, 9], 0.0)
+        den += vis[v].astype(np.int64)
+    return plain, absg, den
+
+
+def adam(param, grad, m, v, lr: float, step: int, beta1=0.9, beta2=0.999, eps=1e-15):
+    """One Adam step (Kingma and Ba, with bias correction), float64.
+
+    m <- b1 m + (1-b1) g;  v <- b2 v + (1-b2) g^2;
+    p <- p - lr * (m / (1-b1^t)) / (sqrt(v / (1-b2^t)) + eps).
+    """
+    p = np.array(param, np.float64)
+    g = np.asarray(grad, np.float64)
+    m = beta1 * np.asarray(m, np.float64) + (1.0 - beta1) * g
+    v = beta2 * np.asarray(v, np.float64) + (1.0 - beta2) * g * g
+    mhat = m / (1.0 - beta1 ** step)
+    vhat = v / (1.0 - beta2 ** step)
+    p = p - lr * mhat / (np.sqrt(vhat) + eps)
+    return p, m, v
+
+
+def render_all(scene, projs=None, bg=None, tol_alpha=0.0, tol_T=0.0):
+    """Full-image forward render of every view; returns [V,3,H,W] colour etc."""
+    projs = project_views(scene) if projs is None else projs
+    outs = []
+    for v, c in enumerate(scene.cameras):
+        ys, xs = np.meshgrid(np.arange(c.height), np.arange(c.width), indexing="ij")
+        pix = np.stack([np.full(xs.size, v), xs.ravel(), ys.ravel()], axis=1)
+        outs.append((pix, render(projs, scene.cameras, scene.background if bg is None else bg,
+                                 pix, tol_alpha, tol_T)))
+    return outs
