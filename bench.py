@@ -1,0 +1,456 @@
+#!/usr/bin/env python
+"""Benchmark of the differentiable EWA splatting training step on B200.
+
+One step = gs_project -> gs_bin_sort -> gs_rasterize_fwd -> gs_rasterize_bwd
+(screen space) -> gs_project_bwd -> gs_densify_stats -> gs_adam_step, on the
+1,000,000-Gaussian SH3 scene at 1920x1080 (fx = fy = 1200) with an upstream
+image gradient N(0, 1e-2), synthetic and seeded. The metric is the step time
+and its pixel throughput (Mpix/s = rendered pixels / step time).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs one process per GPU under torch.distributed (NCCL): each rank
+renders its own view of the same Gaussians (views on an orbit of radius 8),
+the parameter gradients are summed across ranks with one all-reduce, and every
+rank applies the same Adam step (weak scaling: one view per GPU).
+
+Rank 0 prints one JSON line. ``--impl reference`` times the float64 CPU
+oracle on the host cores on a bounded sample of the same workload instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "train_1m_1080p"
+METRIC = "fwd+bwd train-step ms & Mpix/s at 1M Gaussians 1080p; % of roofline"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--sort-mode", default="presort", choices=["presort", "full64"])
+    ap.add_argument("--n", type=int, default=None, help="override the Gaussian count")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- helpers
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), sm_max_mhz=float(d.get("sm_max_mhz", 1965.0)),
+                    source="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, sm_max_mhz=1965.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["nvidia-smi unavailable"])
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(name)
+        os.unlink(self.path)
+        return dict(sm_mhz=statistics.median(sm) if sm else None,
+                    sm_max_mhz=max(smax) if smax else None, reasons=sorted(reasons),
+                    samples=len(sm))
+
+
+def orbit_camera(scene, k: int, count: int):
+    from gaussian_splatting_differentiable_ewa_b200 import scenes as S
+    c0 = scene.cameras[0]
+    a = 2.0 * math.pi * k / count
+    centre = (8.0 * math.sin(a), 0.0, -8.0 * math.cos(a))
+    return S.Camera(viewmat=S.look_at(centre).astype(np.float32), fx=c0.fx, fy=c0.fy, cx=c0.cx,
+                    cy=c0.cy, width=c0.width, height=c0.height,
+                    campos=np.asarray(centre, np.float32))
+
+
+# ----------------------------------------------------------------- work model
+
+def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float) -> dict:
+    """Algorithmic bytes (and exp evaluations) per launch of each call.
+
+    Bytes count the data the definition has to move once: parameters read,
+    outputs written, 59 real floats per Gaussian (pad lanes excluded)."""
+    n, V = sp.n, sp.V
+    P = V * sp.W * sp.H
+    rec = 48
+    p59 = 59 * 4
+    if sort_mode == "full64":
+        passes = 6 if V * ((sp.W + 15) // 16) * ((sp.H + 15) // 16) > 256 else 5
+        sort_bytes = n_pairs * (12 + passes * 24 + 8) + V * n * 16
+    else:
+        sort_bytes = n_pairs * (8 + 2 * 16 + 4) + V * n * (16 + 4 * 24 + 12)
+    return {
+        "gs_project": dict(bytes=V * n * (p59 + rec + 4), exps=0.0),
+        "gs_bin_sort": dict(bytes=sort_bytes, exps=0.0),
+        "gs_rasterize_fwd": dict(bytes=n_pairs * (4 + rec) + P * 20, exps=exps),
+        "gs_rasterize_bwd": dict(bytes=n_pairs * (4 + rec) + P * 20 + V * n * 48 * 2, exps=exps),
+        "gs_project_bwd": dict(bytes=V * n * (p59 + 48 + 4) + n * p59, exps=0.0),
+        "gs_densify_stats": dict(bytes=V * n * (12 + 4) + n * 24, exps=0.0),
+        "gs_adam_step": dict(bytes=n * 59 * 28, exps=0.0),
+    }
+
+
+def sfu_peak_gexps(sm_mhz: float, sms: int = 148) -> float:
+    # MUFU.EX2: 16 results per SM per clock (4 per SM sub-partition)
+    return sms * 16 * sm_mhz * 1e6 / 1e9
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def cpu_baseline(scene, sample_pixels: int = 4096, seed: int = 5):
+    """Time the float64 oracle as it stands on host cores over a bounded
+    sample and extrapolate to one full step. Returns (dict, n_exp_mean)."""
+    from oracle import oracle as O
+    from gaussian_splatting_differentiable_ewa_b200 import scenes as S
+    c = scene.cameras[0]
+    rng = np.random.default_rng(seed)
+    pix = np.stack([np.zeros(sample_pixels, np.int64), rng.integers(0, c.width, sample_pixels),
+                    rng.integers(0, c.height, sample_pixels)], 1).astype(np.int32)
+    t0 = time.perf_counter()
+    projs = O.project_views(scene)
+    t1 = time.perf_counter()
+    ref = O.render(projs, scene.cameras, scene.background, pix)
+    t2 = time.perf_counter()
+    dL = S.make_upstream_grad(1, c.height, c.width, seed=1)
+    gC = dL[0][:, pix[:, 2], pix[:, 1]].T
+    g2 = O.render_bwd(projs, scene.cameras, scene.background, pix, gC)
+    t3 = time.perf_counter()
+    # the projection backward over every Gaussian (as in a full step)
+    g2_full = g2.copy()
+    g2_full[..., :9] += 1e-3
+    O.project_bwd(scene, projs, g2_full)
+    t4 = time.perf_counter()
+    n = scene.n
+    p = np.zeros(59 * n)
+    O.adam(p, p + 1e-3, p, p, 1e-3, 1)
+    t5 = time.perf_counter()
+    P = c.width * c.height
+    scale = P / sample_pixels
+    step_s = (t1 - t0) + (t2 - t1 + t3 - t2) * scale + (t4 - t3) + (t5 - t4)
+    out = dict(value=P / step_s / 1e6, unit="Mpix/s", cores=O.num_threads(), kind="oracle",
+               sample=("float64 oracle: projection, projection backward and Adam over all %d "
+                       "Gaussians; render + render backward on %d random pixels, extrapolated "
+                       "linearly to %d pixels" % (n, sample_pixels, P)),
+               step_s=step_s, measured_s=t5 - t0)
+    return out, float(ref["n_exp"].mean())
+
+
+def run_reference(args):
+    """--impl reference: the oracle timed on the host, rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from oracle import oracle as O
+    from gaussian_splatting_differentiable_ewa_b200 import scenes as S
+    scene = S.make_scene(WORKLOAD, n=args.n)
+    c = scene.cameras[0]
+    P = c.width * c.height
+    n = scene.n
+    sub = max(1, n // 16)
+    small = S.make_scene(WORKLOAD, n=sub)
+    projs_full = O.project_views(scene)
+    rng = np.random.default_rng(7)
+    dL = S.make_upstream_grad(1, c.height, c.width, seed=1)
+    n_pix = 512
+    times = []
+    for it in range(args.warmup + args.steps):
+        pix = np.stack([np.zeros(n_pix, np.int64), rng.integers(0, c.width, n_pix),
+                        rng.integers(0, c.height, n_pix)], 1).astype(np.int32)
+        gC = dL[0][:, pix[:, 2], pix[:, 1]].T
+        t0 = time.perf_counter()
+        pr = O.project_views(small)
+        t1 = time.perf_counter()
+        O.render(projs_full, scene.cameras, scene.background, pix)
+        g2 = O.render_bwd(projs_full, scene.cameras, scene.background, pix, gC)
+        t2 = time.perf_counter()
+        g2s = np.full((1, sub, 10), 1e-3)
+        O.project_bwd(small, pr, g2s)
+        p = np.zeros(59 * sub)
+        O.adam(p, p + 1e-3, p, p, 1e-3, 1)
+        t3 = time.perf_counter()
+        step = (t1 - t0) * n / sub + (t2 - t1) * P / n_pix + (t3 - t2) * n / sub
+        if it >= args.warmup:
+            times.append(step)
+    ms = 1000.0 * float(np.mean(times))
+    value = P / (ms / 1000.0) / 1e6
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "Mpix/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "gaussians": n, "width": c.width, "height": c.height,
+                   "sh_degree": 3, "views_per_gpu": 1},
+        "cpu_baseline": {"value": value, "unit": "Mpix/s", "cores": O.num_threads(),
+                         "kind": "oracle",
+                         "sample": "per step: projection, projection backward and Adam on "
+                                   "%d of %d Gaussians, render + backward on %d random pixels; "
+                                   "each part extrapolated linearly to the full step"
+                                   % (sub, n, n_pix)},
+        "e2e": {"value": value, "unit": "Mpix/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- our path
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from gaussian_splatting_differentiable_ewa_b200 import api
+    from gaussian_splatting_differentiable_ewa_b200 import scenes as S
+    from gaussian_splatting_differentiable_ewa_b200.pipeline import Splatter
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    mode = api.GS_SORT_PRESORT if args.sort_mode == "presort" else api.GS_SORT_FULL64
+
+    scene = S.make_scene(WORKLOAD, n=args.n)
+    if world > 1:
+        scene.cameras = [orbit_camera(scene, rank, world)]
+    c = scene.cameras[0]
+    sp = Splatter(scene, sort_mode=mode)
+    need = sp.ensure_capacity()
+    dL_host = S.make_upstream_grad(1, c.height, c.width, seed=1)
+    dL = torch.as_tensor(dL_host).cuda()
+    stream = torch.cuda.current_stream()
+    pixels = c.width * c.height
+
+    def step(events=None):
+        def mark(k):
+            if events is not None:
+                events[k].record(stream)
+        mark(0)
+        sp.project()
+        mark(1)
+        sp.bin_sort()
+        mark(2)
+        sp.rasterize_fwd()
+        mark(3)
+        sp.rasterize_bwd(dL, with_params=False)
+        mark(4)
+        sp.project_bwd()
+        mark(5)
+        if world > 1:
+            dist.all_reduce(sp.grad_flat)
+        mark(6)
+        sp.densify_stats()
+        mark(7)
+        sp.adam_step()
+        mark(8)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    assert sp.status() == api.GS_OK, "device status after warm-up"
+
+    names = ["gs_project", "gs_bin_sort", "gs_rasterize_fwd", "gs_rasterize_bwd",
+             "gs_project_bwd", "all_reduce", "gs_densify_stats", "gs_adam_step"]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for k in range(args.steps):
+        step(ev[k])
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = start.elapsed_time(end)
+    per_call = {nm: float(np.mean([ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(args.steps)]))
+                for i, nm in enumerate(names)}
+    if world > 1:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms = elapsed_ms / args.steps
+    value = world * pixels / (ms / 1000.0) / 1e6
+    n_pairs = int(sp.n_pairs.item())
+    status = sp.status()
+
+    # end to end through the C calls from host buffers: the upstream gradient
+    # goes host -> device and the rendered image device -> host every step
+    e2e = None
+    if not args.no_e2e:
+        h_in = torch.from_numpy(dL_host).pin_memory()
+        h_out = torch.empty(sp.image.shape, dtype=torch.float32).pin_memory()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            dL.copy_(h_in, non_blocking=True)
+            step()
+            h_out.copy_(sp.image, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1) / args.steps
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * pixels / (e_ms / 1000.0) / 1e6, "unit": "Mpix/s",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": int(h_in.numel() * 4),
+               "d2h_bytes_per_step": int(h_out.numel() * 4)}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    # CPU baseline and the exp count of the blend kernels (oracle, rank 0, N=1)
+    cpu = None
+    exps = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu, nexp_mean = cpu_baseline(scene)
+        exps = nexp_mean * pixels
+    pk = peaks()
+    work = algorithmic_work(sp, n_pairs, args.sort_mode, exps or 0.0)
+    kernels = {}
+    for nm in names:
+        if nm not in work:
+            continue
+        t = per_call[nm] / 1000.0
+        w = work[nm]
+        kernels[nm] = dict(ms=per_call[nm], gbs=w["bytes"] / t / 1e9,
+                           hbm_frac=w["bytes"] / t / 1e9 / pk["hbm_gbs"])
+        if w["exps"]:
+            kernels[nm]["gexps"] = w["exps"] / t / 1e9
+    dom = max(kernels, key=lambda k: kernels[k]["ms"])
+    sm_for_peak = pk["sm_max_mhz"]
+    if work[dom]["exps"] and exps:
+        peak = sfu_peak_gexps(sm_for_peak)
+        ach = work[dom]["exps"] / (per_call[dom] / 1000.0) / 1e9
+        roof = {"kernel": dom, "bound": "alu", "achieved": ach, "peak": peak, "unit": "Gexp/s",
+                "frac": ach / peak, "traffic": None,
+                "peak_source": "148 SM x 16 MUFU.EX2/clk x %.0f MHz (max SM clock)" % sm_for_peak}
+    else:
+        ach = work[dom]["bytes"] / (per_call[dom] / 1000.0) / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": ach / pk["hbm_gbs"], "traffic": None,
+                "peak_source": pk["source"]}
+    # step roofline: sum over calls of max(bytes / HBM, exps / SFU)
+    bound_s = 0.0
+    for nm, w in work.items():
+        bound_s += max(w["bytes"] / (pk["hbm_gbs"] * 1e9),
+                       (w["exps"] / (sfu_peak_gexps(sm_for_peak) * 1e9)) if w["exps"] else 0.0)
+    launches_per_step = {"presort": 1 + 10 + 1 + 1 + 1 + 1 + 1,
+                         "full64": 1 + 9 + 1 + 1 + 1 + 1 + 1}[args.sort_mode]
+    line = {
+        "metric": METRIC, "value": value, "unit": "Mpix/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "gaussians": sp.n, "width": c.width, "height": c.height,
+                   "sh_degree": 3, "views_per_gpu": 1, "pairs": n_pairs,
+                   "sort_mode": args.sort_mode,
+                   "l2": "working set larger than L2 (0.7 GB of parameters and Adam state "
+                         "rewritten every step)",
+                   "parallelism": "dp%d (one view per GPU, gradient all-reduce)" % world
+                   if world > 1 else "single GPU"},
+        "roofline": roof,
+        "step_roofline": {"bound_ms": bound_s * 1000.0, "frac": bound_s * 1000.0 / ms},
+        "kernels": kernels,
+        "cpu_baseline": None if cpu is None else {k: cpu[k] for k in
+                                                  ("value", "unit", "cores", "kind", "sample")},
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+        "device_status": api.status_string(status),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

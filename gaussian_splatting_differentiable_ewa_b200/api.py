@@ -1,0 +1,249 @@
+"""ctypes binding of ``libgs_b200.so`` -- the C ABI declared in ``include/gs.h``.
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels. The structs mirror gs.h field for field; the functions keep the C
+names. Loading fails loudly when the library has not been built -- there is
+no fallback implementation.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libgs_b200.so")
+
+GS_OK = 0
+GS_ERR_INVALID_ARG = 1
+GS_ERR_CAPACITY = 2
+GS_ERR_OVERFLOW = 3
+GS_ERR_DEVICE_TIMEOUT = 4
+GS_ERR_NONFINITE = 5
+GS_ERR_CUDA = 6
+
+GS_SORT_FULL64 = 0
+GS_SORT_PRESORT = 1
+
+GS_TILE = 16
+GS_MAX_VIEWS = 32
+GS_RECORD_FLOATS = 12
+GS_GRAD2D_FLOATS = 12
+
+_c = ctypes
+_vp = _c.c_void_p
+
+
+class GsCamera(_c.Structure):
+    _fields_ = [("viewmat", _c.c_float * 12), ("fx", _c.c_float), ("fy", _c.c_float),
+                ("cx", _c.c_float), ("cy", _c.c_float), ("width", _c.c_int32),
+                ("height", _c.c_int32), ("campos", _c.c_float * 3), ("reserved", _c.c_float)]
+
+
+class GsParams(_c.Structure):
+    _fields_ = [("means", _vp), ("log_scales", _vp), ("quats", _vp), ("opacity_logit", _vp),
+                ("sh", _vp), ("sh_degree", _c.c_int32), ("reserved", _c.c_int32),
+                ("n", _c.c_int64)]
+
+
+class GsGrads(_c.Structure):
+    _fields_ = [("means", _vp), ("log_scales", _vp), ("quats", _vp), ("opacity_logit", _vp),
+                ("sh", _vp)]
+
+
+class GsProjected(_c.Structure):
+    _fields_ = [("records", _vp), ("radii", _vp)]
+
+
+class GsBinned(_c.Structure):
+    _fields_ = [("ids", _vp), ("ranges", _vp), ("n_pairs", _vp), ("pair_capacity", _c.c_int64)]
+
+
+class GsAdamGroup(_c.Structure):
+    _fields_ = [("param", _vp), ("grad", _vp), ("exp_avg", _vp), ("exp_avg_sq", _vp),
+                ("count", _c.c_int64), ("lr", _c.c_float), ("reserved", _c.c_float)]
+
+
+# (name, restype, argtypes) for every symbol gs.h declares
+SIGNATURES = [
+    ("gs_abi_version", _c.c_int32, []),
+    ("gs_status_string", _c.c_char_p, [_c.c_int]),
+    ("gs_workspace_size", _c.c_size_t,
+     [_c.c_int64, _c.c_int32, _c.POINTER(GsCamera), _c.c_int64, _c.c_int32]),
+    ("gs_project", _c.c_int,
+     [_c.POINTER(GsParams), _c.POINTER(GsCamera), _c.c_int32, _c.POINTER(GsProjected), _vp]),
+    ("gs_bin_sort", _c.c_int,
+     [_c.POINTER(GsProjected), _c.POINTER(GsCamera), _c.c_int32, _c.c_int64, _c.c_int32,
+      _c.POINTER(GsBinned), _vp, _c.c_size_t, _vp]),
+    ("gs_rasterize_fwd", _c.c_int,
+     [_c.POINTER(GsProjected), _c.POINTER(GsBinned), _c.POINTER(GsCamera), _c.c_int32,
+      _c.c_int64, _c.POINTER(_c.c_float), _vp, _vp, _vp, _vp]),
+    ("gs_rasterize_bwd", _c.c_int,
+     [_c.POINTER(GsParams), _c.POINTER(GsProjected), _c.POINTER(GsBinned),
+      _c.POINTER(GsCamera), _c.c_int32, _c.POINTER(_c.c_float), _vp, _vp, _vp, _vp,
+      _c.POINTER(GsGrads), _vp]),
+    ("gs_project_bwd", _c.c_int,
+     [_c.POINTER(GsParams), _c.POINTER(GsCamera), _c.c_int32, _vp, _vp, _c.POINTER(GsGrads),
+      _vp]),
+    ("gs_densify_stats", _c.c_int,
+     [_vp, _vp, _c.c_int32, _c.c_int64, _vp, _vp, _vp, _vp]),
+    ("gs_adam_step", _c.c_int,
+     [_c.POINTER(GsAdamGroup), _c.c_int32, _c.c_float, _c.c_float, _c.c_float, _c.c_int64, _vp]),
+    ("gs_get_status", _c.c_int, [_vp, _vp]),
+]
+
+_LIB = None
+
+
+class GsError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__("%s failed: %s (status %d)" % (where, status_string(status), status))
+        self.status = status
+
+
+def lib():
+    """Load libgs_b200.so (no fallback: raises if it was not built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libgs_b200.so is not built (run "
+                               "gaussian_splatting_differentiable_ewa_b200/build.py)")
+        L = _c.CDLL(LIB_PATH)
+        for name, res, args in SIGNATURES:
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _LIB = L
+    return _LIB
+
+
+def status_string(status: int) -> str:
+    try:
+        return lib().gs_status_string(int(status)).decode()
+    except Exception:  # library not loadable
+        return "status %d" % status
+
+
+def _check(status: int, where: str) -> None:
+    if status != GS_OK:
+        raise GsError(status, where)
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    return int(t.data_ptr())
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return None
+    h = getattr(stream, "cuda_stream", stream)
+    return int(h) if h else None
+
+
+def cameras(cams: Sequence) -> ctypes.Array:
+    """Array of GsCamera from objects with viewmat/fx/fy/cx/cy/width/height/campos."""
+    arr = (GsCamera * len(cams))()
+    for k, c in enumerate(cams):
+        d = c if isinstance(c, dict) else c.as_dict()
+        vm = [float(x) for x in np.asarray(d["viewmat"], np.float32).reshape(12)]
+        arr[k].viewmat[:] = vm
+        arr[k].fx, arr[k].fy = float(d["fx"]), float(d["fy"])
+        arr[k].cx, arr[k].cy = float(d["cx"]), float(d["cy"])
+        arr[k].width, arr[k].height = int(d["width"]), int(d["height"])
+        arr[k].campos[:] = [float(x) for x in d["campos"]]
+    return arr
+
+
+def params(means, log_scales, quats, opacity_logit, sh, sh_degree: int) -> GsParams:
+    return GsParams(_ptr(means), _ptr(log_scales), _ptr(quats), _ptr(opacity_logit), _ptr(sh),
+                    int(sh_degree), 0, int(means.shape[0]))
+
+
+def grads(means, log_scales, quats, opacity_logit, sh) -> GsGrads:
+    return GsGrads(_ptr(means), _ptr(log_scales), _ptr(quats), _ptr(opacity_logit), _ptr(sh))
+
+
+def projected(records, radii) -> GsProjected:
+    return GsProjected(_ptr(records), _ptr(radii))
+
+
+def binned(ids, ranges, n_pairs, capacity: int) -> GsBinned:
+    return GsBinned(_ptr(ids), _ptr(ranges), _ptr(n_pairs), int(capacity))
+
+
+def _floats3(bg) -> ctypes.Array:
+    a = (_c.c_float * 3)()
+    a[:] = [float(x) for x in bg]
+    return a
+
+
+# ---------------------------------------------------------------- C calls
+
+def gs_abi_version() -> int:
+    return int(lib().gs_abi_version())
+
+
+def gs_workspace_size(n: int, cams_arr, n_views: int, pair_capacity: int, sort_mode: int) -> int:
+    return int(lib().gs_workspace_size(int(n), int(n_views), cams_arr, int(pair_capacity),
+                                       int(sort_mode)))
+
+
+def gs_project(p: GsParams, cams_arr, n_views: int, out: GsProjected, stream=None) -> None:
+    _check(lib().gs_project(_c.byref(p), cams_arr, int(n_views), _c.byref(out), _stream(stream)),
+           "gs_project")
+
+
+def gs_bin_sort(proj: GsProjected, cams_arr, n_views: int, n: int, sort_mode: int,
+                out: GsBinned, ws, stream=None) -> None:
+    _check(lib().gs_bin_sort(_c.byref(proj), cams_arr, int(n_views), int(n), int(sort_mode),
+                             _c.byref(out), _ptr(ws), int(ws.numel() * ws.element_size()),
+                             _stream(stream)), "gs_bin_sort")
+
+
+def gs_rasterize_fwd(proj: GsProjected, bins: GsBinned, cams_arr, n_views: int, n: int, bg,
+                     image, final_T, n_contrib, stream=None) -> None:
+    _check(lib().gs_rasterize_fwd(_c.byref(proj), _c.byref(bins), cams_arr, int(n_views), int(n),
+                                  _floats3(bg), _ptr(image), _ptr(final_T), _ptr(n_contrib),
+                                  _stream(stream)), "gs_rasterize_fwd")
+
+
+def gs_rasterize_bwd(p: GsParams, proj: GsProjected, bins: GsBinned, cams_arr, n_views: int, bg,
+                     dL_dimage, final_T, n_contrib, grad2d, g: Optional[GsGrads],
+                     stream=None) -> None:
+    _check(lib().gs_rasterize_bwd(_c.byref(p), _c.byref(proj), _c.byref(bins), cams_arr,
+                                  int(n_views), _floats3(bg), _ptr(dL_dimage), _ptr(final_T),
+                                  _ptr(n_contrib), _ptr(grad2d),
+                                  None if g is None else _c.byref(g), _stream(stream)),
+           "gs_rasterize_bwd")
+
+
+def gs_project_bwd(p: GsParams, cams_arr, n_views: int, radii, grad2d, g: GsGrads,
+                   stream=None) -> None:
+    _check(lib().gs_project_bwd(_c.byref(p), cams_arr, int(n_views), _ptr(radii), _ptr(grad2d),
+                                _c.byref(g), _stream(stream)), "gs_project_bwd")
+
+
+def gs_densify_stats(grad2d, radii, n_views: int, n: int, accum_plain, accum_abs, denom,
+                     stream=None) -> None:
+    _check(lib().gs_densify_stats(_ptr(grad2d), _ptr(radii), int(n_views), int(n),
+                                  _ptr(accum_plain), _ptr(accum_abs), _ptr(denom),
+                                  _stream(stream)), "gs_densify_stats")
+
+
+def gs_adam_step(groups: Sequence[tuple], beta1: float, beta2: float, eps: float, step: int,
+                 stream=None) -> None:
+    """groups: (param, grad, exp_avg, exp_avg_sq, lr) tensors / float."""
+    arr = (GsAdamGroup * len(groups))()
+    for k, (p, g, m, v, lr) in enumerate(groups):
+        arr[k] = GsAdamGroup(_ptr(p), _ptr(g), _ptr(m), _ptr(v), int(p.numel()), float(lr), 0.0)
+    _check(lib().gs_adam_step(arr, len(groups), float(beta1), float(beta2), float(eps), int(step),
+                              _stream(stream)), "gs_adam_step")
+
+
+def gs_get_status(ws, stream=None) -> int:
+    return int(lib().gs_get_status(_ptr(ws), _stream(stream)))

@@ -1,0 +1,330 @@
+// capi.cu -- the extern "C" entry points declared in include/gs.h.
+//
+// Host-side argument checks, workspace carving and kernel launches. Nothing
+// here allocates device memory or keeps state between calls.
+
+#include <cstdint>
+#include <cstring>
+#include <cuda_runtime.h>
+
+#include "gs_internal.h"
+
+using namespace gsb;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kControlBytes = 4096;  // status word, counters, device scalars
+constexpr size_t kStatusOffset = 0;
+constexpr size_t kCountersOffset = 64;   // 16 x uint32
+constexpr size_t kNItemsOffset = 256;    // int64
+constexpr size_t kHistBytes = 8 * 256 * sizeof(unsigned long long);
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+int bits_for(uint64_t max_value) {
+  int b = 0;
+  while (max_value) { ++b; max_value >>= 1; }
+  return b;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct Layout {
+  int pair_passes = 0;
+  int presort_passes = 0;
+  int key_bytes = 8;
+  int64_t region_words = 0;
+  size_t off_hist = 0, off_phist = 0, off_emit_lb = 0, off_lb = 0, off_keys0 = 0, off_keys1 = 0,
+         off_vals1 = 0, off_pkeys0 = 0, off_pkeys1 = 0, off_pvals0 = 0, off_pvals1 = 0;
+  size_t total = 0;
+};
+
+bool check_cams(const gs_camera* cams, int32_t n_views) {
+  if (!cams || n_views < 1 || n_views > GS_MAX_VIEWS) return false;
+  for (int v = 0; v < n_views; ++v) {
+    if (cams[v].width <= 0 || cams[v].height <= 0) return false;
+    if (cams[v].width != cams[0].width || cams[v].height != cams[0].height) return false;
+  }
+  const Grid g = grid_of(cams[0]);
+  if (g.tiles_x > 65535 || g.tiles_y > 65535) return false;
+  return true;
+}
+
+bool make_layout(int64_t n, int32_t n_views, const gs_camera* cams, int64_t capacity, int32_t mode,
+                 Layout& L) {
+  if (n < 0 || n >= (1ll << 31) || capacity < 0) return false;
+  if (mode != GS_SORT_FULL64 && mode != GS_SORT_PRESORT) return false;
+  if (!check_cams(cams, n_views)) return false;
+  const Grid g = grid_of(cams[0]);
+  const uint64_t tiles = (uint64_t)g.tiles_per_view * (uint64_t)n_views;
+  if (tiles >= (1ull << 32)) return false;
+  const int tile_bits = bits_for(tiles - 1);
+  const int64_t items = n * n_views;
+  if (mode == GS_SORT_FULL64) {
+    L.key_bytes = 8;
+    L.pair_passes = (32 + tile_bits + 7) / 8;
+    L.presort_passes = 0;
+  } else {
+    L.key_bytes = 4;
+    L.pair_passes = (tile_bits + 7) / 8;
+    L.presort_passes = 4 + (n_views > 1 ? 1 : 0);
+  }
+  const int regions = L.pair_passes > L.presort_passes ? L.pair_passes : L.presort_passes;
+  int64_t parts = sort_partitions(capacity);
+  if (mode == GS_SORT_PRESORT) {
+    const int64_t p2 = sort_partitions(items);
+    if (p2 > parts) parts = p2;
+  }
+  L.region_words = parts * 256;
+  size_t off = kControlBytes;
+  L.off_hist = off; off = align_up(off + kHistBytes);
+  L.off_phist = off; off = align_up(off + kHistBytes);
+  L.off_emit_lb = off; off = align_up(off + (size_t)emit_blocks(items) * 8);
+  L.off_lb = off; off = align_up(off + (size_t)(regions > 0 ? regions : 1) * L.region_words * 8);
+  L.off_keys0 = off; off = align_up(off + (size_t)capacity * L.key_bytes);
+  L.off_keys1 = off; off = align_up(off + (size_t)capacity * L.key_bytes);
+  L.off_vals1 = off; off = align_up(off + (size_t)capacity * 4);
+  if (mode == GS_SORT_PRESORT) {
+    L.off_pkeys0 = off; off = align_up(off + (size_t)items * 8);
+    L.off_pkeys1 = off; off = align_up(off + (size_t)items * 8);
+    L.off_pvals0 = off; off = align_up(off + (size_t)items * 4);
+    L.off_pvals1 = off; off = align_up(off + (size_t)items * 4);
+  }
+  L.total = off;
+  return true;
+}
+
+CamSet pack_cams(const gs_camera* cams, int32_t n_views) {
+  CamSet s;
+  std::memset(&s, 0, sizeof(s));
+  for (int v = 0; v < n_views; ++v) s.c[v] = cams[v];
+  return s;
+}
+
+inline gs_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GS_OK : GS_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t gs_abi_version(void) { return GS_ABI_VERSION; }
+
+const char* gs_status_string(gs_status s) {
+  switch (s) {
+    case GS_OK: return "ok";
+    case GS_ERR_INVALID_ARG: return "invalid argument";
+    case GS_ERR_CAPACITY: return "pair capacity exceeded";
+    case GS_ERR_OVERFLOW: return "size exceeds a 32-bit field";
+    case GS_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
+    case GS_ERR_NONFINITE: return "non-finite input";
+    case GS_ERR_CUDA: return "CUDA runtime error";
+  }
+  return "unknown status";
+}
+
+size_t gs_workspace_size(int64_t n, int32_t n_views, const gs_camera* cams, int64_t pair_capacity,
+                         int32_t sort_mode) {
+  Layout L;
+  if (!make_layout(n, n_views, cams, pair_capacity, sort_mode, L)) return 0;
+  return L.total;
+}
+
+gs_status gs_project(const gs_params* params, const gs_camera* cams, int32_t n_views,
+                     gs_projected* out, void* stream) {
+  if (!params || !out || !check_cams(cams, n_views)) return GS_ERR_INVALID_ARG;
+  const gs_params& p = *params;
+  if (p.n < 0) return GS_ERR_INVALID_ARG;
+  if (p.n >= (1ll << 31) || p.n * n_views >= (1ll << 40)) return GS_ERR_OVERFLOW;
+  if (p.sh_degree < 0 || p.sh_degree > 3) return GS_ERR_INVALID_ARG;
+  if (p.n == 0) return GS_OK;
+  if (!p.means || !p.log_scales || !p.quats || !p.opacity_logit || !p.sh || !out->records ||
+      !out->radii)
+    return GS_ERR_INVALID_ARG;
+  if (!aligned(p.means, 16) || !aligned(p.log_scales, 16) || !aligned(p.quats, 16) ||
+      !aligned(out->records, 16))
+    return GS_ERR_INVALID_ARG;
+  const CamSet cs = pack_cams(cams, n_views);
+  return cuda_status(launch_project(p, cs, n_views, out->records, out->radii,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n_views, int64_t n,
+                      int32_t sort_mode, gs_binned* out, void* ws, size_t ws_bytes,
+                      void* stream) {
+  if (!proj || !out || !ws) return GS_ERR_INVALID_ARG;
+  if (n >= (1ll << 31)) return GS_ERR_OVERFLOW;
+  Layout L;
+  if (!make_layout(n, n_views, cams, out->pair_capacity, sort_mode, L)) return GS_ERR_INVALID_ARG;
+  if (ws_bytes < L.total || !aligned(ws, kAlign)) return GS_ERR_INVALID_ARG;
+  if (!out->ids || !out->ranges || !out->n_pairs) return GS_ERR_INVALID_ARG;
+  if (n > 0 && (!proj->records || !aligned(proj->records, 16))) return GS_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  const Grid g = grid_of(cams[0]);
+  const int64_t tiles = (int64_t)g.tiles_per_view * n_views;
+  const int64_t items = n * n_views;
+
+  if (cudaMemsetAsync(w + kCountersOffset, 0, 16 * sizeof(uint32_t), st) != cudaSuccess ||
+      cudaMemsetAsync(w + L.off_hist, 0, kHistBytes, st) != cudaSuccess ||
+      cudaMemsetAsync(w + L.off_phist, 0, kHistBytes, st) != cudaSuccess ||
+      cudaMemsetAsync(w + L.off_emit_lb, 0, (size_t)emit_blocks(items) * 8, st) != cudaSuccess ||
+      cudaMemsetAsync(out->ranges, 0, (size_t)tiles * 2 * sizeof(int64_t), st) != cudaSuccess)
+    return GS_ERR_CUDA;
+
+  BinSortArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.records = proj->records;
+  a.n = (int)n;
+  a.n_views = n_views;
+  a.mode = sort_mode;
+  a.grid = g;
+  a.capacity = out->pair_capacity;
+  a.pair_passes = L.pair_passes;
+  a.presort_passes = L.presort_passes;
+  a.emit_buf = L.pair_passes & 1;
+  a.keys[0] = reinterpret_cast<uint64_t*>(w + L.off_keys0);
+  a.keys[1] = reinterpret_cast<uint64_t*>(w + L.off_keys1);
+  a.vals[0] = out->ids;
+  a.vals[1] = reinterpret_cast<uint32_t*>(w + L.off_vals1);
+  if (sort_mode == GS_SORT_PRESORT) {
+    a.pkeys[0] = reinterpret_cast<uint64_t*>(w + L.off_pkeys0);
+    a.pkeys[1] = reinterpret_cast<uint64_t*>(w + L.off_pkeys1);
+    a.pvals[0] = reinterpret_cast<uint32_t*>(w + L.off_pvals0);
+    a.pvals[1] = reinterpret_cast<uint32_t*>(w + L.off_pvals1);
+  }
+  a.hist = reinterpret_cast<unsigned long long*>(w + L.off_hist);
+  a.presort_hist = reinterpret_cast<unsigned long long*>(w + L.off_phist);
+  a.lookback = reinterpret_cast<uint64_t*>(w + L.off_lb);
+  a.lookback_region_words = L.region_words;
+  a.emit_lookback = reinterpret_cast<uint64_t*>(w + L.off_emit_lb);
+  a.counters = reinterpret_cast<uint32_t*>(w + kCountersOffset);
+  a.status = reinterpret_cast<uint32_t*>(w + kStatusOffset);
+  a.n_pairs = out->n_pairs;
+  a.n_items_dev = reinterpret_cast<int64_t*>(w + kNItemsOffset);
+  a.ranges = out->ranges;
+  a.n_tiles = tiles;
+  return cuda_status(launch_bin_sort(a, st));
+}
+
+gs_status gs_rasterize_fwd(const gs_projected* proj, const gs_binned* bins, const gs_camera* cams,
+                           int32_t n_views, int64_t n, const float* bg, float* image,
+                           float* final_T, uint32_t* n_contrib, void* stream) {
+  if (!proj || !bins || !bg || !check_cams(cams, n_views)) return GS_ERR_INVALID_ARG;
+  if (n < 0) return GS_ERR_INVALID_ARG;
+  if (n >= (1ll << 31)) return GS_ERR_OVERFLOW;
+  if (!image || !final_T || !n_contrib || !bins->ranges || !bins->ids) return GS_ERR_INVALID_ARG;
+  if (n > 0 && (!proj->records || !aligned(proj->records, 16))) return GS_ERR_INVALID_ARG;
+  const Grid g = grid_of(cams[0]);
+  return cuda_status(launch_raster_fwd(proj->records, bins->ids, bins->ranges, bins->pair_capacity,
+                                       g, n_views, (int)n, bg, image, final_T, n_contrib, nullptr,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+namespace {
+
+gs_status check_grads_args(const gs_params& p, const gs_grads* grads, bool need) {
+  if (!grads) return need ? GS_ERR_INVALID_ARG : GS_OK;
+  if (p.n > 0 && (!p.means || !p.log_scales || !p.quats || !p.opacity_logit || !p.sh ||
+                  !grads->means || !grads->log_scales || !grads->quats ||
+                  !grads->opacity_logit || !grads->sh))
+    return GS_ERR_INVALID_ARG;
+  if (!aligned(p.means, 16) || !aligned(p.log_scales, 16) || !aligned(p.quats, 16) ||
+      !aligned(grads->means, 16) || !aligned(grads->log_scales, 16) ||
+      !aligned(grads->quats, 16))
+    return GS_ERR_INVALID_ARG;
+  return GS_OK;
+}
+
+}  // namespace
+
+gs_status gs_project_bwd(const gs_params* params, const gs_camera* cams, int32_t n_views,
+                         const int32_t* radii, const float* grad2d, gs_grads* grads,
+                         void* stream) {
+  if (!params || !check_cams(cams, n_views)) return GS_ERR_INVALID_ARG;
+  const gs_params& p = *params;
+  if (p.n < 0 || p.sh_degree < 0 || p.sh_degree > 3) return GS_ERR_INVALID_ARG;
+  if (p.n >= (1ll << 31)) return GS_ERR_OVERFLOW;
+  const gs_status s = check_grads_args(p, grads, true);
+  if (s != GS_OK) return s;
+  if (p.n == 0) return GS_OK;
+  if (!radii || !grad2d || !aligned(grad2d, 16)) return GS_ERR_INVALID_ARG;
+  const CamSet cs = pack_cams(cams, n_views);
+  return cuda_status(launch_project_bwd(p, cs, n_views, grad2d, radii, *grads,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+gs_status gs_rasterize_bwd(const gs_params* params, const gs_projected* proj,
+                           const gs_binned* bins, const gs_camera* cams, int32_t n_views,
+                           const float* bg, const float* dL_dimage, const float* final_T,
+                           const uint32_t* n_contrib, float* grad2d, gs_grads* grads,
+                           void* stream) {
+  if (!params || !proj || !bins || !bg || !check_cams(cams, n_views)) return GS_ERR_INVALID_ARG;
+  const gs_params& p = *params;
+  if (p.n < 0 || p.sh_degree < 0 || p.sh_degree > 3) return GS_ERR_INVALID_ARG;
+  if (p.n >= (1ll << 31)) return GS_ERR_OVERFLOW;
+  if (!dL_dimage || !final_T || !n_contrib || !bins->ranges || !bins->ids)
+    return GS_ERR_INVALID_ARG;
+  if (p.n > 0 && (!proj->records || !proj->radii || !grad2d)) return GS_ERR_INVALID_ARG;
+  if (!aligned(grad2d, 16)) return GS_ERR_INVALID_ARG;
+  const gs_status s = check_grads_args(p, grads, false);
+  if (s != GS_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Grid g = grid_of(cams[0]);
+  if (cudaMemsetAsync(grad2d, 0, (size_t)p.n * n_views * GS_GRAD2D_FLOATS * sizeof(float), st) !=
+      cudaSuccess)
+    return GS_ERR_CUDA;
+  cudaError_t e = launch_raster_bwd(proj->records, bins->ids, bins->ranges, bins->pair_capacity, g,
+                                    n_views, (int)p.n, bg, dL_dimage, final_T, n_contrib, grad2d,
+                                    nullptr, st);
+  if (e != cudaSuccess) return GS_ERR_CUDA;
+  if (!grads) return GS_OK;
+  const CamSet cs = pack_cams(cams, n_views);
+  return cuda_status(launch_project_bwd(p, cs, n_views, grad2d, proj->radii, *grads, st));
+}
+
+gs_status gs_densify_stats(const float* grad2d, const int32_t* radii, int32_t n_views, int64_t n,
+                           float* accum_plain, float* accum_abs, int32_t* denom, void* stream) {
+  if (n < 0 || n_views < 1 || n_views > GS_MAX_VIEWS) return GS_ERR_INVALID_ARG;
+  if (n >= (1ll << 31)) return GS_ERR_OVERFLOW;
+  if (n == 0) return GS_OK;
+  if (!grad2d || !radii || !accum_plain || !accum_abs || !denom || !aligned(grad2d, 16))
+    return GS_ERR_INVALID_ARG;
+  return cuda_status(launch_densify(grad2d, radii, n_views, (int)n, accum_plain, accum_abs, denom,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+gs_status gs_adam_step(const gs_adam_group* groups, int32_t n_groups, float beta1, float beta2,
+                       float eps, int64_t step, void* stream) {
+  if (!groups || n_groups < 1 || n_groups > 8 || step < 1) return GS_ERR_INVALID_ARG;
+  if (!(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f) || !(eps >= 0.f))
+    return GS_ERR_INVALID_ARG;
+  for (int k = 0; k < n_groups; ++k) {
+    const gs_adam_group& gr = groups[k];
+    if (gr.count < 0) return GS_ERR_INVALID_ARG;
+    if (gr.count == 0) continue;
+    if (!gr.param || !gr.grad || !gr.exp_avg || !gr.exp_avg_sq) return GS_ERR_INVALID_ARG;
+    if (!aligned(gr.param, 16) || !aligned(gr.grad, 16) || !aligned(gr.exp_avg, 16) ||
+        !aligned(gr.exp_avg_sq, 16))
+      return GS_ERR_INVALID_ARG;
+  }
+  return cuda_status(
+      launch_adam(groups, n_groups, beta1, beta2, eps, step, static_cast<cudaStream_t>(stream)));
+}
+
+gs_status gs_get_status(void* ws, void* stream) {
+  if (!ws) return GS_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return GS_ERR_CUDA;
+  uint32_t word = 0;
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  if (cudaMemcpy(&word, w + kStatusOffset, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return GS_ERR_CUDA;
+  if (cudaMemset(w + kStatusOffset, 0, sizeof(uint32_t)) != cudaSuccess) return GS_ERR_CUDA;
+  if (word & kStatusTimeout) return GS_ERR_DEVICE_TIMEOUT;
+  if (word & kStatusBounds) return GS_ERR_OVERFLOW;
+  if (word & kStatusCapacity) return GS_ERR_CAPACITY;
+  return GS_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,181 @@
+// gs_device.cuh -- device-side helpers shared by the sm_100a kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/gs.h"
+
+namespace gsb {
+
+// Method constants (the task's stated values; the pages print none of them).
+constexpr int kTile = GS_TILE;                 // 16x16 pixel tiles
+constexpr int kTilePixels = kTile * kTile;     // 256 threads per raster block
+constexpr double kNear = 0.2;                  // near-plane cull
+constexpr double kLowPass = 0.3;               // + 0.3 I on the 2D covariance
+constexpr float kAlphaMax = 0.99f;             // alpha clamp
+constexpr float kAlphaMin = 1.0f / 255.0f;     // alpha skip threshold
+constexpr float kTMin = 1e-4f;                 // transmittance stop
+constexpr int kMaxRadius = 1 << 30;            // radius saturation
+
+// Status bits OR-ed into the workspace status word.
+constexpr uint32_t kStatusCapacity = 1u << 0;
+constexpr uint32_t kStatusTimeout = 1u << 1;
+constexpr uint32_t kStatusBounds = 1u << 2;
+
+// Spin limit of every device-side wait (iterations of ~100 ns each).
+constexpr uint32_t kSpinLimit = 20u * 1000u * 1000u;
+
+// Cameras travel in the kernel parameter block.
+struct CamSet {
+  gs_camera c[GS_MAX_VIEWS];
+};
+
+struct Grid {
+  int width, height, tiles_x, tiles_y, tiles_per_view;
+};
+
+__host__ __device__ inline Grid grid_of(const gs_camera& c) {
+  Grid g;
+  g.width = c.width;
+  g.height = c.height;
+  g.tiles_x = (c.width + kTile - 1) / kTile;
+  g.tiles_y = (c.height + kTile - 1) / kTile;
+  g.tiles_per_view = g.tiles_x * g.tiles_y;
+  return g;
+}
+
+// Record field offsets (floats), see gs.h.
+enum RecField {
+  R_U = 0, R_V = 1, R_CA = 2, R_CB = 3, R_CC = 4, R_OPAC = 5,
+  R_R = 6, R_G = 7, R_B = 8, R_DEPTH = 9, R_TX = 10, R_TY = 11
+};
+// Screen-space gradient fields (floats), see gs.h.
+enum G2Field {
+  G_U = 0, G_V = 1, G_CA = 2, G_CB = 3, G_CC = 4, G_OPAC = 5,
+  G_R = 6, G_G = 7, G_B = 8, G_ABS = 9
+};
+
+// Per-pixel opacity of one splat. Forward and backward both call this, so
+// their skip / stop decisions are taken on identical float values.
+//   q = a dx^2 + 2 b dx dy + c dy^2,  d = pixel centre - mean
+//   alpha_raw = o exp(-q/2),  alpha = min(0.99, alpha_raw)
+struct SplatEval {
+  float dx, dy, G, alpha_raw, alpha;
+};
+
+__device__ __forceinline__ SplatEval splat_eval(float px, float py, float u, float v, float ca,
+                                                float cb, float cc, float o) {
+  SplatEval e;
+  e.dx = px - u;
+  e.dy = py - v;
+  float power = -0.5f * (ca * e.dx * e.dx + cc * e.dy * e.dy) - cb * e.dx * e.dy;
+  e.G = __expf(power);
+  e.alpha_raw = o * e.G;
+  e.alpha = fminf(kAlphaMax, e.alpha_raw);
+  return e;
+}
+
+// ---------------------------------------------------------------- PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// One TMA bulk copy global -> shared, completing `bytes` on `bar`.
+// dst and src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes,
+                                              uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait on an mbarrier phase; on timeout flags the status and returns
+// false (the caller must not touch the buffer).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  uint32_t* status) {
+  for (uint32_t it = 0; it < kSpinLimit; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (it > 64) __nanosleep(64);
+  }
+  if (status) atomicOr(status, kStatusTimeout);
+  return false;
+}
+
+// Vector float reduction into global memory (sm_90+), 16-byte aligned.
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+
+// 64-bit relaxed device-scope load / store for decoupled look-back words.
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Look-back word: [63:62] flag (0 empty, 1 aggregate, 2 inclusive prefix),
+// [61:0] count.
+constexpr uint64_t kLbAggregate = 1ull << 62;
+constexpr uint64_t kLbPrefix = 2ull << 62;
+constexpr uint64_t kLbValueMask = (1ull << 62) - 1;
+
+// Wait (bounded) until a look-back word is non-empty; returns it. On timeout
+// flags the status and returns an inclusive-prefix word of 0 so that the
+// caller terminates.
+__device__ __forceinline__ uint64_t lookback_wait(const uint64_t* p, uint32_t* status) {
+  uint64_t w = ld_relaxed_u64(p);
+  uint32_t it = 0;
+  while ((w >> 62) == 0) {
+    if (++it > kSpinLimit) {
+      atomicOr(status, kStatusTimeout);
+      return kLbPrefix;
+    }
+    if (it > 32) __nanosleep(100);
+    w = ld_relaxed_u64(p);
+  }
+  return w;
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+}  // namespace gsb

@@ -1,0 +1,64 @@
+// gs_internal.h -- launchers shared between the kernel files and the C ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "gs_device.cuh"
+
+namespace gsb {
+
+struct BinSortArgs {
+  const float* records;
+  int n;
+  int n_views;
+  int mode;
+  Grid grid;
+  int64_t capacity;
+  int pair_passes;     // radix passes over the pair keys
+  int presort_passes;  // radix passes over the per-Gaussian depth keys
+  int emit_buf;        // which key/value buffer the emission writes
+  uint64_t* keys[2];   // pair keys (64-bit, or 32-bit in presort mode)
+  uint32_t* vals[2];   // pair ids; the final one is the caller's ids array
+  uint64_t* pkeys[2];  // presort keys
+  uint32_t* pvals[2];  // presort values
+  unsigned long long* hist;          // [8][256] pair-key digit histograms
+  unsigned long long* presort_hist;  // [8][256]
+  uint64_t* lookback;                // [passes][region_words]
+  int64_t lookback_region_words;
+  uint64_t* emit_lookback;           // [emit blocks]
+  uint32_t* counters;                // [16] dynamic block counters
+  uint32_t* status;
+  int64_t* n_pairs;
+  int64_t* n_items_dev;
+  int64_t* ranges;
+  int64_t n_tiles;     // n_views * tiles per view
+};
+
+cudaError_t launch_project(const gs_params& p, const CamSet& cams, int n_views, float* records,
+                           int* radii, cudaStream_t stream);
+cudaError_t launch_project_bwd(const gs_params& p, const CamSet& cams, int n_views,
+                               const float* grad2d, const int* radii, const gs_grads& g,
+                               cudaStream_t stream);
+cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream);
+cudaError_t launch_raster_fwd(const float* records, const uint32_t* ids, const int64_t* ranges,
+                              int64_t capacity, const Grid& g, int n_views, int n,
+                              const float bg[3], float* image,
+                              float* final_T, uint32_t* n_contrib, uint32_t* status,
+                              cudaStream_t stream);
+cudaError_t launch_raster_bwd(const float* records, const uint32_t* ids, const int64_t* ranges,
+                              int64_t capacity, const Grid& g, int n_views, int n,
+                              const float bg[3],
+                              const float* dL_dimage, const float* final_T,
+                              const uint32_t* n_contrib, float* grad2d, uint32_t* status,
+                              cudaStream_t stream);
+cudaError_t launch_densify(const float* grad2d, const int* radii, int n_views, int n,
+                           float* accum_plain, float* accum_abs, int* denom, cudaStream_t stream);
+cudaError_t launch_adam(const gs_adam_group* groups, int n_groups, float b1, float b2, float eps,
+                        int64_t step, cudaStream_t stream);
+
+int64_t sort_partitions(int64_t items);
+int64_t emit_blocks(int64_t items);
+
+}  // namespace gsb

@@ -1,0 +1,471 @@
+// project.cu -- EWA projection of 3D Gaussians and its backward, sm_100a.
+//
+// Forward ("Better Gaussian Splatting in Julia", pwwt.cn sec. 3.2
+// project_gaussian; lshu.cn sec. 3.2: world -> camera -> pixel with division
+// by depth, 3D covariance through the Jacobian of that map): one thread per
+// Gaussian, looping over the views so the parameters are read once. The
+// geometry that ends in a discrete decision (depth key, radius, tile
+// rectangle) is evaluated in double, so that the decision is the exact one up
+// to double rounding; colour is evaluated in float.
+//
+// Backward: chain rule of the same map, float, one thread per Gaussian,
+// summing the views in registers before one write of every gradient.
+
+#include <cuda_runtime.h>
+
+#include "gs_internal.h"
+
+namespace gsb {
+namespace {
+
+// Real spherical harmonics on the unit sphere, index l*l + l + m, l <= 3,
+// with the Condon-Shortley phase carried into the real form:
+//   Y_l0 = K_l0 P_l(z);  Y_lm = sqrt2 K_l|m| P_l^|m|(z) {cos m phi, sin |m| phi}.
+// Normalisation constants:
+constexpr float kY0 = 0.28209479177387814f;   // 1 / (2 sqrt(pi))
+constexpr float kY1 = 0.48860251190291992f;   // sqrt(3 / (4 pi))
+constexpr float kY2a = 1.0925484305920792f;   // sqrt(15 / pi) / 2
+constexpr float kY2b = 0.31539156525252005f;  // sqrt(5 / pi) / 4
+constexpr float kY2c = 0.54627421529603959f;  // sqrt(15 / pi) / 4
+constexpr float kY3a = 0.59004358992664352f;  // sqrt(35 / (2 pi)) / 4
+constexpr float kY3b = 2.8906114426405538f;   // sqrt(105 / pi) / 2
+constexpr float kY3c = 0.45704579946446572f;  // sqrt(21 / (2 pi)) / 4
+constexpr float kY3d = 0.37317633259011546f;  // sqrt(7 / pi) / 4
+constexpr float kY3e = 1.4453057213202769f;   // sqrt(105 / pi) / 4
+
+template <int DEG>
+__device__ __forceinline__ void sh_basis(float x, float y, float z, float* Y) {
+  Y[0] = kY0;
+  if (DEG >= 1) {
+    Y[1] = -kY1 * y;
+    Y[2] = kY1 * z;
+    Y[3] = -kY1 * x;
+  }
+  if (DEG >= 2) {
+    float xx = x * x, yy = y * y, zz = z * z;
+    Y[4] = kY2a * x * y;
+    Y[5] = -kY2a * y * z;
+    Y[6] = kY2b * (3.f * zz - 1.f);
+    Y[7] = -kY2a * x * z;
+    Y[8] = kY2c * (xx - yy);
+    if (DEG >= 3) {
+      Y[9] = -kY3a * y * (3.f * xx - yy);
+      Y[10] = kY3b * x * y * z;
+      Y[11] = -kY3c * y * (5.f * zz - 1.f);
+      Y[12] = kY3d * z * (5.f * zz - 3.f);
+      Y[13] = -kY3c * x * (5.f * zz - 1.f);
+      Y[14] = kY3e * z * (xx - yy);
+      Y[15] = -kY3a * x * (xx - 3.f * yy);
+    }
+  }
+}
+
+// Partial derivatives of the polynomials above with respect to x, y, z taken
+// as independent variables (the caller projects onto the sphere's tangent
+// plane, which removes the difference between equivalent forms on the sphere).
+template <int DEG>
+__device__ __forceinline__ void sh_basis_grad(float x, float y, float z, float* gx, float* gy,
+                                              float* gz) {
+  gx[0] = gy[0] = gz[0] = 0.f;
+  if (DEG >= 1) {
+    gx[1] = 0.f;    gy[1] = -kY1;  gz[1] = 0.f;
+    gx[2] = 0.f;    gy[2] = 0.f;   gz[2] = kY1;
+    gx[3] = -kY1;   gy[3] = 0.f;   gz[3] = 0.f;
+  }
+  if (DEG >= 2) {
+    gx[4] = kY2a * y;          gy[4] = kY2a * x;          gz[4] = 0.f;
+    gx[5] = 0.f;               gy[5] = -kY2a * z;         gz[5] = -kY2a * y;
+    gx[6] = 0.f;               gy[6] = 0.f;               gz[6] = 6.f * kY2b * z;
+    gx[7] = -kY2a * z;         gy[7] = 0.f;               gz[7] = -kY2a * x;
+    gx[8] = 2.f * kY2c * x;    gy[8] = -2.f * kY2c * y;   gz[8] = 0.f;
+    if (DEG >= 3) {
+      float xx = x * x, yy = y * y, zz = z * z;
+      gx[9] = -6.f * kY3a * x * y;          gy[9] = -3.f * kY3a * (xx - yy);    gz[9] = 0.f;
+      gx[10] = kY3b * y * z;                gy[10] = kY3b * x * z;              gz[10] = kY3b * x * y;
+      gx[11] = 0.f;                         gy[11] = -kY3c * (5.f * zz - 1.f);  gz[11] = -10.f * kY3c * y * z;
+      gx[12] = 0.f;                         gy[12] = 0.f;                       gz[12] = kY3d * (15.f * zz - 3.f);
+      gx[13] = -kY3c * (5.f * zz - 1.f);    gy[13] = 0.f;                       gz[13] = -10.f * kY3c * x * z;
+      gx[14] = 2.f * kY3e * x * z;          gy[14] = -2.f * kY3e * y * z;       gz[14] = kY3e * (xx - yy);
+      gx[15] = -3.f * kY3a * (xx - yy);     gy[15] = 6.f * kY3a * x * y;        gz[15] = 0.f;
+    }
+  }
+}
+
+// Rotation matrix of the normalised quaternion (w, x, y, z).
+template <typename T>
+__device__ __forceinline__ void quat_to_rot(T w, T x, T y, T z, T R[3][3]) {
+  R[0][0] = T(1) - T(2) * (y * y + z * z);
+  R[0][1] = T(2) * (x * y - w * z);
+  R[0][2] = T(2) * (x * z + w * y);
+  R[1][0] = T(2) * (x * y + w * z);
+  R[1][1] = T(1) - T(2) * (x * x + z * z);
+  R[1][2] = T(2) * (y * z - w * x);
+  R[2][0] = T(2) * (x * z - w * y);
+  R[2][1] = T(2) * (y * z + w * x);
+  R[2][2] = T(1) - T(2) * (x * x + y * y);
+}
+
+__device__ __forceinline__ long long floor_tile(double a) {
+  return static_cast<long long>(floor(a * (1.0 / kTile)));
+}
+
+template <int DEG>
+__global__ void __launch_bounds__(256) k_project(const float4* __restrict__ means,
+                                                 const float4* __restrict__ log_scales,
+                                                 const float4* __restrict__ quats,
+                                                 const float* __restrict__ logit,
+                                                 const float* __restrict__ sh, int n, int n_views,
+                                                 CamSet cams, float4* __restrict__ records,
+                                                 int* __restrict__ radii) {
+  constexpr int K = (DEG + 1) * (DEG + 1);
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float4 m = __ldg(&means[i]);
+  const float4 ls = __ldg(&log_scales[i]);
+  const float4 q = __ldg(&quats[i]);
+  const float lg = __ldg(&logit[i]);
+
+  // view-independent: M = R diag(exp(s)) in double
+  double qw = q.x, qx = q.y, qy = q.z, qz = q.w;
+  double qinv = 1.0 / sqrt(qw * qw + qx * qx + qy * qy + qz * qz);
+  qw *= qinv; qx *= qinv; qy *= qinv; qz *= qinv;
+  double R[3][3];
+  quat_to_rot<double>(qw, qx, qy, qz, R);
+  const double s[3] = {exp((double)ls.x), exp((double)ls.y), exp((double)ls.z)};
+  double M[3][3];
+#pragma unroll
+  for (int a = 0; a < 3; ++a)
+#pragma unroll
+    for (int b = 0; b < 3; ++b) M[a][b] = R[a][b] * s[b];
+  const float opac = (float)(1.0 / (1.0 + exp(-(double)lg)));
+
+  float coef[K * 3];
+  const float* shi = sh + (size_t)i * K * 3;
+#pragma unroll
+  for (int k = 0; k < K * 3; ++k) coef[k] = __ldg(&shi[k]);
+
+  const Grid g = grid_of(cams.c[0]);
+  for (int v = 0; v < n_views; ++v) {
+    const gs_camera& c = cams.c[v];
+    const double mx = m.x, my = m.y, mz = m.z;
+    const double W[3][3] = {{c.viewmat[0], c.viewmat[1], c.viewmat[2]},
+                            {c.viewmat[4], c.viewmat[5], c.viewmat[6]},
+                            {c.viewmat[8], c.viewmat[9], c.viewmat[10]}};
+    const double tx = fma(W[0][0], mx, fma(W[0][1], my, fma(W[0][2], mz, (double)c.viewmat[3])));
+    const double ty = fma(W[1][0], mx, fma(W[1][1], my, fma(W[1][2], mz, (double)c.viewmat[7])));
+    const double tz = fma(W[2][0], mx, fma(W[2][1], my, fma(W[2][2], mz, (double)c.viewmat[11])));
+    // sort key: float32 depth as a fixed chain of correctly rounded fmas of
+    // the float inputs, so it is one well-defined float; it also decides the
+    // near-plane cull
+    const float key = __fmaf_rn(c.viewmat[8], m.x,
+                                __fmaf_rn(c.viewmat[9], m.y, __fmaf_rn(c.viewmat[10], m.z, c.viewmat[11])));
+    float rec[12];
+#pragma unroll
+    for (int k = 0; k < 12; ++k) rec[k] = 0.f;
+    int radius = 0;
+    bool ok = key >= (float)kNear;
+    long long x0 = 1, x1 = 0, y0 = 1, y1 = 0;
+    if (ok) {
+      const double iz = 1.0 / tz;
+      const double fx = c.fx, fy = c.fy;
+      const double a0 = fx * iz, a2 = -fx * tx * iz * iz;
+      const double b1 = fy * iz, b2 = -fy * ty * iz * iz;
+      // rows of T = J W
+      double T0[3], T1[3];
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        T0[j] = a0 * W[0][j] + a2 * W[2][j];
+        T1[j] = b1 * W[1][j] + b2 * W[2][j];
+      }
+      // V = T M, cov2d = V V^T + 0.3 I
+      double V0[3], V1[3];
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        V0[k] = T0[0] * M[0][k] + T0[1] * M[1][k] + T0[2] * M[2][k];
+        V1[k] = T1[0] * M[0][k] + T1[1] * M[1][k] + T1[2] * M[2][k];
+      }
+      const double A = V0[0] * V0[0] + V0[1] * V0[1] + V0[2] * V0[2] + kLowPass;
+      const double B = V0[0] * V1[0] + V0[1] * V1[1] + V0[2] * V1[2];
+      const double C = V1[0] * V1[0] + V1[1] * V1[1] + V1[2] * V1[2] + kLowPass;
+      const double det = A * C - B * B;
+      ok = det > 0.0;
+      if (ok) {
+        const double idet = 1.0 / det;
+        const double mid = 0.5 * (A + C);
+        const double lam = mid + sqrt(0.25 * (A - C) * (A - C) + B * B);
+        double rd = ceil(3.0 * sqrt(lam));
+        if (!(rd <= (double)kMaxRadius)) rd = (double)kMaxRadius;
+        radius = (int)rd;
+        const double u = fx * tx * iz + (double)c.cx;
+        const double vv = fy * ty * iz + (double)c.cy;
+        const long long fx0 = floor_tile(u - radius), fx1 = floor_tile(u + radius);
+        const long long fy0 = floor_tile(vv - radius), fy1 = floor_tile(vv + radius);
+        x0 = fx0 < 0 ? 0 : fx0;
+        x1 = fx1 > g.tiles_x - 1 ? g.tiles_x - 1 : fx1;
+        y0 = fy0 < 0 ? 0 : fy0;
+        y1 = fy1 > g.tiles_y - 1 ? g.tiles_y - 1 : fy1;
+        ok = (x0 <= x1) && (y0 <= y1);
+        if (ok) {
+          rec[R_U] = (float)u;
+          rec[R_V] = (float)vv;
+          rec[R_CA] = (float)(C * idet);
+          rec[R_CB] = (float)(-B * idet);
+          rec[R_CC] = (float)(A * idet);
+          rec[R_OPAC] = opac;
+          rec[R_DEPTH] = key;
+          // colour: SH at the direction from the camera centre to the mean
+          float dxv = m.x - c.campos[0], dyv = m.y - c.campos[1], dzv = m.z - c.campos[2];
+          float inv = rsqrtf(dxv * dxv + dyv * dyv + dzv * dzv);
+          float Y[16];
+          sh_basis<DEG>(dxv * inv, dyv * inv, dzv * inv, Y);
+#pragma unroll
+          for (int ch = 0; ch < 3; ++ch) {
+            float acc = 0.5f;
+#pragma unroll
+            for (int k = 0; k < K; ++k) acc = fmaf(Y[k], coef[k * 3 + ch], acc);
+            rec[R_R + ch] = fmaxf(acc, 0.f);
+          }
+        }
+      }
+    }
+    if (!ok) {
+      radius = 0;
+      x0 = 1; x1 = 0; y0 = 1; y1 = 0;
+#pragma unroll
+      for (int k = 0; k < 10; ++k) rec[k] = 0.f;
+    }
+    rec[R_TX] = __uint_as_float((uint32_t)x0 | ((uint32_t)x1 << 16));
+    rec[R_TY] = __uint_as_float((uint32_t)y0 | ((uint32_t)y1 << 16));
+    float4* out = records + ((size_t)v * n + i) * 3;
+    out[0] = make_float4(rec[0], rec[1], rec[2], rec[3]);
+    out[1] = make_float4(rec[4], rec[5], rec[6], rec[7]);
+    out[2] = make_float4(rec[8], rec[9], rec[10], rec[11]);
+    radii[(size_t)v * n + i] = radius;
+  }
+}
+
+// Backward of k_project for the raw parameters, summing every view in which
+// the Gaussian was visible (radius > 0).
+template <int DEG>
+__global__ void __launch_bounds__(128) k_project_bwd(
+    const float4* __restrict__ means, const float4* __restrict__ log_scales,
+    const float4* __restrict__ quats, const float* __restrict__ logit,
+    const float* __restrict__ sh, const float4* __restrict__ grad2d,
+    const int* __restrict__ radii, int n, int n_views, CamSet cams, float4* __restrict__ g_means,
+    float4* __restrict__ g_log_scales, float4* __restrict__ g_quats, float* __restrict__ g_logit,
+    float* __restrict__ g_sh) {
+  constexpr int K = (DEG + 1) * (DEG + 1);
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float4 m = __ldg(&means[i]);
+  const float4 ls = __ldg(&log_scales[i]);
+  const float4 q = __ldg(&quats[i]);
+  const float lg = __ldg(&logit[i]);
+
+  const float qn2 = q.x * q.x + q.y * q.y + q.z * q.z + q.w * q.w;
+  const float qinv = rsqrtf(qn2);
+  const float qw = q.x * qinv, qx = q.y * qinv, qy = q.z * qinv, qz = q.w * qinv;
+  float R[3][3];
+  quat_to_rot<float>(qw, qx, qy, qz, R);
+  const float s[3] = {__expf(ls.x), __expf(ls.y), __expf(ls.z)};
+  float M[3][3];
+#pragma unroll
+  for (int a = 0; a < 3; ++a)
+#pragma unroll
+    for (int b = 0; b < 3; ++b) M[a][b] = R[a][b] * s[b];
+  const float opac = 1.f / (1.f + __expf(-lg));
+
+  float dM[3][3] = {{0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}};
+  float dmu[3] = {0.f, 0.f, 0.f};
+  float dopac = 0.f;
+  float dsh[K * 3];
+#pragma unroll
+  for (int k = 0; k < K * 3; ++k) dsh[k] = 0.f;
+  const float* shi = sh + (size_t)i * K * 3;
+
+  for (int v = 0; v < n_views; ++v) {
+    if (radii[(size_t)v * n + i] <= 0) continue;
+    const float4* G4 = grad2d + ((size_t)v * n + i) * 3;
+    const float4 ga = G4[0], gb = G4[1], gc = G4[2];
+    const float G[9] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w, gc.x};
+    const gs_camera& c = cams.c[v];
+    const float W[3][3] = {{c.viewmat[0], c.viewmat[1], c.viewmat[2]},
+                           {c.viewmat[4], c.viewmat[5], c.viewmat[6]},
+                           {c.viewmat[8], c.viewmat[9], c.viewmat[10]}};
+    const float tx = W[0][0] * m.x + W[0][1] * m.y + W[0][2] * m.z + c.viewmat[3];
+    const float ty = W[1][0] * m.x + W[1][1] * m.y + W[1][2] * m.z + c.viewmat[7];
+    const float tz = W[2][0] * m.x + W[2][1] * m.y + W[2][2] * m.z + c.viewmat[11];
+    const float iz = 1.f / tz, iz2 = iz * iz;
+    const float fx = c.fx, fy = c.fy;
+    const float a0 = fx * iz, a2 = -fx * tx * iz2, b1 = fy * iz, b2 = -fy * ty * iz2;
+    float T0[3], T1[3];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      T0[j] = a0 * W[0][j] + a2 * W[2][j];
+      T1[j] = b1 * W[1][j] + b2 * W[2][j];
+    }
+    float V0[3], V1[3];
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      V0[k] = T0[0] * M[0][k] + T0[1] * M[1][k] + T0[2] * M[2][k];
+      V1[k] = T1[0] * M[0][k] + T1[1] * M[1][k] + T1[2] * M[2][k];
+    }
+    const float n0 = V0[0] * V0[0] + V0[1] * V0[1] + V0[2] * V0[2];
+    const float n1 = V1[0] * V1[0] + V1[1] * V1[1] + V1[2] * V1[2];
+    const float A = n0 + 0.3f;
+    const float B = V0[0] * V1[0] + V0[1] * V1[1] + V0[2] * V1[2];
+    const float C = n1 + 0.3f;
+    // det = (A-0.3)(C-0.3) - B^2 + 0.3 (A + C - 0.6) + 0.09, with the first
+    // part written as |V0 x V1|^2 (Lagrange's identity) to avoid cancellation
+    const float cx_ = V0[1] * V1[2] - V0[2] * V1[1];
+    const float cy_ = V0[2] * V1[0] - V0[0] * V1[2];
+    const float cz_ = V0[0] * V1[1] - V0[1] * V1[0];
+    const float det = cx_ * cx_ + cy_ * cy_ + cz_ * cz_ + 0.3f * (n0 + n1) + 0.09f;
+    const float id2 = 1.f / (det * det);
+    // conic (a, b, c) = (C, -B, A) / det
+    const float dA = (-C * C * G[G_CA] + B * C * G[G_CB] - B * B * G[G_CC]) * id2;
+    const float dB = (2.f * B * C * G[G_CA] - (A * C + B * B) * G[G_CB] + 2.f * A * B * G[G_CC]) * id2;
+    const float dC = (-B * B * G[G_CA] + A * B * G[G_CB] - A * A * G[G_CC]) * id2;
+    float dV0[3], dV1[3];
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      dV0[k] = 2.f * dA * V0[k] + dB * V1[k];
+      dV1[k] = dB * V0[k] + 2.f * dC * V1[k];
+    }
+    float dT0[3], dT1[3];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      dT0[j] = dV0[0] * M[j][0] + dV0[1] * M[j][1] + dV0[2] * M[j][2];
+      dT1[j] = dV1[0] * M[j][0] + dV1[1] * M[j][1] + dV1[2] * M[j][2];
+#pragma unroll
+      for (int k = 0; k < 3; ++k) dM[j][k] += T0[j] * dV0[k] + T1[j] * dV1[k];
+    }
+    const float da0 = dT0[0] * W[0][0] + dT0[1] * W[0][1] + dT0[2] * W[0][2];
+    const float da2 = dT0[0] * W[2][0] + dT0[1] * W[2][1] + dT0[2] * W[2][2];
+    const float db1 = dT1[0] * W[1][0] + dT1[1] * W[1][1] + dT1[2] * W[1][2];
+    const float db2 = dT1[0] * W[2][0] + dT1[1] * W[2][1] + dT1[2] * W[2][2];
+    const float gu = G[G_U], gv = G[G_V];
+    const float dtx = gu * fx * iz - da2 * fx * iz2;
+    const float dty = gv * fy * iz - db2 * fy * iz2;
+    const float dtz = -gu * fx * tx * iz2 - gv * fy * ty * iz2 - da0 * fx * iz2 - db1 * fy * iz2 +
+                      2.f * da2 * fx * tx * iz2 * iz + 2.f * db2 * fy * ty * iz2 * iz;
+#pragma unroll
+    for (int j = 0; j < 3; ++j) dmu[j] += W[0][j] * dtx + W[1][j] * dty + W[2][j] * dtz;
+    dopac += G[G_OPAC];
+
+    // colour: rgb_c = max(0, sum_k Y_k(d) sh_kc + 0.5), d = normalize(mu - campos)
+    const float wx = m.x - c.campos[0], wy = m.y - c.campos[1], wz = m.z - c.campos[2];
+    const float winv = rsqrtf(wx * wx + wy * wy + wz * wz);
+    const float dx = wx * winv, dy = wy * winv, dz = wz * winv;
+    float Y[16], gx[16], gy[16], gz[16];
+    sh_basis<DEG>(dx, dy, dz, Y);
+    sh_basis_grad<DEG>(dx, dy, dz, gx, gy, gz);
+    float gdx = 0.f, gdy = 0.f, gdz = 0.f;
+#pragma unroll
+    for (int ch = 0; ch < 3; ++ch) {
+      float raw = 0.5f;
+#pragma unroll
+      for (int k = 0; k < K; ++k) raw = fmaf(Y[k], __ldg(&shi[k * 3 + ch]), raw);
+      if (!(raw > 0.f)) continue;
+      const float gcol = G[G_R + ch];
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        const float cf = __ldg(&shi[k * 3 + ch]);
+        dsh[k * 3 + ch] += Y[k] * gcol;
+        gdx += gcol * cf * gx[k];
+        gdy += gcol * cf * gy[k];
+        gdz += gcol * cf * gz[k];
+      }
+    }
+    // through d = w / |w|: (I - d d^T) / |w|
+    const float dd = gdx * dx + gdy * dy + gdz * dz;
+    dmu[0] += (gdx - dx * dd) * winv;
+    dmu[1] += (gdy - dy * dd) * winv;
+    dmu[2] += (gdz - dz * dd) * winv;
+  }
+
+  // M = R diag(s): dL/ds_k = sum_j dM_jk R_jk, dL/dR_jk = dM_jk s_k
+  float dls[3];
+#pragma unroll
+  for (int k = 0; k < 3; ++k)
+    dls[k] = (dM[0][k] * R[0][k] + dM[1][k] * R[1][k] + dM[2][k] * R[2][k]) * s[k];
+  float dR[3][3];
+#pragma unroll
+  for (int j = 0; j < 3; ++j)
+#pragma unroll
+    for (int k = 0; k < 3; ++k) dR[j][k] = dM[j][k] * s[k];
+  // rotation matrix entries as functions of the unit quaternion (w, x, y, z)
+  float dqw = 2.f * (-qz * dR[0][1] + qy * dR[0][2] + qz * dR[1][0] - qx * dR[1][2] -
+                     qy * dR[2][0] + qx * dR[2][1]);
+  float dqx = 2.f * (qy * dR[0][1] + qz * dR[0][2] + qy * dR[1][0] - qw * dR[1][2] +
+                     qz * dR[2][0] + qw * dR[2][1]) -
+              4.f * qx * (dR[1][1] + dR[2][2]);
+  float dqy = 2.f * (qx * dR[0][1] + qw * dR[0][2] + qx * dR[1][0] + qz * dR[1][2] -
+                     qw * dR[2][0] + qz * dR[2][1]) -
+              4.f * qy * (dR[0][0] + dR[2][2]);
+  float dqz = 2.f * (-qw * dR[0][1] + qx * dR[0][2] + qw * dR[1][0] + qy * dR[1][2] +
+                     qx * dR[2][0] + qy * dR[2][1]) -
+              4.f * qz * (dR[0][0] + dR[1][1]);
+  // through the normalisation q_hat = q / |q|
+  const float proj = dqw * qw + dqx * qx + dqy * qy + dqz * qz;
+  dqw = (dqw - qw * proj) * qinv;
+  dqx = (dqx - qx * proj) * qinv;
+  dqy = (dqy - qy * proj) * qinv;
+  dqz = (dqz - qz * proj) * qinv;
+
+  g_means[i] = make_float4(dmu[0], dmu[1], dmu[2], 0.f);
+  g_log_scales[i] = make_float4(dls[0], dls[1], dls[2], 0.f);
+  g_quats[i] = make_float4(dqw, dqx, dqy, dqz);
+  g_logit[i] = dopac * opac * (1.f - opac);
+  float* gsh = g_sh + (size_t)i * K * 3;
+#pragma unroll
+  for (int k = 0; k < K * 3; ++k) gsh[k] = dsh[k];
+}
+
+}  // namespace
+
+cudaError_t launch_project(const gs_params& p, const CamSet& cams, int n_views, float* records,
+                           int* radii, cudaStream_t stream) {
+  const int n = (int)p.n;
+  if (n == 0) return cudaSuccess;
+  const int threads = 256;
+  const int blocks = (n + threads - 1) / threads;
+  auto m = reinterpret_cast<const float4*>(p.means);
+  auto s = reinterpret_cast<const float4*>(p.log_scales);
+  auto q = reinterpret_cast<const float4*>(p.quats);
+  auto r = reinterpret_cast<float4*>(records);
+  switch (p.sh_degree) {
+    case 0: k_project<0><<<blocks, threads, 0, stream>>>(m, s, q, p.opacity_logit, p.sh, n, n_views, cams, r, radii); break;
+    case 1: k_project<1><<<blocks, threads, 0, stream>>>(m, s, q, p.opacity_logit, p.sh, n, n_views, cams, r, radii); break;
+    case 2: k_project<2><<<blocks, threads, 0, stream>>>(m, s, q, p.opacity_logit, p.sh, n, n_views, cams, r, radii); break;
+    default: k_project<3><<<blocks, threads, 0, stream>>>(m, s, q, p.opacity_logit, p.sh, n, n_views, cams, r, radii); break;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_project_bwd(const gs_params& p, const CamSet& cams, int n_views,
+                               const float* grad2d, const int* radii, const gs_grads& g,
+                               cudaStream_t stream) {
+  const int n = (int)p.n;
+  if (n == 0) return cudaSuccess;
+  const int threads = 128;
+  const int blocks = (n + threads - 1) / threads;
+  auto m = reinterpret_cast<const float4*>(p.means);
+  auto s = reinterpret_cast<const float4*>(p.log_scales);
+  auto q = reinterpret_cast<const float4*>(p.quats);
+  auto g2 = reinterpret_cast<const float4*>(grad2d);
+  auto gm = reinterpret_cast<float4*>(g.means);
+  auto gs = reinterpret_cast<float4*>(g.log_scales);
+  auto gq = reinterpret_cast<float4*>(g.quats);
+#define GS_PBWD(D) k_project_bwd<D><<<blocks, threads, 0, stream>>>(m, s, q, p.opacity_logit, p.sh, g2, radii, n, n_views, cams, gm, gs, gq, g.opacity_logit, g.sh)
+  switch (p.sh_degree) {
+    case 0: GS_PBWD(0); break;
+    case 1: GS_PBWD(1); break;
+    case 2: GS_PBWD(2); break;
+    default: GS_PBWD(3); break;
+  }
+#undef GS_PBWD
+  return cudaGetLastError();
+}
+
+}  // namespace gsb

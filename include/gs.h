@@ -1,0 +1,270 @@
+/*
+ * gs.h -- C ABI of the B200 (sm_100a) differentiable EWA Gaussian-splatting
+ * library (libgs_b200.so).
+ *
+ * The calls follow the pipeline the pages state: project the 3D Gaussians,
+ * assign them to tiles and depth-sort, blend per pixel, and differentiate it
+ * ("Better Gaussian Splatting in Julia", pwwt.cn, sec. 3.2-3.3 and 5.4; the
+ * second Julia page, lshu.cn, sec. 3.2 `rasterize` pseudocode and sec. 1
+ * capability table), accumulate the plain and absolute view-space gradients
+ * used for densification (jsqmd.com, sec. 2 table and sec. 3.1), and take one
+ * Adam step over every parameter (lshu.cn sec. 3.3 and 5.3).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every array argument is a DEVICE pointer owned by the caller, except the
+ *    camera array, the background colour and the Adam group table, which are
+ *    HOST pointers read before the call returns. The library never allocates
+ *    or frees device memory and keeps no state between calls.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream). Every call only enqueues work on that stream and returns
+ *    without synchronising, except gs_get_status.
+ *  - Argument errors are detected on the host before anything is enqueued and
+ *    returned at once (GS_ERR_INVALID_ARG, GS_ERR_OVERFLOW). A failed launch
+ *    returns GS_ERR_CUDA. Conditions only the device can see (pair capacity
+ *    exceeded, a bounded wait that gave up) are OR-ed into the status word at
+ *    the start of the workspace and read back by gs_get_status.
+ *  - Pixel (x, y) has its centre at (x + 0.5, y + 0.5); tiles are 16 x 16
+ *    pixels; tile index within a view is ty * tiles_x + tx, and the global
+ *    tile index of view v is v * tiles_per_view + tile.
+ *  - All views of one call share width and height.
+ */
+#ifndef GS_B200_H
+#define GS_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GS_ABI_VERSION 1
+#define GS_TILE 16            /* tile edge in pixels */
+#define GS_MAX_VIEWS 32       /* views per call */
+#define GS_RECORD_FLOATS 12   /* floats per projected record */
+#define GS_GRAD2D_FLOATS 12   /* floats per screen-space gradient record */
+
+typedef enum gs_status {
+  GS_OK = 0,
+  GS_ERR_INVALID_ARG = 1,     /* bad pointer, size, degree, view count, layout */
+  GS_ERR_CAPACITY = 2,        /* more Gaussian x tile pairs than pair_capacity */
+  GS_ERR_OVERFLOW = 3,        /* a size exceeds a 32-bit field it must fit */
+  GS_ERR_DEVICE_TIMEOUT = 4,  /* a bounded device-side wait gave up */
+  GS_ERR_NONFINITE = 5,       /* reserved: non-finite input detected */
+  GS_ERR_CUDA = 6             /* a CUDA runtime call or launch failed */
+} gs_status;
+
+/* Sort strategy of gs_bin_sort; both give bit-identical per-tile lists. */
+typedef enum gs_sort_mode {
+  /* Emit one 64-bit key (global tile << 32 | float bits of depth) per
+   * Gaussian x tile pair and radix-sort the keys (least significant digit
+   * first, 8-bit digits, single-sweep passes). */
+  GS_SORT_FULL64 = 0,
+  /* Radix-sort the Gaussians of each view once by (view << 32 | depth bits),
+   * emit the pairs in that order, then radix-sort the pairs stably by global
+   * tile alone. Same order as FULL64, fewer bytes per pair. */
+  GS_SORT_PRESORT = 1
+} gs_sort_mode;
+
+/* Pinhole camera (lshu.cn sec. 3.2: "camera intrinsics and extrinsics").
+ * viewmat: row-major 3x4 [R | t] mapping world to camera coordinates
+ * (x right, y down, z forward). u = fx * x / z + cx, v = fy * y / z + cy.
+ * campos: camera centre in world coordinates (origin of the SH view
+ * direction). 88 bytes. */
+typedef struct gs_camera {
+  float viewmat[12];
+  float fx, fy, cx, cy;
+  int32_t width, height;
+  float campos[3];
+  float reserved;
+} gs_camera;
+
+/* Raw (un-activated) Gaussian parameters, structure of arrays
+ * (pwwt.cn sec. 1.1 and 3.1; lshu.cn sec. 3.1 table):
+ *   means          float [n][4]  x, y, z, (pad, ignored)
+ *   log_scales     float [n][4]  log of the per-axis scale, (pad, ignored)
+ *   quats          float [n][4]  rotation quaternion w, x, y, z (normalised
+ *                                inside; need not be unit)
+ *   opacity_logit  float [n]     opacity = sigmoid(logit)
+ *   sh             float [n][(sh_degree+1)^2][3]  real SH colour coefficients
+ * The float4 arrays must be 16-byte aligned. */
+typedef struct gs_params {
+  const float* means;
+  const float* log_scales;
+  const float* quats;
+  const float* opacity_logit;
+  const float* sh;
+  int32_t sh_degree;  /* 0..3 */
+  int32_t reserved;
+  int64_t n;          /* number of Gaussians, 0 <= n < 2^31 */
+} gs_params;
+
+/* Gradients of the raw parameters: same layouts as gs_params (pad lanes are
+ * written as 0). Overwritten, not accumulated, by gs_rasterize_bwd. */
+typedef struct gs_grads {
+  float* means;
+  float* log_scales;
+  float* quats;
+  float* opacity_logit;
+  float* sh;
+} gs_grads;
+
+/* Output of gs_project, per view v and Gaussian i (record index v*n + i):
+ * records [n_views][n][12] floats, 16-byte aligned:
+ *   0 u        1 v          pixel coordinates of the mean
+ *   2 conic_a  3 conic_b    4 conic_c   inverse 2D covariance [[a, b], [b, c]]
+ *   5 opacity  6 r  7 g  8 b            activated opacity, colour
+ *   9 depth                 camera-space z, rounded to float (the sort key)
+ *  10 tile_x  (bits) tx0 | tx1 << 16   inclusive tile range touched
+ *  11 tile_y  (bits) ty0 | ty1 << 16   (tx0 > tx1 marks a culled Gaussian)
+ * radii [n_views][n] int32: ceil(3 sqrt(lambda_max)) of the 2D covariance,
+ *   0 when culled (the densification visibility filter). */
+typedef struct gs_projected {
+  float* records;
+  int32_t* radii;
+} gs_projected;
+
+/* Output of gs_bin_sort.
+ *   ids     uint32 [pair_capacity]  Gaussian index (within its view) of each
+ *           pair, ordered by global tile, then depth key, then index
+ *   ranges  int64 [n_views * tiles_per_view][2]  [start, end) of each tile's
+ *           slice of ids (start == end for an empty tile)
+ *   n_pairs int64 [1]  number of pairs (always written, also on overflow) */
+typedef struct gs_binned {
+  uint32_t* ids;
+  int64_t* ranges;
+  int64_t* n_pairs;
+  int64_t pair_capacity;
+} gs_binned;
+
+/* One Adam parameter group (lshu.cn sec. 3.3 per-group learning rates). */
+typedef struct gs_adam_group {
+  float* param;
+  const float* grad;
+  float* exp_avg;     /* first moment m */
+  float* exp_avg_sq;  /* second moment v */
+  int64_t count;      /* floats in the group */
+  float lr;
+  float reserved;
+} gs_adam_group;
+
+/* ABI version of the loaded library (GS_ABI_VERSION). */
+int32_t gs_abi_version(void);
+
+/* Static text for a status code. */
+const char* gs_status_string(gs_status status);
+
+/* Bytes of workspace gs_bin_sort needs for n Gaussians, n_views views of
+ * cams[0]'s size, pair_capacity pairs and the given sort mode. Returns 0 for
+ * invalid arguments. The workspace must be 256-byte aligned; its first 256
+ * bytes hold the device status word and counters; zero them once (e.g.
+ * cudaMemset) before the workspace is first used. */
+size_t gs_workspace_size(int64_t n, int32_t n_views, const gs_camera* cams,
+                         int64_t pair_capacity, int32_t sort_mode);
+
+/* EWA projection (pwwt.cn sec. 3.2 `project_gaussian`: world -> camera ->
+ * pixel with division by depth, covariance through the Jacobian of that map;
+ * lshu.cn sec. 3.2). Per view and Gaussian: R from the normalised quaternion,
+ * Sigma = R diag(exp(2 s)) R^T, t = W mu + T, J = [[fx/z, 0, -fx x/z^2],
+ * [0, fy/z, -fy y/z^2]], cov2d = J W Sigma W^T J^T + 0.3 I, conic = cov2d^-1,
+ * radius = ceil(3 sqrt(lambda_max)), colour = max(0, sum_k Y_k(d) sh_k + 0.5)
+ * with d = normalize(mu - campos), opacity = sigmoid(logit), tile rectangle
+ * floor((u -+ radius)/16) clamped to the grid. Culled when z < 0.2, the 2D
+ * covariance is not positive definite, or the rectangle is empty.
+ * Geometry (camera-space mean, covariance, radius, rectangle, depth key) is
+ * evaluated in double precision and rounded to float at the end; colour in
+ * float. Writes out->records and out->radii for all n_views * n records. */
+gs_status gs_project(const gs_params* params, const gs_camera* cams, int32_t n_views,
+                     gs_projected* out, void* stream);
+
+/* Tile binning with depth sort (pwwt.cn sec. 3.3 steps 1-2 and 4.3 tiles;
+ * lshu.cn sec. 3.2 `assign_to_tiles` and `sort_by_depth!`). Every Gaussian
+ * with a non-empty rectangle emits one pair per tile it touches; the pairs
+ * are ordered by global tile, then by the float bits of its depth key, then
+ * by Gaussian index (the order of a stable sort on the 64-bit key
+ * tile << 32 | depth bits over pairs emitted in index order).
+ * `n` is the per-view Gaussian count used by gs_project. `ws` must hold
+ * gs_workspace_size(n, n_views, cams, out->pair_capacity, sort_mode) bytes.
+ * If more than pair_capacity pairs are needed, nothing is emitted, n_pairs
+ * still receives the count, every range is empty and GS_ERR_CAPACITY is
+ * raised in the status word. */
+gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n_views,
+                      int64_t n, int32_t sort_mode, gs_binned* out, void* ws,
+                      size_t ws_bytes, void* stream);
+
+/* Forward rasterisation, one 16x16 tile per thread block and one thread per
+ * pixel (pwwt.cn sec. 5.4 tile mode; lshu.cn sec. 3.2 `blend`, sec. 7.3).
+ * For each pixel, front to back over its tile's list:
+ *   alpha = min(0.99, o exp(-q/2)), q = d^T conic d, d = pixel centre - mean;
+ *   skip when alpha < 1/255; T' = T (1 - alpha); stop (without adding it)
+ *   when T' < 1e-4; C += colour * alpha * T; T = T'.
+ * Then C += T * bg[c]. Outputs (device):
+ *   image     float [n_views][3][H][W]
+ *   final_T   float [n_views][H][W]  transmittance after the last contributor
+ *   n_contrib uint32 [n_views][H][W] 1 + position in the tile's list of the
+ *             last contributing Gaussian (0 if none)
+ * `bg` is a host pointer to 3 floats. */
+gs_status gs_rasterize_fwd(const gs_projected* proj, const gs_binned* bins,
+                           const gs_camera* cams, int32_t n_views, int64_t n,
+                           const float* bg, float* image, float* final_T,
+                           uint32_t* n_contrib, void* stream);
+
+/* Backward of gs_rasterize_fwd and gs_project (lshu.cn sec. 1
+ * "differentiable rasterisation"). Given dL/dimage [n_views][3][H][W] and the
+ * forward's final_T and n_contrib, replays each pixel's list back to front
+ * and writes, per view and Gaussian, grad2d [n_views][n][12]:
+ *   0 dL/du  1 dL/dv  2 dL/dconic_a  3 dL/dconic_b  4 dL/dconic_c
+ *   5 dL/dopacity  6..8 dL/d(r, g, b)
+ *   9 sum over pixels of ||(dL/du, dL/dv)|| (the absolute view-space
+ *     gradient, jsqmd.com sec. 2 table)   10, 11 zero
+ * (0 and 1 together are the view's plain view-space gradient), then the
+ * gradients of the raw parameters summed over views into *grads
+ * (overwritten; see gs_project_bwd). grad2d is overwritten. With
+ * grads == NULL only grad2d is computed. */
+gs_status gs_rasterize_bwd(const gs_params* params, const gs_projected* proj,
+                           const gs_binned* bins, const gs_camera* cams, int32_t n_views,
+                           const float* bg, const float* dL_dimage, const float* final_T,
+                           const uint32_t* n_contrib, float* grad2d, gs_grads* grads,
+                           void* stream);
+
+/* Projection backward alone (the second half of gs_rasterize_bwd): the
+ * gradients of the raw parameters from the screen-space gradients grad2d
+ * [n_views][n][12] (fields 0..8 as written by gs_rasterize_bwd), summed over
+ * the views in which radii[v][i] > 0, by the chain rule of gs_project:
+ * conic -> 2D covariance -> (J W, R, scale) -> log-scale, quaternion (through
+ * its normalisation), mean (through J and the pixel coordinates); colour ->
+ * SH coefficients and, through the view direction, the mean; opacity ->
+ * logit. *grads is overwritten. */
+gs_status gs_project_bwd(const gs_params* params, const gs_camera* cams, int32_t n_views,
+                         const int32_t* radii, const float* grad2d, gs_grads* grads,
+                         void* stream);
+
+/* Densification statistics (jsqmd.com sec. 2 table and sec. 3.1
+ * `add_densification_stats`): for each view v and Gaussian i with
+ * radii[v][i] > 0, accumulate
+ *   accum_plain[i] += ||(grad2d[v][i][0], grad2d[v][i][1])||,
+ *   accum_abs[i]   += grad2d[v][i][9],
+ *   denom[i]       += 1.
+ * The three outputs accumulate across calls (the caller zeroes them). */
+gs_status gs_densify_stats(const float* grad2d, const int32_t* radii, int32_t n_views,
+                           int64_t n, float* accum_plain, float* accum_abs,
+                           int32_t* denom, void* stream);
+
+/* Adam step over up to 8 groups (lshu.cn sec. 3.3 and 5.3; Kingma and Ba):
+ * m = b1 m + (1-b1) g; v = b2 v + (1-b2) g^2;
+ * p -= lr * (m / (1 - b1^step)) / (sqrt(v / (1 - b2^step)) + eps).
+ * `groups` is a host array; step >= 1. Each group's arrays must be 16-byte
+ * aligned. */
+gs_status gs_adam_step(const gs_adam_group* groups, int32_t n_groups, float beta1,
+                       float beta2, float eps, int64_t step, void* stream);
+
+/* Synchronise `stream`, return the status word accumulated in workspace `ws`
+ * by device-side checks since the last call, and clear it. */
+gs_status gs_get_status(void* ws, void* stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* GS_B200_H */

@@ -194,6 +194,7 @@ struct Proj {
   S opacity;
   S rgb[3];
   double depth;    // camera-space z of the mean
+  float key;       // float32 depth (the sort key), see project_one
   double lam;      // larger eigenvalue of the 2D covariance
   int valid;
   int clamp_mask;  // bit c set when colour channel c was clamped at 0
@@ -209,7 +210,14 @@ Proj<S> project_one(const S mu[3], const S ls[3], const S q[4], const S& logit,
   for (int i = 0; i < 3; ++i)
     t[i] = cam.R[i][0] * mu[0] + cam.R[i][1] * mu[1] + cam.R[i][2] * mu[2] + cam.t[i];
   P.depth = val(t[2]);
-  P.valid = P.depth >= kNear ? 1 : 0;
+  // The sort key is a float: the depth is taken in float32 as the fused
+  // multiply-add chain fma(R20, x, fma(R21, y, fma(R22, z, t2))) of the float
+  // inputs (every step correctly rounded), so that it is one well-defined
+  // float; the near-plane cull compares that float with 0.2f.
+  P.key = std::fma((float)cam.R[2][0], (float)val(mu[0]),
+                   std::fma((float)cam.R[2][1], (float)val(mu[1]),
+                            std::fma((float)cam.R[2][2], (float)val(mu[2]), (float)cam.t[2])));
+  P.valid = P.key >= (float)kNear ? 1 : 0;
   // rotation matrix of the normalised quaternion (w, x, y, z)
   S qn = dsqrt(q[0] * q[0] + q[1] * q[1] + q[2] * q[2] + q[3] * q[3]);
   S w = q[0] / qn, x = q[1] / qn, y = q[2] / qn, z = q[3] / qn;
@@ -310,14 +318,15 @@ void orc_sh_basis(int64_t n, const double* dirs, int deg, double* out) {
 //   geom[n][16]: u, v, depth, A, B, C, conic a, b, c, opacity, r, g, b, lam,
 //                3 sqrt(lam), camera-space z
 //   ints[n][8]: valid, radius, tx0, tx1, ty0, ty1, clamp_mask, ambiguous
-//   depth_key[n]: float32 rounding of depth (the sort key)
+//   depth_key[n]: float32 depth (the sort key)
 // A Gaussian is culled (valid 0, radius 0, empty rectangle) when its depth is
 // below the near plane, its 2D covariance is not positive definite, or its
 // tile rectangle is empty after clamping to the grid. `ambiguous` is set when a
-// discrete decision (ceil of the radius, floor of a rectangle edge, the near
-// plane, the float32 rounding of the depth) lies within `tol` (relative) of its
-// threshold, so that a float64 computation in another order may decide it the
-// other way.
+// discrete decision taken on a double (ceil of the radius, floor of a
+// rectangle edge) lies within `tol` (relative) of its threshold, so that a
+// double computation in another order may decide it the other way. The depth
+// key and the near-plane cull are float32 decisions defined exactly (see
+// project_one) and are never ambiguous.
 void orc_project(int64_t n, const double* means, const double* log_scales, const double* quats,
                  const double* logit, const double* sh, int deg, const double* cam_packed,
                  double tol, double* geom, int32_t* ints, float* depth_key) {
@@ -348,13 +357,7 @@ void orc_project(int64_t n, const double* means, const double* log_scales, const
       y1 = std::min((long long)cam.tiles_y - 1, tile_floor(e[3]));
       if (x0 > x1 || y0 > y1) { P.valid = 0; }
     }
-    if (std::fabs(P.depth - kNear) < tol * kNear) amb = 1;
-    float key = (float)P.depth;
-    if (std::isfinite(P.depth) && P.depth > 0) {
-      double lo = (double)std::nextafter(key, 0.0f), hi = (double)std::nextafter(key, 1e30f);
-      double m0 = 0.5 * (lo + (double)key), m1 = 0.5 * (hi + (double)key);
-      if (std::fabs(P.depth - m0) < tol * P.depth || std::fabs(P.depth - m1) < tol * P.depth) amb = 1;
-    }
+    float key = P.key;
     if (!P.valid) { r = 0; x0 = 1; x1 = 0; y0 = 1; y1 = 0; }
     o[0] = P.valid; o[1] = (int32_t)r;
     o[2] = (int32_t)x0; o[3] = (int32_t)x1; o[4] = (int32_t)y0; o[5] = (int32_t)y1;

@@ -91,7 +91,7 @@ def _raw(scene):
             _f64(scene.opacity_logit), _f64(scene.sh.reshape(n, k, 3)))
 
 
-def project(scene, cam, tol: float = 1e-9) -> Dict[str, np.ndarray]:
+def project(scene, cam, tol: float = 1e-12) -> Dict[str, np.ndarray]:
     """Project every Gaussian of ``scene`` into ``cam`` (float64)."""
     m, s, q, lg, sh = _raw(scene)
     n = scene.n
@@ -109,7 +109,7 @@ def project(scene, cam, tol: float = 1e-9) -> Dict[str, np.ndarray]:
         clamp=ints[:, 6].copy(), ambiguous=ints[:, 7].copy(), key=key)
 
 
-def project_views(scene, tol: float = 1e-9) -> List[Dict[str, np.ndarray]]:
+def project_views(scene, tol: float = 1e-12) -> List[Dict[str, np.ndarray]]:
     return [project(scene, c, tol) for c in scene.cameras]
 
 

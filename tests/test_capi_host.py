@@ -1,0 +1,77 @@
+"""Host-side checks of the C-ABI library that need no GPU: it loads, exports
+every function include/gs.h declares, and rejects bad arguments before any
+CUDA call."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from gaussian_splatting_differentiable_ewa_b200 import api
+from gaussian_splatting_differentiable_ewa_b200 import scenes as S
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "gs.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gs_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = api.lib()
+    names = _declared()
+    assert len(names) >= 10
+    for name in names:
+        assert hasattr(L, name), name
+    assert {s[0] for s in api.SIGNATURES} == set(names)
+
+
+def test_abi_version_and_status_strings():
+    assert api.gs_abi_version() == 1
+    for s in range(7):
+        assert api.status_string(s) not in ("", "unknown status")
+
+
+def test_workspace_size_validates_and_grows():
+    sc = S.make_scene("train_1m_1080p", n=1000)
+    cams = api.cameras(sc.cameras)
+    a = api.gs_workspace_size(1000, cams, 1, 10_000, api.GS_SORT_FULL64)
+    b = api.gs_workspace_size(1000, cams, 1, 1_000_000, api.GS_SORT_FULL64)
+    c = api.gs_workspace_size(1000, cams, 1, 1_000_000, api.GS_SORT_PRESORT)
+    assert 0 < a < b and c > 0
+    assert b - a >= (1_000_000 - 10_000) * 20  # two 8-byte key buffers + 4-byte ids
+    assert api.gs_workspace_size(-1, cams, 1, 10, 0) == 0
+    assert api.gs_workspace_size(10, cams, 0, 10, 0) == 0
+    assert api.gs_workspace_size(10, cams, 1, -5, 0) == 0
+    assert api.gs_workspace_size(10, cams, 1, 10, 7) == 0
+    # views of different sizes are rejected
+    two = api.cameras([sc.cameras[0], S.make_scene("fwd_1k_128", n=1).cameras[0]])
+    assert api.gs_workspace_size(10, two, 2, 10, 0) == 0
+
+
+def test_bad_arguments_are_rejected_before_any_cuda_call():
+    L = api.lib()
+    sc = S.make_scene("fwd_1k_128", n=10)
+    cams = api.cameras(sc.cameras)
+    p = api.GsParams(None, None, None, None, None, 0, 0, 10)
+    out = api.GsProjected(None, None)
+    assert L.gs_project(ctypes.byref(p), cams, 1, ctypes.byref(out), None) == api.GS_ERR_INVALID_ARG
+    p.sh_degree = 4
+    assert L.gs_project(ctypes.byref(p), cams, 1, ctypes.byref(out), None) == api.GS_ERR_INVALID_ARG
+    p.n = 1 << 31
+    p.sh_degree = 0
+    assert L.gs_project(ctypes.byref(p), cams, 1, ctypes.byref(out), None) == api.GS_ERR_OVERFLOW
+    assert L.gs_project(ctypes.byref(p), cams, 0, ctypes.byref(out), None) == api.GS_ERR_INVALID_ARG
+    b = api.GsBinned(None, None, None, 10)
+    assert L.gs_bin_sort(ctypes.byref(out), cams, 1, 10, 0, ctypes.byref(b), None, 0, None) == \
+        api.GS_ERR_INVALID_ARG
+    grp = (api.GsAdamGroup * 1)()
+    assert L.gs_adam_step(grp, 1, 0.9, 0.999, 1e-15, 0, None) == api.GS_ERR_INVALID_ARG
+    assert L.gs_adam_step(grp, 9, 0.9, 0.999, 1e-15, 1, None) == api.GS_ERR_INVALID_ARG
+    assert L.gs_adam_step(grp, 1, 1.5, 0.999, 1e-15, 1, None) == api.GS_ERR_INVALID_ARG
+    assert L.gs_densify_stats(None, None, 0, 10, None, None, None, None) == api.GS_ERR_INVALID_ARG
+    assert L.gs_get_status(None, None) == api.GS_ERR_INVALID_ARG

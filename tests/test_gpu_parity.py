@@ -1,0 +1,290 @@
+"""CUDA path (through the C ABI) against the float64 oracle on seeded inputs.
+
+Small cases run the whole image; larger ones a seeded pixel sample plus full
+tile rows. Every case spans several tiles and a ragged last tile row/column.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from gaussian_splatting_differentiable_ewa_b200 import api
+from gaussian_splatting_differentiable_ewa_b200 import scenes as S
+from gaussian_splatting_differentiable_ewa_b200.pipeline import Splatter
+from oracle import oracle as O
+
+import parity as P
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    ("fwd_1k_128", dict(), "full"),
+    ("fwd_100k_800", dict(n=20000, width=792, height=600), "full"),
+    ("train_1m_1080p", dict(n=40000), "sample"),
+    ("train_6m_8x1080p", dict(n=20000, n_views=3), "sample"),
+]
+MODES = [api.GS_SORT_FULL64, api.GS_SORT_PRESORT]
+
+
+def _pixels(scene, how):
+    return P.full_pixels(scene) if how == "full" else P.pixel_sample(scene)
+
+
+def _setup(name, kw, mode=api.GS_SORT_PRESORT):
+    sc = S.make_scene(name, **kw)
+    sp = Splatter(sc, sort_mode=mode)
+    sp.ensure_capacity()
+    torch.cuda.synchronize()
+    return sc, sp
+
+
+@pytest.mark.parametrize("name,kw,how", CASES)
+def test_project_matches_oracle(name, kw, how):
+    sc = S.make_scene(name, **kw)
+    sp = Splatter(sc, pair_capacity=1)
+    sp.project()
+    torch.cuda.synchronize()
+    rec = sp.records.cpu().numpy()
+    radii = sp.radii.cpu().numpy()
+    for v, p in enumerate(O.project_views(sc)):
+        g = P.unpack_records(rec[v])
+        amb = p["ambiguous"] != 0
+        assert amb.mean() < 1e-3
+        vo = p["valid"] != 0
+        assert np.array_equal(vo[~amb], (radii[v] > 0)[~amb])
+        m = vo & ~amb
+        assert m.sum() > 0.5 * sc.n
+        assert np.array_equal(radii[v][m], p["radius"][m])
+        assert np.array_equal(g["rect"][m], p["rect"][m])
+        assert np.array_equal(g["depth"][m].view(np.uint32), p["key"][m].view(np.uint32))
+        np.testing.assert_allclose(g["xy"][m], p["xy"][m], rtol=1e-6, atol=1e-4)
+        scale = np.sqrt(p["conic"][m, 0] * p["conic"][m, 2])[:, None]
+        assert np.max(np.abs(g["conic"][m] - p["conic"][m]) / scale) < 2e-6
+        np.testing.assert_allclose(g["opacity"][m], p["opacity"][m], rtol=2e-6)
+        np.testing.assert_allclose(g["rgb"][m], p["rgb"][m], atol=2e-5)
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("name,kw,how", CASES)
+def test_binning_bit_exact(name, kw, how, mode):
+    sc, sp = _setup(name, kw, mode)
+    assert sp.status() == api.GS_OK
+    ids = sp.ids.cpu().numpy()
+    ranges = sp.ranges.cpu().numpy()
+    n_pairs = int(sp.n_pairs.item())
+    projs = O.project_views(sc)
+    rects = np.stack([p["rect"] for p in projs])
+    keys = np.stack([p["key"] for p in projs])
+    valid = np.stack([p["valid"] for p in projs]) != 0
+    area = (rects[..., 1] - rects[..., 0] + 1) * (rects[..., 3] - rects[..., 2] + 1)
+    amb = P.ambiguous_tiles(sc, projs)
+    if not amb.any():
+        assert n_pairs == int(area[valid].sum())
+    tiles = ranges.shape[0]
+    sel = np.arange(tiles) if how == "full" else np.unique(
+        np.random.default_rng(0).integers(0, tiles, 400))
+    sel = sel[~amb[sel]]
+    assert P.compare_lists(ids, ranges, rects, keys, sc, sel) == 0
+    # ranges tile the pair array in order
+    nz = ranges[ranges[:, 1] > ranges[:, 0]]
+    assert nz[0, 0] == 0 and nz[-1, 1] == n_pairs
+    assert np.all(nz[1:, 0] == nz[:-1, 1])
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_binning_isolated_with_ties_and_ragged_tail(mode):
+    # screen-space inputs straight from the generator: many equal depth keys
+    # (ties broken by index), culled entries, rectangles clipped by the image
+    W, H, n, V = 200, 136, 3000, 2
+    d = S.make_projected_2d(n, W, H, seed=3, n_views=V)
+    tx, ty = (W + 15) // 16, (H + 15) // 16
+    rects = np.zeros((V, n, 4), np.int32)
+    u, v, r = d["xy"][..., 0].astype(np.float64), d["xy"][..., 1].astype(np.float64), d["radius"]
+    rects[..., 0] = np.maximum(0, np.floor((u - r) / 16))
+    rects[..., 1] = np.minimum(tx - 1, np.floor((u + r) / 16))
+    rects[..., 2] = np.maximum(0, np.floor((v - r) / 16))
+    rects[..., 3] = np.minimum(ty - 1, np.floor((v + r) / 16))
+    bad = (r == 0) | (rects[..., 0] > rects[..., 1]) | (rects[..., 2] > rects[..., 3])
+    rects[bad] = [1, 0, 1, 0]
+    projs = [dict(xy=d["xy"][k], conic=np.zeros((n, 3)), opacity=np.zeros(n), rgb=np.zeros((n, 3)),
+                  key=d["depth"][k], rect=rects[k], valid=(~bad[k]).astype(np.int32))
+             for k in range(V)]
+    rec = torch.as_tensor(P.pack_records(projs)).cuda()
+    sc = S.make_scene("fwd_1k_128", n=n, width=W, height=H, n_views=1)
+    sc.cameras = sc.cameras * V
+    sp = Splatter(sc, sort_mode=mode, pair_capacity=int(((rects[..., 1] - rects[..., 0] + 1) * (rects[..., 3] - rects[..., 2] + 1))[~bad].sum()))
+    sp.records.copy_(rec)
+    sp.bin_sort()
+    assert sp.status() == api.GS_OK
+    ids, ranges = sp.ids.cpu().numpy(), sp.ranges.cpu().numpy()
+    assert P.compare_lists(ids, ranges, rects, d["depth"], sc, np.arange(ranges.shape[0])) == 0
+
+
+@pytest.mark.parametrize("name,kw,how", CASES)
+def test_render_matches_oracle(name, kw, how):
+    sc, sp = _setup(name, kw)
+    sp.rasterize_fwd()
+    torch.cuda.synchronize()
+    pix = _pixels(sc, how)
+    projs = O.project_views(sc)
+    ref = O.render(projs, sc.cameras, sc.background, pix, P.WIN_ALPHA, P.WIN_T)
+    ref["flags"] = ref["flags"] | (4 * P.ambiguous_pixels(sc, projs, pix))
+    st = P.compare_render(sp.image.cpu().numpy(), sp.final_T.cpu().numpy(),
+                          sp.n_contrib.cpu().numpy(), ref, pix)
+    print(name, st)
+    assert st["flagged"] <= 0.02 * st["n"]
+    assert st["max_abs"] <= P.MAX_ABS
+    assert st["mean_abs"] <= P.MEAN_ABS
+    assert st["nc_mismatch"] == 0
+    assert st["T_max_rel"] < 1e-3
+
+
+@pytest.mark.parametrize("name,kw,how", CASES)
+def test_backward_and_densify_match_oracle(name, kw, how):
+    sc, sp = _setup(name, kw)
+    sp.rasterize_fwd()
+    torch.cuda.synchronize()
+    projs = O.project_views(sc)
+    pix = _pixels(sc, how)
+    ref = O.render(projs, sc.cameras, sc.background, pix, P.WIN_ALPHA, P.WIN_T)
+    keep = pix[(ref["flags"] == 0) & ~P.ambiguous_pixels(sc, projs, pix)]
+    c = sc.cameras[0]
+    dL = S.make_upstream_grad(sc.n_views, c.height, c.width, seed=1)
+    mask = np.zeros_like(dL)
+    mask[keep[:, 0], :, keep[:, 2], keep[:, 1]] = 1.0
+    dL = dL * mask
+    sp.rasterize_bwd(torch.as_tensor(dL).cuda())
+    sp.densify_stats()
+    torch.cuda.synchronize()
+    g2_ref = O.render_bwd(projs, sc.cameras, sc.background, keep,
+                          dL[keep[:, 0], :, keep[:, 2], keep[:, 1]])
+    g2 = sp.grad2d.cpu().numpy()
+    for f in range(10):
+        e = P.rel_l2(g2[..., f], g2_ref[..., f])
+        assert e < P.REL_L2, ("grad2d field", f, e)
+    gr = O.project_bwd(sc, projs, g2_ref)
+    for k, t in sp.grads.items():
+        gpu = t.cpu().numpy()
+        if k in ("means", "log_scales"):
+            gpu = gpu[:, :3]
+        e = P.rel_l2(gpu.reshape(gr[k].shape), gr[k])
+        assert e < P.REL_L2, (k, e)
+    valid = np.stack([p["valid"] for p in projs])
+    plain, absg, den = O.densify_stats(g2_ref, valid)
+    assert P.rel_l2(sp.accum_plain.cpu().numpy(), plain) < P.REL_L2
+    assert P.rel_l2(sp.accum_abs.cpu().numpy(), absg) < P.REL_L2
+    assert np.array_equal(sp.denom.cpu().numpy(), den)
+
+
+def test_adam_matches_oracle_on_generated_inputs():
+    rng = np.random.default_rng(11)
+    sizes = [4 * 1000, 4 * 1000, 4 * 1000, 1000, 48 * 1000 + 3]
+    lrs = [1.6e-4, 5e-3, 1e-3, 5e-2, 2.5e-3]
+    groups, ref = [], []
+    for sz, lr in zip(sizes, lrs):
+        p = rng.normal(size=sz).astype(np.float32)
+        g = rng.normal(size=sz).astype(np.float32) * rng.choice([0, 1e-6, 1.0], size=sz).astype(np.float32)
+        m = (rng.normal(size=sz) * 0.1).astype(np.float32)
+        v = (rng.random(size=sz) * 0.01).astype(np.float32)
+        t = [torch.as_tensor(a).cuda() for a in (p, g, m, v)]
+        groups.append((t[0], t[1], t[2], t[3], lr))
+        # the kernel receives float32 hyper-parameters; the oracle takes the
+        # same values, widened exactly
+        ref.append(O.adam(p, g, m, v, float(np.float32(lr)), 7, float(np.float32(0.9)),
+                          float(np.float32(0.999)), float(np.float32(1e-15))))
+    api.gs_adam_step(groups, 0.9, 0.999, 1e-15, 7)
+    torch.cuda.synchronize()
+    for (p, g, m, v, lr), (rp, rm, rv) in zip(groups, ref):
+        assert P.rel_l2(m.cpu().numpy(), rm) < 1e-6
+        assert P.rel_l2(v.cpu().numpy(), rv) < 1e-6
+        assert P.rel_l2(p.cpu().numpy(), rp) < 1e-6
+
+
+def test_train_step_adam_state_matches_oracle():
+    sc, sp = _setup("fwd_1k_128", dict(n=800), api.GS_SORT_FULL64)
+    p0 = {k: t.clone() for k, t in sp.param_list}
+    c = sc.cameras[0]
+    dL = S.make_upstream_grad(1, c.height, c.width, seed=1)
+    sp.train_step(torch.as_tensor(dL).cuda())
+    torch.cuda.synchronize()
+    projs = O.project_views(sc)
+    pix = P.full_pixels(sc)
+    g2 = O.render_bwd(projs, sc.cameras, sc.background, pix, dL[0].reshape(3, -1).T)
+    gr = O.project_bwd(sc, projs, g2)
+    for k, t in sp.param_list:
+        g = gr[k].reshape(-1)
+        p = p0[k].cpu().numpy().astype(np.float64)
+        if k in ("means", "log_scales"):
+            p = p[:, :3]
+            m_gpu = sp.exp_avg[k].cpu().numpy()[:, :3].reshape(-1)
+            v_gpu = sp.exp_avg_sq[k].cpu().numpy()[:, :3].reshape(-1)
+            p_gpu = t.cpu().numpy()[:, :3].reshape(-1)
+        else:
+            m_gpu = sp.exp_avg[k].cpu().numpy().reshape(-1)
+            v_gpu = sp.exp_avg_sq[k].cpu().numpy().reshape(-1)
+            p_gpu = t.cpu().numpy().reshape(-1)
+        rp, rm, rv = O.adam(p.reshape(-1), g, np.zeros_like(g), np.zeros_like(g), sp.lr[k], 1)
+        assert P.rel_l2(m_gpu, rm) < P.REL_L2, k
+        assert P.rel_l2(v_gpu, rv) < P.REL_L2, k
+        # the first step moves each parameter by lr * sign(g): compare where
+        # the gradient is not vanishingly small
+        big = np.abs(g) > 1e-3 * np.sqrt(np.mean(g * g) + 1e-300)
+        assert P.rel_l2((p_gpu - p.reshape(-1))[big], (rp - p.reshape(-1))[big]) < P.REL_L2, k
+
+
+def test_capacity_exceeded_reports_and_empties():
+    sc = S.make_scene("fwd_1k_128", n=500)
+    sp = Splatter(sc, pair_capacity=10)
+    sp.forward()
+    assert sp.status() == api.GS_ERR_CAPACITY
+    projs = O.project_views(sc)
+    r = projs[0]["rect"]
+    need = int(((r[:, 1] - r[:, 0] + 1) * (r[:, 3] - r[:, 2] + 1))[projs[0]["valid"] != 0].sum())
+    assert int(sp.n_pairs.item()) == need
+    assert int(sp.ranges.abs().sum().item()) == 0
+    assert torch.all(sp.final_T == 1.0)
+    assert sp.status() == api.GS_OK  # cleared by the previous read
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_empty_and_all_culled(mode):
+    for n, behind in ((0, False), (50, True)):
+        sc = S.make_scene("fwd_1k_128", n=max(n, 1))
+        if n == 0:
+            for k in ("means", "log_scales", "quats", "opacity_logit", "sh"):
+                setattr(sc, k, getattr(sc, k)[:0])
+        if behind:
+            sc.means[:, 2] = -5.0
+        sc.background = np.array([0.25, 0.5, 0.75], np.float32)
+        sp = Splatter(sc, sort_mode=mode, pair_capacity=16)
+        sp.forward()
+        dL = torch.ones((1, 3, 128, 128), device="cuda")
+        sp.rasterize_bwd(dL)
+        torch.cuda.synchronize()
+        assert sp.status() == api.GS_OK
+        assert int(sp.n_pairs.item()) == 0
+        img = sp.image.cpu().numpy()
+        for ch in range(3):
+            assert np.all(img[0, ch] == sc.background[ch])
+        assert torch.all(sp.n_contrib == 0)
+        for t in sp.grads.values():
+            assert torch.all(t == 0)
+
+
+def test_single_gaussian_centred_on_pixel_gives_o_c():
+    cam = S.Camera(viewmat=np.concatenate([np.eye(3), np.zeros((3, 1))], 1).astype(np.float32),
+                   fx=100.0, fy=100.0, cx=20.5, cy=17.5, width=40, height=36,
+                   campos=np.zeros(3, np.float32))
+    logit = np.float32(0.4)
+    sc = S.Scene("one", means=np.array([[0, 0, 3.0, 0]], np.float32),
+                 log_scales=np.array([[-4.0, -4.0, -4.0, 0]], np.float32),
+                 quats=np.array([[1, 0, 0, 0]], np.float32), opacity_logit=np.array([logit]),
+                 sh=np.array([[[0.3, -0.2, 0.4]]], np.float32), sh_degree=0, cameras=[cam],
+                 background=np.zeros(3, np.float32))
+    sp = Splatter(sc, pair_capacity=64)
+    sp.forward()
+    torch.cuda.synchronize()
+    o = 1.0 / (1.0 + np.exp(-np.float64(logit)))
+    rgb = 0.5 + 0.28209479177387814 * np.array([0.3, -0.2, 0.4])
+    got = sp.image.cpu().numpy()[0, :, 17, 20]
+    np.testing.assert_allclose(got, o * rgb, atol=1e-6)
