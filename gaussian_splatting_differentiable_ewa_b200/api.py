@@ -93,7 +93,12 @@ SIGNATURES = [
     ("gs_adam_step", _c.c_int,
      [_c.POINTER(GsAdamGroup), _c.c_int32, _c.c_float, _c.c_float, _c.c_float, _c.c_int64, _vp]),
     ("gs_get_status", _c.c_int, [_vp, _vp]),
+    ("gs_bin_sort_noalloc", _c.c_int,
+     [_c.POINTER(GsProjected), _c.POINTER(GsCamera), _c.c_int32, _c.c_int64, _c.c_int32,
+      _c.POINTER(GsBinned), _vp, _vp]),
 ]
+
+GS_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 _LIB = None
 
@@ -247,3 +252,13 @@ def gs_adam_step(groups: Sequence[tuple], beta1: float, beta2: float, eps: float
 
 def gs_get_status(ws, stream=None) -> int:
     return int(lib().gs_get_status(_ptr(ws), _stream(stream)))
+
+
+def gs_bin_sort_noalloc(proj: GsProjected, cams_arr, n_views: int, n: int, sort_mode: int,
+                        out: GsBinned, device_status=None, stream=None) -> None:
+    """gs_bin_sort without a workspace argument, for callers that cannot
+    allocate device memory: the library's fixed scratch array is used instead
+    (see include/gs.h for its size limit and the no-overlap rule)."""
+    _check(lib().gs_bin_sort_noalloc(_c.byref(proj), cams_arr, int(n_views), int(n),
+                                     int(sort_mode), _c.byref(out), _ptr(device_status),
+                                     _stream(stream)), "gs_bin_sort_noalloc")

@@ -5,6 +5,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <cuda_runtime.h>
 
 #include "gs_internal.h"
@@ -310,6 +311,65 @@ gs_status gs_adam_step(const gs_adam_group* groups, int32_t n_groups, float beta
   }
   return cuda_status(
       launch_adam(groups, n_groups, beta1, beta2, eps, step, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// gs_bin_sort_noalloc: gs_bin_sort with its workspace in a fixed device array,
+// for callers that cannot allocate device memory themselves.
+namespace {
+
+// The scratch. In host code this name is a host-side stand-in, not a device
+// address: the address is looked up once per device with
+// cudaGetSymbolAddress and passed to the kernels.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GS_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch on the current device (looked up on the
+// first call for that device).
+gs_status noalloc_scratch(void** addr) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GS_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return GS_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GS_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *addr = g_noalloc_addr[dev];
+  return GS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+gs_status gs_bin_sort_noalloc(const gs_projected* proj, const gs_camera* cams, int32_t n_views,
+                              int64_t n, int32_t sort_mode, gs_binned* out,
+                              int32_t* device_status, void* stream) {
+  if (!proj || !out) return GS_ERR_INVALID_ARG;
+  const size_t need = gs_workspace_size(n, n_views, cams, out->pair_capacity, sort_mode);
+  if (need == 0 || need > (size_t)GS_NOALLOC_SCRATCH_BYTES) return GS_ERR_INVALID_ARG;
+  void* ws = nullptr;
+  gs_status s = noalloc_scratch(&ws);
+  if (s != GS_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the array keeps the previous call's contents: start from a clear status
+  // word (gs_bin_sort clears the counters, histograms and look-back state it
+  // relies on)
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), st) != cudaSuccess) return GS_ERR_CUDA;
+  s = gs_bin_sort(proj, cams, n_views, n, sort_mode, out, ws, GS_NOALLOC_SCRATCH_BYTES, stream);
+  if (s != GS_OK) return s;
+  if (device_status &&
+      cudaMemcpyAsync(device_status, ws, sizeof(int32_t), cudaMemcpyDeviceToDevice, st) !=
+          cudaSuccess)
+    return GS_ERR_CUDA;
+  return GS_OK;
 }
 
 gs_status gs_get_status(void* ws, void* stream) {

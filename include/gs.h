@@ -193,6 +193,32 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
                       int64_t n, int32_t sort_mode, gs_binned* out, void* ws,
                       size_t ws_bytes, void* stream);
 
+/* Size of the fixed scratch array that gs_bin_sort_noalloc uses. */
+#define GS_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* gs_bin_sort for callers that must not allocate device memory. (The pages
+ * have no counterpart; this is a library convenience.) Some callers cannot
+ * call cudaMalloc: code that runs inside a host application owning the
+ * device's memory budget (a plug-in or an engine's render thread), or a loop
+ * that cannot afford the device-wide synchronisation and the late
+ * out-of-memory failure a fresh allocation can bring. This entry point takes
+ * the same inputs and outputs as gs_bin_sort but no workspace: its scratch is
+ * a fixed array of GS_NOALLOC_SCRATCH_BYTES inside the library, which every
+ * GPU that uses this entry point holds from its first call until the process
+ * exits. The first call on a device looks up the array's device address
+ * (with that device current); make that first call before any stream
+ * capture. Requests whose gs_workspace_size exceeds GS_NOALLOC_SCRATCH_BYTES
+ * are rejected with GS_ERR_INVALID_ARG before anything is enqueued. All calls
+ * share the one array: calls whose work overlaps on the GPU (for example on
+ * two streams) race and corrupt each other's results; serialise them.
+ * Each call starts with a cleared status word; if `device_status` (a device
+ * int32, may be NULL) is given, the call's device-side status bits (1 pair
+ * capacity exceeded, 2 a bounded wait gave up, 4 an index out of range) are
+ * copied there at the end, in stream order. */
+gs_status gs_bin_sort_noalloc(const gs_projected* proj, const gs_camera* cams, int32_t n_views,
+                              int64_t n, int32_t sort_mode, gs_binned* out,
+                              int32_t* device_status, void* stream);
+
 /* Forward rasterisation, one 16x16 tile per thread block and one thread per
  * pixel (pwwt.cn sec. 5.4 tile mode; lshu.cn sec. 3.2 `blend`, sec. 7.3).
  * For each pixel, front to back over its tile's list:
