@@ -55,7 +55,7 @@ class GsGrads(_c.Structure):
 
 
 class GsProjected(_c.Structure):
-    _fields_ = [("records", _vp), ("radii", _vp)]
+    _fields_ = [("records", _vp), ("bins", _vp), ("radii", _vp)]
 
 
 class GsBinned(_c.Structure):
@@ -173,8 +173,8 @@ def grads(means, log_scales, quats, opacity_logit, sh) -> GsGrads:
     return GsGrads(_ptr(means), _ptr(log_scales), _ptr(quats), _ptr(opacity_logit), _ptr(sh))
 
 
-def projected(records, radii) -> GsProjected:
-    return GsProjected(_ptr(records), _ptr(radii))
+def projected(records, bins, radii) -> GsProjected:
+    return GsProjected(_ptr(records), _ptr(bins), _ptr(radii))
 
 
 def binned(ids, ranges, n_pairs, capacity: int) -> GsBinned:

@@ -72,25 +72,63 @@ __device__ __forceinline__ uint32_t block_exclusive_scan_256(uint32_t x, uint32_
   return r;
 }
 
-// Decoupled look-back for one value per block (thread 0 of the block).
-// Publishes the block aggregate, walks back to the nearest inclusive prefix,
-// publishes its own inclusive prefix, and returns the exclusive prefix.
-__device__ uint64_t block_lookback(uint64_t* lb, uint32_t idx, uint64_t aggregate,
-                                   uint32_t* status) {
+// Exclusive prefix of partition p from the look-back words of partitions
+// p-1, p-2, ... (word of partition j at base[j * stride]): one thread walks
+// back 8 partitions per round trip (8 independent loads), waiting only on
+// words still empty, until it reaches an inclusive prefix.
+__device__ __forceinline__ uint64_t windowed_lookback(const uint64_t* base, int64_t stride,
+                                                      int64_t p, uint32_t* status) {
+  constexpr int kWin = 8;
+  uint64_t excl = 0;
+  int64_t j = p - 1;
+  while (j >= 0) {
+    uint64_t w[kWin];
+#pragma unroll
+    for (int k = 0; k < kWin; ++k) w[k] = (j - k >= 0) ? ld_relaxed_u64(base + (j - k) * stride) : 0ull;
+    bool found = false;
+#pragma unroll
+    for (int k = 0; k < kWin; ++k) {
+      if (found || j - k < 0) continue;
+      uint64_t v = w[k];
+      if ((v >> 62) == 0) v = lookback_wait(base + (j - k) * stride, status);
+      excl += v & kLbValueMask;
+      if ((v >> 62) == 2) found = true;
+    }
+    if (found) break;
+    j -= kWin;
+  }
+  return excl;
+}
+
+// Decoupled look-back for one value per block, run by warp 0 of the block.
+// Publishes the block aggregate, then the warp reads 32 predecessors per
+// round trip and sums them back to the nearest inclusive prefix; publishes
+// the block's inclusive prefix and returns the exclusive prefix (to all lanes
+// of warp 0).
+__device__ uint64_t warp_block_lookback(uint64_t* lb, uint32_t idx, uint64_t aggregate,
+                                        uint32_t* status) {
+  const int lane = threadIdx.x & 31;
   if (idx == 0) {
-    st_relaxed_u64(&lb[0], kLbPrefix | aggregate);
+    if (lane == 0) st_relaxed_u64(&lb[0], kLbPrefix | aggregate);
     return 0;
   }
-  st_relaxed_u64(&lb[idx], kLbAggregate | aggregate);
+  if (lane == 0) st_relaxed_u64(&lb[idx], kLbAggregate | aggregate);
   uint64_t excl = 0;
-  int64_t j = (int64_t)idx - 1;
-  while (j >= 0) {
-    uint64_t w = lookback_wait(&lb[j], status);
-    excl += w & kLbValueMask;
-    if ((w >> 62) == 2) break;
-    --j;
+  int64_t base = (int64_t)idx - 1;
+  while (true) {
+    const int64_t j = base - lane;
+    uint64_t w = j >= 0 ? ld_relaxed_u64(&lb[j]) : kLbPrefix;
+    if ((w >> 62) == 0) w = lookback_wait(&lb[j], status);
+    const uint32_t pre = __ballot_sync(0xffffffffu, (w >> 62) == 2);
+    const int first = pre ? __ffs(pre) - 1 : 32;  // nearest inclusive prefix
+    uint64_t val = lane <= first ? (w & kLbValueMask) : 0ull;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) val += __shfl_xor_sync(0xffffffffu, val, o);
+    excl += val;
+    if (pre) break;
+    base -= 32;
   }
-  st_relaxed_u64(&lb[idx], kLbPrefix | (excl + aggregate));
+  if (lane == 0) st_relaxed_u64(&lb[idx], kLbPrefix | (excl + aggregate));
   return excl;
 }
 
@@ -109,7 +147,7 @@ struct KeyTraits<uint32_t> {
 // Presort keys: (view << 32 | depth bits) for visible Gaussians, all ones for
 // culled ones, value = Gaussian index within its view. Also histograms the
 // key digits of the presort passes.
-__global__ void __launch_bounds__(256) k_depth_keys(const float4* __restrict__ records, int n,
+__global__ void __launch_bounds__(256) k_depth_keys(const float4* __restrict__ bins, int n,
                                                    int n_views, int passes,
                                                    uint64_t* __restrict__ keys,
                                                    uint32_t* __restrict__ vals,
@@ -122,12 +160,12 @@ __global__ void __launch_bounds__(256) k_depth_keys(const float4* __restrict__ r
   const int64_t total = (int64_t)n * n_views;
   for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < total;
        j += (int64_t)gridDim.x * blockDim.x) {
-    const float4 r2 = __ldg(&records[j * 3 + 2]);
-    const uint32_t txw = __float_as_uint(r2.z), tyw = __float_as_uint(r2.w);
+    const float4 r2 = __ldg(&bins[j]);  // depth key, tile_x, tile_y
+    const uint32_t txw = __float_as_uint(r2.y), tyw = __float_as_uint(r2.z);
     const bool vis = (txw & 0xffffu) <= (txw >> 16) && (tyw & 0xffffu) <= (tyw >> 16);
     const int view = (int)(j / n);
     const uint64_t key =
-        vis ? (((uint64_t)view << 32) | (uint64_t)__float_as_uint(r2.y)) : ~0ull;
+        vis ? (((uint64_t)view << 32) | (uint64_t)__float_as_uint(r2.x)) : ~0ull;
     keys[j] = key;
     vals[j] = (uint32_t)(j - (int64_t)view * n);
     for (int d = 0; d < passes; ++d) atomicAdd(&s_hist[d][(key >> (8 * d)) & 0xff], 1u);
@@ -141,14 +179,14 @@ __global__ void __launch_bounds__(256) k_depth_keys(const float4* __restrict__ r
 
 // ---------------------------------------------------------------------------
 // Fused pair count + scan + emission.
-// MODE 0 (full 64-bit keys): items are the n_views * n records in index
+// MODE 0 (full 64-bit keys): items are the n_views * n Gaussians in index
 //   order; key = (global tile << 32) | depth bits.
 // MODE 1 (presorted): items are the presorted (key, index) list; key = global
 //   tile (32-bit).
 // Histograms: digit d of the emitted keys into hist[d][256] for d < passes.
 template <int MODE, typename K>
 __global__ void __launch_bounds__(kEmitThreads) k_emit(
-    const float4* __restrict__ records, const uint64_t* __restrict__ pkeys,
+    const float4* __restrict__ bins, const uint64_t* __restrict__ pkeys,
     const uint32_t* __restrict__ pvals, int n, int n_views, Grid g, int passes,
     K* __restrict__ keys_out, uint32_t* __restrict__ ids_out, int64_t capacity,
     int64_t* __restrict__ n_pairs, unsigned long long* __restrict__ hist,
@@ -189,15 +227,15 @@ __global__ void __launch_bounds__(kEmitThreads) k_emit(
         rec_index = (int64_t)(view < 0 ? 0 : view) * n + id;
       }
       if (view >= 0) {
-        const float4 r2 = __ldg(&records[rec_index * 3 + 2]);
-        const uint32_t txw = __float_as_uint(r2.z), tyw = __float_as_uint(r2.w);
+        const float4 r2 = __ldg(&bins[rec_index]);
+        const uint32_t txw = __float_as_uint(r2.y), tyw = __float_as_uint(r2.z);
         const uint32_t x0 = txw & 0xffffu, x1 = txw >> 16, y0 = tyw & 0xffffu, y1 = tyw >> 16;
         if (x0 <= x1 && y0 <= y1) {
           const uint32_t w = x1 - x0 + 1;
           c = w * (y1 - y0 + 1);
           rx = x0 | (w << 16);
           ry = y0 | ((uint32_t)view << 16);
-          depth = __float_as_uint(r2.y);
+          depth = __float_as_uint(r2.x);
         }
       }
     }
@@ -215,13 +253,15 @@ __global__ void __launch_bounds__(kEmitThreads) k_emit(
     s_off[threadIdx.x * kEmitItemsPerThread + k] = toff;
     toff += cnt[k];
   }
-  if (threadIdx.x == 0) {
-    s_off[kEmitItems] = block_total;
-    const uint64_t base = block_lookback(lookback, bidx, block_total, status);
-    s_base = base;
-    const uint32_t n_blocks = (uint32_t)((n_items + kEmitItems - 1) / kEmitItems);
-    if (bidx == n_blocks - 1) *n_pairs = (int64_t)(base + block_total);
-    if ((int64_t)(base + block_total) > capacity) atomicOr(status, kStatusCapacity);
+  if (threadIdx.x < 32) {
+    const uint64_t base = warp_block_lookback(lookback, bidx, block_total, status);
+    if (threadIdx.x == 0) {
+      s_off[kEmitItems] = block_total;
+      s_base = base;
+      const uint32_t n_blocks = (uint32_t)((n_items + kEmitItems - 1) / kEmitItems);
+      if (bidx == n_blocks - 1) *n_pairs = (int64_t)(base + block_total);
+      if ((int64_t)(base + block_total) > capacity) atomicOr(status, kStatusCapacity);
+    }
   }
   __syncthreads();
   const uint64_t base = s_base;
@@ -376,13 +416,7 @@ __global__ void __launch_bounds__(kSortThreads, 2) k_onesweep(
         st_relaxed_u64(lb, kLbPrefix | (uint64_t)count);
       } else {
         st_relaxed_u64(lb, kLbAggregate | (uint64_t)count);
-        int64_t j = p - 1;
-        while (j >= 0) {
-          const uint64_t w = lookback_wait(lookback + j * kRadix + b, status);
-          excl += w & kLbValueMask;
-          if ((w >> 62) == 2) break;
-          --j;
-        }
+        excl = windowed_lookback(lookback + b, kRadix, p, status);
         st_relaxed_u64(lb, kLbPrefix | (excl + count));
       }
       s_gbase[b] = s_gexcl[b] + excl;
@@ -420,30 +454,65 @@ __global__ void __launch_bounds__(kSortThreads, 2) k_onesweep(
   }
 }
 
+// Tile id of a sorted key.
+template <typename K>
+__device__ __forceinline__ uint32_t tile_of(K k) {
+  return (uint32_t)(((uint64_t)k) >> (KeyTraits<K>::kBits == 64 ? 32 : 0));
+}
+
+// [start, end) of every tile present in the sorted keys. Each thread takes 8
+// consecutive keys with vector loads (a full chunk) and compares neighbours.
 template <typename K>
 __global__ void k_ranges(const K* __restrict__ keys, const int64_t* __restrict__ n_ptr,
                          int64_t capacity, int64_t n_tiles, int64_t* __restrict__ ranges,
                          uint32_t* __restrict__ status) {
   const int64_t n = *n_ptr;
   if (n > capacity) return;
-  constexpr int kShift = KeyTraits<K>::kBits == 64 ? 32 : 0;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const uint32_t t = (uint32_t)(keys[i] >> kShift);
-    if ((int64_t)t >= n_tiles || (i > 0 && (int64_t)(uint32_t)(keys[i - 1] >> kShift) >= n_tiles)) {
-      atomicOr(status, kStatusBounds);
-      continue;
-    }
-    if (i == 0) {
-      ranges[2 * (int64_t)t] = 0;
-    } else {
-      const uint32_t tp = (uint32_t)(keys[i - 1] >> kShift);
-      if (tp != t) {
-        ranges[2 * (int64_t)t] = i;
-        ranges[2 * (int64_t)tp + 1] = i;
+  constexpr int C = 8;
+  const int64_t chunks = (n + C - 1) / C;
+  for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < chunks;
+       c += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i0 = c * C;
+    uint32_t t[C];
+    if (i0 + C <= n) {
+      if (KeyTraits<K>::kBits == 32) {
+        const uint4* p4 = reinterpret_cast<const uint4*>(keys + i0);
+        const uint4 a = p4[0], b = p4[1];
+        t[0] = a.x; t[1] = a.y; t[2] = a.z; t[3] = a.w;
+        t[4] = b.x; t[5] = b.y; t[6] = b.z; t[7] = b.w;
+      } else {
+        const ulonglong2* p2 = reinterpret_cast<const ulonglong2*>(keys + i0);
+#pragma unroll
+        for (int q = 0; q < C / 2; ++q) {
+          const ulonglong2 v = p2[q];
+          t[2 * q] = (uint32_t)(v.x >> 32);
+          t[2 * q + 1] = (uint32_t)(v.y >> 32);
+        }
       }
+    } else {
+#pragma unroll
+      for (int k = 0; k < C; ++k) t[k] = i0 + k < n ? tile_of(keys[i0 + k]) : 0u;
     }
-    if (i == n - 1) ranges[2 * (int64_t)t + 1] = n;
+    uint32_t prev = i0 > 0 ? tile_of(keys[i0 - 1]) : 0xffffffffu;
+#pragma unroll
+    for (int k = 0; k < C; ++k) {
+      const int64_t i = i0 + k;
+      if (i >= n) break;
+      const uint32_t cur = t[k];
+      if ((int64_t)cur >= n_tiles) {
+        atomicOr(status, kStatusBounds);
+        prev = cur;
+        continue;
+      }
+      if (i == 0) {
+        ranges[2 * (int64_t)cur] = 0;
+      } else if (cur != prev) {
+        ranges[2 * (int64_t)cur] = i;
+        if ((int64_t)prev < n_tiles) ranges[2 * (int64_t)prev + 1] = i;
+      }
+      if (i == n - 1) ranges[2 * (int64_t)cur + 1] = n;
+      prev = cur;
+    }
   }
 }
 
@@ -506,7 +575,7 @@ int64_t emit_blocks(int64_t items) { return (items + kEmitItems - 1) / kEmitItem
 cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
   cudaError_t e;
   const int64_t n_items = (int64_t)a.n * a.n_views;
-  const auto rec4 = reinterpret_cast<const float4*>(a.records);
+  const auto rec4 = reinterpret_cast<const float4*>(a.bins);
   if (n_items == 0) {
     return cudaMemsetAsync(a.n_pairs, 0, sizeof(int64_t), stream);
   }

@@ -140,13 +140,13 @@ gs_status gs_project(const gs_params* params, const gs_camera* cams, int32_t n_v
   if (p.sh_degree < 0 || p.sh_degree > 3) return GS_ERR_INVALID_ARG;
   if (p.n == 0) return GS_OK;
   if (!p.means || !p.log_scales || !p.quats || !p.opacity_logit || !p.sh || !out->records ||
-      !out->radii)
+      !out->bins || !out->radii)
     return GS_ERR_INVALID_ARG;
   if (!aligned(p.means, 16) || !aligned(p.log_scales, 16) || !aligned(p.quats, 16) ||
-      !aligned(out->records, 16))
+      !aligned(out->records, 16) || !aligned(out->bins, 16))
     return GS_ERR_INVALID_ARG;
   const CamSet cs = pack_cams(cams, n_views);
-  return cuda_status(launch_project(p, cs, n_views, out->records, out->radii,
+  return cuda_status(launch_project(p, cs, n_views, out->records, out->bins, out->radii,
                                     static_cast<cudaStream_t>(stream)));
 }
 
@@ -159,7 +159,7 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
   if (!make_layout(n, n_views, cams, out->pair_capacity, sort_mode, L)) return GS_ERR_INVALID_ARG;
   if (ws_bytes < L.total || !aligned(ws, kAlign)) return GS_ERR_INVALID_ARG;
   if (!out->ids || !out->ranges || !out->n_pairs) return GS_ERR_INVALID_ARG;
-  if (n > 0 && (!proj->records || !aligned(proj->records, 16))) return GS_ERR_INVALID_ARG;
+  if (n > 0 && (!proj->bins || !aligned(proj->bins, 16))) return GS_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   unsigned char* w = static_cast<unsigned char*>(ws);
   const Grid g = grid_of(cams[0]);
@@ -175,7 +175,7 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
 
   BinSortArgs a;
   std::memset(&a, 0, sizeof(a));
-  a.records = proj->records;
+  a.bins = proj->bins;
   a.n = (int)n;
   a.n_views = n_views;
   a.mode = sort_mode;

@@ -45,11 +45,12 @@ __host__ __device__ inline Grid grid_of(const gs_camera& c) {
   return g;
 }
 
-// Record field offsets (floats), see gs.h.
+// Raster record field offsets (floats), see gs.h.
 enum RecField {
   R_U = 0, R_V = 1, R_CA = 2, R_CB = 3, R_CC = 4, R_OPAC = 5,
-  R_R = 6, R_G = 7, R_B = 8, R_DEPTH = 9, R_TX = 10, R_TY = 11
+  R_R = 6, R_G = 7, R_B = 8, R_HX = 9, R_HY = 10, R_SPARE = 11
 };
+// Binning record (one float4): depth key, tile_x word, tile_y word, 0.
 // Screen-space gradient fields (floats), see gs.h.
 enum G2Field {
   G_U = 0, G_V = 1, G_CA = 2, G_CB = 3, G_CC = 4, G_OPAC = 5,

@@ -10,7 +10,7 @@
 namespace gsb {
 
 struct BinSortArgs {
-  const float* records;
+  const float* bins;    // [n_views][n][4] binning records
   int n;
   int n_views;
   int mode;
@@ -37,7 +37,7 @@ struct BinSortArgs {
 };
 
 cudaError_t launch_project(const gs_params& p, const CamSet& cams, int n_views, float* records,
-                           int* radii, cudaStream_t stream);
+                           float* bins, int* radii, cudaStream_t stream);
 cudaError_t launch_project_bwd(const gs_params& p, const CamSet& cams, int n_views,
                                const float* grad2d, const int* radii, const gs_grads& g,
                                cudaStream_t stream);

@@ -109,6 +109,36 @@ __device__ __forceinline__ long long floor_tile(double a) {
   return static_cast<long long>(floor(a * (1.0 / kTile)));
 }
 
+// Colour from the SH coefficients of one Gaussian at unit direction (x, y, z):
+// rgb_c = max(0, sum_k Y_k sh_kc + 0.5). Coefficients are read with 16-byte
+// loads when the per-Gaussian block is a multiple of 16 bytes.
+template <int DEG>
+__device__ __forceinline__ void sh_colour(const float* __restrict__ shi, float x, float y, float z,
+                                          float rgb[3]) {
+  constexpr int K = (DEG + 1) * (DEG + 1);
+  float Y[16];
+  sh_basis<DEG>(x, y, z, Y);
+  float acc[3] = {0.5f, 0.5f, 0.5f};
+  if ((K * 3) % 4 == 0) {
+    const float4* s4 = reinterpret_cast<const float4*>(shi);
+#pragma unroll
+    for (int q = 0; q < K * 3 / 4; ++q) {
+      const float4 c = __ldg(&s4[q]);
+      const float cv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int idx = 4 * q + e;
+        acc[idx % 3] = fmaf(Y[idx / 3], cv[e], acc[idx % 3]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int idx = 0; idx < K * 3; ++idx) acc[idx % 3] = fmaf(Y[idx / 3], __ldg(&shi[idx]), acc[idx % 3]);
+  }
+#pragma unroll
+  for (int ch = 0; ch < 3; ++ch) rgb[ch] = fmaxf(acc[ch], 0.f);
+}
+
 template <int DEG>
 __global__ void __launch_bounds__(256) k_project(const float4* __restrict__ means,
                                                  const float4* __restrict__ log_scales,
@@ -116,6 +146,7 @@ __global__ void __launch_bounds__(256) k_project(const float4* __restrict__ mean
                                                  const float* __restrict__ logit,
                                                  const float* __restrict__ sh, int n, int n_views,
                                                  CamSet cams, float4* __restrict__ records,
+                                                 float4* __restrict__ bins,
                                                  int* __restrict__ radii) {
   constexpr int K = (DEG + 1) * (DEG + 1);
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -137,12 +168,10 @@ __global__ void __launch_bounds__(256) k_project(const float4* __restrict__ mean
   for (int a = 0; a < 3; ++a)
 #pragma unroll
     for (int b = 0; b < 3; ++b) M[a][b] = R[a][b] * s[b];
-  const float opac = (float)(1.0 / (1.0 + exp(-(double)lg)));
-
-  float coef[K * 3];
+  const double opac_d = 1.0 / (1.0 + exp(-(double)lg));
+  // alpha >= 1/255 needs q <= Q = 2 ln(255 o); Q <= 0: the splat never counts
+  const double Qa = 2.0 * log(255.0 * opac_d);
   const float* shi = sh + (size_t)i * K * 3;
-#pragma unroll
-  for (int k = 0; k < K * 3; ++k) coef[k] = __ldg(&shi[k]);
 
   const Grid g = grid_of(cams.c[0]);
   for (int v = 0; v < n_views; ++v) {
@@ -211,20 +240,26 @@ __global__ void __launch_bounds__(256) k_project(const float4* __restrict__ mean
           rec[R_CA] = (float)(C * idet);
           rec[R_CB] = (float)(-B * idet);
           rec[R_CC] = (float)(A * idet);
-          rec[R_OPAC] = opac;
-          rec[R_DEPTH] = key;
+          rec[R_OPAC] = (float)opac_d;
+          // half-widths of the box around {q <= Q}, with Q padded (0.2 % +
+          // 1e-4) well beyond the float rounding of the rasteriser's alpha
+          // test, so the box holds every pixel that test can accept
+          const double Qp = Qa + 2e-3 * fabs(Qa) + 1e-4;
+          if (Qp > 0.0) {
+            rec[R_HX] = (float)(sqrt(Qp * A) + 1e-2);
+            rec[R_HY] = (float)(sqrt(Qp * C) + 1e-2);
+          } else {
+            rec[R_HX] = -1.f;
+            rec[R_HY] = -1.f;
+          }
           // colour: SH at the direction from the camera centre to the mean
           float dxv = m.x - c.campos[0], dyv = m.y - c.campos[1], dzv = m.z - c.campos[2];
           float inv = rsqrtf(dxv * dxv + dyv * dyv + dzv * dzv);
-          float Y[16];
-          sh_basis<DEG>(dxv * inv, dyv * inv, dzv * inv, Y);
-#pragma unroll
-          for (int ch = 0; ch < 3; ++ch) {
-            float acc = 0.5f;
-#pragma unroll
-            for (int k = 0; k < K; ++k) acc = fmaf(Y[k], coef[k * 3 + ch], acc);
-            rec[R_R + ch] = fmaxf(acc, 0.f);
-          }
+          float rgb[3];
+          sh_colour<DEG>(shi, dxv * inv, dyv * inv, dzv * inv, rgb);
+          rec[R_R] = rgb[0];
+          rec[R_G] = rgb[1];
+          rec[R_B] = rgb[2];
         }
       }
     }
@@ -232,15 +267,18 @@ __global__ void __launch_bounds__(256) k_project(const float4* __restrict__ mean
       radius = 0;
       x0 = 1; x1 = 0; y0 = 1; y1 = 0;
 #pragma unroll
-      for (int k = 0; k < 10; ++k) rec[k] = 0.f;
+      for (int k = 0; k < 12; ++k) rec[k] = 0.f;
+      rec[R_HX] = -1.f;
+      rec[R_HY] = -1.f;
     }
-    rec[R_TX] = __uint_as_float((uint32_t)x0 | ((uint32_t)x1 << 16));
-    rec[R_TY] = __uint_as_float((uint32_t)y0 | ((uint32_t)y1 << 16));
-    float4* out = records + ((size_t)v * n + i) * 3;
+    const size_t r = (size_t)v * n + i;
+    float4* out = records + r * 3;
     out[0] = make_float4(rec[0], rec[1], rec[2], rec[3]);
     out[1] = make_float4(rec[4], rec[5], rec[6], rec[7]);
     out[2] = make_float4(rec[8], rec[9], rec[10], rec[11]);
-    radii[(size_t)v * n + i] = radius;
+    bins[r] = make_float4(key, __uint_as_float((uint32_t)x0 | ((uint32_t)x1 << 16)),
+                          __uint_as_float((uint32_t)y0 | ((uint32_t)y1 << 16)), 0.f);
+    radii[r] = radius;
   }
 }
 
@@ -425,7 +463,7 @@ __global__ void __launch_bounds__(128) k_project_bwd(
 }  // namespace
 
 cudaError_t launch_project(const gs_params& p, const CamSet& cams, int n_views, float* records,
-                           int* radii, cudaStream_t stream) {
+                           float* bins, int* radii, cudaStream_t stream) {
   const int n = (int)p.n;
   if (n == 0) return cudaSuccess;
   const int threads = 256;
@@ -434,12 +472,15 @@ cudaError_t launch_project(const gs_params& p, const CamSet& cams, int n_views, 
   auto s = reinterpret_cast<const float4*>(p.log_scales);
   auto q = reinterpret_cast<const float4*>(p.quats);
   auto r = reinterpret_cast<float4*>(records);
+  auto b = reinterpret_cast<float4*>(bins);
+#define GS_PFWD(D) k_project<D><<<blocks, threads, 0, stream>>>(m, s, q, p.opacity_logit, p.sh, n, n_views, cams, r, b, radii)
   switch (p.sh_degree) {
-    case 0: k_project<0><<<blocks, threads, 0, stream>>>(m, s, q, p.opacity_logit, p.sh, n, n_views, cams, r, radii); break;
-    case 1: k_project<1><<<blocks, threads, 0, stream>>>(m, s, q, p.opacity_logit, p.sh, n, n_views, cams, r, radii); break;
-    case 2: k_project<2><<<blocks, threads, 0, stream>>>(m, s, q, p.opacity_logit, p.sh, n, n_views, cams, r, radii); break;
-    default: k_project<3><<<blocks, threads, 0, stream>>>(m, s, q, p.opacity_logit, p.sh, n, n_views, cams, r, radii); break;
+    case 0: GS_PFWD(0); break;
+    case 1: GS_PFWD(1); break;
+    case 2: GS_PFWD(2); break;
+    default: GS_PFWD(3); break;
   }
+#undef GS_PFWD
   return cudaGetLastError();
 }
 

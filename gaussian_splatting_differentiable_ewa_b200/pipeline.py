@@ -56,6 +56,7 @@ class Splatter:
                            ("sh", self.sh)]
         n, V = self.n, self.V
         self.records = torch.empty((V, n, api.GS_RECORD_FLOATS), dtype=f32, device=dev)
+        self.bins = torch.empty((V, n, 4), dtype=f32, device=dev)
         self.radii = torch.empty((V, n), dtype=torch.int32, device=dev)
         self.image = torch.empty((V, 3, self.H, self.W), dtype=f32, device=dev)
         self.final_T = torch.empty((V, self.H, self.W), dtype=f32, device=dev)
@@ -85,7 +86,7 @@ class Splatter:
         self.c_params = api.params(self.means, self.log_scales, self.quats, self.opacity_logit,
                                    self.sh, self.deg)
         self.c_grads = api.grads(*[self.grads[k] for k, _ in self.param_list])
-        self.c_proj = api.projected(self.records, self.radii)
+        self.c_proj = api.projected(self.records, self.bins, self.radii)
         self._alloc_pairs(int(pair_capacity) if pair_capacity is not None else 0)
 
     # ------------------------------------------------------------ buffers

@@ -111,17 +111,26 @@ typedef struct gs_grads {
 } gs_grads;
 
 /* Output of gs_project, per view v and Gaussian i (record index v*n + i):
- * records [n_views][n][12] floats, 16-byte aligned:
+ * records [n_views][n][12] floats, 16-byte aligned (what the rasteriser reads):
  *   0 u        1 v          pixel coordinates of the mean
  *   2 conic_a  3 conic_b    4 conic_c   inverse 2D covariance [[a, b], [b, c]]
  *   5 opacity  6 r  7 g  8 b            activated opacity, colour
- *   9 depth                 camera-space z, rounded to float (the sort key)
- *  10 tile_x  (bits) tx0 | tx1 << 16   inclusive tile range touched
- *  11 tile_y  (bits) ty0 | ty1 << 16   (tx0 > tx1 marks a culled Gaussian)
+ *   9 hx      10 hy         half-widths of a box around the ellipse where
+ *                           alpha >= 1/255 (q <= Q = 2 ln(255 o)): sqrt(Qp
+ *                           cov_xx) + 0.01 and sqrt(Qp cov_yy) + 0.01 with
+ *                           Qp = Q + 0.002 |Q| + 1e-4; -1 when Qp <= 0
+ *  11 zero
+ * bins [n_views][n][4] floats, 16-byte aligned (what the binning reads):
+ *   0 depth key: camera-space z as the float fma chain
+ *     fma(W20, x, fma(W21, y, fma(W22, z, t2))) of the float inputs
+ *   1 tile_x  (bits) tx0 | tx1 << 16   inclusive tile range touched
+ *   2 tile_y  (bits) ty0 | ty1 << 16   (tx0 > tx1 marks a culled Gaussian)
+ *   3 zero
  * radii [n_views][n] int32: ceil(3 sqrt(lambda_max)) of the 2D covariance,
  *   0 when culled (the densification visibility filter). */
 typedef struct gs_projected {
   float* records;
+  float* bins;
   int32_t* radii;
 } gs_projected;
 

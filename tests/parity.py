@@ -38,36 +38,33 @@ def oracle_projs(scene):
     return O.project_views(scene)
 
 
-def unpack_records(rec: np.ndarray) -> dict:
-    """GPU records [V, n, 12] -> named fields."""
-    tx = rec[..., 10].view(np.uint32)
-    ty = rec[..., 11].view(np.uint32)
+def unpack_records(rec: np.ndarray, bins: np.ndarray) -> dict:
+    """GPU records [V, n, 12] and binning records [V, n, 4] -> named fields."""
+    tx = bins[..., 1].view(np.uint32)
+    ty = bins[..., 2].view(np.uint32)
     rect = np.stack([tx & 0xFFFF, tx >> 16, ty & 0xFFFF, ty >> 16], -1).astype(np.int32)
     return dict(xy=rec[..., 0:2], conic=rec[..., 2:5], opacity=rec[..., 5], rgb=rec[..., 6:9],
-                depth=rec[..., 9], rect=rect)
+                hx=rec[..., 9], hy=rec[..., 10], depth=bins[..., 0], rect=rect)
 
 
-def pack_records(projs) -> np.ndarray:
-    """Oracle projections -> float32 records in the library's layout [V, n, 12]."""
+def pack_bins(projs) -> np.ndarray:
+    """Oracle projections -> float32 binning records in the library's layout
+    [V, n, 4]: depth key, packed tile ranges."""
     V = len(projs)
     n = projs[0]["xy"].shape[0]
-    rec = np.zeros((V, n, 12), np.float32)
+    out = np.zeros((V, n, 4), np.float32)
     for v, p in enumerate(projs):
-        rec[v, :, 0:2] = p["xy"]
-        rec[v, :, 2:5] = p["conic"]
-        rec[v, :, 5] = p["opacity"]
-        rec[v, :, 6:9] = p["rgb"]
-        rec[v, :, 9] = p["key"]
+        out[v, :, 0] = p["key"]
         r = p["rect"].astype(np.int64)
         tx = (r[:, 0] & 0xFFFF) | ((r[:, 1] & 0xFFFF) << 16)
         ty = (r[:, 2] & 0xFFFF) | ((r[:, 3] & 0xFFFF) << 16)
-        rec[v, :, 10] = tx.astype(np.uint32).view(np.float32)
-        rec[v, :, 11] = ty.astype(np.uint32).view(np.float32)
+        out[v, :, 1] = tx.astype(np.uint32).view(np.float32)
+        out[v, :, 2] = ty.astype(np.uint32).view(np.float32)
         bad = p["valid"] == 0
-        rec[v, bad, :10] = 0
-        rec[v, bad, 10] = np.uint32(1).view(np.float32)
-        rec[v, bad, 11] = np.uint32(1).view(np.float32)
-    return rec
+        out[v, bad, 0] = 0
+        out[v, bad, 1] = np.uint32(1).view(np.float32)
+        out[v, bad, 2] = np.uint32(1).view(np.float32)
+    return out
 
 
 def ambiguous_tiles(scene, projs) -> np.ndarray:

@@ -45,9 +45,10 @@ def test_project_matches_oracle(name, kw, how):
     sp.project()
     torch.cuda.synchronize()
     rec = sp.records.cpu().numpy()
+    bins = sp.bins.cpu().numpy()
     radii = sp.radii.cpu().numpy()
     for v, p in enumerate(O.project_views(sc)):
-        g = P.unpack_records(rec[v])
+        g = P.unpack_records(rec[v], bins[v])
         amb = p["ambiguous"] != 0
         assert amb.mean() < 1e-3
         vo = p["valid"] != 0
@@ -62,6 +63,15 @@ def test_project_matches_oracle(name, kw, how):
         assert np.max(np.abs(g["conic"][m] - p["conic"][m]) / scale) < 2e-6
         np.testing.assert_allclose(g["opacity"][m], p["opacity"][m], rtol=2e-6)
         np.testing.assert_allclose(g["rgb"][m], p["rgb"][m], atol=2e-5)
+        # the culling box holds the whole alpha >= 1/255 ellipse: its
+        # half-widths are at least sqrt(Q cov_xx), sqrt(Q cov_yy)
+        Q = 2 * np.log(255 * p["opacity"][m])
+        need_x = np.sqrt(np.maximum(Q, 0) * p["cov"][m, 0])
+        need_y = np.sqrt(np.maximum(Q, 0) * p["cov"][m, 2])
+        reach = Q > 0
+        assert np.all(g["hx"][m][reach] >= need_x[reach])
+        assert np.all(g["hy"][m][reach] >= need_y[reach])
+        assert np.all(g["hx"][m][Q < -1e-3] < 0)
 
 
 @pytest.mark.parametrize("mode", MODES)
@@ -109,11 +119,11 @@ def test_binning_isolated_with_ties_and_ragged_tail(mode):
     projs = [dict(xy=d["xy"][k], conic=np.zeros((n, 3)), opacity=np.zeros(n), rgb=np.zeros((n, 3)),
                   key=d["depth"][k], rect=rects[k], valid=(~bad[k]).astype(np.int32))
              for k in range(V)]
-    rec = torch.as_tensor(P.pack_records(projs)).cuda()
+    bins = torch.as_tensor(P.pack_bins(projs)).cuda()
     sc = S.make_scene("fwd_1k_128", n=n, width=W, height=H, n_views=1)
     sc.cameras = sc.cameras * V
     sp = Splatter(sc, sort_mode=mode, pair_capacity=int(((rects[..., 1] - rects[..., 0] + 1) * (rects[..., 3] - rects[..., 2] + 1))[~bad].sum()))
-    sp.records.copy_(rec)
+    sp.bins.copy_(bins)
     sp.bin_sort()
     assert sp.status() == api.GS_OK
     ids, ranges = sp.ids.cpu().numpy(), sp.ranges.cpu().numpy()
