@@ -74,11 +74,13 @@ __device__ __forceinline__ uint32_t block_exclusive_scan_256(uint32_t x, uint32_
 
 // Exclusive prefix of partition p from the look-back words of partitions
 // p-1, p-2, ... (word of partition j at base[j * stride]): one thread walks
-// back 8 partitions per round trip (8 independent loads), waiting only on
-// words still empty, until it reaches an inclusive prefix.
+// back kWin partitions per round trip (kWin independent loads), waiting only
+// on words still empty, until it reaches an inclusive prefix. The window
+// matters for throughput: with B partitions in flight a partition sums about
+// B aggregates, i.e. B / kWin round trips.
+template <int kWin>
 __device__ __forceinline__ uint64_t windowed_lookback(const uint64_t* base, int64_t stride,
                                                       int64_t p, uint32_t* status) {
-  constexpr int kWin = 8;
   uint64_t excl = 0;
   int64_t j = p - 1;
   while (j >= 0) {
@@ -158,17 +160,29 @@ __global__ void __launch_bounds__(256) k_depth_keys(const float4* __restrict__ b
   for (int k = threadIdx.x; k < 8 * kRadix; k += blockDim.x) (&s_hist[0][0])[k] = 0u;
   __syncthreads();
   const int64_t total = (int64_t)n * n_views;
-  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < total;
-       j += (int64_t)gridDim.x * blockDim.x) {
-    const float4 r2 = __ldg(&bins[j]);  // depth key, tile_x, tile_y
-    const uint32_t txw = __float_as_uint(r2.y), tyw = __float_as_uint(r2.z);
-    const bool vis = (txw & 0xffffu) <= (txw >> 16) && (tyw & 0xffffu) <= (tyw >> 16);
-    const int view = (int)(j / n);
-    const uint64_t key =
-        vis ? (((uint64_t)view << 32) | (uint64_t)__float_as_uint(r2.x)) : ~0ull;
-    keys[j] = key;
-    vals[j] = (uint32_t)(j - (int64_t)view * n);
-    for (int d = 0; d < passes; ++d) atomicAdd(&s_hist[d][(key >> (8 * d)) & 0xff], 1u);
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const uint32_t lt = lanemask_lt();
+  // uniform trip count per warp so the match.any below sees every lane
+  for (int64_t j0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); j0 < total;
+       j0 += stride) {
+    const int64_t j = j0 + (threadIdx.x & 31);
+    const bool in = j < total;
+    uint64_t key = ~0ull;
+    if (in) {
+      const float4 r2 = __ldg(&bins[j]);  // depth key, tile_x, tile_y
+      const uint32_t txw = __float_as_uint(r2.y), tyw = __float_as_uint(r2.z);
+      const bool vis = (txw & 0xffffu) <= (txw >> 16) && (tyw & 0xffffu) <= (tyw >> 16);
+      const int view = (int)(j / n);
+      key = vis ? (((uint64_t)view << 32) | (uint64_t)__float_as_uint(r2.x)) : ~0ull;
+      keys[j] = key;
+      vals[j] = (uint32_t)(j - (int64_t)view * n);
+    }
+    // warp-aggregated histogram: one shared atomic per distinct digit
+    for (int d = 0; d < passes; ++d) {
+      const uint32_t dv = in ? (uint32_t)((key >> (8 * d)) & 0xff) : 256u;
+      const uint32_t peers = __match_any_sync(0xffffffffu, dv);
+      if (in && (peers & lt) == 0) atomicAdd(&s_hist[d][dv], (uint32_t)__popc(peers));
+    }
   }
   __syncthreads();
   for (int k = threadIdx.x; k < passes * kRadix; k += blockDim.x) {
@@ -183,7 +197,17 @@ __global__ void __launch_bounds__(256) k_depth_keys(const float4* __restrict__ b
 //   order; key = (global tile << 32) | depth bits.
 // MODE 1 (presorted): items are the presorted (key, index) list; key = global
 //   tile (32-bit).
-// Histograms: digit d of the emitted keys into hist[d][256] for d < passes.
+// An item's pairs are its rectangle's tiles in row-major order.
+// Counting: each thread takes 4 consecutive items; block scan; decoupled
+// look-back for the block's global offset.
+// Emission, window by window of the block's pairs: thread t takes pairs
+// 8t .. 8t+7 of the window (4 in MODE 0) -- one binary search over the item
+// offsets, then row / column stepping -- and stages them in shared memory
+// (one pad word per 32 so the strided writes hit distinct banks); the block
+// then writes the window out with coalesced stores.
+// Histograms of the following radix passes (digit d into hist[d][256] for
+// d < passes): depth digits once per item weighted by its pair count, tile
+// byte 0 per pair, higher tile bytes as per-thread runs.
 template <int MODE, typename K>
 __global__ void __launch_bounds__(kEmitThreads) k_emit(
     const float4* __restrict__ bins, const uint64_t* __restrict__ pkeys,
@@ -192,12 +216,18 @@ __global__ void __launch_bounds__(kEmitThreads) k_emit(
     int64_t* __restrict__ n_pairs, unsigned long long* __restrict__ hist,
     uint64_t* __restrict__ lookback, uint32_t* __restrict__ block_counter,
     uint32_t* __restrict__ status) {
+  constexpr int kPer = MODE == 0 ? 4 : 8;           // pairs per thread per window
+  constexpr int kWin = kPer * kEmitThreads;         // pairs per window
+  constexpr int kWinPad = kWin + kWin / 32;
+  constexpr int kTileDigit0 = MODE == 0 ? 4 : 0;    // digit index of tile byte 0
   __shared__ uint32_t s_off[kEmitItems + 1];
-  __shared__ uint32_t s_rect[kEmitItems];   // x0 | width << 16
-  __shared__ uint32_t s_rect2[kEmitItems];  // y0 | view << 16
+  __shared__ uint32_t s_rx[kEmitItems];   // x0 | width << 16
+  __shared__ uint32_t s_ry[kEmitItems];   // y0 | view << 16
   __shared__ uint32_t s_id[kEmitItems];
-  __shared__ uint32_t s_depth[kEmitItems];
+  __shared__ uint32_t s_depth[MODE == 0 ? kEmitItems : 1];
   __shared__ uint32_t s_hist[8][kRadix];
+  __shared__ K s_key[kWinPad];
+  __shared__ uint32_t s_sid[kWinPad];
   __shared__ uint32_t s_warp[9];
   __shared__ uint64_t s_base;
 
@@ -215,18 +245,18 @@ __global__ void __launch_bounds__(kEmitThreads) k_emit(
     uint32_t c = 0, rx = 0, ry = 0, id = 0, depth = 0;
     if (item < n_items) {
       int64_t rec_index;
-      int view;
+      int vw;
       if (MODE == 0) {
-        view = (int)(item / n);
-        id = (uint32_t)(item - (int64_t)view * n);
+        vw = (int)(item / n);
+        id = (uint32_t)(item - (int64_t)vw * n);
         rec_index = item;
       } else {
         const uint64_t pk = pkeys[item];
-        view = pk == ~0ull ? -1 : (int)(pk >> 32);
+        vw = pk == ~0ull ? -1 : (int)(pk >> 32);
         id = pvals[item];
-        rec_index = (int64_t)(view < 0 ? 0 : view) * n + id;
+        rec_index = (int64_t)(vw < 0 ? 0 : vw) * n + id;
       }
-      if (view >= 0) {
+      if (vw >= 0) {
         const float4 r2 = __ldg(&bins[rec_index]);
         const uint32_t txw = __float_as_uint(r2.y), tyw = __float_as_uint(r2.z);
         const uint32_t x0 = txw & 0xffffu, x1 = txw >> 16, y0 = tyw & 0xffffu, y1 = tyw >> 16;
@@ -234,16 +264,16 @@ __global__ void __launch_bounds__(kEmitThreads) k_emit(
           const uint32_t w = x1 - x0 + 1;
           c = w * (y1 - y0 + 1);
           rx = x0 | (w << 16);
-          ry = y0 | ((uint32_t)view << 16);
+          ry = y0 | ((uint32_t)vw << 16);
           depth = __float_as_uint(r2.x);
         }
       }
     }
     cnt[k] = c;
-    s_rect[threadIdx.x * kEmitItemsPerThread + k] = rx;
-    s_rect2[threadIdx.x * kEmitItemsPerThread + k] = ry;
-    s_id[threadIdx.x * kEmitItemsPerThread + k] = id;
-    s_depth[threadIdx.x * kEmitItemsPerThread + k] = depth;
+    s_rx[li] = rx;
+    s_ry[li] = ry;
+    s_id[li] = id;
+    if (MODE == 0) s_depth[li] = depth;
     tsum += c;
   }
   uint32_t block_total;
@@ -278,31 +308,78 @@ __global__ void __launch_bounds__(kEmitThreads) k_emit(
     }
   }
 
-  const int tiles_x = g.tiles_x, tpv = g.tiles_per_view;
-  for (uint32_t j = threadIdx.x; j < block_total; j += kEmitThreads) {
-    // item owning pair j: largest k with s_off[k] <= j
-    int lo = 0, hi = kEmitItems - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_off[mid] <= j) lo = mid; else hi = mid - 1;
+  const uint32_t tiles_x = (uint32_t)g.tiles_x, tpv = (uint32_t)g.tiles_per_view;
+  const int n_tile_digits = passes - kTileDigit0;
+  for (uint32_t w0 = 0; w0 < block_total; w0 += kWin) {
+    const uint32_t p0 = w0 + threadIdx.x * kPer;
+    if (p0 < block_total) {
+      // item owning pair p0: largest k with s_off[k] <= p0 (skips empty items)
+      int lo = 0, hi = kEmitItems - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_off[mid] <= p0) lo = mid; else hi = mid - 1;
+      }
+      int k = lo;
+      uint32_t end_k = s_off[k + 1];
+      uint32_t rx = s_rx[k], ry = s_ry[k];
+      uint32_t w = rx >> 16;
+      const uint32_t local = p0 - s_off[k];
+      uint32_t row = local / w, col = local - row * w;
+      uint32_t id = s_id[k];
+      uint32_t depth = MODE == 0 ? s_depth[k] : 0u;
+      uint32_t run_v[3] = {0u, 0u, 0u}, run_n[3] = {0u, 0u, 0u};
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const uint32_t p = p0 + i;
+        if (p >= block_total) break;
+        if (p >= end_k) {  // next item that has pairs
+          do {
+            ++k;
+            end_k = s_off[k + 1];
+          } while (p >= end_k);
+          rx = s_rx[k];
+          ry = s_ry[k];
+          w = rx >> 16;
+          row = 0;
+          col = 0;
+          id = s_id[k];
+          if (MODE == 0) depth = s_depth[k];
+        }
+        const uint32_t tile = (ry >> 16) * tpv + ((ry & 0xffffu) + row) * tiles_x + (rx & 0xffffu) + col;
+        const uint32_t q = p - w0;
+        const uint32_t si = q + (q >> 5);
+        s_key[si] = MODE == 0 ? (K)(((uint64_t)tile << 32) | depth) : (K)tile;
+        s_sid[si] = id;
+        atomicAdd(&s_hist[kTileDigit0][tile & 255u], 1u);
+#pragma unroll
+        for (int dd = 1; dd < 4; ++dd) {
+          if (dd >= n_tile_digits) break;
+          const uint32_t dv = (tile >> (8 * dd)) & 255u;
+          if (run_n[dd - 1] && dv != run_v[dd - 1]) {
+            atomicAdd(&s_hist[kTileDigit0 + dd][run_v[dd - 1]], run_n[dd - 1]);
+            run_n[dd - 1] = 0;
+          }
+          run_v[dd - 1] = dv;
+          ++run_n[dd - 1];
+        }
+        if (++col == w) {
+          col = 0;
+          ++row;
+        }
+      }
+#pragma unroll
+      for (int dd = 1; dd < 4; ++dd)
+        if (run_n[dd - 1]) atomicAdd(&s_hist[kTileDigit0 + dd][run_v[dd - 1]], run_n[dd - 1]);
     }
-    const uint32_t local = j - s_off[lo];
-    const uint32_t rx = s_rect[lo], ry = s_rect2[lo];
-    const uint32_t w = rx >> 16;
-    const uint32_t ty = (ry & 0xffffu) + local / w;
-    const uint32_t tx = (rx & 0xffffu) + local % w;
-    const uint32_t view = ry >> 16;
-    const uint32_t tile = view * (uint32_t)tpv + ty * (uint32_t)tiles_x + tx;
-    K key;
-    if (MODE == 0) key = (K)(((uint64_t)tile << 32) | (uint64_t)s_depth[lo]);
-    else key = (K)tile;
-    keys_out[base + j] = key;
-    ids_out[base + j] = s_id[lo];
-    const int first_pair_digit = MODE == 0 ? 4 : 0;
-    for (int d = first_pair_digit; d < passes; ++d)
-      atomicAdd(&s_hist[d][(uint32_t)(((uint64_t)key) >> (8 * d)) & 0xff], 1u);
+    __syncthreads();
+    const uint32_t m = min((uint32_t)kWin, block_total - w0);
+    for (uint32_t q = threadIdx.x; q < m; q += kEmitThreads) {
+      const uint32_t si = q + (q >> 5);
+      keys_out[base + w0 + q] = s_key[si];
+      ids_out[base + w0 + q] = s_sid[si];
+    }
+    __syncthreads();
   }
-  __syncthreads();
   for (int k = threadIdx.x; k < passes * kRadix; k += kEmitThreads) {
     const uint32_t c = (&s_hist[0][0])[k];
     if (c) atomicAdd(&hist[k], (unsigned long long)c);
@@ -324,9 +401,30 @@ __global__ void k_clear_lookback(uint64_t* __restrict__ lb, const int64_t* __res
   }
 }
 
-// One stable LSD radix pass over digit (key >> shift) & 0xff.
+// Blocks per SM of the radix pass, by key width (register budget).
 template <typename K>
-__global__ void __launch_bounds__(kSortThreads, 2) k_onesweep(
+struct SortOcc;
+template <>
+struct SortOcc<uint32_t> {
+  static constexpr int kBlocks = 3;
+};
+template <>
+struct SortOcc<uint64_t> {
+  static constexpr int kBlocks = 2;
+};
+
+// One stable LSD radix pass over digit (key >> shift) & 0xff.
+// Per partition of kSortTile keys: (1) all keys and values are loaded first
+// (independent loads in flight together); (2) per-warp digit counts with
+// shared-memory atomics; (3) per digit, the counts over warps give each
+// warp's offset and the block's count, which is published to the look-back
+// array at once, before ranking; (4) each warp ranks its keys stably with
+// match.any over warp-striped steps; (5) scatter into shared memory in
+// sorted order; (6) look-back for the global offset of every digit (32
+// predecessors per round trip); (7) write runs of equal digits to global
+// memory.
+template <typename K>
+__global__ void __launch_bounds__(kSortThreads, SortOcc<K>::kBlocks) k_onesweep(
     const K* __restrict__ keys_in, const uint32_t* __restrict__ vals_in,
     K* __restrict__ keys_out, uint32_t* __restrict__ vals_out,
     const int64_t* __restrict__ n_ptr, int64_t capacity, int shift,
@@ -351,7 +449,6 @@ __global__ void __launch_bounds__(kSortThreads, 2) k_onesweep(
   // global exclusive prefix of this digit's histogram (same for every block)
   {
     const unsigned long long c = hist[tid];
-    // 64-bit exclusive scan over 256 threads
     unsigned long long incl = c;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -367,77 +464,83 @@ __global__ void __launch_bounds__(kSortThreads, 2) k_onesweep(
     __syncthreads();
   }
 
+  uint32_t* wh = s_whist + warp * (kRadix + 1);
+  const uint32_t lt = lanemask_lt();
   while (true) {
     if (tid == 0) s_part = atomicAdd(part_counter, 1u);
     for (int k = tid; k < kSortWarps * (kRadix + 1); k += kSortThreads) s_whist[k] = 0u;
     __syncthreads();
     const int64_t p = s_part;
     if (p >= parts) break;
-    const int64_t tile_first = p * kSortTile;
+    const int64_t first = p * kSortTile + warp * (kSortItems * 32);
 
-    // load (warp-striped) and rank within the warp, stably
+    // (1) loads, warp-striped: step `it` of this warp covers 32 consecutive keys
     K key[kSortItems];
     uint32_t val[kSortItems];
-    uint32_t rank[kSortItems];
-    uint32_t dig[kSortItems];
-    uint32_t* wh = s_whist + warp * (kRadix + 1);
-    const uint32_t lt = lanemask_lt();
 #pragma unroll
     for (int it = 0; it < kSortItems; ++it) {
-      const int64_t idx = tile_first + warp * (kSortItems * 32) + it * 32 + lane;
-      const bool valid = idx < n;
-      key[it] = valid ? keys_in[idx] : (K)0;
-      val[it] = valid ? vals_in[idx] : 0u;
-      const uint32_t d = valid ? (uint32_t)((key[it] >> shift) & 0xff) : (uint32_t)kRadix;
-      dig[it] = d;
+      const int64_t idx = first + it * 32 + lane;
+      key[it] = idx < n ? keys_in[idx] : (K)0;
+      val[it] = idx < n ? vals_in[idx] : 0u;
+    }
+    // (2) per-warp digit counts (digit 256 marks an empty slot)
+#pragma unroll
+    for (int it = 0; it < kSortItems; ++it) {
+      const int64_t idx = first + it * 32 + lane;
+      const uint32_t d = idx < n ? (uint32_t)((key[it] >> shift) & 0xff) : (uint32_t)kRadix;
+      atomicAdd(&wh[d], 1u);
+    }
+    __syncthreads();
+    // (3) per digit: warp offsets, block count, early aggregate
+    const int b = tid;  // 256 threads == 256 digits
+    uint32_t count = 0;
+#pragma unroll
+    for (int w = 0; w < kSortWarps; ++w) {
+      const uint32_t c = s_whist[w * (kRadix + 1) + b];
+      s_whist[w * (kRadix + 1) + b] = count;
+      count += c;
+    }
+    uint64_t* lb = lookback + p * kRadix + b;
+    st_relaxed_u64(lb, (p == 0 ? kLbPrefix : kLbAggregate) | (uint64_t)count);
+    uint32_t tot;
+    const uint32_t lstart = block_exclusive_scan_256(count, s_scan, tot);
+    s_lstart[b] = lstart;
+    // running position of each digit for this warp = local start + warp offset
+#pragma unroll
+    for (int w = 0; w < kSortWarps; ++w) s_whist[w * (kRadix + 1) + b] += lstart;
+    __syncthreads();
+    // (4) stable rank within the warp -> final position within the partition
+    uint32_t pos[kSortItems];
+#pragma unroll
+    for (int it = 0; it < kSortItems; ++it) {
+      const int64_t idx = first + it * 32 + lane;
+      const uint32_t d = idx < n ? (uint32_t)((key[it] >> shift) & 0xff) : (uint32_t)kRadix;
       const uint32_t peers = __match_any_sync(0xffffffffu, d);
       const uint32_t before = wh[d];
       __syncwarp();
       if ((peers & lt) == 0) wh[d] = before + __popc(peers);
       __syncwarp();
-      rank[it] = before + __popc(peers & lt);
+      pos[it] = before + __popc(peers & lt);
     }
-    __syncthreads();
-
-    // per digit: counts over warps -> exclusive warp offsets, block count
-    uint32_t count = 0;
-    {
-      const int b = tid;  // 256 threads == 256 digits
-#pragma unroll
-      for (int w = 0; w < kSortWarps; ++w) {
-        const uint32_t c = s_whist[w * (kRadix + 1) + b];
-        s_whist[w * (kRadix + 1) + b] = count;
-        count += c;
-      }
-      // decoupled look-back across partitions for this digit
-      uint64_t* lb = lookback + p * kRadix + b;
-      uint64_t excl = 0;
-      if (p == 0) {
-        st_relaxed_u64(lb, kLbPrefix | (uint64_t)count);
-      } else {
-        st_relaxed_u64(lb, kLbAggregate | (uint64_t)count);
-        excl = windowed_lookback(lookback + b, kRadix, p, status);
-        st_relaxed_u64(lb, kLbPrefix | (excl + count));
-      }
-      s_gbase[b] = s_gexcl[b] + excl;
-    }
-    uint32_t tot;
-    const uint32_t lstart = block_exclusive_scan_256(count, s_scan, tot);
-    s_lstart[tid] = lstart;
-    __syncthreads();
-
-    // scatter into shared memory in sorted order
+    // (5) scatter into shared memory in sorted order (frees the registers)
 #pragma unroll
     for (int it = 0; it < kSortItems; ++it) {
-      const uint32_t d = dig[it];
-      if (d < (uint32_t)kRadix) {
-        const uint32_t pos = s_lstart[d] + s_whist[warp * (kRadix + 1) + d] + rank[it];
-        s_keys[pos] = key[it];
-        s_vals[pos] = val[it];
+      const int64_t idx = first + it * 32 + lane;
+      if (idx < n) {
+        s_keys[pos[it]] = key[it];
+        s_vals[pos[it]] = val[it];
       }
     }
+    // (6) look-back: global start of each digit's run from this partition
+    uint64_t excl = 0;
+    if (p > 0) {
+      excl = windowed_lookback<32>(lookback + b, kRadix, p, status);
+      st_relaxed_u64(lb, kLbPrefix | (excl + count));
+    }
+    s_gbase[b] = s_gexcl[b] + excl;
     __syncthreads();
-    const int64_t remain = n - tile_first;
+    // (7) write runs of equal digits out
+    const int64_t remain = n - p * kSortTile;
     const int valid_count = remain < kSortTile ? (int)remain : kSortTile;
     for (int j = tid; j < valid_count; j += kSortThreads) {
       const K k = s_keys[j];
