@@ -5,18 +5,25 @@
 // Julia", pwwt.cn sec. 3.3 steps 1-2 and 4.3; lshu.cn sec. 3.2
 // assign_to_tiles / sort_by_depth!), ties broken by Gaussian index.
 //
-//  k_emit      one pass over the Gaussians: per-Gaussian pair counts, a
-//              single-pass scan (decoupled look-back between blocks), and
-//              load-balanced emission of (key, id) pairs by the whole block;
-//              the digit histograms of the following radix passes are
-//              accumulated on the way, so the sort needs no upsweep pass.
-//  k_onesweep  one least-significant-digit pass of a stable radix sort with
-//              8-bit digits: warp-level ranking with match.any, per-digit
-//              decoupled look-back across partitions, scatter through shared
-//              memory so global writes are runs of equal digits.
-//  k_ranges    [start, end) of each tile in the sorted pairs.
-// Every device-side wait is bounded (kSpinLimit) and reports through the
-// status word instead of hanging.
+//  k_depth_keys    (presort mode) per-Gaussian (view, depth) keys + digit
+//                  histograms.
+//  k_emit          one pass over the Gaussians: pair counts, a single-pass
+//                  scan across blocks (decoupled look-back, one warp reading
+//                  32 predecessors per round trip) and emission of the
+//                  (key, id) pairs through shared-memory staging; the digit
+//                  histograms of every following radix pass are accumulated
+//                  on the way.
+//  k_radix_count / k_radix_scan / k_radix_scatter
+//                  one stable least-significant-digit radix pass with 8-bit
+//                  digits, reduce-then-scan: per-partition digit counts, a
+//                  per-digit scan over partitions, then a scatter that ranks
+//                  each partition's keys stably (ballots over warp-striped
+//                  steps), stages them in shared memory and writes runs of
+//                  equal digits.
+//  k_ranges        [start, end) of each tile in the sorted pairs.
+// The emission's look-back waits are bounded (kSpinLimit) and report through
+// the status word instead of hanging; the radix passes never wait on other
+// blocks.
 
 #include <cuda_runtime.h>
 
@@ -72,34 +79,34 @@ __device__ __forceinline__ uint32_t block_exclusive_scan_256(uint32_t x, uint32_
   return r;
 }
 
-// Exclusive prefix of partition p from the look-back words of partitions
-// p-1, p-2, ... (word of partition j at base[j * stride]): one thread walks
-// back kWin partitions per round trip (kWin independent loads), waiting only
-// on words still empty, until it reaches an inclusive prefix. The window
-// matters for throughput: with B partitions in flight a partition sums about
-// B aggregates, i.e. B / kWin round trips.
-template <int kWin>
-__device__ __forceinline__ uint64_t windowed_lookback(const uint64_t* base, int64_t stride,
-                                                      int64_t p, uint32_t* status) {
-  uint64_t excl = 0;
-  int64_t j = p - 1;
-  while (j >= 0) {
-    uint64_t w[kWin];
+// Exclusive block-wide scan of one uint64 per thread (256 threads).
+__device__ __forceinline__ uint64_t block_exclusive_scan_256_u64(uint64_t x, uint64_t* s_warp,
+                                                                 uint64_t& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint64_t incl = x;
 #pragma unroll
-    for (int k = 0; k < kWin; ++k) w[k] = (j - k >= 0) ? ld_relaxed_u64(base + (j - k) * stride) : 0ull;
-    bool found = false;
-#pragma unroll
-    for (int k = 0; k < kWin; ++k) {
-      if (found || j - k < 0) continue;
-      uint64_t v = w[k];
-      if ((v >> 62) == 0) v = lookback_wait(base + (j - k) * stride, status);
-      excl += v & kLbValueMask;
-      if ((v >> 62) == 2) found = true;
-    }
-    if (found) break;
-    j -= kWin;
+  for (int o = 1; o < 32; o <<= 1) {
+    uint64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
   }
-  return excl;
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    uint64_t w = lane < 8 ? s_warp[lane] : 0ull;
+    uint64_t wi = w;
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      uint64_t y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
+    }
+    if (lane < 8) s_warp[lane] = wi - w;
+    if (lane == 7) s_warp[8] = wi;
+  }
+  __syncthreads();
+  total = s_warp[8];
+  uint64_t r = s_warp[warp] + incl - x;
+  __syncthreads();
+  return r;
 }
 
 // Decoupled look-back for one value per block, run by warp 0 of the block.
@@ -139,10 +146,12 @@ struct KeyTraits;
 template <>
 struct KeyTraits<uint64_t> {
   static constexpr int kBits = 64;
+  static constexpr int kBlocks = 2;  // radix scatter blocks per SM (registers)
 };
 template <>
 struct KeyTraits<uint32_t> {
   static constexpr int kBits = 32;
+  static constexpr int kBlocks = 3;
 };
 
 // ---------------------------------------------------------------------------
@@ -191,7 +200,6 @@ __global__ void __launch_bounds__(256) k_depth_keys(const float4* __restrict__ b
   }
 }
 
-// ---------------------------------------------------------------------------
 // Fused pair count + scan + emission.
 // MODE 0 (full 64-bit keys): items are the n_views * n Gaussians in index
 //   order; key = (global tile << 32) | depth bits.
@@ -386,174 +394,180 @@ __global__ void __launch_bounds__(kEmitThreads) k_emit(
   }
 }
 
-// Clear the look-back words of `passes` regions for the pair count now in
-// *n_items (device), partitions of kSortTile keys.
-__global__ void k_clear_lookback(uint64_t* __restrict__ lb, const int64_t* __restrict__ n_items,
-                                 int64_t capacity, int passes, int64_t region_words) {
-  const int64_t n = *n_items;
-  if (n > capacity) return;
-  const int64_t words = ((n + kSortTile - 1) / kSortTile) * kRadix;
-  for (int p = 0; p < passes; ++p) {
-    uint64_t* base = lb + p * region_words;
-    for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < words;
-         w += (int64_t)gridDim.x * blockDim.x)
-      base[w] = 0ull;
+// ---------------------------------------------------------------------------
+// Radix pass, reduce-then-scan. Partition p holds keys [p * kSortTile, ...).
+// counts / offsets: uint64 [256][stride], digit-major.
+
+// (1) digit counts of one partition (per-warp shared histograms).
+template <typename K>
+__global__ void __launch_bounds__(kSortThreads) k_radix_count(
+    const K* __restrict__ keys, const int64_t* __restrict__ n_ptr, int64_t capacity, int shift,
+    uint64_t* __restrict__ counts, int64_t stride) {
+  __shared__ uint32_t s_h[kSortWarps][kRadix];
+  const int64_t n = *n_ptr;
+  if (n > capacity || n <= 0) return;
+  const int64_t p = blockIdx.x;
+  if (p * kSortTile >= n) return;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int k = tid; k < kSortWarps * kRadix; k += kSortThreads) (&s_h[0][0])[k] = 0u;
+  const int64_t first = p * kSortTile + warp * (kSortItems * 32);
+  K key[kSortItems];
+#pragma unroll
+  for (int it = 0; it < kSortItems; ++it) {
+    const int64_t idx = first + it * 32 + lane;
+    key[it] = idx < n ? keys[idx] : (K)0;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int it = 0; it < kSortItems; ++it) {
+    const int64_t idx = first + it * 32 + lane;
+    if (idx < n) atomicAdd(&s_h[warp][(uint32_t)((key[it] >> shift) & 0xff)], 1u);
+  }
+  __syncthreads();
+  uint32_t c = 0;
+#pragma unroll
+  for (int w = 0; w < kSortWarps; ++w) c += s_h[w][tid];
+  counts[(int64_t)tid * stride + p] = c;
+}
+
+// (2) per digit (one block each): exclusive scan of its counts over the
+// partitions, plus the number of keys with a smaller digit, in place.
+__global__ void __launch_bounds__(256) k_radix_scan(uint64_t* __restrict__ counts, int64_t stride,
+                                                   const int64_t* __restrict__ n_ptr,
+                                                   int64_t capacity,
+                                                   const unsigned long long* __restrict__ hist) {
+  __shared__ uint64_t s_warp[9];
+  __shared__ uint64_t s_base;
+  const int64_t n = *n_ptr;
+  if (n > capacity || n <= 0) return;
+  const int64_t parts = (n + kSortTile - 1) / kSortTile;
+  const int d = blockIdx.x;
+  const int tid = threadIdx.x;
+  if (tid < 32) {
+    uint64_t s = 0;
+    for (int k = tid; k < d; k += 32) s += hist[k];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (tid == 0) s_base = s;
+  }
+  uint64_t* row = counts + (int64_t)d * stride;
+  // thread t scans partitions [t * chunk, (t + 1) * chunk)
+  const int64_t chunk = (parts + 255) / 256;
+  const int64_t b0 = (int64_t)tid * chunk;
+  const int64_t b1 = min(parts, b0 + chunk);
+  uint64_t sum = 0;
+  for (int64_t q = b0; q < b1; ++q) sum += row[q];
+  uint64_t tot;
+  uint64_t run = block_exclusive_scan_256_u64(sum, s_warp, tot) + s_base;
+  for (int64_t q = b0; q < b1; ++q) {
+    const uint64_t c = row[q];
+    row[q] = run;
+    run += c;
   }
 }
 
-// Blocks per SM of the radix pass, by key width (register budget).
-template <typename K>
-struct SortOcc;
-template <>
-struct SortOcc<uint32_t> {
-  static constexpr int kBlocks = 3;
-};
-template <>
-struct SortOcc<uint64_t> {
-  static constexpr int kBlocks = 2;
-};
+// Lanes of the warp holding the same value d (d < 512): the intersection over
+// the 9 bits of d of the ballot of lanes agreeing on that bit. Costs the same
+// whatever the values (unlike match.any, whose cost grows with the number of
+// distinct values).
+__device__ __forceinline__ uint32_t warp_peers_9bit(uint32_t d) {
+  uint32_t peers = 0xffffffffu;
+#pragma unroll
+  for (int b = 0; b < 9; ++b) {
+    const uint32_t bal = __ballot_sync(0xffffffffu, (d >> b) & 1u);
+    peers &= ((d >> b) & 1u) ? bal : ~bal;
+  }
+  return peers;
+}
 
-// One stable LSD radix pass over digit (key >> shift) & 0xff.
-// Per partition of kSortTile keys: (1) all keys and values are loaded first
-// (independent loads in flight together); (2) per-warp digit counts with
-// shared-memory atomics; (3) per digit, the counts over warps give each
-// warp's offset and the block's count, which is published to the look-back
-// array at once, before ranking; (4) each warp ranks its keys stably with
-// match.any over warp-striped steps; (5) scatter into shared memory in
-// sorted order; (6) look-back for the global offset of every digit (32
-// predecessors per round trip); (7) write runs of equal digits to global
-// memory.
+// (3) stable scatter of one partition: loads (warp-striped), per-warp digit
+// counts, block-local digit starts, ranking by ballots, staging in shared
+// memory in sorted order, then runs of equal digits written at their global
+// offsets.
 template <typename K>
-__global__ void __launch_bounds__(kSortThreads, SortOcc<K>::kBlocks) k_onesweep(
+__global__ void __launch_bounds__(kSortThreads, KeyTraits<K>::kBlocks) k_radix_scatter(
     const K* __restrict__ keys_in, const uint32_t* __restrict__ vals_in,
     K* __restrict__ keys_out, uint32_t* __restrict__ vals_out,
     const int64_t* __restrict__ n_ptr, int64_t capacity, int shift,
-    const unsigned long long* __restrict__ hist, uint64_t* __restrict__ lookback,
-    uint32_t* __restrict__ part_counter, uint32_t* __restrict__ status) {
+    const uint64_t* __restrict__ offsets, int64_t stride, uint32_t* __restrict__ status) {
   // layout: 64-bit arrays first so every carve-out is naturally aligned
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  uint64_t* s_gexcl = reinterpret_cast<uint64_t*>(smem_raw);            // [256]
-  uint64_t* s_gbase = s_gexcl + kRadix;                                 // [256]
+  uint64_t* s_gbase = reinterpret_cast<uint64_t*>(smem_raw);            // [256]
   K* s_keys = reinterpret_cast<K*>(s_gbase + kRadix);                   // [tile]
   uint32_t* s_vals = reinterpret_cast<uint32_t*>(s_keys + kSortTile);   // [tile]
   uint32_t* s_whist = s_vals + kSortTile;                               // [warps][257]
   uint32_t* s_lstart = s_whist + kSortWarps * (kRadix + 1);             // [256]
   uint32_t* s_scan = s_lstart + kRadix;                                 // [16]
-  __shared__ uint32_t s_part;
 
   const int64_t n = *n_ptr;
   if (n > capacity || n <= 0) return;
-  const int64_t parts = (n + kSortTile - 1) / kSortTile;
+  const int64_t p = blockIdx.x;
+  if (p * kSortTile >= n) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-  // global exclusive prefix of this digit's histogram (same for every block)
-  {
-    const unsigned long long c = hist[tid];
-    unsigned long long incl = c;
+  for (int k = tid; k < kSortWarps * (kRadix + 1); k += kSortThreads) s_whist[k] = 0u;
+  const int64_t first = p * kSortTile + warp * (kSortItems * 32);
+  K key[kSortItems];
+  uint32_t val[kSortItems];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    __shared__ unsigned long long s_w[8];
-    if (lane == 31) s_w[warp] = incl;
-    __syncthreads();
-    unsigned long long wo = 0;
-    for (int w = 0; w < warp; ++w) wo += s_w[w];
-    s_gexcl[tid] = wo + incl - c;
-    __syncthreads();
+  for (int it = 0; it < kSortItems; ++it) {
+    const int64_t idx = first + it * 32 + lane;
+    key[it] = idx < n ? keys_in[idx] : (K)0;
+    val[it] = idx < n ? vals_in[idx] : 0u;
   }
-
+  s_gbase[tid] = offsets[(int64_t)tid * stride + p];
+  __syncthreads();
   uint32_t* wh = s_whist + warp * (kRadix + 1);
+#pragma unroll
+  for (int it = 0; it < kSortItems; ++it) {
+    const int64_t idx = first + it * 32 + lane;
+    const uint32_t d = idx < n ? (uint32_t)((key[it] >> shift) & 0xff) : (uint32_t)kRadix;
+    atomicAdd(&wh[d], 1u);
+  }
+  __syncthreads();
+  // per digit: warp offsets, block count, block-local start
+  uint32_t count = 0;
+#pragma unroll
+  for (int w = 0; w < kSortWarps; ++w) {
+    const uint32_t c = s_whist[w * (kRadix + 1) + tid];
+    s_whist[w * (kRadix + 1) + tid] = count;
+    count += c;
+  }
+  uint32_t tot;
+  const uint32_t lstart = block_exclusive_scan_256(count, s_scan, tot);
+  s_lstart[tid] = lstart;
+#pragma unroll
+  for (int w = 0; w < kSortWarps; ++w) s_whist[w * (kRadix + 1) + tid] += lstart;
+  __syncthreads();
+  // stable rank within the warp -> position within the partition
   const uint32_t lt = lanemask_lt();
-  while (true) {
-    if (tid == 0) s_part = atomicAdd(part_counter, 1u);
-    for (int k = tid; k < kSortWarps * (kRadix + 1); k += kSortThreads) s_whist[k] = 0u;
-    __syncthreads();
-    const int64_t p = s_part;
-    if (p >= parts) break;
-    const int64_t first = p * kSortTile + warp * (kSortItems * 32);
-
-    // (1) loads, warp-striped: step `it` of this warp covers 32 consecutive keys
-    K key[kSortItems];
-    uint32_t val[kSortItems];
 #pragma unroll
-    for (int it = 0; it < kSortItems; ++it) {
-      const int64_t idx = first + it * 32 + lane;
-      key[it] = idx < n ? keys_in[idx] : (K)0;
-      val[it] = idx < n ? vals_in[idx] : 0u;
+  for (int it = 0; it < kSortItems; ++it) {
+    const int64_t idx = first + it * 32 + lane;
+    const uint32_t d = idx < n ? (uint32_t)((key[it] >> shift) & 0xff) : (uint32_t)kRadix;
+    const uint32_t peers = warp_peers_9bit(d);
+    const uint32_t before = wh[d];
+    __syncwarp();
+    if ((peers & lt) == 0) wh[d] = before + __popc(peers);
+    __syncwarp();
+    if (idx < n) {
+      const uint32_t pos = before + __popc(peers & lt);
+      s_keys[pos] = key[it];
+      s_vals[pos] = val[it];
     }
-    // (2) per-warp digit counts (digit 256 marks an empty slot)
-#pragma unroll
-    for (int it = 0; it < kSortItems; ++it) {
-      const int64_t idx = first + it * 32 + lane;
-      const uint32_t d = idx < n ? (uint32_t)((key[it] >> shift) & 0xff) : (uint32_t)kRadix;
-      atomicAdd(&wh[d], 1u);
+  }
+  __syncthreads();
+  const int64_t remain = n - p * kSortTile;
+  const int valid_count = remain < kSortTile ? (int)remain : kSortTile;
+  for (int j = tid; j < valid_count; j += kSortThreads) {
+    const K k = s_keys[j];
+    const uint32_t d = (uint32_t)((k >> shift) & 0xff);
+    const uint64_t gpos = s_gbase[d] + (uint64_t)(j - (int)s_lstart[d]);
+    if (gpos < (uint64_t)n) {
+      keys_out[gpos] = k;
+      vals_out[gpos] = s_vals[j];
+    } else {
+      atomicOr(status, kStatusBounds);
     }
-    __syncthreads();
-    // (3) per digit: warp offsets, block count, early aggregate
-    const int b = tid;  // 256 threads == 256 digits
-    uint32_t count = 0;
-#pragma unroll
-    for (int w = 0; w < kSortWarps; ++w) {
-      const uint32_t c = s_whist[w * (kRadix + 1) + b];
-      s_whist[w * (kRadix + 1) + b] = count;
-      count += c;
-    }
-    uint64_t* lb = lookback + p * kRadix + b;
-    st_relaxed_u64(lb, (p == 0 ? kLbPrefix : kLbAggregate) | (uint64_t)count);
-    uint32_t tot;
-    const uint32_t lstart = block_exclusive_scan_256(count, s_scan, tot);
-    s_lstart[b] = lstart;
-    // running position of each digit for this warp = local start + warp offset
-#pragma unroll
-    for (int w = 0; w < kSortWarps; ++w) s_whist[w * (kRadix + 1) + b] += lstart;
-    __syncthreads();
-    // (4) stable rank within the warp -> final position within the partition
-    uint32_t pos[kSortItems];
-#pragma unroll
-    for (int it = 0; it < kSortItems; ++it) {
-      const int64_t idx = first + it * 32 + lane;
-      const uint32_t d = idx < n ? (uint32_t)((key[it] >> shift) & 0xff) : (uint32_t)kRadix;
-      const uint32_t peers = __match_any_sync(0xffffffffu, d);
-      const uint32_t before = wh[d];
-      __syncwarp();
-      if ((peers & lt) == 0) wh[d] = before + __popc(peers);
-      __syncwarp();
-      pos[it] = before + __popc(peers & lt);
-    }
-    // (5) scatter into shared memory in sorted order (frees the registers)
-#pragma unroll
-    for (int it = 0; it < kSortItems; ++it) {
-      const int64_t idx = first + it * 32 + lane;
-      if (idx < n) {
-        s_keys[pos[it]] = key[it];
-        s_vals[pos[it]] = val[it];
-      }
-    }
-    // (6) look-back: global start of each digit's run from this partition
-    uint64_t excl = 0;
-    if (p > 0) {
-      excl = windowed_lookback<32>(lookback + b, kRadix, p, status);
-      st_relaxed_u64(lb, kLbPrefix | (excl + count));
-    }
-    s_gbase[b] = s_gexcl[b] + excl;
-    __syncthreads();
-    // (7) write runs of equal digits out
-    const int64_t remain = n - p * kSortTile;
-    const int valid_count = remain < kSortTile ? (int)remain : kSortTile;
-    for (int j = tid; j < valid_count; j += kSortThreads) {
-      const K k = s_keys[j];
-      const uint32_t d = (uint32_t)((k >> shift) & 0xff);
-      const uint64_t gpos = s_gbase[d] + (uint64_t)(j - (int)s_lstart[d]);
-      if (gpos < (uint64_t)n) {
-        keys_out[gpos] = k;
-        vals_out[gpos] = s_vals[j];
-      } else {
-        atomicOr(status, kStatusBounds);
-      }
-    }
-    __syncthreads();
   }
 }
 
@@ -619,55 +633,49 @@ __global__ void k_ranges(const K* __restrict__ keys, const int64_t* __restrict__
   }
 }
 
-size_t sort_smem_bytes(int key_bytes) {
-  return (size_t)kRadix * 8 * 2 + (size_t)kSortTile * key_bytes + (size_t)kSortTile * 4 +
+size_t scatter_smem_bytes(int key_bytes) {
+  return (size_t)kRadix * 8 + (size_t)kSortTile * key_bytes + (size_t)kSortTile * 4 +
          (size_t)kSortWarps * (kRadix + 1) * 4 + (size_t)kRadix * 4 + 16 * 4;
 }
 
+// `passes` radix passes starting at digit `first_digit`, ping-ponging between
+// (keys_a, vals_a) and (keys_b, vals_b); grid sized for `max_items`.
 template <typename K>
-cudaError_t run_onesweep_passes(K* keys_a, uint32_t* vals_a, K* keys_b, uint32_t* vals_b,
-                                const int64_t* n_ptr, int64_t capacity, int first_digit,
-                                int passes, const unsigned long long* hist,
-                                uint64_t* lookback, int64_t region_words, uint32_t* counters,
-                                uint32_t* status, int grid, cudaStream_t stream) {
-  const size_t smem = sort_smem_bytes(sizeof(K));
-  cudaError_t e = cudaFuncSetAttribute(k_onesweep<K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+cudaError_t run_radix_passes(K* keys_a, uint32_t* vals_a, K* keys_b, uint32_t* vals_b,
+                             const int64_t* n_ptr, int64_t capacity, int64_t max_items,
+                             int first_digit, int passes, const unsigned long long* hist,
+                             uint64_t* counts, int64_t stride, uint32_t* status,
+                             cudaStream_t stream) {
+  const size_t smem = scatter_smem_bytes(sizeof(K));
+  cudaError_t e = cudaFuncSetAttribute(k_radix_scatter<K>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  const int64_t parts = (max_items + kSortTile - 1) / kSortTile;
+  if (parts == 0) return cudaSuccess;
   K* kin = keys_a;
   uint32_t* vin = vals_a;
   K* kout = keys_b;
   uint32_t* vout = vals_b;
   for (int p = 0; p < passes; ++p) {
     const int d = first_digit + p;
-    k_onesweep<K><<<grid, kSortThreads, smem, stream>>>(
-        kin, vin, kout, vout, n_ptr, capacity, 8 * d, hist + (size_t)d * kRadix,
-        lookback + (size_t)p * region_words, counters + p, status);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    k_radix_count<K><<<(unsigned)parts, kSortThreads, 0, stream>>>(kin, n_ptr, capacity, 8 * d,
+                                                                   counts, stride);
+    k_radix_scan<<<kRadix, 256, 0, stream>>>(counts, stride, n_ptr, capacity,
+                                             hist + (size_t)d * kRadix);
+    k_radix_scatter<K><<<(unsigned)parts, kSortThreads, smem, stream>>>(
+        kin, vin, kout, vout, n_ptr, capacity, 8 * d, counts, stride, status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     K* tk = kin; kin = kout; kout = tk;
     uint32_t* tv = vin; vin = vout; vout = tv;
   }
   return cudaSuccess;
 }
 
-int sort_grid(int key_bytes, int64_t max_items) {
-  int dev = 0, sms = 148, per_sm = 2;
+int num_sms() {
+  int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const size_t smem = sort_smem_bytes(key_bytes);
-  if (key_bytes == 8) {
-    cudaFuncSetAttribute(k_onesweep<uint64_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_onesweep<uint64_t>, kSortThreads, smem);
-  } else {
-    cudaFuncSetAttribute(k_onesweep<uint32_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_onesweep<uint32_t>, kSortThreads, smem);
-  }
-  if (per_sm < 1) per_sm = 1;
-  const int64_t parts = (max_items + kSortTile - 1) / kSortTile;
-  int64_t grid = (int64_t)sms * per_sm;
-  if (parts < grid) grid = parts;
-  return grid < 1 ? 1 : (int)grid;
+  return sms;
 }
 
 }  // namespace
@@ -678,74 +686,57 @@ int64_t emit_blocks(int64_t items) { return (items + kEmitItems - 1) / kEmitItem
 cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
   cudaError_t e;
   const int64_t n_items = (int64_t)a.n * a.n_views;
-  const auto rec4 = reinterpret_cast<const float4*>(a.bins);
+  const auto bins4 = reinterpret_cast<const float4*>(a.bins);
   if (n_items == 0) {
     return cudaMemsetAsync(a.n_pairs, 0, sizeof(int64_t), stream);
   }
-  const int64_t lb_region = a.lookback_region_words;
+  const int sms = num_sms();
+  const int64_t eb = emit_blocks(n_items);
   if (a.mode == GS_SORT_PRESORT) {
     // 1) keys (view << 32 | depth) over all Gaussians of all views
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     int64_t blocks = (n_items + 255) / 256;
     if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
-    k_depth_keys<<<(int)blocks, 256, 0, stream>>>(rec4, a.n, a.n_views, a.presort_passes,
-                                                 a.pkeys[0], a.pvals[0], a.presort_hist,
-                                                 a.n_items_dev);
+    k_depth_keys<<<(int)blocks, 256, 0, stream>>>(bins4, a.n, a.n_views, a.presort_passes,
+                                                  a.pkeys[0], a.pvals[0], a.presort_hist,
+                                                  a.n_items_dev);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // the presort look-back regions are sized for n_items (host-known)
-    e = cudaMemsetAsync(a.lookback, 0,
-                        (size_t)a.presort_passes * lb_region * sizeof(uint64_t), stream);
-    if (e != cudaSuccess) return e;
-    e = run_onesweep_passes<uint64_t>(a.pkeys[0], a.pvals[0], a.pkeys[1], a.pvals[1],
-                                      a.n_items_dev, n_items, 0, a.presort_passes,
-                                      a.presort_hist, a.lookback, lb_region, a.counters + 8,
-                                      a.status, sort_grid(8, n_items), stream);
+    e = run_radix_passes<uint64_t>(a.pkeys[0], a.pvals[0], a.pkeys[1], a.pvals[1], a.n_items_dev,
+                                   n_items, n_items, 0, a.presort_passes, a.presort_hist,
+                                   a.counts, a.counts_stride, a.status, stream);
     if (e != cudaSuccess) return e;
     const int fin = a.presort_passes & 1;
     // 2) emission in depth order, 32-bit tile keys
-    const int64_t eb = emit_blocks(n_items);
     k_emit<1, uint32_t><<<(unsigned)eb, kEmitThreads, 0, stream>>>(
-        rec4, a.pkeys[fin], a.pvals[fin], a.n, a.n_views, a.grid, a.pair_passes,
+        bins4, a.pkeys[fin], a.pvals[fin], a.n, a.n_views, a.grid, a.pair_passes,
         reinterpret_cast<uint32_t*>(a.keys[a.emit_buf]), a.vals[a.emit_buf], a.capacity,
         a.n_pairs, a.hist, a.emit_lookback, a.counters + 0, a.status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_clear_lookback<<<sms * 4, 256, 0, stream>>>(a.lookback, a.n_pairs, a.capacity,
-                                                  a.pair_passes, lb_region);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    e = run_onesweep_passes<uint32_t>(
+    e = run_radix_passes<uint32_t>(
         reinterpret_cast<uint32_t*>(a.keys[a.emit_buf]), a.vals[a.emit_buf],
         reinterpret_cast<uint32_t*>(a.keys[a.emit_buf ^ 1]), a.vals[a.emit_buf ^ 1], a.n_pairs,
-        a.capacity, 0, a.pair_passes, a.hist, a.lookback, lb_region, a.counters + 1, a.status,
-        sort_grid(4, a.capacity), stream);
+        a.capacity, a.capacity, 0, a.pair_passes, a.hist, a.counts, a.counts_stride, a.status,
+        stream);
     if (e != cudaSuccess) return e;
     const int out = a.emit_buf ^ (a.pair_passes & 1);
     k_ranges<uint32_t><<<sms * 4, 256, 0, stream>>>(reinterpret_cast<uint32_t*>(a.keys[out]),
-                                                   a.n_pairs, a.capacity, a.n_tiles, a.ranges, a.status);
+                                                   a.n_pairs, a.capacity, a.n_tiles, a.ranges,
+                                                   a.status);
     return cudaGetLastError();
   }
   // full 64-bit keys
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t eb = emit_blocks(n_items);
   k_emit<0, uint64_t><<<(unsigned)eb, kEmitThreads, 0, stream>>>(
-      rec4, nullptr, nullptr, a.n, a.n_views, a.grid, a.pair_passes, a.keys[a.emit_buf],
+      bins4, nullptr, nullptr, a.n, a.n_views, a.grid, a.pair_passes, a.keys[a.emit_buf],
       a.vals[a.emit_buf], a.capacity, a.n_pairs, a.hist, a.emit_lookback, a.counters + 0,
       a.status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  k_clear_lookback<<<sms * 4, 256, 0, stream>>>(a.lookback, a.n_pairs, a.capacity, a.pair_passes,
-                                                lb_region);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  e = run_onesweep_passes<uint64_t>(a.keys[a.emit_buf], a.vals[a.emit_buf], a.keys[a.emit_buf ^ 1],
-                                    a.vals[a.emit_buf ^ 1], a.n_pairs, a.capacity, 0,
-                                    a.pair_passes, a.hist, a.lookback, lb_region, a.counters + 1,
-                                    a.status, sort_grid(8, a.capacity), stream);
+  e = run_radix_passes<uint64_t>(a.keys[a.emit_buf], a.vals[a.emit_buf], a.keys[a.emit_buf ^ 1],
+                                 a.vals[a.emit_buf ^ 1], a.n_pairs, a.capacity, a.capacity, 0,
+                                 a.pair_passes, a.hist, a.counts, a.counts_stride, a.status,
+                                 stream);
   if (e != cudaSuccess) return e;
   const int out = a.emit_buf ^ (a.pair_passes & 1);
   k_ranges<uint64_t><<<sms * 4, 256, 0, stream>>>(a.keys[out], a.n_pairs, a.capacity, a.n_tiles,
-                                                 a.ranges, a.status);
+                                                  a.ranges, a.status);
   return cudaGetLastError();
 }
 

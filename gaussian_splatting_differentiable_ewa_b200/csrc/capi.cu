@@ -35,8 +35,8 @@ struct Layout {
   int pair_passes = 0;
   int presort_passes = 0;
   int key_bytes = 8;
-  int64_t region_words = 0;
-  size_t off_hist = 0, off_phist = 0, off_emit_lb = 0, off_lb = 0, off_keys0 = 0, off_keys1 = 0,
+  int64_t counts_stride = 0;
+  size_t off_hist = 0, off_phist = 0, off_emit_lb = 0, off_counts = 0, off_keys0 = 0, off_keys1 = 0,
          off_vals1 = 0, off_pkeys0 = 0, off_pkeys1 = 0, off_pvals0 = 0, off_pvals1 = 0;
   size_t total = 0;
 };
@@ -71,18 +71,17 @@ bool make_layout(int64_t n, int32_t n_views, const gs_camera* cams, int64_t capa
     L.pair_passes = (tile_bits + 7) / 8;
     L.presort_passes = 4 + (n_views > 1 ? 1 : 0);
   }
-  const int regions = L.pair_passes > L.presort_passes ? L.pair_passes : L.presort_passes;
   int64_t parts = sort_partitions(capacity);
   if (mode == GS_SORT_PRESORT) {
     const int64_t p2 = sort_partitions(items);
     if (p2 > parts) parts = p2;
   }
-  L.region_words = parts * 256;
+  L.counts_stride = parts > 0 ? parts : 1;
   size_t off = kControlBytes;
   L.off_hist = off; off = align_up(off + kHistBytes);
   L.off_phist = off; off = align_up(off + kHistBytes);
   L.off_emit_lb = off; off = align_up(off + (size_t)emit_blocks(items) * 8);
-  L.off_lb = off; off = align_up(off + (size_t)(regions > 0 ? regions : 1) * L.region_words * 8);
+  L.off_counts = off; off = align_up(off + (size_t)256 * L.counts_stride * 8);
   L.off_keys0 = off; off = align_up(off + (size_t)capacity * L.key_bytes);
   L.off_keys1 = off; off = align_up(off + (size_t)capacity * L.key_bytes);
   L.off_vals1 = off; off = align_up(off + (size_t)capacity * 4);
@@ -196,8 +195,8 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
   }
   a.hist = reinterpret_cast<unsigned long long*>(w + L.off_hist);
   a.presort_hist = reinterpret_cast<unsigned long long*>(w + L.off_phist);
-  a.lookback = reinterpret_cast<uint64_t*>(w + L.off_lb);
-  a.lookback_region_words = L.region_words;
+  a.counts = reinterpret_cast<uint64_t*>(w + L.off_counts);
+  a.counts_stride = L.counts_stride;
   a.emit_lookback = reinterpret_cast<uint64_t*>(w + L.off_emit_lb);
   a.counters = reinterpret_cast<uint32_t*>(w + kCountersOffset);
   a.status = reinterpret_cast<uint32_t*>(w + kStatusOffset);

@@ -25,8 +25,8 @@ struct BinSortArgs {
   uint32_t* pvals[2];  // presort values
   unsigned long long* hist;          // [8][256] pair-key digit histograms
   unsigned long long* presort_hist;  // [8][256]
-  uint64_t* lookback;                // [passes][region_words]
-  int64_t lookback_region_words;
+  uint64_t* counts;                  // [256][counts_stride] radix digit counts / offsets
+  int64_t counts_stride;             // partitions of the largest pass
   uint64_t* emit_lookback;           // [emit blocks]
   uint32_t* counters;                // [16] dynamic block counters
   uint32_t* status;

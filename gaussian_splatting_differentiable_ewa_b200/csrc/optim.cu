@@ -81,17 +81,18 @@ __global__ void __launch_bounds__(kAdamThreads) k_adam(AdamTable t, float b1, fl
   for (int k = 0; k < kAdamVecPerThread; ++k) {
     const int64_t e = base + ((int64_t)k * kAdamThreads + threadIdx.x) * 4;
     if (e + 4 <= count) {
-      float4 p = *reinterpret_cast<float4*>(P + e);
-      const float4 g = __ldg(reinterpret_cast<const float4*>(G + e));
-      float4 m = *reinterpret_cast<float4*>(M + e);
-      float4 v = *reinterpret_cast<float4*>(V + e);
+      // every float is read and written once per step: stream past L2
+      float4 p = __ldcs(reinterpret_cast<const float4*>(P + e));
+      const float4 g = __ldcs(reinterpret_cast<const float4*>(G + e));
+      float4 m = __ldcs(reinterpret_cast<const float4*>(M + e));
+      float4 v = __ldcs(reinterpret_cast<const float4*>(V + e));
       adam_one(p.x, g.x, m.x, v.x, lr, b1, b2, eps, bc1, bc2);
       adam_one(p.y, g.y, m.y, v.y, lr, b1, b2, eps, bc1, bc2);
       adam_one(p.z, g.z, m.z, v.z, lr, b1, b2, eps, bc1, bc2);
       adam_one(p.w, g.w, m.w, v.w, lr, b1, b2, eps, bc1, bc2);
-      *reinterpret_cast<float4*>(P + e) = p;
-      *reinterpret_cast<float4*>(M + e) = m;
-      *reinterpret_cast<float4*>(V + e) = v;
+      __stcs(reinterpret_cast<float4*>(P + e), p);
+      __stcs(reinterpret_cast<float4*>(M + e), m);
+      __stcs(reinterpret_cast<float4*>(V + e), v);
     } else {
       for (int64_t f = e; f < count && f < e + 4; ++f) {
         float p = P[f], m = M[f], v = V[f];

@@ -109,12 +109,42 @@ __device__ __forceinline__ long long floor_tile(double a) {
   return static_cast<long long>(floor(a * (1.0 / kTile)));
 }
 
-// Colour from the SH coefficients of one Gaussian at unit direction (x, y, z):
-// rgb_c = max(0, sum_k Y_k sh_kc + 0.5). Coefficients are read with 16-byte
-// loads when the per-Gaussian block is a multiple of 16 bytes.
+constexpr int kProjThreads = 128;     // projection backward block
+constexpr int kProjFwdThreads = 256;  // projection forward block
+constexpr int kShStride = kProjThreads + 1;  // padded row: conflict-free banks
+
+// Stage the SH coefficients of Gaussians [i0, i0 + cnt) in shared memory,
+// coefficient-major with a padded row (s[c * kShStride + local i]), using
+// coalesced loads of the contiguous global block.
+template <int K3>
+__device__ __forceinline__ void stage_sh(const float* __restrict__ sh, int64_t i0, int cnt,
+                                         float* __restrict__ s) {
+  const float* src = sh + i0 * K3;
+  const int total = cnt * K3;
+  for (int e = threadIdx.x; e < total; e += kProjThreads) {
+    const int i = e / K3, c = e - i * K3;
+    s[c * kShStride + i] = __ldg(&src[e]);
+  }
+}
+
+// Write staged values back to the contiguous global block (coalesced).
+template <int K3>
+__device__ __forceinline__ void unstage_sh(float* __restrict__ dst, int64_t i0, int cnt,
+                                           const float* __restrict__ s) {
+  float* d = dst + i0 * K3;
+  const int total = cnt * K3;
+  for (int e = threadIdx.x; e < total; e += kProjThreads) {
+    const int i = e / K3, c = e - i * K3;
+    d[e] = s[c * kShStride + i];
+  }
+}
+
+// Colour from the SH coefficients of one Gaussian read straight from global
+// memory (16-byte loads when the per-Gaussian block allows) at unit direction
+// (x, y, z): rgb_c = max(0, sum_k Y_k sh_kc + 0.5).
 template <int DEG>
-__device__ __forceinline__ void sh_colour(const float* __restrict__ shi, float x, float y, float z,
-                                          float rgb[3]) {
+__device__ __forceinline__ void sh_colour_global(const float* __restrict__ shi, float x, float y,
+                                                 float z, float rgb[3]) {
   constexpr int K = (DEG + 1) * (DEG + 1);
   float Y[16];
   sh_basis<DEG>(x, y, z, Y);
@@ -140,16 +170,17 @@ __device__ __forceinline__ void sh_colour(const float* __restrict__ shi, float x
 }
 
 template <int DEG>
-__global__ void __launch_bounds__(256) k_project(const float4* __restrict__ means,
-                                                 const float4* __restrict__ log_scales,
-                                                 const float4* __restrict__ quats,
-                                                 const float* __restrict__ logit,
-                                                 const float* __restrict__ sh, int n, int n_views,
-                                                 CamSet cams, float4* __restrict__ records,
-                                                 float4* __restrict__ bins,
-                                                 int* __restrict__ radii) {
+__global__ void __launch_bounds__(kProjFwdThreads) k_project(const float4* __restrict__ means,
+                                                          const float4* __restrict__ log_scales,
+                                                          const float4* __restrict__ quats,
+                                                          const float* __restrict__ logit,
+                                                          const float* __restrict__ sh, int n,
+                                                          int n_views, CamSet cams,
+                                                          float4* __restrict__ records,
+                                                          float4* __restrict__ bins,
+                                                          int* __restrict__ radii) {
   constexpr int K = (DEG + 1) * (DEG + 1);
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const int i = blockIdx.x * kProjFwdThreads + threadIdx.x;
   if (i >= n) return;
   const float4 m = __ldg(&means[i]);
   const float4 ls = __ldg(&log_scales[i]);
@@ -256,7 +287,7 @@ __global__ void __launch_bounds__(256) k_project(const float4* __restrict__ mean
           float dxv = m.x - c.campos[0], dyv = m.y - c.campos[1], dzv = m.z - c.campos[2];
           float inv = rsqrtf(dxv * dxv + dyv * dyv + dzv * dzv);
           float rgb[3];
-          sh_colour<DEG>(shi, dxv * inv, dyv * inv, dzv * inv, rgb);
+          sh_colour_global<DEG>(shi, dxv * inv, dyv * inv, dzv * inv, rgb);
           rec[R_R] = rgb[0];
           rec[R_G] = rgb[1];
           rec[R_B] = rgb[2];
@@ -284,8 +315,11 @@ __global__ void __launch_bounds__(256) k_project(const float4* __restrict__ mean
 
 // Backward of k_project for the raw parameters, summing every view in which
 // the Gaussian was visible (radius > 0).
+// SH coefficients come in, and SH gradients go out, through shared memory
+// (coefficient-major, coalesced global traffic); the SH gradients are summed
+// over views in shared memory rather than in registers.
 template <int DEG>
-__global__ void __launch_bounds__(128) k_project_bwd(
+__global__ void __launch_bounds__(kProjThreads) k_project_bwd(
     const float4* __restrict__ means, const float4* __restrict__ log_scales,
     const float4* __restrict__ quats, const float* __restrict__ logit,
     const float* __restrict__ sh, const float4* __restrict__ grad2d,
@@ -293,8 +327,18 @@ __global__ void __launch_bounds__(128) k_project_bwd(
     float4* __restrict__ g_log_scales, float4* __restrict__ g_quats, float* __restrict__ g_logit,
     float* __restrict__ g_sh) {
   constexpr int K = (DEG + 1) * (DEG + 1);
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n) return;
+  constexpr int K3 = K * 3;
+  extern __shared__ float s_pb[];
+  float* s_coef = s_pb;                    // [K3][kShStride]
+  float* s_dsh = s_pb + K3 * kShStride;    // [K3][kShStride]
+  const int64_t i0 = (int64_t)blockIdx.x * kProjThreads;
+  const int cnt = (int)min((int64_t)kProjThreads, (int64_t)n - i0);
+  stage_sh<K3>(sh, i0, cnt, s_coef);
+#pragma unroll
+  for (int c = 0; c < K3; ++c) s_dsh[c * kShStride + threadIdx.x] = 0.f;
+  __syncthreads();
+  const int i = (int)i0 + threadIdx.x;
+  if (i < n) {
   const float4 m = __ldg(&means[i]);
   const float4 ls = __ldg(&log_scales[i]);
   const float4 q = __ldg(&quats[i]);
@@ -316,10 +360,8 @@ __global__ void __launch_bounds__(128) k_project_bwd(
   float dM[3][3] = {{0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}};
   float dmu[3] = {0.f, 0.f, 0.f};
   float dopac = 0.f;
-  float dsh[K * 3];
-#pragma unroll
-  for (int k = 0; k < K * 3; ++k) dsh[k] = 0.f;
-  const float* shi = sh + (size_t)i * K * 3;
+  const float* cf_t = s_coef + threadIdx.x;
+  float* dsh_t = s_dsh + threadIdx.x;
 
   for (int v = 0; v < n_views; ++v) {
     if (radii[(size_t)v * n + i] <= 0) continue;
@@ -403,13 +445,13 @@ __global__ void __launch_bounds__(128) k_project_bwd(
     for (int ch = 0; ch < 3; ++ch) {
       float raw = 0.5f;
 #pragma unroll
-      for (int k = 0; k < K; ++k) raw = fmaf(Y[k], __ldg(&shi[k * 3 + ch]), raw);
+      for (int k = 0; k < K; ++k) raw = fmaf(Y[k], cf_t[(k * 3 + ch) * kShStride], raw);
       if (!(raw > 0.f)) continue;
       const float gcol = G[G_R + ch];
 #pragma unroll
       for (int k = 0; k < K; ++k) {
-        const float cf = __ldg(&shi[k * 3 + ch]);
-        dsh[k * 3 + ch] += Y[k] * gcol;
+        const float cf = cf_t[(k * 3 + ch) * kShStride];
+        dsh_t[(k * 3 + ch) * kShStride] += Y[k] * gcol;
         gdx += gcol * cf * gx[k];
         gdy += gcol * cf * gy[k];
         gdz += gcol * cf * gz[k];
@@ -455,9 +497,9 @@ __global__ void __launch_bounds__(128) k_project_bwd(
   g_log_scales[i] = make_float4(dls[0], dls[1], dls[2], 0.f);
   g_quats[i] = make_float4(dqw, dqx, dqy, dqz);
   g_logit[i] = dopac * opac * (1.f - opac);
-  float* gsh = g_sh + (size_t)i * K * 3;
-#pragma unroll
-  for (int k = 0; k < K * 3; ++k) gsh[k] = dsh[k];
+  }
+  __syncthreads();
+  unstage_sh<K3>(g_sh, i0, cnt, s_dsh);
 }
 
 }  // namespace
@@ -466,7 +508,7 @@ cudaError_t launch_project(const gs_params& p, const CamSet& cams, int n_views, 
                            float* bins, int* radii, cudaStream_t stream) {
   const int n = (int)p.n;
   if (n == 0) return cudaSuccess;
-  const int threads = 256;
+  const int threads = kProjFwdThreads;
   const int blocks = (n + threads - 1) / threads;
   auto m = reinterpret_cast<const float4*>(p.means);
   auto s = reinterpret_cast<const float4*>(p.log_scales);
@@ -489,8 +531,10 @@ cudaError_t launch_project_bwd(const gs_params& p, const CamSet& cams, int n_vie
                                cudaStream_t stream) {
   const int n = (int)p.n;
   if (n == 0) return cudaSuccess;
-  const int threads = 128;
+  const int threads = kProjThreads;
   const int blocks = (n + threads - 1) / threads;
+  const int K3 = 3 * (p.sh_degree + 1) * (p.sh_degree + 1);
+  const size_t smem = (size_t)2 * K3 * kShStride * sizeof(float);
   auto m = reinterpret_cast<const float4*>(p.means);
   auto s = reinterpret_cast<const float4*>(p.log_scales);
   auto q = reinterpret_cast<const float4*>(p.quats);
@@ -498,7 +542,10 @@ cudaError_t launch_project_bwd(const gs_params& p, const CamSet& cams, int n_vie
   auto gm = reinterpret_cast<float4*>(g.means);
   auto gs = reinterpret_cast<float4*>(g.log_scales);
   auto gq = reinterpret_cast<float4*>(g.quats);
-#define GS_PBWD(D) k_project_bwd<D><<<blocks, threads, 0, stream>>>(m, s, q, p.opacity_logit, p.sh, g2, radii, n, n_views, cams, gm, gs, gq, g.opacity_logit, g.sh)
+#define GS_PBWD(D)                                                                            \
+  cudaFuncSetAttribute(k_project_bwd<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+  k_project_bwd<D><<<blocks, threads, smem, stream>>>(m, s, q, p.opacity_logit, p.sh, g2, radii, n, \
+                                                      n_views, cams, gm, gs, gq, g.opacity_logit, g.sh)
   switch (p.sh_degree) {
     case 0: GS_PBWD(0); break;
     case 1: GS_PBWD(1); break;
