@@ -117,34 +117,35 @@ class ClockSampler:
                     samples=len(sm))
 
 
-def orbit_camera(scene, k: int, count: int):
-    from gaussian_splatting_differentiable_ewa_b200 import scenes as S
-    c0 = scene.cameras[0]
-    a = 2.0 * math.pi * k / count
-    centre = (8.0 * math.sin(a), 0.0, -8.0 * math.cos(a))
-    return S.Camera(viewmat=S.look_at(centre).astype(np.float32), fx=c0.fx, fy=c0.fy, cx=c0.cx,
-                    cy=c0.cy, width=c0.width, height=c0.height,
-                    campos=np.asarray(centre, np.float32))
-
-
 # ----------------------------------------------------------------- work model
+
+def sort_passes(sp, sort_mode: str):
+    """(presort passes, pair passes) of gs_bin_sort for this workload."""
+    tiles = sp.V * ((sp.W + 15) // 16) * ((sp.H + 15) // 16)
+    tile_bits = max(int(tiles - 1).bit_length(), 0)
+    if sort_mode == "full64":
+        return 0, (32 + tile_bits + 7) // 8
+    return 4 + (1 if sp.V > 1 else 0), (tile_bits + 7) // 8
+
 
 def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float) -> dict:
     """Algorithmic bytes (and exp evaluations) per launch of each call.
 
     Bytes count the data the definition has to move once: parameters read,
-    outputs written, 59 real floats per Gaussian (pad lanes excluded)."""
+    outputs written, 59 real floats per Gaussian (pad lanes excluded); a radix
+    pass reads and writes every key and value once; the blend kernels read
+    every list entry's id and record once."""
     n, V = sp.n, sp.V
     P = V * sp.W * sp.H
     rec = 48
     p59 = 59 * 4
+    pre, pair = sort_passes(sp, sort_mode)
     if sort_mode == "full64":
-        passes = 6 if V * ((sp.W + 15) // 16) * ((sp.H + 15) // 16) > 256 else 5
-        sort_bytes = n_pairs * (12 + passes * 24 + 8) + V * n * 16
+        sort_bytes = n_pairs * (12 + pair * 24 + 8) + V * n * 16
     else:
-        sort_bytes = n_pairs * (8 + 2 * 16 + 4) + V * n * (16 + 4 * 24 + 12)
+        sort_bytes = n_pairs * (8 + pair * 16 + 4) + V * n * (16 + pre * 24 + 12)
     return {
-        "gs_project": dict(bytes=V * n * (p59 + rec + 4), exps=0.0),
+        "gs_project": dict(bytes=V * n * (p59 + rec + 16 + 4), exps=0.0),
         "gs_bin_sort": dict(bytes=sort_bytes, exps=0.0),
         "gs_rasterize_fwd": dict(bytes=n_pairs * (4 + rec) + P * 20, exps=exps),
         "gs_rasterize_bwd": dict(bytes=n_pairs * (4 + rec) + P * 20 + V * n * 48 * 2, exps=exps),
@@ -152,6 +153,46 @@ def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float) -> dict:
         "gs_densify_stats": dict(bytes=V * n * (12 + 4) + n * 24, exps=0.0),
         "gs_adam_step": dict(bytes=n * 59 * 28, exps=0.0),
     }
+
+
+def launches_per_step(sp, sort_mode: str) -> int:
+    """Library kernels launched by one step (memsets excluded)."""
+    pre, pair = sort_passes(sp, sort_mode)
+    sort = (1 + 3 * pre if sort_mode == "presort" else 0) + 1 + 3 * pair + 1
+    return 1 + sort + 1 + 1 + 1 + 1 + 1
+
+
+# C call -> (kernel, source file) for the ncu traffic lookup
+KERNEL_OF = {
+    "gs_project": ("k_project", "project.cu"),
+    "gs_rasterize_fwd": ("k_raster_fwd", "raster.cu"),
+    "gs_rasterize_bwd": ("k_raster_bwd", "raster.cu"),
+    "gs_project_bwd": ("k_project_bwd", "project.cu"),
+    "gs_adam_step": ("k_adam", "optim.cu"),
+}
+
+
+def profiled_traffic(call: str, workload: str):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+    the committed ncu summary of this kernel and workload, or None when there
+    is none or the kernel's source changed since it was captured."""
+    import hashlib
+    import re
+    if call not in KERNEL_OF:
+        return None
+    kernel, src = KERNEL_OF[call]
+    prof = os.path.join(ROOT, "profiles", "%s_%s.md" % (kernel, workload))
+    srcp = os.path.join(ROOT, "gaussian_splatting_differentiable_ewa_b200", "csrc", src)
+    try:
+        text = open(prof).read()
+        sha = hashlib.sha256(open(srcp, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    m_sha = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
+    m_t = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
+    if not m_sha or not m_t or m_sha.group(1) != sha:
+        return None
+    return int(m_t.group(1))
 
 
 def sfu_peak_gexps(sm_mhz: float, sms: int = 148) -> float:
@@ -278,9 +319,10 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
     mode = api.GS_SORT_PRESORT if args.sort_mode == "presort" else api.GS_SORT_FULL64
 
+    from gaussian_splatting_differentiable_ewa_b200 import dist as gdist
     scene = S.make_scene(WORKLOAD, n=args.n)
     if world > 1:
-        scene.cameras = [orbit_camera(scene, rank, world)]
+        scene.cameras = [gdist.orbit_view(scene, rank, world)]
     c = scene.cameras[0]
     sp = Splatter(scene, sort_mode=mode)
     need = sp.ensure_capacity()
@@ -304,8 +346,7 @@ def run_ours(args):
         mark(4)
         sp.project_bwd()
         mark(5)
-        if world > 1:
-            dist.all_reduce(sp.grad_flat)
+        gdist.allreduce_grads(sp.grad_flat)
         mark(6)
         sp.densify_stats()
         mark(7)
@@ -336,13 +377,9 @@ def run_ours(args):
     clk = clocks.stop()
     if world > 1:
         dist.barrier()
-    elapsed_ms = start.elapsed_time(end)
+    elapsed_ms = gdist.max_over_ranks(start.elapsed_time(end), device="cuda")
     per_call = {nm: float(np.mean([ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(args.steps)]))
                 for i, nm in enumerate(names)}
-    if world > 1:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
     ms = elapsed_ms / args.steps
     value = world * pixels / (ms / 1000.0) / 1e6
     n_pairs = int(sp.n_pairs.item())
@@ -366,11 +403,7 @@ def run_ours(args):
             h_out.copy_(sp.image, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1) / args.steps
-        if world > 1:
-            t = torch.tensor([e_ms], dtype=torch.float64, device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = gdist.max_over_ranks(e0.elapsed_time(e1) / args.steps, device="cuda")
         e2e = {"value": world * pixels / (e_ms / 1000.0) / 1e6, "unit": "Mpix/s",
                "ms_per_step": e_ms, "h2d_bytes_per_step": int(h_in.numel() * 4),
                "d2h_bytes_per_step": int(h_out.numel() * 4)}
@@ -401,24 +434,26 @@ def run_ours(args):
             kernels[nm]["gexps"] = w["exps"] / t / 1e9
     dom = max(kernels, key=lambda k: kernels[k]["ms"])
     sm_for_peak = pk["sm_max_mhz"]
-    if work[dom]["exps"] and exps:
+    t_hbm = work[dom]["bytes"] / (pk["hbm_gbs"] * 1e9)
+    t_sfu = (work[dom]["exps"] / (sfu_peak_gexps(sm_for_peak) * 1e9)) if exps else 0.0
+    if t_sfu > t_hbm:
         peak = sfu_peak_gexps(sm_for_peak)
         ach = work[dom]["exps"] / (per_call[dom] / 1000.0) / 1e9
         roof = {"kernel": dom, "bound": "alu", "achieved": ach, "peak": peak, "unit": "Gexp/s",
-                "frac": ach / peak, "traffic": None,
+                "frac": ach / peak, "traffic": profiled_traffic(dom, WORKLOAD),
                 "peak_source": "148 SM x 16 MUFU.EX2/clk x %.0f MHz (max SM clock)" % sm_for_peak}
     else:
         ach = work[dom]["bytes"] / (per_call[dom] / 1000.0) / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"],
-                "unit": "GB/s", "frac": ach / pk["hbm_gbs"], "traffic": None,
-                "peak_source": pk["source"]}
+                "unit": "GB/s", "frac": ach / pk["hbm_gbs"],
+                "traffic": profiled_traffic(dom, WORKLOAD),
+                "peak_source": pk["source"] + " (MEASURED_PEAKS.json copy bandwidth)"}
     # step roofline: sum over calls of max(bytes / HBM, exps / SFU)
     bound_s = 0.0
     for nm, w in work.items():
         bound_s += max(w["bytes"] / (pk["hbm_gbs"] * 1e9),
                        (w["exps"] / (sfu_peak_gexps(sm_for_peak) * 1e9)) if w["exps"] else 0.0)
-    launches_per_step = {"presort": 1 + 10 + 1 + 1 + 1 + 1 + 1,
-                         "full64": 1 + 9 + 1 + 1 + 1 + 1 + 1}[args.sort_mode]
+    n_launch = launches_per_step(sp, args.sort_mode)
     line = {
         "metric": METRIC, "value": value, "unit": "Mpix/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
@@ -437,7 +472,7 @@ def run_ours(args):
         "cpu_baseline": None if cpu is None else {k: cpu[k] for k in
                                                   ("value", "unit", "cores", "kind", "sample")},
         "e2e": e2e,
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": n_launch * args.steps,
         "clocks": clk,
         "device_status": api.status_string(status),
     }
