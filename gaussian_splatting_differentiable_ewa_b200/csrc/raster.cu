@@ -1,11 +1,15 @@
 // raster.cu -- tile rasteriser, forward and backward, sm_100a.
 //
-// One 16x16 tile per 256-thread block, one thread per pixel ("Better Gaussian
-// Splatting in Julia", pwwt.cn sec. 5.4: a pixel block per thread group, each
-// group compositing serially, groups in parallel -- no atomics on pixels).
-// Each warp owns an 8x4 pixel block of the tile.
+// One 16x16 tile per 128-thread block ("Better Gaussian Splatting in Julia",
+// pwwt.cn sec. 5.4: a pixel block per thread group, each group compositing
+// serially, groups in parallel -- no atomics on pixels). Each warp owns an 8x8
+// pixel block of the tile and each thread two pixels of one column, four rows
+// apart: (x, y) and (x, y + 4). The pair shares its x offset from every
+// Gaussian centre, and its per-pixel arithmetic runs two-wide on the FP32x2
+// pipe (__ffma2_rn / __fadd2_rn / __fmul2_rn: each half rounds exactly like
+// the scalar operation, so pixel results do not depend on the pairing).
 //
-// The tile's depth-sorted list is consumed in batches of 256 records; each
+// The tile's depth-sorted list is consumed in batches of 128 records; each
 // thread stages one 48-byte record into shared memory with a TMA bulk copy
 // (cp.async.bulk completing on an mbarrier), double-buffered so the next batch
 // is in flight while the current one is blended. When a batch lands, thread j
@@ -17,17 +21,17 @@
 //
 // Forward (pwwt.cn sec. 3.3 `composite`, front to back; lshu.cn sec. 3.2
 // `blend`): alpha = min(0.99, o exp(-q/2)); skip alpha < 1/255; stop before a
-// Gaussian that would take T below 1e-4; a warp stops once all its lanes are
+// Gaussian that would take T below 1e-4; a warp stops once all its pixels are
 // done and a block once all its warps are (votes).
 //
 // Backward: each pixel replays its contributors back to front, recovering
-// T_k = T_{k+1} / (1 - alpha_k) and the colour behind,
+// T_k = T_{k+1} / (1 - alpha_k), with B_k the colour composited behind k,
 //   dC/dc_k = alpha_k T_k,
 //   dC/dalpha_k = T_k (c_k - B_k) - T_final bg / (1 - alpha_k),
-// B_k = alpha_{k+1} c_{k+1} + (1 - alpha_{k+1}) B_{k+1}. Per Gaussian the warp
-// sums its lanes' ten terms with a transposing butterfly (16 shuffles, each
-// lane ends with one total), the block sums its warps in shared memory, and
-// three 4-float vector atomics go to global memory.
+//   B_{k-1} = B_k + alpha_k (c_k - B_k).
+// Per Gaussian a thread adds its two pixels' ten terms, the warp sums its
+// lanes with a transposing butterfly (14 shuffles), the block sums its warps
+// in shared memory, and three 4-float vector atomics go to global memory.
 
 #include <cuda_runtime.h>
 
@@ -36,12 +40,15 @@
 namespace gsb {
 namespace {
 
-constexpr int kBatch = kTilePixels;              // records per batch
+constexpr int kThreads = 128;                    // 4 warps, 8x8 pixels each
+constexpr int kWarps = kThreads / 32;
+constexpr int kBatch = kThreads;                 // records per batch
 constexpr int kRecBytes = GS_RECORD_FLOATS * 4;  // 48
-constexpr int kWarps = kTilePixels / 32;         // 8 warps, 8x4 pixels each
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2AlphaMin = -7.994353436858858f;  // log2(1/255)
+
+static_assert(kTilePixels == 2 * kThreads, "two pixels per thread");
 
 // Evaluation-form record slots (after the per-batch rewrite in shared memory):
 // 0 u, 1 v, 2 A = -log2(e)/2 conic_a, 3 B = -log2(e) conic_b,
@@ -55,6 +62,8 @@ struct RasterGeom {
   int64_t capacity;  // length of ids
 };
 
+__device__ __forceinline__ float2 f2(float x) { return make_float2(x, x); }
+
 // A tile's [start, end) slice, clipped to the ids buffer (a malformed range
 // renders as empty instead of reading outside the buffer).
 __device__ __forceinline__ void tile_range(const int64_t* ranges, int tile, int64_t capacity,
@@ -64,8 +73,10 @@ __device__ __forceinline__ void tile_range(const int64_t* ranges, int tile, int6
   if (start < 0 || end > capacity || end < start) start = end = 0;
 }
 
+// The thread's pixel pair: (px, py) and (px, py + 4).
 struct TilePix {
   int view, x0, y0, px, py;
+  bool in0, in1;
 };
 
 __device__ __forceinline__ TilePix tile_pixel(const Grid& g, int tile) {
@@ -77,21 +88,27 @@ __device__ __forceinline__ TilePix tile_pixel(const Grid& g, int tile) {
   t.y0 = ty * kTile;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   t.px = t.x0 + 8 * (warp & 1) + (lane & 7);
-  t.py = t.y0 + 4 * (warp >> 1) + (lane >> 3);
+  t.py = t.y0 + 8 * (warp >> 1) + (lane >> 3);
+  t.in0 = t.px < g.width && t.py < g.height;
+  t.in1 = t.px < g.width && t.py + 4 < g.height;
   return t;
 }
 
-// log2 of the unclamped alpha at pixel centre (pxc, pyc): the one
-// expression both directions use, so their skip / stop decisions agree.
-__device__ __forceinline__ float eval_log2_alpha(const float* r, float pxc, float pyc, float& dx,
-                                                 float& dy) {
+// log2 of the unclamped alpha at the pair's pixel centres (pxc, pyc.x) and
+// (pxc, pyc.y); per pixel it is fma(A dx, dx, fma(B dx, dy, fma(C dy, dy, lo)))
+// with dx = pxc - u, dy = pyc - v. Both directions call this one function, so
+// their skip / stop decisions agree bit for bit.
+__device__ __forceinline__ float2 eval_log2_alpha(const float* r, float pxc, float2 pyc, float& dx,
+                                                  float2& dy) {
   dx = pxc - r[E_U];
-  dy = pyc - r[E_V];
-  return fmaf(r[E_A] * dx, dx, fmaf(r[E_B] * dx, dy, fmaf(r[E_C] * dy, dy, r[E_LO])));
+  dy = __fadd2_rn(pyc, f2(-r[E_V]));
+  float2 t = __ffma2_rn(__fmul2_rn(f2(r[E_C]), dy), dy, f2(r[E_LO]));
+  t = __ffma2_rn(f2(r[E_B] * dx), dy, t);
+  return __ffma2_rn(f2(r[E_A] * dx), f2(dx), t);
 }
 
 // Rewrite record j of a landed batch into evaluation form and return the
-// 8-bit mask of warps whose pixel block its alpha >= 1/255 box overlaps.
+// 4-bit mask of warps whose 8x8 pixel block its alpha >= 1/255 box overlaps.
 __device__ __forceinline__ uint32_t prepare_record(float* r, int x0, int y0) {
   const float u = r[R_U], v = r[R_V], hx = r[R_HX], hy = r[R_HY];
   const float o = r[R_OPAC];
@@ -102,17 +119,14 @@ __device__ __forceinline__ uint32_t prepare_record(float* r, int x0, int y0) {
   r[E_LO] = __log2f(o);
   r[E_IO] = 1.f / o;
   if (!(hx >= 0.f)) return 0u;
-  // pixel-centre extents of the warp blocks: x blocks of 8, y blocks of 4
+  // pixel-centre extents of the warp blocks: 8 wide, 8 high
   uint32_t xm = 0, ym = 0;
 #pragma unroll
-  for (int bx = 0; bx < 2; ++bx) {
-    const float lo = (float)(x0 + 8 * bx) + 0.5f, hi = lo + 7.f;
-    if (u + hx >= lo && u - hx <= hi) xm |= 1u << bx;
-  }
-#pragma unroll
-  for (int by = 0; by < 4; ++by) {
-    const float lo = (float)(y0 + 4 * by) + 0.5f, hi = lo + 3.f;
-    if (v + hy >= lo && v - hy <= hi) ym |= 1u << by;
+  for (int bi = 0; bi < 2; ++bi) {
+    const float xlo = (float)(x0 + 8 * bi) + 0.5f, xhi = xlo + 7.f;
+    if (u + hx >= xlo && u - hx <= xhi) xm |= 1u << bi;
+    const float ylo = (float)(y0 + 8 * bi) + 0.5f, yhi = ylo + 7.f;
+    if (v + hy >= ylo && v - hy <= yhi) ym |= 1u << bi;
   }
   uint32_t mask = 0;
 #pragma unroll
@@ -139,7 +153,7 @@ __device__ __forceinline__ int warp_list(const uint8_t* s_mask, uint8_t* list, i
   return cnt;
 }
 
-__global__ void __launch_bounds__(kTilePixels) k_raster_fwd(
+__global__ void __launch_bounds__(kThreads) k_raster_fwd(
     const float* __restrict__ records, const uint32_t* __restrict__ ids,
     const int64_t* __restrict__ ranges, RasterGeom geo, float bg0, float bg1, float bg2,
     float* __restrict__ image, float* __restrict__ final_T, uint32_t* __restrict__ n_contrib,
@@ -151,7 +165,6 @@ __global__ void __launch_bounds__(kTilePixels) k_raster_fwd(
 
   const int tile = blockIdx.x;
   const TilePix tp = tile_pixel(geo.g, tile);
-  const bool inside = tp.px < geo.g.width && tp.py < geo.g.height;
   int64_t start, end;
   tile_range(ranges, tile, geo.capacity, start, end);
   const int64_t cnt = end - start;
@@ -180,14 +193,15 @@ __global__ void __launch_bounds__(kTilePixels) k_raster_fwd(
     }
   };
 
-  const float pxc = (float)tp.px + 0.5f, pyc = (float)tp.py + 0.5f;
-  float T = 1.f, c0 = 0.f, c1 = 0.f, c2 = 0.f;
-  uint32_t last = 0;
-  bool done = !inside;
+  const float pxc = (float)tp.px + 0.5f;
+  const float2 pyc = make_float2((float)tp.py + 0.5f, (float)tp.py + 4.5f);
+  float2 T = f2(1.f), c0 = f2(0.f), c1 = f2(0.f), c2 = f2(0.f);
+  uint32_t last0 = 0, last1 = 0;
+  bool done0 = !tp.in0, done1 = !tp.in1;
   if (nb > 0) issue(0);
   int b = 0;
   for (; b < nb; ++b) {
-    if (!__syncthreads_or(!done)) break;  // block vote; also frees buffer (b+1)&1
+    if (!__syncthreads_or(!(done0 && done1))) break;  // block vote; frees buffer (b+1)&1
     if (b + 1 < nb) issue(b + 1);
     const int buf = b & 1;
     if (!__syncthreads_and(mbar_wait_bounded(&s_bar[buf], (uint32_t)((b >> 1) & 1), status))) {
@@ -196,81 +210,103 @@ __global__ void __launch_bounds__(kTilePixels) k_raster_fwd(
     }
     const int64_t rem = cnt - (int64_t)b * kBatch;
     const int m = rem < kBatch ? (int)rem : kBatch;
-    if ((int)threadIdx.x < m) s_mask[threadIdx.x] = (uint8_t)prepare_record(&s_rec[buf][threadIdx.x][0], tp.x0, tp.y0);
+    if ((int)threadIdx.x < m)
+      s_mask[threadIdx.x] = (uint8_t)prepare_record(&s_rec[buf][threadIdx.x][0], tp.x0, tp.y0);
     __syncthreads();
     const int wc = warp_list(s_mask, s_list[warp], m);
     for (int k = 0; k < wc; ++k) {
-      if ((k & 3) == 0 && __all_sync(0xffffffffu, done)) break;  // warp vote
-      if (done) continue;
+      const bool both_done = done0 && done1;
+      if ((k & 3) == 0 && __all_sync(0xffffffffu, both_done)) break;  // warp vote
+      if (both_done) continue;
       const int j = s_list[warp][k];
       const float* r = &s_rec[buf][j][0];
-      float dx, dy;
-      const float p = eval_log2_alpha(r, pxc, pyc, dx, dy);
-      if (p < kLog2AlphaMin) continue;  // alpha < 1/255
-      const float a = fminf(kAlphaMax, exp2f(p));
-      const float Tn = T * (1.f - a);
-      if (Tn < kTMin) {
-        done = true;
-        continue;
+      float dx;
+      float2 dy;
+      const float2 p = eval_log2_alpha(r, pxc, pyc, dx, dy);
+      bool ok0 = !done0 && p.x >= kLog2AlphaMin;  // alpha >= 1/255
+      bool ok1 = !done1 && p.y >= kLog2AlphaMin;
+      if (!(ok0 || ok1)) continue;
+      const float2 a = make_float2(fminf(kAlphaMax, exp2f(p.x)), fminf(kAlphaMax, exp2f(p.y)));
+      const float2 Tn = __fmul2_rn(T, __fadd2_rn(f2(1.f), make_float2(-a.x, -a.y)));
+      if (ok0 && Tn.x < kTMin) {
+        done0 = true;
+        ok0 = false;
       }
-      const float w = a * T;
-      c0 = fmaf(r[E_R], w, c0);
-      c1 = fmaf(r[E_G], w, c1);
-      c2 = fmaf(r[E_BL], w, c2);
-      T = Tn;
-      last = (uint32_t)(b * kBatch + j + 1);
+      if (ok1 && Tn.y < kTMin) {
+        done1 = true;
+        ok1 = false;
+      }
+      float2 w = __fmul2_rn(a, T);
+      w.x = ok0 ? w.x : 0.f;
+      w.y = ok1 ? w.y : 0.f;
+      c0 = __ffma2_rn(f2(r[E_R]), w, c0);
+      c1 = __ffma2_rn(f2(r[E_G]), w, c1);
+      c2 = __ffma2_rn(f2(r[E_BL]), w, c2);
+      const uint32_t pos1 = (uint32_t)(b * kBatch + j + 1);
+      if (ok0) {
+        T.x = Tn.x;
+        last0 = pos1;
+      }
+      if (ok1) {
+        T.y = Tn.y;
+        last1 = pos1;
+      }
     }
   }
   // a batch issued but not consumed must land before the block exits
   if (b < nb) mbar_wait_bounded(&s_bar[b & 1], (uint32_t)((b >> 1) & 1), status);
 
-  if (inside) {
-    const size_t hw = (size_t)geo.g.width * geo.g.height;
+  const size_t hw = (size_t)geo.g.width * geo.g.height;
+  float* img = image + (size_t)tp.view * 3 * hw;
+  float* tf = final_T + (size_t)tp.view * hw;
+  uint32_t* nc = n_contrib + (size_t)tp.view * hw;
+  if (tp.in0) {
     const size_t pix = (size_t)tp.py * geo.g.width + tp.px;
-    float* img = image + (size_t)tp.view * 3 * hw;
-    img[pix] = c0 + T * bg0;
-    img[hw + pix] = c1 + T * bg1;
-    img[2 * hw + pix] = c2 + T * bg2;
-    final_T[(size_t)tp.view * hw + pix] = T;
-    n_contrib[(size_t)tp.view * hw + pix] = last;
+    img[pix] = fmaf(T.x, bg0, c0.x);
+    img[hw + pix] = fmaf(T.x, bg1, c1.x);
+    img[2 * hw + pix] = fmaf(T.x, bg2, c2.x);
+    tf[pix] = T.x;
+    nc[pix] = last0;
+  }
+  if (tp.in1) {
+    const size_t pix = (size_t)(tp.py + 4) * geo.g.width + tp.px;
+    img[pix] = fmaf(T.y, bg0, c0.y);
+    img[hw + pix] = fmaf(T.y, bg1, c1.y);
+    img[2 * hw + pix] = fmaf(T.y, bg2, c2.y);
+    tf[pix] = T.y;
+    nc[pix] = last1;
   }
 }
 
-// Transposing butterfly: v[0..15] per lane in, the warp total of value
-// (lane >> 1) & 15 out (lanes 2k and 2k+1 both hold total k). 16 shuffles.
-__device__ __forceinline__ float warp_sum16(const float (&v)[16]) {
+// Warp sum of ten per-lane values by a transposing butterfly: each exchange
+// sends the half of the live values the partner keeps, so the live set halves
+// per step (5, 3, 2, 2, 2 shuffles). On return lane l holds in `t0` the total
+// of value ((l>>2)&1) + 3((l>>3)&1) + 5((l>>4)&1) -- one of 0,1,3,4,5,6,8,9 --
+// and in `t1` the total of value 2 + 5((l>>4)&1), i.e. 2 or 7.
+__device__ __forceinline__ void warp_sum10(const float (&v)[10], float& t0, float& t1) {
   const int lane = threadIdx.x & 31;
-  float a[8];
-  const bool h16 = lane & 16;
+  const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4;
+  float a[5];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const float send = h16 ? v[k] : v[k + 8];
-    const float keep = h16 ? v[k + 8] : v[k];
+  for (int k = 0; k < 5; ++k) {
+    const float send = h16 ? v[k] : v[k + 5];
+    const float keep = h16 ? v[k + 5] : v[k];
     a[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
   }
-  float b[4];
-  const bool h8 = lane & 8;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const float send = h8 ? a[k] : a[k + 4];
-    const float keep = h8 ? a[k + 4] : a[k];
-    b[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-  }
-  float c[2];
-  const bool h4 = lane & 4;
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const float send = h4 ? b[k] : b[k + 2];
-    const float keep = h4 ? b[k + 2] : b[k];
-    c[k] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-  }
-  const bool h2 = lane & 2;
-  float d = (h2 ? c[1] : c[0]) + __shfl_xor_sync(0xffffffffu, h2 ? c[0] : c[1], 2);
-  d += __shfl_xor_sync(0xffffffffu, d, 1);
-  return d;
+  const float b0 = (h8 ? a[3] : a[0]) + __shfl_xor_sync(0xffffffffu, h8 ? a[0] : a[3], 8);
+  const float b1 = (h8 ? a[4] : a[1]) + __shfl_xor_sync(0xffffffffu, h8 ? a[1] : a[4], 8);
+  const float b2 = a[2] + __shfl_xor_sync(0xffffffffu, a[2], 8);
+  float c0 = (h4 ? b1 : b0) + __shfl_xor_sync(0xffffffffu, h4 ? b0 : b1, 4);
+  float c1 = b2 + __shfl_xor_sync(0xffffffffu, b2, 4);
+  c0 += __shfl_xor_sync(0xffffffffu, c0, 2);
+  c1 += __shfl_xor_sync(0xffffffffu, c1, 2);
+  c0 += __shfl_xor_sync(0xffffffffu, c0, 1);
+  c1 += __shfl_xor_sync(0xffffffffu, c1, 1);
+  t0 = c0;
+  t1 = c1;
 }
 
-__global__ void __launch_bounds__(kTilePixels) k_raster_bwd(
+__global__ void __launch_bounds__(kThreads) k_raster_bwd(
     const float* __restrict__ records, const uint32_t* __restrict__ ids,
     const int64_t* __restrict__ ranges, RasterGeom geo, float bg0, float bg1, float bg2,
     const float* __restrict__ dL_dimage, const float* __restrict__ final_T,
@@ -286,33 +322,46 @@ __global__ void __launch_bounds__(kTilePixels) k_raster_bwd(
 
   const int tile = blockIdx.x;
   const TilePix tp = tile_pixel(geo.g, tile);
-  const bool inside = tp.px < geo.g.width && tp.py < geo.g.height;
   const size_t hw = (size_t)geo.g.width * geo.g.height;
-  const size_t pix = (size_t)tp.py * geo.g.width + tp.px;
+  const size_t pix0 = (size_t)tp.py * geo.g.width + tp.px;
+  const size_t pix1 = pix0 + 4 * (size_t)geo.g.width;
   int64_t start, end;
   tile_range(ranges, tile, geo.capacity, start, end);
   const float* rec_view = records + (size_t)tp.view * geo.n * GS_RECORD_FLOATS;
   float* g2_view = grad2d + (size_t)tp.view * geo.n * GS_GRAD2D_FLOATS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // per-pixel state
-  float T = 1.f, Tfin = 1.f, g0 = 0.f, g1 = 0.f, g2 = 0.f;
-  uint32_t my_nc = 0;
-  if (inside) {
-    Tfin = final_T[(size_t)tp.view * hw + pix];
-    T = Tfin;
-    my_nc = n_contrib[(size_t)tp.view * hw + pix];
+  // per-pixel state, pixel 0 in .x and pixel 1 in .y; an outside pixel has
+  // no contributors and zero upstream gradient
+  float2 Tfin = f2(1.f), g0 = f2(0.f), g1 = f2(0.f), g2 = f2(0.f);
+  uint32_t nc0 = 0, nc1 = 0;
+  {
+    const float* tf = final_T + (size_t)tp.view * hw;
+    const uint32_t* nc = n_contrib + (size_t)tp.view * hw;
     const float* gi = dL_dimage + (size_t)tp.view * 3 * hw;
-    g0 = gi[pix];
-    g1 = gi[hw + pix];
-    g2 = gi[2 * hw + pix];
+    if (tp.in0) {
+      Tfin.x = tf[pix0];
+      nc0 = nc[pix0];
+      g0.x = gi[pix0];
+      g1.x = gi[hw + pix0];
+      g2.x = gi[2 * hw + pix0];
+    }
+    if (tp.in1) {
+      Tfin.y = tf[pix1];
+      nc1 = nc[pix1];
+      g0.y = gi[pix1];
+      g1.y = gi[hw + pix1];
+      g2.y = gi[2 * hw + pix1];
+    }
   }
-  const float bgg = bg0 * g0 + bg1 * g1 + bg2 * g2;
-  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f;  // colour behind, seen from just behind
-  float last_a = 0.f, last_r = 0.f, last_g = 0.f, last_b = 0.f;
+  // T_final (bg . dL/dC): the background's share of dC/dalpha, before 1/(1-alpha)
+  const float2 tfbg =
+      __fmul2_rn(Tfin, __ffma2_rn(f2(bg2), g2, __ffma2_rn(f2(bg1), g1, __fmul2_rn(f2(bg0), g0))));
+  float2 T = Tfin;
+  float2 acc0 = f2(0.f), acc1 = f2(0.f), acc2 = f2(0.f);  // colour behind
 
   // the longest prefix any pixel of the tile used
-  const uint32_t wm = __reduce_max_sync(0xffffffffu, my_nc);
+  const uint32_t wm = __reduce_max_sync(0xffffffffu, max(nc0, nc1));
   if (lane == 0) s_wmax[warp] = wm;
   if (threadIdx.x == 0) {
     mbar_init(&s_bar[0], 1);
@@ -344,7 +393,8 @@ __global__ void __launch_bounds__(kTilePixels) k_raster_bwd(
     }
   };
 
-  const float pxc = (float)tp.px + 0.5f, pyc = (float)tp.py + 0.5f;
+  const float pxc = (float)tp.px + 0.5f;
+  const float2 pyc = make_float2((float)tp.py + 0.5f, (float)tp.py + 4.5f);
   if (nb > 0) issue(0);
   for (int it = 0; it < nb; ++it) {
     const int b = nb - 1 - it;
@@ -357,68 +407,80 @@ __global__ void __launch_bounds__(kTilePixels) k_raster_bwd(
       break;
     if ((int)threadIdx.x < m)
       s_mask[threadIdx.x] = (uint8_t)prepare_record(&s_rec[buf][threadIdx.x][0], tp.x0, tp.y0);
-#pragma unroll
-    for (int k = 0; k < GS_GRAD2D_FLOATS; ++k) s_acc[threadIdx.x][k] = 0.f;
+    {
+      float4* z = reinterpret_cast<float4*>(&s_acc[threadIdx.x][0]);
+      z[0] = z[1] = z[2] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     __syncthreads();
     const int wc = warp_list(s_mask, s_list[warp], m);
     for (int k = wc - 1; k >= 0; --k) {
       const int j = s_list[warp][k];
       const uint32_t pos = (uint32_t)(b * kBatch + j);
-      bool contrib = inside && pos < my_nc;
-      float v[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = 0.f;
-      if (contrib) {
-        const float* r = &s_rec[buf][j][0];
-        float dx, dy;
-        const float p = eval_log2_alpha(r, pxc, pyc, dx, dy);
-        if (p < kLog2AlphaMin) {
-          contrib = false;
-        } else {
-          const float a_raw = exp2f(p);
-          const float a = fminf(kAlphaMax, a_raw);
-          const float one_m = 1.f - a;
-          T = T / one_m;  // transmittance in front of this Gaussian
-          const float w = a * T;
-          const float cr = r[E_R], cg = r[E_G], cbl = r[E_BL];
-          v[6] = w * g0;
-          v[7] = w * g1;
-          v[8] = w * g2;
-          acc0 = last_a * last_r + (1.f - last_a) * acc0;
-          acc1 = last_a * last_g + (1.f - last_a) * acc1;
-          acc2 = last_a * last_b + (1.f - last_a) * acc2;
-          const float dLda = T * ((cr - acc0) * g0 + (cg - acc1) * g1 + (cbl - acc2) * g2) -
-                             Tfin * bgg / one_m;
-          last_a = a;
-          last_r = cr;
-          last_g = cg;
-          last_b = cbl;
-          if (a_raw < kAlphaMax) {
-            const float dpow = a * dLda;       // d alpha / d (-q/2) = alpha
-            v[5] = a * r[E_IO] * dLda;         // d alpha / d opacity = alpha / o
-            // -q/2 = ln2 (A dx^2 + B dx dy + C dy^2) with dx = px - u
-            const float du = -dpow * kLn2 * (2.f * r[E_A] * dx + r[E_B] * dy);
-            const float dv = -dpow * kLn2 * (r[E_B] * dx + 2.f * r[E_C] * dy);
-            v[0] = du;
-            v[1] = dv;
-            v[2] = -0.5f * dx * dx * dpow;
-            v[3] = -dx * dy * dpow;
-            v[4] = -0.5f * dy * dy * dpow;
-            v[9] = sqrtf(du * du + dv * dv);
-          }
-        }
-      }
-      const uint32_t bal = __ballot_sync(0xffffffffu, contrib);
+      const float* r = &s_rec[buf][j][0];
+      float dx;
+      float2 dy;
+      const float2 p = eval_log2_alpha(r, pxc, pyc, dx, dy);
+      const bool ok0 = pos < nc0 && p.x >= kLog2AlphaMin;
+      const bool ok1 = pos < nc1 && p.y >= kLog2AlphaMin;
+      const uint32_t bal = __ballot_sync(0xffffffffu, ok0 || ok1);
       if (bal == 0u) continue;
+      // a pixel that does not blend this Gaussian takes alpha = 0, which
+      // leaves its T and colour-behind unchanged and adds nothing below
+      const float2 araw = make_float2(exp2f(p.x), exp2f(p.y));
+      const float2 a = make_float2(ok0 ? fminf(kAlphaMax, araw.x) : 0.f,
+                                   ok1 ? fminf(kAlphaMax, araw.y) : 0.f);
+      const float2 one_m = __fadd2_rn(f2(1.f), make_float2(-a.x, -a.y));
+      const float2 inv = make_float2(ok0 ? 1.f / one_m.x : 1.f, ok1 ? 1.f / one_m.y : 1.f);
+      T = __fmul2_rn(T, inv);  // transmittance in front of this Gaussian
+      const float2 w = __fmul2_rn(a, T);
+      const float2 d0 = __fadd2_rn(f2(r[E_R]), make_float2(-acc0.x, -acc0.y));
+      const float2 d1 = __fadd2_rn(f2(r[E_G]), make_float2(-acc1.x, -acc1.y));
+      const float2 d2 = __fadd2_rn(f2(r[E_BL]), make_float2(-acc2.x, -acc2.y));
+      float2 s = __fmul2_rn(d0, g0);
+      s = __ffma2_rn(d1, g1, s);
+      s = __ffma2_rn(d2, g2, s);
+      const float2 bgt = __fmul2_rn(tfbg, inv);
+      const float2 dLda = __ffma2_rn(T, s, make_float2(-bgt.x, -bgt.y));
+      acc0 = __ffma2_rn(a, d0, acc0);
+      acc1 = __ffma2_rn(a, d1, acc1);
+      acc2 = __ffma2_rn(a, d2, acc2);
+      // d alpha / d(-q/2) = alpha below the clamp, 0 on it
+      float2 dpow = __fmul2_rn(a, dLda);
+      dpow.x = araw.x < kAlphaMax ? dpow.x : 0.f;
+      dpow.y = araw.y < kAlphaMax ? dpow.y : 0.f;
+      // -q/2 = ln2 (A dx^2 + B dx dy + C dy^2) with dx = px - u, dy = py - v
+      const float2 dpl = __fmul2_rn(dpow, f2(-kLn2));
+      const float adx2 = 2.f * r[E_A] * dx, bdx = r[E_B] * dx;
+      const float2 du = __fmul2_rn(dpl, __ffma2_rn(f2(r[E_B]), dy, f2(adx2)));
+      const float2 dv = __fmul2_rn(dpl, __ffma2_rn(f2(2.f * r[E_C]), dy, f2(bdx)));
+      const float2 dyd = __fmul2_rn(dy, dpow);
+      const float2 dy2d = __fmul2_rn(dy, dyd);
+      const float2 wg0 = __fmul2_rn(w, g0), wg1 = __fmul2_rn(w, g1), wg2 = __fmul2_rn(w, g2);
+      const float2 n2 = __ffma2_rn(dv, dv, __fmul2_rn(du, du));
+      const float sd = dpow.x + dpow.y;
+      float v[10];
+      v[0] = du.x + du.y;
+      v[1] = dv.x + dv.y;
+      v[2] = -0.5f * dx * dx * sd;
+      v[3] = -dx * (dyd.x + dyd.y);
+      v[4] = -0.5f * (dy2d.x + dy2d.y);
+      v[5] = r[E_IO] * sd;  // d alpha / d opacity = alpha / o
+      v[6] = wg0.x + wg0.y;
+      v[7] = wg1.x + wg1.y;
+      v[8] = wg2.x + wg2.y;
+      v[9] = sqrtf(n2.x) + sqrtf(n2.y);
       if (__popc(bal) == 1) {
-        if (contrib) {
+        if (ok0 || ok1) {
 #pragma unroll
           for (int e = 0; e < 10; ++e) atomicAdd(&s_acc[j][e], v[e]);
         }
       } else {
-        const float tot = warp_sum16(v);
-        const int idx = (lane >> 1) & 15;
-        if ((lane & 1) == 0 && idx < 10) atomicAdd(&s_acc[j][idx], tot);
+        float t0, t1;
+        warp_sum10(v, t0, t1);
+        const bool first = (lane & 3) == 0;
+        const int e = first ? ((lane >> 2) & 1) + 3 * ((lane >> 3) & 1) + 5 * ((lane >> 4) & 1)
+                            : 2 + 5 * ((lane >> 4) & 1);
+        if (first || (lane & 15) == 2) atomicAdd(&s_acc[j][e], first ? t0 : t1);
       }
     }
     __syncthreads();
@@ -447,8 +509,8 @@ cudaError_t launch_raster_fwd(const float* records, const uint32_t* ids, const i
   const int64_t tiles = (int64_t)g.tiles_per_view * n_views;
   if (tiles == 0) return cudaSuccess;
   RasterGeom geo{g, n, n > 0 ? capacity : 0};
-  k_raster_fwd<<<(unsigned)tiles, kTilePixels, 0, stream>>>(records, ids, ranges, geo, bg[0], bg[1],
-                                                            bg[2], image, final_T, n_contrib, status);
+  k_raster_fwd<<<(unsigned)tiles, kThreads, 0, stream>>>(records, ids, ranges, geo, bg[0], bg[1],
+                                                         bg[2], image, final_T, n_contrib, status);
   return cudaGetLastError();
 }
 
@@ -460,9 +522,9 @@ cudaError_t launch_raster_bwd(const float* records, const uint32_t* ids, const i
   const int64_t tiles = (int64_t)g.tiles_per_view * n_views;
   if (tiles == 0) return cudaSuccess;
   RasterGeom geo{g, n, n > 0 ? capacity : 0};
-  k_raster_bwd<<<(unsigned)tiles, kTilePixels, 0, stream>>>(records, ids, ranges, geo, bg[0], bg[1],
-                                                            bg[2], dL_dimage, final_T, n_contrib,
-                                                            grad2d, status);
+  k_raster_bwd<<<(unsigned)tiles, kThreads, 0, stream>>>(records, ids, ranges, geo, bg[0], bg[1],
+                                                         bg[2], dL_dimage, final_T, n_contrib,
+                                                         grad2d, status);
   return cudaGetLastError();
 }
 
