@@ -5,21 +5,21 @@
 // Julia", pwwt.cn sec. 3.3 steps 1-2 and 4.3; lshu.cn sec. 3.2
 // assign_to_tiles / sort_by_depth!), ties broken by Gaussian index.
 //
-//  k_depth_keys    (presort mode) per-Gaussian (view, depth) keys + digit
-//                  histograms.
+//  k_depth_keys    (presort mode) per-Gaussian (view, depth) keys.
 //  k_emit          one pass over the Gaussians: pair counts, a single-pass
 //                  scan across blocks (decoupled look-back, one warp reading
 //                  32 predecessors per round trip) and emission of the
-//                  (key, id) pairs through shared-memory staging; the digit
-//                  histograms of every following radix pass are accumulated
-//                  on the way.
+//                  (key, id) pairs through shared-memory staging.
 //  k_radix_count / k_radix_scan / k_radix_scatter
-//                  one stable least-significant-digit radix pass with 8-bit
-//                  digits, reduce-then-scan: per-partition digit counts, a
-//                  per-digit scan over partitions, then a scatter that ranks
-//                  each partition's keys stably (ballots over warp-striped
-//                  steps), stages them in shared memory and writes runs of
-//                  equal digits.
+//                  one stable least-significant-digit radix pass with digits
+//                  of up to 8 bits, reduce-then-scan: per-partition digit
+//                  counts, a per-digit scan over partitions (with the digit
+//                  totals), then a scatter that ranks each partition's keys
+//                  stably (ballots over warp-striped steps), stages them in
+//                  shared memory and writes runs of equal digits. The tile
+//                  bits of the 32-bit pair keys are split evenly over the
+//                  fewest passes (13 bits: 7 + 6), so each key costs one
+//                  ballot per bit of its pass.
 //  k_ranges        [start, end) of each tile in the sorted pairs.
 // The emission's look-back waits are bounded (kSpinLimit) and report through
 // the status word instead of hanging; the radix passes never wait on other
@@ -38,9 +38,9 @@ constexpr int kEmitItems = kEmitThreads * kEmitItemsPerThread;
 
 constexpr int kSortThreads = 256;
 constexpr int kSortWarps = kSortThreads / 32;
-constexpr int kSortItems = 16;
+constexpr int kSortItems = 16;                        // pair passes
 constexpr int kSortTile = kSortThreads * kSortItems;  // keys per partition
-constexpr int kRadix = 256;
+constexpr int kPresortItems = 4;                      // per-Gaussian depth passes
 
 __device__ __forceinline__ uint32_t get_block_index(uint32_t* counter) {
   __shared__ uint32_t s_idx;
@@ -75,36 +75,6 @@ __device__ __forceinline__ uint32_t block_exclusive_scan_256(uint32_t x, uint32_
   __syncthreads();
   total = s_warp[8];
   uint32_t r = s_warp[warp] + incl - x;
-  __syncthreads();
-  return r;
-}
-
-// Exclusive block-wide scan of one uint64 per thread (256 threads).
-__device__ __forceinline__ uint64_t block_exclusive_scan_256_u64(uint64_t x, uint64_t* s_warp,
-                                                                 uint64_t& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint64_t incl = x;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    uint64_t y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) s_warp[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    uint64_t w = lane < 8 ? s_warp[lane] : 0ull;
-    uint64_t wi = w;
-#pragma unroll
-    for (int o = 1; o < 8; o <<= 1) {
-      uint64_t y = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += y;
-    }
-    if (lane < 8) s_warp[lane] = wi - w;
-    if (lane == 7) s_warp[8] = wi;
-  }
-  __syncthreads();
-  total = s_warp[8];
-  uint64_t r = s_warp[warp] + incl - x;
   __syncthreads();
   return r;
 }
@@ -146,57 +116,29 @@ struct KeyTraits;
 template <>
 struct KeyTraits<uint64_t> {
   static constexpr int kBits = 64;
-  static constexpr int kBlocks = 2;  // radix scatter blocks per SM (registers)
 };
 template <>
 struct KeyTraits<uint32_t> {
   static constexpr int kBits = 32;
-  static constexpr int kBlocks = 3;
 };
 
 // ---------------------------------------------------------------------------
 // Presort keys: (view << 32 | depth bits) for visible Gaussians, all ones for
-// culled ones, value = Gaussian index within its view. Also histograms the
-// key digits of the presort passes.
+// culled ones, value = Gaussian index within its view.
 __global__ void __launch_bounds__(256) k_depth_keys(const float4* __restrict__ bins, int n,
-                                                   int n_views, int passes,
-                                                   uint64_t* __restrict__ keys,
+                                                   int n_views, uint64_t* __restrict__ keys,
                                                    uint32_t* __restrict__ vals,
-                                                   unsigned long long* __restrict__ hist,
                                                    int64_t* __restrict__ n_items_out) {
   if (blockIdx.x == 0 && threadIdx.x == 0) *n_items_out = (int64_t)n * n_views;
-  __shared__ uint32_t s_hist[8][kRadix];
-  for (int k = threadIdx.x; k < 8 * kRadix; k += blockDim.x) (&s_hist[0][0])[k] = 0u;
-  __syncthreads();
   const int64_t total = (int64_t)n * n_views;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  const uint32_t lt = lanemask_lt();
-  // uniform trip count per warp so the match.any below sees every lane
-  for (int64_t j0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); j0 < total;
-       j0 += stride) {
-    const int64_t j = j0 + (threadIdx.x & 31);
-    const bool in = j < total;
-    uint64_t key = ~0ull;
-    if (in) {
-      const float4 r2 = __ldg(&bins[j]);  // depth key, tile_x, tile_y
-      const uint32_t txw = __float_as_uint(r2.y), tyw = __float_as_uint(r2.z);
-      const bool vis = (txw & 0xffffu) <= (txw >> 16) && (tyw & 0xffffu) <= (tyw >> 16);
-      const int view = (int)(j / n);
-      key = vis ? (((uint64_t)view << 32) | (uint64_t)__float_as_uint(r2.x)) : ~0ull;
-      keys[j] = key;
-      vals[j] = (uint32_t)(j - (int64_t)view * n);
-    }
-    // warp-aggregated histogram: one shared atomic per distinct digit
-    for (int d = 0; d < passes; ++d) {
-      const uint32_t dv = in ? (uint32_t)((key >> (8 * d)) & 0xff) : 256u;
-      const uint32_t peers = __match_any_sync(0xffffffffu, dv);
-      if (in && (peers & lt) == 0) atomicAdd(&s_hist[d][dv], (uint32_t)__popc(peers));
-    }
-  }
-  __syncthreads();
-  for (int k = threadIdx.x; k < passes * kRadix; k += blockDim.x) {
-    const uint32_t c = (&s_hist[0][0])[k];
-    if (c) atomicAdd(&hist[k], (unsigned long long)c);
+  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < total;
+       j += (int64_t)gridDim.x * blockDim.x) {
+    const float4 r2 = __ldg(&bins[j]);  // depth key, tile_x, tile_y
+    const uint32_t txw = __float_as_uint(r2.y), tyw = __float_as_uint(r2.z);
+    const bool vis = (txw & 0xffffu) <= (txw >> 16) && (tyw & 0xffffu) <= (tyw >> 16);
+    const int view = (int)(j / n);
+    keys[j] = vis ? (((uint64_t)view << 32) | (uint64_t)__float_as_uint(r2.x)) : ~0ull;
+    vals[j] = (uint32_t)(j - (int64_t)view * n);
   }
 }
 
@@ -213,27 +155,21 @@ __global__ void __launch_bounds__(256) k_depth_keys(const float4* __restrict__ b
 // offsets, then row / column stepping -- and stages them in shared memory
 // (one pad word per 32 so the strided writes hit distinct banks); the block
 // then writes the window out with coalesced stores.
-// Histograms of the following radix passes (digit d into hist[d][256] for
-// d < passes): depth digits once per item weighted by its pair count, tile
-// byte 0 per pair, higher tile bytes as per-thread runs.
 template <int MODE, typename K>
 __global__ void __launch_bounds__(kEmitThreads) k_emit(
     const float4* __restrict__ bins, const uint64_t* __restrict__ pkeys,
-    const uint32_t* __restrict__ pvals, int n, int n_views, Grid g, int passes,
+    const uint32_t* __restrict__ pvals, int n, int n_views, Grid g,
     K* __restrict__ keys_out, uint32_t* __restrict__ ids_out, int64_t capacity,
-    int64_t* __restrict__ n_pairs, unsigned long long* __restrict__ hist,
-    uint64_t* __restrict__ lookback, uint32_t* __restrict__ block_counter,
+    int64_t* __restrict__ n_pairs, uint64_t* __restrict__ lookback, uint32_t* __restrict__ block_counter,
     uint32_t* __restrict__ status) {
   constexpr int kPer = MODE == 0 ? 4 : 8;           // pairs per thread per window
   constexpr int kWin = kPer * kEmitThreads;         // pairs per window
   constexpr int kWinPad = kWin + kWin / 32;
-  constexpr int kTileDigit0 = MODE == 0 ? 4 : 0;    // digit index of tile byte 0
   __shared__ uint32_t s_off[kEmitItems + 1];
   __shared__ uint32_t s_rx[kEmitItems];   // x0 | width << 16
   __shared__ uint32_t s_ry[kEmitItems];   // y0 | view << 16
   __shared__ uint32_t s_id[kEmitItems];
   __shared__ uint32_t s_depth[MODE == 0 ? kEmitItems : 1];
-  __shared__ uint32_t s_hist[8][kRadix];
   __shared__ K s_key[kWinPad];
   __shared__ uint32_t s_sid[kWinPad];
   __shared__ uint32_t s_warp[9];
@@ -242,7 +178,6 @@ __global__ void __launch_bounds__(kEmitThreads) k_emit(
   const uint32_t bidx = get_block_index(block_counter);
   const int64_t n_items = (int64_t)n * n_views;
   const int64_t first = (int64_t)bidx * kEmitItems;
-  for (int k = threadIdx.x; k < 8 * kRadix; k += kEmitThreads) (&s_hist[0][0])[k] = 0u;
 
   uint32_t cnt[kEmitItemsPerThread];
   uint32_t tsum = 0;
@@ -305,19 +240,7 @@ __global__ void __launch_bounds__(kEmitThreads) k_emit(
   const uint64_t base = s_base;
   if ((int64_t)(base + block_total) > capacity) return;  // nothing is emitted
 
-  // depth digits are shared by all pairs of a Gaussian: count them per item
-  if (MODE == 0) {
-#pragma unroll
-    for (int k = 0; k < kEmitItemsPerThread; ++k) {
-      if (!cnt[k]) continue;
-      const uint32_t dbits = s_depth[threadIdx.x * kEmitItemsPerThread + k];
-#pragma unroll
-      for (int d = 0; d < 4; ++d) atomicAdd(&s_hist[d][(dbits >> (8 * d)) & 0xff], cnt[k]);
-    }
-  }
-
   const uint32_t tiles_x = (uint32_t)g.tiles_x, tpv = (uint32_t)g.tiles_per_view;
-  const int n_tile_digits = passes - kTileDigit0;
   for (uint32_t w0 = 0; w0 < block_total; w0 += kWin) {
     const uint32_t p0 = w0 + threadIdx.x * kPer;
     if (p0 < block_total) {
@@ -335,7 +258,6 @@ __global__ void __launch_bounds__(kEmitThreads) k_emit(
       uint32_t row = local / w, col = local - row * w;
       uint32_t id = s_id[k];
       uint32_t depth = MODE == 0 ? s_depth[k] : 0u;
-      uint32_t run_v[3] = {0u, 0u, 0u}, run_n[3] = {0u, 0u, 0u};
 #pragma unroll
       for (int i = 0; i < kPer; ++i) {
         const uint32_t p = p0 + i;
@@ -358,26 +280,11 @@ __global__ void __launch_bounds__(kEmitThreads) k_emit(
         const uint32_t si = q + (q >> 5);
         s_key[si] = MODE == 0 ? (K)(((uint64_t)tile << 32) | depth) : (K)tile;
         s_sid[si] = id;
-        atomicAdd(&s_hist[kTileDigit0][tile & 255u], 1u);
-#pragma unroll
-        for (int dd = 1; dd < 4; ++dd) {
-          if (dd >= n_tile_digits) break;
-          const uint32_t dv = (tile >> (8 * dd)) & 255u;
-          if (run_n[dd - 1] && dv != run_v[dd - 1]) {
-            atomicAdd(&s_hist[kTileDigit0 + dd][run_v[dd - 1]], run_n[dd - 1]);
-            run_n[dd - 1] = 0;
-          }
-          run_v[dd - 1] = dv;
-          ++run_n[dd - 1];
-        }
         if (++col == w) {
           col = 0;
           ++row;
         }
       }
-#pragma unroll
-      for (int dd = 1; dd < 4; ++dd)
-        if (run_n[dd - 1]) atomicAdd(&s_hist[kTileDigit0 + dd][run_v[dd - 1]], run_n[dd - 1]);
     }
     __syncthreads();
     const uint32_t m = min((uint32_t)kWin, block_total - w0);
@@ -388,181 +295,217 @@ __global__ void __launch_bounds__(kEmitThreads) k_emit(
     }
     __syncthreads();
   }
-  for (int k = threadIdx.x; k < passes * kRadix; k += kEmitThreads) {
-    const uint32_t c = (&s_hist[0][0])[k];
-    if (c) atomicAdd(&hist[k], (unsigned long long)c);
-  }
 }
 
 // ---------------------------------------------------------------------------
-// Radix pass, reduce-then-scan. Partition p holds keys [p * kSortTile, ...).
-// counts / offsets: uint64 [256][stride], digit-major.
+// Radix pass, reduce-then-scan, on a BITS-wide digit (key >> shift) & (2^BITS
+// - 1). Partition p holds keys [p * TILE, (p + 1) * TILE), TILE = 256 * ITEMS.
+// counts: uint32 [2^BITS][stride], digit-major. Positions are 32-bit (the
+// caller keeps every key count below 2^31).
+
+template <int ITEMS>
+struct SortTile {
+  static constexpr int kItems = kSortThreads * ITEMS;
+};
 
 // (1) digit counts of one partition (per-warp shared histograms).
-template <typename K>
+template <typename K, int BITS, int ITEMS>
 __global__ void __launch_bounds__(kSortThreads) k_radix_count(
     const K* __restrict__ keys, const int64_t* __restrict__ n_ptr, int64_t capacity, int shift,
-    uint64_t* __restrict__ counts, int64_t stride) {
-  __shared__ uint32_t s_h[kSortWarps][kRadix];
-  const int64_t n = *n_ptr;
-  if (n > capacity || n <= 0) return;
-  const int64_t p = blockIdx.x;
-  if (p * kSortTile >= n) return;
+    uint32_t* __restrict__ counts, int64_t stride) {
+  constexpr int R = 1 << BITS;
+  constexpr uint32_t M = R - 1;
+  constexpr int TILE = SortTile<ITEMS>::kItems;
+  __shared__ uint32_t s_h[kSortWarps][R];
+  const int64_t n64 = *n_ptr;
+  if (n64 > capacity || n64 <= 0) return;
+  const uint32_t n = (uint32_t)n64;
+  const uint32_t p = blockIdx.x;
+  if (p * (uint32_t)TILE >= n) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int k = tid; k < kSortWarps * kRadix; k += kSortThreads) (&s_h[0][0])[k] = 0u;
-  const int64_t first = p * kSortTile + warp * (kSortItems * 32);
-  K key[kSortItems];
+  for (int k = tid; k < kSortWarps * R; k += kSortThreads) (&s_h[0][0])[k] = 0u;
+  const uint32_t first = p * (uint32_t)TILE + (uint32_t)warp * (ITEMS * 32) + lane;
+  K key[ITEMS];
 #pragma unroll
-  for (int it = 0; it < kSortItems; ++it) {
-    const int64_t idx = first + it * 32 + lane;
+  for (int it = 0; it < ITEMS; ++it) {
+    const uint32_t idx = first + it * 32;
     key[it] = idx < n ? keys[idx] : (K)0;
   }
   __syncthreads();
 #pragma unroll
-  for (int it = 0; it < kSortItems; ++it) {
-    const int64_t idx = first + it * 32 + lane;
-    if (idx < n) atomicAdd(&s_h[warp][(uint32_t)((key[it] >> shift) & 0xff)], 1u);
+  for (int it = 0; it < ITEMS; ++it) {
+    const uint32_t idx = first + it * 32;
+    if (idx < n) atomicAdd(&s_h[warp][(uint32_t)(key[it] >> shift) & M], 1u);
   }
   __syncthreads();
-  uint32_t c = 0;
+  for (int d = tid; d < R; d += kSortThreads) {
+    uint32_t c = 0;
 #pragma unroll
-  for (int w = 0; w < kSortWarps; ++w) c += s_h[w][tid];
-  counts[(int64_t)tid * stride + p] = c;
+    for (int w = 0; w < kSortWarps; ++w) c += s_h[w][d];
+    counts[(int64_t)d * stride + p] = c;
+  }
 }
 
 // (2) per digit (one block each): exclusive scan of its counts over the
-// partitions, plus the number of keys with a smaller digit, in place.
-__global__ void __launch_bounds__(256) k_radix_scan(uint64_t* __restrict__ counts, int64_t stride,
+// partitions, in place (coalesced 4-wide loads), and the digit's total.
+__global__ void __launch_bounds__(256) k_radix_scan(uint32_t* __restrict__ counts, int64_t stride,
                                                    const int64_t* __restrict__ n_ptr,
-                                                   int64_t capacity,
-                                                   const unsigned long long* __restrict__ hist) {
-  __shared__ uint64_t s_warp[9];
-  __shared__ uint64_t s_base;
+                                                   int64_t capacity, int tile,
+                                                   uint32_t* __restrict__ totals) {
+  __shared__ uint32_t s_warp[9];
   const int64_t n = *n_ptr;
   if (n > capacity || n <= 0) return;
-  const int64_t parts = (n + kSortTile - 1) / kSortTile;
-  const int d = blockIdx.x;
-  const int tid = threadIdx.x;
-  if (tid < 32) {
-    uint64_t s = 0;
-    for (int k = tid; k < d; k += 32) s += hist[k];
+  const int64_t parts = (n + tile - 1) / tile;
+  uint32_t* row = counts + (int64_t)blockIdx.x * stride;
+  uint32_t carry = 0;
+  for (int64_t base = 0; base < parts; base += 4 * 256) {
+    const int64_t i0 = base + 4 * (int64_t)threadIdx.x;
+    const bool full = i0 + 4 <= parts;
+    uint32_t v[4];
+    if (full) {
+      const uint4 q = *reinterpret_cast<const uint4*>(row + i0);
+      v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+    } else {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (tid == 0) s_base = s;
+      for (int k = 0; k < 4; ++k) v[k] = i0 + k < parts ? row[i0 + k] : 0u;
+    }
+    uint32_t tot;
+    uint32_t run = carry + block_exclusive_scan_256(v[0] + v[1] + v[2] + v[3], s_warp, tot);
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      o[k] = run;
+      run += v[k];
+    }
+    if (full) {
+      *reinterpret_cast<uint4*>(row + i0) = make_uint4(o[0], o[1], o[2], o[3]);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (i0 + k < parts) row[i0 + k] = o[k];
+    }
+    carry += tot;
   }
-  uint64_t* row = counts + (int64_t)d * stride;
-  // thread t scans partitions [t * chunk, (t + 1) * chunk)
-  const int64_t chunk = (parts + 255) / 256;
-  const int64_t b0 = (int64_t)tid * chunk;
-  const int64_t b1 = min(parts, b0 + chunk);
-  uint64_t sum = 0;
-  for (int64_t q = b0; q < b1; ++q) sum += row[q];
-  uint64_t tot;
-  uint64_t run = block_exclusive_scan_256_u64(sum, s_warp, tot) + s_base;
-  for (int64_t q = b0; q < b1; ++q) {
-    const uint64_t c = row[q];
-    row[q] = run;
-    run += c;
-  }
+  if (threadIdx.x == 0) totals[blockIdx.x] = carry;
 }
 
-// Lanes of the warp holding the same value d (d < 512): the intersection over
-// the 9 bits of d of the ballot of lanes agreeing on that bit. Costs the same
+// Lanes of the warp holding the same BITS-bit value d: the intersection over
+// the bits of d of the ballot of lanes agreeing on that bit. Costs the same
 // whatever the values (unlike match.any, whose cost grows with the number of
 // distinct values).
-__device__ __forceinline__ uint32_t warp_peers_9bit(uint32_t d) {
+template <int BITS>
+__device__ __forceinline__ uint32_t warp_peers(uint32_t d) {
   uint32_t peers = 0xffffffffu;
 #pragma unroll
-  for (int b = 0; b < 9; ++b) {
+  for (int b = 0; b < BITS; ++b) {
     const uint32_t bal = __ballot_sync(0xffffffffu, (d >> b) & 1u);
     peers &= ((d >> b) & 1u) ? bal : ~bal;
   }
   return peers;
 }
 
+template <typename K, int ITEMS>
+struct ScatterOcc {
+  static constexpr int kBlocks = sizeof(K) == 4 ? 3 : (ITEMS > 8 ? 2 : 4);
+};
+
+template <typename K, int BITS, int ITEMS>
+size_t scatter_smem_bytes() {
+  constexpr int R = 1 << BITS;
+  return (size_t)SortTile<ITEMS>::kItems * (sizeof(K) + 4) + (size_t)(kSortWarps + 1) * R * 4;
+}
+
 // (3) stable scatter of one partition: loads (warp-striped), per-warp digit
 // counts, block-local digit starts, ranking by ballots, staging in shared
 // memory in sorted order, then runs of equal digits written at their global
-// offsets.
-template <typename K>
-__global__ void __launch_bounds__(kSortThreads, KeyTraits<K>::kBlocks) k_radix_scatter(
+// offsets. Keys past the end take the largest digit: they rank after every
+// real key of the partition and are never written.
+template <typename K, int BITS, int ITEMS>
+__global__ void __launch_bounds__(kSortThreads, (ScatterOcc<K, ITEMS>::kBlocks)) k_radix_scatter(
     const K* __restrict__ keys_in, const uint32_t* __restrict__ vals_in,
     K* __restrict__ keys_out, uint32_t* __restrict__ vals_out,
     const int64_t* __restrict__ n_ptr, int64_t capacity, int shift,
-    const uint64_t* __restrict__ offsets, int64_t stride, uint32_t* __restrict__ status) {
-  // layout: 64-bit arrays first so every carve-out is naturally aligned
+    const uint32_t* __restrict__ offsets, int64_t stride, const uint32_t* __restrict__ totals,
+    uint32_t* __restrict__ status) {
+  constexpr int R = 1 << BITS;
+  constexpr uint32_t M = R - 1;
+  constexpr int TILE = SortTile<ITEMS>::kItems;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  uint64_t* s_gbase = reinterpret_cast<uint64_t*>(smem_raw);            // [256]
-  K* s_keys = reinterpret_cast<K*>(s_gbase + kRadix);                   // [tile]
-  uint32_t* s_vals = reinterpret_cast<uint32_t*>(s_keys + kSortTile);   // [tile]
-  uint32_t* s_whist = s_vals + kSortTile;                               // [warps][257]
-  uint32_t* s_lstart = s_whist + kSortWarps * (kRadix + 1);             // [256]
-  uint32_t* s_scan = s_lstart + kRadix;                                 // [16]
+  K* s_keys = reinterpret_cast<K*>(smem_raw);                          // [TILE]
+  uint32_t* s_vals = reinterpret_cast<uint32_t*>(s_keys + TILE);       // [TILE]
+  uint32_t* s_whist = s_vals + TILE;                                   // [warps][R]
+  uint32_t* s_delta = s_whist + kSortWarps * R;                        // [R]
+  __shared__ uint32_t s_scan[9];
 
-  const int64_t n = *n_ptr;
-  if (n > capacity || n <= 0) return;
-  const int64_t p = blockIdx.x;
-  if (p * kSortTile >= n) return;
+  const int64_t n64 = *n_ptr;
+  if (n64 > capacity || n64 <= 0) return;
+  const uint32_t n = (uint32_t)n64;
+  const uint32_t p = blockIdx.x;
+  if (p * (uint32_t)TILE >= n) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int k = tid; k < kSortWarps * (kRadix + 1); k += kSortThreads) s_whist[k] = 0u;
-  const int64_t first = p * kSortTile + warp * (kSortItems * 32);
-  K key[kSortItems];
-  uint32_t val[kSortItems];
+  for (int k = tid; k < kSortWarps * R; k += kSortThreads) s_whist[k] = 0u;
+  const uint32_t first = p * (uint32_t)TILE + (uint32_t)warp * (ITEMS * 32) + lane;
+  K key[ITEMS];
+  uint32_t val[ITEMS];
 #pragma unroll
-  for (int it = 0; it < kSortItems; ++it) {
-    const int64_t idx = first + it * 32 + lane;
+  for (int it = 0; it < ITEMS; ++it) {
+    const uint32_t idx = first + it * 32;
     key[it] = idx < n ? keys_in[idx] : (K)0;
     val[it] = idx < n ? vals_in[idx] : 0u;
   }
-  s_gbase[tid] = offsets[(int64_t)tid * stride + p];
+  // digit d's keys of this partition start at totals(< d) + offsets[d][p]
+  const uint32_t gbase = tid < R ? offsets[(int64_t)tid * stride + p] : 0u;
+  const uint32_t dtotal = tid < R ? totals[tid] : 0u;
   __syncthreads();
-  uint32_t* wh = s_whist + warp * (kRadix + 1);
+  uint32_t* wh = s_whist + warp * R;
 #pragma unroll
-  for (int it = 0; it < kSortItems; ++it) {
-    const int64_t idx = first + it * 32 + lane;
-    const uint32_t d = idx < n ? (uint32_t)((key[it] >> shift) & 0xff) : (uint32_t)kRadix;
+  for (int it = 0; it < ITEMS; ++it) {
+    const uint32_t idx = first + it * 32;
+    const uint32_t d = idx < n ? ((uint32_t)(key[it] >> shift) & M) : M;
     atomicAdd(&wh[d], 1u);
   }
-  __syncthreads();
+  uint32_t all;
+  const uint32_t dbase = block_exclusive_scan_256(dtotal, s_scan, all);  // syncs the block
   // per digit: warp offsets, block count, block-local start
   uint32_t count = 0;
+  if (tid < R) {
 #pragma unroll
-  for (int w = 0; w < kSortWarps; ++w) {
-    const uint32_t c = s_whist[w * (kRadix + 1) + tid];
-    s_whist[w * (kRadix + 1) + tid] = count;
-    count += c;
+    for (int w = 0; w < kSortWarps; ++w) {
+      const uint32_t c = s_whist[w * R + tid];
+      s_whist[w * R + tid] = count;
+      count += c;
+    }
   }
   uint32_t tot;
   const uint32_t lstart = block_exclusive_scan_256(count, s_scan, tot);
-  s_lstart[tid] = lstart;
+  if (tid < R) {
+    s_delta[tid] = dbase + gbase - lstart;  // local slot j -> global position j + delta
 #pragma unroll
-  for (int w = 0; w < kSortWarps; ++w) s_whist[w * (kRadix + 1) + tid] += lstart;
+    for (int w = 0; w < kSortWarps; ++w) s_whist[w * R + tid] += lstart;
+  }
   __syncthreads();
   // stable rank within the warp -> position within the partition
   const uint32_t lt = lanemask_lt();
 #pragma unroll
-  for (int it = 0; it < kSortItems; ++it) {
-    const int64_t idx = first + it * 32 + lane;
-    const uint32_t d = idx < n ? (uint32_t)((key[it] >> shift) & 0xff) : (uint32_t)kRadix;
-    const uint32_t peers = warp_peers_9bit(d);
+  for (int it = 0; it < ITEMS; ++it) {
+    const uint32_t idx = first + it * 32;
+    const uint32_t d = idx < n ? ((uint32_t)(key[it] >> shift) & M) : M;
+    const uint32_t peers = warp_peers<BITS>(d);
     const uint32_t before = wh[d];
     __syncwarp();
     if ((peers & lt) == 0) wh[d] = before + __popc(peers);
     __syncwarp();
-    if (idx < n) {
-      const uint32_t pos = before + __popc(peers & lt);
-      s_keys[pos] = key[it];
-      s_vals[pos] = val[it];
-    }
+    const uint32_t pos = before + __popc(peers & lt);
+    s_keys[pos] = key[it];
+    s_vals[pos] = val[it];
   }
   __syncthreads();
-  const int64_t remain = n - p * kSortTile;
-  const int valid_count = remain < kSortTile ? (int)remain : kSortTile;
-  for (int j = tid; j < valid_count; j += kSortThreads) {
+  const uint32_t remain = n - p * (uint32_t)TILE;
+  const uint32_t valid = remain < (uint32_t)TILE ? remain : (uint32_t)TILE;
+  for (uint32_t j = tid; j < valid; j += kSortThreads) {
     const K k = s_keys[j];
-    const uint32_t d = (uint32_t)((k >> shift) & 0xff);
-    const uint64_t gpos = s_gbase[d] + (uint64_t)(j - (int)s_lstart[d]);
-    if (gpos < (uint64_t)n) {
+    const uint32_t gpos = j + s_delta[(uint32_t)(k >> shift) & M];
+    if (gpos < n) {
       keys_out[gpos] = k;
       vals_out[gpos] = s_vals[j];
     } else {
@@ -633,38 +576,55 @@ __global__ void k_ranges(const K* __restrict__ keys, const int64_t* __restrict__
   }
 }
 
-size_t scatter_smem_bytes(int key_bytes) {
-  return (size_t)kRadix * 8 + (size_t)kSortTile * key_bytes + (size_t)kSortTile * 4 +
-         (size_t)kSortWarps * (kRadix + 1) * 4 + (size_t)kRadix * 4 + 16 * 4;
-}
 
-// `passes` radix passes starting at digit `first_digit`, ping-ponging between
-// (keys_a, vals_a) and (keys_b, vals_b); grid sized for `max_items`.
-template <typename K>
-cudaError_t run_radix_passes(K* keys_a, uint32_t* vals_a, K* keys_b, uint32_t* vals_b,
-                             const int64_t* n_ptr, int64_t capacity, int64_t max_items,
-                             int first_digit, int passes, const unsigned long long* hist,
-                             uint64_t* counts, int64_t stride, uint32_t* status,
-                             cudaStream_t stream) {
-  const size_t smem = scatter_smem_bytes(sizeof(K));
-  cudaError_t e = cudaFuncSetAttribute(k_radix_scatter<K>,
+template <typename K, int BITS, int ITEMS>
+cudaError_t radix_pass(const K* kin, const uint32_t* vin, K* kout, uint32_t* vout,
+                       const int64_t* n_ptr, int64_t capacity, int64_t parts, int shift,
+                       uint32_t* counts, int64_t stride, uint32_t* totals, uint32_t* status,
+                       cudaStream_t stream) {
+  const size_t smem = scatter_smem_bytes<K, BITS, ITEMS>();
+  cudaError_t e = cudaFuncSetAttribute(k_radix_scatter<K, BITS, ITEMS>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int64_t parts = (max_items + kSortTile - 1) / kSortTile;
+  k_radix_count<K, BITS, ITEMS><<<(unsigned)parts, kSortThreads, 0, stream>>>(
+      kin, n_ptr, capacity, shift, counts, stride);
+  k_radix_scan<<<1u << BITS, 256, 0, stream>>>(counts, stride, n_ptr, capacity,
+                                               SortTile<ITEMS>::kItems, totals);
+  k_radix_scatter<K, BITS, ITEMS><<<(unsigned)parts, kSortThreads, smem, stream>>>(
+      kin, vin, kout, vout, n_ptr, capacity, shift, counts, stride, totals, status);
+  return cudaGetLastError();
+}
+
+// The plan's passes, ping-ponging between (keys_a, vals_a) and (keys_b,
+// vals_b); grids sized for `max_items`, the device count read from n_ptr.
+template <typename K, int ITEMS>
+cudaError_t run_radix_passes(K* keys_a, uint32_t* vals_a, K* keys_b, uint32_t* vals_b,
+                             const int64_t* n_ptr, int64_t capacity, int64_t max_items,
+                             const RadixPlan& plan, uint32_t* counts, int64_t stride,
+                             uint32_t* totals, uint32_t* status, cudaStream_t stream) {
+  const int64_t parts = (max_items + SortTile<ITEMS>::kItems - 1) / SortTile<ITEMS>::kItems;
   if (parts == 0) return cudaSuccess;
   K* kin = keys_a;
   uint32_t* vin = vals_a;
   K* kout = keys_b;
   uint32_t* vout = vals_b;
-  for (int p = 0; p < passes; ++p) {
-    const int d = first_digit + p;
-    k_radix_count<K><<<(unsigned)parts, kSortThreads, 0, stream>>>(kin, n_ptr, capacity, 8 * d,
-                                                                   counts, stride);
-    k_radix_scan<<<kRadix, 256, 0, stream>>>(counts, stride, n_ptr, capacity,
-                                             hist + (size_t)d * kRadix);
-    k_radix_scatter<K><<<(unsigned)parts, kSortThreads, smem, stream>>>(
-        kin, vin, kout, vout, n_ptr, capacity, 8 * d, counts, stride, status);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  for (int p = 0; p < plan.passes; ++p) {
+    const int sh = plan.shift[p];
+    cudaError_t e = cudaErrorInvalidValue;
+    if constexpr (sizeof(K) == 4) {
+      switch (plan.bits[p]) {
+        case 4: e = radix_pass<K, 4, ITEMS>(kin, vin, kout, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream); break;
+        case 5: e = radix_pass<K, 5, ITEMS>(kin, vin, kout, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream); break;
+        case 6: e = radix_pass<K, 6, ITEMS>(kin, vin, kout, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream); break;
+        case 7: e = radix_pass<K, 7, ITEMS>(kin, vin, kout, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream); break;
+        case 8: e = radix_pass<K, 8, ITEMS>(kin, vin, kout, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream); break;
+        default: break;
+      }
+    } else {
+      if (plan.bits[p] == 8)
+        e = radix_pass<K, 8, ITEMS>(kin, vin, kout, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream);
+    }
+    if (e != cudaSuccess) return e;
     K* tk = kin; kin = kout; kout = tk;
     uint32_t* tv = vin; vin = vout; vout = tv;
   }
@@ -680,7 +640,26 @@ int num_sms() {
 
 }  // namespace
 
-int64_t sort_partitions(int64_t items) { return (items + kSortTile - 1) / kSortTile; }
+RadixPlan make_radix_plan(int key_bits, bool balanced) {
+  RadixPlan pl;
+  pl.passes = (key_bits + 7) / 8;
+  int shift = 0;
+  for (int i = 0; i < pl.passes; ++i) {
+    int w = 8;
+    if (balanced) w = key_bits / pl.passes + (i < key_bits % pl.passes ? 1 : 0);
+    pl.shift[i] = shift;
+    // a digit wider than its share also covers bits of the next pass (or
+    // zero bits above the key), which keeps the final order unchanged
+    pl.bits[i] = w < 4 ? 4 : w;
+    shift += w;
+  }
+  return pl;
+}
+
+int64_t pair_partitions(int64_t items) { return (items + kSortTile - 1) / kSortTile; }
+int64_t presort_partitions(int64_t items) {
+  return (items + SortTile<kPresortItems>::kItems - 1) / SortTile<kPresortItems>::kItems;
+}
 int64_t emit_blocks(int64_t items) { return (items + kEmitItems - 1) / kEmitItems; }
 
 cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
@@ -693,31 +672,31 @@ cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
   const int sms = num_sms();
   const int64_t eb = emit_blocks(n_items);
   if (a.mode == GS_SORT_PRESORT) {
-    // 1) keys (view << 32 | depth) over all Gaussians of all views
+    // 1) keys (view << 32 | depth) over all Gaussians of all views, sorted
     int64_t blocks = (n_items + 255) / 256;
     if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
-    k_depth_keys<<<(int)blocks, 256, 0, stream>>>(bins4, a.n, a.n_views, a.presort_passes,
-                                                  a.pkeys[0], a.pvals[0], a.presort_hist,
+    k_depth_keys<<<(int)blocks, 256, 0, stream>>>(bins4, a.n, a.n_views, a.pkeys[0], a.pvals[0],
                                                   a.n_items_dev);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    e = run_radix_passes<uint64_t>(a.pkeys[0], a.pvals[0], a.pkeys[1], a.pvals[1], a.n_items_dev,
-                                   n_items, n_items, 0, a.presort_passes, a.presort_hist,
-                                   a.counts, a.counts_stride, a.status, stream);
+    e = run_radix_passes<uint64_t, kPresortItems>(a.pkeys[0], a.pvals[0], a.pkeys[1], a.pvals[1],
+                                                  a.n_items_dev, n_items, n_items, a.presort,
+                                                  a.counts, a.counts_stride, a.totals, a.status,
+                                                  stream);
     if (e != cudaSuccess) return e;
-    const int fin = a.presort_passes & 1;
+    const int fin = a.presort.passes & 1;
     // 2) emission in depth order, 32-bit tile keys
     k_emit<1, uint32_t><<<(unsigned)eb, kEmitThreads, 0, stream>>>(
-        bins4, a.pkeys[fin], a.pvals[fin], a.n, a.n_views, a.grid, a.pair_passes,
+        bins4, a.pkeys[fin], a.pvals[fin], a.n, a.n_views, a.grid,
         reinterpret_cast<uint32_t*>(a.keys[a.emit_buf]), a.vals[a.emit_buf], a.capacity,
-        a.n_pairs, a.hist, a.emit_lookback, a.counters + 0, a.status);
+        a.n_pairs, a.emit_lookback, a.counters + 0, a.status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    e = run_radix_passes<uint32_t>(
+    // 3) stable sort by tile
+    e = run_radix_passes<uint32_t, kSortItems>(
         reinterpret_cast<uint32_t*>(a.keys[a.emit_buf]), a.vals[a.emit_buf],
         reinterpret_cast<uint32_t*>(a.keys[a.emit_buf ^ 1]), a.vals[a.emit_buf ^ 1], a.n_pairs,
-        a.capacity, a.capacity, 0, a.pair_passes, a.hist, a.counts, a.counts_stride, a.status,
-        stream);
+        a.capacity, a.capacity, a.pairs, a.counts, a.counts_stride, a.totals, a.status, stream);
     if (e != cudaSuccess) return e;
-    const int out = a.emit_buf ^ (a.pair_passes & 1);
+    const int out = a.emit_buf ^ (a.pairs.passes & 1);
     k_ranges<uint32_t><<<sms * 4, 256, 0, stream>>>(reinterpret_cast<uint32_t*>(a.keys[out]),
                                                    a.n_pairs, a.capacity, a.n_tiles, a.ranges,
                                                    a.status);
@@ -725,16 +704,15 @@ cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
   }
   // full 64-bit keys
   k_emit<0, uint64_t><<<(unsigned)eb, kEmitThreads, 0, stream>>>(
-      bins4, nullptr, nullptr, a.n, a.n_views, a.grid, a.pair_passes, a.keys[a.emit_buf],
-      a.vals[a.emit_buf], a.capacity, a.n_pairs, a.hist, a.emit_lookback, a.counters + 0,
-      a.status);
+      bins4, nullptr, nullptr, a.n, a.n_views, a.grid, a.keys[a.emit_buf], a.vals[a.emit_buf],
+      a.capacity, a.n_pairs, a.emit_lookback, a.counters + 0, a.status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  e = run_radix_passes<uint64_t>(a.keys[a.emit_buf], a.vals[a.emit_buf], a.keys[a.emit_buf ^ 1],
-                                 a.vals[a.emit_buf ^ 1], a.n_pairs, a.capacity, a.capacity, 0,
-                                 a.pair_passes, a.hist, a.counts, a.counts_stride, a.status,
-                                 stream);
+  e = run_radix_passes<uint64_t, kSortItems>(a.keys[a.emit_buf], a.vals[a.emit_buf],
+                                             a.keys[a.emit_buf ^ 1], a.vals[a.emit_buf ^ 1],
+                                             a.n_pairs, a.capacity, a.capacity, a.pairs, a.counts,
+                                             a.counts_stride, a.totals, a.status, stream);
   if (e != cudaSuccess) return e;
-  const int out = a.emit_buf ^ (a.pair_passes & 1);
+  const int out = a.emit_buf ^ (a.pairs.passes & 1);
   k_ranges<uint64_t><<<sms * 4, 256, 0, stream>>>(a.keys[out], a.n_pairs, a.capacity, a.n_tiles,
                                                   a.ranges, a.status);
   return cudaGetLastError();

@@ -19,7 +19,8 @@ constexpr size_t kControlBytes = 4096;  // status word, counters, device scalars
 constexpr size_t kStatusOffset = 0;
 constexpr size_t kCountersOffset = 64;   // 16 x uint32
 constexpr size_t kNItemsOffset = 256;    // int64
-constexpr size_t kHistBytes = 8 * 256 * sizeof(unsigned long long);
+constexpr size_t kHistBytes = 256 * sizeof(uint32_t);  // digit totals of the current pass
+constexpr int64_t kMaxPairCapacity = GS_MAX_PAIR_CAPACITY;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -32,11 +33,10 @@ int bits_for(uint64_t max_value) {
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct Layout {
-  int pair_passes = 0;
-  int presort_passes = 0;
+  RadixPlan pairs, presort;
   int key_bytes = 8;
   int64_t counts_stride = 0;
-  size_t off_hist = 0, off_phist = 0, off_emit_lb = 0, off_counts = 0, off_keys0 = 0, off_keys1 = 0,
+  size_t off_hist = 0, off_emit_lb = 0, off_counts = 0, off_keys0 = 0, off_keys1 = 0,
          off_vals1 = 0, off_pkeys0 = 0, off_pkeys1 = 0, off_pvals0 = 0, off_pvals1 = 0;
   size_t total = 0;
 };
@@ -54,7 +54,8 @@ bool check_cams(const gs_camera* cams, int32_t n_views) {
 
 bool make_layout(int64_t n, int32_t n_views, const gs_camera* cams, int64_t capacity, int32_t mode,
                  Layout& L) {
-  if (n < 0 || n >= (1ll << 31) || capacity < 0) return false;
+  // pair positions are 32-bit inside the sort
+  if (n < 0 || n >= (1ll << 31) || capacity < 0 || capacity > kMaxPairCapacity) return false;
   if (mode != GS_SORT_FULL64 && mode != GS_SORT_PRESORT) return false;
   if (!check_cams(cams, n_views)) return false;
   const Grid g = grid_of(cams[0]);
@@ -64,24 +65,22 @@ bool make_layout(int64_t n, int32_t n_views, const gs_camera* cams, int64_t capa
   const int64_t items = n * n_views;
   if (mode == GS_SORT_FULL64) {
     L.key_bytes = 8;
-    L.pair_passes = (32 + tile_bits + 7) / 8;
-    L.presort_passes = 0;
+    L.pairs = make_radix_plan(32 + tile_bits, false);
   } else {
     L.key_bytes = 4;
-    L.pair_passes = (tile_bits + 7) / 8;
-    L.presort_passes = 4 + (n_views > 1 ? 1 : 0);
+    L.pairs = make_radix_plan(tile_bits, true);
+    L.presort = make_radix_plan(32 + bits_for((uint64_t)n_views - 1), false);
   }
-  int64_t parts = sort_partitions(capacity);
+  int64_t parts = pair_partitions(capacity);
   if (mode == GS_SORT_PRESORT) {
-    const int64_t p2 = sort_partitions(items);
+    const int64_t p2 = presort_partitions(items);
     if (p2 > parts) parts = p2;
   }
-  L.counts_stride = parts > 0 ? parts : 1;
+  L.counts_stride = parts > 0 ? (parts + 3) / 4 * 4 : 4;
   size_t off = kControlBytes;
   L.off_hist = off; off = align_up(off + kHistBytes);
-  L.off_phist = off; off = align_up(off + kHistBytes);
   L.off_emit_lb = off; off = align_up(off + (size_t)emit_blocks(items) * 8);
-  L.off_counts = off; off = align_up(off + (size_t)256 * L.counts_stride * 8);
+  L.off_counts = off; off = align_up(off + (size_t)256 * L.counts_stride * 4);
   L.off_keys0 = off; off = align_up(off + (size_t)capacity * L.key_bytes);
   L.off_keys1 = off; off = align_up(off + (size_t)capacity * L.key_bytes);
   L.off_vals1 = off; off = align_up(off + (size_t)capacity * 4);
@@ -166,8 +165,6 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
   const int64_t items = n * n_views;
 
   if (cudaMemsetAsync(w + kCountersOffset, 0, 16 * sizeof(uint32_t), st) != cudaSuccess ||
-      cudaMemsetAsync(w + L.off_hist, 0, kHistBytes, st) != cudaSuccess ||
-      cudaMemsetAsync(w + L.off_phist, 0, kHistBytes, st) != cudaSuccess ||
       cudaMemsetAsync(w + L.off_emit_lb, 0, (size_t)emit_blocks(items) * 8, st) != cudaSuccess ||
       cudaMemsetAsync(out->ranges, 0, (size_t)tiles * 2 * sizeof(int64_t), st) != cudaSuccess)
     return GS_ERR_CUDA;
@@ -180,9 +177,9 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
   a.mode = sort_mode;
   a.grid = g;
   a.capacity = out->pair_capacity;
-  a.pair_passes = L.pair_passes;
-  a.presort_passes = L.presort_passes;
-  a.emit_buf = L.pair_passes & 1;
+  a.pairs = L.pairs;
+  a.presort = L.presort;
+  a.emit_buf = L.pairs.passes & 1;
   a.keys[0] = reinterpret_cast<uint64_t*>(w + L.off_keys0);
   a.keys[1] = reinterpret_cast<uint64_t*>(w + L.off_keys1);
   a.vals[0] = out->ids;
@@ -193,9 +190,8 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
     a.pvals[0] = reinterpret_cast<uint32_t*>(w + L.off_pvals0);
     a.pvals[1] = reinterpret_cast<uint32_t*>(w + L.off_pvals1);
   }
-  a.hist = reinterpret_cast<unsigned long long*>(w + L.off_hist);
-  a.presort_hist = reinterpret_cast<unsigned long long*>(w + L.off_phist);
-  a.counts = reinterpret_cast<uint64_t*>(w + L.off_counts);
+  a.totals = reinterpret_cast<uint32_t*>(w + L.off_hist);
+  a.counts = reinterpret_cast<uint32_t*>(w + L.off_counts);
   a.counts_stride = L.counts_stride;
   a.emit_lookback = reinterpret_cast<uint64_t*>(w + L.off_emit_lb);
   a.counters = reinterpret_cast<uint32_t*>(w + kCountersOffset);

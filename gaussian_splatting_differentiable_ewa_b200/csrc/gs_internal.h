@@ -9,6 +9,18 @@
 
 namespace gsb {
 
+// Digits of a least-significant-digit radix sort: pass i orders by
+// (key >> shift[i]) & (2^bits[i] - 1).
+struct RadixPlan {
+  int passes = 0;
+  int shift[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  int bits[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+};
+
+// `key_bits` significant bits in the fewest passes of at most 8 bits; with
+// `balanced` the bits are split evenly (13 -> 7 + 6), else 8 per pass.
+RadixPlan make_radix_plan(int key_bits, bool balanced);
+
 struct BinSortArgs {
   const float* bins;    // [n_views][n][4] binning records
   int n;
@@ -16,17 +28,16 @@ struct BinSortArgs {
   int mode;
   Grid grid;
   int64_t capacity;
-  int pair_passes;     // radix passes over the pair keys
-  int presort_passes;  // radix passes over the per-Gaussian depth keys
+  RadixPlan pairs;     // radix passes over the pair keys
+  RadixPlan presort;   // radix passes over the per-Gaussian depth keys
   int emit_buf;        // which key/value buffer the emission writes
   uint64_t* keys[2];   // pair keys (64-bit, or 32-bit in presort mode)
   uint32_t* vals[2];   // pair ids; the final one is the caller's ids array
   uint64_t* pkeys[2];  // presort keys
   uint32_t* pvals[2];  // presort values
-  unsigned long long* hist;          // [8][256] pair-key digit histograms
-  unsigned long long* presort_hist;  // [8][256]
-  uint64_t* counts;                  // [256][counts_stride] radix digit counts / offsets
-  int64_t counts_stride;             // partitions of the largest pass
+  uint32_t* totals;                  // [256] keys per digit of the current pass
+  uint32_t* counts;                  // [256][counts_stride] radix digit counts / offsets
+  int64_t counts_stride;             // partitions of the largest pass, a multiple of 4
   uint64_t* emit_lookback;           // [emit blocks]
   uint32_t* counters;                // [16] dynamic block counters
   uint32_t* status;
@@ -58,7 +69,8 @@ cudaError_t launch_densify(const float* grad2d, const int* radii, int n_views, i
 cudaError_t launch_adam(const gs_adam_group* groups, int n_groups, float b1, float b2, float eps,
                         int64_t step, cudaStream_t stream);
 
-int64_t sort_partitions(int64_t items);
+int64_t pair_partitions(int64_t items);     // radix partitions over pair keys
+int64_t presort_partitions(int64_t items);  // radix partitions over depth keys
 int64_t emit_blocks(int64_t items);
 
 }  // namespace gsb

@@ -44,6 +44,7 @@ extern "C" {
 #define GS_MAX_VIEWS 32       /* views per call */
 #define GS_RECORD_FLOATS 12   /* floats per projected record */
 #define GS_GRAD2D_FLOATS 12   /* floats per screen-space gradient record */
+#define GS_MAX_PAIR_CAPACITY ((int64_t)1 << 31) /* pair positions are 32-bit */
 
 typedef enum gs_status {
   GS_OK = 0,
@@ -166,7 +167,8 @@ const char* gs_status_string(gs_status status);
 
 /* Bytes of workspace gs_bin_sort needs for n Gaussians, n_views views of
  * cams[0]'s size, pair_capacity pairs and the given sort mode. Returns 0 for
- * invalid arguments. The workspace must be 256-byte aligned; its first 256
+ * invalid arguments, pair_capacity above GS_MAX_PAIR_CAPACITY included. The
+ * workspace must be 256-byte aligned; its first 256
  * bytes hold the device status word and counters; zero them once (e.g.
  * cudaMemset) before the workspace is first used. */
 size_t gs_workspace_size(int64_t n, int32_t n_views, const gs_camera* cams,
