@@ -7,8 +7,8 @@
 // backward), plus a visibility count.
 //
 // Adam (lshu.cn sec. 3.3 / 5.3, per-group learning rates): one launch over
-// every group, float4-vectorised, IEEE square root and division so the step
-// does not depend on fast-math approximations.
+// every group, float4-vectorised, streaming loads and stores (each float is
+// touched once per step), square root and division on the SFU.
 
 #include <cuda_runtime.h>
 
@@ -57,17 +57,20 @@ constexpr int kAdamThreads = 256;
 constexpr int kAdamVecPerThread = 4;
 constexpr int64_t kAdamFloatsPerBlock = (int64_t)kAdamThreads * kAdamVecPerThread * 4;
 
+// One Adam update; ibc1 = 1 / (1 - b1^t), ibc2 = 1 / (1 - b2^t). The square
+// root and the division use the SFU (a few ulp on the step, far inside the
+// update's own scale), which keeps the kernel on HBM rather than on the
+// multi-instruction IEEE sequences.
 __device__ __forceinline__ void adam_one(float& p, float g, float& m, float& v, float lr, float b1,
-                                         float b2, float eps, float bc1, float bc2) {
+                                         float b2, float eps, float ibc1, float ibc2) {
   m = fmaf(b1, m, (1.f - b1) * g);
   v = fmaf(b2, v, (1.f - b2) * g * g);
-  const float mhat = __fdiv_rn(m, bc1);
-  const float vhat = __fdiv_rn(v, bc2);
-  p -= lr * __fdiv_rn(mhat, __fadd_rn(__fsqrt_rn(vhat), eps));
+  const float denom = sqrtf(v * ibc2) + eps;
+  p -= __fdividef(lr * (m * ibc1), denom);
 }
 
 __global__ void __launch_bounds__(kAdamThreads) k_adam(AdamTable t, float b1, float b2, float eps,
-                                                       float bc1, float bc2) {
+                                                       float ibc1, float ibc2) {
   int gi = 0;
   while (gi + 1 < t.n_groups && (int64_t)blockIdx.x >= t.block_start[gi + 1]) ++gi;
   const int64_t count = t.count[gi];
@@ -86,17 +89,17 @@ __global__ void __launch_bounds__(kAdamThreads) k_adam(AdamTable t, float b1, fl
       const float4 g = __ldcs(reinterpret_cast<const float4*>(G + e));
       float4 m = __ldcs(reinterpret_cast<const float4*>(M + e));
       float4 v = __ldcs(reinterpret_cast<const float4*>(V + e));
-      adam_one(p.x, g.x, m.x, v.x, lr, b1, b2, eps, bc1, bc2);
-      adam_one(p.y, g.y, m.y, v.y, lr, b1, b2, eps, bc1, bc2);
-      adam_one(p.z, g.z, m.z, v.z, lr, b1, b2, eps, bc1, bc2);
-      adam_one(p.w, g.w, m.w, v.w, lr, b1, b2, eps, bc1, bc2);
+      adam_one(p.x, g.x, m.x, v.x, lr, b1, b2, eps, ibc1, ibc2);
+      adam_one(p.y, g.y, m.y, v.y, lr, b1, b2, eps, ibc1, ibc2);
+      adam_one(p.z, g.z, m.z, v.z, lr, b1, b2, eps, ibc1, ibc2);
+      adam_one(p.w, g.w, m.w, v.w, lr, b1, b2, eps, ibc1, ibc2);
       __stcs(reinterpret_cast<float4*>(P + e), p);
       __stcs(reinterpret_cast<float4*>(M + e), m);
       __stcs(reinterpret_cast<float4*>(V + e), v);
     } else {
       for (int64_t f = e; f < count && f < e + 4; ++f) {
         float p = P[f], m = M[f], v = V[f];
-        adam_one(p, G[f], m, v, lr, b1, b2, eps, bc1, bc2);
+        adam_one(p, G[f], m, v, lr, b1, b2, eps, ibc1, ibc2);
         P[f] = p;
         M[f] = m;
         V[f] = v;
@@ -134,7 +137,8 @@ cudaError_t launch_adam(const gs_adam_group* groups, int n_groups, float b1, flo
   if (blocks == 0) return cudaSuccess;
   const double bc1 = 1.0 - pow((double)b1, (double)step);
   const double bc2 = 1.0 - pow((double)b2, (double)step);
-  k_adam<<<(unsigned)blocks, kAdamThreads, 0, stream>>>(t, b1, b2, eps, (float)bc1, (float)bc2);
+  k_adam<<<(unsigned)blocks, kAdamThreads, 0, stream>>>(t, b1, b2, eps, (float)(1.0 / bc1),
+                                                        (float)(1.0 / bc2));
   return cudaGetLastError();
 }
 

@@ -11,13 +11,15 @@
 //
 // The tile's depth-sorted list is consumed in batches of 128 records; each
 // thread stages one 48-byte record into shared memory with a TMA bulk copy
-// (cp.async.bulk completing on an mbarrier), double-buffered so the next batch
-// is in flight while the current one is blended. When a batch lands, thread j
+// (cp.async.bulk completing on an mbarrier). When a batch lands, thread j
 // rewrites record j into evaluation form (log2-scaled conic, log2 opacity) and
 // marks which warps' pixel blocks its alpha >= 1/255 box reaches; every warp
 // then compacts the batch to the records that can touch its pixels (ballot +
 // popc, order kept) and walks only those. The box is conservative, so the
 // skipped records are exactly ones every pixel of the block would skip.
+// The forward writes the evaluation form to a separate array of (x, x) pairs,
+// so the landing buffer is free for the next batch's copy at once; the
+// backward rewrites records in place (scalar form) and double-buffers.
 //
 // Forward (pwwt.cn sec. 3.3 `composite`, front to back; lshu.cn sec. 3.2
 // `blend`): alpha = min(0.99, o exp(-q/2)); skip alpha < 1/255; stop before a
@@ -50,11 +52,11 @@ constexpr float kLog2AlphaMin = -7.994353436858858f;  // log2(1/255)
 
 static_assert(kTilePixels == 2 * kThreads, "two pixels per thread");
 
-// Evaluation-form record slots (after the per-batch rewrite in shared memory):
-// 0 u, 1 v, 2 A = -log2(e)/2 conic_a, 3 B = -log2(e) conic_b,
-// 4 C = -log2(e)/2 conic_c, 5 log2(opacity), 6..8 colour, 9 1/opacity.
-enum EvalSlot { E_U = 0, E_V = 1, E_A = 2, E_B = 3, E_C = 4, E_LO = 5, E_R = 6, E_G = 7,
-                E_BL = 8, E_IO = 9 };
+// Evaluation form of a record, one (x, x) pair per field, so the two-pixel
+// arithmetic takes every operand straight from shared memory:
+// -u, -v, A = -log2(e)/2 conic_a, B = -log2(e) conic_b, C = -log2(e)/2 conic_c,
+// log2(opacity), colour r g b, 2C. 80 bytes per record (the forward's form).
+enum EvPair { V_NU = 0, V_NV, V_A, V_B, V_C, V_LO, V_R, V_G, V_BL, V_C2, kEvPairs };
 
 struct RasterGeom {
   Grid g;
@@ -94,32 +96,12 @@ __device__ __forceinline__ TilePix tile_pixel(const Grid& g, int tile) {
   return t;
 }
 
-// log2 of the unclamped alpha at the pair's pixel centres (pxc, pyc.x) and
-// (pxc, pyc.y); per pixel it is fma(A dx, dx, fma(B dx, dy, fma(C dy, dy, lo)))
-// with dx = pxc - u, dy = pyc - v. Both directions call this one function, so
-// their skip / stop decisions agree bit for bit.
-__device__ __forceinline__ float2 eval_log2_alpha(const float* r, float pxc, float2 pyc, float& dx,
-                                                  float2& dy) {
-  dx = pxc - r[E_U];
-  dy = __fadd2_rn(pyc, f2(-r[E_V]));
-  float2 t = __ffma2_rn(__fmul2_rn(f2(r[E_C]), dy), dy, f2(r[E_LO]));
-  t = __ffma2_rn(f2(r[E_B] * dx), dy, t);
-  return __ffma2_rn(f2(r[E_A] * dx), f2(dx), t);
-}
-
-// Rewrite record j of a landed batch into evaluation form and return the
-// 4-bit mask of warps whose 8x8 pixel block its alpha >= 1/255 box overlaps.
-__device__ __forceinline__ uint32_t prepare_record(float* r, int x0, int y0) {
-  const float u = r[R_U], v = r[R_V], hx = r[R_HX], hy = r[R_HY];
-  const float o = r[R_OPAC];
-  const float ca = r[R_CA], cb = r[R_CB], cc = r[R_CC];
-  r[E_A] = -0.5f * kLog2e * ca;
-  r[E_B] = -kLog2e * cb;
-  r[E_C] = -0.5f * kLog2e * cc;
-  r[E_LO] = __log2f(o);
-  r[E_IO] = 1.f / o;
+// 4-bit mask of the warps whose 8x8 pixel block the alpha >= 1/255 box
+// [u - hx, u + hx] x [v - hy, v + hy] overlaps, on pixel-centre extents (a
+// record without a box, hx < 0 or NaN, reaches none).
+__device__ __forceinline__ uint32_t warp_block_mask(float u, float v, float hx, float hy, int x0,
+                                                    int y0) {
   if (!(hx >= 0.f)) return 0u;
-  // pixel-centre extents of the warp blocks: 8 wide, 8 high
   uint32_t xm = 0, ym = 0;
 #pragma unroll
   for (int bi = 0; bi < 2; ++bi) {
@@ -133,6 +115,74 @@ __device__ __forceinline__ uint32_t prepare_record(float* r, int x0, int y0) {
   for (int w = 0; w < kWarps; ++w)
     if (((xm >> (w & 1)) & 1u) && ((ym >> (w >> 1)) & 1u)) mask |= 1u << w;
   return mask;
+}
+
+// log2 of the unclamped alpha at the pair's pixel centres (pxc, pyc.x) and
+// (pxc, pyc.y); per pixel it is fma(A dx, dx, fma(B dx, dy, fma(C dy, dy, lo)))
+// with dx = pxc - u, dy = pyc - v. dx, A dx and B dx come out as (x, x)
+// pairs. Both directions call this one function, so their skip / stop
+// decisions agree bit for bit.
+__device__ __forceinline__ float2 eval_log2_alpha(const float2* e, float2 pxc, float2 pyc,
+                                                  float2& dx, float2& dy, float2& adx,
+                                                  float2& bdx) {
+  dx = __fadd2_rn(pxc, e[V_NU]);
+  dy = __fadd2_rn(pyc, e[V_NV]);
+  float2 t = __ffma2_rn(__fmul2_rn(e[V_C], dy), dy, e[V_LO]);
+  bdx = __fmul2_rn(e[V_B], dx);
+  t = __ffma2_rn(bdx, dy, t);
+  adx = __fmul2_rn(e[V_A], dx);
+  return __ffma2_rn(adx, dx, t);
+}
+
+// Write the evaluation form of raw record r and return the 4-bit mask of
+// warps whose 8x8 pixel block its alpha >= 1/255 box overlaps.
+__device__ __forceinline__ uint32_t prepare_record(const float* r, float2* e, int x0, int y0) {
+  const float u = r[R_U], v = r[R_V], hx = r[R_HX], hy = r[R_HY];
+  const float o = r[R_OPAC];
+  const float A = -0.5f * kLog2e * r[R_CA], B = -kLog2e * r[R_CB], C = -0.5f * kLog2e * r[R_CC];
+  float4* e4 = reinterpret_cast<float4*>(e);
+  e4[0] = make_float4(-u, -u, -v, -v);
+  e4[1] = make_float4(A, A, B, B);
+  const float lo = __log2f(o);
+  e4[2] = make_float4(C, C, lo, lo);
+  e4[3] = make_float4(r[R_R], r[R_R], r[R_G], r[R_G]);
+  e4[4] = make_float4(r[R_B], r[R_B], 2.f * C, 2.f * C);
+  return warp_block_mask(u, v, hx, hy, x0, y0);
+}
+
+// Backward: records are rewritten in place into a scalar evaluation form
+// (slots after the per-batch rewrite in shared memory):
+// 0 u, 1 v, 2 A = -log2(e)/2 conic_a, 3 B = -log2(e) conic_b,
+// 4 C = -log2(e)/2 conic_c, 5 log2(opacity), 6..8 colour, 9 1/opacity.
+enum EvalSlot { E_U = 0, E_V = 1, E_A = 2, E_B = 3, E_C = 4, E_LO = 5, E_R = 6, E_G = 7,
+                E_BL = 8, E_IO = 9 };
+
+// eval_log2_alpha on a scalar evaluation record: per pixel the same IEEE
+// operations in the same order (pxc - u, pyc - v, C dy, fma(C dy, dy, lo),
+// B dx, fma(B dx, dy, .), A dx, fma(A dx, dx, .)), so the backward's skip
+// decisions are bit-identical to the forward's.
+__device__ __forceinline__ float2 eval_log2_alpha_s(const float* r, float pxc, float2 pyc, float& dx,
+                                                  float2& dy) {
+  dx = pxc - r[E_U];
+  dy = __fadd2_rn(pyc, f2(-r[E_V]));
+  float2 t = __ffma2_rn(__fmul2_rn(f2(r[E_C]), dy), dy, f2(r[E_LO]));
+  t = __ffma2_rn(f2(r[E_B] * dx), dy, t);
+  return __ffma2_rn(f2(r[E_A] * dx), f2(dx), t);
+}
+
+// Rewrite record j of a landed batch in place into the scalar evaluation form
+// and return the 4-bit mask of warps whose 8x8 pixel block its alpha >= 1/255
+// box overlaps.
+__device__ __forceinline__ uint32_t prepare_record_s(float* r, int x0, int y0) {
+  const float u = r[R_U], v = r[R_V], hx = r[R_HX], hy = r[R_HY];
+  const float o = r[R_OPAC];
+  const float ca = r[R_CA], cb = r[R_CB], cc = r[R_CC];
+  r[E_A] = -0.5f * kLog2e * ca;
+  r[E_B] = -kLog2e * cb;
+  r[E_C] = -0.5f * kLog2e * cc;
+  r[E_LO] = __log2f(o);
+  r[E_IO] = 1.f / o;
+  return warp_block_mask(u, v, hx, hy, x0, y0);
 }
 
 // Warp-wide compaction of the batch entries whose mask has this warp's bit,
@@ -158,8 +208,9 @@ __global__ void __launch_bounds__(kThreads) k_raster_fwd(
     const int64_t* __restrict__ ranges, RasterGeom geo, float bg0, float bg1, float bg2,
     float* __restrict__ image, float* __restrict__ final_T, uint32_t* __restrict__ n_contrib,
     uint32_t* __restrict__ status) {
-  __shared__ __align__(128) float s_rec[2][kBatch][GS_RECORD_FLOATS];
-  __shared__ __align__(8) uint64_t s_bar[2];
+  __shared__ __align__(128) float s_rec[kBatch][GS_RECORD_FLOATS];
+  __shared__ __align__(16) float2 s_ev[kBatch][kEvPairs];
+  __shared__ __align__(8) uint64_t s_bar;
   __shared__ uint8_t s_mask[kBatch];
   __shared__ uint8_t s_list[kWarps][kBatch];
 
@@ -173,88 +224,98 @@ __global__ void __launch_bounds__(kThreads) k_raster_fwd(
   const int warp = threadIdx.x >> 5;
 
   if (threadIdx.x == 0) {
-    mbar_init(&s_bar[0], 1);
-    mbar_init(&s_bar[1], 1);
+    mbar_init(&s_bar, 1);
     fence_mbar_init();
   }
   __syncthreads();
 
+  // batch b's records land in s_rec (one copy in flight at a time: a batch
+  // is converted into s_ev as soon as it lands, which frees s_rec for the
+  // next one while the current batch is blended)
   auto issue = [&](int b) {
-    const int buf = b & 1;
     const int64_t first = start + (int64_t)b * kBatch;
     const int64_t rem = end - first;
     const int m = rem < kBatch ? (int)rem : kBatch;
-    if (threadIdx.x == 0) mbar_arrive_expect_tx(&s_bar[buf], (uint32_t)(m * kRecBytes));
+    if (threadIdx.x == 0) mbar_arrive_expect_tx(&s_bar, (uint32_t)(m * kRecBytes));
     if ((int)threadIdx.x < m) {
       uint32_t id = __ldg(&ids[first + threadIdx.x]);
       if (id >= (uint32_t)geo.n) id = 0;  // never read outside the records
-      bulk_copy_g2s(&s_rec[buf][threadIdx.x][0], rec_view + (size_t)id * GS_RECORD_FLOATS,
-                    kRecBytes, &s_bar[buf]);
+      bulk_copy_g2s(&s_rec[threadIdx.x][0], rec_view + (size_t)id * GS_RECORD_FLOATS, kRecBytes,
+                    &s_bar);
     }
   };
 
-  const float pxc = (float)tp.px + 0.5f;
+  const float kInf = __int_as_float(0x7f800000);
+  const float2 pxc = f2((float)tp.px + 0.5f);
   const float2 pyc = make_float2((float)tp.py + 0.5f, (float)tp.py + 4.5f);
-  float2 T = f2(1.f), c0 = f2(0.f), c1 = f2(0.f), c2 = f2(0.f);
+  const float2 one = f2(1.f), mone = f2(-1.f);
+  float2 T = one, c0 = f2(0.f), c1 = f2(0.f), c2 = f2(0.f);
   uint32_t last0 = 0, last1 = 0;
-  bool done0 = !tp.in0, done1 = !tp.in1;
-  if (nb > 0) issue(0);
+  // a pixel takes a Gaussian when log2(alpha) >= its threshold: log2(1/255)
+  // while it composites, +inf once it is done (or outside the image)
+  float thr0 = tp.in0 ? kLog2AlphaMin : kInf, thr1 = tp.in1 ? kLog2AlphaMin : kInf;
+  bool done = !(tp.in0 || tp.in1);
+  bool pending = nb > 0;  // batch b's copy is in flight
+  if (pending) issue(0);
   int b = 0;
   for (; b < nb; ++b) {
-    if (!__syncthreads_or(!(done0 && done1))) break;  // block vote; frees buffer (b+1)&1
-    if (b + 1 < nb) issue(b + 1);
-    const int buf = b & 1;
-    if (!__syncthreads_and(mbar_wait_bounded(&s_bar[buf], (uint32_t)((b >> 1) & 1), status))) {
-      b = nb;  // a copy never landed: give up on the tile
+    if (!__syncthreads_or(!done)) break;  // block vote; the previous batch is finished
+    if (!__syncthreads_and(mbar_wait_bounded(&s_bar, (uint32_t)(b & 1), status))) {
+      pending = false;  // a copy never landed: give up on the tile
       break;
     }
+    pending = false;
     const int64_t rem = cnt - (int64_t)b * kBatch;
     const int m = rem < kBatch ? (int)rem : kBatch;
     if ((int)threadIdx.x < m)
-      s_mask[threadIdx.x] = (uint8_t)prepare_record(&s_rec[buf][threadIdx.x][0], tp.x0, tp.y0);
-    __syncthreads();
+      s_mask[threadIdx.x] =
+          (uint8_t)prepare_record(&s_rec[threadIdx.x][0], &s_ev[threadIdx.x][0], tp.x0, tp.y0);
+    __syncthreads();  // s_rec is free again
+    if (b + 1 < nb) {
+      issue(b + 1);
+      pending = true;
+    }
     const int wc = warp_list(s_mask, s_list[warp], m);
+    const uint32_t pos0 = (uint32_t)(b * kBatch + 1);
     for (int k = 0; k < wc; ++k) {
-      const bool both_done = done0 && done1;
-      if ((k & 3) == 0 && __all_sync(0xffffffffu, both_done)) break;  // warp vote
-      if (both_done) continue;
+      if ((k & 3) == 0 && __all_sync(0xffffffffu, done)) break;  // warp vote
       const int j = s_list[warp][k];
-      const float* r = &s_rec[buf][j][0];
-      float dx;
-      float2 dy;
-      const float2 p = eval_log2_alpha(r, pxc, pyc, dx, dy);
-      bool ok0 = !done0 && p.x >= kLog2AlphaMin;  // alpha >= 1/255
-      bool ok1 = !done1 && p.y >= kLog2AlphaMin;
+      const float2* e = &s_ev[j][0];
+      float2 dx, dy, adx, bdx;
+      const float2 p = eval_log2_alpha(e, pxc, pyc, dx, dy, adx, bdx);
+      bool ok0 = p.x >= thr0, ok1 = p.y >= thr1;
       if (!(ok0 || ok1)) continue;
-      const float2 a = make_float2(fminf(kAlphaMax, exp2f(p.x)), fminf(kAlphaMax, exp2f(p.y)));
-      const float2 Tn = __fmul2_rn(T, __fadd2_rn(f2(1.f), make_float2(-a.x, -a.y)));
-      if (ok0 && Tn.x < kTMin) {
-        done0 = true;
-        ok0 = false;
+      float2 a = make_float2(ok0 ? fminf(kAlphaMax, exp2f(p.x)) : 0.f,
+                             ok1 ? fminf(kAlphaMax, exp2f(p.y)) : 0.f);
+      float2 Tn = __fmul2_rn(T, __ffma2_rn(a, mone, one));  // T (1 - alpha)
+      if (Tn.x < kTMin || Tn.y < kTMin) {
+        // the pixel stops before this Gaussian: it takes no part in it
+        if (Tn.x < kTMin) {
+          a.x = 0.f;
+          Tn.x = T.x;
+          thr0 = kInf;
+          ok0 = false;
+        }
+        if (Tn.y < kTMin) {
+          a.y = 0.f;
+          Tn.y = T.y;
+          thr1 = kInf;
+          ok1 = false;
+        }
+        done = thr0 == kInf && thr1 == kInf;
       }
-      if (ok1 && Tn.y < kTMin) {
-        done1 = true;
-        ok1 = false;
-      }
-      float2 w = __fmul2_rn(a, T);
-      w.x = ok0 ? w.x : 0.f;
-      w.y = ok1 ? w.y : 0.f;
-      c0 = __ffma2_rn(f2(r[E_R]), w, c0);
-      c1 = __ffma2_rn(f2(r[E_G]), w, c1);
-      c2 = __ffma2_rn(f2(r[E_BL]), w, c2);
-      const uint32_t pos1 = (uint32_t)(b * kBatch + j + 1);
-      if (ok0) {
-        T.x = Tn.x;
-        last0 = pos1;
-      }
-      if (ok1) {
-        T.y = Tn.y;
-        last1 = pos1;
-      }
+      const float2 w = __fmul2_rn(a, T);
+      c0 = __ffma2_rn(e[V_R], w, c0);
+      c1 = __ffma2_rn(e[V_G], w, c1);
+      c2 = __ffma2_rn(e[V_BL], w, c2);
+      T = Tn;
+      const uint32_t pos1 = pos0 + (uint32_t)j;
+      last0 = ok0 ? pos1 : last0;
+      last1 = ok1 ? pos1 : last1;
     }
   }
   // a batch issued but not consumed must land before the block exits
-  if (b < nb) mbar_wait_bounded(&s_bar[b & 1], (uint32_t)((b >> 1) & 1), status);
+  if (pending) mbar_wait_bounded(&s_bar, (uint32_t)(b & 1), status);
 
   const size_t hw = (size_t)geo.g.width * geo.g.height;
   float* img = image + (size_t)tp.view * 3 * hw;
@@ -406,7 +467,7 @@ __global__ void __launch_bounds__(kThreads) k_raster_bwd(
     if (!__syncthreads_and(mbar_wait_bounded(&s_bar[buf], (uint32_t)((it >> 1) & 1), status)))
       break;
     if ((int)threadIdx.x < m)
-      s_mask[threadIdx.x] = (uint8_t)prepare_record(&s_rec[buf][threadIdx.x][0], tp.x0, tp.y0);
+      s_mask[threadIdx.x] = (uint8_t)prepare_record_s(&s_rec[buf][threadIdx.x][0], tp.x0, tp.y0);
     {
       float4* z = reinterpret_cast<float4*>(&s_acc[threadIdx.x][0]);
       z[0] = z[1] = z[2] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -419,7 +480,7 @@ __global__ void __launch_bounds__(kThreads) k_raster_bwd(
       const float* r = &s_rec[buf][j][0];
       float dx;
       float2 dy;
-      const float2 p = eval_log2_alpha(r, pxc, pyc, dx, dy);
+      const float2 p = eval_log2_alpha_s(r, pxc, pyc, dx, dy);
       const bool ok0 = pos < nc0 && p.x >= kLog2AlphaMin;
       const bool ok1 = pos < nc1 && p.y >= kLog2AlphaMin;
       const uint32_t bal = __ballot_sync(0xffffffffu, ok0 || ok1);
