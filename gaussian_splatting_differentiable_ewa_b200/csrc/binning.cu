@@ -10,6 +10,13 @@
 //                  scan across blocks (decoupled look-back, one warp reading
 //                  32 predecessors per round trip) and emission of the
 //                  (key, id) pairs through shared-memory staging.
+//  k_col_count / k_emit_cols
+//                  (presort mode, up to 256 tile columns) emission already
+//                  ordered by tile column: per-block column counts from a
+//                  difference array, their scan, then lanes owning columns
+//                  append their pairs in depth order through shared-memory
+//                  buffers written out warp-wide. Keys are row << cbits |
+//                  column; the radix passes then sort by row alone.
 //  k_radix_count / k_radix_scan / k_radix_scatter
 //                  one stable least-significant-digit radix pass with digits
 //                  of up to 8 bits, reduce-then-scan: per-partition digit
@@ -40,7 +47,11 @@ constexpr int kSortThreads = 256;
 constexpr int kSortWarps = kSortThreads / 32;
 constexpr int kSortItems = 16;                        // pair passes
 constexpr int kSortTile = kSortThreads * kSortItems;  // keys per partition
-constexpr int kPresortItems = 4;                      // per-Gaussian depth passes
+constexpr int kPresortItems = 8;                      // per-Gaussian depth passes
+constexpr int kColItems = 256;     // Gaussians per column-emission block
+constexpr int kColBuf = 32;        // pairs a column stages before a warp-wide write
+constexpr int kMaxColumns = 256;   // widest tile grid the column emission takes
+constexpr int kColPitch = 33;      // buffer row: conflict-free along and across columns
 
 __device__ __forceinline__ uint32_t get_block_index(uint32_t* counter) {
   __shared__ uint32_t s_idx;
@@ -139,6 +150,214 @@ __global__ void __launch_bounds__(256) k_depth_keys(const float4* __restrict__ b
     const int view = (int)(j / n);
     keys[j] = vis ? (((uint64_t)view << 32) | (uint64_t)__float_as_uint(r2.x)) : ~0ull;
     vals[j] = (uint32_t)(j - (int64_t)view * n);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Column emission (presort mode, images up to kMaxColumns tiles wide).
+// A pair's key is row << cbits | column, row = view * tiles_y + tile row:
+// ordering by it is ordering by global tile. The emission hands out pairs
+// already ordered by column (stable in depth order), which is the first
+// least-significant-digit pass of that order; the radix passes that follow
+// sort by row only.
+
+// Rectangle of presorted item `item`; false for a culled or empty one.
+__device__ __forceinline__ bool presorted_rect(const float4* __restrict__ bins,
+                                               const uint64_t* __restrict__ pkeys,
+                                               const uint32_t* __restrict__ pvals, int n,
+                                               int64_t item, uint32_t& rx, uint32_t& ry,
+                                               uint32_t& view, uint32_t& id) {
+  const uint64_t pk = pkeys[item];
+  if (pk == ~0ull) return false;
+  view = (uint32_t)(pk >> 32);
+  id = pvals[item];
+  const float4 r2 = __ldg(&bins[(int64_t)view * n + id]);
+  rx = __float_as_uint(r2.y);  // x0 | x1 << 16
+  ry = __float_as_uint(r2.z);  // y0 | y1 << 16
+  return (rx & 0xffffu) <= (rx >> 16) && (ry & 0xffffu) <= (ry >> 16);
+}
+
+// (1) pairs per tile column of each block of kColItems presorted Gaussians:
+// a difference array over columns weighted by the rectangle's height, then a
+// prefix over the columns. Also adds the block's pairs to the 64-bit total.
+__global__ void __launch_bounds__(kColItems) k_col_count(
+    const float4* __restrict__ bins, const uint64_t* __restrict__ pkeys,
+    const uint32_t* __restrict__ pvals, int n, int n_views, Grid g, uint32_t* __restrict__ counts,
+    int64_t stride, unsigned long long* __restrict__ pair_total, uint4* __restrict__ crect) {
+  __shared__ int s_diff[kMaxColumns + 1];
+  __shared__ uint32_t s_warp[9];
+  const int64_t items = (int64_t)n * n_views;
+  for (int c = threadIdx.x; c <= kMaxColumns; c += kColItems) s_diff[c] = 0;
+  __syncthreads();
+  const int64_t item = (int64_t)blockIdx.x * kColItems + threadIdx.x;
+  uint32_t rx, ry, view, id;
+  uint64_t mine = 0;
+  if (item < items) {
+    if (presorted_rect(bins, pkeys, pvals, n, item, rx, ry, view, id)) {
+      const int h = (int)((ry >> 16) - (ry & 0xffffu) + 1);
+      atomicAdd(&s_diff[rx & 0xffffu], h);
+      atomicAdd(&s_diff[(rx >> 16) + 1], -h);
+      mine = (uint64_t)h * ((rx >> 16) - (rx & 0xffffu) + 1);
+      crect[item] = make_uint4(rx, ry, view * (uint32_t)g.tiles_y, id);
+    } else {
+      crect[item] = make_uint4(1u, 0u, 0u, 0u);  // empty: x0 > x1
+    }
+  }
+  // the block's pair total: warp sums, then one 64-bit atomic per block
+  __shared__ unsigned long long s_tot[kColItems / 32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
+  if ((threadIdx.x & 31) == 0) s_tot[threadIdx.x >> 5] = mine;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long b = 0;
+#pragma unroll
+    for (int w = 0; w < kColItems / 32; ++w) b += s_tot[w];
+    if (b) atomicAdd(pair_total, b);
+  }
+  const int t = threadIdx.x;
+  const int d = t < g.tiles_x ? s_diff[t] : 0;
+  uint32_t tot;
+  const uint32_t excl = block_exclusive_scan_256((uint32_t)d, s_warp, tot);
+  if (t < g.tiles_x) counts[(int64_t)t * stride + blockIdx.x] = excl + (uint32_t)d;
+}
+
+// (3) emission. Block (b, w) -- one warp -- takes Gaussian block b's pairs in
+// tile columns 32w .. 32w + 31; lane l owns column 32w + l (its buffer and
+// its next global position). The warp compacts the block's Gaussians to those
+// whose rectangle reaches its columns (depth order kept) and walks them,
+// writing a rectangle's pairs at once, one lane per (row, column) pair, each
+// into its column's buffer in shared memory after the pairs already there. A
+// column whose buffer cannot take the rectangle's rows is first written out
+// by the whole warp to the column's next global positions (coalesced), so a
+// column's pairs leave in depth order. One warp per block lets the scheduler
+// balance column groups of very different load (the image centre against its
+// edges). offsets: [column][block] exclusive scans over blocks; totals: pairs
+// per column; crect: the presorted rectangles (x0 | x1 << 16, y0 | y1 << 16,
+// first row of the view, Gaussian index).
+
+// Warp-wide write of the first `count` (<= 32) pairs of buffer column `bc`
+// to global positions base, base + 1, ...
+__device__ __forceinline__ void flush_column(uint32_t* __restrict__ keys_out,
+                                             uint32_t* __restrict__ ids_out, int64_t capacity,
+                                             const uint32_t* s_bk, const uint32_t* s_bi, int bc,
+                                             uint32_t base, uint32_t count,
+                                             uint32_t* __restrict__ status) {
+  const uint32_t lane = threadIdx.x & 31;
+  if (lane < count) {
+    const uint32_t pos = base + lane;
+    if ((int64_t)pos < capacity) {
+      keys_out[pos] = s_bk[lane * kColPitch + bc];
+      ids_out[pos] = s_bi[lane * kColPitch + bc];
+    } else {
+      atomicOr(status, kStatusBounds);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(32) k_emit_cols(
+    const uint4* __restrict__ crect, int64_t items, Grid g, int cbits,
+    const uint32_t* __restrict__ offsets, int64_t stride, const uint32_t* __restrict__ totals,
+    const unsigned long long* __restrict__ pair_total, uint32_t* __restrict__ keys_out,
+    uint32_t* __restrict__ ids_out, int64_t capacity, int64_t* __restrict__ n_pairs,
+    uint32_t* __restrict__ status) {
+  __shared__ uint32_t s_bk[kColBuf * kColPitch], s_bi[kColBuf * kColPitch];
+  __shared__ uint4 s_rect[kColItems];  // this warp's rectangles, compacted
+  const int lane = threadIdx.x;
+  const unsigned long long total = *pair_total;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && lane == 0) {
+    *n_pairs = (int64_t)total;
+    if ((int64_t)total > capacity) atomicOr(status, kStatusCapacity);
+  }
+  if ((int64_t)total > capacity) return;  // nothing is emitted
+  const uint32_t wlo = 32u * blockIdx.y, col = wlo + (uint32_t)lane;
+  // first position of this block's pairs in column col: pairs of lower
+  // columns plus column col's pairs from earlier blocks
+  uint32_t below = 0;
+  for (uint32_t c = (uint32_t)lane; c < wlo; c += 32) below += totals[c];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) below += __shfl_xor_sync(0xffffffffu, below, o);
+  uint32_t tot_c = col < (uint32_t)g.tiles_x ? totals[col] : 0u;
+  uint32_t incl = tot_c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  uint32_t gofs = below + incl - tot_c;
+  if (col < (uint32_t)g.tiles_x) gofs += offsets[(int64_t)col * stride + blockIdx.x];
+  // compact the block's rectangles that reach columns wlo .. wlo + 31
+  const uint32_t lt = lanemask_lt();
+  int cnt = 0;
+  const int64_t first = (int64_t)blockIdx.x * kColItems;
+#pragma unroll 2
+  for (int c = 0; c < kColItems / 32; ++c) {
+    const int64_t item = first + c * 32 + lane;
+    uint4 r = make_uint4(1u, 0u, 0u, 0u);
+    if (item < items) r = crect[item];
+    const uint32_t x0 = r.x & 0xffffu, x1 = r.x >> 16;
+    const bool hit = x0 <= x1 && x1 >= wlo && x0 <= wlo + 31u;
+    const uint32_t bal = __ballot_sync(0xffffffffu, hit);
+    if (hit) s_rect[cnt + __popc(bal & lt)] = r;
+    cnt += __popc(bal);
+  }
+  __syncwarp();
+  uint32_t fill = 0;
+  for (int k = 0; k < cnt; ++k) {
+    const uint4 r = s_rect[k];
+    // this warp's columns of the rectangle
+    const uint32_t cx0 = max(r.x & 0xffffu, wlo);
+    const uint32_t cx1 = min(r.x >> 16, wlo + 31u);
+    const uint32_t wp = cx1 - cx0 + 1;
+    const float inv_wp = 1.f / (float)wp;
+    const bool owner = col >= cx0 && col <= cx1;
+    const uint32_t y0 = r.y & 0xffffu, h = (r.y >> 16) - y0 + 1;
+    const uint32_t row0 = r.z + y0;
+    for (uint32_t r0 = 0; r0 < h; r0 += kColBuf) {  // row chunks, uniform across the warp
+      const uint32_t hc = min(h - r0, (uint32_t)kColBuf);
+      // make room: columns that cannot take hc more pairs are written out
+      uint32_t need = __ballot_sync(0xffffffffu, owner && fill + hc > kColBuf);
+      if (need) {
+        __syncwarp();
+        do {
+          const int L = __ffs(need) - 1;
+          need &= need - 1;
+          flush_column(keys_out, ids_out, capacity, s_bk, s_bi, L,
+                       __shfl_sync(0xffffffffu, gofs, L), __shfl_sync(0xffffffffu, fill, L),
+                       status);
+          if (lane == L) {
+            gofs += fill;
+            fill = 0;
+          }
+        } while (need);
+        __syncwarp();
+      }
+      // the chunk's wp * hc pairs, 32 at a time: pair p is row p / wp, column
+      // cx0 + p % wp, written after that column's fill pairs
+      const uint32_t np = wp * hc;
+      for (uint32_t p0 = 0; p0 < np; p0 += 32) {
+        const uint32_t p = p0 + (uint32_t)lane;
+        const uint32_t rr = min((uint32_t)(((float)p + 0.5f) * inv_wp), hc - 1);
+        const uint32_t cc = min(p - rr * wp, wp - 1);
+        const uint32_t bc = cx0 + cc - wlo;  // buffer column = owning lane
+        const uint32_t f = __shfl_sync(0xffffffffu, fill, (int)bc);
+        if (p < np) {
+          const int at = (int)(f + rr) * kColPitch + (int)bc;
+          s_bk[at] = ((row0 + r0 + rr) << cbits) | (wlo + bc);
+          s_bi[at] = r.w;
+        }
+      }
+      if (owner) fill += hc;
+    }
+  }
+  // what is left in each column's buffer
+  __syncwarp();
+  uint32_t left = __ballot_sync(0xffffffffu, fill > 0);
+  while (left) {
+    const int L = __ffs(left) - 1;
+    left &= left - 1;
+    flush_column(keys_out, ids_out, capacity, s_bk, s_bi, L, __shfl_sync(0xffffffffu, gofs, L),
+                 __shfl_sync(0xffffffffu, fill, L), status);
   }
 }
 
@@ -522,10 +741,12 @@ __device__ __forceinline__ uint32_t tile_of(K k) {
 
 // [start, end) of every tile present in the sorted keys. Each thread takes 8
 // consecutive keys with vector loads (a full chunk) and compares neighbours.
+// cbits > 0: 32-bit keys are row << cbits | column (column emission), decoded
+// to row * tiles_x + column; the decoding is monotone, so runs stay runs.
 template <typename K>
 __global__ void k_ranges(const K* __restrict__ keys, const int64_t* __restrict__ n_ptr,
-                         int64_t capacity, int64_t n_tiles, int64_t* __restrict__ ranges,
-                         uint32_t* __restrict__ status) {
+                         int64_t capacity, int64_t n_tiles, int cbits, uint32_t tiles_x,
+                         int64_t* __restrict__ ranges, uint32_t* __restrict__ status) {
   const int64_t n = *n_ptr;
   if (n > capacity) return;
   constexpr int C = 8;
@@ -554,6 +775,12 @@ __global__ void k_ranges(const K* __restrict__ keys, const int64_t* __restrict__
       for (int k = 0; k < C; ++k) t[k] = i0 + k < n ? tile_of(keys[i0 + k]) : 0u;
     }
     uint32_t prev = i0 > 0 ? tile_of(keys[i0 - 1]) : 0xffffffffu;
+    if (cbits > 0) {
+      const uint32_t cm = (1u << cbits) - 1u;
+#pragma unroll
+      for (int k = 0; k < C; ++k) t[k] = (t[k] >> cbits) * tiles_x + (t[k] & cm);
+      if (i0 > 0) prev = (prev >> cbits) * tiles_x + (prev & cm);
+    }
 #pragma unroll
     for (int k = 0; k < C; ++k) {
       const int64_t i = i0 + k;
@@ -661,6 +888,8 @@ int64_t presort_partitions(int64_t items) {
   return (items + SortTile<kPresortItems>::kItems - 1) / SortTile<kPresortItems>::kItems;
 }
 int64_t emit_blocks(int64_t items) { return (items + kEmitItems - 1) / kEmitItems; }
+int64_t column_blocks(int64_t items) { return (items + kColItems - 1) / kColItems; }
+bool column_emission(const Grid& g) { return g.tiles_x <= kMaxColumns; }
 
 cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
   cudaError_t e;
@@ -684,6 +913,32 @@ cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
                                                   stream);
     if (e != cudaSuccess) return e;
     const int fin = a.presort.passes & 1;
+    if (a.column_emit) {
+      // 2) pairs per column and block, their scan, emission by column
+      const int64_t cb = column_blocks(n_items);
+      k_col_count<<<(unsigned)cb, kColItems, 0, stream>>>(bins4, a.pkeys[fin], a.pvals[fin], a.n,
+                                                          a.n_views, a.grid, a.counts,
+                                                          a.counts_stride, a.pair_total, a.crect);
+      k_radix_scan<<<(unsigned)a.grid.tiles_x, 256, 0, stream>>>(
+          a.counts, a.counts_stride, a.n_items_dev, n_items, kColItems, a.totals);
+      const dim3 grid((unsigned)cb, (unsigned)((a.grid.tiles_x + 31) / 32));
+      k_emit_cols<<<grid, 32, 0, stream>>>(
+          a.crect, n_items, a.grid, a.cbits, a.counts, a.counts_stride, a.totals, a.pair_total,
+          reinterpret_cast<uint32_t*>(a.keys[a.emit_buf]), a.vals[a.emit_buf], a.capacity,
+          a.n_pairs, a.status);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      // 3) stable sort by row
+      e = run_radix_passes<uint32_t, kSortItems>(
+          reinterpret_cast<uint32_t*>(a.keys[a.emit_buf]), a.vals[a.emit_buf],
+          reinterpret_cast<uint32_t*>(a.keys[a.emit_buf ^ 1]), a.vals[a.emit_buf ^ 1], a.n_pairs,
+          a.capacity, a.capacity, a.pairs, a.counts, a.counts_stride, a.totals, a.status, stream);
+      if (e != cudaSuccess) return e;
+      const int out = a.emit_buf ^ (a.pairs.passes & 1);
+      k_ranges<uint32_t><<<sms * 4, 256, 0, stream>>>(
+          reinterpret_cast<uint32_t*>(a.keys[out]), a.n_pairs, a.capacity, a.n_tiles, a.cbits,
+          (uint32_t)a.grid.tiles_x, a.ranges, a.status);
+      return cudaGetLastError();
+    }
     // 2) emission in depth order, 32-bit tile keys
     k_emit<1, uint32_t><<<(unsigned)eb, kEmitThreads, 0, stream>>>(
         bins4, a.pkeys[fin], a.pvals[fin], a.n, a.n_views, a.grid,
@@ -698,8 +953,8 @@ cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     const int out = a.emit_buf ^ (a.pairs.passes & 1);
     k_ranges<uint32_t><<<sms * 4, 256, 0, stream>>>(reinterpret_cast<uint32_t*>(a.keys[out]),
-                                                   a.n_pairs, a.capacity, a.n_tiles, a.ranges,
-                                                   a.status);
+                                                   a.n_pairs, a.capacity, a.n_tiles, 0, 0u,
+                                                   a.ranges, a.status);
     return cudaGetLastError();
   }
   // full 64-bit keys
@@ -714,7 +969,7 @@ cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const int out = a.emit_buf ^ (a.pairs.passes & 1);
   k_ranges<uint64_t><<<sms * 4, 256, 0, stream>>>(a.keys[out], a.n_pairs, a.capacity, a.n_tiles,
-                                                  a.ranges, a.status);
+                                                  0, 0u, a.ranges, a.status);
   return cudaGetLastError();
 }
 

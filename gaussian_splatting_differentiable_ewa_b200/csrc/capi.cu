@@ -19,6 +19,7 @@ constexpr size_t kControlBytes = 4096;  // status word, counters, device scalars
 constexpr size_t kStatusOffset = 0;
 constexpr size_t kCountersOffset = 64;   // 16 x uint32
 constexpr size_t kNItemsOffset = 256;    // int64
+constexpr size_t kPairTotalOffset = 264; // uint64
 constexpr size_t kHistBytes = 256 * sizeof(uint32_t);  // digit totals of the current pass
 constexpr int64_t kMaxPairCapacity = GS_MAX_PAIR_CAPACITY;
 
@@ -34,10 +35,13 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 struct Layout {
   RadixPlan pairs, presort;
+  bool column_emit = false;
+  int cbits = 0;
   int key_bytes = 8;
   int64_t counts_stride = 0;
   size_t off_hist = 0, off_emit_lb = 0, off_counts = 0, off_keys0 = 0, off_keys1 = 0,
-         off_vals1 = 0, off_pkeys0 = 0, off_pkeys1 = 0, off_pvals0 = 0, off_pvals1 = 0;
+         off_vals1 = 0, off_pkeys0 = 0, off_pkeys1 = 0, off_pvals0 = 0, off_pvals1 = 0,
+         off_crect = 0;
   size_t total = 0;
 };
 
@@ -68,13 +72,24 @@ bool make_layout(int64_t n, int32_t n_views, const gs_camera* cams, int64_t capa
     L.pairs = make_radix_plan(32 + tile_bits, false);
   } else {
     L.key_bytes = 4;
-    L.pairs = make_radix_plan(tile_bits, true);
     L.presort = make_radix_plan(32 + bits_for((uint64_t)n_views - 1), false);
+    L.column_emit = column_emission(g);
+    if (L.column_emit) {
+      // keys row << cbits | column; the radix passes sort the row bits
+      L.cbits = bits_for((uint64_t)g.tiles_x - 1);
+      if (L.cbits == 0) L.cbits = 1;
+      L.pairs = make_radix_plan(bits_for((uint64_t)g.tiles_y * n_views - 1), true);
+      for (int i = 0; i < L.pairs.passes; ++i) L.pairs.shift[i] += L.cbits;
+    } else {
+      L.pairs = make_radix_plan(tile_bits, true);
+    }
   }
   int64_t parts = pair_partitions(capacity);
   if (mode == GS_SORT_PRESORT) {
     const int64_t p2 = presort_partitions(items);
     if (p2 > parts) parts = p2;
+    const int64_t p3 = column_blocks(items);
+    if (p3 > parts) parts = p3;
   }
   L.counts_stride = parts > 0 ? (parts + 3) / 4 * 4 : 4;
   size_t off = kControlBytes;
@@ -89,6 +104,9 @@ bool make_layout(int64_t n, int32_t n_views, const gs_camera* cams, int64_t capa
     L.off_pkeys1 = off; off = align_up(off + (size_t)items * 8);
     L.off_pvals0 = off; off = align_up(off + (size_t)items * 4);
     L.off_pvals1 = off; off = align_up(off + (size_t)items * 4);
+    if (L.column_emit) {
+      L.off_crect = off; off = align_up(off + (size_t)items * 16);
+    }
   }
   L.total = off;
   return true;
@@ -165,6 +183,7 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
   const int64_t items = n * n_views;
 
   if (cudaMemsetAsync(w + kCountersOffset, 0, 16 * sizeof(uint32_t), st) != cudaSuccess ||
+      cudaMemsetAsync(w + kPairTotalOffset, 0, sizeof(uint64_t), st) != cudaSuccess ||
       cudaMemsetAsync(w + L.off_emit_lb, 0, (size_t)emit_blocks(items) * 8, st) != cudaSuccess ||
       cudaMemsetAsync(out->ranges, 0, (size_t)tiles * 2 * sizeof(int64_t), st) != cudaSuccess)
     return GS_ERR_CUDA;
@@ -177,6 +196,8 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
   a.mode = sort_mode;
   a.grid = g;
   a.capacity = out->pair_capacity;
+  a.column_emit = L.column_emit;
+  a.cbits = L.cbits;
   a.pairs = L.pairs;
   a.presort = L.presort;
   a.emit_buf = L.pairs.passes & 1;
@@ -198,6 +219,8 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
   a.status = reinterpret_cast<uint32_t*>(w + kStatusOffset);
   a.n_pairs = out->n_pairs;
   a.n_items_dev = reinterpret_cast<int64_t*>(w + kNItemsOffset);
+  a.pair_total = reinterpret_cast<unsigned long long*>(w + kPairTotalOffset);
+  if (L.column_emit) a.crect = reinterpret_cast<uint4*>(w + L.off_crect);
   a.ranges = out->ranges;
   a.n_tiles = tiles;
   return cuda_status(launch_bin_sort(a, st));

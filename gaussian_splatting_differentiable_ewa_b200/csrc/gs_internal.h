@@ -28,6 +28,8 @@ struct BinSortArgs {
   int mode;
   Grid grid;
   int64_t capacity;
+  bool column_emit;    // presort mode: emission ordered by tile column
+  int cbits;           // column bits of a column-emission key (row << cbits | column)
   RadixPlan pairs;     // radix passes over the pair keys
   RadixPlan presort;   // radix passes over the per-Gaussian depth keys
   int emit_buf;        // which key/value buffer the emission writes
@@ -43,6 +45,8 @@ struct BinSortArgs {
   uint32_t* status;
   int64_t* n_pairs;
   int64_t* n_items_dev;
+  unsigned long long* pair_total;  // column emission: exact pair count
+  uint4* crect;                      // column emission: presorted rectangles [n_views * n]
   int64_t* ranges;
   int64_t n_tiles;     // n_views * tiles per view
 };
@@ -71,6 +75,8 @@ cudaError_t launch_adam(const gs_adam_group* groups, int n_groups, float b1, flo
 
 int64_t pair_partitions(int64_t items);     // radix partitions over pair keys
 int64_t presort_partitions(int64_t items);  // radix partitions over depth keys
+int64_t column_blocks(int64_t items);       // column-emission blocks
+bool column_emission(const Grid& g);        // presort mode emits by column on this grid
 int64_t emit_blocks(int64_t items);
 
 }  // namespace gsb

@@ -60,34 +60,32 @@ __device__ __forceinline__ void sh_basis(float x, float y, float z, float* Y) {
   }
 }
 
-// Partial derivatives of the polynomials above with respect to x, y, z taken
-// as independent variables (the caller projects onto the sphere's tangent
-// plane, which removes the difference between equivalent forms on the sphere).
+// sum_k w_k grad Y_k: the gradient of the polynomials above with respect to
+// x, y, z taken as independent variables, weighted by w (the caller projects
+// onto the sphere's tangent plane, which removes the difference between
+// equivalent forms on the sphere). Accumulates into (gx, gy, gz).
 template <int DEG>
-__device__ __forceinline__ void sh_basis_grad(float x, float y, float z, float* gx, float* gy,
-                                              float* gz) {
-  gx[0] = gy[0] = gz[0] = 0.f;
+__device__ __forceinline__ void sh_dir_grad(float x, float y, float z, const float* w, float& gx,
+                                            float& gy, float& gz) {
   if (DEG >= 1) {
-    gx[1] = 0.f;    gy[1] = -kY1;  gz[1] = 0.f;
-    gx[2] = 0.f;    gy[2] = 0.f;   gz[2] = kY1;
-    gx[3] = -kY1;   gy[3] = 0.f;   gz[3] = 0.f;
+    gy -= kY1 * w[1];
+    gz += kY1 * w[2];
+    gx -= kY1 * w[3];
   }
   if (DEG >= 2) {
-    gx[4] = kY2a * y;          gy[4] = kY2a * x;          gz[4] = 0.f;
-    gx[5] = 0.f;               gy[5] = -kY2a * z;         gz[5] = -kY2a * y;
-    gx[6] = 0.f;               gy[6] = 0.f;               gz[6] = 6.f * kY2b * z;
-    gx[7] = -kY2a * z;         gy[7] = 0.f;               gz[7] = -kY2a * x;
-    gx[8] = 2.f * kY2c * x;    gy[8] = -2.f * kY2c * y;   gz[8] = 0.f;
-    if (DEG >= 3) {
-      float xx = x * x, yy = y * y, zz = z * z;
-      gx[9] = -6.f * kY3a * x * y;          gy[9] = -3.f * kY3a * (xx - yy);    gz[9] = 0.f;
-      gx[10] = kY3b * y * z;                gy[10] = kY3b * x * z;              gz[10] = kY3b * x * y;
-      gx[11] = 0.f;                         gy[11] = -kY3c * (5.f * zz - 1.f);  gz[11] = -10.f * kY3c * y * z;
-      gx[12] = 0.f;                         gy[12] = 0.f;                       gz[12] = kY3d * (15.f * zz - 3.f);
-      gx[13] = -kY3c * (5.f * zz - 1.f);    gy[13] = 0.f;                       gz[13] = -10.f * kY3c * x * z;
-      gx[14] = 2.f * kY3e * x * z;          gy[14] = -2.f * kY3e * y * z;       gz[14] = kY3e * (xx - yy);
-      gx[15] = -3.f * kY3a * (xx - yy);     gy[15] = 6.f * kY3a * x * y;        gz[15] = 0.f;
-    }
+    gx += kY2a * (y * w[4] - z * w[7]) + 2.f * kY2c * x * w[8];
+    gy += kY2a * (x * w[4] - z * w[5]) - 2.f * kY2c * y * w[8];
+    gz += 6.f * kY2b * z * w[6] - kY2a * (y * w[5] + x * w[7]);
+  }
+  if (DEG >= 3) {
+    const float xx = x * x, yy = y * y, zz = z * z;
+    const float p5 = 5.f * zz - 1.f;
+    gx += -6.f * kY3a * x * y * w[9] + kY3b * y * z * w[10] - kY3c * p5 * w[13] +
+          2.f * kY3e * x * z * w[14] - 3.f * kY3a * (xx - yy) * w[15];
+    gy += -3.f * kY3a * (xx - yy) * w[9] + kY3b * x * z * w[10] - kY3c * p5 * w[11] -
+          2.f * kY3e * y * z * w[14] + 6.f * kY3a * x * y * w[15];
+    gz += kY3b * x * y * w[10] - 10.f * kY3c * y * z * w[11] + kY3d * (15.f * zz - 3.f) * w[12] -
+          10.f * kY3c * x * z * w[13] + kY3e * (xx - yy) * w[14];
   }
 }
 
@@ -170,7 +168,7 @@ __device__ __forceinline__ void sh_colour_global(const float* __restrict__ shi, 
 }
 
 template <int DEG>
-__global__ void __launch_bounds__(kProjFwdThreads) k_project(const float4* __restrict__ means,
+__global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __restrict__ means,
                                                           const float4* __restrict__ log_scales,
                                                           const float4* __restrict__ quats,
                                                           const float* __restrict__ logit,
@@ -317,9 +315,10 @@ __global__ void __launch_bounds__(kProjFwdThreads) k_project(const float4* __res
 // the Gaussian was visible (radius > 0).
 // SH coefficients come in, and SH gradients go out, through shared memory
 // (coefficient-major, coalesced global traffic); the SH gradients are summed
-// over views in shared memory rather than in registers.
-template <int DEG>
-__global__ void __launch_bounds__(kProjThreads) k_project_bwd(
+// over views in shared memory rather than in registers. With ALIAS (one view)
+// the gradients overwrite the staged coefficients slot by slot.
+template <int DEG, bool ALIAS>
+__global__ void __launch_bounds__(kProjThreads, 6) k_project_bwd(
     const float4* __restrict__ means, const float4* __restrict__ log_scales,
     const float4* __restrict__ quats, const float* __restrict__ logit,
     const float* __restrict__ sh, const float4* __restrict__ grad2d,
@@ -329,13 +328,15 @@ __global__ void __launch_bounds__(kProjThreads) k_project_bwd(
   constexpr int K = (DEG + 1) * (DEG + 1);
   constexpr int K3 = K * 3;
   extern __shared__ float s_pb[];
-  float* s_coef = s_pb;                    // [K3][kShStride]
-  float* s_dsh = s_pb + K3 * kShStride;    // [K3][kShStride]
+  float* s_coef = s_pb;                                 // [K3][kShStride]
+  float* s_dsh = ALIAS ? s_pb : s_pb + K3 * kShStride;  // [K3][kShStride]
   const int64_t i0 = (int64_t)blockIdx.x * kProjThreads;
   const int cnt = (int)min((int64_t)kProjThreads, (int64_t)n - i0);
   stage_sh<K3>(sh, i0, cnt, s_coef);
+  if (!ALIAS) {
 #pragma unroll
-  for (int c = 0; c < K3; ++c) s_dsh[c * kShStride + threadIdx.x] = 0.f;
+    for (int c = 0; c < K3; ++c) s_dsh[c * kShStride + threadIdx.x] = 0.f;
+  }
   __syncthreads();
   const int i = (int)i0 + threadIdx.x;
   if (i < n) {
@@ -363,8 +364,10 @@ __global__ void __launch_bounds__(kProjThreads) k_project_bwd(
   const float* cf_t = s_coef + threadIdx.x;
   float* dsh_t = s_dsh + threadIdx.x;
 
+  bool touched = false;
   for (int v = 0; v < n_views; ++v) {
     if (radii[(size_t)v * n + i] <= 0) continue;
+    touched = true;
     const float4* G4 = grad2d + ((size_t)v * n + i) * 3;
     const float4 ga = G4[0], gb = G4[1], gc = G4[2];
     const float G[9] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w, gc.x};
@@ -437,31 +440,40 @@ __global__ void __launch_bounds__(kProjThreads) k_project_bwd(
     const float wx = m.x - c.campos[0], wy = m.y - c.campos[1], wz = m.z - c.campos[2];
     const float winv = rsqrtf(wx * wx + wy * wy + wz * wz);
     const float dx = wx * winv, dy = wy * winv, dz = wz * winv;
-    float Y[16], gx[16], gy[16], gz[16];
+    float Y[16], wk[16];
     sh_basis<DEG>(dx, dy, dz, Y);
-    sh_basis_grad<DEG>(dx, dy, dz, gx, gy, gz);
-    float gdx = 0.f, gdy = 0.f, gdz = 0.f;
+#pragma unroll
+    for (int k = 0; k < K; ++k) wk[k] = 0.f;
 #pragma unroll
     for (int ch = 0; ch < 3; ++ch) {
       float raw = 0.5f;
 #pragma unroll
       for (int k = 0; k < K; ++k) raw = fmaf(Y[k], cf_t[(k * 3 + ch) * kShStride], raw);
-      if (!(raw > 0.f)) continue;
-      const float gcol = G[G_R + ch];
+      // a clamped channel passes no gradient; with one view the gradient slot
+      // is the coefficient's own (read above), written once
+      const float gcol = raw > 0.f ? G[G_R + ch] : 0.f;
 #pragma unroll
       for (int k = 0; k < K; ++k) {
         const float cf = cf_t[(k * 3 + ch) * kShStride];
-        dsh_t[(k * 3 + ch) * kShStride] += Y[k] * gcol;
-        gdx += gcol * cf * gx[k];
-        gdy += gcol * cf * gy[k];
-        gdz += gcol * cf * gz[k];
+        if (ALIAS)
+          dsh_t[(k * 3 + ch) * kShStride] = Y[k] * gcol;
+        else
+          dsh_t[(k * 3 + ch) * kShStride] += Y[k] * gcol;
+        wk[k] = fmaf(gcol, cf, wk[k]);
       }
     }
+    float gdx = 0.f, gdy = 0.f, gdz = 0.f;
+    sh_dir_grad<DEG>(dx, dy, dz, wk, gdx, gdy, gdz);
     // through d = w / |w|: (I - d d^T) / |w|
     const float dd = gdx * dx + gdy * dy + gdz * dz;
     dmu[0] += (gdx - dx * dd) * winv;
     dmu[1] += (gdy - dy * dd) * winv;
     dmu[2] += (gdz - dz * dd) * winv;
+  }
+
+  if (ALIAS && !touched) {  // no view wrote this Gaussian's slots
+#pragma unroll
+    for (int c = 0; c < K3; ++c) dsh_t[c * kShStride] = 0.f;
   }
 
   // M = R diag(s): dL/ds_k = sum_j dM_jk R_jk, dL/dR_jk = dM_jk s_k
@@ -534,7 +546,8 @@ cudaError_t launch_project_bwd(const gs_params& p, const CamSet& cams, int n_vie
   const int threads = kProjThreads;
   const int blocks = (n + threads - 1) / threads;
   const int K3 = 3 * (p.sh_degree + 1) * (p.sh_degree + 1);
-  const size_t smem = (size_t)2 * K3 * kShStride * sizeof(float);
+  const bool alias = n_views == 1;
+  const size_t smem = (size_t)(alias ? 1 : 2) * K3 * kShStride * sizeof(float);
   auto m = reinterpret_cast<const float4*>(p.means);
   auto s = reinterpret_cast<const float4*>(p.log_scales);
   auto q = reinterpret_cast<const float4*>(p.quats);
@@ -542,10 +555,18 @@ cudaError_t launch_project_bwd(const gs_params& p, const CamSet& cams, int n_vie
   auto gm = reinterpret_cast<float4*>(g.means);
   auto gs = reinterpret_cast<float4*>(g.log_scales);
   auto gq = reinterpret_cast<float4*>(g.quats);
-#define GS_PBWD(D)                                                                            \
-  cudaFuncSetAttribute(k_project_bwd<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
-  k_project_bwd<D><<<blocks, threads, smem, stream>>>(m, s, q, p.opacity_logit, p.sh, g2, radii, n, \
-                                                      n_views, cams, gm, gs, gq, g.opacity_logit, g.sh)
+#define GS_PBWD1(D, AL)                                                                      \
+  cudaFuncSetAttribute(k_project_bwd<D, AL>, cudaFuncAttributeMaxDynamicSharedMemorySize,      \
+                       (int)smem);                                                              \
+  k_project_bwd<D, AL><<<blocks, threads, smem, stream>>>(m, s, q, p.opacity_logit, p.sh, g2,   \
+                                                          radii, n, n_views, cams, gm, gs, gq,  \
+                                                          g.opacity_logit, g.sh)
+#define GS_PBWD(D)            \
+  if (alias) {                \
+    GS_PBWD1(D, true);        \
+  } else {                    \
+    GS_PBWD1(D, false);       \
+  }
   switch (p.sh_degree) {
     case 0: GS_PBWD(0); break;
     case 1: GS_PBWD(1); break;
@@ -553,6 +574,7 @@ cudaError_t launch_project_bwd(const gs_params& p, const CamSet& cams, int n_vie
     default: GS_PBWD(3); break;
   }
 #undef GS_PBWD
+#undef GS_PBWD1
   return cudaGetLastError();
 }
 
