@@ -10,6 +10,14 @@
 //                  scan across blocks (decoupled look-back, one warp reading
 //                  32 predecessors per round trip) and emission of the
 //                  (key, id) pairs through shared-memory staging.
+//  k_tile_count / k_tile_base / k_emit_tiles
+//                  (presort mode, tile grids up to ~40k tiles) every pair
+//                  straight to its final position: per (Gaussian block,
+//                  tile) counts from a 2-D difference array, their scans over
+//                  blocks and over tiles (which are also the ranges), then
+//                  one warp per (block, 32 x 16 tile region) streams the
+//                  block's rectangles in depth order and writes each pair at
+//                  its tile's next position.
 //  k_col_count / k_emit_cols
 //                  (presort mode, up to 256 tile columns) emission already
 //                  ordered by tile column: per-block column counts from a
@@ -52,6 +60,9 @@ constexpr int kColItems = 256;     // Gaussians per column-emission block
 constexpr int kColBuf = 32;        // pairs a column stages before a warp-wide write
 constexpr int kMaxColumns = 256;   // widest tile grid the column emission takes
 constexpr int kColPitch = 33;      // buffer row: conflict-free along and across columns
+constexpr int kRegionCols = 32;    // tile-emission region: kRegionCols x kRegionRows tiles
+constexpr int kRegionRows = 16;
+constexpr int kTileDiffBytes = 160 * 1024;  // largest tile-count difference array
 
 __device__ __forceinline__ uint32_t get_block_index(uint32_t* counter) {
   __shared__ uint32_t s_idx;
@@ -139,7 +150,11 @@ struct KeyTraits<uint32_t> {
 __global__ void __launch_bounds__(256) k_depth_keys(const float4* __restrict__ bins, int n,
                                                    int n_views, uint64_t* __restrict__ keys,
                                                    uint32_t* __restrict__ vals,
-                                                   int64_t* __restrict__ n_items_out) {
+                                                   int64_t* __restrict__ n_items_out,
+                                                   uint32_t* __restrict__ n_visible) {
+  __shared__ uint32_t s_vis[GS_MAX_VIEWS];
+  if (threadIdx.x < GS_MAX_VIEWS) s_vis[threadIdx.x] = 0u;
+  __syncthreads();
   if (blockIdx.x == 0 && threadIdx.x == 0) *n_items_out = (int64_t)n * n_views;
   const int64_t total = (int64_t)n * n_views;
   for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < total;
@@ -150,16 +165,22 @@ __global__ void __launch_bounds__(256) k_depth_keys(const float4* __restrict__ b
     const int view = (int)(j / n);
     keys[j] = vis ? (((uint64_t)view << 32) | (uint64_t)__float_as_uint(r2.x)) : ~0ull;
     vals[j] = (uint32_t)(j - (int64_t)view * n);
+    if (vis) atomicAdd(&s_vis[view], 1u);
   }
+  __syncthreads();
+  if (threadIdx.x < n_views && s_vis[threadIdx.x]) atomicAdd(&n_visible[threadIdx.x], s_vis[threadIdx.x]);
 }
 
 // ---------------------------------------------------------------------------
-// Column emission (presort mode, images up to kMaxColumns tiles wide).
-// A pair's key is row << cbits | column, row = view * tiles_y + tile row:
-// ordering by it is ordering by global tile. The emission hands out pairs
-// already ordered by column (stable in depth order), which is the first
-// least-significant-digit pass of that order; the radix passes that follow
-// sort by row only.
+// Tile emission (presort mode, tile grids whose difference array fits in
+// shared memory). Every pair goes straight to its final position:
+// view v's presorted Gaussians are cut into blocks of `gsize`; for block b and
+// tile t, cnt(t, b) = number of the block's rectangles covering t. A scan
+// over b (per tile) and one over t give pair (t, Gaussian g of block b) the
+// position base(t) + sum_{b' < b} cnt(t, b') + (rank of g among the block's
+// Gaussians covering t), which is depth order within the tile -- the order
+// of the stable (tile, depth) sort -- and the ranges are the scans
+// themselves. No pair keys, no sort of the pairs.
 
 // Rectangle of presorted item `item`; false for a culled or empty one.
 __device__ __forceinline__ bool presorted_rect(const float4* __restrict__ bins,
@@ -176,6 +197,242 @@ __device__ __forceinline__ bool presorted_rect(const float4* __restrict__ bins,
   ry = __float_as_uint(r2.z);  // y0 | y1 << 16
   return (rx & 0xffffu) <= (rx >> 16) && (ry & 0xffffu) <= (ry >> 16);
 }
+
+// Start of view v's visible Gaussians in the presorted order (sorted by
+// (view, depth) with culled ones last) and their number.
+__device__ __forceinline__ void view_span(const uint32_t* __restrict__ n_visible, int v,
+                                          int64_t& start, int64_t& count) {
+  int64_t s0 = 0;
+  for (int u = 0; u < v; ++u) s0 += n_visible[u];
+  start = s0;
+  count = n_visible[v];
+}
+
+// (1) cnt(t, b) for block (b, v): a 2-D difference array over the view's
+// tile grid (+1 / -1 at the rectangle's four corners), summed along rows then
+// columns. Also the packed rectangles (x0 | x1 << 16, y0 | y1 << 16, 0, id)
+// for the emission and the exact pair total. Grid (blocks per view, views).
+__global__ void __launch_bounds__(256) k_tile_count(
+    const float4* __restrict__ bins, const uint64_t* __restrict__ pkeys,
+    const uint32_t* __restrict__ pvals, int n, Grid g, int gsize,
+    const uint32_t* __restrict__ n_visible, uint32_t* __restrict__ counts, int64_t stride,
+    unsigned long long* __restrict__ pair_total, uint4* __restrict__ crect,
+    int64_t* __restrict__ scan_n) {
+  extern __shared__ int s_d[];  // [tiles_y + 1][tiles_x + 1]
+  __shared__ unsigned long long s_tot[8];
+  const int v = blockIdx.y, b = blockIdx.x;
+  if (b == 0 && v == 0 && threadIdx.x == 0) *scan_n = gridDim.x;
+  int64_t vs, nv;
+  view_span(n_visible, v, vs, nv);
+  const int64_t first = vs + (int64_t)b * gsize;
+  const int64_t last = min(vs + nv, first + gsize);
+  const int W = g.tiles_x + 1, H = g.tiles_y + 1;
+  for (int k = threadIdx.x; k < W * H; k += 256) s_d[k] = 0;
+  __syncthreads();
+  uint64_t mine = 0;
+  // four items per thread at a time: all their loads issue before any use
+  for (int64_t base = first + threadIdx.x; base < last; base += 4 * 256) {
+    uint64_t pk[4];
+    uint32_t id[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t item = base + u * 256;
+      pk[u] = item < last ? pkeys[item] : ~0ull;
+      id[u] = item < last ? pvals[item] : 0u;
+    }
+    float4 r2[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      r2[u] = pk[u] != ~0ull ? __ldg(&bins[(int64_t)(pk[u] >> 32) * n + id[u]])
+                             : make_float4(0.f, __uint_as_float(1u), 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t item = base + u * 256;
+      if (item >= last) break;
+      const uint32_t rx = __float_as_uint(r2[u].y), ry = __float_as_uint(r2[u].z);
+      const int x0 = rx & 0xffffu, x1 = rx >> 16, y0 = ry & 0xffffu, y1 = ry >> 16;
+      if (x0 <= x1 && y0 <= y1) {
+        atomicAdd(&s_d[y0 * W + x0], 1);
+        atomicAdd(&s_d[y0 * W + x1 + 1], -1);
+        atomicAdd(&s_d[(y1 + 1) * W + x0], -1);
+        atomicAdd(&s_d[(y1 + 1) * W + x1 + 1], 1);
+        mine += (uint64_t)(x1 - x0 + 1) * (uint64_t)(y1 - y0 + 1);
+        crect[item] = make_uint4(rx, ry, 0u, id[u]);
+      } else {
+        crect[item] = make_uint4(1u, 0u, 0u, 0u);  // empty: x0 > x1
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
+  if ((threadIdx.x & 31) == 0) s_tot[threadIdx.x >> 5] = mine;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long t = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += s_tot[w];
+    if (t) atomicAdd(pair_total, t);
+  }
+  // running sums along each row, then down each column
+  for (int r = threadIdx.x; r < H - 1; r += 256) {
+    int acc = 0;
+    for (int c = 0; c < W - 1; ++c) {
+      acc += s_d[r * W + c];
+      s_d[r * W + c] = acc;
+    }
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < W - 1; c += 256) {
+    int acc = 0;
+    for (int r = 0; r < H - 1; ++r) {
+      acc += s_d[r * W + c];
+      s_d[r * W + c] = acc;
+    }
+  }
+  __syncthreads();
+  const int tpv = g.tiles_per_view;
+  for (int t = threadIdx.x; t < tpv; t += 256) {
+    const int r = t / g.tiles_x, c = t - r * g.tiles_x;
+    counts[((int64_t)v * tpv + t) * stride + b] = (uint32_t)s_d[r * W + c];
+  }
+}
+
+// (2b) base(t): exclusive scan of the tile totals over all tiles (one block),
+// the ranges, the pair count and the capacity check.
+__global__ void __launch_bounds__(1024) k_tile_base(
+    const uint32_t* __restrict__ tile_totals, int64_t n_tiles,
+    const unsigned long long* __restrict__ pair_total, int64_t capacity,
+    uint32_t* __restrict__ tile_base, int64_t* __restrict__ ranges, int64_t* __restrict__ n_pairs,
+    uint32_t* __restrict__ status) {
+  __shared__ uint32_t s_w[32];
+  const unsigned long long total = *pair_total;
+  if (threadIdx.x == 0) {
+    *n_pairs = (int64_t)total;
+    if ((int64_t)total > capacity) atomicOr(status, kStatusCapacity);
+  }
+  if ((int64_t)total > capacity) return;  // every range stays empty
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t carry = 0;
+  for (int64_t base = 0; base < n_tiles; base += 1024) {
+    const int64_t t = base + threadIdx.x;
+    const uint32_t x = t < n_tiles ? tile_totals[t] : 0u;
+    uint32_t incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_w[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const uint32_t w = s_w[lane];
+      uint32_t wi = w;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += y;
+      }
+      s_w[lane] = wi - w;
+    }
+    __syncthreads();
+    const uint32_t start = carry + s_w[warp] + incl - x;
+    if (t < n_tiles) {
+      tile_base[t] = start;
+      ranges[2 * t] = start;
+      ranges[2 * t + 1] = (int64_t)start + x;
+    }
+    __syncthreads();
+    if (threadIdx.x == 1023) s_w[0] = start + x;  // carry into the next chunk
+    __syncthreads();
+    carry = s_w[0];
+    __syncthreads();
+  }
+}
+
+// (3) emission. Block (b, region, v) -- one warp -- places Gaussian block b's
+// pairs in a region of kRegionCols x kRegionRows tiles. Every tile of the
+// region keeps the position of its next pair in shared memory (base(t) plus
+// the pairs earlier blocks put there); the warp streams the block's
+// rectangles in depth order, 32 per coalesced load, and for each one that
+// reaches the region writes its pairs at once, one lane per tile (a rectangle
+// has one pair per tile, so no two lanes share a counter), straight to their
+// final positions.
+__global__ void __launch_bounds__(32) k_emit_tiles(
+    const uint4* __restrict__ crect, int gsize, const uint32_t* __restrict__ n_visible, Grid g,
+    const uint32_t* __restrict__ offsets, int64_t stride, const uint32_t* __restrict__ tile_base,
+    const unsigned long long* __restrict__ pair_total, uint32_t* __restrict__ ids_out,
+    int64_t capacity, uint32_t* __restrict__ status) {
+  constexpr int kTiles = kRegionCols * kRegionRows;
+  __shared__ uint32_t s_next[kTiles];
+  if ((int64_t)*pair_total > capacity) return;
+  const int lane = threadIdx.x;
+  const int v = blockIdx.z, b = blockIdx.x;
+  const int ncg = (g.tiles_x + kRegionCols - 1) / kRegionCols;
+  const int c0 = kRegionCols * (blockIdx.y % ncg), r0 = kRegionRows * (blockIdx.y / ncg);
+  const int c1 = min(c0 + kRegionCols, g.tiles_x) - 1, r1 = min(r0 + kRegionRows, g.tiles_y) - 1;
+  int64_t vs, nv;
+  view_span(n_visible, v, vs, nv);
+  const int64_t first = vs + (int64_t)b * gsize;
+  const int64_t last = min(vs + nv, first + gsize);
+  if (first >= last) return;
+  const int tpv = g.tiles_per_view;
+  for (int li = lane; li < kTiles; li += 32) {
+    const int r = r0 + li / kRegionCols, c = c0 + li % kRegionCols;
+    uint32_t next = 0;
+    if (r <= r1 && c <= c1) {
+      const int64_t t = (int64_t)v * tpv + (int64_t)r * g.tiles_x + c;
+      next = tile_base[t] + offsets[t * stride + b];
+    }
+    s_next[li] = next;
+  }
+  __syncwarp();
+  uint4 cur = make_uint4(1u, 0u, 0u, 0u), nxt = make_uint4(1u, 0u, 0u, 0u);
+  if (first + lane < last) cur = crect[first + lane];
+  if (first + 32 + lane < last) nxt = crect[first + 32 + lane];
+  for (int64_t i0 = first; i0 < last; i0 += 32) {
+    // two batches in flight while this one is placed
+    uint4 nxt2 = make_uint4(1u, 0u, 0u, 0u);
+    if (i0 + 64 + lane < last) nxt2 = crect[i0 + 64 + lane];
+    const int x0 = cur.x & 0xffffu, x1 = cur.x >> 16, y0 = cur.y & 0xffffu, y1 = cur.y >> 16;
+    uint32_t hits = __ballot_sync(0xffffffffu,
+                                  x0 <= x1 && x1 >= c0 && x0 <= c1 && y1 >= r0 && y0 <= r1);
+    while (hits) {
+      const int L = __ffs(hits) - 1;
+      hits &= hits - 1;
+      const uint32_t rx = __shfl_sync(0xffffffffu, cur.x, L);
+      const uint32_t ry = __shfl_sync(0xffffffffu, cur.y, L);
+      const uint32_t id = __shfl_sync(0xffffffffu, cur.w, L);
+      const int cx0 = max((int)(rx & 0xffffu), c0), cx1 = min((int)(rx >> 16), c1);
+      const int ry0 = max((int)(ry & 0xffffu), r0), ry1 = min((int)(ry >> 16), r1);
+      const int wp = cx1 - cx0 + 1;
+      const int np = wp * (ry1 - ry0 + 1);
+      const float inv_wp = 1.f / (float)wp;
+      for (int p0 = 0; p0 < np; p0 += 32) {
+        const int p = p0 + lane;
+        if (p < np) {
+          const int rr = min((int)(((float)p + 0.5f) * inv_wp), ry1 - ry0);
+          const int cc = p - rr * wp;
+          const int li = (ry0 - r0 + rr) * kRegionCols + (cx0 - c0 + cc);
+          const uint32_t pos = s_next[li];
+          s_next[li] = pos + 1;
+          if ((int64_t)pos < capacity) ids_out[pos] = id;
+          else atomicOr(status, kStatusBounds);
+        }
+      }
+      __syncwarp();
+    }
+    cur = nxt;
+    nxt = nxt2;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Column emission (presort mode, images up to kMaxColumns tiles wide).
+// A pair's key is row << cbits | column, row = view * tiles_y + tile row:
+// ordering by it is ordering by global tile. The emission hands out pairs
+// already ordered by column (stable in depth order), which is the first
+// least-significant-digit pass of that order; the radix passes that follow
+// sort by row only.
 
 // (1) pairs per tile column of each block of kColItems presorted Gaussians:
 // a difference array over columns weighted by the rectangle's height, then a
@@ -890,6 +1147,10 @@ int64_t presort_partitions(int64_t items) {
 int64_t emit_blocks(int64_t items) { return (items + kEmitItems - 1) / kEmitItems; }
 int64_t column_blocks(int64_t items) { return (items + kColItems - 1) / kColItems; }
 bool column_emission(const Grid& g) { return g.tiles_x <= kMaxColumns; }
+bool tile_emission(const Grid& g) {
+  return (int64_t)(g.tiles_x + 1) * (g.tiles_y + 1) * (int64_t)sizeof(int) <= kTileDiffBytes;
+}
+int tile_gsize(int64_t n) { return n <= (2 << 20) ? 1024 : 4096; }
 
 cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
   cudaError_t e;
@@ -905,7 +1166,7 @@ cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
     int64_t blocks = (n_items + 255) / 256;
     if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
     k_depth_keys<<<(int)blocks, 256, 0, stream>>>(bins4, a.n, a.n_views, a.pkeys[0], a.pvals[0],
-                                                  a.n_items_dev);
+                                                  a.n_items_dev, a.n_visible);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     e = run_radix_passes<uint64_t, kPresortItems>(a.pkeys[0], a.pvals[0], a.pkeys[1], a.pvals[1],
                                                   a.n_items_dev, n_items, n_items, a.presort,
@@ -913,6 +1174,27 @@ cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
                                                   stream);
     if (e != cudaSuccess) return e;
     const int fin = a.presort.passes & 1;
+    if (a.tile_emit) {
+      // 2) pairs per (tile, Gaussian block), their scans, placement
+      const Grid& g = a.grid;
+      const size_t dsmem = (size_t)(g.tiles_x + 1) * (g.tiles_y + 1) * sizeof(int);
+      if ((e = cudaFuncSetAttribute(k_tile_count, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)dsmem)) != cudaSuccess)
+        return e;
+      k_tile_count<<<dim3((unsigned)a.tile_bpv, (unsigned)a.n_views), 256, dsmem, stream>>>(
+          bins4, a.pkeys[fin], a.pvals[fin], a.n, g, a.gsize, a.n_visible, a.counts,
+          a.counts_stride, a.pair_total, a.crect, a.scan_n);
+      k_radix_scan<<<(unsigned)a.n_tiles, 256, 0, stream>>>(a.counts, a.counts_stride, a.scan_n,
+                                                            a.tile_bpv, 1, a.tile_totals);
+      k_tile_base<<<1, 1024, 0, stream>>>(a.tile_totals, a.n_tiles, a.pair_total, a.capacity,
+                                          a.tile_base, a.ranges, a.n_pairs, a.status);
+      const unsigned regions = (unsigned)(((g.tiles_x + kRegionCols - 1) / kRegionCols) *
+                                          ((g.tiles_y + kRegionRows - 1) / kRegionRows));
+      k_emit_tiles<<<dim3((unsigned)a.tile_bpv, regions, (unsigned)a.n_views), 32, 0, stream>>>(
+          a.crect, a.gsize, a.n_visible, g, a.counts, a.counts_stride, a.tile_base, a.pair_total,
+          a.vals[0], a.capacity, a.status);
+      return cudaGetLastError();
+    }
     if (a.column_emit) {
       // 2) pairs per column and block, their scan, emission by column
       const int64_t cb = column_blocks(n_items);

@@ -20,6 +20,8 @@ constexpr size_t kStatusOffset = 0;
 constexpr size_t kCountersOffset = 64;   // 16 x uint32
 constexpr size_t kNItemsOffset = 256;    // int64
 constexpr size_t kPairTotalOffset = 264; // uint64
+constexpr size_t kNVisibleOffset = 512;  // uint32 [GS_MAX_VIEWS]
+constexpr size_t kScanNOffset = 640;     // int64
 constexpr size_t kHistBytes = 256 * sizeof(uint32_t);  // digit totals of the current pass
 constexpr int64_t kMaxPairCapacity = GS_MAX_PAIR_CAPACITY;
 
@@ -35,13 +37,15 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 struct Layout {
   RadixPlan pairs, presort;
+  bool tile_emit = false;
+  int gsize = 0, tile_bpv = 0;
   bool column_emit = false;
   int cbits = 0;
   int key_bytes = 8;
   int64_t counts_stride = 0;
   size_t off_hist = 0, off_emit_lb = 0, off_counts = 0, off_keys0 = 0, off_keys1 = 0,
          off_vals1 = 0, off_pkeys0 = 0, off_pkeys1 = 0, off_pvals0 = 0, off_pvals1 = 0,
-         off_crect = 0;
+         off_crect = 0, off_tile_totals = 0, off_tile_base = 0;
   size_t total = 0;
 };
 
@@ -73,8 +77,12 @@ bool make_layout(int64_t n, int32_t n_views, const gs_camera* cams, int64_t capa
   } else {
     L.key_bytes = 4;
     L.presort = make_radix_plan(32 + bits_for((uint64_t)n_views - 1), false);
-    L.column_emit = column_emission(g);
-    if (L.column_emit) {
+    L.tile_emit = tile_emission(g);
+    L.column_emit = !L.tile_emit && column_emission(g);
+    if (L.tile_emit) {
+      L.gsize = tile_gsize(n);
+      L.tile_bpv = (int)((n + L.gsize - 1) / L.gsize);
+    } else if (L.column_emit) {
       // keys row << cbits | column; the radix passes sort the row bits
       L.cbits = bits_for((uint64_t)g.tiles_x - 1);
       if (L.cbits == 0) L.cbits = 1;
@@ -88,24 +96,33 @@ bool make_layout(int64_t n, int32_t n_views, const gs_camera* cams, int64_t capa
   if (mode == GS_SORT_PRESORT) {
     const int64_t p2 = presort_partitions(items);
     if (p2 > parts) parts = p2;
-    const int64_t p3 = column_blocks(items);
+    const int64_t p3 = L.tile_emit ? L.tile_bpv : column_blocks(items);
     if (p3 > parts) parts = p3;
   }
   L.counts_stride = parts > 0 ? (parts + 3) / 4 * 4 : 4;
+  // counts rows: radix digits, tile columns, or every tile of every view
+  const int64_t rows = L.tile_emit && (int64_t)tiles > 256 ? (int64_t)tiles : 256;
   size_t off = kControlBytes;
   L.off_hist = off; off = align_up(off + kHistBytes);
   L.off_emit_lb = off; off = align_up(off + (size_t)emit_blocks(items) * 8);
-  L.off_counts = off; off = align_up(off + (size_t)256 * L.counts_stride * 4);
-  L.off_keys0 = off; off = align_up(off + (size_t)capacity * L.key_bytes);
-  L.off_keys1 = off; off = align_up(off + (size_t)capacity * L.key_bytes);
-  L.off_vals1 = off; off = align_up(off + (size_t)capacity * 4);
+  L.off_counts = off; off = align_up(off + (size_t)rows * L.counts_stride * 4);
+  // pair keys and the second id buffer: not needed when pairs are placed
+  // straight at their positions
+  const int64_t kcap = L.tile_emit ? 0 : capacity;
+  L.off_keys0 = off; off = align_up(off + (size_t)kcap * L.key_bytes);
+  L.off_keys1 = off; off = align_up(off + (size_t)kcap * L.key_bytes);
+  L.off_vals1 = off; off = align_up(off + (size_t)kcap * 4);
   if (mode == GS_SORT_PRESORT) {
     L.off_pkeys0 = off; off = align_up(off + (size_t)items * 8);
     L.off_pkeys1 = off; off = align_up(off + (size_t)items * 8);
     L.off_pvals0 = off; off = align_up(off + (size_t)items * 4);
     L.off_pvals1 = off; off = align_up(off + (size_t)items * 4);
-    if (L.column_emit) {
+    if (L.column_emit || L.tile_emit) {
       L.off_crect = off; off = align_up(off + (size_t)items * 16);
+    }
+    if (L.tile_emit) {
+      L.off_tile_totals = off; off = align_up(off + (size_t)tiles * 4);
+      L.off_tile_base = off; off = align_up(off + (size_t)tiles * 4);
     }
   }
   L.total = off;
@@ -184,6 +201,7 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
 
   if (cudaMemsetAsync(w + kCountersOffset, 0, 16 * sizeof(uint32_t), st) != cudaSuccess ||
       cudaMemsetAsync(w + kPairTotalOffset, 0, sizeof(uint64_t), st) != cudaSuccess ||
+      cudaMemsetAsync(w + kNVisibleOffset, 0, GS_MAX_VIEWS * sizeof(uint32_t), st) != cudaSuccess ||
       cudaMemsetAsync(w + L.off_emit_lb, 0, (size_t)emit_blocks(items) * 8, st) != cudaSuccess ||
       cudaMemsetAsync(out->ranges, 0, (size_t)tiles * 2 * sizeof(int64_t), st) != cudaSuccess)
     return GS_ERR_CUDA;
@@ -196,6 +214,9 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
   a.mode = sort_mode;
   a.grid = g;
   a.capacity = out->pair_capacity;
+  a.tile_emit = L.tile_emit;
+  a.gsize = L.gsize;
+  a.tile_bpv = L.tile_bpv;
   a.column_emit = L.column_emit;
   a.cbits = L.cbits;
   a.pairs = L.pairs;
@@ -220,7 +241,13 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
   a.n_pairs = out->n_pairs;
   a.n_items_dev = reinterpret_cast<int64_t*>(w + kNItemsOffset);
   a.pair_total = reinterpret_cast<unsigned long long*>(w + kPairTotalOffset);
-  if (L.column_emit) a.crect = reinterpret_cast<uint4*>(w + L.off_crect);
+  if (L.column_emit || L.tile_emit) a.crect = reinterpret_cast<uint4*>(w + L.off_crect);
+  a.n_visible = reinterpret_cast<uint32_t*>(w + kNVisibleOffset);
+  a.scan_n = reinterpret_cast<int64_t*>(w + kScanNOffset);
+  if (L.tile_emit) {
+    a.tile_totals = reinterpret_cast<uint32_t*>(w + L.off_tile_totals);
+    a.tile_base = reinterpret_cast<uint32_t*>(w + L.off_tile_base);
+  }
   a.ranges = out->ranges;
   a.n_tiles = tiles;
   return cuda_status(launch_bin_sort(a, st));

@@ -28,6 +28,9 @@ struct BinSortArgs {
   int mode;
   Grid grid;
   int64_t capacity;
+  bool tile_emit;      // presort mode: pairs placed straight at their positions
+  int gsize;           // tile emission: Gaussians per block
+  int tile_bpv;        // tile emission: blocks per view
   bool column_emit;    // presort mode: emission ordered by tile column
   int cbits;           // column bits of a column-emission key (row << cbits | column)
   RadixPlan pairs;     // radix passes over the pair keys
@@ -46,7 +49,11 @@ struct BinSortArgs {
   int64_t* n_pairs;
   int64_t* n_items_dev;
   unsigned long long* pair_total;  // column emission: exact pair count
-  uint4* crect;                      // column emission: presorted rectangles [n_views * n]
+  uint4* crect;                      // tile / column emission: presorted rectangles [n_views * n]
+  uint32_t* n_visible;               // [GS_MAX_VIEWS] visible Gaussians per view
+  uint32_t* tile_totals;             // tile emission: pairs per tile [n_tiles]
+  uint32_t* tile_base;               // tile emission: first position of each tile [n_tiles]
+  int64_t* scan_n;                   // tile emission: blocks per view, for the scan
   int64_t* ranges;
   int64_t n_tiles;     // n_views * tiles per view
 };
@@ -77,6 +84,8 @@ int64_t pair_partitions(int64_t items);     // radix partitions over pair keys
 int64_t presort_partitions(int64_t items);  // radix partitions over depth keys
 int64_t column_blocks(int64_t items);       // column-emission blocks
 bool column_emission(const Grid& g);        // presort mode emits by column on this grid
+bool tile_emission(const Grid& g);          // presort mode places pairs directly on this grid
+int tile_gsize(int64_t n);                  // tile emission: Gaussians per block
 int64_t emit_blocks(int64_t items);
 
 }  // namespace gsb

@@ -102,12 +102,13 @@ def test_binning_bit_exact(name, kw, how, mode):
 
 
 @pytest.mark.parametrize("mode", MODES)
-@pytest.mark.parametrize("W,H", [(200, 136), (4096, 48), (4300, 40)])
+@pytest.mark.parametrize("W,H", [(200, 136), (4300, 40), (4096, 2576), (8192, 1296)])
 def test_binning_isolated_with_ties_and_ragged_tail(mode, W, H):
     # screen-space inputs straight from the generator: many equal depth keys
     # (ties broken by index), culled entries, rectangles clipped by the image.
-    # Widths: 13 tile columns, exactly 256 (the widest grid emitted by
-    # column in presort mode) and 269 (emitted by tile id instead).
+    # Grids in presort mode: 13 x 9 and 269 x 3 tiles place pairs straight at
+    # their positions; 256 x 161 (too many tiles for that) emits by column;
+    # 512 x 81 (too wide for columns too) emits by tile id.
     n, V = 3000, 2
     d = S.make_projected_2d(n, W, H, seed=3, n_views=V)
     tx, ty = (W + 15) // 16, (H + 15) // 16
