@@ -119,13 +119,22 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- work model
 
-def sort_passes(sp, sort_mode: str):
-    """(presort passes, pair passes) of gs_bin_sort for this workload."""
-    tiles = sp.V * ((sp.W + 15) // 16) * ((sp.H + 15) // 16)
+def sort_plan(sp, sort_mode: str) -> dict:
+    """How gs_bin_sort treats this workload (mirrors the library's choice):
+    presort passes, pair passes, emission path and tile-placement blocks."""
+    tx, ty = (sp.W + 15) // 16, (sp.H + 15) // 16
+    tiles = sp.V * tx * ty
     tile_bits = max(int(tiles - 1).bit_length(), 0)
     if sort_mode == "full64":
-        return 0, (32 + tile_bits + 7) // 8
-    return 4 + (1 if sp.V > 1 else 0), (tile_bits + 7) // 8
+        return dict(path="tile_id", pre=0, pair=(32 + tile_bits + 7) // 8, bpv=0, tiles=tiles)
+    pre = (32 + max(int(sp.V - 1).bit_length(), 0) + 7) // 8
+    if (tx + 1) * (ty + 1) * 4 <= 160 * 1024:
+        gsize = 1024 if sp.n <= (2 << 20) else 4096
+        return dict(path="tiles", pre=pre, pair=0, bpv=-(-sp.n // gsize), tiles=tiles)
+    if tx <= 256:
+        rows = max(int(sp.V * ty - 1).bit_length(), 0)
+        return dict(path="columns", pre=pre, pair=(rows + 7) // 8, bpv=0, tiles=tiles)
+    return dict(path="tile_id", pre=pre, pair=(tile_bits + 7) // 8, bpv=0, tiles=tiles)
 
 
 def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float) -> dict:
@@ -133,15 +142,22 @@ def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float) -> dict:
 
     Bytes count the data the definition has to move once: parameters read,
     outputs written, 59 real floats per Gaussian (pad lanes excluded); a radix
-    pass reads and writes every key and value once; the blend kernels read
-    every list entry's id and record once."""
+    pass reads and writes every key and value once; placing pairs straight at
+    their positions writes every id once, reads every packed rectangle once
+    and reads and writes the (tile, Gaussian block) count table once; the
+    blend kernels read every list entry's id and record once."""
     n, V = sp.n, sp.V
     P = V * sp.W * sp.H
     rec = 48
     p59 = 59 * 4
-    pre, pair = sort_passes(sp, sort_mode)
+    plan = sort_plan(sp, sort_mode)
+    pre, pair = plan["pre"], plan["pair"]
     if sort_mode == "full64":
         sort_bytes = n_pairs * (12 + pair * 24 + 8) + V * n * 16
+    elif plan["path"] == "tiles":
+        table = plan["tiles"] * plan["bpv"] * 4
+        sort_bytes = (n_pairs * 4 + V * n * (16 + 12 + pre * 24 + 12 + 16 + 16)
+                      + 3 * table + plan["tiles"] * 24)
     else:
         sort_bytes = n_pairs * (8 + pair * 16 + 4) + V * n * (16 + pre * 24 + 12)
     return {
@@ -157,8 +173,16 @@ def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float) -> dict:
 
 def launches_per_step(sp, sort_mode: str) -> int:
     """Library kernels launched by one step (memsets excluded)."""
-    pre, pair = sort_passes(sp, sort_mode)
-    sort = (1 + 3 * pre if sort_mode == "presort" else 0) + 1 + 3 * pair + 1
+    plan = sort_plan(sp, sort_mode)
+    pre, pair = plan["pre"], plan["pair"]
+    if sort_mode == "full64":
+        sort = 1 + 3 * pair + 1                 # emit, passes, ranges
+    elif plan["path"] == "tiles":
+        sort = 1 + 3 * pre + 4                  # keys, presort, count, scan, base, place
+    elif plan["path"] == "columns":
+        sort = 1 + 3 * pre + 3 + 3 * pair + 1   # ..., count, scan, emit, row passes, ranges
+    else:
+        sort = 1 + 3 * pre + 1 + 3 * pair + 1
     return 1 + sort + 1 + 1 + 1 + 1 + 1
 
 
@@ -462,6 +486,7 @@ def run_ours(args):
         "config": {"workload": WORKLOAD, "gaussians": sp.n, "width": c.width, "height": c.height,
                    "sh_degree": 3, "views_per_gpu": 1, "pairs": n_pairs,
                    "sort_mode": args.sort_mode,
+                   "sort_path": sort_plan(sp, args.sort_mode)["path"],
                    "l2": "working set larger than L2 (0.7 GB of parameters and Adam state "
                          "rewritten every step)",
                    "parallelism": "dp%d (one view per GPU, gradient all-reduce)" % world

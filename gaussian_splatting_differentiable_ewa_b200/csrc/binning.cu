@@ -62,6 +62,7 @@ constexpr int kMaxColumns = 256;   // widest tile grid the column emission takes
 constexpr int kColPitch = 33;      // buffer row: conflict-free along and across columns
 constexpr int kRegionCols = 32;    // tile-emission region: kRegionCols x kRegionRows tiles
 constexpr int kRegionRows = 16;
+constexpr int kEmitWarps = 1;      // tile-emission regions (one per warp) per block
 constexpr int kTileDiffBytes = 160 * 1024;  // largest tile-count difference array
 
 __device__ __forceinline__ uint32_t get_block_index(uint32_t* counter) {
@@ -198,6 +199,13 @@ __device__ __forceinline__ bool presorted_rect(const float4* __restrict__ bins,
   return (rx & 0xffffu) <= (rx >> 16) && (ry & 0xffffu) <= (ry >> 16);
 }
 
+// Count table entry of (global tile t, Gaussian block b): groups of 8 tiles,
+// block-major inside a group, so a block writes 8 neighbouring tiles' counts
+// as one 32-byte run and a group's entries over all blocks are contiguous.
+__device__ __forceinline__ int64_t tcount_index(int64_t t, int64_t b, int64_t stride) {
+  return ((t >> 3) * stride + b) * 8 + (t & 7);
+}
+
 // Start of view v's visible Gaussians in the presorted order (sorted by
 // (view, depth) with culled ones last) and their number.
 __device__ __forceinline__ void view_span(const uint32_t* __restrict__ n_visible, int v,
@@ -293,7 +301,76 @@ __global__ void __launch_bounds__(256) k_tile_count(
   const int tpv = g.tiles_per_view;
   for (int t = threadIdx.x; t < tpv; t += 256) {
     const int r = t / g.tiles_x, c = t - r * g.tiles_x;
-    counts[((int64_t)v * tpv + t) * stride + b] = (uint32_t)s_d[r * W + c];
+    counts[tcount_index((int64_t)v * tpv + t, b, stride)] = (uint32_t)s_d[r * W + c];
+  }
+}
+
+// (2a) per tile: exclusive scan of cnt(t, b) over the blocks b, in place, and
+// the tile's total. One block per group of 8 tiles; thread i takes blocks
+// i, i + 256, ... with the group's 8 counts of a block in two 16-byte loads,
+// scanning the 8 tiles side by side.
+__global__ void __launch_bounds__(256) k_tile_scan(uint32_t* __restrict__ counts, int64_t stride,
+                                                  int bpv, int64_t n_tiles,
+                                                  uint32_t* __restrict__ totals) {
+  __shared__ uint32_t s_w[8][9];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t g = blockIdx.x;
+  uint4* grp = reinterpret_cast<uint4*>(counts + g * stride * 8);
+  uint32_t carry[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int b0 = 0; b0 < bpv; b0 += 256) {
+    const int b = b0 + (int)threadIdx.x;
+    uint32_t x[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (b < bpv) {
+      const uint4 lo = grp[2 * b], hi = grp[2 * b + 1];
+      x[0] = lo.x; x[1] = lo.y; x[2] = lo.z; x[3] = lo.w;
+      x[4] = hi.x; x[5] = hi.y; x[6] = hi.z; x[7] = hi.w;
+    }
+    uint32_t inc[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) inc[k] = x[k];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc[k], o);
+        if (lane >= o) inc[k] += y;
+      }
+    }
+    if (lane == 31) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) s_w[warp][k] = inc[k];
+    }
+    __syncthreads();
+    uint32_t before[8], chunk[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      uint32_t pre = 0, all = 0;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        const uint32_t s = s_w[w][k];
+        pre += w < warp ? s : 0u;
+        all += s;
+      }
+      before[k] = pre;
+      chunk[k] = all;
+    }
+    if (b < bpv) {
+      uint32_t o[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) o[k] = carry[k] + before[k] + inc[k] - x[k];
+      grp[2 * b] = make_uint4(o[0], o[1], o[2], o[3]);
+      grp[2 * b + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) carry[k] += chunk[k];
+    __syncthreads();
+  }
+  if (threadIdx.x < 8) {
+    const int64_t t = g * 8 + threadIdx.x;
+    uint32_t c = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) c = k == (int)threadIdx.x ? carry[k] : c;
+    if (t < n_tiles) totals[t] = c;
   }
 }
 
@@ -349,26 +426,29 @@ __global__ void __launch_bounds__(1024) k_tile_base(
   }
 }
 
-// (3) emission. Block (b, region, v) -- one warp -- places Gaussian block b's
-// pairs in a region of kRegionCols x kRegionRows tiles. Every tile of the
+// (3) emission. Each warp of block (b, ., v) places Gaussian block b's pairs
+// in one region of kRegionCols x kRegionRows tiles. Every tile of the
 // region keeps the position of its next pair in shared memory (base(t) plus
 // the pairs earlier blocks put there); the warp streams the block's
 // rectangles in depth order, 32 per coalesced load, and for each one that
 // reaches the region writes its pairs at once, one lane per tile (a rectangle
 // has one pair per tile, so no two lanes share a counter), straight to their
 // final positions.
-__global__ void __launch_bounds__(32) k_emit_tiles(
+__global__ void __launch_bounds__(32 * kEmitWarps) k_emit_tiles(
     const uint4* __restrict__ crect, int gsize, const uint32_t* __restrict__ n_visible, Grid g,
-    const uint32_t* __restrict__ offsets, int64_t stride, const uint32_t* __restrict__ tile_base,
-    const unsigned long long* __restrict__ pair_total, uint32_t* __restrict__ ids_out,
-    int64_t capacity, uint32_t* __restrict__ status) {
+    int n_regions, const uint32_t* __restrict__ offsets, int64_t stride,
+    const uint32_t* __restrict__ tile_base, const unsigned long long* __restrict__ pair_total,
+    uint32_t* __restrict__ ids_out, int64_t capacity, uint32_t* __restrict__ status) {
   constexpr int kTiles = kRegionCols * kRegionRows;
-  __shared__ uint32_t s_next[kTiles];
+  __shared__ uint32_t s_next_all[kEmitWarps][kTiles];
   if ((int64_t)*pair_total > capacity) return;
-  const int lane = threadIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int region = blockIdx.y * kEmitWarps + warp;  // warps of a block: regions side by side
+  if (region >= n_regions) return;
+  uint32_t* s_next = s_next_all[warp];
   const int v = blockIdx.z, b = blockIdx.x;
   const int ncg = (g.tiles_x + kRegionCols - 1) / kRegionCols;
-  const int c0 = kRegionCols * (blockIdx.y % ncg), r0 = kRegionRows * (blockIdx.y / ncg);
+  const int c0 = kRegionCols * (region % ncg), r0 = kRegionRows * (region / ncg);
   const int c1 = min(c0 + kRegionCols, g.tiles_x) - 1, r1 = min(r0 + kRegionRows, g.tiles_y) - 1;
   int64_t vs, nv;
   view_span(n_visible, v, vs, nv);
@@ -381,7 +461,7 @@ __global__ void __launch_bounds__(32) k_emit_tiles(
     uint32_t next = 0;
     if (r <= r1 && c <= c1) {
       const int64_t t = (int64_t)v * tpv + (int64_t)r * g.tiles_x + c;
-      next = tile_base[t] + offsets[t * stride + b];
+      next = tile_base[t] + offsets[tcount_index(t, b, stride)];
     }
     s_next[li] = next;
   }
@@ -1184,15 +1264,17 @@ cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
       k_tile_count<<<dim3((unsigned)a.tile_bpv, (unsigned)a.n_views), 256, dsmem, stream>>>(
           bins4, a.pkeys[fin], a.pvals[fin], a.n, g, a.gsize, a.n_visible, a.counts,
           a.counts_stride, a.pair_total, a.crect, a.scan_n);
-      k_radix_scan<<<(unsigned)a.n_tiles, 256, 0, stream>>>(a.counts, a.counts_stride, a.scan_n,
-                                                            a.tile_bpv, 1, a.tile_totals);
+      k_tile_scan<<<(unsigned)((a.n_tiles + 7) / 8), 256, 0, stream>>>(
+          a.counts, a.counts_stride, a.tile_bpv, a.n_tiles, a.tile_totals);
       k_tile_base<<<1, 1024, 0, stream>>>(a.tile_totals, a.n_tiles, a.pair_total, a.capacity,
                                           a.tile_base, a.ranges, a.n_pairs, a.status);
-      const unsigned regions = (unsigned)(((g.tiles_x + kRegionCols - 1) / kRegionCols) *
-                                          ((g.tiles_y + kRegionRows - 1) / kRegionRows));
-      k_emit_tiles<<<dim3((unsigned)a.tile_bpv, regions, (unsigned)a.n_views), 32, 0, stream>>>(
-          a.crect, a.gsize, a.n_visible, g, a.counts, a.counts_stride, a.tile_base, a.pair_total,
-          a.vals[0], a.capacity, a.status);
+      const int regions = ((g.tiles_x + kRegionCols - 1) / kRegionCols) *
+                          ((g.tiles_y + kRegionRows - 1) / kRegionRows);
+      const unsigned rblocks = (unsigned)((regions + kEmitWarps - 1) / kEmitWarps);
+      k_emit_tiles<<<dim3((unsigned)a.tile_bpv, rblocks, (unsigned)a.n_views), 32 * kEmitWarps,
+                     0, stream>>>(a.crect, a.gsize, a.n_visible, g, regions, a.counts,
+                                  a.counts_stride, a.tile_base, a.pair_total, a.vals[0],
+                                  a.capacity, a.status);
       return cudaGetLastError();
     }
     if (a.column_emit) {

@@ -101,7 +101,9 @@ bool make_layout(int64_t n, int32_t n_views, const gs_camera* cams, int64_t capa
   }
   L.counts_stride = parts > 0 ? (parts + 3) / 4 * 4 : 4;
   // counts rows: radix digits, tile columns, or every tile of every view
-  const int64_t rows = L.tile_emit && (int64_t)tiles > 256 ? (int64_t)tiles : 256;
+  // (rounded up to whole groups of 8 tiles)
+  const int64_t trows = ((int64_t)tiles + 7) / 8 * 8;
+  const int64_t rows = L.tile_emit && trows > 256 ? trows : 256;
   size_t off = kControlBytes;
   L.off_hist = off; off = align_up(off + kHistBytes);
   L.off_emit_lb = off; off = align_up(off + (size_t)emit_blocks(items) * 8);
