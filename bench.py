@@ -129,7 +129,7 @@ def sort_plan(sp, sort_mode: str) -> dict:
         return dict(path="tile_id", pre=0, pair=(32 + tile_bits + 7) // 8, bpv=0, tiles=tiles)
     pre = (32 + max(int(sp.V - 1).bit_length(), 0) + 7) // 8
     if (tx + 1) * (ty + 1) * 4 <= 160 * 1024:
-        gsize = 1024 if sp.n <= (2 << 20) else 4096
+        gsize = 768 if sp.n <= (2 << 20) else 4096
         return dict(path="tiles", pre=pre, pair=0, bpv=-(-sp.n // gsize), tiles=tiles)
     if tx <= 256:
         rows = max(int(sp.V * ty - 1).bit_length(), 0)

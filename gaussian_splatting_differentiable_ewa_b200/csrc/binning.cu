@@ -1230,7 +1230,7 @@ bool column_emission(const Grid& g) { return g.tiles_x <= kMaxColumns; }
 bool tile_emission(const Grid& g) {
   return (int64_t)(g.tiles_x + 1) * (g.tiles_y + 1) * (int64_t)sizeof(int) <= kTileDiffBytes;
 }
-int tile_gsize(int64_t n) { return n <= (2 << 20) ? 1024 : 4096; }
+int tile_gsize(int64_t n) { return n <= (2 << 20) ? 768 : 4096; }
 
 cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
   cudaError_t e;
