@@ -3,7 +3,9 @@
 // Forward ("Better Gaussian Splatting in Julia", pwwt.cn sec. 3.2
 // project_gaussian; lshu.cn sec. 3.2: world -> camera -> pixel with division
 // by depth, 3D covariance through the Jacobian of that map): one thread per
-// Gaussian, looping over the views so the parameters are read once. The
+// Gaussian, looping over the views so the parameters are read once; a block's
+// SH coefficients arrive in shared memory by one TMA bulk copy issued at the
+// start, overlapping the geometry. The
 // geometry that ends in a discrete decision (depth key, radius, tile
 // rectangle) is evaluated in double, so that the decision is the exact one up
 // to double rounding; colour is evaluated in float.
@@ -167,6 +169,35 @@ __device__ __forceinline__ void sh_colour_global(const float* __restrict__ shi, 
   for (int ch = 0; ch < 3; ++ch) rgb[ch] = fmaxf(acc[ch], 0.f);
 }
 
+// Colour from the SH coefficients of one Gaussian staged in shared memory
+// (16-byte loads), same arithmetic as sh_colour_global.
+template <int DEG>
+__device__ __forceinline__ void sh_colour_smem(const float* __restrict__ shi, float x, float y,
+                                               float z, float rgb[3]) {
+  constexpr int K = (DEG + 1) * (DEG + 1);
+  float Y[16];
+  sh_basis<DEG>(x, y, z, Y);
+  float acc[3] = {0.5f, 0.5f, 0.5f};
+  if ((K * 3) % 4 == 0) {
+    const float4* s4 = reinterpret_cast<const float4*>(shi);
+#pragma unroll
+    for (int q = 0; q < K * 3 / 4; ++q) {
+      const float4 c = s4[q];
+      const float cv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int idx = 4 * q + e;
+        acc[idx % 3] = fmaf(Y[idx / 3], cv[e], acc[idx % 3]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int idx = 0; idx < K * 3; ++idx) acc[idx % 3] = fmaf(Y[idx / 3], shi[idx], acc[idx % 3]);
+  }
+#pragma unroll
+  for (int ch = 0; ch < 3; ++ch) rgb[ch] = fmaxf(acc[ch], 0.f);
+}
+
 template <int DEG>
 __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __restrict__ means,
                                                           const float4* __restrict__ log_scales,
@@ -178,8 +209,27 @@ __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __
                                                           float4* __restrict__ bins,
                                                           int* __restrict__ radii) {
   constexpr int K = (DEG + 1) * (DEG + 1);
+  // the block's SH coefficients are one contiguous range: a full block with a
+  // 16-byte-aligned array fetches them with one bulk copy that lands while
+  // the geometry is computed
+  extern __shared__ __align__(16) float s_sh[];  // [kProjFwdThreads][K * 3]
+  __shared__ __align__(8) uint64_t s_bar;
+  const int64_t i0 = (int64_t)blockIdx.x * kProjFwdThreads;
+  const bool staged = ((reinterpret_cast<uintptr_t>(sh) & 15) == 0) &&
+                      i0 + kProjFwdThreads <= (int64_t)n;
+  if (staged) {
+    if (threadIdx.x == 0) {
+      constexpr uint32_t bytes = kProjFwdThreads * K * 3 * sizeof(float);
+      mbar_init(&s_bar, 1);
+      fence_mbar_init();
+      mbar_arrive_expect_tx(&s_bar, bytes);
+      bulk_copy_g2s(s_sh, sh + i0 * K * 3, bytes, &s_bar);
+    }
+    __syncthreads();
+  }
+  bool sh_ready = !staged;
   const int i = blockIdx.x * kProjFwdThreads + threadIdx.x;
-  if (i >= n) return;
+  if (i >= n) return;  // only in a partial block, which is not staged
   const float4 m = __ldg(&means[i]);
   const float4 ls = __ldg(&log_scales[i]);
   const float4 q = __ldg(&quats[i]);
@@ -285,7 +335,13 @@ __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __
           float dxv = m.x - c.campos[0], dyv = m.y - c.campos[1], dzv = m.z - c.campos[2];
           float inv = rsqrtf(dxv * dxv + dyv * dyv + dzv * dzv);
           float rgb[3];
-          sh_colour_global<DEG>(shi, dxv * inv, dyv * inv, dzv * inv, rgb);
+          if (staged) {
+            if (!sh_ready) sh_ready = mbar_wait_bounded(&s_bar, 0u, nullptr);
+            sh_colour_smem<DEG>(s_sh + (size_t)threadIdx.x * K * 3, dxv * inv, dyv * inv,
+                                dzv * inv, rgb);
+          } else {
+            sh_colour_global<DEG>(shi, dxv * inv, dyv * inv, dzv * inv, rgb);
+          }
           rec[R_R] = rgb[0];
           rec[R_G] = rgb[1];
           rec[R_B] = rgb[2];
@@ -309,6 +365,8 @@ __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __
                           __uint_as_float((uint32_t)y0 | ((uint32_t)y1 << 16)), 0.f);
     radii[r] = radius;
   }
+  // a staged copy lands before the block exits, even if no view needed it
+  if (staged && !sh_ready) mbar_wait_bounded(&s_bar, 0u, nullptr);
 }
 
 // Backward of k_project for the raw parameters, summing every view in which
@@ -527,7 +585,13 @@ cudaError_t launch_project(const gs_params& p, const CamSet& cams, int n_views, 
   auto q = reinterpret_cast<const float4*>(p.quats);
   auto r = reinterpret_cast<float4*>(records);
   auto b = reinterpret_cast<float4*>(bins);
-#define GS_PFWD(D) k_project<D><<<blocks, threads, 0, stream>>>(m, s, q, p.opacity_logit, p.sh, n, n_views, cams, r, b, radii)
+#define GS_PFWD(D)                                                                          \
+  {                                                                                         \
+    const int smem = threads * 3 * (D + 1) * (D + 1) * (int)sizeof(float);                  \
+    cudaFuncSetAttribute(k_project<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);   \
+    k_project<D><<<blocks, threads, smem, stream>>>(m, s, q, p.opacity_logit, p.sh, n, n_views, \
+                                                    cams, r, b, radii);                     \
+  }
   switch (p.sh_degree) {
     case 0: GS_PFWD(0); break;
     case 1: GS_PFWD(1); break;

@@ -17,6 +17,10 @@ from oracle import oracle as O
 
 # Flag windows: relative distance of alpha from 1/255 and of the trial
 # transmittance from 1e-4 below which float32 and float64 may decide apart.
+# With cancellation in the quadratic form of an elongated Gaussian the
+# kernel's alpha can sit 2e-5 relative from the float64 value (a flip seen at
+# a distance between 2e-5 and 2e-4); every near-opaque layer multiplies that
+# by alpha / (1 - alpha) in the trial T.
 WIN_ALPHA = 2e-4
 WIN_T = 2e-3
 
