@@ -11,7 +11,9 @@
 // to double rounding; colour is evaluated in float.
 //
 // Backward: chain rule of the same map, float, one thread per Gaussian,
-// summing the views in registers before one write of every gradient.
+// summing the views in registers before one write of every gradient; the
+// block's SH coefficients stream into shared memory (cp.async) while the
+// parameters load and the view-independent part is computed.
 
 #include <cuda_runtime.h>
 
@@ -114,17 +116,26 @@ constexpr int kProjFwdThreads = 256;  // projection forward block
 constexpr int kShStride = kProjThreads + 1;  // padded row: conflict-free banks
 
 // Stage the SH coefficients of Gaussians [i0, i0 + cnt) in shared memory,
-// coefficient-major with a padded row (s[c * kShStride + local i]), using
-// coalesced loads of the contiguous global block.
+// coefficient-major with a padded row (s[c * kShStride + local i]), by
+// asynchronous 4-byte copies (cp.async) of the contiguous global block: the
+// caller keeps working and calls cp_async_wait_all() + __syncthreads() before
+// the reads.
 template <int K3>
-__device__ __forceinline__ void stage_sh(const float* __restrict__ sh, int64_t i0, int cnt,
-                                         float* __restrict__ s) {
+__device__ __forceinline__ void stage_sh_async(const float* __restrict__ sh, int64_t i0, int cnt,
+                                               float* __restrict__ s) {
   const float* src = sh + i0 * K3;
   const int total = cnt * K3;
   for (int e = threadIdx.x; e < total; e += kProjThreads) {
     const int i = e / K3, c = e - i * K3;
-    s[c * kShStride + i] = __ldg(&src[e]);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(&s[c * kShStride + i])),
+                 "l"(src + e)
+                 : "memory");
   }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 // Write staged values back to the contiguous global block (coalesced).
@@ -390,18 +401,20 @@ __global__ void __launch_bounds__(kProjThreads, 6) k_project_bwd(
   float* s_dsh = ALIAS ? s_pb : s_pb + K3 * kShStride;  // [K3][kShStride]
   const int64_t i0 = (int64_t)blockIdx.x * kProjThreads;
   const int cnt = (int)min((int64_t)kProjThreads, (int64_t)n - i0);
-  stage_sh<K3>(sh, i0, cnt, s_coef);
+  // the coefficients stream into shared memory while the parameters load and
+  // the view-independent part is computed
+  stage_sh_async<K3>(sh, i0, cnt, s_coef);
   if (!ALIAS) {
 #pragma unroll
     for (int c = 0; c < K3; ++c) s_dsh[c * kShStride + threadIdx.x] = 0.f;
   }
-  __syncthreads();
   const int i = (int)i0 + threadIdx.x;
-  if (i < n) {
-  const float4 m = __ldg(&means[i]);
-  const float4 ls = __ldg(&log_scales[i]);
-  const float4 q = __ldg(&quats[i]);
-  const float lg = __ldg(&logit[i]);
+  const bool live = i < n;
+  const int il = live ? i : (int)i0;  // a dead thread computes on a valid index, writes nothing
+  const float4 m = __ldg(&means[il]);
+  const float4 ls = __ldg(&log_scales[il]);
+  const float4 q = __ldg(&quats[il]);
+  const float lg = __ldg(&logit[il]);
 
   const float qn2 = q.x * q.x + q.y * q.y + q.z * q.z + q.w * q.w;
   const float qinv = rsqrtf(qn2);
@@ -421,7 +434,9 @@ __global__ void __launch_bounds__(kProjThreads, 6) k_project_bwd(
   float dopac = 0.f;
   const float* cf_t = s_coef + threadIdx.x;
   float* dsh_t = s_dsh + threadIdx.x;
-
+  cp_async_wait_all();
+  __syncthreads();
+  if (live) {
   bool touched = false;
   for (int v = 0; v < n_views; ++v) {
     if (radii[(size_t)v * n + i] <= 0) continue;
