@@ -409,24 +409,27 @@ def run_ours(args):
     n_pairs = int(sp.n_pairs.item())
     status = sp.status()
 
-    # end to end through the C calls from host buffers: the upstream gradient
-    # goes host -> device and the rendered image device -> host every step
+    # end to end through the library's host-fed step (Splatter.train_from_host):
+    # every step uploads its upstream gradient from pinned host memory and
+    # downloads the rendered image to it, on a copy stream overlapping the
+    # compute stream
     e2e = None
     if not args.no_e2e:
         h_in = torch.from_numpy(dL_host).pin_memory()
         h_out = torch.empty(sp.image.shape, dtype=torch.float32).pin_memory()
+        sp.stream = torch.cuda.Stream()
+        hook = (lambda: gdist.allreduce_grads(sp.grad_flat)) if world > 1 else None
+        sp.train_from_host([h_in] * 3, [h_out] * 3, grad_hook=hook)  # warm-up
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
+        e0.record(sp.stream)
+        sp.train_from_host([h_in] * args.steps, [h_out] * args.steps, grad_hook=hook)
+        e1.record(sp.stream)
         torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(args.steps):
-            dL.copy_(h_in, non_blocking=True)
-            step()
-            h_out.copy_(sp.image, non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize()
+        sp.stream = None
         e_ms = gdist.max_over_ranks(e0.elapsed_time(e1) / args.steps, device="cuda")
         e2e = {"value": world * pixels / (e_ms / 1000.0) / 1e6, "unit": "Mpix/s",
                "ms_per_step": e_ms, "h2d_bytes_per_step": int(h_in.numel() * 4),

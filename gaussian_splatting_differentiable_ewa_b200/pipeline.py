@@ -159,5 +159,66 @@ class Splatter:
         if adam:
             self.adam_step()
 
+    def train_from_host(self, dL_host, image_host, adam: bool = True, grad_hook=None) -> None:
+        """Training steps fed from host memory, copies overlapped with compute.
+
+        Step k uploads ``dL_host[k]`` (pinned, [V][3][H][W] float32), runs one
+        training step and downloads the rendered image into ``image_host[k]``
+        (pinned). The copies run on a second stream: step k + 1's gradient
+        uploads (into the other of two device buffers) while step k computes,
+        and step k's image downloads while its backward runs; events order the
+        next forward after that download and each upload after the backward
+        that last read its buffer. Everything is enqueued; the caller
+        synchronises. ``self.stream`` must be a stream other than the legacy
+        default stream (which would serialise the two). ``grad_hook()``, if
+        given, runs on the compute stream between the backward and the
+        statistics (e.g. the gradient all-reduce of a multi-GPU step)."""
+        comp = self.stream
+        if comp is None:
+            raise ValueError("train_from_host needs Splatter(stream=...) on a created stream")
+        n = len(dL_host)
+        if n != len(image_host):
+            raise ValueError("one image buffer per gradient")
+        if getattr(self, "_copy_stream", None) is None:
+            self._copy_stream = torch.cuda.Stream(device=self.device)
+            self._dL_dev = [torch.empty((self.V, 3, self.H, self.W), dtype=torch.float32,
+                                        device=self.device) for _ in range(2)]
+        cs = self._copy_stream
+        uploaded = [torch.cuda.Event(), torch.cuda.Event()]
+        consumed = [torch.cuda.Event(), torch.cuda.Event()]
+        rendered = torch.cuda.Event()
+        downloaded = torch.cuda.Event()
+        cs.wait_stream(comp)  # nothing earlier on the compute stream is overtaken
+        with torch.cuda.stream(cs):
+            self._dL_dev[0].copy_(dL_host[0], non_blocking=True)
+            uploaded[0].record(cs)
+        for k in range(n):
+            buf = k & 1
+            self.project()
+            self.bin_sort()
+            if k > 0:
+                comp.wait_event(downloaded)  # the previous image has left
+            self.rasterize_fwd()
+            rendered.record(comp)
+            cs.wait_event(rendered)
+            with torch.cuda.stream(cs):
+                image_host[k].copy_(self.image, non_blocking=True)
+                downloaded.record(cs)
+                if k + 1 < n:
+                    if k >= 1:
+                        cs.wait_event(consumed[buf ^ 1])  # step k - 1's backward is done with it
+                    self._dL_dev[buf ^ 1].copy_(dL_host[k + 1], non_blocking=True)
+                    uploaded[buf ^ 1].record(cs)
+            comp.wait_event(uploaded[buf])
+            self.rasterize_bwd(self._dL_dev[buf])
+            consumed[buf].record(comp)
+            if grad_hook is not None:
+                with torch.cuda.stream(comp):
+                    grad_hook()
+            self.densify_stats()
+            if adam:
+                self.adam_step()
+        comp.wait_event(downloaded)  # the last image is on the host when comp is done
+
     def status(self) -> int:
         return api.gs_get_status(self.ws, self.stream)
