@@ -248,3 +248,94 @@ def render_all(scene, projs=None, bg=None, tol_alpha=0.0, tol_T=0.0):
         outs.append((pix, render(projs, scene.cameras, scene.background if bg is None else bg,
                                  pix, tol_alpha, tol_T)))
     return outs
+
+
+# --------------------------------------------------------------- densify_and_prune
+
+DP_PRUNE, DP_KEEP, DP_CLONE, DP_SPLIT = 0, 1, 2, 3
+PARAM_NAMES = ("means", "log_scales", "quats", "opacity_logit", "sh")
+
+
+def _rotate(q, u):
+    """u rotated by the unit quaternion q = (w, x, y, z): the sandwich product
+    q (0, u) q*, written as u + 2w (v x u) + 2 v x (v x u) with v = (x, y, z)."""
+    w = q[..., :1]
+    v = q[..., 1:]
+    t = 2.0 * np.cross(v, u)
+    return u + w * t + np.cross(v, t)
+
+
+def densify_decisions(log_scales, opacity_logit, accum, denom, grad_threshold, log_scale_split,
+                      logit_min_opacity, log_max_scale):
+    """Per-Gaussian decision of densify_and_prune (absolute-gradient
+    densification page, sec. 1 and 3.3: the average gradient accum / denom
+    against a threshold; clone a small Gaussian, split a large one, prune a
+    faint or oversized one). Taken in float32 like the kernel: the gradient
+    test as accum > threshold * denom (denom > 0), the scale and opacity tests
+    on the raw log-scale and logit against float32 thresholds. Pruning wins.
+    Returns the codes DP_PRUNE / DP_KEEP / DP_CLONE / DP_SPLIT."""
+    f = np.float32
+    ls = np.asarray(log_scales, f)
+    lg = np.asarray(opacity_logit, f).reshape(-1)
+    acc = np.asarray(accum, f).reshape(-1)
+    den = np.asarray(denom).reshape(-1)
+    max_ls = ls.max(axis=1)
+    hot = (den > 0) & (acc > f(grad_threshold) * den.astype(f))
+    large = max_ls > f(log_scale_split)
+    prune = (lg < f(logit_min_opacity)) | (max_ls > f(log_max_scale))
+    code = np.full(len(lg), DP_KEEP, np.int32)
+    code[hot & ~large] = DP_CLONE
+    code[hot & large] = DP_SPLIT
+    code[prune] = DP_PRUNE
+    return code
+
+
+def densify_and_prune(params: dict, moments: dict, accum, denom, z, grad_threshold,
+                      log_scale_split, logit_min_opacity, log_max_scale,
+                      split_shrink: float = 1.6):
+    """densify_and_prune in float64, Gaussian by Gaussian in index order:
+      prune -> nothing;  keep -> the Gaussian (its Adam moments kept);
+      clone -> the Gaussian, then an exact copy (moments zero);
+      split -> two children c = 0, 1 (moments zero): mean + R (s * z[i, c]),
+               log-scale - ln(split_shrink), everything else copied;
+    R the rotation of the normalised quaternion, s = exp(log-scale), z the
+    caller's standard normal draws [N][2][3].
+    params: name -> array [N, ...]; moments: name -> (m, v) of the same shapes.
+    Returns (params_out, moments_out, codes)."""
+    code = densify_decisions(params["log_scales"], params["opacity_logit"], accum, denom,
+                             grad_threshold, log_scale_split, logit_min_opacity, log_max_scale)
+    P = {k: np.asarray(params[k], np.float64) for k in PARAM_NAMES}
+    n = len(code)
+    z = np.asarray(z, np.float64).reshape(n, 2, 3)
+    q = P["quats"] / np.linalg.norm(P["quats"], axis=1, keepdims=True)
+    s = np.exp(P["log_scales"])
+    out = {k: [] for k in PARAM_NAMES}
+    mom = {k: ([], []) for k in PARAM_NAMES}
+    for i in range(n):
+        c = code[i]
+        if c == DP_PRUNE:
+            continue
+        if c in (DP_KEEP, DP_CLONE):
+            for k in PARAM_NAMES:
+                out[k].append(P[k][i])
+                mom[k][0].append(np.asarray(moments[k][0], np.float64)[i])
+                mom[k][1].append(np.asarray(moments[k][1], np.float64)[i])
+        if c == DP_CLONE:
+            for k in PARAM_NAMES:
+                out[k].append(P[k][i])
+                mom[k][0].append(np.zeros_like(P[k][i]))
+                mom[k][1].append(np.zeros_like(P[k][i]))
+        if c == DP_SPLIT:
+            for ch in range(2):
+                child = {k: P[k][i].copy() for k in PARAM_NAMES}
+                child["means"] = P["means"][i] + _rotate(q[i], s[i] * z[i, ch])
+                child["log_scales"] = P["log_scales"][i] - np.log(split_shrink)
+                for k in PARAM_NAMES:
+                    out[k].append(child[k])
+                    mom[k][0].append(np.zeros_like(P[k][i]))
+                    mom[k][1].append(np.zeros_like(P[k][i]))
+    shapes = {k: P[k].shape[1:] for k in PARAM_NAMES}
+    params_out = {k: (np.array(out[k]).reshape((-1,) + shapes[k])) for k in PARAM_NAMES}
+    moments_out = {k: (np.array(mom[k][0]).reshape((-1,) + shapes[k]),
+                       np.array(mom[k][1]).reshape((-1,) + shapes[k])) for k in PARAM_NAMES}
+    return params_out, moments_out, code

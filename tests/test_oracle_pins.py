@@ -472,3 +472,95 @@ def test_adam_closed_forms():
     np.testing.assert_allclose(p2, p1 - lr * m_hat / (np.sqrt(v_hat) + eps), rtol=1e-12)
     p3, _, _ = O.adam(p0, np.zeros(100), z, z, lr, 1)
     assert np.array_equal(p3, p0)
+
+
+# ------------------------------------------------------------ densify_and_prune
+
+def _dp_set(n, K=1, seed=0):
+    rng = np.random.default_rng(seed)
+    params = dict(means=rng.normal(size=(n, 3)), log_scales=rng.uniform(-4, -1, (n, 3)),
+                  quats=rng.normal(size=(n, 4)), opacity_logit=rng.normal(size=n),
+                  sh=rng.normal(size=(n, K, 3)))
+    params = {k: v.astype(np.float32).astype(np.float64) for k, v in params.items()}
+    moments = {k: (rng.normal(size=v.shape), rng.random(v.shape)) for k, v in params.items()}
+    return params, moments
+
+
+def test_dp_rotation_is_the_axis_angle_rotation():
+    # the sandwich product agrees with Rodrigues' formula for angle t about a
+    rng = np.random.default_rng(3)
+    for _ in range(20):
+        a = rng.normal(size=3)
+        a /= np.linalg.norm(a)
+        t = rng.uniform(-np.pi, np.pi)
+        q = np.concatenate([[np.cos(t / 2)], np.sin(t / 2) * a])
+        u = rng.normal(size=3)
+        rod = u * np.cos(t) + np.cross(a, u) * np.sin(t) + a * np.dot(a, u) * (1 - np.cos(t))
+        np.testing.assert_allclose(O._rotate(q, u), rod, atol=1e-12)
+
+
+def test_dp_split_child_closed_form():
+    params, moments = _dp_set(1)
+    params["quats"][0] = [3.0, 0.0, 0.0, 0.0]          # identity after normalisation
+    params["log_scales"][0] = np.log([2.0, 1.0, 0.5])
+    params["opacity_logit"][0] = 2.0
+    z = np.array([[[1.0, -1.0, 2.0], [0.0, 0.5, 0.0]]])
+    out, mom, code = O.densify_and_prune(params, moments, [1.0], [1], z, 0.5,
+                                         np.log(1.5), -10.0, 10.0)
+    assert code.tolist() == [O.DP_SPLIT]
+    mu = params["means"][0]
+    np.testing.assert_allclose(out["means"], [mu + [2.0, -1.0, 1.0], mu + [0.0, 0.5, 0.0]],
+                               atol=1e-12)
+    np.testing.assert_allclose(out["log_scales"],
+                               np.log([[1.25, 0.625, 0.3125]] * 2), atol=1e-12)
+    for k in ("quats", "opacity_logit", "sh"):
+        assert np.array_equal(out[k], np.stack([params[k][0]] * 2))
+        assert not mom[k][0].any() and not mom[k][1].any()
+
+
+def test_dp_decisions_order_copies_and_moments():
+    # 0 keep (cold), 1 clone (hot, small), 2 split (hot, large), 3 prune (faint),
+    # 4 prune beats split (hot, large, faint), 5 keep (never seen: denom 0),
+    # 6 prune (oversized)
+    params, moments = _dp_set(7, K=4)
+    small, large = np.log(0.01), np.log(0.2)
+    params["log_scales"][:] = small
+    params["log_scales"][[2, 4], 1] = large
+    params["log_scales"][6, 2] = np.log(5.0)
+    params["opacity_logit"][:] = 1.0
+    params["opacity_logit"][[3, 4]] = -8.0
+    accum = np.array([0.1, 3.0, 3.0, 3.0, 3.0, 3.0, 0.1])
+    denom = np.array([1, 2, 2, 2, 2, 0, 1])
+    z = np.random.default_rng(1).normal(size=(7, 2, 3))
+    out, mom, code = O.densify_and_prune(params, moments, accum, denom, z, 1.0, np.log(0.1),
+                                         -5.0, np.log(1.0))
+    assert code.tolist() == [O.DP_KEEP, O.DP_CLONE, O.DP_SPLIT, O.DP_PRUNE, O.DP_PRUNE,
+                             O.DP_KEEP, O.DP_PRUNE]
+    # layout: g0, g1, g1 (clone), child 2a, child 2b, g5
+    assert len(out["means"]) == 6
+    for k in O.PARAM_NAMES:
+        for row, src in ((0, 0), (1, 1), (2, 1), (5, 5)):
+            assert np.array_equal(out[k][row], params[k][src]), (k, row)
+        for row, src in ((0, 0), (1, 1), (5, 5)):                 # kept: moments kept
+            assert np.array_equal(mom[k][0][row], moments[k][0][src])
+            assert np.array_equal(mom[k][1][row], moments[k][1][src])
+        for row in (2, 3, 4):                                       # new: moments zero
+            assert not mom[k][0][row].any() and not mom[k][1][row].any()
+    # children: the scales shrink by 1.6, the offsets are R (s * z)
+    assert np.allclose(out["log_scales"][3], params["log_scales"][2] - np.log(1.6))
+    d = out["means"][3:5] - params["means"][2]
+    assert np.allclose(np.linalg.norm(d, axis=1),
+                       np.linalg.norm(np.exp(params["log_scales"][2]) * z[2], axis=1))
+
+
+def test_dp_threshold_is_strict_and_exact_in_float32():
+    # accum == threshold * denom exactly is not above it; one ulp more is
+    params, moments = _dp_set(2)
+    params["log_scales"][:] = -5.0
+    params["opacity_logit"][:] = 0.0
+    thr = np.float32(0.0002)
+    acc = np.array([np.float32(thr * np.float32(3)),
+                    np.nextafter(np.float32(thr * np.float32(3)), np.float32(1))])
+    code = O.densify_decisions(params["log_scales"], params["opacity_logit"], acc, [3, 3],
+                               thr, np.log(0.1), -10.0, 10.0)
+    assert code.tolist() == [O.DP_KEEP, O.DP_CLONE]
