@@ -305,6 +305,8 @@ def densify_and_prune(params: dict, moments: dict, accum, denom, z, grad_thresho
     code = densify_decisions(params["log_scales"], params["opacity_logit"], accum, denom,
                              grad_threshold, log_scale_split, logit_min_opacity, log_max_scale)
     P = {k: np.asarray(params[k], np.float64) for k in PARAM_NAMES}
+    Mo = {k: (np.asarray(moments[k][0], np.float64), np.asarray(moments[k][1], np.float64))
+          for k in PARAM_NAMES}
     n = len(code)
     z = np.asarray(z, np.float64).reshape(n, 2, 3)
     q = P["quats"] / np.linalg.norm(P["quats"], axis=1, keepdims=True)
@@ -318,8 +320,8 @@ def densify_and_prune(params: dict, moments: dict, accum, denom, z, grad_thresho
         if c in (DP_KEEP, DP_CLONE):
             for k in PARAM_NAMES:
                 out[k].append(P[k][i])
-                mom[k][0].append(np.asarray(moments[k][0], np.float64)[i])
-                mom[k][1].append(np.asarray(moments[k][1], np.float64)[i])
+                mom[k][0].append(Mo[k][0][i])
+                mom[k][1].append(Mo[k][1][i])
         if c == DP_CLONE:
             for k in PARAM_NAMES:
                 out[k].append(P[k][i])
