@@ -324,6 +324,49 @@ def run_reference(args):
 
 # ----------------------------------------------------------------- our path
 
+def measure_densify(sp) -> dict:
+    """One gs_densify_and_prune call on the Splatter's accumulated statistics
+    (absolute gradients, the page's threshold 0.0002), timed with CUDA events
+    after an untimed call. Algorithmic bytes: 59 real floats of parameters,
+    Adam m and v read per Gaussian plus its statistics and draws, and the same
+    59 x 3 floats written per output Gaussian."""
+    import torch
+    from gaussian_splatting_differentiable_ewa_b200 import api
+    n = sp.n
+    names = [k for k, _ in sp.param_list]
+    like = lambda t: torch.empty((2 * n,) + tuple(t.shape[1:]), dtype=t.dtype,  # noqa: E731
+                                 device=t.device)
+    out = [like(t) for _, t in sp.param_list]
+    m_out = [like(t) for _, t in sp.param_list]
+    v_out = [like(t) for _, t in sp.param_list]
+    n_out = torch.zeros(1, dtype=torch.int64, device="cuda")
+    codes = torch.empty(n, dtype=torch.int8, device="cuda")
+    ws = torch.zeros((api.gs_densify_workspace_size(n) + 255) // 256 * 256 // 8,
+                     dtype=torch.int64, device="cuda")
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(0)
+    z = torch.randn((n, 2, 3), generator=gen, device="cuda")
+    dp = api.densify_params(0.0002, 0.05, 0.005, 1.0)
+    args = (sp.c_params, api.grads(*[sp.exp_avg[k] for k in names]),
+            api.grads(*[sp.exp_avg_sq[k] for k in names]), sp.accum_abs, sp.denom, z, dp,
+            api.grads(*out), api.grads(*m_out), api.grads(*v_out), 2 * n, n_out, codes, ws)
+    api.gs_densify_and_prune(*args)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    api.gs_densify_and_prune(*args)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    m = int(n_out.item())
+    counts = torch.bincount(codes.long(), minlength=4).cpu().tolist()
+    nbytes = n * (59 * 4 * 3 + 4 + 4 + 24) + m * 59 * 4 * 3
+    pk = peaks()
+    return dict(ms=ms, gbs=nbytes / (ms / 1e3) / 1e9,
+                hbm_frac=nbytes / (ms / 1e3) / 1e9 / pk["hbm_gbs"], n_in=n, n_out=m,
+                pruned=counts[0], kept=counts[1], cloned=counts[2], split=counts[3])
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -435,6 +478,12 @@ def run_ours(args):
                "ms_per_step": e_ms, "h2d_bytes_per_step": int(h_in.numel() * 4),
                "d2h_bytes_per_step": int(h_out.numel() * 4)}
 
+    # densify_and_prune once, on the statistics the timed steps accumulated
+    # (not part of the step: it runs every few hundred steps)
+    extras = {}
+    if world == 1:
+        extras["gs_densify_and_prune"] = measure_densify(sp)
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -497,6 +546,7 @@ def run_ours(args):
         "roofline": roof,
         "step_roofline": {"bound_ms": bound_s * 1000.0, "frac": bound_s * 1000.0 / ms},
         "kernels": kernels,
+        "extras": extras,
         "cpu_baseline": None if cpu is None else {k: cpu[k] for k in
                                                   ("value", "unit", "cores", "kind", "sample")},
         "e2e": e2e,

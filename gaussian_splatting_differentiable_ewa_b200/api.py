@@ -67,6 +67,12 @@ class GsAdamGroup(_c.Structure):
                 ("count", _c.c_int64), ("lr", _c.c_float), ("reserved", _c.c_float)]
 
 
+class GsDensifyParams(_c.Structure):
+    _fields_ = [("grad_threshold", _c.c_float), ("log_scale_split", _c.c_float),
+                ("logit_min_opacity", _c.c_float), ("log_max_scale", _c.c_float),
+                ("log_split_shrink", _c.c_float), ("reserved", _c.c_int32)]
+
+
 # (name, restype, argtypes) for every symbol gs.h declares
 SIGNATURES = [
     ("gs_abi_version", _c.c_int32, []),
@@ -93,6 +99,11 @@ SIGNATURES = [
     ("gs_adam_step", _c.c_int,
      [_c.POINTER(GsAdamGroup), _c.c_int32, _c.c_float, _c.c_float, _c.c_float, _c.c_int64, _vp]),
     ("gs_get_status", _c.c_int, [_vp, _vp]),
+    ("gs_densify_workspace_size", _c.c_size_t, [_c.c_int64]),
+    ("gs_densify_and_prune", _c.c_int,
+     [_c.POINTER(GsParams), _c.POINTER(GsGrads), _c.POINTER(GsGrads), _vp, _vp, _vp,
+      _c.POINTER(GsDensifyParams), _c.POINTER(GsGrads), _c.POINTER(GsGrads), _c.POINTER(GsGrads),
+      _c.c_int64, _vp, _vp, _vp, _c.c_size_t, _vp]),
     ("gs_bin_sort_noalloc", _c.c_int,
      [_c.POINTER(GsProjected), _c.POINTER(GsCamera), _c.c_int32, _c.c_int64, _c.c_int32,
       _c.POINTER(GsBinned), _vp, _vp]),
@@ -252,6 +263,30 @@ def gs_adam_step(groups: Sequence[tuple], beta1: float, beta2: float, eps: float
 
 def gs_get_status(ws, stream=None) -> int:
     return int(lib().gs_get_status(_ptr(ws), _stream(stream)))
+
+
+def densify_params(grad_threshold: float, scale_split: float, min_opacity: float,
+                   max_scale: float, split_shrink: float = 1.6) -> GsDensifyParams:
+    """Thresholds in the units of the call: log-scales and a logit (float32)."""
+    import math
+    return GsDensifyParams(float(grad_threshold), float(math.log(scale_split)),
+                           float(math.log(min_opacity / (1.0 - min_opacity))),
+                           float(math.log(max_scale)), float(math.log(split_shrink)), 0)
+
+
+def gs_densify_workspace_size(n: int) -> int:
+    return int(lib().gs_densify_workspace_size(int(n)))
+
+
+def gs_densify_and_prune(params: GsParams, m_in: GsGrads, v_in: GsGrads, accum, denom, z,
+                         dp: GsDensifyParams, out: GsGrads, m_out: GsGrads, v_out: GsGrads,
+                         out_capacity: int, n_out, codes, ws, stream=None) -> None:
+    _check(lib().gs_densify_and_prune(_c.byref(params), _c.byref(m_in), _c.byref(v_in),
+                                      _ptr(accum), _ptr(denom), _ptr(z), _c.byref(dp),
+                                      _c.byref(out), _c.byref(m_out), _c.byref(v_out),
+                                      int(out_capacity), _ptr(n_out), _ptr(codes), _ptr(ws),
+                                      int(ws.numel() * ws.element_size()), _stream(stream)),
+           "gs_densify_and_prune")
 
 
 def gs_bin_sort_noalloc(proj: GsProjected, cams_arr, n_views: int, n: int, sort_mode: int,

@@ -419,6 +419,59 @@ gs_status gs_bin_sort_noalloc(const gs_projected* proj, const gs_camera* cams, i
   return GS_OK;
 }
 
+size_t gs_densify_workspace_size(int64_t n) {
+  if (n < 0 || n >= (1ll << 31)) return 0;
+  size_t off = kControlBytes;
+  off = align_up(off + (size_t)densify_blocks(n) * sizeof(uint32_t));
+  off = align_up(off + (size_t)n);  // codes, when the caller passes none
+  return off;
+}
+
+namespace {
+bool dp_tensors(const gs_grads* g, bool need, gsb::DpTensorPtrs& t) {
+  if (!g) return !need;
+  t = gsb::DpTensorPtrs{g->means, g->log_scales, g->quats, g->opacity_logit, g->sh};
+  return t.means && t.log_scales && t.quats && t.logit && t.sh && aligned(t.means, 16) &&
+         aligned(t.log_scales, 16) && aligned(t.quats, 16) && aligned(t.sh, 16);
+}
+}  // namespace
+
+gs_status gs_densify_and_prune(const gs_params* in, const gs_grads* m_in, const gs_grads* v_in,
+                               const float* accum, const int32_t* denom, const float* z,
+                               const gs_densify_params* dp, gs_grads* out, gs_grads* m_out,
+                               gs_grads* v_out, int64_t out_capacity, int64_t* n_out,
+                               int8_t* codes, void* ws, size_t ws_bytes, void* stream) {
+  if (!in || !dp || !n_out || !ws || !m_in || !v_in || !out || !m_out || !v_out)
+    return GS_ERR_INVALID_ARG;
+  if (in->n < 0 || in->sh_degree < 0 || in->sh_degree > 3 || out_capacity < 0)
+    return GS_ERR_INVALID_ARG;
+  if (in->n >= (1ll << 31) || out_capacity >= (1ll << 31)) return GS_ERR_OVERFLOW;
+  const size_t need = gs_densify_workspace_size(in->n);
+  if (ws_bytes < need || !aligned(ws, kAlign)) return GS_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int n = (int)in->n;
+  if (n == 0) return cuda_status(cudaMemsetAsync(n_out, 0, sizeof(int64_t), st));
+  gs_grads pin{const_cast<float*>(in->means), const_cast<float*>(in->log_scales),
+               const_cast<float*>(in->quats), const_cast<float*>(in->opacity_logit),
+               const_cast<float*>(in->sh)};
+  gsb::DpTensorPtrs tp, tm, tv, op, om, ov;
+  if (!dp_tensors(&pin, true, tp) || !dp_tensors(m_in, true, tm) || !dp_tensors(v_in, true, tv) ||
+      !dp_tensors(out, true, op) || !dp_tensors(m_out, true, om) || !dp_tensors(v_out, true, ov))
+    return GS_ERR_INVALID_ARG;
+  if (!accum || !denom || !z) return GS_ERR_INVALID_ARG;
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  uint32_t* block_counts = reinterpret_cast<uint32_t*>(w + kControlBytes);
+  int8_t* code_buf = codes ? codes
+                           : reinterpret_cast<int8_t*>(
+                                 w + align_up(kControlBytes + (size_t)densify_blocks(n) * 4));
+  gsb::DensifyArgs a{dp->grad_threshold, dp->log_scale_split, dp->logit_min_opacity,
+                     dp->log_max_scale, dp->log_split_shrink};
+  const int k3 = 3 * (in->sh_degree + 1) * (in->sh_degree + 1);
+  return cuda_status(gsb::launch_densify_and_prune(
+      tp, tm, tv, accum, denom, z, n, k3, a, code_buf, block_counts, out_capacity, n_out,
+      reinterpret_cast<uint32_t*>(w + kStatusOffset), op, om, ov, st));
+}
+
 gs_status gs_get_status(void* ws, void* stream) {
   if (!ws) return GS_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -88,4 +88,29 @@ bool tile_emission(const Grid& g);          // presort mode places pairs directl
 int tile_gsize(int64_t n);                  // tile emission: Gaussians per block
 int64_t emit_blocks(int64_t items);
 
+// densify_and_prune (densify.cu)
+struct DensifyArgs {
+  float grad_threshold;     // densify when accum > grad_threshold * denom, denom > 0
+  float log_scale_split;    // split when the largest log-scale exceeds this, else clone
+  float logit_min_opacity;  // prune when the opacity logit is below this
+  float log_max_scale;      // prune when the largest log-scale exceeds this
+  float log_split_shrink;   // a child's log-scales are the parent's minus this
+};
+struct DpTensorPtrs {       // the five parameter-shaped arrays (params, moments)
+  float* means;             // float4 [n]
+  float* log_scales;        // float4 [n]
+  float* quats;             // float4 [n]
+  float* logit;             // [n]
+  float* sh;                // [n][K][3]
+};
+int64_t densify_blocks(int64_t n);
+cudaError_t launch_densify_and_prune(const DpTensorPtrs& p_in, const DpTensorPtrs& m_in,
+                                     const DpTensorPtrs& v_in, const float* accum,
+                                     const int32_t* denom, const float* z, int n, int k3,
+                                     const DensifyArgs& args, int8_t* codes,
+                                     uint32_t* block_counts, int64_t capacity, int64_t* n_out,
+                                     uint32_t* status, const DpTensorPtrs& p_out,
+                                     const DpTensorPtrs& m_out, const DpTensorPtrs& v_out,
+                                     cudaStream_t stream);
+
 }  // namespace gsb

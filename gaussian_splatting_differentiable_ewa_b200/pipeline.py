@@ -46,21 +46,37 @@ class Splatter:
             t = torch.as_tensor(np.ascontiguousarray(a, np.float32))
             return (t if shape is None else t.reshape(shape)).to(dev).contiguous()
 
-        self.means = up(scene.means)
-        self.log_scales = up(scene.log_scales)
-        self.quats = up(scene.quats)
-        self.opacity_logit = up(scene.opacity_logit)
-        self.sh = up(scene.sh, (self.n, self.K, 3))
-        self.param_list = [("means", self.means), ("log_scales", self.log_scales),
-                           ("quats", self.quats), ("opacity_logit", self.opacity_logit),
-                           ("sh", self.sh)]
-        n, V = self.n, self.V
-        self.records = torch.empty((V, n, api.GS_RECORD_FLOATS), dtype=f32, device=dev)
-        self.bins = torch.empty((V, n, 4), dtype=f32, device=dev)
-        self.radii = torch.empty((V, n), dtype=torch.int32, device=dev)
+        self._alloc_gaussians(up(scene.means), up(scene.log_scales), up(scene.quats),
+                              up(scene.opacity_logit), up(scene.sh, (self.n, self.K, 3)))
+        V = self.V
         self.image = torch.empty((V, 3, self.H, self.W), dtype=f32, device=dev)
         self.final_T = torch.empty((V, self.H, self.W), dtype=f32, device=dev)
         self.n_contrib = torch.empty((V, self.H, self.W), dtype=torch.int32, device=dev)
+        tiles = ((self.W + 15) // 16) * ((self.H + 15) // 16) * V
+        self.ranges = torch.empty((tiles, 2), dtype=torch.int64, device=dev)
+        self.n_pairs = torch.zeros(1, dtype=torch.int64, device=dev)
+        self.capacity = 0
+        self.ids = None
+        self.ws = None
+        self.step_count = 0
+        self._alloc_pairs(int(pair_capacity) if pair_capacity is not None else 0)
+
+    # ------------------------------------------------------------ buffers
+    def _alloc_gaussians(self, means, log_scales, quats, opacity_logit, sh, exp_avg=None,
+                         exp_avg_sq=None) -> None:
+        """Adopt the given parameter tensors (and Adam moments, zero if None) and
+        (re)allocate every buffer whose size follows the Gaussian count."""
+        dev, f32 = self.device, torch.float32
+        self.means, self.log_scales, self.quats = means, log_scales, quats
+        self.opacity_logit, self.sh = opacity_logit, sh
+        self.n = n = int(means.shape[0])
+        V = self.V
+        self.param_list = [("means", self.means), ("log_scales", self.log_scales),
+                           ("quats", self.quats), ("opacity_logit", self.opacity_logit),
+                           ("sh", self.sh)]
+        self.records = torch.empty((V, n, api.GS_RECORD_FLOATS), dtype=f32, device=dev)
+        self.bins = torch.empty((V, n, 4), dtype=f32, device=dev)
+        self.radii = torch.empty((V, n), dtype=torch.int32, device=dev)
         self.grad2d = torch.empty((V, n, api.GS_GRAD2D_FLOATS), dtype=f32, device=dev)
         # gradients live in one flat buffer (one all-reduce across ranks), each
         # group at a 16-byte aligned offset
@@ -71,25 +87,20 @@ class Splatter:
         self.grad_flat = torch.zeros(max(total, 4), dtype=f32, device=dev)
         self.grads = {k: self.grad_flat[offs[k]:offs[k] + t.numel()].view(t.shape)
                       for k, t in self.param_list}
-        self.exp_avg = {k: torch.zeros_like(t) for k, t in self.param_list}
-        self.exp_avg_sq = {k: torch.zeros_like(t) for k, t in self.param_list}
+        self.exp_avg = (exp_avg if exp_avg is not None
+                        else {k: torch.zeros_like(t) for k, t in self.param_list})
+        self.exp_avg_sq = (exp_avg_sq if exp_avg_sq is not None
+                           else {k: torch.zeros_like(t) for k, t in self.param_list})
         self.accum_plain = torch.zeros(n, dtype=f32, device=dev)
         self.accum_abs = torch.zeros(n, dtype=f32, device=dev)
         self.denom = torch.zeros(n, dtype=torch.int32, device=dev)
-        tiles = ((self.W + 15) // 16) * ((self.H + 15) // 16) * V
-        self.ranges = torch.empty((tiles, 2), dtype=torch.int64, device=dev)
-        self.n_pairs = torch.zeros(1, dtype=torch.int64, device=dev)
-        self.capacity = 0
-        self.ids = None
-        self.ws = None
-        self.step_count = 0
         self.c_params = api.params(self.means, self.log_scales, self.quats, self.opacity_logit,
                                    self.sh, self.deg)
         self.c_grads = api.grads(*[self.grads[k] for k, _ in self.param_list])
         self.c_proj = api.projected(self.records, self.bins, self.radii)
-        self._alloc_pairs(int(pair_capacity) if pair_capacity is not None else 0)
+        if getattr(self, "ws", None) is not None:
+            self._alloc_pairs(self.capacity)  # the workspace follows the count too
 
-    # ------------------------------------------------------------ buffers
     def _alloc_pairs(self, capacity: int) -> None:
         self.capacity = int(capacity)
         self.ids = torch.empty(max(self.capacity, 1), dtype=torch.int32, device=self.device)
@@ -219,6 +230,54 @@ class Splatter:
             if adam:
                 self.adam_step()
         comp.wait_event(downloaded)  # the last image is on the host when comp is done
+
+    def densify_and_prune(self, grad_threshold: float = 0.0002, scale_split: float = 0.05,
+                          min_opacity: float = 0.005, max_scale: float = 1.0,
+                          split_shrink: float = 1.6, use_abs: bool = True, z=None,
+                          seed: int = 0) -> torch.Tensor:
+        """Clone, split and prune (gs_densify_and_prune) with this Splatter's
+        accumulated view-space gradient statistics (the absolute ones when
+        use_abs, else the plain ones), then adopt the new Gaussian set: every
+        per-Gaussian buffer is reallocated and the statistics restart from
+        zero. z: standard normal draws float32 [n][2][3] for the split
+        children (drawn on the device from `seed` when None). Returns the
+        per-Gaussian codes (0 pruned, 1 kept, 2 cloned, 3 split)."""
+        n, dev = self.n, self.device
+        if z is None:
+            gen = torch.Generator(device=dev)
+            gen.manual_seed(int(seed))
+            z = torch.randn((n, 2, 3), generator=gen, device=dev, dtype=torch.float32)
+        cap = 2 * n
+        names = [k for k, _ in self.param_list]
+
+        def like(t):
+            return torch.empty((cap,) + tuple(t.shape[1:]), dtype=t.dtype, device=dev)
+
+        out = {k: like(t) for k, t in self.param_list}
+        m_out = {k: like(t) for k, t in self.param_list}
+        v_out = {k: like(t) for k, t in self.param_list}
+        n_out = torch.zeros(1, dtype=torch.int64, device=dev)
+        codes = torch.empty(max(n, 1), dtype=torch.int8, device=dev)
+        ws = torch.zeros((api.gs_densify_workspace_size(n) + 255) // 256 * 256 // 8,
+                         dtype=torch.int64, device=dev)
+        dp = api.densify_params(grad_threshold, scale_split, min_opacity, max_scale, split_shrink)
+        api.gs_densify_and_prune(self.c_params,
+                                 api.grads(*[self.exp_avg[k] for k in names]),
+                                 api.grads(*[self.exp_avg_sq[k] for k in names]),
+                                 self.accum_abs if use_abs else self.accum_plain, self.denom,
+                                 z, dp, api.grads(*[out[k] for k in names]),
+                                 api.grads(*[m_out[k] for k in names]),
+                                 api.grads(*[v_out[k] for k in names]), cap, n_out, codes, ws,
+                                 self.stream)
+        st = api.gs_get_status(ws, self.stream)
+        if st != api.GS_OK:
+            raise api.GsError(st, "gs_densify_and_prune")
+        m = int(n_out.item())
+        keep = lambda d: {k: d[k][:m] for k in names}  # noqa: E731
+        o, mo, vo = keep(out), keep(m_out), keep(v_out)
+        self._alloc_gaussians(o["means"], o["log_scales"], o["quats"], o["opacity_logit"],
+                              o["sh"], mo, vo)
+        return codes[:n]
 
     def status(self) -> int:
         return api.gs_get_status(self.ws, self.stream)

@@ -296,6 +296,50 @@ gs_status gs_densify_stats(const float* grad2d, const int32_t* radii, int32_t n_
 gs_status gs_adam_step(const gs_adam_group* groups, int32_t n_groups, float beta1,
                        float beta2, float eps, int64_t step, void* stream);
 
+/* Thresholds of gs_densify_and_prune. The pages fix only the gradient
+ * threshold (0.0002 in the absolute-gradient tutorial's configuration); the
+ * other cut-offs are the caller's. Scale and opacity tests are taken on the
+ * raw parameters, so they are given as a log-scale and a logit. */
+typedef struct gs_densify_params {
+  float grad_threshold;     /* densify when accum > grad_threshold * denom, denom > 0 */
+  float log_scale_split;    /* a densifying Gaussian whose largest log-scale exceeds
+                               this is split, else cloned */
+  float logit_min_opacity;  /* prune when the opacity logit is below this */
+  float log_max_scale;      /* prune when the largest log-scale exceeds this */
+  float log_split_shrink;   /* a child's log-scales: the parent's minus this (ln 1.6) */
+  int32_t reserved;
+} gs_densify_params;
+
+/* Bytes of workspace gs_densify_and_prune needs for n Gaussians (256-byte
+ * aligned; the first 256 bytes hold the status word, as for gs_bin_sort). */
+size_t gs_densify_workspace_size(int64_t n);
+
+/* densify_and_prune (jsqmd.com sec. 1 and 3.3; pwwt.cn sec. 4.2). With the
+ * float32 decisions of gs_densify_params, Gaussian i (index order) becomes:
+ *   pruned (logit < logit_min_opacity or largest log-scale > log_max_scale;
+ *     pruning wins): nothing;
+ *   kept (not densifying): itself, with its Adam moments;
+ *   cloned (densifying, largest log-scale <= log_scale_split): itself with its
+ *     moments, then an exact copy with zero moments;
+ *   split (densifying, larger): two children with zero moments: child c's
+ *     mean is mean + R (exp(log-scale) * z[i][c]) (R the rotation of the
+ *     normalised quaternion, z the caller's standard normal draws,
+ *     float [n][2][3]); its log-scales are the parent's minus
+ *     log_split_shrink; quaternion, logit and SH are copied.
+ * The output Gaussians are compacted in that order into `out`, `m_out`,
+ * `v_out` (the layouts of gs_params, out_capacity Gaussians each; padding
+ * lanes copied); *n_out (device int64) always receives their number. If it
+ * exceeds out_capacity nothing is written and GS_ERR_CAPACITY is raised in
+ * the status word. accum is the view-space gradient accumulator of
+ * gs_densify_stats (plain or absolute), denom its visibility count. codes, if
+ * not NULL, receives int8 [n]: 0 pruned, 1 kept, 2 cloned, 3 split. Outputs
+ * must not overlap the inputs. */
+gs_status gs_densify_and_prune(const gs_params* in, const gs_grads* m_in, const gs_grads* v_in,
+                               const float* accum, const int32_t* denom, const float* z,
+                               const gs_densify_params* dp, gs_grads* out, gs_grads* m_out,
+                               gs_grads* v_out, int64_t out_capacity, int64_t* n_out,
+                               int8_t* codes, void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronise `stream`, return the status word accumulated in workspace `ws`
  * by device-side checks since the last call, and clear it. */
 gs_status gs_get_status(void* ws, void* stream);

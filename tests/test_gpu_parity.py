@@ -200,32 +200,53 @@ def test_backward_and_densify_match_oracle(name, kw, how):
 
 
 def test_train_from_host_matches_device_steps():
-    # host-fed steps with copies on a second stream give the same images and
-    # parameters as device-fed steps (up to the order of float atomic sums)
+    # host-fed steps (copies on a second stream) against device-fed ones
     sc = S.make_scene("fwd_100k_800", n=20000, width=792, height=600)
     c = sc.cameras[0]
-    dL = S.make_upstream_grad(1, c.height, c.width, seed=1)
     steps = 3
-    ref = Splatter(sc)
-    ref.ensure_capacity()
-    imgs = []
-    for _ in range(steps):
-        ref.train_step(torch.as_tensor(dL).cuda())
-        imgs.append(ref.image.cpu().numpy())
-    torch.cuda.synchronize()
-    sp = Splatter(sc, stream=torch.cuda.Stream())
-    sp.ensure_capacity()
-    h_in = [torch.from_numpy(dL).pin_memory() for _ in range(steps)]
-    h_out = [torch.empty(sp.image.shape, dtype=torch.float32).pin_memory() for _ in range(steps)]
-    sp.train_from_host(h_in, h_out)
-    torch.cuda.synchronize()
-    assert sp.status() == api.GS_OK
-    assert np.array_equal(h_out[0].numpy(), imgs[0])  # same parameters: same bits
+    dLs = [S.make_upstream_grad(1, c.height, c.width, seed=1 + k) for k in range(steps)]
+
+    def device_run(adam):
+        ref = Splatter(sc)
+        ref.ensure_capacity()
+        imgs = []
+        for k in range(steps):
+            ref.train_step(torch.as_tensor(dLs[k]).cuda(), adam=adam)
+            imgs.append(ref.image.cpu().numpy())
+        torch.cuda.synchronize()
+        return ref, imgs
+
+    def host_run(adam):
+        sp = Splatter(sc, stream=torch.cuda.Stream())
+        sp.ensure_capacity()
+        h_in = [torch.from_numpy(d).pin_memory() for d in dLs]
+        h_out = [torch.empty(sp.image.shape, dtype=torch.float32).pin_memory()
+                 for _ in range(steps)]
+        sp.train_from_host(h_in, h_out, adam=adam)
+        torch.cuda.synchronize()
+        assert sp.status() == api.GS_OK
+        return sp, [h.numpy() for h in h_out]
+
+    # fixed parameters: every image is the same bits, and the last step's
+    # gradients (from the last upload) agree to the rounding of their float
+    # atomic sums (~1e-5; another step's gradient would differ by ~1)
+    ref, imgs = device_run(False)
+    sp, outs = host_run(False)
+    for k in range(steps):
+        assert np.array_equal(outs[k], imgs[0])
+    for k in sp.grads:
+        assert P.rel_l2(sp.grads[k].cpu().numpy(), ref.grads[k].cpu().numpy()) < 1e-4, k
+    # with Adam the parameters move between steps (so a download racing the
+    # next forward would show); Adam turns the rounding of a near-zero
+    # gradient into a full +-lr step now and then, hence the loose bounds
+    ref, imgs = device_run(True)
+    sp, outs = host_run(True)
+    assert np.array_equal(outs[0], imgs[0])
     for k in range(1, steps):
-        assert np.abs(h_out[k].numpy() - imgs[k]).max() < 1e-4
+        d = np.abs(outs[k] - imgs[k])
+        assert d.mean() < 2e-5 and d.max() < 5e-2
     for k, t in sp.param_list:
-        r = dict(ref.param_list)[k]
-        assert P.rel_l2(t.cpu().numpy(), r.cpu().numpy()) < 1e-6, k
+        assert P.rel_l2(t.cpu().numpy(), dict(ref.param_list)[k].cpu().numpy()) < 1e-3, k
 
 
 def test_adam_matches_oracle_on_generated_inputs():
@@ -340,3 +361,113 @@ def test_single_gaussian_centred_on_pixel_gives_o_c():
     rgb = 0.5 + 0.28209479177387814 * np.array([0.3, -0.2, 0.4])
     got = sp.image.cpu().numpy()[0, :, 17, 20]
     np.testing.assert_allclose(got, o * rgb, atol=1e-6)
+
+
+def _dp_inputs(n, seed=7):
+    rng = np.random.default_rng(seed)
+    accum = rng.exponential(0.0003, n).astype(np.float32)
+    denom = rng.integers(0, 5, n).astype(np.int32)
+    z = rng.normal(size=(n, 2, 3)).astype(np.float32)
+    return rng, accum, denom, z
+
+
+DP_ARGS = dict(grad_threshold=0.0002, scale_split=0.05, min_opacity=0.2, max_scale=0.12)
+
+
+def _dp_oracle_thresholds():
+    dp = api.densify_params(**DP_ARGS)
+    return (np.float32(dp.grad_threshold), np.float32(dp.log_scale_split),
+            np.float32(dp.logit_min_opacity), np.float32(dp.log_max_scale))
+
+
+def test_densify_and_prune_matches_oracle():
+    sc = S.make_scene("fwd_100k_800", n=20000, width=792, height=600)
+    n = sc.n
+    sp = Splatter(sc)
+    rng, accum, denom, z = _dp_inputs(n)
+    sp.accum_abs.copy_(torch.as_tensor(accum))
+    sp.denom.copy_(torch.as_tensor(denom))
+    mom_in = {}
+    for k, t in sp.param_list:
+        m = rng.normal(size=tuple(t.shape)).astype(np.float32)
+        v = rng.random(tuple(t.shape)).astype(np.float32)
+        sp.exp_avg[k].copy_(torch.as_tensor(m))
+        sp.exp_avg_sq[k].copy_(torch.as_tensor(v))
+        mom_in[k] = (m, v)
+    p_in = {k: t.cpu().numpy() for k, t in sp.param_list}
+    codes = sp.densify_and_prune(**DP_ARGS, z=torch.as_tensor(z).cuda()).cpu().numpy()
+    torch.cuda.synchronize()
+    # the oracle on the same float32 values (means and log-scales without the pad lane)
+    trim = lambda d: {k: (v[:, :3] if k in ("means", "log_scales") else v)  # noqa: E731
+                      for k, v in d.items()}
+    P_in = trim(p_in)
+    M_in = {k: (trim({k: m})[k], trim({k: v})[k]) for k, (m, v) in mom_in.items()}
+    ref, ref_mom, ref_codes = O.densify_and_prune(P_in, M_in, accum, denom, z,
+                                                  *_dp_oracle_thresholds())
+    assert np.array_equal(codes, ref_codes)
+    assert all((codes == c).sum() > 50 for c in range(4))   # every outcome occurs
+    assert sp.n == len(ref["means"])
+    rows = np.repeat(np.arange(n), np.where(codes == 0, 0, np.where(codes == 1, 1, 2)))
+    kind = np.concatenate([[c] * (0 if c == 0 else 1 if c == 1 else 2) for c in codes])
+    first = np.concatenate([[True] if c == 1 else [True, False] if c in (2, 3) else []
+                            for c in codes]).astype(bool)
+    got = trim({k: t.cpu().numpy() for k, t in sp.param_list})
+    got_m = trim({k: sp.exp_avg[k].cpu().numpy() for k, _ in sp.param_list})
+    got_v = trim({k: sp.exp_avg_sq[k].cpu().numpy() for k, _ in sp.param_list})
+    copies = kind != 3
+    for k in got:
+        # kept and cloned Gaussians: the float32 inputs, bit for bit
+        assert np.array_equal(got[k][copies], P_in[k][rows[copies]].astype(np.float32)), k
+        # moments: kept for the originals, zero for clones and split children
+        keep_m = copies & first
+        assert np.array_equal(got_m[k][keep_m], M_in[k][0][rows[keep_m]]), k
+        assert np.array_equal(got_v[k][keep_m], M_in[k][1][rows[keep_m]]), k
+        assert not got_m[k][~keep_m].any() and not got_v[k][~keep_m].any(), k
+    split = kind == 3
+    np.testing.assert_allclose(got["means"][split], ref["means"][split], rtol=0, atol=2e-6)
+    np.testing.assert_allclose(got["log_scales"][split], ref["log_scales"][split], rtol=0,
+                               atol=2e-6)
+    for k in ("quats", "opacity_logit", "sh"):
+        assert np.array_equal(got[k][split], P_in[k][rows[split]].astype(np.float32)), k
+
+
+def test_densify_and_prune_capacity_and_empty():
+    sc = S.make_scene("fwd_1k_128", n=500)
+    sp = Splatter(sc)
+    n = sc.n
+    _, accum, denom, z = _dp_inputs(n, seed=3)
+    accum[:] = 1.0                                   # everything densifies
+    denom[:] = 1
+    names = [k for k, _ in sp.param_list]
+    like = lambda t, c: torch.empty((c,) + tuple(t.shape[1:]), dtype=t.dtype,  # noqa: E731
+                                    device=t.device)
+    cap = n // 2
+    out = [like(t, cap) for _, t in sp.param_list]
+    m_out = [like(t, cap) for _, t in sp.param_list]
+    v_out = [like(t, cap) for _, t in sp.param_list]
+    n_out = torch.full((1,), -1, dtype=torch.int64, device="cuda")
+    ws = torch.zeros((api.gs_densify_workspace_size(n) + 255) // 256 * 256 // 8,
+                     dtype=torch.int64, device="cuda")
+    sentinel = out[0].clone()
+    api.gs_densify_and_prune(sp.c_params, api.grads(*[sp.exp_avg[k] for k in names]),
+                             api.grads(*[sp.exp_avg_sq[k] for k in names]),
+                             torch.as_tensor(accum).cuda(), torch.as_tensor(denom).cuda(),
+                             torch.as_tensor(z).cuda(),
+                             api.densify_params(0.0002, 0.05, 1e-6, 100.0),   # prunes nothing
+                             api.grads(*out), api.grads(*m_out), api.grads(*v_out), cap, n_out,
+                             None, ws)
+    assert api.gs_get_status(ws) == api.GS_ERR_CAPACITY
+    assert int(n_out.item()) == 2 * n                # every Gaussian cloned or split
+    assert torch.equal(out[0], sentinel)             # nothing written
+    # n = 0: the count is written, nothing else
+    sc0 = S.make_scene("fwd_1k_128", n=1)
+    sp0 = Splatter(sc0)
+    sp0.c_params.n = 0
+    n_out.fill_(-1)
+    api.gs_densify_and_prune(sp0.c_params, api.grads(*[sp0.exp_avg[k] for k in names]),
+                             api.grads(*[sp0.exp_avg_sq[k] for k in names]),
+                             sp0.accum_abs, sp0.denom, torch.zeros(6, device="cuda"),
+                             api.densify_params(**DP_ARGS), api.grads(*out), api.grads(*m_out),
+                             api.grads(*v_out), cap, n_out, None, ws)
+    torch.cuda.synchronize()
+    assert int(n_out.item()) == 0
