@@ -341,3 +341,101 @@ def densify_and_prune(params: dict, moments: dict, accum, denom, z, grad_thresho
     moments_out = {k: (np.array(mom[k][0]).reshape((-1,) + shapes[k]),
                        np.array(mom[k][1]).reshape((-1,) + shapes[k])) for k in PARAM_NAMES}
     return params_out, moments_out, code
+
+
+# --------------------------------------------------------------- photometric loss
+
+# The training objective of the second Julia page (lshu.cn, sec. 3.3): a blend
+# of the L1 error and the structural dissimilarity 1 - SSIM with weight
+# lambda about 0.2. The page fixes nothing else about SSIM, so the constants
+# are those of the SSIM definition itself (Wang, Bovik, Sheikh, Simoncelli
+# 2004): an 11 x 11 Gaussian window of standard deviation 1.5 normalised to
+# sum 1, C1 = (0.01 L)^2 and C2 = (0.03 L)^2 with dynamic range L = 1. The map
+# is taken at every pixel with the image zero-padded outside its border, and
+# both terms are means over the pixels and colour channels of one view.
+SSIM_WINDOW = 11
+SSIM_SIGMA = 1.5
+SSIM_C1 = 0.01 ** 2
+SSIM_C2 = 0.03 ** 2
+LOSS_LAMBDA = 0.2
+
+
+def ssim_window(size: int = SSIM_WINDOW, sigma: float = SSIM_SIGMA) -> np.ndarray:
+    """The 2-D Gaussian window w[i, j] ~ exp(-(di^2 + dj^2) / (2 sigma^2)),
+    di, dj the offsets from the centre, normalised to sum 1."""
+    r = np.arange(size, dtype=np.float64) - (size - 1) / 2.0
+    w = np.exp(-(r[:, None] ** 2 + r[None, :] ** 2) / (2.0 * sigma * sigma))
+    return w / w.sum()
+
+
+def window_filter(img: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """Same-size correlation of the last two axes with the window w, zero
+    outside the image: out[y, x] = sum_ij w[i, j] img[y + i - h, x + j - h]."""
+    img = np.asarray(img, np.float64)
+    s = w.shape[0]
+    h = s // 2
+    H, W = img.shape[-2:]
+    pad = np.zeros(img.shape[:-2] + (H + 2 * h, W + 2 * h))
+    pad[..., h:h + H, h:h + W] = img
+    out = np.zeros(img.shape)
+    for i in range(s):
+        for j in range(s):
+            out += w[i, j] * pad[..., i:i + H, j:j + W]
+    return out
+
+
+def ssim_map(x: np.ndarray, y: np.ndarray, w: Optional[np.ndarray] = None) -> np.ndarray:
+    """SSIM at every pixel of the planes x, y (last two axes): local means,
+    variances and covariance under the window, then
+    S = (2 mx my + C1)(2 sxy + C2) / ((mx^2 + my^2 + C1)(sx^2 + sy^2 + C2))."""
+    w = ssim_window() if w is None else w
+    x = np.asarray(x, np.float64)
+    y = np.asarray(y, np.float64)
+    mx, my = window_filter(x, w), window_filter(y, w)
+    sxx = window_filter(x * x, w) - mx * mx
+    syy = window_filter(y * y, w) - my * my
+    sxy = window_filter(x * y, w) - mx * my
+    return ((2 * mx * my + SSIM_C1) * (2 * sxy + SSIM_C2)
+            / ((mx * mx + my * my + SSIM_C1) * (sxx + syy + SSIM_C2)))
+
+
+def l1_dssim_loss(image: np.ndarray, target: np.ndarray, lam: float = LOSS_LAMBDA):
+    """Loss and its gradient for images [V, 3, H, W] against targets of the
+    same shape, view by view:
+      L_v = (1 - lam) mean|x - y| + lam (1 - mean SSIM(x, y)).
+    The gradient dL_v / dx is the chain rule through the window statistics:
+    with the SSIM map written as S(mx, Exx, Exy) of the windowed moments
+    mx = w*x, Exx = w*(x x), Exy = w*(x y), each pixel q receives
+      dS_mean/dx_q = (1/N) [w'*(dS/dmx) + 2 x_q w'*(dS/dExx) + y_q w'*(dS/dExy)]_q
+    where w'* is the adjoint of the zero-padded correlation (correlation with
+    the flipped window, zero outside). The L1 term contributes
+    sign(x_q - y_q) / N with sign(0) = 0. Returns (terms [V, 3] = loss, mean
+    L1, mean SSIM per view; grad [V, 3, H, W])."""
+    x = np.asarray(image, np.float64)
+    y = np.asarray(target, np.float64)
+    w = ssim_window()
+    wf = w[::-1, ::-1]
+    V = x.shape[0]
+    N = float(np.prod(x.shape[1:]))
+    mx, my = window_filter(x, w), window_filter(y, w)
+    exx, eyy, exy = window_filter(x * x, w), window_filter(y * y, w), window_filter(x * y, w)
+    a1 = 2 * mx * my + SSIM_C1
+    a2 = 2 * (exy - mx * my) + SSIM_C2
+    b1 = mx * mx + my * my + SSIM_C1
+    b2 = (exx - mx * mx) + (eyy - my * my) + SSIM_C2
+    num, den = a1 * a2, b1 * b2
+    S = num / den
+    # partial derivatives of S = num / den with respect to mx, Exx and Exy
+    d_num_mx = 2 * my * a2 + a1 * (-2 * my)
+    d_den_mx = 2 * mx * b2 + b1 * (-2 * mx)
+    d_mx = (d_num_mx * den - num * d_den_mx) / (den * den)
+    d_exx = -num * b1 / (den * den)
+    d_exy = 2 * a1 / den
+    g_ssim = (window_filter(d_mx, wf) + 2 * x * window_filter(d_exx, wf)
+              + y * window_filter(d_exy, wf)) / N
+    diff = x - y
+    l1 = np.abs(diff).reshape(V, -1).mean(axis=1)
+    ssim = S.reshape(V, -1).mean(axis=1)
+    terms = np.stack([(1 - lam) * l1 + lam * (1 - ssim), l1, ssim], axis=1)
+    grad = (1 - lam) * np.sign(diff) / N - lam * g_ssim
+    return terms, grad

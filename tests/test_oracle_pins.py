@@ -564,3 +564,143 @@ def test_dp_threshold_is_strict_and_exact_in_float32():
     code = O.densify_decisions(params["log_scales"], params["opacity_logit"], acc, [3, 3],
                                thr, np.log(0.1), -10.0, 10.0)
     assert code.tolist() == [O.DP_KEEP, O.DP_CLONE]
+
+
+# ---------------------------------------------------------------- L1 + D-SSIM loss
+
+def _gauss1d(size=11, sigma=1.5):
+    """Normalised 1-D Gaussian taps; the 2-D SSIM window is their outer product."""
+    g = np.array([math.exp(-((k - size // 2) ** 2) / (2 * sigma * sigma)) for k in range(size)])
+    return g / g.sum()
+
+
+def test_ssim_window_is_the_normalised_gaussian():
+    w = O.ssim_window()
+    assert w.shape == (11, 11)
+    assert abs(w.sum() - 1.0) < 1e-15
+    c = 5
+    assert w[c, c + 1] / w[c, c] == pytest.approx(math.exp(-1 / 4.5), rel=1e-14)
+    assert w[c + 2, c - 1] / w[c, c] == pytest.approx(math.exp(-5 / 4.5), rel=1e-14)
+    g = _gauss1d()
+    np.testing.assert_allclose(w, np.outer(g, g), rtol=1e-13, atol=0)
+
+
+def test_ssim_of_an_image_with_itself_is_one_and_loss_zero():
+    rng = np.random.default_rng(3)
+    x = rng.random((2, 3, 17, 21))
+    S = O.ssim_map(x, x)
+    np.testing.assert_allclose(S, 1.0, rtol=0, atol=1e-12)
+    terms, grad = O.l1_dssim_loss(x, x)
+    np.testing.assert_allclose(terms, [[0.0, 0.0, 1.0]] * 2, atol=1e-12)
+    assert np.abs(grad).max() < 1e-14
+
+
+def _window_mass(H, W, y, x):
+    """Weight of the 11 x 11 window that falls inside an H x W image at (y, x)."""
+    g = _gauss1d()
+    rows = sum(g[i] for i in range(11) if 0 <= y + i - 5 < H)
+    cols = sum(g[j] for j in range(11) if 0 <= x + j - 5 < W)
+    return rows * cols
+
+
+def test_ssim_of_constant_planes_closed_form():
+    """x = a, y = b everywhere: inside, S = (2ab + C1) / (a^2 + b^2 + C1) (no
+    variance, the contrast-structure factor is C2 / C2); at the border the
+    zero padding leaves window mass m < 1, so mx = a m, var x = a^2 m (1 - m),
+    cov = a b m (1 - m)."""
+    a, b, H, W = 0.5, 0.25, 20, 24
+    S = O.ssim_map(np.full((H, W), a), np.full((H, W), b))
+    assert S[10, 12] == pytest.approx((0.25 + 1e-4) / (0.3125 + 1e-4), rel=1e-13)
+    C1, C2 = 1e-4, 9e-4
+    for (yy, xx) in [(0, 0), (0, 7), (3, 23), (19, 2), (10, 12)]:
+        m = _window_mass(H, W, yy, xx)
+        v = m * (1 - m)
+        want = ((2 * a * b * m * m + C1) * (2 * a * b * v + C2)
+                / (((a * a + b * b) * m * m + C1) * ((a * a + b * b) * v + C2)))
+        assert S[yy, xx] == pytest.approx(want, rel=1e-12), (yy, xx)
+
+
+def test_ssim_of_a_checkerboard_against_its_mean():
+    """x = 0.5 + 0.25 (-1)^(i+j) against y = 0.5: the window's alternating sum
+    A = (sum_k g_k (-1)^k)^2 gives mx = 0.5 + 0.25 s A (s the pixel's parity
+    sign) and var x = 0.0625 (1 - A^2); y has no variance and no covariance."""
+    H, W = 24, 24
+    ii, jj = np.meshgrid(np.arange(H), np.arange(W), indexing="ij")
+    x = 0.5 + 0.25 * (-1.0) ** (ii + jj)
+    y = np.full((H, W), 0.5)
+    S = O.ssim_map(x, y)
+    g = _gauss1d()
+    A = sum(g[k] * (-1) ** (k - 5) for k in range(11)) ** 2
+    C1, C2 = 1e-4, 9e-4
+    for (yy, xx) in [(11, 11), (11, 12), (8, 15)]:
+        s = (-1.0) ** (yy + xx)
+        mx = 0.5 + 0.25 * s * A
+        vx = 0.0625 * (1 - A * A)
+        want = (2 * mx * 0.5 + C1) * C2 / ((mx * mx + 0.25 + C1) * (vx + C2))
+        assert S[yy, xx] == pytest.approx(want, rel=1e-12)
+
+
+def test_ssim_against_brute_force_patch_statistics():
+    """Each pixel's statistics taken directly from its zero-padded 11 x 11
+    patch in centred form, sum w (x - mx)(y - my), instead of the moment maps."""
+    rng = np.random.default_rng(5)
+    H, W = 23, 29
+    x, y = rng.random((H, W)), rng.random((H, W))
+    S = O.ssim_map(x, y)
+    w = np.outer(_gauss1d(), _gauss1d())
+    px = np.pad(x, 5)
+    py = np.pad(y, 5)
+    C1, C2 = 1e-4, 9e-4
+    for (yy, xx) in [(0, 0), (0, 28), (22, 0), (22, 28), (11, 14), (4, 9), (17, 3)]:
+        P = px[yy:yy + 11, xx:xx + 11]
+        Q = py[yy:yy + 11, xx:xx + 11]
+        mx, my = (w * P).sum(), (w * Q).sum()
+        vx, vy = (w * (P - mx) ** 2).sum(), (w * (Q - my) ** 2).sum()
+        cxy = (w * (P - mx) * (Q - my)).sum()
+        lum = (2 * mx * my + C1) / (mx * mx + my * my + C1)
+        cs = (2 * cxy + C2) / (vx + vy + C2)
+        assert S[yy, xx] == pytest.approx(lum * cs, rel=1e-12), (yy, xx)
+
+
+def test_loss_terms_weights_and_symmetry():
+    rng = np.random.default_rng(6)
+    x, y = rng.random((2, 3, 14, 19)), rng.random((2, 3, 14, 19))
+    t0, _ = O.l1_dssim_loss(x, y, lam=0.0)
+    t1, _ = O.l1_dssim_loss(x, y, lam=1.0)
+    t, _ = O.l1_dssim_loss(x, y)
+    np.testing.assert_allclose(t0[:, 0], np.abs(x - y).reshape(2, -1).mean(1), rtol=1e-14)
+    S = O.ssim_map(x, y)
+    np.testing.assert_allclose(t1[:, 0], 1 - S.reshape(2, -1).mean(1), rtol=1e-14)
+    np.testing.assert_allclose(t[:, 0], 0.8 * t0[:, 0] + 0.2 * t1[:, 0], rtol=1e-14)
+    np.testing.assert_allclose(S, O.ssim_map(y, x), rtol=1e-14)
+    assert S.max() <= 1.0 + 1e-12
+
+
+@pytest.mark.parametrize("lam", [0.2, 1.0])
+def test_loss_gradient_matches_central_differences(lam):
+    rng = np.random.default_rng(7)
+    x, y = rng.random((2, 3, 12, 15)), rng.random((2, 3, 12, 15))
+    keep = np.abs(x - y) < 1e-3          # stay off the L1 kink
+    x[keep] += 2e-3
+    _, g = O.l1_dssim_loss(x, y, lam)
+    eps = 1e-6
+    for _ in range(24):
+        idx = tuple(int(rng.integers(0, s)) for s in x.shape)
+        xp, xm = x.copy(), x.copy()
+        xp[idx] += eps
+        xm[idx] -= eps
+        v = idx[0]
+        fd = (O.l1_dssim_loss(xp, y, lam)[0][v, 0] - O.l1_dssim_loss(xm, y, lam)[0][v, 0]) / (2 * eps)
+        assert g[idx] == pytest.approx(fd, rel=1e-6, abs=1e-11), idx
+        # another view's loss does not depend on this pixel
+        o = 1 - v
+        assert O.l1_dssim_loss(xp, y, lam)[0][o, 0] == O.l1_dssim_loss(x, y, lam)[0][o, 0]
+
+
+def test_loss_l1_subgradient_is_zero_where_equal():
+    rng = np.random.default_rng(8)
+    x, y = rng.random((1, 3, 13, 13)), rng.random((1, 3, 13, 13))
+    x[0, 1, 6, 6] = y[0, 1, 6, 6]
+    _, g = O.l1_dssim_loss(x, y, 0.2)
+    _, g1 = O.l1_dssim_loss(x, y, 1.0)
+    assert g[0, 1, 6, 6] == pytest.approx(0.2 * g1[0, 1, 6, 6], rel=1e-13)
