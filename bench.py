@@ -324,6 +324,48 @@ def run_reference(args):
 
 # ----------------------------------------------------------------- our path
 
+# FP32 peak of the part for the ALU-bound loss kernel: 148 SMs x 128 FP32
+# lanes x 2 FLOP per FMA at the maximum SM clock.
+FP32_LANES = 148 * 128
+
+
+def measure_loss(sp, reps: int = 5) -> dict:
+    """gs_l1_dssim (loss, and its gradient) on the Splatter's rendered frame
+    against a seeded target of the same size, each launch timed with CUDA
+    events after an L2 flush (a 256 MB write), mean over `reps` after an
+    untimed launch. Algorithmic work per value: the separable 11-tap window
+    applied along rows and columns to the five SSIM moments and to the three
+    partial maps of the gradient, 2 x 11 x 8 = 176 FMA (352 FLOP); traffic:
+    x and y read, dL/dx written, 12 bytes."""
+    import torch
+    from gaussian_splatting_differentiable_ewa_b200 import api
+    from gaussian_splatting_differentiable_ewa_b200 import scenes as S
+    V, H, W = sp.V, sp.H, sp.W
+    _, tgt = S.make_image_pair(V, H, W, seed=4)
+    target = torch.from_numpy(tgt).cuda()
+    sp.loss(target)
+    torch.cuda.synchronize()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ms = 0.0
+    for _ in range(reps):
+        flush.fill_(1)
+        e0.record()
+        sp.loss(target)
+        e1.record()
+        torch.cuda.synchronize()
+        ms += e0.elapsed_time(e1) / reps
+    values = 3 * V * H * W
+    pk = peaks()
+    tflops = values * 352 / (ms / 1e3) / 1e12
+    fp32_peak = FP32_LANES * 2 * pk["sm_max_mhz"] * 1e6 / 1e12
+    gbs = values * 12 / (ms / 1e3) / 1e9
+    t = sp.loss_terms.cpu().numpy()
+    return dict(ms=ms, values=values, tflops=tflops, fp32_peak_tflops=fp32_peak,
+                alu_frac=tflops / fp32_peak, gbs=gbs, hbm_frac=gbs / pk["hbm_gbs"],
+                loss=float(t[0, 0]), l1=float(t[0, 1]), ssim=float(t[0, 2]))
+
+
 def measure_densify(sp) -> dict:
     """One gs_densify_and_prune call on the Splatter's accumulated statistics
     (absolute gradients, the page's threshold 0.0002), timed with CUDA events
@@ -483,6 +525,7 @@ def run_ours(args):
     extras = {}
     if world == 1:
         extras["gs_densify_and_prune"] = measure_densify(sp)
+        extras["gs_l1_dssim"] = measure_loss(sp)
 
     if world > 1:
         dist.barrier()

@@ -104,6 +104,10 @@ SIGNATURES = [
      [_c.POINTER(GsParams), _c.POINTER(GsGrads), _c.POINTER(GsGrads), _vp, _vp, _vp,
       _c.POINTER(GsDensifyParams), _c.POINTER(GsGrads), _c.POINTER(GsGrads), _c.POINTER(GsGrads),
       _c.c_int64, _vp, _vp, _vp, _c.c_size_t, _vp]),
+    ("gs_l1_dssim_workspace_size", _c.c_size_t, [_c.c_int32]),
+    ("gs_l1_dssim", _c.c_int,
+     [_vp, _vp, _c.c_int32, _c.c_int32, _c.c_int32, _c.c_float, _vp, _vp, _vp, _c.c_size_t,
+      _vp]),
     ("gs_bin_sort_noalloc", _c.c_int,
      [_c.POINTER(GsProjected), _c.POINTER(GsCamera), _c.c_int32, _c.c_int64, _c.c_int32,
       _c.POINTER(GsBinned), _vp, _vp]),
@@ -287,6 +291,20 @@ def gs_densify_and_prune(params: GsParams, m_in: GsGrads, v_in: GsGrads, accum, 
                                       int(out_capacity), _ptr(n_out), _ptr(codes), _ptr(ws),
                                       int(ws.numel() * ws.element_size()), _stream(stream)),
            "gs_densify_and_prune")
+
+
+def gs_l1_dssim_workspace_size(n_views: int) -> int:
+    return int(lib().gs_l1_dssim_workspace_size(int(n_views)))
+
+
+def gs_l1_dssim(image, target, n_views: int, height: int, width: int, lam: float, terms,
+                dL_dimage, ws, stream=None) -> None:
+    """(1 - lam) L1 + lam (1 - SSIM) per view; terms [V, 3] float64 (loss,
+    mean L1, mean SSIM), dL_dimage like image or None."""
+    _check(lib().gs_l1_dssim(_ptr(image), _ptr(target), int(n_views), int(height), int(width),
+                             float(lam), _ptr(terms), _ptr(dL_dimage), _ptr(ws),
+                             int(ws.numel() * ws.element_size()), _stream(stream)),
+           "gs_l1_dssim")
 
 
 def gs_bin_sort_noalloc(proj: GsProjected, cams_arr, n_views: int, n: int, sort_mode: int,

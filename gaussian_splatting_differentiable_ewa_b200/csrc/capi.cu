@@ -472,6 +472,30 @@ gs_status gs_densify_and_prune(const gs_params* in, const gs_grads* m_in, const 
       reinterpret_cast<uint32_t*>(w + kStatusOffset), op, om, ov, st));
 }
 
+size_t gs_l1_dssim_workspace_size(int32_t n_views) {
+  if (n_views < 0) return 0;
+  return (size_t)n_views * 2 * sizeof(double) + 16;
+}
+
+gs_status gs_l1_dssim(const float* image, const float* target, int32_t n_views, int32_t height,
+                      int32_t width, float lambda, double* terms, float* dL_dimage, void* ws,
+                      size_t ws_bytes, void* stream) {
+  if (n_views < 0 || n_views > 21845) return GS_ERR_INVALID_ARG;
+  if (n_views == 0) return GS_OK;
+  if (height < 1 || width < 1 || height > 2097120) return GS_ERR_INVALID_ARG;
+  if (!(lambda >= 0.f && lambda <= 1.f)) return GS_ERR_INVALID_ARG;
+  if (!image || !target || !terms || !ws || !aligned(ws, 8) || !aligned(terms, 8))
+    return GS_ERR_INVALID_ARG;
+  if (!aligned(image, 4) || !aligned(target, 4) || (dL_dimage && !aligned(dL_dimage, 4)))
+    return GS_ERR_INVALID_ARG;
+  if (ws_bytes < gs_l1_dssim_workspace_size(n_views)) return GS_ERR_INVALID_ARG;
+  double* sums = static_cast<double*>(ws);
+  unsigned* done = reinterpret_cast<unsigned*>(sums + 2 * (size_t)n_views);
+  return cuda_status(gsb::launch_l1_dssim(image, target, n_views, height, width, lambda, terms,
+                                          dL_dimage, sums, done,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 gs_status gs_get_status(void* ws, void* stream) {
   if (!ws) return GS_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -113,4 +113,11 @@ cudaError_t launch_densify_and_prune(const DpTensorPtrs& p_in, const DpTensorPtr
                                      const DpTensorPtrs& m_out, const DpTensorPtrs& v_out,
                                      cudaStream_t stream);
 
+// Fused L1 + D-SSIM loss over [n_views][3][H][W] planes; `sums` holds
+// 2 * n_views doubles followed by the block counter `done` (both cleared here).
+size_t loss_smem_bytes();
+cudaError_t launch_l1_dssim(const float* image, const float* target, int n_views, int H, int W,
+                            float lambda, double* terms, float* grad, double* sums,
+                            unsigned* done, cudaStream_t stream);
+
 }  // namespace gsb

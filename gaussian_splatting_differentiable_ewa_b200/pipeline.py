@@ -59,6 +59,7 @@ class Splatter:
         self.ids = None
         self.ws = None
         self.step_count = 0
+        self.loss_terms = None
         self._alloc_pairs(int(pair_capacity) if pair_capacity is not None else 0)
 
     # ------------------------------------------------------------ buffers
@@ -166,6 +167,33 @@ class Splatter:
     def train_step(self, dL_dimage: torch.Tensor, adam: bool = True):
         self.forward()
         self.rasterize_bwd(dL_dimage)
+        self.densify_stats()
+        if adam:
+            self.adam_step()
+
+    def loss(self, target: torch.Tensor, lam: float = 0.2, grad: bool = True) -> torch.Tensor:
+        """(1 - lam) L1 + lam (1 - SSIM) of the rendered image against
+        `target` ([V, 3, H, W] float32 on the device). Leaves the per-view
+        terms (loss, mean L1, mean SSIM) in ``self.loss_terms`` and, with
+        `grad`, dL/dimage in ``self.dL_loss``; returns ``self.loss_terms``."""
+        if tuple(target.shape) != tuple(self.image.shape) or target.dtype != torch.float32:
+            raise ValueError("target must be float32 of the image's shape")
+        if self.loss_terms is None:
+            self.loss_terms = torch.empty((self.V, 3), dtype=torch.float64, device=self.device)
+            self.dL_loss = torch.empty_like(self.image)
+            nb = api.gs_l1_dssim_workspace_size(self.V)
+            self._loss_ws = torch.empty((nb + 7) // 8, dtype=torch.float64, device=self.device)
+        api.gs_l1_dssim(self.image, target.contiguous(), self.V, self.H, self.W, lam,
+                        self.loss_terms, self.dL_loss if grad else None, self._loss_ws,
+                        self.stream)
+        return self.loss_terms
+
+    def train_step_target(self, target: torch.Tensor, lam: float = 0.2, adam: bool = True):
+        """One training step on target images: render, the L1 + D-SSIM loss
+        and its image gradient, then the backward, statistics and Adam."""
+        self.forward()
+        self.loss(target, lam)
+        self.rasterize_bwd(self.dL_loss)
         self.densify_stats()
         if adam:
             self.adam_step()

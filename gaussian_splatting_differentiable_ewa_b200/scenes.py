@@ -261,3 +261,38 @@ def make_projected_2d(n: int, width: int, height: int, seed: int = 2,
     depth = depth + rng.integers(0, 4, size=(n_views, n)) * 1e-3
     return dict(xy=xy.astype(np.float32), radius=radius.astype(np.int32),
                 depth=depth.astype(np.float32))
+
+
+def make_image_pair(n_views: int, height: int, width: int, seed: int = 3,
+                    noise: float = 0.05, tie_frac: float = 0.05):
+    """A rendered-like image and a target for the photometric loss, float32
+    [V, 3, H, W] each, values in [0, 1].
+
+    The target is a smooth field (a few random low-frequency sinusoids per
+    channel) with sharp-edged discs on top, like a render of a few large
+    splats over a background; the image is the target shifted by a slowly
+    varying offset plus white noise of standard deviation `noise`, clipped to
+    [0, 1]. A fraction `tie_frac` of the image's values equals the target's
+    exactly, so that |x - y| has zeros.
+    """
+    rng = np.random.default_rng(seed)
+    yy, xx = np.meshgrid(np.linspace(0, 1, height), np.linspace(0, 1, width), indexing="ij")
+    tgt = np.empty((n_views, 3, height, width))
+    img = np.empty_like(tgt)
+    for v in range(n_views):
+        for c in range(3):
+            f = 0.5 + np.zeros((height, width))
+            for _ in range(4):
+                kx, ky = rng.uniform(0.5, 6.0, 2)
+                f += 0.12 * np.sin(2 * np.pi * (kx * xx + ky * yy) + rng.uniform(0, 2 * np.pi))
+            for _ in range(6):
+                cx, cy, r = rng.uniform(0, 1), rng.uniform(0, 1), rng.uniform(0.03, 0.2)
+                f = np.where((xx - cx) ** 2 + (yy - cy) ** 2 < r * r, rng.uniform(0, 1), f)
+            tgt[v, c] = f
+            off = 0.05 * np.sin(2 * np.pi * (rng.uniform(0.2, 2) * xx + rng.uniform(0, 1)))
+            img[v, c] = f + off + rng.normal(0.0, noise, size=(height, width))
+    tgt = np.clip(tgt, 0.0, 1.0).astype(np.float32)
+    img = np.clip(img, 0.0, 1.0).astype(np.float32)
+    tie = rng.random(img.shape) < tie_frac
+    img[tie] = tgt[tie]
+    return img, tgt

@@ -340,6 +340,31 @@ gs_status gs_densify_and_prune(const gs_params* in, const gs_grads* m_in, const 
                                gs_grads* v_out, int64_t out_capacity, int64_t* n_out,
                                int8_t* codes, void* ws, size_t ws_bytes, void* stream);
 
+/* Bytes of workspace gs_l1_dssim needs for n_views views (sums and a block
+ * counter; 8-byte aligned). */
+size_t gs_l1_dssim_workspace_size(int32_t n_views);
+
+/* Photometric loss and its gradient (second Julia page, lshu.cn, sec. 3.3):
+ *   L_v = (1 - lambda) mean|x - y| + lambda (1 - mean SSIM(x, y))
+ * per view v, the means over its 3 x height x width values. SSIM follows its
+ * own definition (Wang et al. 2004), which the page does not restate: an
+ * 11 x 11 Gaussian window of sigma 1.5 normalised to 1, C1 = 0.01^2,
+ * C2 = 0.03^2 (dynamic range 1), the map taken at every pixel with the
+ * planes zero outside the image.
+ * image, target: float [n_views][3][height][width] (the layout of
+ *   gs_rasterize_fwd's colour), device memory, not overlapping dL_dimage.
+ * terms: device double [n_views][3] receives (L_v, mean L1, mean SSIM).
+ * dL_dimage: device float, image's layout, receives dL_v / dimage (the
+ *   L1 subgradient taken as 0 where x == y); NULL skips the gradient.
+ * ws: device workspace of gs_l1_dssim_workspace_size(n_views) bytes,
+ *   8-byte aligned; owned by the caller and overwritten.
+ * n_views 0 returns GS_OK with nothing done; n_views > 21845, an empty image,
+ * a height above 2,097,120, lambda outside [0, 1] or a NULL pointer is
+ * GS_ERR_INVALID_ARG. One launch on `stream`. */
+gs_status gs_l1_dssim(const float* image, const float* target, int32_t n_views, int32_t height,
+                      int32_t width, float lambda, double* terms, float* dL_dimage, void* ws,
+                      size_t ws_bytes, void* stream);
+
 /* Synchronise `stream`, return the status word accumulated in workspace `ws`
  * by device-side checks since the last call, and clear it. */
 gs_status gs_get_status(void* ws, void* stream);
