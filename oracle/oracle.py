@@ -439,3 +439,138 @@ def l1_dssim_loss(image: np.ndarray, target: np.ndarray, lam: float = LOSS_LAMBD
     terms = np.stack([(1 - lam) * l1 + lam * (1 - ssim), l1, ssim], axis=1)
     grad = (1 - lam) * np.sign(diff) / N - lam * g_ssim
     return terms, grad
+
+
+# --------------------------------------------------------------- quantised SH state
+
+# The Spirula VRAM page (sec. 魔法一, quantised training): SH coefficients are
+# stored as 8- or 16-bit fixed point, every 256 units sharing one (min, max)
+# pair that decodes them; gradients stay float32; the Adam moments are 16-bit
+# words in a transposed layout. Readings where the page is silent: a unit is
+# one SH value; the layout is coefficient-major ([3K][N], N padded to a
+# multiple of 256), so a group is one coefficient of 256 consecutive
+# Gaussians; a code q decodes to min + q (max - min) / (2^b - 1); encoding
+# takes the group's min and max and rounds (x - min) (2^b - 1) / (max - min),
+# in float32 like the kernel, to nearest-even or stochastically (floor of
+# t + u, u uniform from SplitMix64); the 16-bit Adam words are bfloat16,
+# rounded to nearest-even from float32.
+Q_GROUP = 256
+_GAMMA = np.uint64(0x9E3779B97F4A7C15)
+
+
+def splitmix64(seed: int, counter) -> np.ndarray:
+    """Output number `counter` + 1 of SplitMix64 started at `seed` (Steele,
+    Lea and Flood 2014): z = seed + (counter + 1) gamma, then the variant-13
+    mix z ^= z >> 30; z *= 0xBF58476D1CE4E5B9; z ^= z >> 27;
+    z *= 0x94D049BB133111EB; z ^= z >> 31 (all mod 2^64)."""
+    with np.errstate(over="ignore"):
+        c = np.asarray(counter, np.uint64)
+        z = np.uint64(seed) + (c + np.uint64(1)) * _GAMMA
+        z = (z ^ (z >> np.uint64(30))) * np.uint64(0xBF58476D1CE4E5B9)
+        z = (z ^ (z >> np.uint64(27))) * np.uint64(0x94D049BB133111EB)
+        return z ^ (z >> np.uint64(31))
+
+
+def sr_uniform(seed: int, step: int, coef, gauss) -> np.ndarray:
+    """The stochastic-rounding draw of SH value (coefficient j, Gaussian n) at
+    Adam step t: counter = t 2^37 + j 2^31 + n, u = (top 24 bits) / 2^24, a
+    float32 in [0, 1)."""
+    c = ((np.uint64(step) << np.uint64(37)) + (np.asarray(coef, np.uint64) << np.uint64(31))
+         + np.asarray(gauss, np.uint64))
+    return ((splitmix64(seed, c) >> np.uint64(40)).astype(np.float64) / 2.0 ** 24).astype(
+        np.float32)
+
+
+def to_bf16(x) -> np.ndarray:
+    """bfloat16 bits (uint16) of float32(x), rounded to nearest-even."""
+    b = np.asarray(np.asarray(x, np.float32)).view(np.uint32).astype(np.uint64)
+    r = (b + np.uint64(0x7FFF) + ((b >> np.uint64(16)) & np.uint64(1))) >> np.uint64(16)
+    return r.astype(np.uint16)
+
+
+def from_bf16(h) -> np.ndarray:
+    return (np.asarray(h, np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32).astype(
+        np.float64)
+
+
+def _sh_transposed(sh: np.ndarray, n_pad: int) -> np.ndarray:
+    """[N][K][3] -> [3K][n_pad] (value j = 3 k + channel), zero padding."""
+    n = sh.shape[0]
+    t = np.zeros((sh.shape[1] * 3, n_pad), np.asarray(sh).dtype)
+    t[:, :n] = np.asarray(sh).reshape(n, -1).T
+    return t
+
+
+def quantize_groups(x: np.ndarray, n: int, bits: int, rounding: int = 0, seed: int = 0,
+                    step: int = 0):
+    """Codes and (min, max) bounds of float32 values x [3K][n_pad], groups of
+    256 along the Gaussian axis over the first n Gaussians only. The decision
+    is taken in float32: range = max - min, inv = (2^b - 1) / range,
+    t = (x - min) inv, then rint(t) (rounding 0) or floor(t + u) (rounding 1),
+    clamped to [0, 2^b - 1]; a group with max == min gets code 0."""
+    f = np.float32
+    x = np.asarray(x, f)
+    k3, n_pad = x.shape
+    qmax = (1 << bits) - 1
+    codes = np.zeros((k3, n_pad), np.uint16 if bits == 16 else np.uint8)
+    bounds = np.zeros((k3, n_pad // Q_GROUP, 2), f)
+    for g in range(n_pad // Q_GROUP):
+        a, b = g * Q_GROUP, min((g + 1) * Q_GROUP, n)
+        if b <= a:
+            continue
+        blk = x[:, a:b]
+        lo, hi = blk.min(axis=1), blk.max(axis=1)
+        bounds[:, g, 0], bounds[:, g, 1] = lo, hi
+        rng = (hi - lo).astype(f)
+        flat = rng == 0
+        inv = np.where(flat, f(0), f(qmax) / np.where(flat, f(1), rng)).astype(f)
+        t = ((blk - lo[:, None]).astype(f) * inv[:, None]).astype(f)
+        if rounding == 0:
+            q = np.rint(t)
+        else:
+            u = sr_uniform(seed, step, np.arange(k3)[:, None], np.arange(a, b)[None, :])
+            q = np.floor((t + u).astype(f))
+        codes[:, a:b] = np.clip(q, 0, qmax).astype(codes.dtype)
+    return codes, bounds
+
+
+def dequantize_groups(codes: np.ndarray, bounds: np.ndarray, n: int, bits: int) -> np.ndarray:
+    """x = min + q (max - min) / (2^b - 1) in float64 -> [3K][n]."""
+    qmax = (1 << bits) - 1
+    c = np.asarray(codes, np.float64)[:, :n]
+    g = np.arange(n) // Q_GROUP
+    lo = np.asarray(bounds, np.float64)[:, g, 0]
+    hi = np.asarray(bounds, np.float64)[:, g, 1]
+    return lo + c * (hi - lo) / qmax
+
+
+def sh_quantize(sh: np.ndarray, bits: int):
+    """Quantised SH state of float32 SH [N][K][3]: (codes [3K][n_pad], bounds
+    [3K][n_pad / 256][2]) with round-to-nearest."""
+    n = sh.shape[0]
+    n_pad = -(-n // Q_GROUP) * Q_GROUP
+    return quantize_groups(_sh_transposed(np.asarray(sh, np.float32), n_pad), n, bits)
+
+
+def adam_sh_quant(codes, bounds, grad_sh, m16, v16, n: int, bits: int, lr: float, step: int,
+                  beta1=0.9, beta2=0.999, eps=1e-15, rounding: int = 0, seed: int = 0):
+    """One Adam step on quantised SH: decode the parameters, update the
+    bfloat16 moments with the float32 gradient (grad_sh [N][K][3]), take the
+    Adam step (as ``adam``), store the moments back as bfloat16 and re-encode
+    the parameters with their groups' new min and max (the float32 value of
+    the new parameter is quantised, like the kernel's). Returns (codes,
+    bounds, m16, v16, p_new [3K][n] float64)."""
+    n_pad = codes.shape[1]
+    p = dequantize_groups(codes, bounds, n, bits)
+    g = _sh_transposed(np.asarray(grad_sh, np.float64), n_pad)[:, :n]
+    m = from_bf16(m16[:, :n])
+    v = from_bf16(v16[:, :n])
+    p, m, v = adam(p, g, m, v, lr, step, beta1, beta2, eps)
+    m_out = np.array(m16, copy=True)
+    v_out = np.array(v16, copy=True)
+    m_out[:, :n] = to_bf16(m)
+    v_out[:, :n] = to_bf16(v)
+    x = np.zeros((codes.shape[0], n_pad), np.float32)
+    x[:, :n] = p.astype(np.float32)
+    c, b = quantize_groups(x, n, bits, rounding, seed, step)
+    return c, b, m_out, v_out, p

@@ -704,3 +704,111 @@ def test_loss_l1_subgradient_is_zero_where_equal():
     _, g = O.l1_dssim_loss(x, y, 0.2)
     _, g1 = O.l1_dssim_loss(x, y, 1.0)
     assert g[0, 1, 6, 6] == pytest.approx(0.2 * g1[0, 1, 6, 6], rel=1e-13)
+
+
+# ---------------------------------------------------------------- quantised SH state
+
+def test_splitmix64_published_sequence():
+    """The first three outputs of SplitMix64 seeded with 0, as published with
+    the generator (and used to seed the xoshiro family)."""
+    out = [int(v) for v in O.splitmix64(0, np.arange(3))]
+    assert out == [0xE220A8397B1DCDAF, 0x6E789E6AA1B965F4, 0x06C45D188009454F]
+
+
+def test_bf16_rounding_closed_forms():
+    assert int(O.to_bf16(1.0)) == 0x3F80
+    assert int(O.to_bf16(-2.0)) == 0xC000
+    assert int(O.to_bf16(1 + 2 ** -8)) == 0x3F80          # tie -> even
+    assert int(O.to_bf16(1 + 3 * 2 ** -8)) == 0x3F82      # tie -> even (up)
+    assert int(O.to_bf16(1 + 2 ** -8 + 2 ** -20)) == 0x3F81  # above the tie
+    assert int(O.to_bf16(0.0)) == 0 and int(O.to_bf16(-0.0)) == 0x8000
+    rng = np.random.default_rng(1)
+    x = rng.normal(0, 1, 10000) * 10.0 ** rng.integers(-20, 20, 10000)
+    back = O.from_bf16(O.to_bf16(x))
+    assert np.all(np.abs(back - x) <= np.abs(x) * 2.0 ** -8)
+
+
+def test_quantize_groups_structure_and_error_bound():
+    """Groups are one coefficient of 256 consecutive Gaussians; the group's
+    min and max are exact codes 0 and 2^b - 1; nearest rounding is off by at
+    most half a step (plus float32 rounding of the scale)."""
+    rng = np.random.default_rng(2)
+    n, K = 700, 4                           # 3 groups, the last one ragged
+    sh = rng.normal(0, 1, (n, K, 3)).astype(np.float32)
+    sh[256:512, 2, 1] = 0.25                # one constant group
+    for bits in (8, 16):
+        codes, bounds = O.sh_quantize(sh, bits)
+        qmax = (1 << bits) - 1
+        assert codes.shape == (12, 768) and bounds.shape == (12, 3, 2)
+        j = 2 * 3 + 1
+        grp = sh[256:512, 2, 1]
+        assert bounds[j, 1, 0] == grp.min() and bounds[j, 1, 1] == grp.max()
+        assert np.all(codes[j, 256:512] == 0)
+        x = O.dequantize_groups(codes, bounds, n, bits)
+        assert np.all(x[j, 256:512] == 0.25)
+        vals = sh.reshape(n, -1).T
+        for jj in range(12):
+            for g in range(3):
+                a, b = 256 * g, min(256 * (g + 1), n)
+                blk = vals[jj, a:b]
+                assert bounds[jj, g, 0] == blk.min() and bounds[jj, g, 1] == blk.max()
+                if blk.max() > blk.min():
+                    assert codes[jj, a + int(np.argmin(blk))] == 0
+                    assert codes[jj, a + int(np.argmax(blk))] == qmax
+                    step = (float(blk.max()) - float(blk.min())) / qmax
+                    err = np.abs(x[jj, a:b] - blk)
+                    # half a step, plus the float32 rounding of t = (x - min) inv
+                    # (a few ulps of t <= 2^b - 1)
+                    assert err.max() <= step * (0.5 + 4 * qmax * 2.0 ** -24) + 1e-6 * abs(blk).max()
+        assert np.all(codes[:, n:] == 0)    # padding untouched
+
+
+def test_stochastic_rounding_is_unbiased_and_adjacent():
+    rng = np.random.default_rng(3)
+    x = np.zeros((1, 256), np.float32)
+    x[0] = rng.uniform(-1, 1, 256).astype(np.float32)
+    x[0, 0], x[0, 1] = -1.0, 1.0            # pin the range to exactly [-1, 1]
+    qmax = 255
+    step = 2.0 / qmax
+    t = (x[0].astype(np.float64) + 1.0) / step
+    acc = np.zeros(256)
+    S = 400
+    for s in range(S):
+        c, b = O.quantize_groups(x, 256, 8, rounding=1, seed=1234, step=s + 1)
+        q = c[0].astype(np.float64)
+        assert np.all((q == np.floor(t + 1e-6)) | (q == np.floor(t + 1e-6) + 1)
+                      | (q == np.ceil(t - 1e-6)))
+        acc += -1.0 + q * step
+    mean = acc / S
+    # each draw's error is within one step with variance <= step^2 / 4
+    assert np.all(np.abs(mean - x[0]) < 5 * step / 2 / np.sqrt(S))
+
+
+def test_adam_on_quantised_state_against_plain_adam():
+    """16-bit codes with nearest rounding: the re-encoded parameters equal the
+    plain Adam step from the decoded values within half a step of the new
+    groups, and the moments are the bfloat16 of the plain moments."""
+    rng = np.random.default_rng(4)
+    n, K = 600, 4
+    sh = rng.normal(0, 0.5, (n, K, 3)).astype(np.float32)
+    codes, bounds = O.sh_quantize(sh, 16)
+    n_pad = codes.shape[1]
+    m16 = O.to_bf16(rng.normal(0, 1e-3, (12, n_pad)))
+    v16 = O.to_bf16(rng.uniform(0, 1e-6, (12, n_pad)))
+    grad = rng.normal(0, 1e-3, (n, K, 3)).astype(np.float32)
+    c2, b2, m2, v2, p_new = O.adam_sh_quant(codes, bounds, grad, m16, v16, n, 16, lr=2.5e-3,
+                                            step=3)
+    p0 = O.dequantize_groups(codes, bounds, n, 16)
+    g = grad.reshape(n, -1).T.astype(np.float64)
+    m0, v0 = O.from_bf16(m16[:, :n]), O.from_bf16(v16[:, :n])
+    m1 = 0.9 * m0 + 0.1 * g
+    v1 = 0.999 * v0 + 0.001 * g * g
+    p1 = p0 - 2.5e-3 * (m1 / (1 - 0.9 ** 3)) / (np.sqrt(v1 / (1 - 0.999 ** 3)) + 1e-15)
+    np.testing.assert_allclose(p_new, p1, rtol=1e-12, atol=1e-15)
+    assert np.array_equal(m2[:, :n], O.to_bf16(m1)) and np.array_equal(v2[:, :n], O.to_bf16(v1))
+    x = O.dequantize_groups(c2, b2, n, 16)
+    step = (b2[:, :, 1] - b2[:, :, 0]).astype(np.float64) / 65535
+    tol = step[:, np.arange(n) // 256] * (0.5 + 4 * 65535 * 2.0 ** -24) + 1e-7
+    assert np.all(np.abs(x - p1) <= tol)
+    # the moments' padding lanes are left alone
+    assert np.array_equal(m2[:, n:], m16[:, n:])
