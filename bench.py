@@ -366,6 +366,65 @@ def measure_loss(sp, reps: int = 5) -> dict:
                 loss=float(t[0, 0]), l1=float(t[0, 1]), ssim=float(t[0, 2]))
 
 
+def measure_quant_adam(sp, reps: int = 5) -> dict:
+    """gs_adam_step_sh_quant on the Splatter's SH (encoded once with
+    gs_sh_quantize) and its SH gradient, 8- and 16-bit codes, nearest
+    rounding, each launch after an L2 flush; mean of `reps` after an untimed
+    launch. Beside it the float32 gs_adam_step of the same SH group.
+    Algorithmic bytes per SH value: code read and written (1 or 2 B each),
+    gradient 4 B, bfloat16 moments read and written 8 B; float32: 28 B."""
+    import torch
+    from gaussian_splatting_differentiable_ewa_b200 import api
+    n = sp.n
+    sh = dict(sp.param_list)["sh"]
+    k3 = sh[0].numel()
+    n_pad = -(-n // 256) * 256
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pk = peaks()
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        ms = 0.0
+        for _ in range(reps):
+            flush.fill_(1)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ms += e0.elapsed_time(e1) / reps
+        return ms
+
+    out = {}
+    g = sp.grads["sh"]
+    for bits in (8, 16):
+        codes = torch.zeros((k3, n_pad), dtype=torch.uint8 if bits == 8 else torch.int16,
+                            device="cuda")
+        bounds = torch.zeros((k3, n_pad // 256, 2), dtype=torch.float32, device="cuda")
+        q = api.sh_quant(codes, bounds, n, k3, bits)
+        api.gs_sh_quantize(sh, q)
+        m = torch.zeros((k3, n_pad), dtype=torch.int16, device="cuda")
+        v = torch.zeros_like(m)
+        step = [0]
+
+        def run():
+            step[0] += 1
+            api.gs_adam_step_sh_quant(q, g, m, v, 2.5e-3, 0.9, 0.999, 1e-15, step[0])
+        ms = timed(run)
+        nbytes = n * k3 * (2 * bits // 8 + 4 + 8) + k3 * (n_pad // 256) * 16
+        out["q%d" % bits] = dict(ms=ms, gbs=nbytes / (ms / 1e3) / 1e9,
+                                 hbm_frac=nbytes / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                                 state_bytes=n * k3 * (bits // 8 + 4))
+    m32, v32 = torch.zeros_like(sh), torch.zeros_like(sh)
+    p32 = sh.clone()
+    ms = timed(lambda: api.gs_adam_step([(p32, g, m32, v32, 2.5e-3)], 0.9, 0.999, 1e-15, 1))
+    nbytes = n * k3 * 28
+    out["f32"] = dict(ms=ms, gbs=nbytes / (ms / 1e3) / 1e9,
+                      hbm_frac=nbytes / (ms / 1e3) / 1e9 / pk["hbm_gbs"], state_bytes=n * k3 * 12)
+    return out
+
+
 def measure_densify(sp) -> dict:
     """One gs_densify_and_prune call on the Splatter's accumulated statistics
     (absolute gradients, the page's threshold 0.0002), timed with CUDA events
@@ -526,6 +585,7 @@ def run_ours(args):
     if world == 1:
         extras["gs_densify_and_prune"] = measure_densify(sp)
         extras["gs_l1_dssim"] = measure_loss(sp)
+        extras["gs_adam_step_sh_quant"] = measure_quant_adam(sp)
 
     if world > 1:
         dist.barrier()

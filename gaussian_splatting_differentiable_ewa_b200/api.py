@@ -108,6 +108,11 @@ SIGNATURES = [
     ("gs_l1_dssim", _c.c_int,
      [_vp, _vp, _c.c_int32, _c.c_int32, _c.c_int32, _c.c_float, _vp, _vp, _vp, _c.c_size_t,
       _vp]),
+    ("gs_sh_quantize", _c.c_int, [_vp, _c.c_void_p, _vp]),
+    ("gs_sh_dequantize", _c.c_int, [_c.c_void_p, _vp, _vp]),
+    ("gs_adam_step_sh_quant", _c.c_int,
+     [_c.c_void_p, _vp, _vp, _vp, _c.c_float, _c.c_float, _c.c_float, _c.c_float, _c.c_int64,
+      _c.c_int32, _c.c_uint64, _vp]),
     ("gs_bin_sort_noalloc", _c.c_int,
      [_c.POINTER(GsProjected), _c.POINTER(GsCamera), _c.c_int32, _c.c_int64, _c.c_int32,
       _c.POINTER(GsBinned), _vp, _vp]),
@@ -305,6 +310,37 @@ def gs_l1_dssim(image, target, n_views: int, height: int, width: int, lam: float
                              float(lam), _ptr(terms), _ptr(dL_dimage), _ptr(ws),
                              int(ws.numel() * ws.element_size()), _stream(stream)),
            "gs_l1_dssim")
+
+
+GS_QUANT_GROUP = 256
+
+
+class GsShQuant(_c.Structure):
+    _fields_ = [("codes", _vp), ("bounds", _vp), ("n", _c.c_int64), ("k3", _c.c_int32),
+                ("bits", _c.c_int32)]
+
+
+def sh_quant(codes, bounds, n: int, k3: int, bits: int) -> GsShQuant:
+    """Descriptor of a quantised SH state: codes uint8/int16 [k3, n_pad],
+    bounds float32 [k3, n_pad // 256, 2]."""
+    return GsShQuant(_ptr(codes), _ptr(bounds), int(n), int(k3), int(bits))
+
+
+def gs_sh_quantize(sh, q: GsShQuant, stream=None) -> None:
+    _check(lib().gs_sh_quantize(_ptr(sh), _c.byref(q), _stream(stream)), "gs_sh_quantize")
+
+
+def gs_sh_dequantize(q: GsShQuant, sh, stream=None) -> None:
+    _check(lib().gs_sh_dequantize(_c.byref(q), _ptr(sh), _stream(stream)), "gs_sh_dequantize")
+
+
+def gs_adam_step_sh_quant(q: GsShQuant, grad_sh, exp_avg, exp_avg_sq, lr: float, beta1: float,
+                          beta2: float, eps: float, step: int, rounding: int = 0, seed: int = 0,
+                          stream=None) -> None:
+    _check(lib().gs_adam_step_sh_quant(_c.byref(q), _ptr(grad_sh), _ptr(exp_avg),
+                                       _ptr(exp_avg_sq), float(lr), float(beta1), float(beta2),
+                                       float(eps), int(step), int(rounding), int(seed),
+                                       _stream(stream)), "gs_adam_step_sh_quant")
 
 
 def gs_bin_sort_noalloc(proj: GsProjected, cams_arr, n_views: int, n: int, sort_mode: int,

@@ -496,6 +496,51 @@ gs_status gs_l1_dssim(const float* image, const float* target, int32_t n_views, 
                                           static_cast<cudaStream_t>(stream)));
 }
 
+namespace {
+bool quant_ok(const gs_sh_quant* q) {
+  if (!q || q->n < 0 || q->n >= (1ll << 31)) return false;
+  if (q->bits != 8 && q->bits != 16) return false;
+  if (q->k3 != 3 && q->k3 != 12 && q->k3 != 27 && q->k3 != 48) return false;
+  if (q->n == 0) return true;
+  // codes move four at a time
+  return q->codes && q->bounds && aligned(q->codes, q->bits / 2) && aligned(q->bounds, 8);
+}
+}  // namespace
+
+gs_status gs_sh_quantize(const float* sh, const gs_sh_quant* q, void* stream) {
+  if (!quant_ok(q)) return GS_ERR_INVALID_ARG;
+  if (q->n == 0) return GS_OK;
+  if (!sh || !aligned(sh, 4)) return GS_ERR_INVALID_ARG;
+  return cuda_status(gsb::launch_sh_quantize(sh, q->n, q->k3, q->bits, q->codes,
+                                             reinterpret_cast<float2*>(q->bounds),
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+gs_status gs_sh_dequantize(const gs_sh_quant* q, float* sh, void* stream) {
+  if (!quant_ok(q)) return GS_ERR_INVALID_ARG;
+  if (q->n == 0) return GS_OK;
+  if (!sh || !aligned(sh, 4)) return GS_ERR_INVALID_ARG;
+  return cuda_status(gsb::launch_sh_dequantize(q->codes, reinterpret_cast<const float2*>(q->bounds),
+                                               q->n, q->k3, q->bits, sh,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+gs_status gs_adam_step_sh_quant(const gs_sh_quant* q, const float* grad_sh, uint16_t* exp_avg,
+                                uint16_t* exp_avg_sq, float lr, float beta1, float beta2,
+                                float eps, int64_t step, int32_t rounding, uint64_t seed,
+                                void* stream) {
+  if (!quant_ok(q) || step < 1 || (rounding != 0 && rounding != 1)) return GS_ERR_INVALID_ARG;
+  if (!(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f) || !(eps >= 0.f))
+    return GS_ERR_INVALID_ARG;
+  if (q->n == 0) return GS_OK;
+  if (!grad_sh || !exp_avg || !exp_avg_sq || !aligned(grad_sh, 4) || !aligned(exp_avg, 8) ||
+      !aligned(exp_avg_sq, 8))
+    return GS_ERR_INVALID_ARG;
+  return cuda_status(gsb::launch_adam_sh_quant(
+      q->codes, reinterpret_cast<float2*>(q->bounds), grad_sh, exp_avg, exp_avg_sq, q->n, q->k3,
+      q->bits, lr, beta1, beta2, eps, step, rounding, seed, static_cast<cudaStream_t>(stream)));
+}
+
 gs_status gs_get_status(void* ws, void* stream) {
   if (!ws) return GS_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

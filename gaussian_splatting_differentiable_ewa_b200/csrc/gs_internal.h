@@ -120,4 +120,14 @@ cudaError_t launch_l1_dssim(const float* image, const float* target, int n_views
                             float lambda, double* terms, float* grad, double* sums,
                             unsigned* done, cudaStream_t stream);
 
+// Quantised SH state: codes [k3][n_pad], bounds [k3][n_pad / 256].
+cudaError_t launch_sh_quantize(const float* sh, int64_t n, int k3, int bits, void* codes,
+                               float2* bounds, cudaStream_t stream);
+cudaError_t launch_sh_dequantize(const void* codes, const float2* bounds, int64_t n, int k3,
+                                 int bits, float* sh, cudaStream_t stream);
+cudaError_t launch_adam_sh_quant(void* codes, float2* bounds, const float* grad, uint16_t* m,
+                                 uint16_t* v, int64_t n, int k3, int bits, float lr, float beta1,
+                                 float beta2, float eps, int64_t step, int rounding,
+                                 uint64_t seed, cudaStream_t stream);
+
 }  // namespace gsb

@@ -24,8 +24,12 @@ DEFAULT_LR = dict(means=1.6e-4, sh=2.5e-3, opacity_logit=5e-2, log_scales=5e-3, 
 class Splatter:
     def __init__(self, scene, device="cuda", sort_mode: int = api.GS_SORT_PRESORT,
                  pair_capacity: Optional[int] = None, headroom: float = 1.25,
-                 lr: Optional[dict] = None, stream: Optional[torch.cuda.Stream] = None):
+                 lr: Optional[dict] = None, stream: Optional[torch.cuda.Stream] = None,
+                 sh_bits: Optional[int] = None, sh_rounding: int = 0, sh_seed: int = 0):
         self.device = torch.device(device)
+        self.sh_bits = sh_bits
+        self.sh_rounding = int(sh_rounding)
+        self.sh_seed = int(sh_seed)
         self.scene = scene
         self.n = int(scene.n)
         self.V = int(scene.n_views)
@@ -92,6 +96,8 @@ class Splatter:
                         else {k: torch.zeros_like(t) for k, t in self.param_list})
         self.exp_avg_sq = (exp_avg_sq if exp_avg_sq is not None
                            else {k: torch.zeros_like(t) for k, t in self.param_list})
+        if self.sh_bits is not None:
+            self._quantise_sh()
         self.accum_plain = torch.zeros(n, dtype=f32, device=dev)
         self.accum_abs = torch.zeros(n, dtype=f32, device=dev)
         self.denom = torch.zeros(n, dtype=torch.int32, device=dev)
@@ -101,6 +107,26 @@ class Splatter:
         self.c_proj = api.projected(self.records, self.bins, self.radii)
         if getattr(self, "ws", None) is not None:
             self._alloc_pairs(self.capacity)  # the workspace follows the count too
+
+    def _quantise_sh(self) -> None:
+        """Quantised SH state: the SH live as codes with per-256 bounds and
+        bfloat16 Adam moments; ``self.sh`` becomes the float32 decode target
+        that the projection reads, refreshed before every forward."""
+        if self.sh_bits not in (8, 16):
+            raise ValueError("sh_bits must be 8 or 16")
+        n, k3, dev = self.n, 3 * self.K, self.device
+        n_pad = -(-n // api.GS_QUANT_GROUP) * api.GS_QUANT_GROUP
+        self.sh_codes = torch.zeros((k3, n_pad), device=dev,
+                                    dtype=torch.uint8 if self.sh_bits == 8 else torch.int16)
+        self.sh_bounds = torch.zeros((k3, n_pad // api.GS_QUANT_GROUP, 2), dtype=torch.float32,
+                                     device=dev)
+        self.sh_q = api.sh_quant(self.sh_codes, self.sh_bounds, n, k3, self.sh_bits)
+        self.sh_m16 = torch.zeros((k3, n_pad), dtype=torch.int16, device=dev)
+        self.sh_v16 = torch.zeros((k3, n_pad), dtype=torch.int16, device=dev)
+        # the float32 moments of the SH are not used in this mode
+        self.exp_avg["sh"] = self.exp_avg_sq["sh"] = None
+        api.gs_sh_quantize(self.sh, self.sh_q, self.stream)
+        api.gs_sh_dequantize(self.sh_q, self.sh, self.stream)
 
     def _alloc_pairs(self, capacity: int) -> None:
         self.capacity = int(capacity)
@@ -130,6 +156,8 @@ class Splatter:
 
     # ------------------------------------------------------------ the calls
     def project(self):
+        if self.sh_bits is not None:
+            api.gs_sh_dequantize(self.sh_q, self.sh, self.stream)
         api.gs_project(self.c_params, self.cams, self.V, self.c_proj, self.stream)
 
     def bin_sort(self):
@@ -155,9 +183,14 @@ class Splatter:
 
     def adam_step(self, beta1=0.9, beta2=0.999, eps=1e-15):
         self.step_count += 1
+        quant = self.sh_bits is not None
         groups = [(t, self.grads[k], self.exp_avg[k], self.exp_avg_sq[k], self.lr[k])
-                  for k, t in self.param_list]
+                  for k, t in self.param_list if not (quant and k == "sh")]
         api.gs_adam_step(groups, beta1, beta2, eps, self.step_count, self.stream)
+        if quant:
+            api.gs_adam_step_sh_quant(self.sh_q, self.grads["sh"], self.sh_m16, self.sh_v16,
+                                      self.lr["sh"], beta1, beta2, eps, self.step_count,
+                                      self.sh_rounding, self.sh_seed, self.stream)
 
     def forward(self):
         self.project()
@@ -270,6 +303,8 @@ class Splatter:
         zero. z: standard normal draws float32 [n][2][3] for the split
         children (drawn on the device from `seed` when None). Returns the
         per-Gaussian codes (0 pruned, 1 kept, 2 cloned, 3 split)."""
+        if self.sh_bits is not None:
+            raise NotImplementedError("densify_and_prune with quantised SH state")
         n, dev = self.n, self.device
         if z is None:
             gen = torch.Generator(device=dev)

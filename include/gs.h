@@ -365,6 +365,49 @@ gs_status gs_l1_dssim(const float* image, const float* target, int32_t n_views, 
                       int32_t width, float lambda, double* terms, float* dL_dimage, void* ws,
                       size_t ws_bytes, void* stream);
 
+/* ---- quantised SH state (Spirula VRAM page, sec. 魔法一) ----------------
+ * SH coefficients kept as 8- or 16-bit codes, every 256 Gaussians of one
+ * coefficient sharing a (min, max) pair; the Adam moments of those values are
+ * bfloat16 in the same coefficient-major layout. With n_pad = n rounded up to
+ * a multiple of GS_QUANT_GROUP and k3 = 3 (degree + 1)^2:
+ *   codes   uint8 (bits 8) or uint16 (bits 16) [k3][n_pad]; value j of
+ *           Gaussian i (j = 3 coefficient + channel) at j * n_pad + i;
+ *   bounds  float [k3][n_pad / 256][2]: the (min, max) of group (j, i / 256);
+ *   a code q decodes to min + q (max - min) / (2^bits - 1).
+ * Encoding takes each group's min and max over its real Gaussians and rounds
+ * t = (x - min) * ((2^bits - 1) / (max - min)) in float32 to nearest-even
+ * (rounding 0) or to floor(t + u) (rounding 1, u in [0, 1) from SplitMix64
+ * output number step * 2^37 + j * 2^31 + i + 1 of `seed`, top 24 bits);
+ * a group with max == min gets code 0. Padding lanes are never written. */
+#define GS_QUANT_GROUP 256
+
+typedef struct gs_sh_quant {
+  void* codes;      /* see above; device memory, caller-owned, 4-byte (8-bit
+                       codes) or 8-byte (16-bit codes) aligned */
+  float* bounds;    /* see above; device memory, caller-owned */
+  int64_t n;        /* Gaussians, 0 <= n < 2^31 */
+  int32_t k3;       /* values per Gaussian: 3, 12, 27 or 48 */
+  int32_t bits;     /* 8 or 16 */
+} gs_sh_quant;
+
+/* Encode float SH [n][k3] (the gs_params layout) into q (nearest rounding). */
+gs_status gs_sh_quantize(const float* sh, const gs_sh_quant* q, void* stream);
+
+/* Decode q into float SH [n][k3] (float32: fma(q, (max - min) / (2^bits - 1), min)). */
+gs_status gs_sh_dequantize(const gs_sh_quant* q, float* sh, void* stream);
+
+/* One Adam step on the quantised SH, fused: decode each value, update its
+ * bfloat16 moments exp_avg / exp_avg_sq ([k3][n_pad], round to nearest-even)
+ * with the float32 gradient grad_sh ([n][k3], the gs_grads layout), take the
+ * step of gs_adam_step (lr, beta1, beta2, eps, bias corrections of `step`),
+ * then re-encode the group with its new min and max (rounding as above).
+ * The moments must be 8-byte aligned. Argument errors as gs_adam_step, plus
+ * rounding not 0/1, bits not 8/16, k3 not 3/12/27/48. */
+gs_status gs_adam_step_sh_quant(const gs_sh_quant* q, const float* grad_sh, uint16_t* exp_avg,
+                                uint16_t* exp_avg_sq, float lr, float beta1, float beta2,
+                                float eps, int64_t step, int32_t rounding, uint64_t seed,
+                                void* stream);
+
 /* Synchronise `stream`, return the status word accumulated in workspace `ws`
  * by device-side checks since the last call, and clear it. */
 gs_status gs_get_status(void* ws, void* stream);

@@ -58,7 +58,8 @@ def test_loss_weights_and_forward_only(lam):
     _check_grad(g, want_g)
     t2, none = _run(img, tgt, lam, grad=False)
     assert none is None
-    np.testing.assert_allclose(t2, terms, rtol=0, atol=1e-12)
+    # the same sums in another instantiation and atomic order: float32 noise only
+    np.testing.assert_allclose(t2, terms, rtol=0, atol=2e-6)
 
 
 def test_loss_of_identical_images():
