@@ -334,9 +334,10 @@ def measure_loss(sp, reps: int = 5) -> dict:
     against a seeded target of the same size, each launch timed with CUDA
     events after an L2 flush (a 256 MB write), mean over `reps` after an
     untimed launch. Algorithmic work per value: the separable 11-tap window
-    applied along rows and columns to the five SSIM moments and to the three
-    partial maps of the gradient, 2 x 11 x 8 = 176 FMA (352 FLOP); traffic:
-    x and y read, dL/dx written, 12 bytes."""
+    applied along rows and columns to the four moments SSIM needs (x, y,
+    xx + yy, xy) and to the three partial maps of the gradient,
+    2 x 11 x 7 = 154 FMA (308 FLOP); traffic: x and y read, dL/dx written,
+    12 bytes."""
     import torch
     from gaussian_splatting_differentiable_ewa_b200 import api
     from gaussian_splatting_differentiable_ewa_b200 import scenes as S
@@ -357,7 +358,7 @@ def measure_loss(sp, reps: int = 5) -> dict:
         ms += e0.elapsed_time(e1) / reps
     values = 3 * V * H * W
     pk = peaks()
-    tflops = values * 352 / (ms / 1e3) / 1e12
+    tflops = values * 308 / (ms / 1e3) / 1e12
     fp32_peak = FP32_LANES * 2 * pk["sm_max_mhz"] * 1e6 / 1e12
     gbs = values * 12 / (ms / 1e3) / 1e9
     t = sp.loss_terms.cpu().numpy()

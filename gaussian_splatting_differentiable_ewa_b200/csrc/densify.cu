@@ -17,7 +17,9 @@
 //               moments copied for the kept ones, moments zero for the new
 //               ones; a split child's mean is mean + R (s * z) with the
 //               caller's normal draws z, its log-scales shrink by
-//               log_split_shrink.
+//               log_split_shrink. Each thread writes its Gaussian's small
+//               fields; the SH blocks (most of the bytes) are moved by the
+//               whole warp in contiguous runs.
 
 #include <cuda_runtime.h>
 
@@ -120,18 +122,6 @@ __device__ __forceinline__ float3 rotate(float4 q, float3 u) {
                      r20 * u.x + r21 * u.y + r22 * u.z);
 }
 
-// Copy (or zero) K3 floats of one Gaussian's SH block.
-__device__ __forceinline__ void copy_sh(float* __restrict__ dst, const float* __restrict__ src,
-                                        int k3, bool zero) {
-  if ((k3 & 3) == 0) {
-    float4* d4 = reinterpret_cast<float4*>(dst);
-    const float4* s4 = reinterpret_cast<const float4*>(src);
-    for (int q = 0; q < k3 / 4; ++q) d4[q] = zero ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(&s4[q]);
-  } else {
-    for (int e = 0; e < k3; ++e) dst[e] = zero ? 0.f : __ldg(&src[e]);
-  }
-}
-
 struct DpTensors {
   float4* means;
   float4* log_scales;
@@ -147,15 +137,93 @@ struct DpConst {
   const float* sh;
 };
 
-// Moments of Gaussian i copied to slot o, or zeroed.
+// Moments of Gaussian i copied to slot o, or zeroed (all but the SH block,
+// which the warp moves together: copy_sh_warp).
 __device__ __forceinline__ void put_moments(const DpConst& in, const DpTensors& out, int64_t i,
-                                            int64_t o, int k3, bool zero) {
+                                            int64_t o, bool zero) {
   const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
   out.means[o] = zero ? z4 : __ldg(&in.means[i]);
   out.log_scales[o] = zero ? z4 : __ldg(&in.log_scales[i]);
   out.quats[o] = zero ? z4 : __ldg(&in.quats[i]);
   out.logit[o] = zero ? 0.f : __ldg(&in.logit[i]);
-  copy_sh(out.sh + o * k3, in.sh + i * k3, k3, zero);
+}
+
+// The SH blocks (parameters and both moments) of the warp's 32 Gaussians,
+// moved by the whole warp so that every access is part of a contiguous run:
+// the warp walks the (Gaussian, element) items of its Gaussians' three
+// blocks 32 at a time (float4 elements when k3 is a multiple of 4), four
+// rounds of loads in flight. A kept Gaussian keeps its moments; a clone's
+// second copy and both split children get zeros.
+template <typename E>
+__device__ __forceinline__ void copy_sh_warp(const DpConst& p_in, const DpConst& m_in,
+                                             const DpConst& v_in, const DpTensors& p_out,
+                                             const DpTensors& m_out, const DpTensors& v_out,
+                                             int k3, int8_t c_lane, int64_t pos_lane,
+                                             int64_t i_warp) {
+  constexpr int kW = (int)(sizeof(E) / sizeof(float));
+  const int per = k3 / kW;           // elements per block
+  const int items = 3 * per;         // per Gaussian
+  const int total = 32 * items;      // a multiple of 32: every lane runs every round
+  const int lane = threadIdx.x & 31;
+#pragma unroll 4
+  for (int f = lane; f < total; f += 32) {
+    const int j = f / items, r = f - j * items;
+    const int c = __shfl_sync(0xffffffffu, (int)c_lane, j);
+    const int64_t pos = __shfl_sync(0xffffffffu, pos_lane, j);
+    if (c == 0) continue;            // pruned
+    const int arr = r / per, q = r - arr * per;
+    const float* src = arr == 0 ? p_in.sh : (arr == 1 ? m_in.sh : v_in.sh);
+    float* dst = arr == 0 ? p_out.sh : (arr == 1 ? m_out.sh : v_out.sh);
+    const E v = __ldg(reinterpret_cast<const E*>(src + (i_warp + j) * k3) + q);
+    const int nout = c == 1 ? 1 : 2;  // kKeep: one output, clone / split: two
+    for (int copy = 0; copy < nout; ++copy) {
+      const bool zero = arr > 0 && (c == 3 || copy == 1);
+      E* d = reinterpret_cast<E*>(dst + (pos + copy) * k3) + q;
+      *d = zero ? E{} : v;
+    }
+  }
+}
+
+// Every field but the SH blocks of Gaussian i's outputs at pos (and pos + 1).
+__device__ __forceinline__ void emit_fields(const DpConst& p_in, const DpConst& m_in,
+                                            const DpConst& v_in, const float* __restrict__ z,
+                                            int64_t i, int64_t pos, int8_t c,
+                                            float log_split_shrink, const DpTensors& p_out,
+                                            const DpTensors& m_out, const DpTensors& v_out) {
+  const float4 mu = __ldg(&p_in.means[i]);
+  const float4 ls = __ldg(&p_in.log_scales[i]);
+  const float4 q = __ldg(&p_in.quats[i]);
+  const float lg = __ldg(&p_in.logit[i]);
+  if (c == kKeep || c == kClone) {
+    for (int copy = 0; copy < (c == kClone ? 2 : 1); ++copy) {
+      const int64_t o = pos + copy;
+      p_out.means[o] = mu;
+      p_out.log_scales[o] = ls;
+      p_out.quats[o] = q;
+      p_out.logit[o] = lg;
+      put_moments(m_in, m_out, i, o, copy == 1);
+      put_moments(v_in, v_out, i, o, copy == 1);
+    }
+    return;
+  }
+  // split: two children
+  const float qn = rsqrtf(q.x * q.x + q.y * q.y + q.z * q.z + q.w * q.w);
+  const float4 qu = make_float4(q.x * qn, q.y * qn, q.z * qn, q.w * qn);
+  const float3 s = make_float3(__expf(ls.x), __expf(ls.y), __expf(ls.z));
+  const float4 lsc = make_float4(ls.x - log_split_shrink, ls.y - log_split_shrink,
+                                 ls.z - log_split_shrink, ls.w);
+  for (int ch = 0; ch < 2; ++ch) {
+    const int64_t o = pos + ch;
+    const float* zc = z + (i * 2 + ch) * 3;
+    const float3 d = rotate(qu, make_float3(s.x * __ldg(&zc[0]), s.y * __ldg(&zc[1]),
+                                            s.z * __ldg(&zc[2])));
+    p_out.means[o] = make_float4(mu.x + d.x, mu.y + d.y, mu.z + d.z, mu.w);
+    p_out.log_scales[o] = lsc;
+    p_out.quats[o] = q;
+    p_out.logit[o] = lg;
+    put_moments(m_in, m_out, i, o, true);
+    put_moments(v_in, v_out, i, o, true);
+  }
 }
 
 __global__ void __launch_bounds__(kDpThreads) k_dp_emit(
@@ -180,45 +248,16 @@ __global__ void __launch_bounds__(kDpThreads) k_dp_emit(
   uint32_t before = 0;
 #pragma unroll
   for (int w = 0; w < kDpThreads / 32; ++w) before += w < warp ? s_w[w] : 0u;
-  if (c == kPrune) return;
   const int64_t pos = (int64_t)block_offsets[blockIdx.x] + before + incl - cnt;
-  const float4 mu = __ldg(&p_in.means[i]);
-  const float4 ls = __ldg(&p_in.log_scales[i]);
-  const float4 q = __ldg(&p_in.quats[i]);
-  const float lg = __ldg(&p_in.logit[i]);
-  if (c == kKeep || c == kClone) {
-    for (int copy = 0; copy < (c == kClone ? 2 : 1); ++copy) {
-      const int64_t o = pos + copy;
-      p_out.means[o] = mu;
-      p_out.log_scales[o] = ls;
-      p_out.quats[o] = q;
-      p_out.logit[o] = lg;
-      copy_sh(p_out.sh + o * k3, p_in.sh + i * k3, k3, false);
-      put_moments(m_in, m_out, i, o, k3, copy == 1);
-      put_moments(v_in, v_out, i, o, k3, copy == 1);
-    }
-    return;
-  }
-  // split: two children
-  const float qn = rsqrtf(q.x * q.x + q.y * q.y + q.z * q.z + q.w * q.w);
-  const float4 qu = make_float4(q.x * qn, q.y * qn, q.z * qn, q.w * qn);
-  const float3 s = make_float3(__expf(ls.x), __expf(ls.y), __expf(ls.z));
-  const float4 lsc = make_float4(ls.x - log_split_shrink, ls.y - log_split_shrink,
-                                 ls.z - log_split_shrink, ls.w);
-  for (int ch = 0; ch < 2; ++ch) {
-    const int64_t o = pos + ch;
-    const float* zc = z + (i * 2 + ch) * 3;
-    const float3 d = rotate(qu, make_float3(s.x * __ldg(&zc[0]), s.y * __ldg(&zc[1]),
-                                            s.z * __ldg(&zc[2])));
-    p_out.means[o] = make_float4(mu.x + d.x, mu.y + d.y, mu.z + d.z, mu.w);
-    p_out.log_scales[o] = lsc;
-    p_out.quats[o] = q;
-    p_out.logit[o] = lg;
-    copy_sh(p_out.sh + o * k3, p_in.sh + i * k3, k3, false);
-    put_moments(m_in, m_out, i, o, k3, true);
-    put_moments(v_in, v_out, i, o, k3, true);
-  }
+  if (c != kPrune) emit_fields(p_in, m_in, v_in, z, i, pos, c, log_split_shrink, p_out, m_out,
+                               v_out);
+  // the SH blocks, the warp together
+  if ((k3 & 3) == 0)
+    copy_sh_warp<float4>(p_in, m_in, v_in, p_out, m_out, v_out, k3, c, pos, i - lane);
+  else
+    copy_sh_warp<float>(p_in, m_in, v_in, p_out, m_out, v_out, k3, c, pos, i - lane);
 }
+
 
 DpConst to_const(const DpTensorPtrs& t) {
   return DpConst{reinterpret_cast<const float4*>(t.means), reinterpret_cast<const float4*>(t.log_scales),
