@@ -75,3 +75,29 @@ def test_bad_arguments_are_rejected_before_any_cuda_call():
     assert L.gs_adam_step(grp, 1, 1.5, 0.999, 1e-15, 1, None) == api.GS_ERR_INVALID_ARG
     assert L.gs_densify_stats(None, None, 0, 10, None, None, None, None) == api.GS_ERR_INVALID_ARG
     assert L.gs_get_status(None, None) == api.GS_ERR_INVALID_ARG
+
+
+def test_loss_and_quant_arguments_are_rejected_before_any_cuda_call():
+    L = api.lib()
+    assert api.gs_l1_dssim_workspace_size(3) == 3 * 16 + 16
+    assert api.gs_l1_dssim_workspace_size(-1) == 0
+    p = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+    bad = [(p, p, 1, 0, 8, 0.2, p, None, p, 64),        # empty image
+           (p, p, 1, 8, 8, 1.5, p, None, p, 64),        # lambda outside [0, 1]
+           (None, p, 1, 8, 8, 0.2, p, None, p, 64),     # no image
+           (p, p, 1, 8, 8, 0.2, p, None, p, 8),         # workspace too small
+           (p, p, 21846, 8, 8, 0.2, p, None, p, 1 << 20)]
+    for a in bad:
+        assert L.gs_l1_dssim(*a, None) == api.GS_ERR_INVALID_ARG, a
+    assert L.gs_l1_dssim(None, None, 0, 0, 0, 0.2, None, None, None, 0, None) == api.GS_OK
+    q = api.GsShQuant(16, 16, 100, 12, 12)              # 12-bit codes
+    assert L.gs_sh_quantize(p, ctypes.byref(q), None) == api.GS_ERR_INVALID_ARG
+    q = api.GsShQuant(16, 16, 100, 10, 8)               # k3 not 3 (K) for K in 1, 4, 9, 16
+    assert L.gs_sh_dequantize(ctypes.byref(q), p, None) == api.GS_ERR_INVALID_ARG
+    q = api.GsShQuant(16, 16, 100, 12, 8)
+    assert L.gs_adam_step_sh_quant(ctypes.byref(q), p, p, p, 1e-3, 0.9, 0.999, 1e-15, 1, 2, 0,
+                                   None) == api.GS_ERR_INVALID_ARG   # rounding 2
+    assert L.gs_adam_step_sh_quant(ctypes.byref(q), p, p, p, 1e-3, 1.0, 0.999, 1e-15, 1, 0, 0,
+                                   None) == api.GS_ERR_INVALID_ARG   # beta1 1
+    q = api.GsShQuant(None, None, 0, 12, 8)
+    assert L.gs_sh_quantize(None, ctypes.byref(q), None) == api.GS_OK
