@@ -433,14 +433,16 @@ __global__ void __launch_bounds__(1024) k_tile_base(
 // rectangles in depth order, 32 per coalesced load, and for each one that
 // reaches the region writes its pairs at once, one lane per tile (a rectangle
 // has one pair per tile, so no two lanes share a counter), straight to their
-// final positions.
+// final positions. The counters' rows are padded by one word so that the
+// tiles of a rectangle's column sit in different banks.
+constexpr int kNextPitch = kRegionCols + 1;
 __global__ void __launch_bounds__(32 * kEmitWarps) k_emit_tiles(
     const uint4* __restrict__ crect, int gsize, const uint32_t* __restrict__ n_visible, Grid g,
     int n_regions, const uint32_t* __restrict__ offsets, int64_t stride,
     const uint32_t* __restrict__ tile_base, const unsigned long long* __restrict__ pair_total,
     uint32_t* __restrict__ ids_out, int64_t capacity, uint32_t* __restrict__ status) {
   constexpr int kTiles = kRegionCols * kRegionRows;
-  __shared__ uint32_t s_next_all[kEmitWarps][kTiles];
+  __shared__ uint32_t s_next_all[kEmitWarps][kRegionRows * kNextPitch];
   if ((int64_t)*pair_total > capacity) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int region = blockIdx.y * kEmitWarps + warp;  // warps of a block: regions side by side
@@ -457,13 +459,14 @@ __global__ void __launch_bounds__(32 * kEmitWarps) k_emit_tiles(
   if (first >= last) return;
   const int tpv = g.tiles_per_view;
   for (int li = lane; li < kTiles; li += 32) {
-    const int r = r0 + li / kRegionCols, c = c0 + li % kRegionCols;
+    const int rr = li / kRegionCols, cc = li % kRegionCols;
+    const int r = r0 + rr, c = c0 + cc;
     uint32_t next = 0;
     if (r <= r1 && c <= c1) {
       const int64_t t = (int64_t)v * tpv + (int64_t)r * g.tiles_x + c;
       next = tile_base[t] + offsets[tcount_index(t, b, stride)];
     }
-    s_next[li] = next;
+    s_next[rr * kNextPitch + cc] = next;
   }
   __syncwarp();
   uint4 cur = make_uint4(1u, 0u, 0u, 0u), nxt = make_uint4(1u, 0u, 0u, 0u);
@@ -492,7 +495,7 @@ __global__ void __launch_bounds__(32 * kEmitWarps) k_emit_tiles(
         if (p < np) {
           const int rr = min((int)(((float)p + 0.5f) * inv_wp), ry1 - ry0);
           const int cc = p - rr * wp;
-          const int li = (ry0 - r0 + rr) * kRegionCols + (cx0 - c0 + cc);
+          const int li = (ry0 - r0 + rr) * kNextPitch + (cx0 - c0 + cc);
           const uint32_t pos = s_next[li];
           s_next[li] = pos + 1;
           if ((int64_t)pos < capacity) ids_out[pos] = id;
