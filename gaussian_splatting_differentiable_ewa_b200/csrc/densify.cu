@@ -226,7 +226,7 @@ __device__ __forceinline__ void emit_fields(const DpConst& p_in, const DpConst& 
   }
 }
 
-__global__ void __launch_bounds__(kDpThreads) k_dp_emit(
+__global__ void __launch_bounds__(kDpThreads, 6) k_dp_emit(
     DpConst p_in, DpConst m_in, DpConst v_in, const float* __restrict__ z, int n, int k3,
     float log_split_shrink, const int8_t* __restrict__ codes,
     const uint32_t* __restrict__ block_offsets, const int64_t* __restrict__ n_out,
