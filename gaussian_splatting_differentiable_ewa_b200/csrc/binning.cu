@@ -152,7 +152,8 @@ __global__ void __launch_bounds__(256) k_depth_keys(const float4* __restrict__ b
                                                    int n_views, uint64_t* __restrict__ keys,
                                                    uint32_t* __restrict__ vals,
                                                    int64_t* __restrict__ n_items_out,
-                                                   uint32_t* __restrict__ n_visible) {
+                                                   uint32_t* __restrict__ n_visible,
+                                                   uint32_t* __restrict__ status) {
   __shared__ uint32_t s_vis[GS_MAX_VIEWS];
   if (threadIdx.x < GS_MAX_VIEWS) s_vis[threadIdx.x] = 0u;
   __syncthreads();
@@ -161,6 +162,7 @@ __global__ void __launch_bounds__(256) k_depth_keys(const float4* __restrict__ b
   for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < total;
        j += (int64_t)gridDim.x * blockDim.x) {
     const float4 r2 = __ldg(&bins[j]);  // depth key, tile_x, tile_y
+    if (__float_as_uint(r2.x) == kNonfiniteKeyBits) atomicOr(status, kStatusNonfinite);
     const uint32_t txw = __float_as_uint(r2.y), tyw = __float_as_uint(r2.z);
     const bool vis = (txw & 0xffffu) <= (txw >> 16) && (tyw & 0xffffu) <= (tyw >> 16);
     const int view = (int)(j / n);
@@ -760,6 +762,8 @@ __global__ void __launch_bounds__(kEmitThreads) k_emit(
       }
       if (vw >= 0) {
         const float4 r2 = __ldg(&bins[rec_index]);
+        if (MODE == 0 && __float_as_uint(r2.x) == kNonfiniteKeyBits)
+          atomicOr(status, kStatusNonfinite);
         const uint32_t txw = __float_as_uint(r2.y), tyw = __float_as_uint(r2.z);
         const uint32_t x0 = txw & 0xffffu, x1 = txw >> 16, y0 = tyw & 0xffffu, y1 = tyw >> 16;
         if (x0 <= x1 && y0 <= y1) {
@@ -1249,7 +1253,7 @@ cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
     int64_t blocks = (n_items + 255) / 256;
     if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
     k_depth_keys<<<(int)blocks, 256, 0, stream>>>(bins4, a.n, a.n_views, a.pkeys[0], a.pvals[0],
-                                                  a.n_items_dev, a.n_visible);
+                                                  a.n_items_dev, a.n_visible, a.status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     e = run_radix_passes<uint64_t, kPresortItems>(a.pkeys[0], a.pvals[0], a.pkeys[1], a.pvals[1],
                                                   a.n_items_dev, n_items, n_items, a.presort,

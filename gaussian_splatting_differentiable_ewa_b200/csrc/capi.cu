@@ -553,6 +553,7 @@ gs_status gs_get_status(void* ws, void* stream) {
   if (word & kStatusTimeout) return GS_ERR_DEVICE_TIMEOUT;
   if (word & kStatusBounds) return GS_ERR_OVERFLOW;
   if (word & kStatusCapacity) return GS_ERR_CAPACITY;
+  if (word & kStatusNonfinite) return GS_ERR_NONFINITE;
   return GS_OK;
 }
 

@@ -19,7 +19,8 @@
 //               caller's normal draws z, its log-scales shrink by
 //               log_split_shrink. Each thread writes its Gaussian's small
 //               fields; the SH blocks (most of the bytes) are moved by the
-//               whole warp in contiguous runs.
+//               whole warp in contiguous runs; six blocks per SM (40
+//               registers) keep more of those runs in flight.
 
 #include <cuda_runtime.h>
 

@@ -22,6 +22,12 @@ constexpr int kMaxRadius = 1 << 30;            // radius saturation
 constexpr uint32_t kStatusCapacity = 1u << 0;
 constexpr uint32_t kStatusTimeout = 1u << 1;
 constexpr uint32_t kStatusBounds = 1u << 2;
+constexpr uint32_t kStatusNonfinite = 1u << 3;
+
+// Depth key that marks a Gaussian culled for a non-finite parameter or
+// colour (a quiet NaN no depth computation produces); the binning raises
+// kStatusNonfinite when it meets one.
+constexpr uint32_t kNonfiniteKeyBits = 0x7FC0BAD0u;
 
 // Spin limit of every device-side wait (iterations of ~100 ns each).
 constexpr uint32_t kSpinLimit = 20u * 1000u * 1000u;

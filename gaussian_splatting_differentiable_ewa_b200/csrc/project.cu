@@ -154,7 +154,7 @@ __device__ __forceinline__ void unstage_sh(float* __restrict__ dst, int64_t i0, 
 // memory (16-byte loads when the per-Gaussian block allows) at unit direction
 // (x, y, z): rgb_c = max(0, sum_k Y_k sh_kc + 0.5).
 template <int DEG>
-__device__ __forceinline__ void sh_colour_global(const float* __restrict__ shi, float x, float y,
+__device__ __forceinline__ bool sh_colour_global(const float* __restrict__ shi, float x, float y,
                                                  float z, float rgb[3]) {
   constexpr int K = (DEG + 1) * (DEG + 1);
   float Y[16];
@@ -178,12 +178,13 @@ __device__ __forceinline__ void sh_colour_global(const float* __restrict__ shi, 
   }
 #pragma unroll
   for (int ch = 0; ch < 3; ++ch) rgb[ch] = fmaxf(acc[ch], 0.f);
+  return isfinite(acc[0] + acc[1] + acc[2]);  // before the clamp, which drops a NaN
 }
 
 // Colour from the SH coefficients of one Gaussian staged in shared memory
 // (16-byte loads), same arithmetic as sh_colour_global.
 template <int DEG>
-__device__ __forceinline__ void sh_colour_smem(const float* __restrict__ shi, float x, float y,
+__device__ __forceinline__ bool sh_colour_smem(const float* __restrict__ shi, float x, float y,
                                                float z, float rgb[3]) {
   constexpr int K = (DEG + 1) * (DEG + 1);
   float Y[16];
@@ -207,6 +208,7 @@ __device__ __forceinline__ void sh_colour_smem(const float* __restrict__ shi, fl
   }
 #pragma unroll
   for (int ch = 0; ch < 3; ++ch) rgb[ch] = fmaxf(acc[ch], 0.f);
+  return isfinite(acc[0] + acc[1] + acc[2]);  // before the clamp, which drops a NaN
 }
 
 template <int DEG>
@@ -245,6 +247,12 @@ __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __
   const float4 ls = __ldg(&log_scales[i]);
   const float4 q = __ldg(&quats[i]);
   const float lg = __ldg(&logit[i]);
+  // a non-finite parameter or a zero quaternion culls the Gaussian in every
+  // view and marks its depth key
+  const bool finite_in = isfinite(m.x) && isfinite(m.y) && isfinite(m.z) && isfinite(ls.x) &&
+                         isfinite(ls.y) && isfinite(ls.z) && isfinite(q.x) && isfinite(q.y) &&
+                         isfinite(q.z) && isfinite(q.w) && isfinite(lg) &&
+                         (q.x != 0.f || q.y != 0.f || q.z != 0.f || q.w != 0.f);
 
   // view-independent: M = R diag(exp(s)) in double
   double qw = q.x, qx = q.y, qy = q.z, qz = q.w;
@@ -282,7 +290,8 @@ __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __
 #pragma unroll
     for (int k = 0; k < 12; ++k) rec[k] = 0.f;
     int radius = 0;
-    bool ok = key >= (float)kNear;
+    bool nonfinite = !finite_in;
+    bool ok = finite_in && key >= (float)kNear;
     long long x0 = 1, x1 = 0, y0 = 1, y1 = 0;
     if (ok) {
       const double iz = 1.0 / tz;
@@ -346,16 +355,22 @@ __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __
           float dxv = m.x - c.campos[0], dyv = m.y - c.campos[1], dzv = m.z - c.campos[2];
           float inv = rsqrtf(dxv * dxv + dyv * dyv + dzv * dzv);
           float rgb[3];
+          bool colour_finite;
           if (staged) {
             if (!sh_ready) sh_ready = mbar_wait_bounded(&s_bar, 0u, nullptr);
-            sh_colour_smem<DEG>(s_sh + (size_t)threadIdx.x * K * 3, dxv * inv, dyv * inv,
-                                dzv * inv, rgb);
+            colour_finite = sh_colour_smem<DEG>(s_sh + (size_t)threadIdx.x * K * 3, dxv * inv,
+                                                dyv * inv, dzv * inv, rgb);
           } else {
-            sh_colour_global<DEG>(shi, dxv * inv, dyv * inv, dzv * inv, rgb);
+            colour_finite = sh_colour_global<DEG>(shi, dxv * inv, dyv * inv, dzv * inv, rgb);
           }
           rec[R_R] = rgb[0];
           rec[R_G] = rgb[1];
           rec[R_B] = rgb[2];
+          // a non-finite SH coefficient shows in the colour
+          if (!colour_finite) {
+            ok = false;
+            nonfinite = true;
+          }
         }
       }
     }
@@ -372,7 +387,8 @@ __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __
     out[0] = make_float4(rec[0], rec[1], rec[2], rec[3]);
     out[1] = make_float4(rec[4], rec[5], rec[6], rec[7]);
     out[2] = make_float4(rec[8], rec[9], rec[10], rec[11]);
-    bins[r] = make_float4(key, __uint_as_float((uint32_t)x0 | ((uint32_t)x1 << 16)),
+    bins[r] = make_float4(nonfinite ? __uint_as_float(kNonfiniteKeyBits) : key,
+                          __uint_as_float((uint32_t)x0 | ((uint32_t)x1 << 16)),
                           __uint_as_float((uint32_t)y0 | ((uint32_t)y1 << 16)), 0.f);
     radii[r] = radius;
   }

@@ -22,8 +22,9 @@
  *  - Argument errors are detected on the host before anything is enqueued and
  *    returned at once (GS_ERR_INVALID_ARG, GS_ERR_OVERFLOW). A failed launch
  *    returns GS_ERR_CUDA. Conditions only the device can see (pair capacity
- *    exceeded, a bounded wait that gave up) are OR-ed into the status word at
- *    the start of the workspace and read back by gs_get_status.
+ *    exceeded, a bounded wait that gave up, a Gaussian culled for non-finite
+ *    values) are OR-ed into the status word at the start of the workspace and
+ *    read back by gs_get_status.
  *  - Pixel (x, y) has its centre at (x + 0.5, y + 0.5); tiles are 16 x 16
  *    pixels; tile index within a view is ty * tiles_x + tx, and the global
  *    tile index of view v is v * tiles_per_view + tile.
@@ -52,7 +53,7 @@ typedef enum gs_status {
   GS_ERR_CAPACITY = 2,        /* more Gaussian x tile pairs than pair_capacity */
   GS_ERR_OVERFLOW = 3,        /* a size exceeds a 32-bit field it must fit */
   GS_ERR_DEVICE_TIMEOUT = 4,  /* a bounded device-side wait gave up */
-  GS_ERR_NONFINITE = 5,       /* reserved: non-finite input detected */
+  GS_ERR_NONFINITE = 5,       /* a Gaussian with a non-finite parameter or colour was culled */
   GS_ERR_CUDA = 6             /* a CUDA runtime call or launch failed */
 } gs_status;
 
@@ -185,7 +186,11 @@ size_t gs_workspace_size(int64_t n, int32_t n_views, const gs_camera* cams,
  * covariance is not positive definite, or the rectangle is empty.
  * Geometry (camera-space mean, covariance, radius, rectangle, depth key) is
  * evaluated in double precision and rounded to float at the end; colour in
- * float. Writes out->records and out->radii for all n_views * n records. */
+ * float. A Gaussian with a non-finite mean, log-scale, quaternion, logit or
+ * colour (a non-finite SH coefficient), or a zero quaternion, is culled in
+ * every view and its depth key marked; gs_bin_sort on those records raises
+ * GS_ERR_NONFINITE in its status word (the rest of the frame is unaffected).
+ * Writes out->records and out->radii for all n_views * n records. */
 gs_status gs_project(const gs_params* params, const gs_camera* cams, int32_t n_views,
                      gs_projected* out, void* stream);
 
@@ -409,7 +414,9 @@ gs_status gs_adam_step_sh_quant(const gs_sh_quant* q, const float* grad_sh, uint
                                 void* stream);
 
 /* Synchronise `stream`, return the status word accumulated in workspace `ws`
- * by device-side checks since the last call, and clear it. */
+ * by device-side checks since the last call, and clear it. Several conditions
+ * report the most severe: GS_ERR_DEVICE_TIMEOUT, then GS_ERR_OVERFLOW (an
+ * index out of range was clipped), GS_ERR_CAPACITY, GS_ERR_NONFINITE. */
 gs_status gs_get_status(void* ws, void* stream);
 
 #ifdef __cplusplus

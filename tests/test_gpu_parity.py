@@ -471,3 +471,34 @@ def test_densify_and_prune_capacity_and_empty():
                              api.grads(*v_out), cap, n_out, None, ws)
     torch.cuda.synchronize()
     assert int(n_out.item()) == 0
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_nonfinite_gaussians_are_culled_and_reported(mode):
+    """A NaN mean, an infinite log-scale, a NaN SH coefficient and a zero
+    quaternion: those Gaussians get radius 0 in every view, gs_bin_sort raises
+    GS_ERR_NONFINITE, and the frame is bit for bit the frame of the scene
+    without them."""
+    sc = S.make_scene("fwd_100k_800", n=3000, width=200, height=152)
+    bad = [3, 70, 1500, 2999]
+    sc.means[3, 0] = np.nan
+    sc.log_scales[70, 1] = np.inf
+    sc.sh[1500, 2, 1] = np.nan
+    sc.quats[2999] = 0.0
+    sp = Splatter(sc, sort_mode=mode)
+    sp.ensure_capacity()
+    sp.forward()
+    torch.cuda.synchronize()
+    assert sp.status() == api.GS_ERR_NONFINITE
+    assert np.all(sp.radii.cpu().numpy()[:, bad] == 0)
+    img = sp.image.cpu().numpy()
+    keep = np.setdiff1d(np.arange(sc.n), bad)
+    sc2 = S.make_scene("fwd_100k_800", n=3000, width=200, height=152)
+    for k in ("means", "log_scales", "quats", "opacity_logit", "sh"):
+        setattr(sc2, k, np.ascontiguousarray(getattr(sc2, k)[keep]))
+    sp2 = Splatter(sc2, sort_mode=mode)
+    sp2.ensure_capacity()
+    sp2.forward()
+    torch.cuda.synchronize()
+    assert sp2.status() == api.GS_OK
+    assert np.array_equal(img, sp2.image.cpu().numpy())
