@@ -10,9 +10,10 @@ and its pixel throughput (Mpix/s = rendered pixels / step time).
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 N > 1 runs one process per GPU under torch.distributed (NCCL): each rank
-renders its own view of the same Gaussians (views on an orbit of radius 8),
-the parameter gradients are summed across ranks with one all-reduce, and every
-rank applies the same Adam step (weak scaling: one view per GPU).
+renders its own view of the same Gaussians (views on an orbit of radius 8);
+the flat gradient buffer is reduce-scattered, each rank runs Adam on its
+1/N slice of the parameters, and an all-gather hands every rank the updated
+parameters (weak scaling: one view per GPU).
 
 Rank 0 prints one JSON line. ``--impl reference`` times the float64 CPU
 oracle on the host cores on a bounded sample of the same workload instead.
@@ -494,6 +495,8 @@ def run_ours(args):
         scene.cameras = [gdist.orbit_view(scene, rank, world)]
     c = scene.cameras[0]
     sp = Splatter(scene, sort_mode=mode)
+    if world > 1:
+        sp.shard_optimizer(rank, world)
     need = sp.ensure_capacity()
     dL_host = S.make_upstream_grad(1, c.height, c.width, seed=1)
     dL = torch.as_tensor(dL_host).cuda()
@@ -515,12 +518,10 @@ def run_ours(args):
         mark(4)
         sp.project_bwd()
         mark(5)
-        gdist.allreduce_grads(sp.grad_flat)
-        mark(6)
         sp.densify_stats()
+        mark(6)
+        sp.adam_step()  # with N > 1: reduce-scatter, Adam on the slice, all-gather
         mark(7)
-        sp.adam_step()
-        mark(8)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -528,8 +529,10 @@ def run_ours(args):
     assert sp.status() == api.GS_OK, "device status after warm-up"
 
     names = ["gs_project", "gs_bin_sort", "gs_rasterize_fwd", "gs_rasterize_bwd",
-             "gs_project_bwd", "all_reduce", "gs_densify_stats", "gs_adam_step"]
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(args.steps)]
+             "gs_project_bwd", "gs_densify_stats",
+             "gs_adam_step" if world == 1 else "reduce_scatter+gs_adam_step+all_gather"]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+          for _ in range(args.steps)]
     clocks = ClockSampler(local)
     if world > 1:
         dist.barrier()
@@ -563,15 +566,14 @@ def run_ours(args):
         h_in = torch.from_numpy(dL_host).pin_memory()
         h_out = torch.empty(sp.image.shape, dtype=torch.float32).pin_memory()
         sp.stream = torch.cuda.Stream()
-        hook = (lambda: gdist.allreduce_grads(sp.grad_flat)) if world > 1 else None
-        sp.train_from_host([h_in] * 3, [h_out] * 3, grad_hook=hook)  # warm-up
+        sp.train_from_host([h_in] * 3, [h_out] * 3)  # warm-up
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         e0.record(sp.stream)
-        sp.train_from_host([h_in] * args.steps, [h_out] * args.steps, grad_hook=hook)
+        sp.train_from_host([h_in] * args.steps, [h_out] * args.steps)
         e1.record(sp.stream)
         torch.cuda.synchronize()
         sp.stream = None
@@ -602,6 +604,8 @@ def run_ours(args):
         exps = nexp_mean * pixels
     pk = peaks()
     work = algorithmic_work(sp, n_pairs, args.sort_mode, exps or 0.0)
+    if world > 1:
+        work["gs_adam_step"]["bytes"] /= world  # each rank updates its slice only
     kernels = {}
     for nm in names:
         if nm not in work:
@@ -645,7 +649,8 @@ def run_ours(args):
                    "sort_path": sort_plan(sp, args.sort_mode)["path"],
                    "l2": "working set larger than L2 (0.7 GB of parameters and Adam state "
                          "rewritten every step)",
-                   "parallelism": "dp%d (one view per GPU, gradient all-reduce)" % world
+                   "parallelism": "dp%d (one view per GPU; gradient reduce-scatter, Adam on "
+                                  "1/%d of the parameters, parameter all-gather)" % (world, world)
                    if world > 1 else "single GPU"},
         "roofline": roof,
         "step_roofline": {"bound_ms": bound_s * 1000.0, "frac": bound_s * 1000.0 / ms},

@@ -1,10 +1,13 @@
 """Multi-GPU plumbing of the training step: one process per GPU, sharded by view.
 
-Every rank holds the same Gaussians and renders its own view; the parameter
-gradients of the step are summed across ranks (one all-reduce over the flat
-gradient buffer, NCCL over NVLink on GPUs), after which every rank applies the
-identical Adam step. Timings are reduced with MAX so a step costs what the
-slowest rank took. Nothing here computes any part of the method.
+Every rank holds the same Gaussians and renders its own view. The parameter
+gradients of the step are summed across ranks with one reduce-scatter over the
+flat gradient buffer (NCCL over NVLink on GPUs): each rank receives the summed
+gradient of its own contiguous slice of the flat parameter buffer, runs Adam
+on that slice only (its optimiser work and moments are 1/world of the whole),
+and one all-gather hands every rank the updated parameters. Timings are
+reduced with MAX so a step costs what the slowest rank took. Nothing here
+computes any part of the method.
 """
 
 from __future__ import annotations
@@ -24,6 +27,40 @@ def orbit_view(scene, rank: int, world: int, radius: float = 8.0):
     return S.Camera(viewmat=S.look_at(centre).astype(np.float32), fx=c0.fx, fy=c0.fy,
                     cx=c0.cx, cy=c0.cy, width=c0.width, height=c0.height,
                     campos=np.asarray(centre, np.float32))
+
+
+def flat_layout(sizes, pad: int):
+    """Offsets of parameter groups [(name, numel), ...] laid end to end in one
+    flat float buffer, each at a 16-byte aligned offset, and the buffer's
+    length rounded up to a multiple of `pad` floats (at least `pad`)."""
+    offsets, total = {}, 0
+    for k, numel in sizes:
+        offsets[k] = total
+        total += (int(numel) + 3) // 4 * 4
+    return offsets, max(-(-total // pad), 1) * pad
+
+
+def shard_bounds(total: int, rank: int, world: int):
+    """This rank's [lo, hi) of a flat buffer of `total` floats: `world` equal
+    contiguous chunks; `total` must be a multiple of 4 * world so that every
+    chunk starts 16-byte aligned."""
+    if world < 1 or not 0 <= rank < world or total % (4 * world):
+        raise ValueError("flat buffer of %d floats does not split in %d aligned chunks"
+                         % (total, world))
+    chunk = total // world
+    return rank * chunk, (rank + 1) * chunk
+
+
+def shard_slices(offsets: dict, sizes: dict, lo: int, hi: int):
+    """The parts of each parameter group inside [lo, hi): (name, a, b) with
+    lo <= a < b <= hi, group `name` occupying [offsets[name], offsets[name] +
+    sizes[name]) of the flat buffer, in group order."""
+    out = []
+    for k, off in offsets.items():
+        a, b = max(lo, off), min(hi, off + sizes[k])
+        if a < b:
+            out.append((k, a, b))
+    return out
 
 
 def allreduce_grads(flat, group=None) -> None:

@@ -9,6 +9,7 @@ libgs_b200.so.
 
 from __future__ import annotations
 
+import contextlib
 import math
 from typing import Optional
 
@@ -16,9 +17,15 @@ import numpy as np
 import torch
 
 from . import api
+from . import dist as gdist
 
 # Per-group Adam learning rates of the 10M-Gaussian training workload.
 DEFAULT_LR = dict(means=1.6e-4, sh=2.5e-3, opacity_logit=5e-2, log_scales=5e-3, quats=1e-3)
+
+# The flat parameter / gradient / moment buffers are padded to a multiple of
+# this many floats, so that they split into 16-byte aligned equal slices for
+# any power-of-two number of ranks up to 256.
+FLAT_PAD = 1024
 
 
 class Splatter:
@@ -30,6 +37,7 @@ class Splatter:
         self.sh_bits = sh_bits
         self.sh_rounding = int(sh_rounding)
         self.sh_seed = int(sh_seed)
+        self._shard = None
         self.scene = scene
         self.n = int(scene.n)
         self.V = int(scene.n_views)
@@ -69,33 +77,56 @@ class Splatter:
     # ------------------------------------------------------------ buffers
     def _alloc_gaussians(self, means, log_scales, quats, opacity_logit, sh, exp_avg=None,
                          exp_avg_sq=None) -> None:
-        """Adopt the given parameter tensors (and Adam moments, zero if None) and
-        (re)allocate every buffer whose size follows the Gaussian count."""
+        """Adopt the given parameter values (and Adam moments, zero if None) and
+        (re)allocate every buffer whose size follows the Gaussian count.
+
+        Parameters, gradients and both moments each live in one flat buffer,
+        every group at a 16-byte aligned offset (the same offsets in all four)
+        and the total padded to a multiple of FLAT_PAD floats, so that one
+        collective moves a whole buffer and equal 16-byte aligned slices of
+        it can be handed to ranks."""
         dev, f32 = self.device, torch.float32
-        self.means, self.log_scales, self.quats = means, log_scales, quats
-        self.opacity_logit, self.sh = opacity_logit, sh
+        src = [("means", means), ("log_scales", log_scales), ("quats", quats),
+               ("opacity_logit", opacity_logit), ("sh", sh)]
         self.n = n = int(means.shape[0])
         V = self.V
-        self.param_list = [("means", self.means), ("log_scales", self.log_scales),
-                           ("quats", self.quats), ("opacity_logit", self.opacity_logit),
-                           ("sh", self.sh)]
+        offs, total = gdist.flat_layout([(k, t.numel()) for k, t in src], FLAT_PAD)
+        self.flat_offsets = offs
+        self.flat_sizes = {k: t.numel() for k, t in src}
+        self.flat_total = total
+
+        def views(buf, names):
+            return {k: buf[offs[k]:offs[k] + t.numel()].view(t.shape)
+                    for k, t in src if k in names}
+
+        names = [k for k, _ in src]
+        self.param_flat = torch.zeros(total, dtype=f32, device=dev)
+        P = views(self.param_flat, names)
+        for k, t in src:
+            P[k].copy_(t)
+        self.means, self.log_scales, self.quats = P["means"], P["log_scales"], P["quats"]
+        self.opacity_logit, self.sh = P["opacity_logit"], P["sh"]
+        self.param_list = [(k, P[k]) for k in names]
         self.records = torch.empty((V, n, api.GS_RECORD_FLOATS), dtype=f32, device=dev)
         self.bins = torch.empty((V, n, 4), dtype=f32, device=dev)
         self.radii = torch.empty((V, n), dtype=torch.int32, device=dev)
         self.grad2d = torch.empty((V, n, api.GS_GRAD2D_FLOATS), dtype=f32, device=dev)
-        # gradients live in one flat buffer (one all-reduce across ranks), each
-        # group at a 16-byte aligned offset
-        offs, total = {}, 0
-        for k, t in self.param_list:
-            offs[k] = total
-            total += (t.numel() + 3) // 4 * 4
-        self.grad_flat = torch.zeros(max(total, 4), dtype=f32, device=dev)
-        self.grads = {k: self.grad_flat[offs[k]:offs[k] + t.numel()].view(t.shape)
-                      for k, t in self.param_list}
-        self.exp_avg = (exp_avg if exp_avg is not None
-                        else {k: torch.zeros_like(t) for k, t in self.param_list})
-        self.exp_avg_sq = (exp_avg_sq if exp_avg_sq is not None
-                           else {k: torch.zeros_like(t) for k, t in self.param_list})
+        self.grad_flat = torch.zeros(total, dtype=f32, device=dev)
+        self.grads = views(self.grad_flat, names)
+        # the moments: with quantised SH the SH moments live beside the codes,
+        # so the float32 moment buffers stop before the SH group
+        m_names = names[:-1] if self.sh_bits is not None else names
+        m_total = offs["sh"] if self.sh_bits is not None else total
+        self.m_flat = torch.zeros(max(m_total, 4), dtype=f32, device=dev)
+        self.v_flat = torch.zeros(max(m_total, 4), dtype=f32, device=dev)
+        self.exp_avg = views(self.m_flat, m_names)
+        self.exp_avg_sq = views(self.v_flat, m_names)
+        for given, mine in ((exp_avg, self.exp_avg), (exp_avg_sq, self.exp_avg_sq)):
+            if given is not None:
+                for k in m_names:
+                    mine[k].copy_(given[k])
+        if self.sh_bits is not None:
+            self.exp_avg["sh"] = self.exp_avg_sq["sh"] = None
         if self.sh_bits is not None:
             self._quantise_sh()
         self.accum_plain = torch.zeros(n, dtype=f32, device=dev)
@@ -105,6 +136,8 @@ class Splatter:
                                    self.sh, self.deg)
         self.c_grads = api.grads(*[self.grads[k] for k, _ in self.param_list])
         self.c_proj = api.projected(self.records, self.bins, self.radii)
+        if getattr(self, "_shard", None) is not None:
+            self._plan_shard()  # the slices follow the buffer size
         if getattr(self, "ws", None) is not None:
             self._alloc_pairs(self.capacity)  # the workspace follows the count too
 
@@ -123,8 +156,6 @@ class Splatter:
         self.sh_q = api.sh_quant(self.sh_codes, self.sh_bounds, n, k3, self.sh_bits)
         self.sh_m16 = torch.zeros((k3, n_pad), dtype=torch.int16, device=dev)
         self.sh_v16 = torch.zeros((k3, n_pad), dtype=torch.int16, device=dev)
-        # the float32 moments of the SH are not used in this mode
-        self.exp_avg["sh"] = self.exp_avg_sq["sh"] = None
         api.gs_sh_quantize(self.sh, self.sh_q, self.stream)
         api.gs_sh_dequantize(self.sh_q, self.sh, self.stream)
 
@@ -183,6 +214,9 @@ class Splatter:
 
     def adam_step(self, beta1=0.9, beta2=0.999, eps=1e-15):
         self.step_count += 1
+        if self._shard is not None:
+            self._sharded_adam_step(beta1, beta2, eps)
+            return
         quant = self.sh_bits is not None
         groups = [(t, self.grads[k], self.exp_avg[k], self.exp_avg_sq[k], self.lr[k])
                   for k, t in self.param_list if not (quant and k == "sh")]
@@ -191,6 +225,73 @@ class Splatter:
             api.gs_adam_step_sh_quant(self.sh_q, self.grads["sh"], self.sh_m16, self.sh_v16,
                                       self.lr["sh"], beta1, beta2, eps, self.step_count,
                                       self.sh_rounding, self.sh_seed, self.stream)
+
+    # ------------------------------------------------------------ sharded optimiser
+    def shard_optimizer(self, rank: int, world: int, group=None) -> None:
+        """Shard the Adam step over `world` ranks that each render their own
+        views of the same Gaussians (torch.distributed initialised, NCCL on
+        GPUs). adam_step then reduce-scatters the flat gradient buffer (every
+        rank gets the sum over ranks of its slice), runs Adam on this rank's
+        contiguous slice of the flat parameter buffer only, and all-gathers
+        the parameters, so every rank ends the step with the same parameters.
+        The moments outside the slice are not kept current on this rank;
+        densify_and_prune gathers them first. world == 1 needs no process
+        group and runs the same slice logic over the whole buffer."""
+        if self.sh_bits is not None:
+            raise NotImplementedError("sharded optimiser with quantised SH state")
+        self._shard = dict(rank=int(rank), world=int(world), group=group)
+        self._plan_shard()
+
+    def _plan_shard(self) -> None:
+        sh = self._shard
+        lo, hi = gdist.shard_bounds(self.flat_total, sh["rank"], sh["world"])
+        sh["lo"], sh["hi"] = lo, hi
+        sh["slices"] = gdist.shard_slices(self.flat_offsets, self.flat_sizes, lo, hi)
+        if sh["world"] > 1:
+            self._grad_shard = torch.empty(hi - lo, dtype=torch.float32, device=self.device)
+            self._param_shard = torch.empty(hi - lo, dtype=torch.float32, device=self.device)
+
+    def _torch_stream(self):
+        return (torch.cuda.stream(self.stream) if self.stream is not None
+                else contextlib.nullcontext())
+
+    def _sharded_adam_step(self, beta1, beta2, eps) -> None:
+        import torch.distributed as dist
+        sh = self._shard
+        lo, hi, world, group = sh["lo"], sh["hi"], sh["world"], sh["group"]
+        if world > 1:
+            with self._torch_stream():
+                dist.reduce_scatter_tensor(self._grad_shard, self.grad_flat, group=group)
+            gsl = self._grad_shard
+        else:
+            gsl = self.grad_flat[lo:hi]
+        groups = [(self.param_flat[a:b], gsl[a - lo:b - lo], self.m_flat[a:b], self.v_flat[a:b],
+                   self.lr[k]) for k, a, b in sh["slices"]]
+        if groups:
+            api.gs_adam_step(groups, beta1, beta2, eps, self.step_count, self.stream)
+        if world > 1:
+            with self._torch_stream():
+                self._param_shard.copy_(self.param_flat[lo:hi])
+                dist.all_gather_into_tensor(self.param_flat, self._param_shard, group=group)
+
+    def _gather_for_densify(self) -> None:
+        """Before densify_and_prune on several ranks: the summed view-space
+        statistics (every rank decides alike) and, when the optimiser is
+        sharded, every rank's slice of the moments."""
+        import torch.distributed as dist
+        if not (dist.is_available() and dist.is_initialized()):
+            return
+        group = self._shard["group"] if self._shard is not None else None
+        if dist.get_world_size(group) < 2:
+            return
+        with self._torch_stream():
+            for t in (self.accum_plain, self.accum_abs, self.denom):
+                dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+            if self._shard is not None:
+                lo, hi = self._shard["lo"], self._shard["hi"]
+                for buf in (self.m_flat, self.v_flat):
+                    part = buf[lo:hi].clone()
+                    dist.all_gather_into_tensor(buf, part, group=group)
 
     def forward(self):
         self.project()
@@ -305,6 +406,7 @@ class Splatter:
         per-Gaussian codes (0 pruned, 1 kept, 2 cloned, 3 split)."""
         if self.sh_bits is not None:
             raise NotImplementedError("densify_and_prune with quantised SH state")
+        self._gather_for_densify()
         n, dev = self.n, self.device
         if z is None:
             gen = torch.Generator(device=dev)

@@ -502,3 +502,27 @@ def test_nonfinite_gaussians_are_culled_and_reported(mode):
     torch.cuda.synchronize()
     assert sp2.status() == api.GS_OK
     assert np.array_equal(img, sp2.image.cpu().numpy())
+
+
+def test_sharded_optimizer_on_one_rank_matches_the_plain_step():
+    """shard_optimizer(0, 1) runs Adam over the slices of the flat buffers
+    (no collectives with one rank): from identical gradients it reaches
+    exactly the parameters and moments of the plain Adam call."""
+    sc = S.make_scene("fwd_100k_800", n=5000, width=256, height=192)
+    dL = torch.as_tensor(S.make_upstream_grad(1, 192, 256, seed=3)).cuda()
+    a = Splatter(sc)
+    a.ensure_capacity()
+    b = Splatter(sc)
+    b.shard_optimizer(0, 1)
+    b.ensure_capacity()
+    assert torch.equal(a.param_flat, b.param_flat)
+    for _ in range(2):
+        a.forward()
+        a.rasterize_bwd(dL)
+        b.grad_flat.copy_(a.grad_flat)
+        a.adam_step()
+        b.adam_step()
+    torch.cuda.synchronize()
+    assert torch.equal(a.param_flat, b.param_flat)
+    assert torch.equal(a.m_flat, b.m_flat) and torch.equal(a.v_flat, b.v_flat)
+    assert not torch.equal(a.param_flat, Splatter(sc).param_flat)   # the steps moved them

@@ -1,8 +1,11 @@
-"""Host-side logic of the multi-GPU step on CPU: two `gloo` ranks.
+"""Host-side logic of the multi-GPU step on CPU: `gloo` ranks.
 
-Each rank gets a distinct orbit view, the flat gradient buffer is summed across
-ranks (so every rank applies the same Adam update), and step times are reduced
-with MAX. No GPU is involved."""
+Each rank gets a distinct orbit view, step times are reduced with MAX, a flat
+buffer summed across ranks is the same everywhere, and the sharded optimiser
+(reduce-scatter of the flat gradient, Adam on each rank's slice, all-gather of
+the parameters) ends with every rank holding the replicated Adam step. The
+Adam arithmetic here is the oracle's; the slicing and the collectives are the
+library's own helpers. No GPU is involved."""
 
 import os
 import socket
@@ -61,3 +64,74 @@ def test_two_gloo_ranks_share_summed_gradients_and_distinct_views():
     assert np.linalg.norm(np.subtract(res[0]["campos"], res[1]["campos"])) > 1.0
     for r in range(world):
         assert abs(np.linalg.norm(res[r]["campos"]) - 8.0) < 1e-5
+
+
+def _shard_worker(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from gaussian_splatting_differentiable_ewa_b200 import dist as gdist
+        from oracle import oracle as O
+        n = 37
+        sizes = [("means", 4 * n), ("log_scales", 4 * n), ("quats", 4 * n),
+                 ("opacity_logit", n), ("sh", 48 * n)]
+        lr = dict(means=1.6e-4, log_scales=5e-3, quats=1e-3, opacity_logit=5e-2, sh=2.5e-3)
+        offs, total = gdist.flat_layout(sizes, 1024)
+        p0 = torch.tensor(np.random.default_rng(7).normal(size=total), dtype=torch.float32)
+        grad = torch.tensor(np.random.default_rng(200 + rank).normal(size=total),
+                            dtype=torch.float32)
+        param, m, v = p0.clone(), torch.zeros(total), torch.zeros(total)
+        lo, hi = gdist.shard_bounds(total, rank, world)
+        shard = torch.empty(hi - lo)
+        dist.reduce_scatter_tensor(shard, grad)          # the summed gradient of the slice
+        for k, a, b in gdist.shard_slices(offs, dict(sizes), lo, hi):
+            pn, mn, vn = O.adam(param[a:b].numpy(), shard[a - lo:b - lo].numpy(),
+                                m[a:b].numpy(), v[a:b].numpy(), lr[k], 1)
+            param[a:b] = torch.tensor(pn, dtype=torch.float32)
+            m[a:b] = torch.tensor(mn, dtype=torch.float32)
+        dist.all_gather_into_tensor(param, param[lo:hi].clone())
+        out[rank] = dict(param=param.numpy().tolist(), offs=offs, total=total, lo=lo, hi=hi)
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_sharded_adam_equals_the_replicated_step(world):
+    """Reduce-scatter of the flat gradient, Adam on each rank's slice only,
+    all-gather of the parameters: every rank ends with the parameters of one
+    Adam step on the summed gradient over the whole buffer (group by group,
+    padding untouched), and the slices tile the buffer."""
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_shard_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    from gaussian_splatting_differentiable_ewa_b200 import dist as gdist
+    from oracle import oracle as O
+    total, offs = res[0]["total"], res[0]["offs"]
+    assert [(res[r]["lo"], res[r]["hi"]) for r in range(world)] == \
+        [(r * total // world, (r + 1) * total // world) for r in range(world)]
+    assert all(res[r]["lo"] % 4 == 0 for r in range(world))
+    n = 37
+    sizes = dict(means=4 * n, log_scales=4 * n, quats=4 * n, opacity_logit=n, sh=48 * n)
+    lr = dict(means=1.6e-4, log_scales=5e-3, quats=1e-3, opacity_logit=5e-2, sh=2.5e-3)
+    p0 = np.random.default_rng(7).normal(size=total).astype(np.float32)
+    g = sum(np.random.default_rng(200 + r).normal(size=total).astype(np.float32)
+            for r in range(world))
+    want = p0.copy()
+    for k, off in offs.items():
+        sl = slice(off, off + sizes[k])
+        pn, _, _ = O.adam(p0[sl], g[sl], np.zeros(sizes[k]), np.zeros(sizes[k]), lr[k], 1)
+        want[sl] = pn.astype(np.float32)
+    for r in range(world):
+        got = np.asarray(res[r]["param"], np.float32)
+        np.testing.assert_allclose(got, want, rtol=0, atol=2e-7)
+    assert np.array_equal(np.asarray(res[0]["param"]), np.asarray(res[world - 1]["param"]))
+    # padding between groups and after the last one keeps its starting value
+    ends = sorted((off + sizes[k], off + (sizes[k] + 3) // 4 * 4) for k, off in offs.items())
+    for a, b in ends + [(max(o + (sizes[k] + 3) // 4 * 4 for k, o in offs.items()), total)]:
+        assert np.array_equal(np.asarray(res[0]["param"], np.float32)[a:b], p0[a:b])
+    assert gdist.shard_slices(offs, sizes, 0, total) == [
+        (k, o, o + sizes[k]) for k, o in offs.items()]
