@@ -64,7 +64,8 @@ def shard_slices(offsets: dict, sizes: dict, lo: int, hi: int):
 
 
 def allreduce_grads(flat, group=None) -> None:
-    """Sum the flat gradient buffer over all ranks, in place."""
+    """Sum a buffer over all ranks, in place (the densify statistics before
+    densify_and_prune; a whole gradient buffer for a replicated optimiser)."""
     import torch.distributed as dist
     if dist.is_initialized() and dist.get_world_size(group) > 1:
         dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)

@@ -1,9 +1,11 @@
 """Buffers and call sequence of one training step, on top of the C ABI.
 
-``Splatter`` owns the device buffers (allocated once with torch, the only
-thing torch is used for besides streams) and runs the six calls in order:
-gs_project -> gs_bin_sort -> gs_rasterize_fwd -> gs_rasterize_bwd ->
-gs_densify_stats -> gs_adam_step. Every step of the computation runs in
+``Splatter`` owns the device buffers (allocated with torch, which is used for
+nothing else besides streams and the collectives of the multi-GPU step) and
+runs the calls in order: gs_project -> gs_bin_sort -> gs_rasterize_fwd ->
+[gs_l1_dssim against a target image] -> gs_rasterize_bwd -> gs_densify_stats
+-> gs_adam_step (or, with quantised SH, gs_adam_step_sh_quant for the SH), and
+gs_densify_and_prune when asked. Every step of the computation runs in
 libgs_b200.so.
 """
 
@@ -286,7 +288,7 @@ class Splatter:
             return
         with self._torch_stream():
             for t in (self.accum_plain, self.accum_abs, self.denom):
-                dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+                gdist.allreduce_grads(t, group)
             if self._shard is not None:
                 lo, hi = self._shard["lo"], self._shard["hi"]
                 for buf in (self.m_flat, self.v_flat):
@@ -345,7 +347,8 @@ class Splatter:
         synchronises. ``self.stream`` must be a stream other than the legacy
         default stream (which would serialise the two). ``grad_hook()``, if
         given, runs on the compute stream between the backward and the
-        statistics (e.g. the gradient all-reduce of a multi-GPU step)."""
+        statistics (e.g. a gradient clip; the multi-GPU exchange is part of
+        adam_step once shard_optimizer was called)."""
         comp = self.stream
         if comp is None:
             raise ValueError("train_from_host needs Splatter(stream=...) on a created stream")
