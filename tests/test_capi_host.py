@@ -101,3 +101,23 @@ def test_loss_and_quant_arguments_are_rejected_before_any_cuda_call():
                                    None) == api.GS_ERR_INVALID_ARG   # beta1 1
     q = api.GsShQuant(None, None, 0, 12, 8)
     assert L.gs_sh_quantize(None, ctypes.byref(q), None) == api.GS_OK
+
+
+def test_densify_thresholds_convert_to_the_raw_parameter_units():
+    """The cut-offs travel as a log-scale and a logit: comparing raw
+    parameters against them decides as comparing activated values against the
+    given thresholds (exp and the logistic function are increasing)."""
+    dp = api.densify_params(0.0002, 0.05, 0.005, 1.0, 1.6)
+    assert dp.grad_threshold == np.float32(0.0002)
+    assert dp.log_scale_split == np.float32(np.log(0.05))
+    assert dp.logit_min_opacity == np.float32(np.log(0.005 / 0.995))
+    assert dp.log_max_scale == 0.0 and dp.log_split_shrink == np.float32(np.log(1.6))
+    rng = np.random.default_rng(3)
+    ls = rng.uniform(-8, 2, 2000).astype(np.float32)
+    lg = rng.uniform(-9, 9, 2000).astype(np.float32)
+    s, o = np.exp(ls.astype(np.float64)), 1 / (1 + np.exp(-lg.astype(np.float64)))
+    far = (np.abs(s - 0.05) > 1e-5) & (np.abs(o - 0.005) > 1e-6)
+    assert np.array_equal((ls > np.float32(dp.log_scale_split))[far], (s > 0.05)[far])
+    assert np.array_equal((lg < np.float32(dp.logit_min_opacity))[far], (o < 0.005)[far])
+    assert 0 < api.gs_densify_workspace_size(1000) < api.gs_densify_workspace_size(10 ** 6)
+    assert api.gs_densify_workspace_size(-1) == 0
