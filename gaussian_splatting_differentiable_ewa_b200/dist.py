@@ -71,6 +71,22 @@ def allreduce_grads(flat, group=None) -> None:
         dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
 
 
+def gather_for_densify(stats, flats, bounds=None, group=None) -> None:
+    """Before densify_and_prune on several ranks: sum each statistics tensor
+    in `stats` over the ranks (every rank then decides alike) and, when the
+    optimiser is sharded (`bounds` = this rank's [lo, hi)), all-gather every
+    rank's slice of each flat moment buffer in `flats`, in place."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) < 2:
+        return
+    for t in stats:
+        dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+    if bounds is not None:
+        lo, hi = bounds
+        for buf in flats:
+            dist.all_gather_into_tensor(buf, buf[lo:hi].clone(), group=group)
+
+
 def max_over_ranks(value: float, device=None) -> float:
     """Largest `value` over all ranks (a step takes as long as its slowest rank)."""
     import torch

@@ -278,22 +278,14 @@ class Splatter:
 
     def _gather_for_densify(self) -> None:
         """Before densify_and_prune on several ranks: the summed view-space
-        statistics (every rank decides alike) and, when the optimiser is
-        sharded, every rank's slice of the moments."""
-        import torch.distributed as dist
-        if not (dist.is_available() and dist.is_initialized()):
-            return
-        group = self._shard["group"] if self._shard is not None else None
-        if dist.get_world_size(group) < 2:
-            return
+        statistics and, when the optimiser is sharded, every rank's slice of
+        the moments (gdist.gather_for_densify)."""
+        sh = self._shard
         with self._torch_stream():
-            for t in (self.accum_plain, self.accum_abs, self.denom):
-                gdist.allreduce_grads(t, group)
-            if self._shard is not None:
-                lo, hi = self._shard["lo"], self._shard["hi"]
-                for buf in (self.m_flat, self.v_flat):
-                    part = buf[lo:hi].clone()
-                    dist.all_gather_into_tensor(buf, part, group=group)
+            gdist.gather_for_densify(
+                (self.accum_plain, self.accum_abs, self.denom), (self.m_flat, self.v_flat),
+                None if sh is None else (sh["lo"], sh["hi"]),
+                None if sh is None else sh["group"])
 
     def forward(self):
         self.project()

@@ -135,3 +135,37 @@ def test_sharded_adam_equals_the_replicated_step(world):
         assert np.array_equal(np.asarray(res[0]["param"], np.float32)[a:b], p0[a:b])
     assert gdist.shard_slices(offs, sizes, 0, total) == [
         (k, o, o + sizes[k]) for k, o in offs.items()]
+
+
+def _densify_worker(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from gaussian_splatting_differentiable_ewa_b200 import dist as gdist
+        total = 1024
+        lo, hi = gdist.shard_bounds(total, rank, world)
+        accum = torch.tensor(np.arange(10, dtype=np.float32) * (rank + 1))
+        denom = torch.tensor(np.full(10, rank + 1, dtype=np.int32))
+        # each rank's moments are current on its own slice only
+        m = torch.full((total,), -1.0)
+        m[lo:hi] = torch.arange(lo, hi, dtype=torch.float32)
+        gdist.gather_for_densify((accum, denom), (m,), (lo, hi))
+        out[rank] = dict(accum=accum.tolist(), denom=denom.tolist(), m=m.tolist())
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_densify_inputs_are_summed_and_gathered_across_ranks():
+    world = 4
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_densify_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    tri = world * (world + 1) // 2
+    for r in range(world):
+        assert res[r]["accum"] == (np.arange(10) * tri).tolist()
+        assert res[r]["denom"] == [tri] * 10
+        assert res[r]["m"] == np.arange(1024, dtype=np.float32).tolist()
