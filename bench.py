@@ -121,21 +121,17 @@ class ClockSampler:
 # ----------------------------------------------------------------- work model
 
 def sort_plan(sp, sort_mode: str) -> dict:
-    """How gs_bin_sort treats this workload (mirrors the library's choice):
-    presort passes, pair passes, emission path and tile-placement blocks."""
-    tx, ty = (sp.W + 15) // 16, (sp.H + 15) // 16
-    tiles = sp.V * tx * ty
-    tile_bits = max(int(tiles - 1).bit_length(), 0)
-    if sort_mode == "full64":
-        return dict(path="tile_id", pre=0, pair=(32 + tile_bits + 7) // 8, bpv=0, tiles=tiles)
-    pre = (32 + max(int(sp.V - 1).bit_length(), 0) + 7) // 8
-    if (tx + 1) * (ty + 1) * 4 <= 160 * 1024:
-        gsize = 768 if sp.n <= (2 << 20) else 4096
-        return dict(path="tiles", pre=pre, pair=0, bpv=-(-sp.n // gsize), tiles=tiles)
-    if tx <= 256:
-        rows = max(int(sp.V * ty - 1).bit_length(), 0)
-        return dict(path="columns", pre=pre, pair=(rows + 7) // 8, bpv=0, tiles=tiles)
-    return dict(path="tile_id", pre=pre, pair=(tile_bits + 7) // 8, bpv=0, tiles=tiles)
+    """How gs_bin_sort treats this workload, as the library plans it
+    (gs_bin_sort_plan): emission path, presort passes, pair passes and the
+    tile-placement blocks per view."""
+    from gaussian_splatting_differentiable_ewa_b200 import api
+    mode = api.GS_SORT_FULL64 if sort_mode == "full64" else api.GS_SORT_PRESORT
+    p = api.gs_bin_sort_plan(sp.n, sp.cams, sp.V, mode)
+    tiles = sp.V * ((sp.W + 15) // 16) * ((sp.H + 15) // 16)
+    path = {api.GS_PATH_TILES: "tiles", api.GS_PATH_COLUMNS: "columns",
+            api.GS_PATH_TILE_ID: "tile_id"}[p.path]
+    return dict(path=path, pre=p.presort_passes, pair=p.pair_passes, bpv=p.blocks_per_view,
+                tiles=tiles)
 
 
 def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float) -> dict:

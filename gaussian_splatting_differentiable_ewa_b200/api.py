@@ -113,6 +113,8 @@ SIGNATURES = [
     ("gs_adam_step_sh_quant", _c.c_int,
      [_c.c_void_p, _vp, _vp, _vp, _c.c_float, _c.c_float, _c.c_float, _c.c_float, _c.c_int64,
       _c.c_int32, _c.c_uint64, _vp]),
+    ("gs_bin_sort_plan", _c.c_int,
+     [_c.c_int64, _c.c_int32, _c.POINTER(GsCamera), _c.c_int32, _c.c_void_p]),
     ("gs_bin_sort_noalloc", _c.c_int,
      [_c.POINTER(GsProjected), _c.POINTER(GsCamera), _c.c_int32, _c.c_int64, _c.c_int32,
       _c.POINTER(GsBinned), _vp, _vp]),
@@ -341,6 +343,23 @@ def gs_adam_step_sh_quant(q: GsShQuant, grad_sh, exp_avg, exp_avg_sq, lr: float,
                                        _ptr(exp_avg_sq), float(lr), float(beta1), float(beta2),
                                        float(eps), int(step), int(rounding), int(seed),
                                        _stream(stream)), "gs_adam_step_sh_quant")
+
+
+GS_PATH_TILE_ID, GS_PATH_COLUMNS, GS_PATH_TILES = 0, 1, 2
+
+
+class GsSortPlan(_c.Structure):
+    _fields_ = [("path", _c.c_int32), ("presort_passes", _c.c_int32),
+                ("pair_passes", _c.c_int32), ("gaussians_per_block", _c.c_int32),
+                ("blocks_per_view", _c.c_int64)]
+
+
+def gs_bin_sort_plan(n: int, cams_arr, n_views: int, sort_mode: int) -> GsSortPlan:
+    """How gs_bin_sort orders the pairs of this request (host only)."""
+    plan = GsSortPlan()
+    _check(lib().gs_bin_sort_plan(int(n), int(n_views), cams_arr, int(sort_mode),
+                                  _c.addressof(plan)), "gs_bin_sort_plan")
+    return plan
 
 
 def gs_bin_sort_noalloc(proj: GsProjected, cams_arr, n_views: int, n: int, sort_mode: int,

@@ -541,6 +541,18 @@ gs_status gs_adam_step_sh_quant(const gs_sh_quant* q, const float* grad_sh, uint
       q->bits, lr, beta1, beta2, eps, step, rounding, seed, static_cast<cudaStream_t>(stream)));
 }
 
+gs_status gs_bin_sort_plan(int64_t n, int32_t n_views, const gs_camera* cams,
+                           int32_t sort_mode, gs_sort_plan* plan) {
+  Layout L;
+  if (!plan || !make_layout(n, n_views, cams, 0, sort_mode, L)) return GS_ERR_INVALID_ARG;
+  plan->path = L.tile_emit ? GS_PATH_TILES : (L.column_emit ? GS_PATH_COLUMNS : GS_PATH_TILE_ID);
+  plan->presort_passes = sort_mode == GS_SORT_PRESORT ? L.presort.passes : 0;
+  plan->pair_passes = L.tile_emit ? 0 : L.pairs.passes;
+  plan->gaussians_per_block = L.tile_emit ? L.gsize : 0;
+  plan->blocks_per_view = L.tile_emit ? L.tile_bpv : 0;
+  return GS_OK;
+}
+
 gs_status gs_get_status(void* ws, void* stream) {
   if (!ws) return GS_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -175,6 +175,29 @@ const char* gs_status_string(gs_status status);
 size_t gs_workspace_size(int64_t n, int32_t n_views, const gs_camera* cams,
                          int64_t pair_capacity, int32_t sort_mode);
 
+/* How gs_bin_sort will order the pairs of a request (host only, no CUDA call):
+ *   path             GS_PATH_TILE_ID (64-bit (tile, depth) keys in full-64
+ *                    mode, or presorted pairs sorted by tile id),
+ *                    GS_PATH_COLUMNS (presorted pairs emitted by tile column,
+ *                    then sorted by row) or GS_PATH_TILES (presorted pairs
+ *                    placed straight at their positions, no pair sort);
+ *   presort_passes   radix passes over the per-Gaussian depth keys (0 in
+ *                    full-64 mode);
+ *   pair_passes      radix passes over the pair keys (0 on GS_PATH_TILES);
+ *   gaussians_per_block, blocks_per_view  the Gaussian blocks of
+ *                    GS_PATH_TILES (0 otherwise).
+ * Returns GS_ERR_INVALID_ARG for a request gs_workspace_size rejects. */
+enum { GS_PATH_TILE_ID = 0, GS_PATH_COLUMNS = 1, GS_PATH_TILES = 2 };
+typedef struct gs_sort_plan {
+  int32_t path;
+  int32_t presort_passes;
+  int32_t pair_passes;
+  int32_t gaussians_per_block;
+  int64_t blocks_per_view;
+} gs_sort_plan;
+gs_status gs_bin_sort_plan(int64_t n, int32_t n_views, const gs_camera* cams,
+                           int32_t sort_mode, gs_sort_plan* plan);
+
 /* EWA projection (pwwt.cn sec. 3.2 `project_gaussian`: world -> camera ->
  * pixel with division by depth, covariance through the Jacobian of that map;
  * lshu.cn sec. 3.2). Per view and Gaussian: R from the normalised quaternion,

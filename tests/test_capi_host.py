@@ -121,3 +121,40 @@ def test_densify_thresholds_convert_to_the_raw_parameter_units():
     assert np.array_equal((lg < np.float32(dp.logit_min_opacity))[far], (o < 0.005)[far])
     assert 0 < api.gs_densify_workspace_size(1000) < api.gs_densify_workspace_size(10 ** 6)
     assert api.gs_densify_workspace_size(-1) == 0
+
+
+def test_sort_plan_follows_the_grid_and_mode():
+    """gs_bin_sort_plan (host only) names the emission path the workspace is
+    laid out for: tile placement while the (tiles + 1)^2 difference array
+    fits, emission by column up to 256 columns, by tile id beyond; radix pass
+    counts of 8-bit digits."""
+    def plan(W, H, n, views, mode):
+        cam = S.make_scene("fwd_1k_128").cameras[0]
+        cam.width, cam.height, cam.cx, cam.cy = W, H, W / 2, H / 2
+        return api.gs_bin_sort_plan(n, api.cameras([cam] * views), views, mode)
+    p = plan(1920, 1080, 1_000_000, 1, api.GS_SORT_PRESORT)
+    assert (p.path, p.presort_passes, p.pair_passes) == (api.GS_PATH_TILES, 4, 0)
+    assert (p.gaussians_per_block, p.blocks_per_view) == (768, 1303)
+    p = plan(1920, 1080, 3_000_000, 1, api.GS_SORT_PRESORT)       # larger blocks past 2M
+    assert (p.gaussians_per_block, p.blocks_per_view) == (4096, 733)
+    p = plan(4096, 2576, 1000, 1, api.GS_SORT_PRESORT)            # 256 x 161 tiles
+    assert (p.path, p.pair_passes) == (api.GS_PATH_COLUMNS, 1)
+    p = plan(8192, 1296, 1000, 1, api.GS_SORT_PRESORT)            # 512 x 81 tiles
+    assert (p.path, p.pair_passes) == (api.GS_PATH_TILE_ID, 2)
+    p = plan(1920, 1080, 1000, 8, api.GS_SORT_PRESORT)            # 3 view bits in the key
+    assert p.presort_passes == 5
+    p = plan(1920, 1080, 1000, 1, api.GS_SORT_FULL64)             # 13 tile bits + 32
+    assert (p.path, p.presort_passes, p.pair_passes) == (api.GS_PATH_TILE_ID, 0, 6)
+    with pytest.raises(api.GsError):
+        plan(1920, 1080, -1, 1, api.GS_SORT_PRESORT)
+
+
+def test_bench_work_model_uses_the_library_plan():
+    import types
+    import bench
+    cams = api.cameras(S.make_scene("train_1m_1080p", n=10).cameras)
+    sp = types.SimpleNamespace(n=1_000_000, V=1, W=1920, H=1080, cams=cams)
+    plan = bench.sort_plan(sp, "presort")
+    assert plan == dict(path="tiles", pre=4, pair=0, bpv=1303, tiles=8160)
+    assert bench.launches_per_step(sp, "presort") == 23
+    assert bench.sort_plan(sp, "full64")["pair"] == 6
