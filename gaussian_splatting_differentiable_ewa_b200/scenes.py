@@ -21,7 +21,7 @@ Any workload can be drawn at a smaller Gaussian count (``n=``) or image size
 (``width=``/``height=``, focal length scaled with the width) with the same
 distributions; parity tests use that to keep the oracle fast.
 
-Readings of the workload text (each is stated in the design doc as well):
+Readings of the workload text:
 
 * ``N(m, s)`` is read as mean m and variance s (the text writes the cluster as
   ``N(0, 0.5^2 I)``), so the higher-order SH draws have std sqrt(0.05) and the
