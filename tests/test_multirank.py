@@ -169,3 +169,79 @@ def test_densify_inputs_are_summed_and_gathered_across_ranks():
         assert res[r]["accum"] == (np.arange(10) * tri).tolist()
         assert res[r]["denom"] == [tri] * 10
         assert res[r]["m"] == np.arange(1024, dtype=np.float32).tolist()
+
+
+def _splatter_worker(rank, world, port, out):
+    """The Splatter's own sharded optimiser and densify gathering on CPU
+    tensors: only the Adam arithmetic (a GPU kernel) is replaced, by the
+    oracle's, so the slicing, collectives and buffer handling are the
+    product code."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from gaussian_splatting_differentiable_ewa_b200 import api
+        from gaussian_splatting_differentiable_ewa_b200 import pipeline
+        from gaussian_splatting_differentiable_ewa_b200 import scenes as S
+        from oracle import oracle as O
+
+        def cpu_adam(groups, beta1, beta2, eps, step, stream=None):
+            for p, g, m, v, lr in groups:
+                pn, mn, vn = O.adam(p.numpy(), g.numpy(), m.numpy(), v.numpy(), lr, step,
+                                    beta1, beta2, eps)
+                p.copy_(torch.from_numpy(pn.astype(np.float32)))
+                m.copy_(torch.from_numpy(mn.astype(np.float32)))
+                v.copy_(torch.from_numpy(vn.astype(np.float32)))
+
+        api.gs_adam_step = cpu_adam
+        sp = pipeline.Splatter(S.make_scene("fwd_1k_128", n=300), device="cpu")
+        sp.shard_optimizer(rank, world)
+        rng = np.random.default_rng(50 + rank)
+        for _ in range(2):
+            sp.grad_flat.copy_(torch.from_numpy(
+                rng.normal(size=sp.flat_total).astype(np.float32)))
+            sp.adam_step()
+        sp.accum_abs.fill_(float(rank + 1))
+        sp.denom.fill_(rank + 1)
+        sp._gather_for_densify()
+        out[rank] = dict(param=sp.param_flat.numpy().tolist(), m=sp.m_flat.numpy().tolist(),
+                         accum=sp.accum_abs.numpy().tolist(), denom=sp.denom.numpy().tolist(),
+                         offs=sp.flat_offsets, sizes=sp.flat_sizes, total=sp.flat_total,
+                         lr=sp.lr)
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_splatter_sharded_optimizer_on_gloo_ranks():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_splatter_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    from gaussian_splatting_differentiable_ewa_b200 import scenes as S
+    from oracle import oracle as O
+    r0 = res[0]
+    total, offs, sizes, lr = r0["total"], r0["offs"], r0["sizes"], r0["lr"]
+    sc = S.make_scene("fwd_1k_128", n=300)
+    start = {"means": sc.means, "log_scales": sc.log_scales, "quats": sc.quats,
+             "opacity_logit": sc.opacity_logit, "sh": sc.sh}
+    p = np.zeros(total, np.float32)
+    for k, off in offs.items():
+        p[off:off + sizes[k]] = np.asarray(start[k], np.float32).reshape(-1)
+    m = np.zeros(total, np.float32)
+    v = np.zeros(total, np.float32)
+    rngs = [np.random.default_rng(50 + r) for r in range(world)]
+    for step in (1, 2):
+        g = sum(rg.normal(size=total).astype(np.float32) for rg in rngs)
+        for k, off in offs.items():
+            sl = slice(off, off + sizes[k])
+            pn, mn, vn = O.adam(p[sl], g[sl], m[sl], v[sl], lr[k], step, 0.9, 0.999, 1e-15)
+            p[sl], m[sl], v[sl] = pn.astype(np.float32), mn.astype(np.float32), vn.astype(np.float32)
+    for r in range(world):
+        np.testing.assert_allclose(np.asarray(res[r]["param"], np.float32), p, rtol=0, atol=1e-6)
+        # after the densify gathering every rank holds every slice of the moments
+        np.testing.assert_allclose(np.asarray(res[r]["m"], np.float32), m, rtol=0, atol=1e-6)
+        assert res[r]["accum"] == [3.0] * 300 and res[r]["denom"] == [3] * 300
+    assert res[0]["param"] == res[1]["param"]
