@@ -208,8 +208,7 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
       cudaMemsetAsync(out->ranges, 0, (size_t)tiles * 2 * sizeof(int64_t), st) != cudaSuccess)
     return GS_ERR_CUDA;
 
-  BinSortArgs a;
-  std::memset(&a, 0, sizeof(a));
+  BinSortArgs a{};
   a.bins = proj->bins;
   a.n = (int)n;
   a.n_views = n_views;

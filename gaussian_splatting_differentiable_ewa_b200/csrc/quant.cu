@@ -105,27 +105,29 @@ __device__ __forceinline__ int lane_pos(int e) {
 template <int K3>
 __device__ __forceinline__ void stage_transposed(const float* __restrict__ src, int cnt,
                                                  float* s, bool vec_ok) {
-  if (K3 % 4 == 0 && vec_ok) {
-    constexpr int kQuads = K3 / 4;
-    const int total = cnt * kQuads;
-    const float4* src4 = reinterpret_cast<const float4*>(src);
+  if constexpr (K3 % 4 == 0) {
+    if (vec_ok) {
+      constexpr int kQuads = K3 / 4;
+      const int total = cnt * kQuads;
+      const float4* src4 = reinterpret_cast<const float4*>(src);
 #pragma unroll 4
-    for (int e = threadIdx.x; e < total; e += kQG) {
-      const int t = e / kQuads;
-      const int j = 4 * (e - t * kQuads);
-      const float4 v = __ldg(src4 + e);
-      s[j * kQPitch + t] = v.x;
-      s[(j + 1) * kQPitch + t] = v.y;
-      s[(j + 2) * kQPitch + t] = v.z;
-      s[(j + 3) * kQPitch + t] = v.w;
+      for (int e = threadIdx.x; e < total; e += kQG) {
+        const int t = e / kQuads;
+        const int j = 4 * (e - t * kQuads);
+        const float4 v = __ldg(src4 + e);
+        s[j * kQPitch + t] = v.x;
+        s[(j + 1) * kQPitch + t] = v.y;
+        s[(j + 2) * kQPitch + t] = v.z;
+        s[(j + 3) * kQPitch + t] = v.w;
+      }
+      return;
     }
-  } else {
-    const int total = cnt * K3;
+  }
+  const int total = cnt * K3;
 #pragma unroll 4
-    for (int e = threadIdx.x; e < total; e += kQG) {
-      const int t = e / K3;
-      s[(e - t * K3) * kQPitch + t] = __ldg(src + e);
-    }
+  for (int e = threadIdx.x; e < total; e += kQG) {
+    const int t = e / K3;
+    s[(e - t * K3) * kQPitch + t] = __ldg(src + e);
   }
 }
 
