@@ -812,3 +812,24 @@ def test_adam_on_quantised_state_against_plain_adam():
     assert np.all(np.abs(x - p1) <= tol)
     # the moments' padding lanes are left alone
     assert np.array_equal(m2[:, n:], m16[:, n:])
+
+
+def test_pure_l1_gradient_is_the_sign_over_n():
+    rng = np.random.default_rng(9)
+    x, y = rng.random((2, 3, 9, 11)), rng.random((2, 3, 9, 11))
+    x[0, 0, 0, 0] = y[0, 0, 0, 0]
+    _, g = O.l1_dssim_loss(x, y, lam=0.0)
+    np.testing.assert_array_equal(g, np.sign(x - y) / (3 * 9 * 11))
+
+
+def test_sixteen_bit_stochastic_rounding_lands_next_to_nearest():
+    """With 16-bit codes a stochastic code is floor(t) or floor(t) + 1, so it
+    is never more than one step from the nearest-rounded code."""
+    rng = np.random.default_rng(10)
+    x = rng.normal(0, 1, (6, 512)).astype(np.float32)
+    cn, bn = O.quantize_groups(x, 500, 16, rounding=0)
+    cs, bs = O.quantize_groups(x, 500, 16, rounding=1, seed=5, step=3)
+    assert np.array_equal(bn, bs)
+    d = np.abs(cn[:, :500].astype(np.int64) - cs[:, :500].astype(np.int64))
+    assert d.max() <= 1 and 0.2 < (d > 0).mean() < 0.8
+    assert np.all(cs[:, 500:] == 0)
