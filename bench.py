@@ -1,13 +1,22 @@
 #!/usr/bin/env python
-"""Benchmark of the differentiable EWA splatting training step on B200.
+"""Benchmark of the differentiable EWA splatting path on B200.
 
-One step = gs_project -> gs_bin_sort -> gs_rasterize_fwd -> gs_rasterize_bwd
-(screen space) -> gs_project_bwd -> gs_densify_stats -> gs_adam_step, on the
-1,000,000-Gaussian SH3 scene at 1920x1080 (fx = fy = 1200) with an upstream
-image gradient N(0, 1e-2), synthetic and seeded. The metric is the step time
-and its pixel throughput (Mpix/s = rendered pixels / step time).
+One step of the default workload (train_1m_1080p: 1,000,000 SH3 Gaussians,
+1920x1080, fx = fy = 1200, upstream image gradient N(0, 1e-2), synthetic and
+seeded) is gs_project -> gs_bin_sort -> gs_rasterize_fwd -> gs_rasterize_bwd
+(screen space) -> gs_project_bwd -> gs_densify_stats -> gs_adam_step. The
+metric is the step time and its pixel throughput (Mpix/s = rendered pixels /
+step time). ``--workload`` selects one of the five workload shapes:
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  fwd_1k_128        forward only (project, bin_sort, rasterize_fwd)
+  fwd_100k_800      forward only
+  train_1m_1080p    the full step above (default)
+  train_6m_8x1080p  8 views, forward + backward + densify statistics summed
+                    over the views, 64-bit (tile << 32 | depth) sort keys
+  train_10m_4k      the full step with the fused Adam update
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
 
 N > 1 runs one process per GPU under torch.distributed (NCCL): each rank
 renders its own view of the same Gaussians (views on an orbit of radius 8);
@@ -36,8 +45,17 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = "train_1m_1080p"
 METRIC = "fwd+bwd train-step ms & Mpix/s at 1M Gaussians 1080p; % of roofline"
+
+# workload -> what one step runs and its default sort mode
+STEPS = {
+    "fwd_1k_128": dict(kind="fwd", sort="presort"),
+    "fwd_100k_800": dict(kind="fwd", sort="presort"),
+    "train_1m_1080p": dict(kind="train", sort="presort"),
+    "train_6m_8x1080p": dict(kind="fwdbwd", sort="full64"),
+    "train_10m_4k": dict(kind="train", sort="presort"),
+}
+DEFAULT_WORKLOAD = "train_1m_1080p"
 
 
 def parse():
@@ -46,11 +64,17 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--sort-mode", default="presort", choices=["presort", "full64"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(STEPS))
+    ap.add_argument("--sort-mode", default=None, choices=["presort", "full64"],
+                    help="default: the workload's own (full64 for the 8-view workload)")
     ap.add_argument("--n", type=int, default=None, help="override the Gaussian count")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    return ap.parse_args()
+    ap.add_argument("--no-extras", action="store_true")
+    args = ap.parse_args()
+    if args.sort_mode is None:
+        args.sort_mode = STEPS[args.workload]["sort"]
+    return args
 
 
 # ----------------------------------------------------------------- helpers
@@ -135,22 +159,36 @@ def sort_plan(sp, sort_mode: str) -> dict:
 
 
 def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float) -> dict:
-    """Algorithmic bytes (and exp evaluations) per launch of each call.
+    """Algorithmic bytes (and exp evaluations) per launch of each call, from
+    the per-unit figures of the hot-path scope table (its measurement part):
 
-    Bytes count the data the definition has to move once: parameters read,
-    outputs written, 59 real floats per Gaussian (pad lanes excluded); a radix
-    pass reads and writes every key and value once; placing pairs straight at
-    their positions writes every id once, reads every packed rectangle once
-    and reads and writes the (tile, Gaussian block) count table once; the
-    blend kernels read every list entry's id and record once."""
+      project       the raw parameters read once ((11 + 3 K) floats: 236 B at
+                    SH3) + 48 B written per Gaussian and view;
+      bin_sort      full-64 keys: 24 B read per Gaussian and view, 12 B
+                    emitted per pair, passes x 24 B + 8 B of histogram per
+                    pair, 8 B per pair for the ranges; the presort paths
+                    (depth presort, pairs placed per tile) move far fewer
+                    bytes and are counted by their own model: every id written
+                    once, the per-Gaussian depth keys sorted (passes x 24 B),
+                    the packed rectangles and the (tile, Gaussian block) count
+                    table read and written once;
+      raster fwd    4 B id + 40 B record per pair + 20 B written per pixel;
+      raster bwd    the same list + 40 B of gradient atomics per pair + 12 B
+                    of dL/dpixel per pixel;
+      project bwd   parameters read and gradients written once, 36 B of
+                    screen-space gradients per Gaussian and view;
+      densify       16 B per Gaussian and view + 24 B per Gaussian;
+      adam          28 B per parameter (p, g, m, v read; p, m, v written).
+
+    Exps: the (pixel, Gaussian) evaluations with alpha >= 1/255 reached
+    before the pixel stops (counted by the oracle on a pixel sample)."""
     n, V = sp.n, sp.V
     P = V * sp.W * sp.H
-    rec = 48
-    p59 = 59 * 4
+    pbytes = (11 + 3 * sp.K) * 4
     plan = sort_plan(sp, sort_mode)
     pre, pair = plan["pre"], plan["pair"]
     if sort_mode == "full64":
-        sort_bytes = n_pairs * (12 + pair * 24 + 8) + V * n * 16
+        sort_bytes = V * n * 24 + n_pairs * (12 + pair * 24 + 8 + 8)
     elif plan["path"] == "tiles":
         table = plan["tiles"] * plan["bpv"] * 4
         sort_bytes = (n_pairs * 4 + V * n * (16 + 12 + pre * 24 + 12 + 16 + 16)
@@ -158,17 +196,17 @@ def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float) -> dict:
     else:
         sort_bytes = n_pairs * (8 + pair * 16 + 4) + V * n * (16 + pre * 24 + 12)
     return {
-        "gs_project": dict(bytes=V * n * (p59 + rec + 16 + 4), exps=0.0),
+        "gs_project": dict(bytes=n * pbytes + V * n * 48, exps=0.0),
         "gs_bin_sort": dict(bytes=sort_bytes, exps=0.0),
-        "gs_rasterize_fwd": dict(bytes=n_pairs * (4 + rec) + P * 20, exps=exps),
-        "gs_rasterize_bwd": dict(bytes=n_pairs * (4 + rec) + P * 20 + V * n * 48 * 2, exps=exps),
-        "gs_project_bwd": dict(bytes=V * n * (p59 + 48 + 4) + n * p59, exps=0.0),
-        "gs_densify_stats": dict(bytes=V * n * (12 + 4) + n * 24, exps=0.0),
-        "gs_adam_step": dict(bytes=n * 59 * 28, exps=0.0),
+        "gs_rasterize_fwd": dict(bytes=n_pairs * 44 + P * 20, exps=exps),
+        "gs_rasterize_bwd": dict(bytes=n_pairs * (44 + 40) + P * 12, exps=exps),
+        "gs_project_bwd": dict(bytes=n * 2 * pbytes + V * n * 36, exps=0.0),
+        "gs_densify_stats": dict(bytes=V * n * 16 + n * 24, exps=0.0),
+        "gs_adam_step": dict(bytes=n * (pbytes // 4) * 28, exps=0.0),
     }
 
 
-def launches_per_step(sp, sort_mode: str) -> int:
+def launches_per_step(sp, sort_mode: str, kind: str = "train") -> int:
     """Library kernels launched by one step (memsets excluded)."""
     plan = sort_plan(sp, sort_mode)
     pre, pair = plan["pre"], plan["pair"]
@@ -180,7 +218,8 @@ def launches_per_step(sp, sort_mode: str) -> int:
         sort = 1 + 3 * pre + 3 + 3 * pair + 1   # ..., count, scan, emit, row passes, ranges
     else:
         sort = 1 + 3 * pre + 1 + 3 * pair + 1
-    return 1 + sort + 1 + 1 + 1 + 1 + 1
+    # project, sort, raster fwd (+ raster bwd, project bwd, densify (+ adam))
+    return 1 + sort + 1 + {"fwd": 0, "fwdbwd": 3, "train": 4}[kind]
 
 
 # C call -> (kernel, source file) for the ncu traffic lookup
@@ -216,6 +255,18 @@ def profiled_traffic(call: str, workload: str):
     return int(m_t.group(1))
 
 
+L2_BYTES = 126 * 1000 * 1000
+
+
+def working_set_bytes(sp) -> int:
+    """Device bytes one step touches: parameters, gradients and both moments,
+    records, binning records, radii, pair ids, images and screen-space
+    gradients."""
+    n, V = sp.n, sp.V
+    return int(4 * sp.flat_total * 4 + V * n * (64 + 16 + 4 + 48) + 4 * sp.capacity
+               + V * sp.W * sp.H * (12 + 4 + 4 + 12))
+
+
 def sfu_peak_gexps(sm_mhz: float, sms: int = 148) -> float:
     # MUFU.EX2: 16 results per SM per clock (4 per SM sub-partition)
     return sms * 16 * sm_mhz * 1e6 / 1e9
@@ -223,80 +274,92 @@ def sfu_peak_gexps(sm_mhz: float, sms: int = 148) -> float:
 
 # ----------------------------------------------------------------- CPU oracle
 
-def cpu_baseline(scene, sample_pixels: int = 4096, seed: int = 5):
-    """Time the float64 oracle as it stands on host cores over a bounded
-    sample and extrapolate to one full step. Returns (dict, n_exp_mean)."""
+def _subset(scene, m: int, seed: int = 3):
+    """The scene restricted to m of its Gaussians (a seeded random subset)."""
+    import copy
+    if m >= scene.n:
+        return scene
+    idx = np.sort(np.random.default_rng(seed).choice(scene.n, m, replace=False))
+    sub = copy.copy(scene)
+    for k in ("means", "log_scales", "quats", "opacity_logit", "sh"):
+        setattr(sub, k, np.ascontiguousarray(getattr(scene, k)[idx]))
+    return sub
+
+
+def cpu_baseline(scene, kind: str, sample_pixels: int = 2048, max_gauss: int = 250_000,
+                 seed: int = 5):
+    """Time the float64 oracle as it stands on the host cores over a bounded
+    sample of one step and extrapolate to the full step:
+      * projection, projection backward and Adam on a seeded subset of at
+        most `max_gauss` Gaussians (all views), scaled by n / subset;
+      * render (and render backward) of `sample_pixels` random pixels of view
+        0 from the projection of every Gaussian into view 0 (its time is not
+        counted again), scaled by the step's pixel count.
+    Returns (dict, n_exp_mean) where n_exp_mean is the oracle's count of
+    alpha >= 1/255 evaluations per pixel on the sample."""
     from oracle import oracle as O
     from gaussian_splatting_differentiable_ewa_b200 import scenes as S
     c = scene.cameras[0]
+    n, V = scene.n, scene.n_views
     rng = np.random.default_rng(seed)
     pix = np.stack([np.zeros(sample_pixels, np.int64), rng.integers(0, c.width, sample_pixels),
                     rng.integers(0, c.height, sample_pixels)], 1).astype(np.int32)
+    sub = _subset(scene, max_gauss)
+    scale_g = n / sub.n
     t0 = time.perf_counter()
-    projs = O.project_views(scene)
+    projs_sub = O.project_views(sub)
     t1 = time.perf_counter()
-    ref = O.render(projs, scene.cameras, scene.background, pix)
+    proj0 = [O.project(scene, c)]
     t2 = time.perf_counter()
-    dL = S.make_upstream_grad(1, c.height, c.width, seed=1)
-    gC = dL[0][:, pix[:, 2], pix[:, 1]].T
-    g2 = O.render_bwd(projs, scene.cameras, scene.background, pix, gC)
+    ref = O.render(proj0, scene.cameras[:1], scene.background, pix)
     t3 = time.perf_counter()
-    # the projection backward over every Gaussian (as in a full step)
-    g2_full = g2.copy()
-    g2_full[..., :9] += 1e-3
-    O.project_bwd(scene, projs, g2_full)
-    t4 = time.perf_counter()
-    n = scene.n
-    p = np.zeros(59 * n)
-    O.adam(p, p + 1e-3, p, p, 1e-3, 1)
-    t5 = time.perf_counter()
-    P = c.width * c.height
-    scale = P / sample_pixels
-    step_s = (t1 - t0) + (t2 - t1 + t3 - t2) * scale + (t4 - t3) + (t5 - t4)
+    t_bwd = t_pb = t_adam = 0.0
+    if kind != "fwd":
+        dL = S.make_upstream_grad(1, c.height, c.width, seed=1)
+        gC = dL[0][:, pix[:, 2], pix[:, 1]].T
+        O.render_bwd(proj0, scene.cameras[:1], scene.background, pix, gC)
+        t4 = time.perf_counter()
+        g2 = np.full((V, sub.n, 10), 1e-3)
+        O.project_bwd(sub, projs_sub, g2)
+        t5 = time.perf_counter()
+        t_bwd, t_pb = t4 - t3, t5 - t4
+        if kind == "train":
+            p = np.zeros(59 * sub.n)
+            O.adam(p, p + 1e-3, p, p, 1e-3, 1)
+            t_adam = time.perf_counter() - t5
+    P = V * c.width * c.height
+    step_s = ((t1 - t0) + t_pb + t_adam) * scale_g + ((t3 - t2) + t_bwd) * P / sample_pixels
+    measured = time.perf_counter() - t0
     out = dict(value=P / step_s / 1e6, unit="Mpix/s", cores=O.num_threads(), kind="oracle",
-               sample=("float64 oracle: projection, projection backward and Adam over all %d "
-                       "Gaussians; render + render backward on %d random pixels, extrapolated "
-                       "linearly to %d pixels" % (n, sample_pixels, P)),
-               step_s=step_s, measured_s=t5 - t0)
+               sample=("float64 oracle: projection%s on %d of %d Gaussians (all %d views), "
+                       "scaled by the Gaussian count; render%s on %d random pixels of view 0, "
+                       "scaled to %d pixels" % (
+                           "" if kind == "fwd" else ", projection backward" +
+                           (" and Adam" if kind == "train" else ""),
+                           sub.n, n, V, "" if kind == "fwd" else " + render backward",
+                           sample_pixels, P)),
+               step_s=step_s, measured_s=measured)
     return out, float(ref["n_exp"].mean())
 
 
 def run_reference(args):
-    """--impl reference: the oracle timed on the host, rank 0 only."""
+    """--impl reference: the oracle timed on the host, rank 0 only; each step
+    a bounded sample of the workload (cpu_baseline's split), extrapolated."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     from oracle import oracle as O
     from gaussian_splatting_differentiable_ewa_b200 import scenes as S
-    scene = S.make_scene(WORKLOAD, n=args.n)
+    kind = STEPS[args.workload]["kind"]
+    scene = S.make_scene(args.workload, n=args.n)
     c = scene.cameras[0]
-    P = c.width * c.height
-    n = scene.n
-    sub = max(1, n // 16)
-    small = S.make_scene(WORKLOAD, n=sub)
-    projs_full = O.project_views(scene)
-    rng = np.random.default_rng(7)
-    dL = S.make_upstream_grad(1, c.height, c.width, seed=1)
-    n_pix = 512
+    P = scene.n_views * c.width * c.height
     times = []
+    cpu = None
     for it in range(args.warmup + args.steps):
-        pix = np.stack([np.zeros(n_pix, np.int64), rng.integers(0, c.width, n_pix),
-                        rng.integers(0, c.height, n_pix)], 1).astype(np.int32)
-        gC = dL[0][:, pix[:, 2], pix[:, 1]].T
-        t0 = time.perf_counter()
-        pr = O.project_views(small)
-        t1 = time.perf_counter()
-        O.render(projs_full, scene.cameras, scene.background, pix)
-        g2 = O.render_bwd(projs_full, scene.cameras, scene.background, pix, gC)
-        t2 = time.perf_counter()
-        g2s = np.full((1, sub, 10), 1e-3)
-        O.project_bwd(small, pr, g2s)
-        p = np.zeros(59 * sub)
-        O.adam(p, p + 1e-3, p, p, 1e-3, 1)
-        t3 = time.perf_counter()
-        step = (t1 - t0) * n / sub + (t2 - t1) * P / n_pix + (t3 - t2) * n / sub
+        cpu, _ = cpu_baseline(scene, kind, sample_pixels=256, max_gauss=50_000, seed=7 + it)
         if it >= args.warmup:
-            times.append(step)
+            times.append(cpu["step_s"])
     ms = 1000.0 * float(np.mean(times))
     value = P / (ms / 1000.0) / 1e6
     line = {
@@ -304,14 +367,11 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "gaussians": n, "width": c.width, "height": c.height,
-                   "sh_degree": 3, "views_per_gpu": 1},
+        "config": {"workload": args.workload, "gaussians": scene.n, "width": c.width,
+                   "height": c.height, "sh_degree": scene.sh_degree,
+                   "views_per_gpu": scene.n_views, "step": kind},
         "cpu_baseline": {"value": value, "unit": "Mpix/s", "cores": O.num_threads(),
-                         "kind": "oracle",
-                         "sample": "per step: projection, projection backward and Adam on "
-                                   "%d of %d Gaussians, render + backward on %d random pixels; "
-                                   "each part extrapolated linearly to the full step"
-                                   % (sub, n, n_pix)},
+                         "kind": "oracle", "sample": "per step: " + cpu["sample"]},
         "e2e": {"value": value, "unit": "Mpix/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -466,6 +526,42 @@ def measure_densify(sp) -> dict:
                 pruned=counts[0], kept=counts[1], cloned=counts[2], split=counts[3])
 
 
+def measure_full64_sort(scene, reps: int = 10) -> dict:
+    """gs_bin_sort with 64-bit (global tile << 32 | depth bits) keys on the
+    workload's projections: one emission of every pair's key, the stable
+    least-significant-digit radix passes over the key bits, the tile ranges.
+    Each launch after an L2 flush, mean of `reps` after an untimed one; bytes
+    by the scope table's figures (see algorithmic_work)."""
+    import torch
+    from gaussian_splatting_differentiable_ewa_b200 import api
+    from gaussian_splatting_differentiable_ewa_b200.pipeline import Splatter
+    sp = Splatter(scene, sort_mode=api.GS_SORT_FULL64)
+    sp.ensure_capacity()
+    sp.project()
+    sp.bin_sort()
+    torch.cuda.synchronize()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ms = 0.0
+    for _ in range(reps):
+        flush.fill_(1)
+        e0.record()
+        sp.bin_sort()
+        e1.record()
+        torch.cuda.synchronize()
+        ms += e0.elapsed_time(e1) / reps
+    assert sp.status() == api.GS_OK
+    n_pairs = int(sp.n_pairs.item())
+    plan = sort_plan(sp, "full64")
+    nbytes = algorithmic_work(sp, n_pairs, "full64", 0.0)["gs_bin_sort"]["bytes"]
+    pk = peaks()
+    out = dict(ms=ms, pairs=n_pairs, passes=plan["pair"], gbs=nbytes / (ms / 1e3) / 1e9,
+               hbm_frac=nbytes / (ms / 1e3) / 1e9 / pk["hbm_gbs"], bytes=nbytes)
+    del sp
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -484,20 +580,28 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     mode = api.GS_SORT_PRESORT if args.sort_mode == "presort" else api.GS_SORT_FULL64
+    kind = STEPS[args.workload]["kind"]
 
     from gaussian_splatting_differentiable_ewa_b200 import dist as gdist
-    scene = S.make_scene(WORKLOAD, n=args.n)
+    scene = S.make_scene(args.workload, n=args.n)
     if world > 1:
         scene.cameras = [gdist.orbit_view(scene, rank, world)]
     c = scene.cameras[0]
     sp = Splatter(scene, sort_mode=mode)
-    if world > 1:
+    if world > 1 and kind == "train":
         sp.shard_optimizer(rank, world)
-    need = sp.ensure_capacity()
-    dL_host = S.make_upstream_grad(1, c.height, c.width, seed=1)
-    dL = torch.as_tensor(dL_host).cuda()
+    sp.ensure_capacity()
+    V = sp.V
+    dL_host = S.make_upstream_grad(V, c.height, c.width, seed=1)
+    dL = torch.as_tensor(dL_host).cuda() if kind != "fwd" else None
     stream = torch.cuda.current_stream()
-    pixels = c.width * c.height
+    pixels = V * c.width * c.height
+
+    names = ["gs_project", "gs_bin_sort", "gs_rasterize_fwd"]
+    if kind != "fwd":
+        names += ["gs_rasterize_bwd", "gs_project_bwd", "gs_densify_stats"]
+    if kind == "train":
+        names += ["gs_adam_step" if world == 1 else "reduce_scatter+gs_adam_step+all_gather"]
 
     def step(events=None):
         def mark(k):
@@ -510,23 +614,23 @@ def run_ours(args):
         mark(2)
         sp.rasterize_fwd()
         mark(3)
+        if kind == "fwd":
+            return
         sp.rasterize_bwd(dL, with_params=False)
         mark(4)
         sp.project_bwd()
         mark(5)
         sp.densify_stats()
         mark(6)
-        sp.adam_step()  # with N > 1: reduce-scatter, Adam on the slice, all-gather
-        mark(7)
+        if kind == "train":
+            sp.adam_step()  # with N > 1: reduce-scatter, Adam on the slice, all-gather
+            mark(7)
 
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize()
     assert sp.status() == api.GS_OK, "device status after warm-up"
 
-    names = ["gs_project", "gs_bin_sort", "gs_rasterize_fwd", "gs_rasterize_bwd",
-             "gs_project_bwd", "gs_densify_stats",
-             "gs_adam_step" if world == 1 else "reduce_scatter+gs_adam_step+all_gather"]
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
           for _ in range(args.steps)]
     clocks = ClockSampler(local)
@@ -535,17 +639,28 @@ def run_ours(args):
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.3)
+    # a working set that fits in L2 is flushed (a 256 MB write) before every
+    # step, outside the step's events, and the step time is the sum of the
+    # steps' own event intervals
+    flush_l2 = working_set_bytes(sp) < L2_BYTES
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if flush_l2 else None
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for k in range(args.steps):
+        if flush_l2:
+            flush.fill_(1)
         step(ev[k])
     end.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
     if world > 1:
         dist.barrier()
-    elapsed_ms = gdist.max_over_ranks(start.elapsed_time(end), device="cuda")
+    if flush_l2:
+        own = sum(ev[k][0].elapsed_time(ev[k][-1]) for k in range(args.steps))
+        elapsed_ms = gdist.max_over_ranks(own, device="cuda")
+    else:
+        elapsed_ms = gdist.max_over_ranks(start.elapsed_time(end), device="cuda")
     per_call = {nm: float(np.mean([ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(args.steps)]))
                 for i, nm in enumerate(names)}
     ms = elapsed_ms / args.steps
@@ -553,38 +668,70 @@ def run_ours(args):
     n_pairs = int(sp.n_pairs.item())
     status = sp.status()
 
-    # end to end through the library's host-fed step (Splatter.train_from_host):
-    # every step uploads its upstream gradient from pinned host memory and
-    # downloads the rendered image to it, on a copy stream overlapping the
-    # compute stream
+    # the measurement protocol of the scope table: 20 warm-up steps, then the
+    # median of 100 steps, each timed by its own events (single GPU)
+    protocol = None
+    if world == 1:
+        for _ in range(20):
+            step()
+        pev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+               for _ in range(100)]
+        for k in range(100):
+            if flush_l2:
+                flush.fill_(1)
+            step(pev[k])
+        torch.cuda.synchronize()
+        st = np.array([pev[k][0].elapsed_time(pev[k][-1]) for k in range(100)])
+        protocol = {"warmup": 20, "steps": 100, "median_ms": float(np.median(st)),
+                    "mean_ms": float(st.mean()), "p10_ms": float(np.percentile(st, 10)),
+                    "p90_ms": float(np.percentile(st, 90)),
+                    "median_mpix_s": pixels / (float(np.median(st)) / 1000.0) / 1e6,
+                    "per_call_median_ms": {
+                        nm: float(np.median([pev[k][i].elapsed_time(pev[k][i + 1])
+                                             for k in range(100)]))
+                        for i, nm in enumerate(names)}}
+
+    # end to end through the library's host-fed calls: every step uploads its
+    # upstream gradient from pinned host memory (training) and downloads the
+    # rendered image to it, on a copy stream overlapping the compute stream
     e2e = None
     if not args.no_e2e:
-        h_in = torch.from_numpy(dL_host).pin_memory()
         h_out = torch.empty(sp.image.shape, dtype=torch.float32).pin_memory()
         sp.stream = torch.cuda.Stream()
-        sp.train_from_host([h_in] * 3, [h_out] * 3)  # warm-up
+        if kind == "fwd":
+            run = lambda k: sp.render_to_host([h_out] * k)  # noqa: E731
+            h2d = 88 * V  # the camera structs, passed by value with every launch
+        else:
+            h_in = torch.from_numpy(dL_host).pin_memory()
+            run = lambda k: sp.train_from_host([h_in] * k, [h_out] * k,  # noqa: E731
+                                               adam=(kind == "train"))
+            h2d = int(h_in.numel() * 4)
+        run(3)  # warm-up
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         e0.record(sp.stream)
-        sp.train_from_host([h_in] * args.steps, [h_out] * args.steps)
+        run(args.steps)
         e1.record(sp.stream)
         torch.cuda.synchronize()
         sp.stream = None
         e_ms = gdist.max_over_ranks(e0.elapsed_time(e1) / args.steps, device="cuda")
         e2e = {"value": world * pixels / (e_ms / 1000.0) / 1e6, "unit": "Mpix/s",
-               "ms_per_step": e_ms, "h2d_bytes_per_step": int(h_in.numel() * 4),
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": int(h_out.numel() * 4)}
 
-    # densify_and_prune once, on the statistics the timed steps accumulated
-    # (not part of the step: it runs every few hundred steps)
+    # beside the step, on the default workload: densify_and_prune once on the
+    # statistics the timed steps accumulated (it runs every few hundred
+    # steps), the loss, the quantised-SH Adam step and the full-64 sort
     extras = {}
-    if world == 1:
+    if world == 1 and not args.no_extras and args.workload == DEFAULT_WORKLOAD:
         extras["gs_densify_and_prune"] = measure_densify(sp)
         extras["gs_l1_dssim"] = measure_loss(sp)
         extras["gs_adam_step_sh_quant"] = measure_quant_adam(sp)
+        if args.sort_mode != "full64":
+            extras["gs_bin_sort_full64"] = measure_full64_sort(scene)
 
     if world > 1:
         dist.barrier()
@@ -596,61 +743,70 @@ def run_ours(args):
     cpu = None
     exps = None
     if world == 1 and not args.no_cpu_baseline:
-        cpu, nexp_mean = cpu_baseline(scene)
+        cpu, nexp_mean = cpu_baseline(scene, kind)
         exps = nexp_mean * pixels
     pk = peaks()
     work = algorithmic_work(sp, n_pairs, args.sort_mode, exps or 0.0)
-    if world > 1:
+    if world > 1 and kind == "train":
         work["gs_adam_step"]["bytes"] /= world  # each rank updates its slice only
     kernels = {}
+    sfu = sfu_peak_gexps(pk["sm_max_mhz"])
     for nm in names:
-        if nm not in work:
+        key = nm if nm in work else "gs_adam_step"
+        if key not in work:
             continue
         t = per_call[nm] / 1000.0
-        w = work[nm]
-        kernels[nm] = dict(ms=per_call[nm], gbs=w["bytes"] / t / 1e9,
-                           hbm_frac=w["bytes"] / t / 1e9 / pk["hbm_gbs"])
+        w = work[key]
+        k = dict(ms=per_call[nm], bytes=w["bytes"], gbs=w["bytes"] / t / 1e9,
+                 hbm_frac=w["bytes"] / t / 1e9 / pk["hbm_gbs"])
+        bound_s = w["bytes"] / (pk["hbm_gbs"] * 1e9)
         if w["exps"]:
-            kernels[nm]["gexps"] = w["exps"] / t / 1e9
+            k["gexps"] = w["exps"] / t / 1e9
+            k["sfu_frac"] = k["gexps"] / sfu
+            bound_s = max(bound_s, w["exps"] / (sfu * 1e9))
+        k["bound_ms"] = bound_s * 1000.0
+        k["roofline_frac"] = bound_s / t
+        kernels[nm] = k
     dom = max(kernels, key=lambda k: kernels[k]["ms"])
-    sm_for_peak = pk["sm_max_mhz"]
-    t_hbm = work[dom]["bytes"] / (pk["hbm_gbs"] * 1e9)
-    t_sfu = (work[dom]["exps"] / (sfu_peak_gexps(sm_for_peak) * 1e9)) if exps else 0.0
+    dk = "gs_adam_step" if dom not in work else dom
+    t_hbm = work[dk]["bytes"] / (pk["hbm_gbs"] * 1e9)
+    t_sfu = (work[dk]["exps"] / (sfu * 1e9)) if exps else 0.0
     if t_sfu > t_hbm:
-        peak = sfu_peak_gexps(sm_for_peak)
-        ach = work[dom]["exps"] / (per_call[dom] / 1000.0) / 1e9
-        roof = {"kernel": dom, "bound": "alu", "achieved": ach, "peak": peak, "unit": "Gexp/s",
-                "frac": ach / peak, "traffic": profiled_traffic(dom, WORKLOAD),
-                "peak_source": "148 SM x 16 MUFU.EX2/clk x %.0f MHz (max SM clock)" % sm_for_peak}
+        ach = work[dk]["exps"] / (per_call[dom] / 1000.0) / 1e9
+        roof = {"kernel": dom, "bound": "alu", "achieved": ach, "peak": sfu, "unit": "Gexp/s",
+                "frac": ach / sfu, "traffic": profiled_traffic(dk, args.workload),
+                "peak_source": "148 SM x 16 MUFU.EX2/clk x %.0f MHz (max SM clock)"
+                               % pk["sm_max_mhz"]}
     else:
-        ach = work[dom]["bytes"] / (per_call[dom] / 1000.0) / 1e9
+        ach = work[dk]["bytes"] / (per_call[dom] / 1000.0) / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"],
                 "unit": "GB/s", "frac": ach / pk["hbm_gbs"],
-                "traffic": profiled_traffic(dom, WORKLOAD),
+                "traffic": profiled_traffic(dk, args.workload),
                 "peak_source": pk["source"] + " (MEASURED_PEAKS.json copy bandwidth)"}
     # step roofline: sum over calls of max(bytes / HBM, exps / SFU)
-    bound_s = 0.0
-    for nm, w in work.items():
-        bound_s += max(w["bytes"] / (pk["hbm_gbs"] * 1e9),
-                       (w["exps"] / (sfu_peak_gexps(sm_for_peak) * 1e9)) if w["exps"] else 0.0)
-    n_launch = launches_per_step(sp, args.sort_mode)
+    bound_ms = sum(k["bound_ms"] for k in kernels.values())
+    n_launch = launches_per_step(sp, args.sort_mode, kind)
     line = {
         "metric": METRIC, "value": value, "unit": "Mpix/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "gaussians": sp.n, "width": c.width, "height": c.height,
-                   "sh_degree": 3, "views_per_gpu": 1, "pairs": n_pairs,
-                   "sort_mode": args.sort_mode,
+        "config": {"workload": args.workload, "step": kind, "gaussians": sp.n,
+                   "width": c.width, "height": c.height, "views_per_gpu": V,
+                   "sh_degree": sp.deg, "pairs": n_pairs, "sort_mode": args.sort_mode,
                    "sort_path": sort_plan(sp, args.sort_mode)["path"],
-                   "l2": "working set larger than L2 (0.7 GB of parameters and Adam state "
-                         "rewritten every step)",
+                   "l2": ("working set %.0f MB inside the 126 MB L2: flushed (256 MB write) "
+                          "before every step, outside the step's own timing"
+                          % (working_set_bytes(sp) / 1e6)) if flush_l2 else
+                         ("working set %.0f MB, larger than the 126 MB L2"
+                          % (working_set_bytes(sp) / 1e6)),
                    "parallelism": "dp%d (one view per GPU; gradient reduce-scatter, Adam on "
                                   "1/%d of the parameters, parameter all-gather)" % (world, world)
                    if world > 1 else "single GPU"},
         "roofline": roof,
-        "step_roofline": {"bound_ms": bound_s * 1000.0, "frac": bound_s * 1000.0 / ms},
+        "step_roofline": {"bound_ms": bound_ms, "frac": bound_ms / ms},
         "kernels": kernels,
+        "protocol": protocol,
         "extras": extras,
         "cpu_baseline": None if cpu is None else {k: cpu[k] for k in
                                                   ("value", "unit", "cores", "kind", "sample")},

@@ -28,9 +28,18 @@ GS_ERR_CUDA = 6
 GS_SORT_FULL64 = 0
 GS_SORT_PRESORT = 1
 
+# bits of the device status word
+GS_STATUS_BIT_CAPACITY = 1
+GS_STATUS_BIT_TIMEOUT = 2
+GS_STATUS_BIT_BOUNDS = 4
+GS_STATUS_BIT_NONFINITE = 8
+
+# gs_debug_stall sites
+GS_STALL_NONE, GS_STALL_EMIT_LOOKBACK, GS_STALL_RASTER_FWD, GS_STALL_RASTER_BWD = 0, 1, 2, 3
+
 GS_TILE = 16
 GS_MAX_VIEWS = 32
-GS_RECORD_FLOATS = 12
+GS_RECORD_FLOATS = 16
 GS_GRAD2D_FLOATS = 12
 
 _c = ctypes
@@ -80,17 +89,18 @@ SIGNATURES = [
     ("gs_workspace_size", _c.c_size_t,
      [_c.c_int64, _c.c_int32, _c.POINTER(GsCamera), _c.c_int64, _c.c_int32]),
     ("gs_project", _c.c_int,
-     [_c.POINTER(GsParams), _c.POINTER(GsCamera), _c.c_int32, _c.POINTER(GsProjected), _vp]),
+     [_c.POINTER(GsParams), _c.POINTER(GsCamera), _c.c_int32, _c.POINTER(GsProjected), _vp,
+      _vp]),
     ("gs_bin_sort", _c.c_int,
      [_c.POINTER(GsProjected), _c.POINTER(GsCamera), _c.c_int32, _c.c_int64, _c.c_int32,
       _c.POINTER(GsBinned), _vp, _c.c_size_t, _vp]),
     ("gs_rasterize_fwd", _c.c_int,
      [_c.POINTER(GsProjected), _c.POINTER(GsBinned), _c.POINTER(GsCamera), _c.c_int32,
-      _c.c_int64, _c.POINTER(_c.c_float), _vp, _vp, _vp, _vp]),
+      _c.c_int64, _c.POINTER(_c.c_float), _vp, _vp, _vp, _vp, _vp]),
     ("gs_rasterize_bwd", _c.c_int,
      [_c.POINTER(GsParams), _c.POINTER(GsProjected), _c.POINTER(GsBinned),
       _c.POINTER(GsCamera), _c.c_int32, _c.POINTER(_c.c_float), _vp, _vp, _vp, _vp,
-      _c.POINTER(GsGrads), _vp]),
+      _c.POINTER(GsGrads), _vp, _vp]),
     ("gs_project_bwd", _c.c_int,
      [_c.POINTER(GsParams), _c.POINTER(GsCamera), _c.c_int32, _vp, _vp, _c.POINTER(GsGrads),
       _vp]),
@@ -115,6 +125,7 @@ SIGNATURES = [
       _c.c_int32, _c.c_uint64, _vp]),
     ("gs_bin_sort_plan", _c.c_int,
      [_c.c_int64, _c.c_int32, _c.POINTER(GsCamera), _c.c_int32, _c.c_void_p]),
+    ("gs_debug_stall", _c.c_int, [_c.c_int32, _c.c_int64, _c.c_double]),
     ("gs_bin_sort_noalloc", _c.c_int,
      [_c.POINTER(GsProjected), _c.POINTER(GsCamera), _c.c_int32, _c.c_int64, _c.c_int32,
       _c.POINTER(GsBinned), _vp, _vp]),
@@ -220,9 +231,9 @@ def gs_workspace_size(n: int, cams_arr, n_views: int, pair_capacity: int, sort_m
                                        int(sort_mode)))
 
 
-def gs_project(p: GsParams, cams_arr, n_views: int, out: GsProjected, stream=None) -> None:
-    _check(lib().gs_project(_c.byref(p), cams_arr, int(n_views), _c.byref(out), _stream(stream)),
-           "gs_project")
+def gs_project(p: GsParams, cams_arr, n_views: int, out: GsProjected, ws, stream=None) -> None:
+    _check(lib().gs_project(_c.byref(p), cams_arr, int(n_views), _c.byref(out), _ptr(ws),
+                            _stream(stream)), "gs_project")
 
 
 def gs_bin_sort(proj: GsProjected, cams_arr, n_views: int, n: int, sort_mode: int,
@@ -233,20 +244,25 @@ def gs_bin_sort(proj: GsProjected, cams_arr, n_views: int, n: int, sort_mode: in
 
 
 def gs_rasterize_fwd(proj: GsProjected, bins: GsBinned, cams_arr, n_views: int, n: int, bg,
-                     image, final_T, n_contrib, stream=None) -> None:
+                     image, final_T, n_contrib, ws, stream=None) -> None:
     _check(lib().gs_rasterize_fwd(_c.byref(proj), _c.byref(bins), cams_arr, int(n_views), int(n),
                                   _floats3(bg), _ptr(image), _ptr(final_T), _ptr(n_contrib),
-                                  _stream(stream)), "gs_rasterize_fwd")
+                                  _ptr(ws), _stream(stream)), "gs_rasterize_fwd")
 
 
 def gs_rasterize_bwd(p: GsParams, proj: GsProjected, bins: GsBinned, cams_arr, n_views: int, bg,
-                     dL_dimage, final_T, n_contrib, grad2d, g: Optional[GsGrads],
+                     dL_dimage, final_T, n_contrib, grad2d, g: Optional[GsGrads], ws,
                      stream=None) -> None:
     _check(lib().gs_rasterize_bwd(_c.byref(p), _c.byref(proj), _c.byref(bins), cams_arr,
                                   int(n_views), _floats3(bg), _ptr(dL_dimage), _ptr(final_T),
                                   _ptr(n_contrib), _ptr(grad2d),
-                                  None if g is None else _c.byref(g), _stream(stream)),
+                                  None if g is None else _c.byref(g), _ptr(ws), _stream(stream)),
            "gs_rasterize_bwd")
+
+
+def gs_debug_stall(site: int, index: int = -1, wait_limit_s: float = 0.0) -> None:
+    """Test hook: make one device-side wait run out (see include/gs.h)."""
+    _check(lib().gs_debug_stall(int(site), int(index), float(wait_limit_s)), "gs_debug_stall")
 
 
 def gs_project_bwd(p: GsParams, cams_arr, n_views: int, radii, grad2d, g: GsGrads,

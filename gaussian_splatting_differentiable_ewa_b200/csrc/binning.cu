@@ -36,9 +36,9 @@
 //                  fewest passes (13 bits: 7 + 6), so each key costs one
 //                  ballot per bit of its pass.
 //  k_ranges        [start, end) of each tile in the sorted pairs.
-// The emission's look-back waits are bounded (kSpinLimit) and report through
-// the status word instead of hanging; the radix passes never wait on other
-// blocks.
+// The emission's look-back waits are bounded in time (WaitCfg) and report
+// through the status word instead of hanging; the radix passes never wait on
+// other blocks.
 
 #include <cuda_runtime.h>
 
@@ -107,20 +107,23 @@ __device__ __forceinline__ uint32_t block_exclusive_scan_256(uint32_t x, uint32_
 // round trip and sums them back to the nearest inclusive prefix; publishes
 // the block's inclusive prefix and returns the exclusive prefix (to all lanes
 // of warp 0).
+// A block whose index is wc.stall (a test hook) publishes nothing, so the
+// waits of its successors run out.
 __device__ uint64_t warp_block_lookback(uint64_t* lb, uint32_t idx, uint64_t aggregate,
-                                        uint32_t* status) {
+                                        uint32_t* status, const WaitCfg& wc) {
   const int lane = threadIdx.x & 31;
+  const bool publish = (int64_t)idx != wc.stall;
   if (idx == 0) {
-    if (lane == 0) st_relaxed_u64(&lb[0], kLbPrefix | aggregate);
+    if (lane == 0 && publish) st_relaxed_u64(&lb[0], kLbPrefix | aggregate);
     return 0;
   }
-  if (lane == 0) st_relaxed_u64(&lb[idx], kLbAggregate | aggregate);
+  if (lane == 0 && publish) st_relaxed_u64(&lb[idx], kLbAggregate | aggregate);
   uint64_t excl = 0;
   int64_t base = (int64_t)idx - 1;
   while (true) {
     const int64_t j = base - lane;
     uint64_t w = j >= 0 ? ld_relaxed_u64(&lb[j]) : kLbPrefix;
-    if ((w >> 62) == 0) w = lookback_wait(&lb[j], status);
+    if ((w >> 62) == 0) w = lookback_wait(&lb[j], wc.limit_ns, status);
     const uint32_t pre = __ballot_sync(0xffffffffu, (w >> 62) == 2);
     const int first = pre ? __ffs(pre) - 1 : 32;  // nearest inclusive prefix
     uint64_t val = lane <= first ? (w & kLbValueMask) : 0ull;
@@ -130,7 +133,7 @@ __device__ uint64_t warp_block_lookback(uint64_t* lb, uint32_t idx, uint64_t agg
     if (pre) break;
     base -= 32;
   }
-  if (lane == 0) st_relaxed_u64(&lb[idx], kLbPrefix | (excl + aggregate));
+  if (lane == 0 && publish) st_relaxed_u64(&lb[idx], kLbPrefix | (excl + aggregate));
   return excl;
 }
 
@@ -722,7 +725,7 @@ __global__ void __launch_bounds__(kEmitThreads) k_emit(
     const uint32_t* __restrict__ pvals, int n, int n_views, Grid g,
     K* __restrict__ keys_out, uint32_t* __restrict__ ids_out, int64_t capacity,
     int64_t* __restrict__ n_pairs, uint64_t* __restrict__ lookback, uint32_t* __restrict__ block_counter,
-    uint32_t* __restrict__ status) {
+    uint32_t* __restrict__ status, WaitCfg wc) {
   constexpr int kPer = MODE == 0 ? 4 : 8;           // pairs per thread per window
   constexpr int kWin = kPer * kEmitThreads;         // pairs per window
   constexpr int kWinPad = kWin + kWin / 32;
@@ -790,7 +793,7 @@ __global__ void __launch_bounds__(kEmitThreads) k_emit(
     toff += cnt[k];
   }
   if (threadIdx.x < 32) {
-    const uint64_t base = warp_block_lookback(lookback, bidx, block_total, status);
+    const uint64_t base = warp_block_lookback(lookback, bidx, block_total, status, wc);
     if (threadIdx.x == 0) {
       s_off[kEmitItems] = block_total;
       s_base = base;
@@ -1314,7 +1317,7 @@ cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
     k_emit<1, uint32_t><<<(unsigned)eb, kEmitThreads, 0, stream>>>(
         bins4, a.pkeys[fin], a.pvals[fin], a.n, a.n_views, a.grid,
         reinterpret_cast<uint32_t*>(a.keys[a.emit_buf]), a.vals[a.emit_buf], a.capacity,
-        a.n_pairs, a.emit_lookback, a.counters + 0, a.status);
+        a.n_pairs, a.emit_lookback, a.counters + 0, a.status, a.wait);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // 3) stable sort by tile
     e = run_radix_passes<uint32_t, kSortItems>(
@@ -1331,7 +1334,7 @@ cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
   // full 64-bit keys
   k_emit<0, uint64_t><<<(unsigned)eb, kEmitThreads, 0, stream>>>(
       bins4, nullptr, nullptr, a.n, a.n_views, a.grid, a.keys[a.emit_buf], a.vals[a.emit_buf],
-      a.capacity, a.n_pairs, a.emit_lookback, a.counters + 0, a.status);
+      a.capacity, a.n_pairs, a.emit_lookback, a.counters + 0, a.status, a.wait);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   e = run_radix_passes<uint64_t, kSortItems>(a.keys[a.emit_buf], a.vals[a.emit_buf],
                                              a.keys[a.emit_buf ^ 1], a.vals[a.emit_buf ^ 1],

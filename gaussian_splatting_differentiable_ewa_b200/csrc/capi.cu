@@ -1,11 +1,13 @@
 // capi.cu -- the extern "C" entry points declared in include/gs.h.
 //
 // Host-side argument checks, workspace carving and kernel launches. Nothing
-// here allocates device memory or keeps state between calls.
+// here allocates device memory or keeps state between calls (the only
+// process-wide setting is the test hook of gs_debug_stall).
 
+#include <atomic>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
-#include <mutex>
 #include <cuda_runtime.h>
 
 #include "gs_internal.h"
@@ -140,6 +142,26 @@ CamSet pack_cams(const gs_camera* cams, int32_t n_views) {
 
 inline gs_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GS_OK : GS_ERR_CUDA; }
 
+// gs_debug_stall's setting: which wait site stalls which block, and the wait
+// limit while it holds.
+std::atomic<int32_t> g_stall_site{GS_STALL_NONE};
+std::atomic<int64_t> g_stall_index{-1};
+std::atomic<uint64_t> g_wait_ns{0};
+
+WaitCfg wait_cfg(int32_t site) {
+  WaitCfg w;
+  const uint64_t ns = g_wait_ns.load();
+  w.limit_ns = ns ? ns : kWaitLimitNs;
+  w.stall = g_stall_site.load() == site ? g_stall_index.load() : -1;
+  return w;
+}
+
+bool status_ws_ok(const void* ws) { return ws && aligned(ws, kAlign); }
+
+uint32_t* status_word(void* ws) {
+  return reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(ws) + kStatusOffset);
+}
+
 }  // namespace
 
 extern "C" {
@@ -167,8 +189,9 @@ size_t gs_workspace_size(int64_t n, int32_t n_views, const gs_camera* cams, int6
 }
 
 gs_status gs_project(const gs_params* params, const gs_camera* cams, int32_t n_views,
-                     gs_projected* out, void* stream) {
-  if (!params || !out || !check_cams(cams, n_views)) return GS_ERR_INVALID_ARG;
+                     gs_projected* out, void* ws, void* stream) {
+  if (!params || !out || !check_cams(cams, n_views) || !status_ws_ok(ws))
+    return GS_ERR_INVALID_ARG;
   const gs_params& p = *params;
   if (p.n < 0) return GS_ERR_INVALID_ARG;
   if (p.n >= (1ll << 31) || p.n * n_views >= (1ll << 40)) return GS_ERR_OVERFLOW;
@@ -182,6 +205,7 @@ gs_status gs_project(const gs_params* params, const gs_camera* cams, int32_t n_v
     return GS_ERR_INVALID_ARG;
   const CamSet cs = pack_cams(cams, n_views);
   return cuda_status(launch_project(p, cs, n_views, out->records, out->bins, out->radii,
+                                    status_word(ws), wait_cfg(GS_STALL_NONE),
                                     static_cast<cudaStream_t>(stream)));
 }
 
@@ -239,6 +263,7 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
   a.emit_lookback = reinterpret_cast<uint64_t*>(w + L.off_emit_lb);
   a.counters = reinterpret_cast<uint32_t*>(w + kCountersOffset);
   a.status = reinterpret_cast<uint32_t*>(w + kStatusOffset);
+  a.wait = wait_cfg(GS_STALL_EMIT_LOOKBACK);
   a.n_pairs = out->n_pairs;
   a.n_items_dev = reinterpret_cast<int64_t*>(w + kNItemsOffset);
   a.pair_total = reinterpret_cast<unsigned long long*>(w + kPairTotalOffset);
@@ -256,15 +281,18 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
 
 gs_status gs_rasterize_fwd(const gs_projected* proj, const gs_binned* bins, const gs_camera* cams,
                            int32_t n_views, int64_t n, const float* bg, float* image,
-                           float* final_T, uint32_t* n_contrib, void* stream) {
-  if (!proj || !bins || !bg || !check_cams(cams, n_views)) return GS_ERR_INVALID_ARG;
+                           float* final_T, uint32_t* n_contrib, void* ws, void* stream) {
+  if (!proj || !bins || !bg || !check_cams(cams, n_views) || !status_ws_ok(ws))
+    return GS_ERR_INVALID_ARG;
   if (n < 0) return GS_ERR_INVALID_ARG;
   if (n >= (1ll << 31)) return GS_ERR_OVERFLOW;
   if (!image || !final_T || !n_contrib || !bins->ranges || !bins->ids) return GS_ERR_INVALID_ARG;
   if (n > 0 && (!proj->records || !aligned(proj->records, 16))) return GS_ERR_INVALID_ARG;
   const Grid g = grid_of(cams[0]);
   return cuda_status(launch_raster_fwd(proj->records, bins->ids, bins->ranges, bins->pair_capacity,
-                                       g, n_views, (int)n, bg, image, final_T, n_contrib, nullptr,
+                                       g, n_views, (int)n, bg, image, final_T, n_contrib,
+                                       status_word(ws),
+                                       wait_cfg(GS_STALL_RASTER_FWD),
                                        static_cast<cudaStream_t>(stream)));
 }
 
@@ -305,8 +333,9 @@ gs_status gs_rasterize_bwd(const gs_params* params, const gs_projected* proj,
                            const gs_binned* bins, const gs_camera* cams, int32_t n_views,
                            const float* bg, const float* dL_dimage, const float* final_T,
                            const uint32_t* n_contrib, float* grad2d, gs_grads* grads,
-                           void* stream) {
-  if (!params || !proj || !bins || !bg || !check_cams(cams, n_views)) return GS_ERR_INVALID_ARG;
+                           void* ws, void* stream) {
+  if (!params || !proj || !bins || !bg || !check_cams(cams, n_views) || !status_ws_ok(ws))
+    return GS_ERR_INVALID_ARG;
   const gs_params& p = *params;
   if (p.n < 0 || p.sh_degree < 0 || p.sh_degree > 3) return GS_ERR_INVALID_ARG;
   if (p.n >= (1ll << 31)) return GS_ERR_OVERFLOW;
@@ -323,7 +352,8 @@ gs_status gs_rasterize_bwd(const gs_params* params, const gs_projected* proj,
     return GS_ERR_CUDA;
   cudaError_t e = launch_raster_bwd(proj->records, bins->ids, bins->ranges, bins->pair_capacity, g,
                                     n_views, (int)p.n, bg, dL_dimage, final_T, n_contrib, grad2d,
-                                    nullptr, st);
+                                    status_word(ws),
+                                    wait_cfg(GS_STALL_RASTER_BWD), st);
   if (e != cudaSuccess) return GS_ERR_CUDA;
   if (!grads) return GS_OK;
   const CamSet cs = pack_cams(cams, n_views);
@@ -371,23 +401,13 @@ namespace {
 // cudaGetSymbolAddress and passed to the kernels.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[GS_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mutex;
-void* g_noalloc_addr[kMaxDevices] = {};
-
-// Device address of the scratch on the current device (looked up on the
-// first call for that device).
+// Device address of the scratch on the current device, looked up on every
+// call (a host-side query, cheap after the first one on a device): a cached
+// address would go stale when a cudaDeviceReset rebuilds the context.
 gs_status noalloc_scratch(void** addr) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GS_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return GS_ERR_INVALID_ARG;
-  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GS_ERR_CUDA;
-    g_noalloc_addr[dev] = p;
-  }
-  *addr = g_noalloc_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GS_ERR_CUDA;
+  *addr = p;
   return GS_OK;
 }
 
@@ -549,6 +569,17 @@ gs_status gs_bin_sort_plan(int64_t n, int32_t n_views, const gs_camera* cams,
   plan->pair_passes = L.tile_emit ? 0 : L.pairs.passes;
   plan->gaussians_per_block = L.tile_emit ? L.gsize : 0;
   plan->blocks_per_view = L.tile_emit ? L.tile_bpv : 0;
+  return GS_OK;
+}
+
+gs_status gs_debug_stall(int32_t site, int64_t index, double wait_limit_s) {
+  if (site < GS_STALL_NONE || site > GS_STALL_RASTER_BWD) return GS_ERR_INVALID_ARG;
+  if (!(wait_limit_s >= 0.0) || wait_limit_s > 60.0) return GS_ERR_INVALID_ARG;
+  if (site != GS_STALL_NONE && index < 0) return GS_ERR_INVALID_ARG;
+  g_stall_site.store(GS_STALL_NONE);
+  g_stall_index.store(site == GS_STALL_NONE ? -1 : index);
+  g_wait_ns.store((uint64_t)std::llround(wait_limit_s * 1e9));
+  g_stall_site.store(site);
   return GS_OK;
 }
 

@@ -29,8 +29,16 @@ constexpr uint32_t kStatusNonfinite = 1u << 3;
 // kStatusNonfinite when it meets one.
 constexpr uint32_t kNonfiniteKeyBits = 0x7FC0BAD0u;
 
-// Spin limit of every device-side wait (iterations of ~100 ns each).
-constexpr uint32_t kSpinLimit = 20u * 1000u * 1000u;
+// Every device-side wait (an mbarrier phase, a look-back flag) gives up after
+// a time limit on the global nanosecond timer, sets kStatusTimeout and
+// returns. `stall` names one block (a raster tile, an emission block) that
+// is made to wait for something that never comes -- a test hook that
+// exercises the timeout path; -1 (the default) stalls nothing.
+struct WaitCfg {
+  uint64_t limit_ns;
+  int64_t stall;
+};
+constexpr uint64_t kWaitLimitNs = 2000ull * 1000ull * 1000ull;  // 2 s
 
 // Cameras travel in the kernel parameter block.
 struct CamSet {
@@ -51,10 +59,15 @@ __host__ __device__ inline Grid grid_of(const gs_camera& c) {
   return g;
 }
 
-// Raster record field offsets (floats), see gs.h.
+// Raster record field offsets (floats), see gs.h. The 2D Gaussian is kept in
+// the form the rasteriser evaluates: the mean split into a float and the
+// float of its remainder (carried in c1, c2), the rows w1, w2 of W with
+// W^T W = (log2(e) / 2) conic, and nlo = -log2(255 opacity), so that
+//   zq = (w1 . d)^2 + (w2 . d)^2 - log2(255 o) = -log2(255 alpha_raw)
+// and a pixel takes the splat iff zq <= 0.
 enum RecField {
-  R_U = 0, R_V = 1, R_CA = 2, R_CB = 3, R_CC = 4, R_OPAC = 5,
-  R_R = 6, R_G = 7, R_B = 8, R_HX = 9, R_HY = 10, R_SPARE = 11
+  R_U = 0, R_V = 1, R_W1X = 2, R_W1Y = 3, R_C1 = 4, R_W2X = 5, R_W2Y = 6, R_C2 = 7,
+  R_NLO = 8, R_R = 9, R_G = 10, R_B = 11, R_HX = 12, R_HY = 13, R_OPAC = 14, R_SPARE = 15
 };
 // Binning record (one float4): depth key, tile_x word, tile_y word, 0.
 // Screen-space gradient fields (floats), see gs.h.
@@ -62,26 +75,6 @@ enum G2Field {
   G_U = 0, G_V = 1, G_CA = 2, G_CB = 3, G_CC = 4, G_OPAC = 5,
   G_R = 6, G_G = 7, G_B = 8, G_ABS = 9
 };
-
-// Per-pixel opacity of one splat. Forward and backward both call this, so
-// their skip / stop decisions are taken on identical float values.
-//   q = a dx^2 + 2 b dx dy + c dy^2,  d = pixel centre - mean
-//   alpha_raw = o exp(-q/2),  alpha = min(0.99, alpha_raw)
-struct SplatEval {
-  float dx, dy, G, alpha_raw, alpha;
-};
-
-__device__ __forceinline__ SplatEval splat_eval(float px, float py, float u, float v, float ca,
-                                                float cb, float cc, float o) {
-  SplatEval e;
-  e.dx = px - u;
-  e.dy = py - v;
-  float power = -0.5f * (ca * e.dx * e.dx + cc * e.dy * e.dy) - cb * e.dx * e.dy;
-  e.G = __expf(power);
-  e.alpha_raw = o * e.G;
-  e.alpha = fminf(kAlphaMax, e.alpha_raw);
-  return e;
-}
 
 // ---------------------------------------------------------------- PTX wrappers
 
@@ -127,13 +120,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait on an mbarrier phase; on timeout flags the status and returns
-// false (the caller must not touch the buffer).
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait on an mbarrier phase: gives up after limit_ns, flags the
+// status (when given) and returns false. After a false return the caller
+// must not read the buffer, and must wait again before exiting if a copy
+// into it may still be in flight.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  uint32_t* status) {
-  for (uint32_t it = 0; it < kSpinLimit; ++it) {
+                                                  uint64_t limit_ns, uint32_t* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (it > 64) __nanosleep(64);
+    if (globaltimer_ns() - t0 > limit_ns) break;
+    __nanosleep(64);
   }
   if (status) atomicOr(status, kStatusTimeout);
   return false;
@@ -162,21 +166,22 @@ constexpr uint64_t kLbAggregate = 1ull << 62;
 constexpr uint64_t kLbPrefix = 2ull << 62;
 constexpr uint64_t kLbValueMask = (1ull << 62) - 1;
 
-// Wait (bounded) until a look-back word is non-empty; returns it. On timeout
-// flags the status and returns an inclusive-prefix word of 0 so that the
-// caller terminates.
-__device__ __forceinline__ uint64_t lookback_wait(const uint64_t* p, uint32_t* status) {
+// Wait (bounded by limit_ns) until a look-back word is non-empty; returns it.
+// On timeout flags the status and returns an inclusive-prefix word of 0 so
+// that the caller terminates.
+__device__ __forceinline__ uint64_t lookback_wait(const uint64_t* p, uint64_t limit_ns,
+                                                  uint32_t* status) {
   uint64_t w = ld_relaxed_u64(p);
-  uint32_t it = 0;
-  while ((w >> 62) == 0) {
-    if (++it > kSpinLimit) {
-      atomicOr(status, kStatusTimeout);
-      return kLbPrefix;
-    }
-    if (it > 32) __nanosleep(100);
+  if ((w >> 62) != 0) return w;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(100);
     w = ld_relaxed_u64(p);
+    if ((w >> 62) != 0) return w;
+    if (globaltimer_ns() - t0 > limit_ns) break;
   }
-  return w;
+  atomicOr(status, kStatusTimeout);
+  return kLbPrefix;
 }
 
 __device__ __forceinline__ uint32_t lanemask_lt() {

@@ -46,6 +46,7 @@ struct BinSortArgs {
   uint64_t* emit_lookback;           // [emit blocks]
   uint32_t* counters;                // [16] dynamic block counters
   uint32_t* status;
+  WaitCfg wait;                      // look-back wait limit (and test stall)
   int64_t* n_pairs;
   int64_t* n_items_dev;
   unsigned long long* pair_total;  // column emission: exact pair count
@@ -59,7 +60,8 @@ struct BinSortArgs {
 };
 
 cudaError_t launch_project(const gs_params& p, const CamSet& cams, int n_views, float* records,
-                           float* bins, int* radii, cudaStream_t stream);
+                           float* bins, int* radii, uint32_t* status, const WaitCfg& wc,
+                           cudaStream_t stream);
 cudaError_t launch_project_bwd(const gs_params& p, const CamSet& cams, int n_views,
                                const float* grad2d, const int* radii, const gs_grads& g,
                                cudaStream_t stream);
@@ -68,13 +70,13 @@ cudaError_t launch_raster_fwd(const float* records, const uint32_t* ids, const i
                               int64_t capacity, const Grid& g, int n_views, int n,
                               const float bg[3], float* image,
                               float* final_T, uint32_t* n_contrib, uint32_t* status,
-                              cudaStream_t stream);
+                              const WaitCfg& wc, cudaStream_t stream);
 cudaError_t launch_raster_bwd(const float* records, const uint32_t* ids, const int64_t* ranges,
                               int64_t capacity, const Grid& g, int n_views, int n,
                               const float bg[3],
                               const float* dL_dimage, const float* final_T,
                               const uint32_t* n_contrib, float* grad2d, uint32_t* status,
-                              cudaStream_t stream);
+                              const WaitCfg& wc, cudaStream_t stream);
 cudaError_t launch_densify(const float* grad2d, const int* radii, int n_views, int n,
                            float* accum_plain, float* accum_abs, int* denom, cudaStream_t stream);
 cudaError_t launch_adam(const gs_adam_group* groups, int n_groups, float b1, float b2, float eps,

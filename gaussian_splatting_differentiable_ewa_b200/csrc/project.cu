@@ -111,6 +111,10 @@ __device__ __forceinline__ long long floor_tile(double a) {
   return static_cast<long long>(floor(a * (1.0 / kTile)));
 }
 
+constexpr double kHalfLog2e = 0.72134752044448170;  // log2(e) / 2
+constexpr double kInvLn2 = 1.4426950408889634;      // 1 / ln 2
+constexpr double kLog2_255 = 7.9943534368588578;    // log2(255)
+
 constexpr int kProjThreads = 128;     // projection backward block
 constexpr int kProjFwdThreads = 256;  // projection forward block
 constexpr int kShStride = kProjThreads + 1;  // padded row: conflict-free banks
@@ -220,7 +224,9 @@ __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __
                                                           int n_views, CamSet cams,
                                                           float4* __restrict__ records,
                                                           float4* __restrict__ bins,
-                                                          int* __restrict__ radii) {
+                                                          int* __restrict__ radii,
+                                                          uint32_t* __restrict__ status,
+                                                          uint64_t wait_ns) {
   constexpr int K = (DEG + 1) * (DEG + 1);
   // the block's SH coefficients are one contiguous range: a full block with a
   // 16-byte-aligned array fetches them with one bulk copy that lands while
@@ -286,9 +292,9 @@ __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __
     // near-plane cull
     const float key = __fmaf_rn(c.viewmat[8], m.x,
                                 __fmaf_rn(c.viewmat[9], m.y, __fmaf_rn(c.viewmat[10], m.z, c.viewmat[11])));
-    float rec[12];
+    float rec[GS_RECORD_FLOATS];
 #pragma unroll
-    for (int k = 0; k < 12; ++k) rec[k] = 0.f;
+    for (int k = 0; k < GS_RECORD_FLOATS; ++k) rec[k] = 0.f;
     int radius = 0;
     bool nonfinite = !finite_in;
     bool ok = finite_in && key >= (float)kNear;
@@ -320,7 +326,8 @@ __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __
       if (ok) {
         const double idet = 1.0 / det;
         const double mid = 0.5 * (A + C);
-        const double lam = mid + sqrt(0.25 * (A - C) * (A - C) + B * B);
+        const double rr = sqrt(0.25 * (A - C) * (A - C) + B * B);
+        const double lam = mid + rr;
         double rd = ceil(3.0 * sqrt(lam));
         if (!(rd <= (double)kMaxRadius)) rd = (double)kMaxRadius;
         radius = (int)rd;
@@ -334,11 +341,36 @@ __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __
         y1 = fy1 > g.tiles_y - 1 ? g.tiles_y - 1 : fy1;
         ok = (x0 <= x1) && (y0 <= y1);
         if (ok) {
-          rec[R_U] = (float)u;
-          rec[R_V] = (float)vv;
-          rec[R_CA] = (float)(C * idet);
-          rec[R_CB] = (float)(-B * idet);
-          rec[R_CC] = (float)(A * idet);
+          // evaluation form: q' = (log2(e)/2) d^T cov^-1 d = (w1 . d)^2 + (w2 . d)^2
+          // with w_i = sqrt(log2(e) / (2 lambda_i)) e_i over the unit eigenvectors
+          // e_i of cov2d (lambda_2 = det / lambda_1 without cancellation; e_1 from
+          // the row of cov2d - lambda_1 I that has no cancellation)
+          const double h = 0.5 * (A - C);
+          double e1x = h >= 0.0 ? h + rr : B, e1y = h >= 0.0 ? B : rr - h;
+          const double en = sqrt(e1x * e1x + e1y * e1y);
+          if (en > 0.0) {
+            e1x /= en;
+            e1y /= en;
+          } else {  // isotropic: any orthonormal pair
+            e1x = 1.0;
+            e1y = 0.0;
+          }
+          const double k1 = sqrt(kHalfLog2e / lam), k2 = sqrt(kHalfLog2e * lam * idet);
+          const float w1x = (float)(k1 * e1x), w1y = (float)(k1 * e1y);
+          const float w2x = (float)(-k2 * e1y), w2y = (float)(k2 * e1x);
+          // the mean as a float plus the float rows applied to its remainder
+          const float uh = (float)u, vh = (float)vv;
+          const double ulo = u - (double)uh, vlo = vv - (double)vh;
+          rec[R_U] = uh;
+          rec[R_V] = vh;
+          rec[R_W1X] = w1x;
+          rec[R_W1Y] = w1y;
+          rec[R_C1] = (float)(-((double)w1x * ulo + (double)w1y * vlo));
+          rec[R_W2X] = w2x;
+          rec[R_W2Y] = w2y;
+          rec[R_C2] = (float)(-((double)w2x * ulo + (double)w2y * vlo));
+          // -log2(255 o), o = 1 / (1 + e^-logit): log2(255) - log2(1 + e^-logit)
+          rec[R_NLO] = (float)(log1p(exp(-(double)lg)) * kInvLn2 - kLog2_255);
           rec[R_OPAC] = (float)opac_d;
           // half-widths of the box around {q <= Q}, with Q padded (0.2 % +
           // 1e-4) well beyond the float rounding of the rasteriser's alpha
@@ -356,11 +388,11 @@ __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __
           float inv = rsqrtf(dxv * dxv + dyv * dyv + dzv * dzv);
           float rgb[3];
           bool colour_finite;
-          if (staged) {
-            if (!sh_ready) sh_ready = mbar_wait_bounded(&s_bar, 0u, nullptr);
+          if (staged && !sh_ready) sh_ready = mbar_wait_bounded(&s_bar, 0u, wait_ns, status);
+          if (sh_ready && staged) {
             colour_finite = sh_colour_smem<DEG>(s_sh + (size_t)threadIdx.x * K * 3, dxv * inv,
                                                 dyv * inv, dzv * inv, rgb);
-          } else {
+          } else {  // not staged, or the staging copy did not land in time
             colour_finite = sh_colour_global<DEG>(shi, dxv * inv, dyv * inv, dzv * inv, rgb);
           }
           rec[R_R] = rgb[0];
@@ -378,22 +410,23 @@ __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __
       radius = 0;
       x0 = 1; x1 = 0; y0 = 1; y1 = 0;
 #pragma unroll
-      for (int k = 0; k < 12; ++k) rec[k] = 0.f;
+      for (int k = 0; k < GS_RECORD_FLOATS; ++k) rec[k] = 0.f;
       rec[R_HX] = -1.f;
       rec[R_HY] = -1.f;
     }
     const size_t r = (size_t)v * n + i;
-    float4* out = records + r * 3;
-    out[0] = make_float4(rec[0], rec[1], rec[2], rec[3]);
-    out[1] = make_float4(rec[4], rec[5], rec[6], rec[7]);
-    out[2] = make_float4(rec[8], rec[9], rec[10], rec[11]);
+    float4* out = records + r * (GS_RECORD_FLOATS / 4);
+#pragma unroll
+    for (int k = 0; k < GS_RECORD_FLOATS / 4; ++k)
+      out[k] = make_float4(rec[4 * k], rec[4 * k + 1], rec[4 * k + 2], rec[4 * k + 3]);
     bins[r] = make_float4(nonfinite ? __uint_as_float(kNonfiniteKeyBits) : key,
                           __uint_as_float((uint32_t)x0 | ((uint32_t)x1 << 16)),
                           __uint_as_float((uint32_t)y0 | ((uint32_t)y1 << 16)), 0.f);
     radii[r] = radius;
   }
   // a staged copy lands before the block exits, even if no view needed it
-  if (staged && !sh_ready) mbar_wait_bounded(&s_bar, 0u, nullptr);
+  // (after a wait that gave up, this waits once more for it)
+  if (staged && !sh_ready) mbar_wait_bounded(&s_bar, 0u, wait_ns, status);
 }
 
 // Backward of k_project for the raw parameters, summing every view in which
@@ -606,7 +639,8 @@ __global__ void __launch_bounds__(kProjThreads, 6) k_project_bwd(
 }  // namespace
 
 cudaError_t launch_project(const gs_params& p, const CamSet& cams, int n_views, float* records,
-                           float* bins, int* radii, cudaStream_t stream) {
+                           float* bins, int* radii, uint32_t* status, const WaitCfg& wc,
+                           cudaStream_t stream) {
   const int n = (int)p.n;
   if (n == 0) return cudaSuccess;
   const int threads = kProjFwdThreads;
@@ -621,7 +655,7 @@ cudaError_t launch_project(const gs_params& p, const CamSet& cams, int n_views, 
     const int smem = threads * 3 * (D + 1) * (D + 1) * (int)sizeof(float);                  \
     cudaFuncSetAttribute(k_project<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);   \
     k_project<D><<<blocks, threads, smem, stream>>>(m, s, q, p.opacity_logit, p.sh, n, n_views, \
-                                                    cams, r, b, radii);                     \
+                                                    cams, r, b, radii, status, wc.limit_ns); \
   }
   switch (p.sh_degree) {
     case 0: GS_PFWD(0); break;

@@ -10,21 +10,34 @@
 // the scalar operation, so pixel results do not depend on the pairing).
 //
 // The tile's depth-sorted list is consumed in batches of 128 records; each
-// thread stages one 48-byte record into shared memory with a TMA bulk copy
+// thread stages one 64-byte record into shared memory with a TMA bulk copy
 // (cp.async.bulk completing on an mbarrier). When a batch lands, thread j
-// rewrites record j into evaluation form (log2-scaled conic, log2 opacity) and
-// marks which warps' pixel blocks its alpha >= 1/255 box reaches; every warp
-// then compacts the batch to the records that can touch its pixels (ballot +
-// popc, order kept) and walks only those. The box is conservative, so the
-// skipped records are exactly ones every pixel of the block would skip.
-// The forward writes the evaluation form to a separate array of (x, x) pairs,
-// so the landing buffer is free for the next batch's copy at once; the
-// backward rewrites records in place (scalar form) and double-buffers.
+// marks which warps' pixel blocks record j's alpha >= 1/255 box reaches;
+// every warp then compacts the batch to the records that can touch its
+// pixels (ballot + popc, order kept) and walks only those. The box is
+// conservative, so the skipped records are exactly ones every pixel of the
+// block would skip. The forward copies each landed record into a separate
+// array of (x, x) pairs, so the landing buffer is free for the next batch's
+// copy at once; the backward reads records in place and double-buffers.
+//
+// Per (pixel, splat) the record's evaluation form (see gs.h) gives
+//   d = P - (uh, vh), p_i = w_i . d + c_i, zq = p1^2 + p2^2 + nlo
+// with zq = -log2(255 alpha_raw): the splat counts iff zq <= 0, and
+// alpha_raw = 2^-zq / 255. Sums of squares of well-scaled terms: the float
+// result stays within a few units of float rounding of zq's magnitude also
+// for elongated splats and for means far from the origin (the mean's float
+// remainder is carried in c_i), with no cancellation as in the conic form.
 //
 // Forward (pwwt.cn sec. 3.3 `composite`, front to back; lshu.cn sec. 3.2
 // `blend`): alpha = min(0.99, o exp(-q/2)); skip alpha < 1/255; stop before a
 // Gaussian that would take T below 1e-4; a warp stops once all its pixels are
 // done and a block once all its warps are (votes).
+//
+// Device-side conditions go to the status word: a list entry naming a
+// Gaussian >= n is clipped to record 0 and masked out (it reaches no pixel),
+// a range outside the ids buffer renders as empty (both kStatusBounds); a
+// batch whose copy does not land within the wait limit ends the tile
+// (kStatusTimeout), after waiting once more for any copy still in flight.
 //
 // Backward: each pixel replays its contributors back to front, recovering
 // T_k = T_{k+1} / (1 - alpha_k), with B_k the colour composited behind k,
@@ -45,18 +58,18 @@ namespace {
 constexpr int kThreads = 128;                    // 4 warps, 8x8 pixels each
 constexpr int kWarps = kThreads / 32;
 constexpr int kBatch = kThreads;                 // records per batch
-constexpr int kRecBytes = GS_RECORD_FLOATS * 4;  // 48
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kLog2AlphaMin = -7.994353436858858f;  // log2(1/255)
+constexpr int kRecBytes = GS_RECORD_FLOATS * 4;  // 64
+constexpr float kInv255 = 1.0f / 255.0f;
+constexpr float kTwoLn2 = 1.3862943611198906f;   // 1 / (log2(e) / 2)
 
 static_assert(kTilePixels == 2 * kThreads, "two pixels per thread");
+static_assert(kRecBytes % 16 == 0, "bulk copies move multiples of 16 bytes");
 
-// Evaluation form of a record, one (x, x) pair per field, so the two-pixel
-// arithmetic takes every operand straight from shared memory:
-// -u, -v, A = -log2(e)/2 conic_a, B = -log2(e) conic_b, C = -log2(e)/2 conic_c,
-// log2(opacity), colour r g b, 2C. 80 bytes per record (the forward's form).
-enum EvPair { V_NU = 0, V_NV, V_A, V_B, V_C, V_LO, V_R, V_G, V_BL, V_C2, kEvPairs };
+// Forward evaluation form of a record, one (x, x) pair per field, so the
+// two-pixel arithmetic takes every operand straight from shared memory:
+// -uh, -vh, w1x, w1y, c1, w2x, w2y, c2, nlo, colour r g b. 96 bytes.
+enum EvPair { V_NU = 0, V_NV, V_W1X, V_W1Y, V_C1, V_W2X, V_W2Y, V_C2, V_NLO, V_R, V_G, V_BL,
+              kEvPairs };
 
 struct RasterGeom {
   Grid g;
@@ -66,13 +79,20 @@ struct RasterGeom {
 
 __device__ __forceinline__ float2 f2(float x) { return make_float2(x, x); }
 
+// alpha_raw = 2^-zq / 255 (zq = -log2(255 alpha_raw)); both directions call
+// this, so their alphas are bit-identical.
+__device__ __forceinline__ float alpha_raw_of(float zq) { return exp2f(-zq) * kInv255; }
+
 // A tile's [start, end) slice, clipped to the ids buffer (a malformed range
-// renders as empty instead of reading outside the buffer).
+// renders as empty instead of reading outside the buffer, and is reported).
 __device__ __forceinline__ void tile_range(const int64_t* ranges, int tile, int64_t capacity,
-                                           int64_t& start, int64_t& end) {
+                                           int64_t& start, int64_t& end, uint32_t* status) {
   start = ranges[2 * (int64_t)tile];
   end = ranges[2 * (int64_t)tile + 1];
-  if (start < 0 || end > capacity || end < start) start = end = 0;
+  if (start < 0 || end > capacity || end < start) {
+    if (threadIdx.x == 0 && status) atomicOr(status, kStatusBounds);
+    start = end = 0;
+  }
 }
 
 // The thread's pixel pair: (px, py) and (px, py + 4).
@@ -117,72 +137,44 @@ __device__ __forceinline__ uint32_t warp_block_mask(float u, float v, float hx, 
   return mask;
 }
 
-// log2 of the unclamped alpha at the pair's pixel centres (pxc, pyc.x) and
-// (pxc, pyc.y); per pixel it is fma(A dx, dx, fma(B dx, dy, fma(C dy, dy, lo)))
-// with dx = pxc - u, dy = pyc - v. dx, A dx and B dx come out as (x, x)
-// pairs. Both directions call this one function, so their skip / stop
-// decisions agree bit for bit.
-__device__ __forceinline__ float2 eval_log2_alpha(const float2* e, float2 pxc, float2 pyc,
-                                                  float2& dx, float2& dy, float2& adx,
-                                                  float2& bdx) {
-  dx = __fadd2_rn(pxc, e[V_NU]);
-  dy = __fadd2_rn(pyc, e[V_NV]);
-  float2 t = __ffma2_rn(__fmul2_rn(e[V_C], dy), dy, e[V_LO]);
-  bdx = __fmul2_rn(e[V_B], dx);
-  t = __ffma2_rn(bdx, dy, t);
-  adx = __fmul2_rn(e[V_A], dx);
-  return __ffma2_rn(adx, dx, t);
+// zq at the pair's pixel centres (pxc, pyc.x) and (pxc, pyc.y):
+//   dx = pxc - uh, dy = pyc - vh, p_i = fma(w_iy, dy, fma(w_ix, dx, c_i)),
+//   zq = fma(p1, p1, fma(p2, p2, nlo)).
+// The backward evaluates the same IEEE operations in the same order
+// (eval_zq_s), so the skip / stop decisions of the two directions agree bit
+// for bit.
+__device__ __forceinline__ float2 eval_zq(const float2* e, float2 pxc, float2 pyc) {
+  const float2 dx = __fadd2_rn(pxc, e[V_NU]);
+  const float2 dy = __fadd2_rn(pyc, e[V_NV]);
+  const float2 p1 = __ffma2_rn(e[V_W1Y], dy, __ffma2_rn(e[V_W1X], dx, e[V_C1]));
+  const float2 p2 = __ffma2_rn(e[V_W2Y], dy, __ffma2_rn(e[V_W2X], dx, e[V_C2]));
+  return __ffma2_rn(p1, p1, __ffma2_rn(p2, p2, e[V_NLO]));
 }
 
-// Write the evaluation form of raw record r and return the 4-bit mask of
-// warps whose 8x8 pixel block its alpha >= 1/255 box overlaps.
+// Write the forward evaluation form of landed record r and return the 4-bit
+// mask of warps whose 8x8 pixel block its alpha >= 1/255 box overlaps.
 __device__ __forceinline__ uint32_t prepare_record(const float* r, float2* e, int x0, int y0) {
-  const float u = r[R_U], v = r[R_V], hx = r[R_HX], hy = r[R_HY];
-  const float o = r[R_OPAC];
-  const float A = -0.5f * kLog2e * r[R_CA], B = -kLog2e * r[R_CB], C = -0.5f * kLog2e * r[R_CC];
+  const float u = r[R_U], v = r[R_V];
   float4* e4 = reinterpret_cast<float4*>(e);
   e4[0] = make_float4(-u, -u, -v, -v);
-  e4[1] = make_float4(A, A, B, B);
-  const float lo = __log2f(o);
-  e4[2] = make_float4(C, C, lo, lo);
-  e4[3] = make_float4(r[R_R], r[R_R], r[R_G], r[R_G]);
-  e4[4] = make_float4(r[R_B], r[R_B], 2.f * C, 2.f * C);
-  return warp_block_mask(u, v, hx, hy, x0, y0);
+  e4[1] = make_float4(r[R_W1X], r[R_W1X], r[R_W1Y], r[R_W1Y]);
+  e4[2] = make_float4(r[R_C1], r[R_C1], r[R_W2X], r[R_W2X]);
+  e4[3] = make_float4(r[R_W2Y], r[R_W2Y], r[R_C2], r[R_C2]);
+  e4[4] = make_float4(r[R_NLO], r[R_NLO], r[R_R], r[R_R]);
+  e4[5] = make_float4(r[R_G], r[R_G], r[R_B], r[R_B]);
+  return warp_block_mask(u, v, r[R_HX], r[R_HY], x0, y0);
 }
 
-// Backward: records are rewritten in place into a scalar evaluation form
-// (slots after the per-batch rewrite in shared memory):
-// 0 u, 1 v, 2 A = -log2(e)/2 conic_a, 3 B = -log2(e) conic_b,
-// 4 C = -log2(e)/2 conic_c, 5 log2(opacity), 6..8 colour, 9 1/opacity.
-enum EvalSlot { E_U = 0, E_V = 1, E_A = 2, E_B = 3, E_C = 4, E_LO = 5, E_R = 6, E_G = 7,
-                E_BL = 8, E_IO = 9 };
-
-// eval_log2_alpha on a scalar evaluation record: per pixel the same IEEE
-// operations in the same order (pxc - u, pyc - v, C dy, fma(C dy, dy, lo),
-// B dx, fma(B dx, dy, .), A dx, fma(A dx, dx, .)), so the backward's skip
-// decisions are bit-identical to the forward's.
-__device__ __forceinline__ float2 eval_log2_alpha_s(const float* r, float pxc, float2 pyc, float& dx,
-                                                  float2& dy) {
-  dx = pxc - r[E_U];
-  dy = __fadd2_rn(pyc, f2(-r[E_V]));
-  float2 t = __ffma2_rn(__fmul2_rn(f2(r[E_C]), dy), dy, f2(r[E_LO]));
-  t = __ffma2_rn(f2(r[E_B] * dx), dy, t);
-  return __ffma2_rn(f2(r[E_A] * dx), f2(dx), t);
-}
-
-// Rewrite record j of a landed batch in place into the scalar evaluation form
-// and return the 4-bit mask of warps whose 8x8 pixel block its alpha >= 1/255
-// box overlaps.
-__device__ __forceinline__ uint32_t prepare_record_s(float* r, int x0, int y0) {
-  const float u = r[R_U], v = r[R_V], hx = r[R_HX], hy = r[R_HY];
-  const float o = r[R_OPAC];
-  const float ca = r[R_CA], cb = r[R_CB], cc = r[R_CC];
-  r[E_A] = -0.5f * kLog2e * ca;
-  r[E_B] = -kLog2e * cb;
-  r[E_C] = -0.5f * kLog2e * cc;
-  r[E_LO] = __log2f(o);
-  r[E_IO] = 1.f / o;
-  return warp_block_mask(u, v, hx, hy, x0, y0);
+// eval_zq on a record in its stored (scalar) form: per pixel the same IEEE
+// operations in the same order (the column offset dx and the inner fmas are
+// shared by the pair); also returns dx, dy and p1, p2 for the gradients.
+__device__ __forceinline__ float2 eval_zq_s(const float* r, float pxc, float2 pyc, float& dx,
+                                            float2& dy, float2& p1, float2& p2) {
+  dx = __fsub_rn(pxc, r[R_U]);
+  dy = __fadd2_rn(pyc, f2(-r[R_V]));
+  p1 = __ffma2_rn(f2(r[R_W1Y]), dy, f2(__fmaf_rn(r[R_W1X], dx, r[R_C1])));
+  p2 = __ffma2_rn(f2(r[R_W2Y]), dy, f2(__fmaf_rn(r[R_W2X], dx, r[R_C2])));
+  return __ffma2_rn(p1, p1, __ffma2_rn(p2, p2, f2(r[R_NLO])));
 }
 
 // Warp-wide compaction of the batch entries whose mask has this warp's bit,
@@ -207,7 +199,7 @@ __global__ void __launch_bounds__(kThreads) k_raster_fwd(
     const float* __restrict__ records, const uint32_t* __restrict__ ids,
     const int64_t* __restrict__ ranges, RasterGeom geo, float bg0, float bg1, float bg2,
     float* __restrict__ image, float* __restrict__ final_T, uint32_t* __restrict__ n_contrib,
-    uint32_t* __restrict__ status) {
+    uint32_t* __restrict__ status, WaitCfg wc) {
   __shared__ __align__(128) float s_rec[kBatch][GS_RECORD_FLOATS];
   __shared__ __align__(16) float2 s_ev[kBatch][kEvPairs];
   __shared__ __align__(8) uint64_t s_bar;
@@ -217,11 +209,13 @@ __global__ void __launch_bounds__(kThreads) k_raster_fwd(
   const int tile = blockIdx.x;
   const TilePix tp = tile_pixel(geo.g, tile);
   int64_t start, end;
-  tile_range(ranges, tile, geo.capacity, start, end);
+  tile_range(ranges, tile, geo.capacity, start, end, status);
   const int64_t cnt = end - start;
   const int nb = (int)((cnt + kBatch - 1) / kBatch);
   const float* rec_view = records + (size_t)tp.view * geo.n * GS_RECORD_FLOATS;
   const int warp = threadIdx.x >> 5;
+  // test hook: this tile issues no copies and waits in vain
+  const bool stalled = (int64_t)tile == wc.stall;
 
   if (threadIdx.x == 0) {
     mbar_init(&s_bar, 1);
@@ -232,14 +226,20 @@ __global__ void __launch_bounds__(kThreads) k_raster_fwd(
   // batch b's records land in s_rec (one copy in flight at a time: a batch
   // is converted into s_ev as soon as it lands, which frees s_rec for the
   // next one while the current batch is blended)
+  bool clipped = false;  // this thread's entry of the batch in flight named no Gaussian
   auto issue = [&](int b) {
+    if (stalled) return;
     const int64_t first = start + (int64_t)b * kBatch;
     const int64_t rem = end - first;
     const int m = rem < kBatch ? (int)rem : kBatch;
     if (threadIdx.x == 0) mbar_arrive_expect_tx(&s_bar, (uint32_t)(m * kRecBytes));
     if ((int)threadIdx.x < m) {
       uint32_t id = __ldg(&ids[first + threadIdx.x]);
-      if (id >= (uint32_t)geo.n) id = 0;  // never read outside the records
+      clipped = id >= (uint32_t)geo.n;
+      if (clipped) {  // never read outside the records
+        id = 0;
+        atomicOr(status, kStatusBounds);
+      }
       bulk_copy_g2s(&s_rec[threadIdx.x][0], rec_view + (size_t)id * GS_RECORD_FLOATS, kRecBytes,
                     &s_bar);
     }
@@ -251,58 +251,60 @@ __global__ void __launch_bounds__(kThreads) k_raster_fwd(
   const float2 one = f2(1.f), mone = f2(-1.f);
   float2 T = one, c0 = f2(0.f), c1 = f2(0.f), c2 = f2(0.f);
   uint32_t last0 = 0, last1 = 0;
-  // a pixel takes a Gaussian when log2(alpha) >= its threshold: log2(1/255)
-  // while it composites, +inf once it is done (or outside the image)
-  float thr0 = tp.in0 ? kLog2AlphaMin : kInf, thr1 = tp.in1 ? kLog2AlphaMin : kInf;
+  // a pixel takes a splat when zq <= its threshold: 0 while it composites,
+  // -inf once it is done (or outside the image)
+  float thr0 = tp.in0 ? 0.f : -kInf, thr1 = tp.in1 ? 0.f : -kInf;
   bool done = !(tp.in0 || tp.in1);
-  bool pending = nb > 0;  // batch b's copy is in flight
-  if (pending) issue(0);
+  bool pending = false;  // batch b's copy is in flight
+  if (nb > 0) {
+    issue(0);
+    pending = !stalled;
+  }
   int b = 0;
   for (; b < nb; ++b) {
     if (!__syncthreads_or(!done)) break;  // block vote; the previous batch is finished
-    if (!__syncthreads_and(mbar_wait_bounded(&s_bar, (uint32_t)(b & 1), status))) {
-      pending = false;  // a copy never landed: give up on the tile
-      break;
-    }
+    if (!__syncthreads_and(mbar_wait_bounded(&s_bar, (uint32_t)(b & 1), wc.limit_ns, status)))
+      break;  // a copy did not land in time: give up on the tile
     pending = false;
     const int64_t rem = cnt - (int64_t)b * kBatch;
     const int m = rem < kBatch ? (int)rem : kBatch;
-    if ((int)threadIdx.x < m)
-      s_mask[threadIdx.x] =
-          (uint8_t)prepare_record(&s_rec[threadIdx.x][0], &s_ev[threadIdx.x][0], tp.x0, tp.y0);
+    if ((int)threadIdx.x < m) {
+      const uint32_t mask = prepare_record(&s_rec[threadIdx.x][0], &s_ev[threadIdx.x][0], tp.x0,
+                                           tp.y0);
+      s_mask[threadIdx.x] = clipped ? 0u : (uint8_t)mask;
+    }
     __syncthreads();  // s_rec is free again
     if (b + 1 < nb) {
       issue(b + 1);
-      pending = true;
+      pending = !stalled;
     }
-    const int wc = warp_list(s_mask, s_list[warp], m);
+    const int wc_n = warp_list(s_mask, s_list[warp], m);
     const uint32_t pos0 = (uint32_t)(b * kBatch + 1);
-    for (int k = 0; k < wc; ++k) {
+    for (int k = 0; k < wc_n; ++k) {
       if ((k & 3) == 0 && __all_sync(0xffffffffu, done)) break;  // warp vote
       const int j = s_list[warp][k];
       const float2* e = &s_ev[j][0];
-      float2 dx, dy, adx, bdx;
-      const float2 p = eval_log2_alpha(e, pxc, pyc, dx, dy, adx, bdx);
-      bool ok0 = p.x >= thr0, ok1 = p.y >= thr1;
+      const float2 zq = eval_zq(e, pxc, pyc);
+      bool ok0 = zq.x <= thr0, ok1 = zq.y <= thr1;
       if (!(ok0 || ok1)) continue;
-      float2 a = make_float2(ok0 ? fminf(kAlphaMax, exp2f(p.x)) : 0.f,
-                             ok1 ? fminf(kAlphaMax, exp2f(p.y)) : 0.f);
+      float2 a = make_float2(ok0 ? fminf(kAlphaMax, alpha_raw_of(zq.x)) : 0.f,
+                             ok1 ? fminf(kAlphaMax, alpha_raw_of(zq.y)) : 0.f);
       float2 Tn = __fmul2_rn(T, __ffma2_rn(a, mone, one));  // T (1 - alpha)
       if (Tn.x < kTMin || Tn.y < kTMin) {
         // the pixel stops before this Gaussian: it takes no part in it
         if (Tn.x < kTMin) {
           a.x = 0.f;
           Tn.x = T.x;
-          thr0 = kInf;
+          thr0 = -kInf;
           ok0 = false;
         }
         if (Tn.y < kTMin) {
           a.y = 0.f;
           Tn.y = T.y;
-          thr1 = kInf;
+          thr1 = -kInf;
           ok1 = false;
         }
-        done = thr0 == kInf && thr1 == kInf;
+        done = thr0 == -kInf && thr1 == -kInf;
       }
       const float2 w = __fmul2_rn(a, T);
       c0 = __ffma2_rn(e[V_R], w, c0);
@@ -315,7 +317,7 @@ __global__ void __launch_bounds__(kThreads) k_raster_fwd(
     }
   }
   // a batch issued but not consumed must land before the block exits
-  if (pending) mbar_wait_bounded(&s_bar, (uint32_t)(b & 1), status);
+  if (pending) mbar_wait_bounded(&s_bar, (uint32_t)(b & 1), wc.limit_ns, status);
 
   const size_t hw = (size_t)geo.g.width * geo.g.height;
   float* img = image + (size_t)tp.view * 3 * hw;
@@ -372,7 +374,7 @@ __global__ void __launch_bounds__(kThreads) k_raster_bwd(
     const int64_t* __restrict__ ranges, RasterGeom geo, float bg0, float bg1, float bg2,
     const float* __restrict__ dL_dimage, const float* __restrict__ final_T,
     const uint32_t* __restrict__ n_contrib, float* __restrict__ grad2d,
-    uint32_t* __restrict__ status) {
+    uint32_t* __restrict__ status, WaitCfg wc) {
   __shared__ __align__(128) float s_rec[2][kBatch][GS_RECORD_FLOATS];
   __shared__ __align__(16) float s_acc[kBatch][GS_GRAD2D_FLOATS];
   __shared__ uint32_t s_id[2][kBatch];
@@ -387,10 +389,11 @@ __global__ void __launch_bounds__(kThreads) k_raster_bwd(
   const size_t pix0 = (size_t)tp.py * geo.g.width + tp.px;
   const size_t pix1 = pix0 + 4 * (size_t)geo.g.width;
   int64_t start, end;
-  tile_range(ranges, tile, geo.capacity, start, end);
+  tile_range(ranges, tile, geo.capacity, start, end, status);
   const float* rec_view = records + (size_t)tp.view * geo.n * GS_RECORD_FLOATS;
   float* g2_view = grad2d + (size_t)tp.view * geo.n * GS_GRAD2D_FLOATS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool stalled = (int64_t)tile == wc.stall;  // test hook, see k_raster_fwd
 
   // per-pixel state, pixel 0 in .x and pixel 1 in .y; an outside pixel has
   // no contributors and zero upstream gradient
@@ -437,8 +440,12 @@ __global__ void __launch_bounds__(kThreads) k_raster_bwd(
   if ((int64_t)maxc < used) used = maxc;
   const int nb = (int)((used + kBatch - 1) / kBatch);
 
-  // batches are consumed from the last (deepest) to the first
+  // batches are consumed from the last (deepest) to the first; iteration it
+  // uses buffer it & 1 and phase (it >> 1) & 1 of that buffer's barrier
+  int pend[2] = {-1, -1};  // iteration whose copy into the buffer is in flight
+  bool clipped[2] = {false, false};
   auto issue = [&](int it) {
+    if (stalled) return;
     const int b = nb - 1 - it;
     const int buf = it & 1;
     const int64_t first = start + (int64_t)b * kBatch;
@@ -447,11 +454,16 @@ __global__ void __launch_bounds__(kThreads) k_raster_bwd(
     if (threadIdx.x == 0) mbar_arrive_expect_tx(&s_bar[buf], (uint32_t)(m * kRecBytes));
     if ((int)threadIdx.x < m) {
       uint32_t id = __ldg(&ids[first + threadIdx.x]);
-      if (id >= (uint32_t)geo.n) id = 0;  // never read outside the records
+      clipped[buf] = id >= (uint32_t)geo.n;
+      if (clipped[buf]) {  // never read outside the records
+        id = 0;
+        atomicOr(status, kStatusBounds);
+      }
       s_id[buf][threadIdx.x] = id;
       bulk_copy_g2s(&s_rec[buf][threadIdx.x][0], rec_view + (size_t)id * GS_RECORD_FLOATS,
                     kRecBytes, &s_bar[buf]);
     }
+    pend[buf] = it;
   };
 
   const float pxc = (float)tp.px + 0.5f;
@@ -464,39 +476,45 @@ __global__ void __launch_bounds__(kThreads) k_raster_bwd(
     if (it + 1 < nb) issue(it + 1);
     const int64_t rem = used - (int64_t)b * kBatch;
     const int m = rem < kBatch ? (int)rem : kBatch;
-    if (!__syncthreads_and(mbar_wait_bounded(&s_bar[buf], (uint32_t)((it >> 1) & 1), status)))
-      break;
-    if ((int)threadIdx.x < m)
-      s_mask[threadIdx.x] = (uint8_t)prepare_record_s(&s_rec[buf][threadIdx.x][0], tp.x0, tp.y0);
+    if (!__syncthreads_and(
+            mbar_wait_bounded(&s_bar[buf], (uint32_t)((it >> 1) & 1), wc.limit_ns, status)))
+      break;  // a copy did not land in time: give up on the tile
+    pend[buf] = -1;
+    if ((int)threadIdx.x < m) {
+      float* r = &s_rec[buf][threadIdx.x][0];
+      const uint32_t mask = warp_block_mask(r[R_U], r[R_V], r[R_HX], r[R_HY], tp.x0, tp.y0);
+      s_mask[threadIdx.x] = clipped[buf] ? 0u : (uint8_t)mask;
+      r[R_OPAC] = 1.f / r[R_OPAC];  // d alpha / d opacity = alpha / o
+    }
     {
       float4* z = reinterpret_cast<float4*>(&s_acc[threadIdx.x][0]);
       z[0] = z[1] = z[2] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
-    const int wc = warp_list(s_mask, s_list[warp], m);
-    for (int k = wc - 1; k >= 0; --k) {
+    const int wc_n = warp_list(s_mask, s_list[warp], m);
+    for (int k = wc_n - 1; k >= 0; --k) {
       const int j = s_list[warp][k];
       const uint32_t pos = (uint32_t)(b * kBatch + j);
       const float* r = &s_rec[buf][j][0];
       float dx;
-      float2 dy;
-      const float2 p = eval_log2_alpha_s(r, pxc, pyc, dx, dy);
-      const bool ok0 = pos < nc0 && p.x >= kLog2AlphaMin;
-      const bool ok1 = pos < nc1 && p.y >= kLog2AlphaMin;
+      float2 dy, p1, p2;
+      const float2 zq = eval_zq_s(r, pxc, pyc, dx, dy, p1, p2);
+      const bool ok0 = pos < nc0 && zq.x <= 0.f;
+      const bool ok1 = pos < nc1 && zq.y <= 0.f;
       const uint32_t bal = __ballot_sync(0xffffffffu, ok0 || ok1);
       if (bal == 0u) continue;
       // a pixel that does not blend this Gaussian takes alpha = 0, which
       // leaves its T and colour-behind unchanged and adds nothing below
-      const float2 araw = make_float2(exp2f(p.x), exp2f(p.y));
+      const float2 araw = make_float2(alpha_raw_of(zq.x), alpha_raw_of(zq.y));
       const float2 a = make_float2(ok0 ? fminf(kAlphaMax, araw.x) : 0.f,
                                    ok1 ? fminf(kAlphaMax, araw.y) : 0.f);
       const float2 one_m = __fadd2_rn(f2(1.f), make_float2(-a.x, -a.y));
       const float2 inv = make_float2(ok0 ? 1.f / one_m.x : 1.f, ok1 ? 1.f / one_m.y : 1.f);
       T = __fmul2_rn(T, inv);  // transmittance in front of this Gaussian
       const float2 w = __fmul2_rn(a, T);
-      const float2 d0 = __fadd2_rn(f2(r[E_R]), make_float2(-acc0.x, -acc0.y));
-      const float2 d1 = __fadd2_rn(f2(r[E_G]), make_float2(-acc1.x, -acc1.y));
-      const float2 d2 = __fadd2_rn(f2(r[E_BL]), make_float2(-acc2.x, -acc2.y));
+      const float2 d0 = __fadd2_rn(f2(r[R_R]), make_float2(-acc0.x, -acc0.y));
+      const float2 d1 = __fadd2_rn(f2(r[R_G]), make_float2(-acc1.x, -acc1.y));
+      const float2 d2 = __fadd2_rn(f2(r[R_B]), make_float2(-acc2.x, -acc2.y));
       float2 s = __fmul2_rn(d0, g0);
       s = __ffma2_rn(d1, g1, s);
       s = __ffma2_rn(d2, g2, s);
@@ -509,11 +527,12 @@ __global__ void __launch_bounds__(kThreads) k_raster_bwd(
       float2 dpow = __fmul2_rn(a, dLda);
       dpow.x = araw.x < kAlphaMax ? dpow.x : 0.f;
       dpow.y = araw.y < kAlphaMax ? dpow.y : 0.f;
-      // -q/2 = ln2 (A dx^2 + B dx dy + C dy^2) with dx = px - u, dy = py - v
-      const float2 dpl = __fmul2_rn(dpow, f2(-kLn2));
-      const float adx2 = 2.f * r[E_A] * dx, bdx = r[E_B] * dx;
-      const float2 du = __fmul2_rn(dpl, __ffma2_rn(f2(r[E_B]), dy, f2(adx2)));
-      const float2 dv = __fmul2_rn(dpl, __ffma2_rn(f2(2.f * r[E_C]), dy, f2(bdx)));
+      // d alpha / d mean = alpha conic d = alpha 2 ln2 W^T (p1, p2)
+      const float2 dpl = __fmul2_rn(dpow, f2(kTwoLn2));
+      const float2 du =
+          __fmul2_rn(dpl, __ffma2_rn(f2(r[R_W1X]), p1, __fmul2_rn(f2(r[R_W2X]), p2)));
+      const float2 dv =
+          __fmul2_rn(dpl, __ffma2_rn(f2(r[R_W1Y]), p1, __fmul2_rn(f2(r[R_W2Y]), p2)));
       const float2 dyd = __fmul2_rn(dy, dpow);
       const float2 dy2d = __fmul2_rn(dy, dyd);
       const float2 wg0 = __fmul2_rn(w, g0), wg1 = __fmul2_rn(w, g1), wg2 = __fmul2_rn(w, g2);
@@ -522,10 +541,11 @@ __global__ void __launch_bounds__(kThreads) k_raster_bwd(
       float v[10];
       v[0] = du.x + du.y;
       v[1] = dv.x + dv.y;
+      // d alpha / d conic = -alpha/2 (dx^2, 2 dx dy, dy^2)
       v[2] = -0.5f * dx * dx * sd;
       v[3] = -dx * (dyd.x + dyd.y);
       v[4] = -0.5f * (dy2d.x + dy2d.y);
-      v[5] = r[E_IO] * sd;  // d alpha / d opacity = alpha / o
+      v[5] = r[R_OPAC] * sd;  // d alpha / d opacity = alpha / o (slot holds 1/o)
       v[6] = wg0.x + wg0.y;
       v[7] = wg1.x + wg1.y;
       v[8] = wg2.x + wg2.y;
@@ -559,6 +579,12 @@ __global__ void __launch_bounds__(kThreads) k_raster_bwd(
       }
     }
   }
+  // after a wait that gave up: copies still in flight land before the block
+  // exits
+#pragma unroll
+  for (int bf = 0; bf < 2; ++bf)
+    if (pend[bf] >= 0)
+      mbar_wait_bounded(&s_bar[bf], (uint32_t)((pend[bf] >> 1) & 1), wc.limit_ns, status);
 }
 
 }  // namespace
@@ -566,12 +592,14 @@ __global__ void __launch_bounds__(kThreads) k_raster_bwd(
 cudaError_t launch_raster_fwd(const float* records, const uint32_t* ids, const int64_t* ranges,
                               int64_t capacity, const Grid& g, int n_views, int n,
                               const float bg[3], float* image, float* final_T,
-                              uint32_t* n_contrib, uint32_t* status, cudaStream_t stream) {
+                              uint32_t* n_contrib, uint32_t* status, const WaitCfg& wc,
+                              cudaStream_t stream) {
   const int64_t tiles = (int64_t)g.tiles_per_view * n_views;
   if (tiles == 0) return cudaSuccess;
   RasterGeom geo{g, n, n > 0 ? capacity : 0};
   k_raster_fwd<<<(unsigned)tiles, kThreads, 0, stream>>>(records, ids, ranges, geo, bg[0], bg[1],
-                                                         bg[2], image, final_T, n_contrib, status);
+                                                         bg[2], image, final_T, n_contrib, status,
+                                                         wc);
   return cudaGetLastError();
 }
 
@@ -579,13 +607,13 @@ cudaError_t launch_raster_bwd(const float* records, const uint32_t* ids, const i
                               int64_t capacity, const Grid& g, int n_views, int n,
                               const float bg[3], const float* dL_dimage, const float* final_T,
                               const uint32_t* n_contrib, float* grad2d, uint32_t* status,
-                              cudaStream_t stream) {
+                              const WaitCfg& wc, cudaStream_t stream) {
   const int64_t tiles = (int64_t)g.tiles_per_view * n_views;
   if (tiles == 0) return cudaSuccess;
   RasterGeom geo{g, n, n > 0 ? capacity : 0};
   k_raster_bwd<<<(unsigned)tiles, kThreads, 0, stream>>>(records, ids, ranges, geo, bg[0], bg[1],
                                                          bg[2], dL_dimage, final_T, n_contrib,
-                                                         grad2d, status);
+                                                         grad2d, status, wc);
   return cudaGetLastError();
 }
 

@@ -191,7 +191,7 @@ class Splatter:
     def project(self):
         if self.sh_bits is not None:
             api.gs_sh_dequantize(self.sh_q, self.sh, self.stream)
-        api.gs_project(self.c_params, self.cams, self.V, self.c_proj, self.stream)
+        api.gs_project(self.c_params, self.cams, self.V, self.c_proj, self.ws, self.stream)
 
     def bin_sort(self):
         api.gs_bin_sort(self.c_proj, self.cams, self.V, self.n, self.sort_mode, self.c_bins,
@@ -199,12 +199,12 @@ class Splatter:
 
     def rasterize_fwd(self):
         api.gs_rasterize_fwd(self.c_proj, self.c_bins, self.cams, self.V, self.n, self.bg,
-                             self.image, self.final_T, self.n_contrib, self.stream)
+                             self.image, self.final_T, self.n_contrib, self.ws, self.stream)
 
     def rasterize_bwd(self, dL_dimage: torch.Tensor, with_params: bool = True):
         api.gs_rasterize_bwd(self.c_params, self.c_proj, self.c_bins, self.cams, self.V, self.bg,
                              dL_dimage, self.final_T, self.n_contrib, self.grad2d,
-                             self.c_grads if with_params else None, self.stream)
+                             self.c_grads if with_params else None, self.ws, self.stream)
 
     def project_bwd(self):
         api.gs_project_bwd(self.c_params, self.cams, self.V, self.radii, self.grad2d,
@@ -387,6 +387,35 @@ class Splatter:
             if adam:
                 self.adam_step()
         comp.wait_event(downloaded)  # the last image is on the host when comp is done
+
+    def render_to_host(self, image_host) -> None:
+        """Forward renders delivered to host memory, copies overlapped with
+        compute: step k renders and downloads the image into ``image_host[k]``
+        (pinned, [V][3][H][W] float32) on a second stream while step k + 1
+        projects and sorts; step k + 1's rasterisation waits for that download.
+        Everything is enqueued; the caller synchronises. ``self.stream`` must
+        be a created stream (see train_from_host)."""
+        comp = self.stream
+        if comp is None:
+            raise ValueError("render_to_host needs Splatter(stream=...) on a created stream")
+        if getattr(self, "_copy_stream", None) is None:
+            self._copy_stream = torch.cuda.Stream(device=self.device)
+        cs = self._copy_stream
+        rendered = torch.cuda.Event()
+        downloaded = torch.cuda.Event()
+        cs.wait_stream(comp)
+        for k in range(len(image_host)):
+            self.project()
+            self.bin_sort()
+            if k > 0:
+                comp.wait_event(downloaded)
+            self.rasterize_fwd()
+            rendered.record(comp)
+            cs.wait_event(rendered)
+            with torch.cuda.stream(cs):
+                image_host[k].copy_(self.image, non_blocking=True)
+                downloaded.record(cs)
+        comp.wait_event(downloaded)
 
     def densify_and_prune(self, grad_threshold: float = 0.0002, scale_split: float = 0.05,
                           min_opacity: float = 0.005, max_scale: float = 1.0,

@@ -52,6 +52,7 @@ __all__ = [
     "make_scene",
     "make_upstream_grad",
     "make_projected_2d",
+    "make_isolated_scene",
 ]
 
 
@@ -296,3 +297,39 @@ def make_image_pair(n_views: int, height: int, width: int, seed: int = 3,
     tie = rng.random(img.shape) < tie_frac
     img[tie] = tgt[tie]
     return img, tgt
+
+
+def make_isolated_scene(side: int = 16, spacing: int = 128, seed: int = 9,
+                        f: float = 600.0, depth: float = 8.0) -> Scene:
+    """side x side Gaussians, one per spacing x spacing pixel cell of a single
+    view (camera at the origin looking down +z), far enough apart that no tile
+    holds two of them, so every pixel sees at most one splat. Log-scales
+    U(-5, -2.3) per axis (2D anisotropy up to ~15), uniform rotations, opacity
+    logits U(-5, 7) (so both the alpha clamp at 0.99 and splats too faint to
+    count occur), a random sub-pixel offset of each mean, and an image of
+    side * spacing pixels squared (means far from the origin, where a float
+    keeps only ~1e-4 px of the mean). Degree-0 colour, DC U(0, 1)."""
+    rng = np.random.default_rng(seed)
+    n = side * side
+    width = height = side * spacing
+    cx = cy = width / 2.0
+    gx, gy = np.meshgrid(np.arange(side), np.arange(side), indexing="xy")
+    px = (gx.ravel() + 0.5) * spacing + rng.uniform(-0.5, 0.5, n)
+    py = (gy.ravel() + 0.5) * spacing + rng.uniform(-0.5, 0.5, n)
+    m3 = np.stack([(px - cx) / f * depth, (py - cy) / f * depth, np.full(n, depth)], 1)
+    s3 = rng.uniform(-5.0, -2.3, size=(n, 3))
+    q = rng.normal(0.0, 1.0, size=(n, 4))
+    q /= np.linalg.norm(q, axis=1, keepdims=True)
+    logit = rng.uniform(-5.0, 7.0, size=n)
+    sh = np.zeros((n, 1, 3))
+    sh[:, 0, :] = rng.uniform(0.0, 1.0, size=(n, 3))
+    means = np.zeros((n, 4), np.float32)
+    means[:, :3] = m3
+    log_scales = np.zeros((n, 4), np.float32)
+    log_scales[:, :3] = s3
+    vm = np.concatenate([np.eye(3), np.zeros((3, 1))], axis=1)
+    return Scene(name="isolated", means=means, log_scales=log_scales,
+                 quats=q.astype(np.float32), opacity_logit=logit.astype(np.float32),
+                 sh=sh.astype(np.float32), sh_degree=0,
+                 cameras=[_camera(vm, (0.0, 0.0, 0.0), f, width, height)],
+                 background=np.zeros(3, np.float32))

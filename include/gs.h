@@ -21,10 +21,14 @@
  *    without synchronising, except gs_get_status.
  *  - Argument errors are detected on the host before anything is enqueued and
  *    returned at once (GS_ERR_INVALID_ARG, GS_ERR_OVERFLOW). A failed launch
- *    returns GS_ERR_CUDA. Conditions only the device can see (pair capacity
- *    exceeded, a bounded wait that gave up, a Gaussian culled for non-finite
- *    values) are OR-ed into the status word at the start of the workspace and
- *    read back by gs_get_status.
+ *    returns GS_ERR_CUDA. Conditions only the device can see are OR-ed into
+ *    the status word at the start of a workspace (the GS_STATUS_BIT_* bits
+ *    below) and read back by gs_get_status: pair capacity exceeded, a
+ *    bounded wait that gave up, an index or range out of bounds (clipped,
+ *    never dereferenced), a Gaussian culled for non-finite values. The calls
+ *    with a device wait or an index to check (gs_project, gs_bin_sort,
+ *    gs_rasterize_fwd, gs_rasterize_bwd) take that workspace; the
+ *    gs_bin_sort workspace serves all of them.
  *  - Pixel (x, y) has its centre at (x + 0.5, y + 0.5); tiles are 16 x 16
  *    pixels; tile index within a view is ty * tiles_x + tx, and the global
  *    tile index of view v is v * tiles_per_view + tile.
@@ -40,12 +44,18 @@
 extern "C" {
 #endif
 
-#define GS_ABI_VERSION 1
+#define GS_ABI_VERSION 2
 #define GS_TILE 16            /* tile edge in pixels */
 #define GS_MAX_VIEWS 32       /* views per call */
-#define GS_RECORD_FLOATS 12   /* floats per projected record */
+#define GS_RECORD_FLOATS 16   /* floats per projected record */
 #define GS_GRAD2D_FLOATS 12   /* floats per screen-space gradient record */
 #define GS_MAX_PAIR_CAPACITY ((int64_t)1 << 31) /* pair positions are 32-bit */
+
+/* Bits of the device status word (the first 4 bytes of a workspace). */
+#define GS_STATUS_BIT_CAPACITY 1u   /* more pairs than pair_capacity: nothing emitted */
+#define GS_STATUS_BIT_TIMEOUT 2u    /* a bounded device-side wait gave up */
+#define GS_STATUS_BIT_BOUNDS 4u     /* an index or range out of bounds was clipped */
+#define GS_STATUS_BIT_NONFINITE 8u  /* a Gaussian with a non-finite value was culled */
 
 typedef enum gs_status {
   GS_OK = 0,
@@ -113,15 +123,31 @@ typedef struct gs_grads {
 } gs_grads;
 
 /* Output of gs_project, per view v and Gaussian i (record index v*n + i):
- * records [n_views][n][12] floats, 16-byte aligned (what the rasteriser reads):
- *   0 u        1 v          pixel coordinates of the mean
- *   2 conic_a  3 conic_b    4 conic_c   inverse 2D covariance [[a, b], [b, c]]
- *   5 opacity  6 r  7 g  8 b            activated opacity, colour
- *   9 hx      10 hy         half-widths of a box around the ellipse where
- *                           alpha >= 1/255 (q <= Q = 2 ln(255 o)): sqrt(Qp
- *                           cov_xx) + 0.01 and sqrt(Qp cov_yy) + 0.01 with
- *                           Qp = Q + 0.002 |Q| + 1e-4; -1 when Qp <= 0
- *  11 zero
+ * records [n_views][n][16] floats, 16-byte aligned (what the rasteriser reads).
+ * The 2D Gaussian (mean (u, v), conic = inverse 2D covariance, opacity o) is
+ * stored in the form the rasteriser evaluates, every field computed in double
+ * precision and rounded to float once:
+ *   0 uh      1 vh       u and v rounded to float
+ *   2 w1x     3 w1y      rows of the 2x2 matrix W = diag(k1, k2) E^T, E the
+ *   5 w2x     6 w2y      unit eigenvectors of the 2D covariance (largest
+ *                        eigenvalue lambda1 first), k_i = sqrt(log2(e) / (2
+ *                        lambda_i)); W^T W = (log2(e) / 2) conic
+ *   4 c1      7 c2       c_i = -(w_i . (u - uh, v - vh)) with the float rows:
+ *                        the part of the mean below float precision
+ *   8 nlo                -log2(255 o)
+ *   9 r  10 g  11 b      colour
+ *  12 hx     13 hy       half-widths of a box around the ellipse where
+ *                        alpha >= 1/255 (q <= Q = 2 ln(255 o)): sqrt(Qp
+ *                        cov_xx) + 0.01 and sqrt(Qp cov_yy) + 0.01 with
+ *                        Qp = Q + 0.002 |Q| + 1e-4; -1 when Qp <= 0
+ *  14 o                  activated opacity
+ *  15 zero
+ * For the pixel centre P and d = P - (uh, vh), p_i = w_i . d + c_i and
+ * zq = p1^2 + p2^2 + nlo equal (log2(e)/2) q - log2(255 o) with
+ * q = (P - mean)^T conic (P - mean): alpha_raw = o exp(-q/2) = 2^-zq / 255,
+ * and alpha_raw >= 1/255 exactly when zq <= 0. (The eigen form is a sum of
+ * squares, so it keeps its relative accuracy for elongated splats, where the
+ * conic form a dx^2 + 2 b dx dy + c dy^2 loses it to cancellation.)
  * bins [n_views][n][4] floats, 16-byte aligned (what the binning reads):
  *   0 depth key: camera-space z as the float fma chain
  *     fma(W20, x, fma(W21, y, fma(W22, z, t2))) of the float inputs
@@ -213,9 +239,13 @@ gs_status gs_bin_sort_plan(int64_t n, int32_t n_views, const gs_camera* cams,
  * colour (a non-finite SH coefficient), or a zero quaternion, is culled in
  * every view and its depth key marked; gs_bin_sort on those records raises
  * GS_ERR_NONFINITE in its status word (the rest of the frame is unaffected).
- * Writes out->records and out->radii for all n_views * n records. */
+ * Writes out->records, out->bins and out->radii for all n_views * n records.
+ * `ws` is a workspace (e.g. gs_bin_sort's) whose status word receives
+ * GS_STATUS_BIT_TIMEOUT if the staging of a block's SH coefficients into
+ * shared memory did not complete in time (the block then reads them from
+ * global memory, so the output is still exact). */
 gs_status gs_project(const gs_params* params, const gs_camera* cams, int32_t n_views,
-                     gs_projected* out, void* stream);
+                     gs_projected* out, void* ws, void* stream);
 
 /* Tile binning with depth sort (pwwt.cn sec. 3.3 steps 1-2 and 4.3 tiles;
  * lshu.cn sec. 3.2 `assign_to_tiles` and `sort_by_depth!`). Every Gaussian
@@ -244,16 +274,21 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
  * the same inputs and outputs as gs_bin_sort but no workspace: its scratch is
  * a fixed array of GS_NOALLOC_SCRATCH_BYTES inside the library, which every
  * GPU that uses this entry point holds from its first call until the process
- * exits. The first call on a device looks up the array's device address
- * (with that device current); make that first call before any stream
- * capture. Requests whose gs_workspace_size exceeds GS_NOALLOC_SCRATCH_BYTES
+ * exits (with eager module loading, CUDA_MODULE_LOADING=EAGER, every context
+ * that loads the library holds it, whether or not it calls this entry
+ * point). Each call looks up the array's device address on the current
+ * device (cudaGetSymbolAddress, a host-side query), so the address stays
+ * right after a cudaDeviceReset; make the first call on a device before any
+ * stream capture. Requests whose gs_workspace_size exceeds GS_NOALLOC_SCRATCH_BYTES
  * are rejected with GS_ERR_INVALID_ARG before anything is enqueued. All calls
  * share the one array: calls whose work overlaps on the GPU (for example on
  * two streams) race and corrupt each other's results; serialise them.
  * Each call starts with a cleared status word; if `device_status` (a device
  * int32, may be NULL) is given, the call's device-side status bits (1 pair
  * capacity exceeded, 2 a bounded wait gave up, 4 an index out of range) are
- * copied there at the end, in stream order. */
+ * copied there at the end, in stream order: the GS_STATUS_BIT_* bits (1 pair
+ * capacity exceeded, 2 a bounded wait gave up, 4 an index or range out of
+ * bounds was clipped, 8 a Gaussian culled for non-finite values was met). */
 gs_status gs_bin_sort_noalloc(const gs_projected* proj, const gs_camera* cams, int32_t n_views,
                               int64_t n, int32_t sort_mode, gs_binned* out,
                               int32_t* device_status, void* stream);
@@ -269,11 +304,19 @@ gs_status gs_bin_sort_noalloc(const gs_projected* proj, const gs_camera* cams, i
  *   final_T   float [n_views][H][W]  transmittance after the last contributor
  *   n_contrib uint32 [n_views][H][W] 1 + position in the tile's list of the
  *             last contributing Gaussian (0 if none)
- * `bg` is a host pointer to 3 floats. */
+ * `bg` is a host pointer to 3 floats. The test alpha_raw >= 1/255 is taken as
+ * zq <= 0 on the record's evaluation form (see gs_projected) and alpha_raw
+ * as 2^-zq / 255 with the SFU exp2. `ws` (device, 256-byte aligned, its
+ * status word zeroed once, e.g. the gs_bin_sort workspace) receives
+ * GS_STATUS_BIT_BOUNDS for a list entry naming a Gaussian >= n or a tile
+ * range outside the ids buffer (the entry reads record 0 and reaches no
+ * pixel; the range renders as empty), and GS_STATUS_BIT_TIMEOUT if a record
+ * batch's copy into shared memory did not complete in time (that tile's
+ * pixels keep what they had composited). */
 gs_status gs_rasterize_fwd(const gs_projected* proj, const gs_binned* bins,
                            const gs_camera* cams, int32_t n_views, int64_t n,
                            const float* bg, float* image, float* final_T,
-                           uint32_t* n_contrib, void* stream);
+                           uint32_t* n_contrib, void* ws, void* stream);
 
 /* Backward of gs_rasterize_fwd and gs_project (lshu.cn sec. 1
  * "differentiable rasterisation"). Given dL/dimage [n_views][3][H][W] and the
@@ -286,12 +329,14 @@ gs_status gs_rasterize_fwd(const gs_projected* proj, const gs_binned* bins,
  * (0 and 1 together are the view's plain view-space gradient), then the
  * gradients of the raw parameters summed over views into *grads
  * (overwritten; see gs_project_bwd). grad2d is overwritten. With
- * grads == NULL only grad2d is computed. */
+ * grads == NULL only grad2d is computed. `ws` as for gs_rasterize_fwd (the
+ * same conditions are reported; a tile whose batch copy timed out adds
+ * nothing further to grad2d). */
 gs_status gs_rasterize_bwd(const gs_params* params, const gs_projected* proj,
                            const gs_binned* bins, const gs_camera* cams, int32_t n_views,
                            const float* bg, const float* dL_dimage, const float* final_T,
                            const uint32_t* n_contrib, float* grad2d, gs_grads* grads,
-                           void* stream);
+                           void* ws, void* stream);
 
 /* Projection backward alone (the second half of gs_rasterize_bwd): the
  * gradients of the raw parameters from the screen-space gradients grad2d
@@ -435,6 +480,26 @@ gs_status gs_adam_step_sh_quant(const gs_sh_quant* q, const float* grad_sh, uint
                                 uint16_t* exp_avg_sq, float lr, float beta1, float beta2,
                                 float eps, int64_t step, int32_t rounding, uint64_t seed,
                                 void* stream);
+
+/* Test hook for the timeout path (the pages have no counterpart). Every
+ * device-side wait of the library (an mbarrier phase in gs_project and the
+ * rasteriser, a look-back flag in gs_bin_sort's emission) gives up after a
+ * time limit, sets GS_STATUS_BIT_TIMEOUT and lets its kernel finish. This
+ * call makes one such wait run out on purpose, without faulting anything:
+ *   GS_STALL_RASTER_FWD / GS_STALL_RASTER_BWD  global tile `index` of the
+ *     next rasteriser calls issues no record copies and waits in vain for
+ *     its first batch (its pixels keep the background / add no gradient);
+ *   GS_STALL_EMIT_LOOKBACK  emission block `index` of gs_bin_sort's
+ *     look-back scan (GS_SORT_FULL64, and GS_SORT_PRESORT on grids that
+ *     sort by tile id) never publishes its prefix, so its successors' waits
+ *     run out;
+ *   GS_STALL_NONE  back to normal.
+ * wait_limit_s (> 0) replaces the default limit of 2 s for every wait while
+ * the setting holds; 0 keeps the default. Process-wide, not thread-safe
+ * against concurrent calls of the library; meant for tests only. */
+enum { GS_STALL_NONE = 0, GS_STALL_EMIT_LOOKBACK = 1, GS_STALL_RASTER_FWD = 2,
+       GS_STALL_RASTER_BWD = 3 };
+gs_status gs_debug_stall(int32_t site, int64_t index, double wait_limit_s);
 
 /* Synchronise `stream`, return the status word accumulated in workspace `ws`
  * by device-side checks since the last call, and clear it. Several conditions

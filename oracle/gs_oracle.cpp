@@ -413,16 +413,37 @@ void orc_tile_lists(int n_views, int64_t n, const int32_t* rects, const float* k
 //   keys[V][n] float32 depth keys; rects[V][n][4]; dims[V][2] = width, height
 //   pix[P][3] = (view, x, y); bg[3]
 //   win_alpha, win_T: relative windows around 1/255 and 1e-4 for flagging
+//   alpha_err[V][n][2] (may be null): for comparing with an implementation
+//     whose alpha of Gaussian i at a pixel with quadratic form q is known to
+//     lie within relative e = alpha_err[i][0] + alpha_err[i][1] q of the
+//     exact one. Then an evaluation is also flagged when its alpha lies within
+//     that relative distance of 1/255, and the trial transmittance when it
+//     lies within the bound rho on the relative error such an implementation's
+//     transmittance can carry: every contributor j multiplies it by (1 - a_j),
+//     adding a_j / (1 - a_j) * e_j to rho (for a clamped alpha the
+//     float32 rounding of 0.99, |0.99f - 0.99| / 0.01) plus 2^-23 for the
+//     float product and difference, and a flagged evaluation (which that
+//     implementation may take or skip) adds a_j / (1 - a_j).
 // Outputs per pixel: color[P][3] (background included), T_final[P],
 //   n_contrib[P] = 1 + list position of the last Gaussian that contributed
-//   (0 if none), flags[P] (bit 0: some alpha within win_alpha of 1/255, bit 1:
-//   some trial transmittance within win_T of 1e-4), n_exp[P] = number of
+//   (0 if none), flags[P] (bit 0: some alpha flagged near 1/255, bit 1: some
+//   trial transmittance flagged near 1e-4), n_exp[P] = number of
 //   Gaussians with alpha >= 1/255 reached before the stop, n_used[P] = number
-//   of contributors, sig[P] = hash of the contributors and their clamp states.
+//   of contributors, sig[P] = hash of the contributors and their clamp states,
+//   flag_dev[P] (may be null) = the sum over flagged evaluations of the most
+//   they can move a colour channel, in units of the largest colour magnitude
+//   c_max in play: a skip taken the other way at k changes the colour by
+//   T_k a_k (c_k - B_k) with B_k the colour behind k, at most 2 T_k a_k c_max,
+//   and a stop taken the other way at k by at most 2 T_k c_max (everything
+//   from k on); entered as 2.02 T_k a_k and 2.02 T_k (a 1 % margin for the
+//   transmittance difference the flips themselves make); flag_T[P] (may be
+//   null) = the sum over flagged evaluations of the most they can move the
+//   final transmittance: T_k a_k / (1 - a_k) for a skip, T_k for a stop.
 void orc_render(int n_views, int64_t n, const double* g2d, const float* keys, const int32_t* rects,
                 const int32_t* dims, int64_t P, const int32_t* pix, const double* bg,
-                double win_alpha, double win_T, double* color, double* T_final, int32_t* n_contrib,
-                int32_t* flags, int64_t* n_exp, int32_t* n_used, uint64_t* sig) {
+                double win_alpha, double win_T, const double* alpha_err, double* color,
+                double* T_final, int32_t* n_contrib, int32_t* flags, int64_t* n_exp,
+                int32_t* n_used, uint64_t* sig, double* flag_dev, double* flag_T) {
   std::vector<int32_t> tx(n_views), ty(n_views);
   for (int v = 0; v < n_views; ++v) {
     tx[v] = (dims[2 * v] + kTile - 1) / kTile;
@@ -457,23 +478,50 @@ void orc_render(int n_views, int64_t n, const double* g2d, const float* keys, co
     int v = pix[3 * p], x = pix[3 * p + 1], y = pix[3 * p + 2];
     int64_t s = tile_req_of_pix[p];
     const double* gv = g2d + (size_t)v * n * 9;
+    const double* ev = alpha_err ? alpha_err + (size_t)v * n * 2 : nullptr;
     double px = x + 0.5, py = y + 0.5;
     double T = 1.0, c[3] = {0, 0, 0};
     int32_t last = 0, fl = 0, used = 0;
     int64_t ne = 0;
     uint64_t h = 1469598103934665603ULL;
+    double rho = 0.0, dev = 0.0, dT = 0.0;
+    const double clamp_err = std::fabs((double)0.99f - kAlphaMax) / (1.0 - kAlphaMax);
+    const double u23 = std::ldexp(1.0, -23);
     for (int64_t k = offs[s]; k < offs[s + 1]; ++k) {
       const double* g = gv + (size_t)ids[k] * 9;
       double d0 = px - g[0], d1 = py - g[1];
       double q = g[2] * d0 * d0 + 2.0 * g[3] * d0 * d1 + g[4] * d1 * d1;
       double araw = g[5] * std::exp(-0.5 * q);
       double a = std::min(kAlphaMax, araw);
-      if (std::fabs(a / kAlphaMin - 1.0) < win_alpha) fl |= 1;
+      const double e = ev ? ev[2 * (size_t)ids[k]] + ev[2 * (size_t)ids[k] + 1] * q : 0.0;
+      bool aflag = std::fabs(a / kAlphaMin - 1.0) < win_alpha;
+      if (ev && std::fabs(araw / kAlphaMin - 1.0) < e) aflag = true;
+      if (aflag) {
+        fl |= 1;
+        const double an = std::max(a, kAlphaMin);
+        dev += 2.02 * T * an;
+        dT += T * an / (1.0 - an);
+        rho += an / (1.0 - an);
+      }
       if (a < kAlphaMin) continue;
       ++ne;
       double Tn = T * (1.0 - a);
-      if (std::fabs(Tn / kTMin - 1.0) < win_T) fl |= 2;
+      // relative error bound of an implementation's trial transmittance
+      double step = u23;
+      if (ev) {
+        if (std::fabs(araw / kAlphaMax - 1.0) < e) step += kAlphaMax * e / (1.0 - kAlphaMax);
+        else if (araw >= kAlphaMax) step += clamp_err;
+        else step += a * e / (1.0 - a);
+      }
+      bool tflag = std::fabs(Tn / kTMin - 1.0) < win_T;
+      if (ev && std::fabs(Tn / kTMin - 1.0) < rho + step) tflag = true;
+      if (tflag) {
+        fl |= 2;
+        dev += 2.02 * T;
+        dT += T;
+      }
       if (Tn < kTMin) break;
+      rho += step;
       for (int ch = 0; ch < 3; ++ch) c[ch] += g[6 + ch] * a * T;
       T = Tn;
       last = (int32_t)(k - offs[s] + 1);
@@ -487,6 +535,8 @@ void orc_render(int n_views, int64_t n, const double* g2d, const float* keys, co
     n_exp[p] = ne;
     n_used[p] = used;
     sig[p] = h;
+    if (flag_dev) flag_dev[p] = dev;
+    if (flag_T) flag_T[p] = dT;
   }
 }
 

@@ -41,8 +41,8 @@ def lib():
         L.orc_tile_lists.argtypes = [ctypes.c_int, ctypes.c_int64, _I32, _F, _I32, _I32,
                                      ctypes.c_int64, _I32, _I64, _I32]
         L.orc_render.argtypes = [ctypes.c_int, ctypes.c_int64, _D, _F, _I32, _I32, ctypes.c_int64,
-                                 _I32, _D, ctypes.c_double, ctypes.c_double, _D, _D, _I32, _I32,
-                                 _I64, _I32, _U64]
+                                 _I32, _D, ctypes.c_double, ctypes.c_double, _D, _D, _D, _I32,
+                                 _I32, _I64, _I32, _U64, _D, _D]
         L.orc_render_bwd.argtypes = [ctypes.c_int, ctypes.c_int64, _D, _F, _I32, _I32,
                                      ctypes.c_int64, _I32, _D, _D, _D]
         L.orc_project_bwd.argtypes = [ctypes.c_int64, _D, _D, _D, _D, _D, ctypes.c_int,
@@ -152,8 +152,17 @@ def tile_lists(rects: np.ndarray, keys: np.ndarray, tiles_xy: Sequence, requests
 
 
 def render(projs: Sequence[dict], cams, bg, pixels: np.ndarray,
-           win_alpha: float = 0.0, win_T: float = 0.0) -> Dict[str, np.ndarray]:
-    """Render the listed pixels ``[(view, x, y)]`` from projected Gaussians."""
+           win_alpha: float = 0.0, win_T: float = 0.0,
+           alpha_err: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
+    """Render the listed pixels ``[(view, x, y)]`` from projected Gaussians.
+
+    ``win_alpha`` / ``win_T`` flag evaluations whose alpha (trial
+    transmittance) lies within that relative distance of 1/255 (1e-4);
+    ``alpha_err`` [V, n, 2], if given, bounds the relative alpha error of the
+    implementation being compared by alpha_err[..., 0] + alpha_err[..., 1] q
+    (q the pixel's quadratic form), which flags by that bound and by the
+    transmittance error bound it implies (see orc_render); ``flag_dev`` /
+    ``flag_T`` receive what the flagged decisions can change."""
     g2d, keys, rects = _stack_views(projs)
     V, n = keys.shape
     pix = np.ascontiguousarray(pixels, np.int32).reshape(-1, 3)
@@ -161,12 +170,17 @@ def render(projs: Sequence[dict], cams, bg, pixels: np.ndarray,
     color = np.zeros((P, 3)); T = np.zeros(P); nc = np.zeros(P, np.int32)
     flags = np.zeros(P, np.int32); nexp = np.zeros(P, np.int64); used = np.zeros(P, np.int32)
     sig = np.zeros(P, np.uint64)
+    fdev = np.zeros(P); fT = np.zeros(P)
     bgd = _f64(bg)
+    ae = None if alpha_err is None else np.ascontiguousarray(alpha_err,
+                                                             np.float64).reshape(V, n, 2)
     lib().orc_render(V, n, _p(g2d, _D), _p(keys, _F), _p(rects, _I32), _p(_dims(cams), _I32),
                      P, _p(pix, _I32), _p(bgd, _D), float(win_alpha), float(win_T),
+                     None if ae is None else _p(ae, _D),
                      _p(color, _D), _p(T, _D), _p(nc, _I32), _p(flags, _I32), _p(nexp, _I64),
-                     _p(used, _I32), _p(sig, _U64))
-    return dict(color=color, T=T, n_contrib=nc, flags=flags, n_exp=nexp, n_used=used, sig=sig)
+                     _p(used, _I32), _p(sig, _U64), _p(fdev, _D), _p(fT, _D))
+    return dict(color=color, T=T, n_contrib=nc, flags=flags, n_exp=nexp, n_used=used, sig=sig,
+                flag_dev=fdev, flag_T=fT)
 
 
 def render_bwd(projs: Sequence[dict], cams, bg, pixels: np.ndarray, dL_dC: np.ndarray) -> np.ndarray:

@@ -43,10 +43,21 @@ int main(void) {
   p.sh_degree = 4; /* degrees stop at 3 */
   gs_projected out;
   memset(&out, 0, sizeof out);
-  CHECK(gs_project(&p, &cam, 1, &out, NULL) == GS_ERR_INVALID_ARG);
+  /* an aligned address that is never dereferenced: every call below returns
+   * before anything is enqueued */
+  void* ws = (void*)(uintptr_t)4096;
+  CHECK(gs_project(&p, &cam, 1, &out, ws, NULL) == GS_ERR_INVALID_ARG);
   p.sh_degree = 0;
   p.n = (int64_t)1 << 31;
-  CHECK(gs_project(&p, &cam, 1, &out, NULL) == GS_ERR_OVERFLOW);
+  CHECK(gs_project(&p, &cam, 1, &out, ws, NULL) == GS_ERR_OVERFLOW);
+  CHECK(gs_project(&p, &cam, 1, &out, NULL, NULL) == GS_ERR_INVALID_ARG); /* no status word */
+
+  CHECK(gs_debug_stall(GS_STALL_RASTER_FWD, -1, 0.0) == GS_ERR_INVALID_ARG);
+  CHECK(gs_debug_stall(7, 0, 0.0) == GS_ERR_INVALID_ARG);
+  CHECK(gs_debug_stall(GS_STALL_NONE, 0, -1.0) == GS_ERR_INVALID_ARG);
+  CHECK(gs_debug_stall(GS_STALL_NONE, 0, 0.0) == GS_OK);
+  CHECK((GS_STATUS_BIT_CAPACITY | GS_STATUS_BIT_TIMEOUT | GS_STATUS_BIT_BOUNDS |
+         GS_STATUS_BIT_NONFINITE) == 15u);
 
   CHECK(gs_l1_dssim_workspace_size(2) == 2 * 16 + 16);
   CHECK(gs_l1_dssim(NULL, NULL, 0, 8, 8, 0.2f, NULL, NULL, NULL, 0, NULL) == GS_OK);

@@ -3,10 +3,30 @@ the same seeded scene and compare them under the stated tolerances.
 
 Tolerances (the task's acceptance criteria):
   * binning: per-tile sorted id lists bit-exact;
-  * rendered colours: max |d| <= 2e-3 and mean |d| <= 1e-5, over pixels whose
-    float64 decisions are not within the flag windows of a threshold
-    (alpha vs 1/255, trial transmittance vs 1e-4); flagged pixels are counted;
+  * rendered colours: max |d| <= 2e-3 and mean |d| <= 1e-5, n_contrib exact
+    and T within 1e-3 relative over pixels none of whose float64 decisions
+    lies within the kernel's error bound of its threshold (alpha vs 1/255,
+    trial transmittance vs 1e-4); a flagged pixel is held to what its flagged
+    decisions can change (the oracle's flag_dev / flag_T);
   * gradients, densify statistics and Adam state: relative L2 <= 1e-3.
+
+The kernel's alpha error bound (alpha_error_bound) is derived from the
+rasteriser's arithmetic on the record's evaluation form: with u = 2^-24,
+d = P - (uh, vh) and p_i = fl(w_iy dy + fl(w_ix dx + c_i)), each p_i is off
+by at most u (4 |w_ix dx| + 3 |w_iy dy| + 3 |c_i|) -- the rounding of dx, of
+the float row w_i, and of the two fmas -- and zq = fl(p1^2 + fl(p2^2 + nlo))
+by at most u (|nlo| + |t| + |zq|) + 2 |p1| dp1 + 2 |p2| dp2 with t the inner
+fma. Where a splat counts, zq <= 0 and q' = p1^2 + p2^2 <= Q' = log2(255 o),
+so |nlo|, |t| and |zq| are at most Q'; writing x = k1 |d . e1|, y = k2
+|d . e2| (q' = x^2 + y^2, |d| <= x / k1 + y / k2, k1 / k2 = 1 / sqrt(kappa),
+kappa = lambda1 / lambda2 of the 2D covariance), 2 |p1| dp1 + 2 |p2| dp2 <=
+8 u (q' + x y (sqrt(kappa) + 1 / sqrt(kappa))) <= 8 u q' (1 + (sqrt(kappa) +
+1 / sqrt(kappa)) / 2). So |zq - zq_exact| <= dz(q') = u (3 Q' + 1 + 8 q' (1 +
+(sqrt(kappa) + 1 / sqrt(kappa)) / 2)) (the 1 covers the c_i terms, at most
+~1e-4 in size), with q' = (log2(e) / 2) q, and alpha_raw = 2^-zq / 255
+carries a relative error of at most ln2 dz(q') + EXP2_REL_ERR (the SFU exp2)
++ 3u (the product by 1/255 and its constant). test_alpha_within_written_bound
+checks the bound on the GPU.
 """
 
 from __future__ import annotations
@@ -15,18 +35,38 @@ import numpy as np
 
 from oracle import oracle as O
 
-# Flag windows: relative distance of alpha from 1/255 and of the trial
-# transmittance from 1e-4 below which float32 and float64 may decide apart.
-# With cancellation in the quadratic form of an elongated Gaussian the
-# kernel's alpha can sit 2e-5 relative from the float64 value (a flip seen at
-# a distance between 2e-5 and 2e-4); every near-opaque layer multiplies that
-# by alpha / (1 - alpha) in the trial T.
-WIN_ALPHA = 2e-4
-WIN_T = 2e-3
-
 MAX_ABS = 2e-3
 MEAN_ABS = 1e-5
 REL_L2 = 1e-3
+
+U24 = 2.0 ** -24
+EXP2_REL_ERR = 2.0 ** -21  # relative error allowed to the SFU's exp2 (ex2.approx)
+HALF_LOG2E = 0.5 / np.log(2.0)
+
+
+def alpha_error_bound(projs) -> np.ndarray:
+    """Relative bound on the rasteriser's alpha_raw for every (view, Gaussian)
+    as [V, n, 2] coefficients (e0, e1) of e0 + e1 q, q the pixel's quadratic
+    form, from the oracle's own projection (see the module docstring)."""
+    out = []
+    for p in projs:
+        o = np.asarray(p["opacity"], np.float64)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            Qp = np.maximum(np.log2(255.0 * o), 0.0)
+            A, B, C = p["cov"][:, 0], p["cov"][:, 1], p["cov"][:, 2]
+            lam1 = np.asarray(p["lam"], np.float64)
+            lam2 = (A * C - B * B) / lam1
+            sk = np.sqrt(np.where(lam2 > 0, lam1 / lam2, 1.0))
+        sk = np.where(np.isfinite(sk) & (sk >= 1.0), sk, 1.0)
+        e0 = np.log(2.0) * U24 * (3.0 * Qp + 1.0) + EXP2_REL_ERR + 3 * U24
+        e1 = np.log(2.0) * U24 * 8.0 * (1.0 + 0.5 * (sk + 1.0 / sk)) * HALF_LOG2E
+        out.append(np.stack([e0, e1], -1))
+    return np.stack(out)
+
+
+def alpha_error_at(bound: np.ndarray, q) -> np.ndarray:
+    """The bound's value e0 + e1 q."""
+    return bound[..., 0] + bound[..., 1] * q
 
 
 def rel_l2(a, b) -> float:
@@ -43,12 +83,27 @@ def oracle_projs(scene):
 
 
 def unpack_records(rec: np.ndarray, bins: np.ndarray) -> dict:
-    """GPU records [V, n, 12] and binning records [V, n, 4] -> named fields."""
+    """GPU records [..., 16] and binning records [..., 4] -> named fields. The
+    evaluation form (float mean, rows w1 w2, offsets c1 c2, -log2(255 o)) is
+    turned back into the mean (the float plus the remainder that solves
+    W r = -c) and the conic W^T W / (log2(e)/2), in float64."""
     tx = bins[..., 1].view(np.uint32)
     ty = bins[..., 2].view(np.uint32)
     rect = np.stack([tx & 0xFFFF, tx >> 16, ty & 0xFFFF, ty >> 16], -1).astype(np.int32)
-    return dict(xy=rec[..., 0:2], conic=rec[..., 2:5], opacity=rec[..., 5], rgb=rec[..., 6:9],
-                hx=rec[..., 9], hy=rec[..., 10], depth=bins[..., 0], rect=rect)
+    r = rec.astype(np.float64)
+    W = np.stack([np.stack([r[..., 2], r[..., 3]], -1), np.stack([r[..., 5], r[..., 6]], -1)], -2)
+    c = np.stack([r[..., 4], r[..., 7]], -1)
+    det = W[..., 0, 0] * W[..., 1, 1] - W[..., 0, 1] * W[..., 1, 0]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        lo_u = (-c[..., 0] * W[..., 1, 1] + c[..., 1] * W[..., 0, 1]) / det
+        lo_v = (-c[..., 1] * W[..., 0, 0] + c[..., 0] * W[..., 1, 0]) / det
+    lo_u = np.where(det != 0, lo_u, 0.0)
+    lo_v = np.where(det != 0, lo_v, 0.0)
+    WtW = np.einsum("...ki,...kj->...ij", W, W) / HALF_LOG2E
+    conic = np.stack([WtW[..., 0, 0], WtW[..., 0, 1], WtW[..., 1, 1]], -1)
+    return dict(xy=np.stack([r[..., 0] + lo_u, r[..., 1] + lo_v], -1), xy_float=rec[..., 0:2],
+                conic=conic, log2_255o=-r[..., 8], opacity=rec[..., 14], rgb=rec[..., 9:12],
+                hx=rec[..., 12], hy=rec[..., 13], depth=bins[..., 0], rect=rect)
 
 
 def pack_bins(projs) -> np.ndarray:
@@ -153,21 +208,39 @@ def full_pixels(scene):
     return np.concatenate(out).astype(np.int32)
 
 
-def compare_render(gpu_image, gpu_T, gpu_nc, ref, pix):
+def colour_max(projs, bg) -> float:
+    """Largest colour magnitude in play (every splat's colour, the background)."""
+    m = max(float(np.max(np.abs(p["rgb"][p["valid"] != 0]), initial=0.0)) for p in projs)
+    return max(m, float(np.max(np.abs(np.asarray(bg, np.float64)))))
+
+
+def compare_render(gpu_image, gpu_T, gpu_nc, ref, pix, cmax=1.0):
     """Colour / transmittance / contributor comparison on listed pixels.
-    Returns a dict of statistics; asserts nothing."""
+    Unflagged pixels are held to the tolerances; a flagged pixel to MAX_ABS
+    plus what its flagged decisions can change (flag_dev * cmax for the
+    colour, 1e-3 T + flag_T for the transmittance). Pixels whose tile list
+    itself is ambiguous (flag bit 2) are only counted. Returns a dict of
+    statistics; asserts nothing."""
     v, x, y = pix[:, 0], pix[:, 1], pix[:, 2]
     g = gpu_image[v, :, y, x].astype(np.float64)           # [P, 3]
     d = np.abs(g - ref["color"])
     flagged = ref["flags"] != 0
+    amb = (ref["flags"] & 4) != 0
     ok = ~flagged
+    fl = flagged & ~amb
+    gT = gpu_T[v, y, x].astype(np.float64)
+    dT = np.abs(gT - ref["T"])
+    fdev = ref.get("flag_dev", np.zeros(len(pix)))
+    fT = ref.get("flag_T", np.zeros(len(pix)))
     stats = dict(
-        n=len(pix), flagged=int(flagged.sum()),
+        n=len(pix), flagged=int(flagged.sum()), ambiguous=int(amb.sum()),
         max_abs=float(d[ok].max()) if ok.any() else 0.0,
         mean_abs=float(d[ok].mean()) if ok.any() else 0.0,
         max_abs_all=float(d.max()),
         nc_mismatch=int((gpu_nc[v, y, x].astype(np.int64) != ref["n_contrib"])[ok].sum()),
-        T_max_rel=float((np.abs(gpu_T[v, y, x] - ref["T"]) / np.maximum(ref["T"], 1e-4))[ok].max())
-        if ok.any() else 0.0,
+        T_max_rel=float((dT / np.maximum(ref["T"], 1e-4))[ok].max()) if ok.any() else 0.0,
+        flagged_excess=float((d.max(1) - (MAX_ABS + fdev * cmax))[fl].max()) if fl.any()
+        else -1.0,
+        flagged_T_excess=float((dT - (1e-3 * ref["T"] + fT))[fl].max()) if fl.any() else -1.0,
     )
     return stats

@@ -31,7 +31,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_status_strings():
-    assert api.gs_abi_version() == 1
+    assert api.gs_abi_version() == 2
     for s in range(7):
         assert api.status_string(s) not in ("", "unknown status")
 
@@ -59,13 +59,30 @@ def test_bad_arguments_are_rejected_before_any_cuda_call():
     cams = api.cameras(sc.cameras)
     p = api.GsParams(None, None, None, None, None, 0, 0, 10)
     out = api.GsProjected(None, None)
-    assert L.gs_project(ctypes.byref(p), cams, 1, ctypes.byref(out), None) == api.GS_ERR_INVALID_ARG
+    # an aligned address that is never dereferenced: each call returns first
+    ws = ctypes.c_void_p(4096)
+    assert L.gs_project(ctypes.byref(p), cams, 1, ctypes.byref(out), ws, None) == \
+        api.GS_ERR_INVALID_ARG
     p.sh_degree = 4
-    assert L.gs_project(ctypes.byref(p), cams, 1, ctypes.byref(out), None) == api.GS_ERR_INVALID_ARG
+    assert L.gs_project(ctypes.byref(p), cams, 1, ctypes.byref(out), ws, None) == \
+        api.GS_ERR_INVALID_ARG
     p.n = 1 << 31
     p.sh_degree = 0
-    assert L.gs_project(ctypes.byref(p), cams, 1, ctypes.byref(out), None) == api.GS_ERR_OVERFLOW
-    assert L.gs_project(ctypes.byref(p), cams, 0, ctypes.byref(out), None) == api.GS_ERR_INVALID_ARG
+    assert L.gs_project(ctypes.byref(p), cams, 1, ctypes.byref(out), ws, None) == \
+        api.GS_ERR_OVERFLOW
+    assert L.gs_project(ctypes.byref(p), cams, 0, ctypes.byref(out), ws, None) == \
+        api.GS_ERR_INVALID_ARG
+    # the status word is required, and must be 256-byte aligned
+    assert L.gs_project(ctypes.byref(p), cams, 1, ctypes.byref(out), None, None) == \
+        api.GS_ERR_INVALID_ARG
+    assert L.gs_project(ctypes.byref(p), cams, 1, ctypes.byref(out), ctypes.c_void_p(4100),
+                        None) == api.GS_ERR_INVALID_ARG
+    bn = api.GsBinned(None, None, None, 10)
+    bg = (ctypes.c_float * 3)()
+    assert L.gs_rasterize_fwd(ctypes.byref(out), ctypes.byref(bn), cams, 1, 10, bg, None, None,
+                              None, None, None) == api.GS_ERR_INVALID_ARG
+    assert L.gs_rasterize_bwd(ctypes.byref(p), ctypes.byref(out), ctypes.byref(bn), cams, 1, bg,
+                              None, None, None, None, None, None, None) == api.GS_ERR_INVALID_ARG
     b = api.GsBinned(None, None, None, 10)
     assert L.gs_bin_sort(ctypes.byref(out), cams, 1, 10, 0, ctypes.byref(b), None, 0, None) == \
         api.GS_ERR_INVALID_ARG
@@ -75,6 +92,15 @@ def test_bad_arguments_are_rejected_before_any_cuda_call():
     assert L.gs_adam_step(grp, 1, 1.5, 0.999, 1e-15, 1, None) == api.GS_ERR_INVALID_ARG
     assert L.gs_densify_stats(None, None, 0, 10, None, None, None, None) == api.GS_ERR_INVALID_ARG
     assert L.gs_get_status(None, None) == api.GS_ERR_INVALID_ARG
+
+
+def test_debug_stall_arguments():
+    assert api.lib().gs_debug_stall(api.GS_STALL_RASTER_FWD, -1, 0.0) == api.GS_ERR_INVALID_ARG
+    assert api.lib().gs_debug_stall(9, 0, 0.0) == api.GS_ERR_INVALID_ARG
+    assert api.lib().gs_debug_stall(api.GS_STALL_NONE, 0, -1.0) == api.GS_ERR_INVALID_ARG
+    assert api.lib().gs_debug_stall(api.GS_STALL_NONE, 0, 61.0) == api.GS_ERR_INVALID_ARG
+    api.gs_debug_stall(api.GS_STALL_RASTER_BWD, 3, 0.05)
+    api.gs_debug_stall(api.GS_STALL_NONE)
 
 
 def test_loss_and_quant_arguments_are_rejected_before_any_cuda_call():

@@ -63,10 +63,17 @@ def test_project_matches_oracle(name, kw, how):
         assert np.array_equal(radii[v][m], p["radius"][m])
         assert np.array_equal(g["rect"][m], p["rect"][m])
         assert np.array_equal(g["depth"][m].view(np.uint32), p["key"][m].view(np.uint32))
-        np.testing.assert_allclose(g["xy"][m], p["xy"][m], rtol=1e-6, atol=1e-4)
+        # the mean: its float part is the float of the oracle's mean (up to a
+        # tie in the rounding), and float part + remainder is the mean far
+        # below float resolution
+        assert np.max(np.abs(g["xy_float"][m] - p["xy"][m].astype(np.float32))
+                      / np.maximum(1.0, np.abs(p["xy"][m]))) <= 2 ** -23
+        assert np.max(np.abs(g["xy"][m] - p["xy"][m])) < 1e-8
         scale = np.sqrt(p["conic"][m, 0] * p["conic"][m, 2])[:, None]
         assert np.max(np.abs(g["conic"][m] - p["conic"][m]) / scale) < 2e-6
         np.testing.assert_allclose(g["opacity"][m], p["opacity"][m], rtol=2e-6)
+        lo2 = np.log2(255.0 * p["opacity"][m])
+        assert np.max(np.abs(g["log2_255o"][m] - lo2) / np.maximum(1.0, np.abs(lo2))) < 2 ** -23
         np.testing.assert_allclose(g["rgb"][m], p["rgb"][m], atol=2e-5)
         # the culling box holds the whole alpha >= 1/255 ellipse: its
         # half-widths are at least sqrt(Q cov_xx), sqrt(Q cov_yy)
@@ -96,8 +103,7 @@ def test_binning_bit_exact(name, kw, how, mode):
     if not amb.any():
         assert n_pairs == int(area[valid].sum())
     tiles = ranges.shape[0]
-    sel = np.arange(tiles) if how == "full" else np.unique(
-        np.random.default_rng(0).integers(0, tiles, 400))
+    sel = np.arange(tiles)  # every tile, at every size
     sel = sel[~amb[sel]]
     assert P.compare_lists(ids, ranges, rects, keys, sc, sel) == 0
     # ranges tile the pair array in order
@@ -144,22 +150,27 @@ def test_render_matches_oracle(name, kw, how):
     sc, sp = _setup(name, kw)
     sp.rasterize_fwd()
     torch.cuda.synchronize()
+    assert sp.status() == api.GS_OK
     pix = _pixels(sc, how)
     projs = O.project_views(sc)
-    ref = O.render(projs, sc.cameras, sc.background, pix, P.WIN_ALPHA, P.WIN_T)
+    ref = O.render(projs, sc.cameras, sc.background, pix,
+                   alpha_err=P.alpha_error_bound(projs))
     ref["flags"] = ref["flags"] | (4 * P.ambiguous_pixels(sc, projs, pix))
     st = P.compare_render(sp.image.cpu().numpy(), sp.final_T.cpu().numpy(),
-                          sp.n_contrib.cpu().numpy(), ref, pix)
+                          sp.n_contrib.cpu().numpy(), ref, pix,
+                          P.colour_max(projs, sc.background))
     print(name, st)
-    # pixels whose alpha lies near 1/255 (or T near 1e-4) are excluded; their
-    # share grows with the number of Gaussians overlapping a pixel (about 3 %
-    # for the 1M-Gaussian benchmark scene), so the bound only keeps the
-    # comparison from becoming vacuous
-    assert st["flagged"] <= 0.05 * st["n"]
+    # flagged: a decision within the kernel's written error bound of its
+    # threshold; such a pixel is still checked against what the decisions
+    # can change
+    assert st["flagged"] <= 1e-3 * st["n"]
+    assert st["ambiguous"] == 0
     assert st["max_abs"] <= P.MAX_ABS
     assert st["mean_abs"] <= P.MEAN_ABS
     assert st["nc_mismatch"] == 0
     assert st["T_max_rel"] < 1e-3
+    assert st["flagged_excess"] <= 0.0
+    assert st["flagged_T_excess"] <= 0.0
 
 
 @pytest.mark.parametrize("name,kw,how", CASES)
@@ -169,13 +180,17 @@ def test_backward_and_densify_match_oracle(name, kw, how):
     torch.cuda.synchronize()
     projs = O.project_views(sc)
     pix = _pixels(sc, how)
-    ref = O.render(projs, sc.cameras, sc.background, pix, P.WIN_ALPHA, P.WIN_T)
-    keep = pix[(ref["flags"] == 0) & ~P.ambiguous_pixels(sc, projs, pix)]
+    assert not P.ambiguous_pixels(sc, projs, pix).any()
+    # the upstream gradient on every checked pixel, flagged ones included (a
+    # sampled case masks it to the sample on both sides, so both compute the
+    # same function)
+    keep = pix
     c = sc.cameras[0]
     dL = S.make_upstream_grad(sc.n_views, c.height, c.width, seed=1)
-    mask = np.zeros_like(dL)
-    mask[keep[:, 0], :, keep[:, 2], keep[:, 1]] = 1.0
-    dL = dL * mask
+    if how != "full":
+        mask = np.zeros_like(dL)
+        mask[keep[:, 0], :, keep[:, 2], keep[:, 1]] = 1.0
+        dL = dL * mask
     sp.rasterize_bwd(torch.as_tensor(dL).cuda())
     sp.densify_stats()
     torch.cuda.synchronize()
@@ -342,6 +357,53 @@ def test_empty_and_all_culled(mode):
         assert torch.all(sp.n_contrib == 0)
         for t in sp.grads.values():
             assert torch.all(t == 0)
+
+
+def test_alpha_within_written_bound():
+    """Every pixel of a scene of isolated splats (at most one per pixel, black
+    background): the kernel's alpha, read off the image as colour / splat
+    colour, lies within the written relative bound of the oracle's float64
+    alpha (parity.alpha_error_bound plus the two roundings of the read-off),
+    and where the oracle does not flag the pixel the two take the same skip
+    decision. Anisotropy up to ~15, clamped and too-faint splats, means near
+    x = 2048 where a float holds the mean to 1e-4 px."""
+    sc = S.make_isolated_scene()
+    side, spacing = 16, 128
+    sp = Splatter(sc)
+    sp.ensure_capacity()
+    sp.rasterize_fwd()
+    torch.cuda.synchronize()
+    assert sp.status() == api.GS_OK
+    projs = O.project_views(sc)
+    bound = P.alpha_error_bound(projs)
+    pix = P.full_pixels(sc)
+    ref = O.render(projs, sc.cameras, sc.background, pix, alpha_err=bound)
+    assert ref["n_used"].max() <= 1                      # isolated
+    gid = (pix[:, 2] // spacing) * side + pix[:, 1] // spacing
+    rgb_o = projs[0]["rgb"][gid]
+    rgb_k = sp.records.cpu().numpy()[0, gid, 9:12].astype(np.float64)
+    ch = np.argmax(rgb_o, axis=1)
+    rows = np.arange(len(pix))
+    img = sp.image.cpu().numpy()[0].reshape(3, -1).T.astype(np.float64)
+    a_o = ref["color"][rows, ch] / rgb_o[rows, ch]
+    a_k = img[rows, ch] / rgb_k[rows, ch]
+    flagged = ref["flags"] != 0
+    assert flagged.mean() < 1e-3
+    # the same decision wherever it is not within the bound of its threshold
+    assert np.array_equal((a_k > 0)[~flagged], (a_o > 0)[~flagged])
+    both = (a_k > 0) & (a_o > 0)
+    assert both.sum() > 20000
+    rel = np.abs(a_k[both] / a_o[both] - 1.0)
+    # the splat's quadratic form at each pixel, for the bound's q term
+    pr = projs[0]
+    d0 = pix[:, 1] + 0.5 - pr["xy"][gid, 0]
+    d1 = pix[:, 2] + 0.5 - pr["xy"][gid, 1]
+    cn = pr["conic"][gid]
+    q = cn[:, 0] * d0 * d0 + 2 * cn[:, 1] * d0 * d1 + cn[:, 2] * d1 * d1
+    lim = P.alpha_error_at(bound[0, gid[both]], q[both]) + 2.0 ** -22
+    print("alpha rel err: max %.2e, max / bound %.3f, median bound %.2e" % (
+        rel.max(), (rel / lim).max(), np.median(lim)))
+    assert np.all(rel <= lim)
 
 
 def test_single_gaussian_centred_on_pixel_gives_o_c():

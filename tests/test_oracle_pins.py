@@ -356,7 +356,75 @@ def _fd_case(seed, deg):
 
 @pytest.mark.parametrize("seed,deg", [(3, 3), (11, 3), (5, 0)])
 def test_gradients_match_central_differences(seed, deg):
-    sc = _fd_case(seed, deg)
+    _check_central_differences(_fd_case(seed, deg), seed)
+
+
+def _clamp_case():
+    """The finite-difference scene with both clamps reached: Gaussian 0 is an
+    opaque (logit 8, opacity 0.99966), round, front-most splat over the image
+    centre, so alpha = min(0.99, o exp(-q/2)) clamps on the pixels within
+    ~0.14 sigma of its mean; Gaussians 1 and 2 have a colour channel (red,
+    blue) whose SH sum is far below 0, so max(0, .) clamps it."""
+    sc = _fd_case(3, 3)
+    sc.means[0, :3] = (0.05, -0.03, -3.0)       # depth 5, in front of the rest
+    sc.log_scales[0, :3] = 0.2
+    sc.opacity_logit[0] = 8.0
+    sc.sh[1, 0, 0] = -4.0
+    sc.sh[2, 0, 2] = -4.0
+    return sc
+
+
+def test_clamp_branches_are_reached_and_match_central_differences():
+    sc = _clamp_case()
+    cam = sc.cameras[0]
+    pr = O.project_views(sc)[0]
+    # the colour clamp holds for red of Gaussian 1 and blue of Gaussian 2
+    assert pr["clamp"][1] & 1 and pr["clamp"][2] & 4
+    assert pr["rgb"][1, 0] == 0.0 and pr["rgb"][2, 2] == 0.0
+    # the alpha clamp holds on a few pixels of Gaussian 0
+    ys, xs = np.meshgrid(np.arange(cam.height) + 0.5, np.arange(cam.width) + 0.5, indexing="ij")
+    d0, d1 = xs - pr["xy"][0, 0], ys - pr["xy"][0, 1]
+    a, b, c = pr["conic"][0]
+    araw = pr["opacity"][0] * np.exp(-0.5 * (a * d0 * d0 + 2 * b * d0 * d1 + c * d1 * d1))
+    assert (araw >= 0.99).sum() >= 3
+    # every gradient, the clamped ones included, against central differences
+    _check_central_differences(sc, 3)
+
+
+def test_clamped_alpha_passes_colour_gradient_only():
+    """On a pixel where the front-most splat's alpha is clamped at 0.99, the
+    pixel's gradient reaches that splat's colour (d C / d c = alpha T = 0.99)
+    and nothing else: its opacity, its conic and its screen-space mean do not
+    move the pixel (the 3D mean still moves it through the view-dependent
+    colour, so the central differences below perturb the logit, the scales
+    and the rotation)."""
+    sc = _clamp_case()
+    cam = sc.cameras[0]
+    pr = O.project_views(sc)
+    x, y = int(pr[0]["xy"][0, 0]), int(pr[0]["xy"][0, 1])
+    pix = np.array([[0, x, y]])
+    d0, d1 = x + 0.5 - pr[0]["xy"][0, 0], y + 0.5 - pr[0]["xy"][0, 1]
+    a, b, c = pr[0]["conic"][0]
+    assert pr[0]["opacity"][0] * np.exp(-0.5 * (a * d0 * d0 + 2 * b * d0 * d1 + c * d1 * d1)) \
+        >= 0.99
+    gC = np.array([[0.3, -0.2, 0.5]])
+    bg = np.array([0.2, 0.5, 0.1])
+    g = O.render_bwd(pr, sc.cameras, bg, pix, gC)[0, 0]
+    assert np.all(g[[0, 1, 2, 3, 4, 5, 9]] == 0.0)
+    np.testing.assert_allclose(g[6:9], 0.99 * gC[0], rtol=1e-12)
+    # the same by central differences of that pixel's colour
+    for k in ("opacity_logit", "log_scales", "quats"):
+        for j in range(getattr(sc, k).reshape(sc.n, -1).shape[1]):
+            vals = []
+            for sgn in (1, -1):
+                s2 = copy.deepcopy(sc)
+                getattr(s2, k).reshape(sc.n, -1)[0, j] += sgn * 1e-5
+                p2 = O.project_views(s2)
+                vals.append((O.render(p2, s2.cameras, bg, pix)["color"] * gC).sum())
+            assert abs(vals[0] - vals[1]) < 1e-12, (k, j)
+
+
+def _check_central_differences(sc, seed):
     cam = sc.cameras[0]
     ys, xs = np.meshgrid(np.arange(cam.height), np.arange(cam.width), indexing="ij")
     pix = np.stack([np.zeros(xs.size, int), xs.ravel(), ys.ravel()], 1)
