@@ -71,6 +71,11 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-protocol", action="store_true",
+                    help="skip the 20 + 100 step median measurement")
+    ap.add_argument("--no-graphs", action="store_true",
+                    help="launch every call's kernels from the host instead of replaying "
+                         "one CUDA graph per call")
     args = ap.parse_args()
     if args.sort_mode is None:
         args.sort_mode = STEPS[args.workload]["sort"]
@@ -592,6 +597,9 @@ def run_ours(args):
         sp.shard_optimizer(rank, world)
     sp.ensure_capacity()
     V = sp.V
+    # the parameters and moments the timed steps start from (Adam moves them;
+    # the protocol run below starts from the same state)
+    start_state = [t.clone() for t in (sp.param_flat, sp.m_flat, sp.v_flat)]
     dL_host = S.make_upstream_grad(V, c.height, c.width, seed=1)
     dL = torch.as_tensor(dL_host).cuda() if kind != "fwd" else None
     stream = torch.cuda.current_stream()
@@ -603,24 +611,35 @@ def run_ours(args):
     if kind == "train":
         names += ["gs_adam_step" if world == 1 else "reduce_scatter+gs_adam_step+all_gather"]
 
+    # one CUDA graph per call (not Adam, whose bias corrections follow the
+    # step count): the call's kernels replay without host launch gaps
+    graphs = None if args.no_graphs else sp.capture_calls(dL)
+    torch.cuda.synchronize()
+
+    def call(name, fn):
+        if graphs is not None and name in graphs:
+            graphs[name].replay()
+        else:
+            fn()
+
     def step(events=None):
         def mark(k):
             if events is not None:
                 events[k].record(stream)
         mark(0)
-        sp.project()
+        call("project", sp.project)
         mark(1)
-        sp.bin_sort()
+        call("bin_sort", sp.bin_sort)
         mark(2)
-        sp.rasterize_fwd()
+        call("rasterize_fwd", sp.rasterize_fwd)
         mark(3)
         if kind == "fwd":
             return
-        sp.rasterize_bwd(dL, with_params=False)
+        call("rasterize_bwd", lambda: sp.rasterize_bwd(dL, with_params=False))
         mark(4)
-        sp.project_bwd()
+        call("project_bwd", sp.project_bwd)
         mark(5)
-        sp.densify_stats()
+        call("densify_stats", sp.densify_stats)
         mark(6)
         if kind == "train":
             sp.adam_step()  # with N > 1: reduce-scatter, Adam on the slice, all-gather
@@ -671,7 +690,9 @@ def run_ours(args):
     # the measurement protocol of the scope table: 20 warm-up steps, then the
     # median of 100 steps, each timed by its own events (single GPU)
     protocol = None
-    if world == 1:
+    if world == 1 and not args.no_protocol:
+        for dst, src in zip((sp.param_flat, sp.m_flat, sp.v_flat), start_state):
+            dst.copy_(src)
         for _ in range(20):
             step()
         pev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
@@ -795,6 +816,8 @@ def run_ours(args):
                    "width": c.width, "height": c.height, "views_per_gpu": V,
                    "sh_degree": sp.deg, "pairs": n_pairs, "sort_mode": args.sort_mode,
                    "sort_path": sort_plan(sp, args.sort_mode)["path"],
+                   "launch": "host launches" if graphs is None else
+                             "one CUDA graph per call (Adam launched from the host)",
                    "l2": ("working set %.0f MB inside the 126 MB L2: flushed (256 MB write) "
                           "before every step, outside the step's own timing"
                           % (working_set_bytes(sp) / 1e6)) if flush_l2 else

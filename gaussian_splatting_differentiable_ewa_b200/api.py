@@ -110,6 +110,9 @@ SIGNATURES = [
      [_c.POINTER(GsAdamGroup), _c.c_int32, _c.c_float, _c.c_float, _c.c_float, _c.c_int64, _vp]),
     ("gs_get_status", _c.c_int, [_vp, _vp]),
     ("gs_densify_workspace_size", _c.c_size_t, [_c.c_int64]),
+    ("gs_densify_params_from_cutoffs", _c.c_int,
+     [_c.c_double, _c.c_double, _c.c_double, _c.c_double, _c.c_double,
+      _c.POINTER(GsDensifyParams)]),
     ("gs_densify_and_prune", _c.c_int,
      [_c.POINTER(GsParams), _c.POINTER(GsGrads), _c.POINTER(GsGrads), _vp, _vp, _vp,
       _c.POINTER(GsDensifyParams), _c.POINTER(GsGrads), _c.POINTER(GsGrads), _c.POINTER(GsGrads),
@@ -294,11 +297,14 @@ def gs_get_status(ws, stream=None) -> int:
 
 def densify_params(grad_threshold: float, scale_split: float, min_opacity: float,
                    max_scale: float, split_shrink: float = 1.6) -> GsDensifyParams:
-    """Thresholds in the units of the call: log-scales and a logit (float32)."""
-    import math
-    return GsDensifyParams(float(grad_threshold), float(math.log(scale_split)),
-                           float(math.log(min_opacity / (1.0 - min_opacity))),
-                           float(math.log(max_scale)), float(math.log(split_shrink)), 0)
+    """gs_densify_params from cut-offs stated as scales and an opacity (the
+    library converts them to log-scales and a logit)."""
+    dp = GsDensifyParams()
+    _check(lib().gs_densify_params_from_cutoffs(float(grad_threshold), float(scale_split),
+                                                float(min_opacity), float(max_scale),
+                                                float(split_shrink), _c.byref(dp)),
+           "gs_densify_params_from_cutoffs")
+    return dp
 
 
 def gs_densify_workspace_size(n: int) -> int:

@@ -438,6 +438,21 @@ gs_status gs_bin_sort_noalloc(const gs_projected* proj, const gs_camera* cams, i
   return GS_OK;
 }
 
+gs_status gs_densify_params_from_cutoffs(double grad_threshold, double scale_split,
+                                         double min_opacity, double max_scale,
+                                         double split_shrink, gs_densify_params* out) {
+  if (!out || !(scale_split > 0.0) || !(max_scale > 0.0) || !(split_shrink > 0.0) ||
+      !(min_opacity > 0.0 && min_opacity < 1.0))
+    return GS_ERR_INVALID_ARG;
+  out->grad_threshold = (float)grad_threshold;
+  out->log_scale_split = (float)std::log(scale_split);
+  out->logit_min_opacity = (float)std::log(min_opacity / (1.0 - min_opacity));
+  out->log_max_scale = (float)std::log(max_scale);
+  out->log_split_shrink = (float)std::log(split_shrink);
+  out->reserved = 0;
+  return GS_OK;
+}
+
 size_t gs_densify_workspace_size(int64_t n) {
   if (n < 0 || n >= (1ll << 31)) return 0;
   size_t off = kControlBytes;

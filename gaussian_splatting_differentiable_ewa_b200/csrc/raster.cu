@@ -137,6 +137,48 @@ __device__ __forceinline__ uint32_t warp_block_mask(float u, float v, float hx, 
   return mask;
 }
 
+// Refines warp_block_mask with the ellipse itself: a warp's 8x8 block of
+// pixel centres [xlo, xlo + 7] x [ylo, ylo + 7] keeps the splat only if the
+// quadratic q'(d) = (w1 . d)^2 + (w2 . d)^2 (d from the float mean) reaches
+// at most Q' = -nlo somewhere on that rectangle: 0 when the mean is inside,
+// else the least value over the four edges (on an edge q' is a parabola in
+// the free coordinate, minimised at its vertex clamped to the edge). Q' is
+// padded (0.2 % + 0.01) well beyond the float rounding of the rasteriser's zq
+// and the mean's float remainder, so no pixel the per-pixel test takes is
+// dropped; the axis-aligned box keeps, on average, ~40 % more (warp, splat)
+// pairs whose ellipse misses the block.
+__device__ __forceinline__ uint32_t warp_block_mask_ellipse(const float* r, uint32_t box, int x0,
+                                                            int y0) {
+  if (box == 0u) return 0u;
+  const float w1x = r[R_W1X], w1y = r[R_W1Y], w2x = r[R_W2X], w2y = r[R_W2Y];
+  const float a = fmaf(w1x, w1x, w2x * w2x), b = fmaf(w1x, w1y, w2x * w2y);
+  const float c = fmaf(w1y, w1y, w2y * w2y);
+  const float ia = 1.f / a, ic = 1.f / c;
+  const float qm = fmaf(-r[R_NLO], 1.002f, 0.01f);
+  const float u = r[R_U], v = r[R_V];
+  uint32_t mask = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    if (!((box >> w) & 1u)) continue;
+    const float ex0 = (float)(x0 + 8 * (w & 1)) + 0.5f - u, ex1 = ex0 + 7.f;
+    const float ey0 = (float)(y0 + 8 * (w >> 1)) + 0.5f - v, ey1 = ey0 + 7.f;
+    bool hit = ex0 <= 0.f && ex1 >= 0.f && ey0 <= 0.f && ey1 >= 0.f;
+    float best = __int_as_float(0x7f800000);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float ex = e ? ex1 : ex0;  // vertical edges
+      const float dy = fminf(fmaxf(-b * ex * ic, ey0), ey1);
+      best = fminf(best, fmaf(a * ex, ex, fmaf(2.f * b * ex, dy, c * dy * dy)));
+      const float ey = e ? ey1 : ey0;  // horizontal edges
+      const float dx = fminf(fmaxf(-b * ey * ia, ex0), ex1);
+      best = fminf(best, fmaf(c * ey, ey, fmaf(2.f * b * ey, dx, a * dx * dx)));
+    }
+    hit = hit || best <= qm;
+    mask |= hit ? 1u << w : 0u;
+  }
+  return mask;
+}
+
 // zq at the pair's pixel centres (pxc, pyc.x) and (pxc, pyc.y):
 //   dx = pxc - uh, dy = pyc - vh, p_i = fma(w_iy, dy, fma(w_ix, dx, c_i)),
 //   zq = fma(p1, p1, fma(p2, p2, nlo)).
@@ -162,7 +204,7 @@ __device__ __forceinline__ uint32_t prepare_record(const float* r, float2* e, in
   e4[3] = make_float4(r[R_W2Y], r[R_W2Y], r[R_C2], r[R_C2]);
   e4[4] = make_float4(r[R_NLO], r[R_NLO], r[R_R], r[R_R]);
   e4[5] = make_float4(r[R_G], r[R_G], r[R_B], r[R_B]);
-  return warp_block_mask(u, v, r[R_HX], r[R_HY], x0, y0);
+  return warp_block_mask_ellipse(r, warp_block_mask(u, v, r[R_HX], r[R_HY], x0, y0), x0, y0);
 }
 
 // eval_zq on a record in its stored (scalar) form: per pixel the same IEEE
@@ -482,7 +524,8 @@ __global__ void __launch_bounds__(kThreads) k_raster_bwd(
     pend[buf] = -1;
     if ((int)threadIdx.x < m) {
       float* r = &s_rec[buf][threadIdx.x][0];
-      const uint32_t mask = warp_block_mask(r[R_U], r[R_V], r[R_HX], r[R_HY], tp.x0, tp.y0);
+      const uint32_t mask = warp_block_mask_ellipse(
+          r, warp_block_mask(r[R_U], r[R_V], r[R_HX], r[R_HY], tp.x0, tp.y0), tp.x0, tp.y0);
       s_mask[threadIdx.x] = clipped[buf] ? 0u : (uint8_t)mask;
       r[R_OPAC] = 1.f / r[R_OPAC];  // d alpha / d opacity = alpha / o
     }
@@ -491,7 +534,9 @@ __global__ void __launch_bounds__(kThreads) k_raster_bwd(
       z[0] = z[1] = z[2] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
-    const int wc_n = warp_list(s_mask, s_list[warp], m);
+    // this warp's pixels use no entry at or past the longest prefix among them
+    const int64_t wlim = (int64_t)wm - (int64_t)b * kBatch;
+    const int wc_n = warp_list(s_mask, s_list[warp], wlim < m ? (wlim > 0 ? (int)wlim : 0) : m);
     for (int k = wc_n - 1; k >= 0; --k) {
       const int j = s_list[warp][k];
       const uint32_t pos = (uint32_t)(b * kBatch + j);

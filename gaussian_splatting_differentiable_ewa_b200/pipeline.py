@@ -287,6 +287,43 @@ class Splatter:
                 None if sh is None else (sh["lo"], sh["hi"]),
                 None if sh is None else sh["group"])
 
+    def capture_calls(self, dL_dimage: Optional[torch.Tensor] = None) -> dict:
+        """CUDA graphs of this Splatter's fixed-shape calls: 'project',
+        'bin_sort', 'rasterize_fwd' and, given an upstream gradient,
+        'rasterize_bwd' (screen space), 'project_bwd' and 'densify_stats'.
+        Every size and pointer of those calls is fixed once ensure_capacity has
+        sized the buffers, so a graph replays the call's kernels with no host
+        launch gaps between them (gs_bin_sort alone is up to 17 launches).
+        Replays run on the current stream. The Adam step is not captured: its
+        bias corrections follow the step count, a host value of the call. The
+        graphs stay valid until a buffer is reallocated (ensure_capacity growing
+        the pairs, densify_and_prune)."""
+        calls = {"project": self.project, "bin_sort": self.bin_sort,
+                 "rasterize_fwd": self.rasterize_fwd}
+        if dL_dimage is not None:
+            calls["rasterize_bwd"] = lambda: self.rasterize_bwd(dL_dimage, with_params=False)
+            calls["project_bwd"] = self.project_bwd
+            calls["densify_stats"] = self.densify_stats
+        saved = self.stream
+        cap = torch.cuda.Stream(device=self.device)
+        cap.wait_stream(torch.cuda.current_stream(self.device))
+        graphs = {}
+        try:
+            for name, fn in calls.items():
+                with torch.cuda.stream(cap):
+                    self.stream = cap
+                    fn()  # the call once outside capture, on the capture stream
+                cap.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=cap):
+                    self.stream = cap
+                    fn()
+                graphs[name] = g
+        finally:
+            self.stream = saved
+        torch.cuda.current_stream(self.device).wait_stream(cap)
+        return graphs
+
     def forward(self):
         self.project()
         self.bin_sort()

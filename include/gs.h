@@ -383,6 +383,17 @@ typedef struct gs_densify_params {
   int32_t reserved;
 } gs_densify_params;
 
+/* The thresholds of gs_densify_and_prune from cut-offs in the units a user
+ * states them in (host only, no CUDA call): the gradient threshold as is, the
+ * scales as scales (log-scale = ln s), the minimum opacity as an opacity
+ * (logit = ln(o / (1 - o))) and the split shrink factor (ln of it; 1.6 in
+ * the usual configuration). Each conversion is taken in double precision and
+ * rounded to float once. GS_ERR_INVALID_ARG unless scale_split, max_scale and
+ * split_shrink are > 0, 0 < min_opacity < 1 and out is not NULL. */
+gs_status gs_densify_params_from_cutoffs(double grad_threshold, double scale_split,
+                                         double min_opacity, double max_scale,
+                                         double split_shrink, gs_densify_params* out);
+
 /* Bytes of workspace gs_densify_and_prune needs for n Gaussians (256-byte
  * aligned; the first 256 bytes hold the status word, as for gs_bin_sort). */
 size_t gs_densify_workspace_size(int64_t n);

@@ -11,22 +11,32 @@ Tolerances (the task's acceptance criteria):
   * gradients, densify statistics and Adam state: relative L2 <= 1e-3.
 
 The kernel's alpha error bound (alpha_error_bound) is derived from the
-rasteriser's arithmetic on the record's evaluation form: with u = 2^-24,
-d = P - (uh, vh) and p_i = fl(w_iy dy + fl(w_ix dx + c_i)), each p_i is off
-by at most u (4 |w_ix dx| + 3 |w_iy dy| + 3 |c_i|) -- the rounding of dx, of
-the float row w_i, and of the two fmas -- and zq = fl(p1^2 + fl(p2^2 + nlo))
-by at most u (|nlo| + |t| + |zq|) + 2 |p1| dp1 + 2 |p2| dp2 with t the inner
-fma. Where a splat counts, zq <= 0 and q' = p1^2 + p2^2 <= Q' = log2(255 o),
-so |nlo|, |t| and |zq| are at most Q'; writing x = k1 |d . e1|, y = k2
-|d . e2| (q' = x^2 + y^2, |d| <= x / k1 + y / k2, k1 / k2 = 1 / sqrt(kappa),
-kappa = lambda1 / lambda2 of the 2D covariance), 2 |p1| dp1 + 2 |p2| dp2 <=
-8 u (q' + x y (sqrt(kappa) + 1 / sqrt(kappa))) <= 8 u q' (1 + (sqrt(kappa) +
-1 / sqrt(kappa)) / 2). So |zq - zq_exact| <= dz(q') = u (3 Q' + 1 + 8 q' (1 +
-(sqrt(kappa) + 1 / sqrt(kappa)) / 2)) (the 1 covers the c_i terms, at most
-~1e-4 in size), with q' = (log2(e) / 2) q, and alpha_raw = 2^-zq / 255
-carries a relative error of at most ln2 dz(q') + EXP2_REL_ERR (the SFU exp2)
-+ 3u (the product by 1/255 and its constant). test_alpha_within_written_bound
-checks the bound on the GPU.
+rasteriser's arithmetic on the record's evaluation form. With u = 2^-24, the
+true offset d = P - mean and its float part dx = fl(P_x - uh), the kernel takes
+a_i = fl(w_ix dx + c_i) and p_i = fl(w_iy dy + a_i) with float rows w_i (off
+the exact rows by u relative each); so p_i is off the exact w_i . d by at most
+u (3 |w_ix dx| + 2 |w_iy dy| + 2 |c_i| + |p_i|) <= u (3 |w_i| |d| + |p_i| +
+2 |c_i|) -- the row, dx and the inner fma for the x term, the row and dy for
+the y term, both fmas for c_i, the outer fma's own rounding. Then zq =
+fl(p1^2 + fl(p2^2 + nlo)) (the squares are exact inside the fmas) is off by at
+most u (|nlo| + |t| + |zq|) + 2 |p1| dp1 + 2 |p2| dp2, t the inner fma. Where
+a splat counts, q' = p1^2 + p2^2 <= Q' = log2(255 o) and zq = q' - Q' <= 0, so
+|nlo| + |t| + |zq| <= 3 Q' - q'. Writing x = |p1| = k1 |d . e1| and y = |p2| =
+k2 |d . e2| (so q' = x^2 + y^2, |d| <= x / k1 + y / k2, k2 / k1 = sqrt(kappa)
+with kappa = lambda1 / lambda2 of the 2D covariance), 2 sum |p_i| 3 |w_i| |d|
+<= 6 (x^2 + y^2 + x y (sqrt(kappa) + 1 / sqrt(kappa))) <= 3 q' (2 + sqrt(kappa)
++ 1 / sqrt(kappa)), and 2 sum |p_i| |p_i| u = 2 u q'. Altogether
+
+    |zq - zq_exact| <= dz(q') = u (3 Q' + 1 + q' (7 + 3 (sqrt(kappa) +
+                                                 1 / sqrt(kappa))))
+
+(the 1 covers the c_i terms: |c_i| <= |w_i| |mean - float mean| < 4e-4 for
+coordinates below 4096), with q' = (log2(e) / 2) q. alpha_raw = fl(2^-zq) *
+fl(1/255) then carries a relative error of at most ln2 dz(q') + EXP2_REL_ERR
+(the SFU exp2 the kernel calls) + 3u (the product, the constant, slack).
+test_alpha_within_written_bound checks the whole bound on the GPU, and
+test_sfu_exp2_error_bound measures EXP2_REL_ERR's part exhaustively over every
+float argument the kernel can pass (0 to 8).
 """
 
 from __future__ import annotations
@@ -39,8 +49,19 @@ MAX_ABS = 2e-3
 MEAN_ABS = 1e-5
 REL_L2 = 1e-3
 
+# A pixel is flagged when one of its alpha >= 1/255 evaluations (or its stop
+# test) falls within the kernel's bound of the threshold, so the flagged share
+# grows with the evaluations per pixel: about 1e-5 per evaluation on the
+# workloads here (the bound is a few e-6 wide in alpha around 1/255). The bar:
+# at most FLAG_RATE flagged pixels per evaluation -- 0.1 % of the pixels at
+# the 1M-Gaussian 1080p workload's 52 evaluations per pixel.
+FLAG_RATE = 2e-5
+
 U24 = 2.0 ** -24
-EXP2_REL_ERR = 2.0 ** -21  # relative error allowed to the SFU's exp2 (ex2.approx)
+# relative error allowed to the SFU exp2: test_sfu_exp2_error_bound measures
+# it over every float argument from 0 to 8 (the largest seen on a B200 is
+# 1.46e-7, at 1.0625)
+EXP2_REL_ERR = 2.0 ** -22
 HALF_LOG2E = 0.5 / np.log(2.0)
 
 
@@ -59,7 +80,7 @@ def alpha_error_bound(projs) -> np.ndarray:
             sk = np.sqrt(np.where(lam2 > 0, lam1 / lam2, 1.0))
         sk = np.where(np.isfinite(sk) & (sk >= 1.0), sk, 1.0)
         e0 = np.log(2.0) * U24 * (3.0 * Qp + 1.0) + EXP2_REL_ERR + 3 * U24
-        e1 = np.log(2.0) * U24 * 8.0 * (1.0 + 0.5 * (sk + 1.0 / sk)) * HALF_LOG2E
+        e1 = np.log(2.0) * U24 * (7.0 + 3.0 * (sk + 1.0 / sk)) * HALF_LOG2E
         out.append(np.stack([e0, e1], -1))
     return np.stack(out)
 

@@ -145,6 +145,14 @@ def test_densify_thresholds_convert_to_the_raw_parameter_units():
     far = (np.abs(s - 0.05) > 1e-5) & (np.abs(o - 0.005) > 1e-6)
     assert np.array_equal((ls > np.float32(dp.log_scale_split))[far], (s > 0.05)[far])
     assert np.array_equal((lg < np.float32(dp.logit_min_opacity))[far], (o < 0.005)[far])
+    L = api.lib()
+    out = api.GsDensifyParams()
+    for bad in ((2e-4, 0.0, 0.005, 1.0, 1.6), (2e-4, 0.05, 0.0, 1.0, 1.6),
+                (2e-4, 0.05, 1.0, 1.0, 1.6), (2e-4, 0.05, 0.005, -1.0, 1.6),
+                (2e-4, 0.05, 0.005, 1.0, 0.0), (2e-4, 0.05, float("nan"), 1.0, 1.6)):
+        assert L.gs_densify_params_from_cutoffs(*bad, ctypes.byref(out)) == api.GS_ERR_INVALID_ARG
+    assert L.gs_densify_params_from_cutoffs(2e-4, 0.05, 0.005, 1.0, 1.6, None) == \
+        api.GS_ERR_INVALID_ARG
     assert 0 < api.gs_densify_workspace_size(1000) < api.gs_densify_workspace_size(10 ** 6)
     assert api.gs_densify_workspace_size(-1) == 0
 

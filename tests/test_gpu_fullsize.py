@@ -59,7 +59,8 @@ def _check_view(sc, sp, v, proj, ids, ranges, rng, n_pix):
         want = oids[off:off + counts[k]]
         off += counts[k]
         s, e = ranges[v * tpv + t]
-        assert np.array_equal(ids[s:e].astype(np.int64), want.astype(np.int64)), (v, t)
+        got = ids[int(s):int(e)].cpu().numpy()  # the tile's slice only (ids can be GBs)
+        assert np.array_equal(got.astype(np.int64), want.astype(np.int64)), (v, t)
     # sampled pixels of this view
     pix = _sample(cam.width, cam.height, 0, n_pix, rng)
     bound = P.alpha_error_bound([proj])
@@ -68,8 +69,8 @@ def _check_view(sc, sp, v, proj, ids, ranges, rng, n_pix):
     fT = sp.final_T[v].cpu().numpy()[None]
     nc = sp.n_contrib[v].cpu().numpy()[None]
     st = P.compare_render(img, fT, nc, ref, pix, P.colour_max([proj], sc.background))
-    print("view", v, st)
-    assert st["flagged"] <= 1e-3 * st["n"]
+    print("view", v, st, "evaluations per pixel %.1f" % ref["n_exp"].mean())
+    assert st["flagged"] <= P.FLAG_RATE * ref["n_exp"].sum()
     assert st["max_abs"] <= P.MAX_ABS and st["mean_abs"] <= P.MEAN_ABS
     assert st["nc_mismatch"] == 0 and st["T_max_rel"] < 1e-3
     assert st["flagged_excess"] <= 0.0 and st["flagged_T_excess"] <= 0.0
@@ -95,7 +96,7 @@ def _run_case(name, mode, n_pix, adam):
     n_pairs = int(sp.n_pairs.item())
     assert n_pairs == need
     print(name, "pairs", n_pairs)
-    ids = sp.ids.cpu().numpy()
+    ids = sp.ids
     ranges = sp.ranges.cpu().numpy()
     rng = np.random.default_rng(17)
     total = 0
@@ -108,7 +109,6 @@ def _run_case(name, mode, n_pix, adam):
         pix_by_view.append(_check_view(sc, sp, v, proj, ids, ranges, rng, n_pix))
         del proj
     assert n_pairs == total
-    del ids
     # backward of an upstream gradient on the sampled pixels
     dL = _upstream(sc, pix_by_view)
     sp.rasterize_bwd(torch.as_tensor(dL).cuda())
@@ -138,9 +138,10 @@ def _run_case(name, mode, n_pix, adam):
         e = P.rel_l2(g2_gpu[..., f], g2_ref[..., f])
         assert e < P.REL_L2, ("grad2d field", f, e)
     # parameter gradients of the touched Gaussians (every other one is 0)
-    sub = S.make_scene(name)
+    import copy
+    sub = copy.copy(sc)
     for k in ("means", "log_scales", "quats", "opacity_logit", "sh"):
-        setattr(sub, k, np.ascontiguousarray(getattr(sub, k)[touched]))
+        setattr(sub, k, np.ascontiguousarray(getattr(sc, k)[touched]))
     projs_sub = O.project_views(sub)
     gr = O.project_bwd(sub, projs_sub, g2_ref)
     tt = torch.as_tensor(touched).cuda()
@@ -150,9 +151,9 @@ def _run_case(name, mode, n_pix, adam):
             gpu = gpu[:, :3]
         e = P.rel_l2(gpu.reshape(gr[k].shape), gr[k])
         assert e < P.REL_L2, (k, e)
-        rest = t.clone()
-        rest[tt] = 0
-        assert not rest.any(), k
+        keep = torch.ones(t.shape[0], dtype=torch.bool, device="cuda")
+        keep[tt] = False
+        assert not t[keep].any(), k
     # densify statistics summed over the views
     plain, absg, _ = O.densify_stats(g2_ref, np.stack(valid)[:, touched])
     assert P.rel_l2(sp.accum_plain[tt].cpu().numpy(), plain) < P.REL_L2

@@ -4,6 +4,8 @@ Small cases run the whole image; larger ones a seeded pixel sample plus full
 tile rows. Every case spans several tiles and a ragged last tile row/column.
 """
 
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -163,7 +165,9 @@ def test_render_matches_oracle(name, kw, how):
     # flagged: a decision within the kernel's written error bound of its
     # threshold; such a pixel is still checked against what the decisions
     # can change
-    assert st["flagged"] <= 1e-3 * st["n"]
+    assert st["flagged"] <= P.FLAG_RATE * ref["n_exp"].sum()
+    if name == "train_1m_1080p" and not kw:
+        assert st["flagged"] <= 1e-3 * st["n"]   # the benchmark workload at full size
     assert st["ambiguous"] == 0
     assert st["max_abs"] <= P.MAX_ABS
     assert st["mean_abs"] <= P.MEAN_ABS
@@ -404,6 +408,25 @@ def test_alpha_within_written_bound():
     print("alpha rel err: max %.2e, max / bound %.3f, median bound %.2e" % (
         rel.max(), (rel / lim).max(), np.median(lim)))
     assert np.all(rel <= lim)
+
+
+def test_sfu_exp2_error_bound(tmp_path):
+    """The float exp2 the rasteriser calls (exp2f built with --use_fast_math,
+    the SFU's approximation) over every float argument from 0 to 8 -- all the
+    kernel passes it, since 2^-zq / 255 is only taken where 0 <= -zq <=
+    log2(255) -- stays within the relative error the comparator's bound
+    allows it (parity.EXP2_REL_ERR). Built with the library's own flags."""
+    import shutil
+    import subprocess
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    src = os.path.join(os.path.dirname(__file__), "probes", "exp2_error.cu")
+    exe = str(tmp_path / "exp2_error")
+    subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O3",
+                    "--use_fast_math", src, "-o", exe], check=True)
+    out = subprocess.run([exe, "0", "8"], capture_output=True, text=True, check=True).stdout
+    print(out.strip())
+    err = float(out.split()[1])
+    assert 0.0 < err <= P.EXP2_REL_ERR
 
 
 def test_single_gaussian_centred_on_pixel_gives_o_c():

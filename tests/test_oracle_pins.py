@@ -283,6 +283,55 @@ def test_single_gaussian_centred_on_pixel_gives_o_c():
     assert abs(r["T"][0] - 0.3) < 1e-15 and r["n_contrib"][0] == 1
 
 
+def test_render_flags_follow_the_given_error_bound():
+    """The comparator inputs of orc_render: with a per-splat relative alpha
+    error bound e, an evaluation whose alpha lies within e of 1/255 is
+    flagged and one outside is not; a trial transmittance is flagged within
+    the transmittance bound the alphas in front imply; flag_dev / flag_T add
+    up what a flagged decision can change (2.02 T a and T a / (1 - a) for a
+    skip, 2.02 T and T for a stop)."""
+    cam = _cam(W=32, H=32)
+    bg = np.zeros(3)
+    pix = np.array([[0, 10, 7]])
+    # one splat centred on the pixel: alpha = o exactly
+    for rel, flagged in ((3e-6, True), (-3e-6, True), (2e-5, False), (-2e-5, False)):
+        o = (1.0 / 255.0) * (1.0 + rel)
+        p = _proj2d([[10.5, 7.5]], [[0.3, 0.1, 0.2]], [o], [[1.0, 1.0, 1.0]], [1.0], 32, 32)
+        err = np.array([[[1e-5, 0.0]]])
+        r = O.render([p], [cam], bg, pix, alpha_err=err)
+        assert bool(r["flags"][0] & 1) == flagged, rel
+        assert (r["flags"][0] & 2) == 0
+        if flagged:
+            np.testing.assert_allclose(r["flag_dev"][0], 2.02 * max(o, 1 / 255.0), rtol=1e-12)
+            a = max(o, 1 / 255.0)
+            np.testing.assert_allclose(r["flag_T"][0], a / (1 - a), rtol=1e-12)
+        else:
+            assert r["flag_dev"][0] == 0.0 and r["flag_T"][0] == 0.0
+        # without a bound nothing is flagged
+        assert O.render([p], [cam], bg, pix)["flags"][0] == 0
+    # the bound grows with q: one pixel away from the centre (q = 0.3),
+    # alpha 4e-6 above 1/255 is inside e1 q for e1 = 2e-5, outside for 1e-5
+    a = 0.3
+    q = a * 1.0 * 1.0
+    o_edge = (1.0 / 255.0) * (1 + 4e-6) / math.exp(-0.5 * q)
+    p = _proj2d([[11.5, 7.5]], [[a, 0.0, a]], [o_edge], [[1.0, 1.0, 1.0]], [1.0], 32, 32)
+    assert O.render([p], [cam], bg, pix, alpha_err=np.array([[[0.0, 2e-5]]]))["flags"][0] & 1
+    assert not O.render([p], [cam], bg, pix, alpha_err=np.array([[[0.0, 1e-5]]]))["flags"][0]
+    # a layer of alpha 0.99 leaves T = 0.01 in front of a second of alpha
+    # 0.99 - 1e-9, whose trial T is a hair (1e-7 relative) above 1e-4: flagged
+    # with a bound, not without
+    xy = [[10.5, 7.5]] * 3
+    opac = [0.99, 0.99 - 1e-9, 0.5]
+    p = _proj2d(xy, [[0.3, 0.0, 0.3]] * 3, opac, [[1.0, 0.0, 0.0]] * 3, [1.0, 2.0, 3.0], 32, 32)
+    r0 = O.render([p], [cam], bg, pix)
+    assert r0["flags"][0] == 0 and r0["n_contrib"][0] == 2
+    r1 = O.render([p], [cam], bg, pix, alpha_err=np.full((1, 3, 2), [1e-6, 0.0]))
+    assert r1["flags"][0] & 2
+    # the stop taken the other way at the second splat, with T = 0.01 in front
+    np.testing.assert_allclose(r1["flag_T"][0], 0.01, rtol=1e-9)
+    np.testing.assert_allclose(r1["flag_dev"][0], 2.02 * 0.01, rtol=1e-9)
+
+
 def test_two_gaussians_front_to_back():
     cam = _cam(W=32, H=32)
     p = _proj2d([[10.2, 7.9], [11.0, 6.5]], [[0.3, 0.1, 0.2], [0.1, -0.02, 0.15]], [0.6, 0.8],
