@@ -1,21 +1,24 @@
 // raster.cu -- tile rasteriser, forward and backward, sm_100a.
 //
-// One 16x16 tile per 128-thread block ("Better Gaussian Splatting in Julia",
+// One 16x16 tile per thread block ("Better Gaussian Splatting in Julia",
 // pwwt.cn sec. 5.4: a pixel block per thread group, each group compositing
-// serially, groups in parallel -- no atomics on pixels). Each warp owns an 8x8
-// pixel block of the tile and each thread two pixels of one column, four rows
-// apart: (x, y) and (x, y + 4). The pair shares its x offset from every
-// Gaussian centre, and its per-pixel arithmetic runs two-wide on the FP32x2
-// pipe (__ffma2_rn / __fadd2_rn / __fmul2_rn: each half rounds exactly like
-// the scalar operation, so pixel results do not depend on the pairing).
+// serially, groups in parallel -- no atomics on pixels). Each thread takes
+// 2 NP pixels of one column, four rows apart -- (x, y), (x, y + 4), ...,
+// (x, y + 4 (2 NP - 1)) -- so a warp owns an 8-column block of 8 NP rows and
+// a tile has 4 / NP warps. A thread's pixels share their x offset from every
+// Gaussian centre (and with it half of the evaluation), and the per-pixel
+// arithmetic runs two-wide on the FP32x2 pipe (__ffma2_rn / __fadd2_rn /
+// __fmul2_rn: each half rounds exactly like the scalar operation, so pixel
+// results do not depend on the grouping).
 //
-// The tile's depth-sorted list is consumed in batches of 128 records; each
-// thread stages one 64-byte record into shared memory with a TMA bulk copy
-// (cp.async.bulk completing on an mbarrier). When a batch lands, thread j
-// marks which warps' pixel blocks record j's alpha >= 1/255 box reaches;
-// every warp then compacts the batch to the records that can touch its
-// pixels (ballot + popc, order kept) and walks only those. The box is
-// conservative, so the skipped records are exactly ones every pixel of the
+// The tile's depth-sorted list is consumed in batches of one record per
+// thread; each thread stages one 64-byte record into shared memory with a TMA
+// bulk copy (cp.async.bulk completing on an mbarrier). When a batch lands,
+// thread j marks which warps' pixel blocks record j's alpha >= 1/255 ellipse
+// reaches (its bounding box, then the ellipse itself against the block's
+// rectangle); every warp then compacts the batch to the records that can
+// touch its pixels (ballot + popc, order kept) and walks only those. The test
+// is conservative, so the skipped records are exactly ones every pixel of the
 // block would skip. The forward copies each landed record into a separate
 // array of (x, x) pairs, so the landing buffer is free for the next batch's
 // copy at once; the backward reads records in place and double-buffers.
@@ -44,9 +47,9 @@
 //   dC/dc_k = alpha_k T_k,
 //   dC/dalpha_k = T_k (c_k - B_k) - T_final bg / (1 - alpha_k),
 //   B_{k-1} = B_k + alpha_k (c_k - B_k).
-// Per Gaussian a thread adds its two pixels' ten terms, the warp sums its
-// lanes with a transposing butterfly (14 shuffles), the block sums its warps
-// in shared memory, and three 4-float vector atomics go to global memory.
+// Per Gaussian a thread adds its pixels' ten terms, the warp sums its lanes
+// with a transposing butterfly (14 shuffles), the block sums its warps in
+// shared memory, and three 4-float vector atomics go to global memory.
 
 #include <cuda_runtime.h>
 
@@ -55,18 +58,30 @@
 namespace gsb {
 namespace {
 
-constexpr int kThreads = 128;                    // 4 warps, 8x8 pixels each
-constexpr int kWarps = kThreads / 32;
-constexpr int kBatch = kThreads;                 // records per batch
+// Pixel pairs per thread of the kernels launched: 1 (two pixels per thread,
+// 128-thread blocks of four warps, each warp an 8 x 8 pixel block). Two pairs
+// (64-thread blocks, 8 x 16 blocks per warp) measured slower on the 1M-splat
+// 1080p frame: forward 0.308 against 0.303 ms, backward 0.613 against 0.584
+// ms -- fewer resident warps (80 and 111 registers) and longer warp lists
+// outweigh the evaluation and reduction shared by four pixels.
+constexpr int kPairs = 1;
+
+template <int NP>
+struct Shape {
+  static constexpr int kThreads = 128 / NP;      // 2 NP pixels per thread, 256 per tile
+  static constexpr int kWarps = kThreads / 32;   // 4 / NP
+  static constexpr int kBatch = kThreads;        // records per batch: one per thread
+  static constexpr int kBlockRows = 8 * NP;      // a warp's block: 8 columns x kBlockRows rows
+};
+
 constexpr int kRecBytes = GS_RECORD_FLOATS * 4;  // 64
 constexpr float kInv255 = 1.0f / 255.0f;
 constexpr float kTwoLn2 = 1.3862943611198906f;   // 1 / (log2(e) / 2)
 
-static_assert(kTilePixels == 2 * kThreads, "two pixels per thread");
 static_assert(kRecBytes % 16 == 0, "bulk copies move multiples of 16 bytes");
 
 // Forward evaluation form of a record, one (x, x) pair per field, so the
-// two-pixel arithmetic takes every operand straight from shared memory:
+// multi-pixel arithmetic takes every operand straight from shared memory:
 // -uh, -vh, w1x, w1y, c1, w2x, w2y, c2, nlo, colour r g b. 96 bytes.
 enum EvPair { V_NU = 0, V_NV, V_W1X, V_W1Y, V_C1, V_W2X, V_W2Y, V_C2, V_NLO, V_R, V_G, V_BL,
               kEvPairs };
@@ -95,14 +110,17 @@ __device__ __forceinline__ void tile_range(const int64_t* ranges, int tile, int6
   }
 }
 
-// The thread's pixel pair: (px, py) and (px, py + 4).
+// The thread's pixels: column px, rows py + 4 i for i < 2 NP; pair k holds
+// rows py + 8k and py + 8k + 4.
+template <int NP>
 struct TilePix {
   int view, x0, y0, px, py;
-  bool in0, in1;
+  bool in[2 * NP];
 };
 
-__device__ __forceinline__ TilePix tile_pixel(const Grid& g, int tile) {
-  TilePix t;
+template <int NP>
+__device__ __forceinline__ TilePix<NP> tile_pixel(const Grid& g, int tile) {
+  TilePix<NP> t;
   t.view = tile / g.tiles_per_view;
   const int tt = tile - t.view * g.tiles_per_view;
   const int ty = tt / g.tiles_x;
@@ -110,45 +128,52 @@ __device__ __forceinline__ TilePix tile_pixel(const Grid& g, int tile) {
   t.y0 = ty * kTile;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   t.px = t.x0 + 8 * (warp & 1) + (lane & 7);
-  t.py = t.y0 + 8 * (warp >> 1) + (lane >> 3);
-  t.in0 = t.px < g.width && t.py < g.height;
-  t.in1 = t.px < g.width && t.py + 4 < g.height;
+  t.py = t.y0 + Shape<NP>::kBlockRows * (warp >> 1) + (lane >> 3);
+#pragma unroll
+  for (int i = 0; i < 2 * NP; ++i) t.in[i] = t.px < g.width && t.py + 4 * i < g.height;
   return t;
 }
 
-// 4-bit mask of the warps whose 8x8 pixel block the alpha >= 1/255 box
-// [u - hx, u + hx] x [v - hy, v + hy] overlaps, on pixel-centre extents (a
-// record without a box, hx < 0 or NaN, reaches none).
+// Mask of the warps whose pixel block (8 columns x kBlockRows rows) the
+// alpha >= 1/255 box [u - hx, u + hx] x [v - hy, v + hy] overlaps, on
+// pixel-centre extents (a record without a box, hx < 0 or NaN, reaches none).
+template <int NP>
 __device__ __forceinline__ uint32_t warp_block_mask(float u, float v, float hx, float hy, int x0,
                                                     int y0) {
+  constexpr int R = Shape<NP>::kBlockRows;
   if (!(hx >= 0.f)) return 0u;
   uint32_t xm = 0, ym = 0;
 #pragma unroll
   for (int bi = 0; bi < 2; ++bi) {
     const float xlo = (float)(x0 + 8 * bi) + 0.5f, xhi = xlo + 7.f;
     if (u + hx >= xlo && u - hx <= xhi) xm |= 1u << bi;
-    const float ylo = (float)(y0 + 8 * bi) + 0.5f, yhi = ylo + 7.f;
+  }
+#pragma unroll
+  for (int bi = 0; bi < kTile / R; ++bi) {
+    const float ylo = (float)(y0 + R * bi) + 0.5f, yhi = ylo + (float)(R - 1);
     if (v + hy >= ylo && v - hy <= yhi) ym |= 1u << bi;
   }
   uint32_t mask = 0;
 #pragma unroll
-  for (int w = 0; w < kWarps; ++w)
+  for (int w = 0; w < Shape<NP>::kWarps; ++w)
     if (((xm >> (w & 1)) & 1u) && ((ym >> (w >> 1)) & 1u)) mask |= 1u << w;
   return mask;
 }
 
-// Refines warp_block_mask with the ellipse itself: a warp's 8x8 block of
-// pixel centres [xlo, xlo + 7] x [ylo, ylo + 7] keeps the splat only if the
-// quadratic q'(d) = (w1 . d)^2 + (w2 . d)^2 (d from the float mean) reaches
-// at most Q' = -nlo somewhere on that rectangle: 0 when the mean is inside,
-// else the least value over the four edges (on an edge q' is a parabola in
-// the free coordinate, minimised at its vertex clamped to the edge). Q' is
-// padded (0.2 % + 0.01) well beyond the float rounding of the rasteriser's zq
-// and the mean's float remainder, so no pixel the per-pixel test takes is
-// dropped; the axis-aligned box keeps, on average, ~40 % more (warp, splat)
-// pairs whose ellipse misses the block.
+// Refines warp_block_mask with the ellipse itself: a warp's block of pixel
+// centres [xlo, xlo + 7] x [ylo, ylo + kBlockRows - 1] keeps the splat only
+// if the quadratic q'(d) = (w1 . d)^2 + (w2 . d)^2 (d from the float mean)
+// reaches at most Q' = -nlo somewhere on that rectangle: 0 when the mean is
+// inside, else the least value over the four edges (on an edge q' is a
+// parabola in the free coordinate, minimised at its vertex clamped to the
+// edge). Q' is padded (0.2 % + 0.01) well beyond the float rounding of the
+// rasteriser's zq and the mean's float remainder, so no pixel the per-pixel
+// test takes is dropped; the axis-aligned box alone keeps ~40 % more (warp,
+// splat) pairs, whose ellipse misses the block.
+template <int NP>
 __device__ __forceinline__ uint32_t warp_block_mask_ellipse(const float* r, uint32_t box, int x0,
                                                             int y0) {
+  constexpr int R = Shape<NP>::kBlockRows;
   if (box == 0u) return 0u;
   const float w1x = r[R_W1X], w1y = r[R_W1Y], w2x = r[R_W2X], w2y = r[R_W2Y];
   const float a = fmaf(w1x, w1x, w2x * w2x), b = fmaf(w1x, w1y, w2x * w2y);
@@ -158,10 +183,10 @@ __device__ __forceinline__ uint32_t warp_block_mask_ellipse(const float* r, uint
   const float u = r[R_U], v = r[R_V];
   uint32_t mask = 0;
 #pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
+  for (int w = 0; w < Shape<NP>::kWarps; ++w) {
     if (!((box >> w) & 1u)) continue;
     const float ex0 = (float)(x0 + 8 * (w & 1)) + 0.5f - u, ex1 = ex0 + 7.f;
-    const float ey0 = (float)(y0 + 8 * (w >> 1)) + 0.5f - v, ey1 = ey0 + 7.f;
+    const float ey0 = (float)(y0 + R * (w >> 1)) + 0.5f - v, ey1 = ey0 + (float)(R - 1);
     bool hit = ex0 <= 0.f && ex1 >= 0.f && ey0 <= 0.f && ey1 >= 0.f;
     float best = __int_as_float(0x7f800000);
 #pragma unroll
@@ -179,22 +204,32 @@ __device__ __forceinline__ uint32_t warp_block_mask_ellipse(const float* r, uint
   return mask;
 }
 
-// zq at the pair's pixel centres (pxc, pyc.x) and (pxc, pyc.y):
-//   dx = pxc - uh, dy = pyc - vh, p_i = fma(w_iy, dy, fma(w_ix, dx, c_i)),
-//   zq = fma(p1, p1, fma(p2, p2, nlo)).
+// The pixel-independent part of the evaluation at column pxc: dx = pxc - uh
+// and a_i = fma(w_ix, dx, c_i), as (x, x) pairs.
+struct EvCol {
+  float2 a1, a2;
+};
+
+__device__ __forceinline__ EvCol eval_col(const float2* e, float2 pxc) {
+  const float2 dx = __fadd2_rn(pxc, e[V_NU]);
+  return EvCol{__ffma2_rn(e[V_W1X], dx, e[V_C1]), __ffma2_rn(e[V_W2X], dx, e[V_C2])};
+}
+
+// zq of a pixel pair of that column at rows pyc.x, pyc.y:
+//   dy = pyc - vh, p_i = fma(w_iy, dy, a_i), zq = fma(p1, p1, fma(p2, p2, nlo)).
 // The backward evaluates the same IEEE operations in the same order
 // (eval_zq_s), so the skip / stop decisions of the two directions agree bit
 // for bit.
-__device__ __forceinline__ float2 eval_zq(const float2* e, float2 pxc, float2 pyc) {
-  const float2 dx = __fadd2_rn(pxc, e[V_NU]);
+__device__ __forceinline__ float2 eval_zq(const float2* e, const EvCol& col, float2 pyc) {
   const float2 dy = __fadd2_rn(pyc, e[V_NV]);
-  const float2 p1 = __ffma2_rn(e[V_W1Y], dy, __ffma2_rn(e[V_W1X], dx, e[V_C1]));
-  const float2 p2 = __ffma2_rn(e[V_W2Y], dy, __ffma2_rn(e[V_W2X], dx, e[V_C2]));
+  const float2 p1 = __ffma2_rn(e[V_W1Y], dy, col.a1);
+  const float2 p2 = __ffma2_rn(e[V_W2Y], dy, col.a2);
   return __ffma2_rn(p1, p1, __ffma2_rn(p2, p2, e[V_NLO]));
 }
 
-// Write the forward evaluation form of landed record r and return the 4-bit
-// mask of warps whose 8x8 pixel block its alpha >= 1/255 box overlaps.
+// Write the forward evaluation form of landed record r and return the mask
+// of warps whose pixel block its alpha >= 1/255 ellipse reaches.
+template <int NP>
 __device__ __forceinline__ uint32_t prepare_record(const float* r, float2* e, int x0, int y0) {
   const float u = r[R_U], v = r[R_V];
   float4* e4 = reinterpret_cast<float4*>(e);
@@ -204,29 +239,37 @@ __device__ __forceinline__ uint32_t prepare_record(const float* r, float2* e, in
   e4[3] = make_float4(r[R_W2Y], r[R_W2Y], r[R_C2], r[R_C2]);
   e4[4] = make_float4(r[R_NLO], r[R_NLO], r[R_R], r[R_R]);
   e4[5] = make_float4(r[R_G], r[R_G], r[R_B], r[R_B]);
-  return warp_block_mask_ellipse(r, warp_block_mask(u, v, r[R_HX], r[R_HY], x0, y0), x0, y0);
+  return warp_block_mask_ellipse<NP>(r, warp_block_mask<NP>(u, v, r[R_HX], r[R_HY], x0, y0), x0,
+                                     y0);
 }
 
-// eval_zq on a record in its stored (scalar) form: per pixel the same IEEE
-// operations in the same order (the column offset dx and the inner fmas are
-// shared by the pair); also returns dx, dy and p1, p2 for the gradients.
-__device__ __forceinline__ float2 eval_zq_s(const float* r, float pxc, float2 pyc, float& dx,
-                                            float2& dy, float2& p1, float2& p2) {
+// eval_col / eval_zq on a record in its stored (scalar) form, the same IEEE
+// operations in the same order (the column part shared by the thread's
+// pixels); also returns dx, dy and p1, p2 for the gradients.
+__device__ __forceinline__ void eval_col_s(const float* r, float pxc, float& dx, float& a1,
+                                           float& a2) {
   dx = __fsub_rn(pxc, r[R_U]);
+  a1 = __fmaf_rn(r[R_W1X], dx, r[R_C1]);
+  a2 = __fmaf_rn(r[R_W2X], dx, r[R_C2]);
+}
+
+__device__ __forceinline__ float2 eval_zq_s(const float* r, float a1, float a2, float2 pyc,
+                                            float2& dy, float2& p1, float2& p2) {
   dy = __fadd2_rn(pyc, f2(-r[R_V]));
-  p1 = __ffma2_rn(f2(r[R_W1Y]), dy, f2(__fmaf_rn(r[R_W1X], dx, r[R_C1])));
-  p2 = __ffma2_rn(f2(r[R_W2Y]), dy, f2(__fmaf_rn(r[R_W2X], dx, r[R_C2])));
+  p1 = __ffma2_rn(f2(r[R_W1Y]), dy, f2(a1));
+  p2 = __ffma2_rn(f2(r[R_W2Y]), dy, f2(a2));
   return __ffma2_rn(p1, p1, __ffma2_rn(p2, p2, f2(r[R_NLO])));
 }
 
-// Warp-wide compaction of the batch entries whose mask has this warp's bit,
-// in batch order. Returns the count.
+// Warp-wide compaction of the batch entries j < m whose mask has this warp's
+// bit, in batch order. Returns the count.
+template <int NP>
 __device__ __forceinline__ int warp_list(const uint8_t* s_mask, uint8_t* list, int m) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t lt = lanemask_lt();
   int cnt = 0;
 #pragma unroll
-  for (int c = 0; c < kBatch / 32; ++c) {
+  for (int c = 0; c < Shape<NP>::kBatch / 32; ++c) {
     const int j = c * 32 + lane;
     const bool bit = j < m && ((s_mask[j] >> warp) & 1u);
     const uint32_t bal = __ballot_sync(0xffffffffu, bit);
@@ -237,19 +280,22 @@ __device__ __forceinline__ int warp_list(const uint8_t* s_mask, uint8_t* list, i
   return cnt;
 }
 
-__global__ void __launch_bounds__(kThreads) k_raster_fwd(
+template <int NP>
+__global__ void __launch_bounds__(Shape<NP>::kThreads) k_raster_fwd(
     const float* __restrict__ records, const uint32_t* __restrict__ ids,
     const int64_t* __restrict__ ranges, RasterGeom geo, float bg0, float bg1, float bg2,
     float* __restrict__ image, float* __restrict__ final_T, uint32_t* __restrict__ n_contrib,
     uint32_t* __restrict__ status, WaitCfg wc) {
+  using Sh = Shape<NP>;
+  constexpr int kBatch = Sh::kBatch;
   __shared__ __align__(128) float s_rec[kBatch][GS_RECORD_FLOATS];
   __shared__ __align__(16) float2 s_ev[kBatch][kEvPairs];
   __shared__ __align__(8) uint64_t s_bar;
   __shared__ uint8_t s_mask[kBatch];
-  __shared__ uint8_t s_list[kWarps][kBatch];
+  __shared__ uint8_t s_list[Sh::kWarps][kBatch];
 
   const int tile = blockIdx.x;
-  const TilePix tp = tile_pixel(geo.g, tile);
+  const TilePix<NP> tp = tile_pixel<NP>(geo.g, tile);
   int64_t start, end;
   tile_range(ranges, tile, geo.capacity, start, end, status);
   const int64_t cnt = end - start;
@@ -289,14 +335,26 @@ __global__ void __launch_bounds__(kThreads) k_raster_fwd(
 
   const float kInf = __int_as_float(0x7f800000);
   const float2 pxc = f2((float)tp.px + 0.5f);
-  const float2 pyc = make_float2((float)tp.py + 0.5f, (float)tp.py + 4.5f);
-  const float2 one = f2(1.f), mone = f2(-1.f);
-  float2 T = one, c0 = f2(0.f), c1 = f2(0.f), c2 = f2(0.f);
-  uint32_t last0 = 0, last1 = 0;
+  float2 pyc[NP];
+  float2 T[NP], c0[NP], c1[NP], c2[NP];
+  uint32_t last[2 * NP];
   // a pixel takes a splat when zq <= its threshold: 0 while it composites,
   // -inf once it is done (or outside the image)
-  float thr0 = tp.in0 ? 0.f : -kInf, thr1 = tp.in1 ? 0.f : -kInf;
-  bool done = !(tp.in0 || tp.in1);
+  float thr[2 * NP];
+  bool done = true;
+#pragma unroll
+  for (int k = 0; k < NP; ++k) {
+    pyc[k] = make_float2((float)(tp.py + 8 * k) + 0.5f, (float)(tp.py + 8 * k) + 4.5f);
+    T[k] = f2(1.f);
+    c0[k] = c1[k] = c2[k] = f2(0.f);
+  }
+#pragma unroll
+  for (int i = 0; i < 2 * NP; ++i) {
+    last[i] = 0;
+    thr[i] = tp.in[i] ? 0.f : -kInf;
+    done = done && !tp.in[i];
+  }
+  const float2 one = f2(1.f), mone = f2(-1.f);
   bool pending = false;  // batch b's copy is in flight
   if (nb > 0) {
     issue(0);
@@ -311,8 +369,8 @@ __global__ void __launch_bounds__(kThreads) k_raster_fwd(
     const int64_t rem = cnt - (int64_t)b * kBatch;
     const int m = rem < kBatch ? (int)rem : kBatch;
     if ((int)threadIdx.x < m) {
-      const uint32_t mask = prepare_record(&s_rec[threadIdx.x][0], &s_ev[threadIdx.x][0], tp.x0,
-                                           tp.y0);
+      const uint32_t mask = prepare_record<NP>(&s_rec[threadIdx.x][0], &s_ev[threadIdx.x][0],
+                                               tp.x0, tp.y0);
       s_mask[threadIdx.x] = clipped ? 0u : (uint8_t)mask;
     }
     __syncthreads();  // s_rec is free again
@@ -320,42 +378,62 @@ __global__ void __launch_bounds__(kThreads) k_raster_fwd(
       issue(b + 1);
       pending = !stalled;
     }
-    const int wc_n = warp_list(s_mask, s_list[warp], m);
+    const int wc_n = warp_list<NP>(s_mask, s_list[warp], m);
     const uint32_t pos0 = (uint32_t)(b * kBatch + 1);
     for (int k = 0; k < wc_n; ++k) {
       if ((k & 3) == 0 && __all_sync(0xffffffffu, done)) break;  // warp vote
       const int j = s_list[warp][k];
       const float2* e = &s_ev[j][0];
-      const float2 zq = eval_zq(e, pxc, pyc);
-      bool ok0 = zq.x <= thr0, ok1 = zq.y <= thr1;
-      if (!(ok0 || ok1)) continue;
-      float2 a = make_float2(ok0 ? fminf(kAlphaMax, alpha_raw_of(zq.x)) : 0.f,
-                             ok1 ? fminf(kAlphaMax, alpha_raw_of(zq.y)) : 0.f);
-      float2 Tn = __fmul2_rn(T, __ffma2_rn(a, mone, one));  // T (1 - alpha)
-      if (Tn.x < kTMin || Tn.y < kTMin) {
-        // the pixel stops before this Gaussian: it takes no part in it
-        if (Tn.x < kTMin) {
-          a.x = 0.f;
-          Tn.x = T.x;
-          thr0 = -kInf;
-          ok0 = false;
-        }
-        if (Tn.y < kTMin) {
-          a.y = 0.f;
-          Tn.y = T.y;
-          thr1 = -kInf;
-          ok1 = false;
-        }
-        done = thr0 == -kInf && thr1 == -kInf;
+      const EvCol col = eval_col(e, pxc);
+      float2 zq[NP];
+      bool ok[2 * NP];
+      bool any = false;
+#pragma unroll
+      for (int q = 0; q < NP; ++q) {
+        zq[q] = eval_zq(e, col, pyc[q]);
+        ok[2 * q] = zq[q].x <= thr[2 * q];
+        ok[2 * q + 1] = zq[q].y <= thr[2 * q + 1];
+        any = any || ok[2 * q] || ok[2 * q + 1];
       }
-      const float2 w = __fmul2_rn(a, T);
-      c0 = __ffma2_rn(e[V_R], w, c0);
-      c1 = __ffma2_rn(e[V_G], w, c1);
-      c2 = __ffma2_rn(e[V_BL], w, c2);
-      T = Tn;
+      if (!any) continue;
       const uint32_t pos1 = pos0 + (uint32_t)j;
-      last0 = ok0 ? pos1 : last0;
-      last1 = ok1 ? pos1 : last1;
+      bool stop = false;
+#pragma unroll
+      for (int q = 0; q < NP; ++q) {
+        bool o0 = ok[2 * q], o1 = ok[2 * q + 1];
+        float2 a = make_float2(o0 ? fminf(kAlphaMax, alpha_raw_of(zq[q].x)) : 0.f,
+                               o1 ? fminf(kAlphaMax, alpha_raw_of(zq[q].y)) : 0.f);
+        float2 Tn = __fmul2_rn(T[q], __ffma2_rn(a, mone, one));  // T (1 - alpha)
+        if (Tn.x < kTMin || Tn.y < kTMin) {
+          // the pixel stops before this Gaussian: it takes no part in it
+          if (Tn.x < kTMin) {
+            a.x = 0.f;
+            Tn.x = T[q].x;
+            thr[2 * q] = -kInf;
+            o0 = false;
+          }
+          if (Tn.y < kTMin) {
+            a.y = 0.f;
+            Tn.y = T[q].y;
+            thr[2 * q + 1] = -kInf;
+            o1 = false;
+          }
+          stop = true;
+        }
+        const float2 w = __fmul2_rn(a, T[q]);
+        c0[q] = __ffma2_rn(e[V_R], w, c0[q]);
+        c1[q] = __ffma2_rn(e[V_G], w, c1[q]);
+        c2[q] = __ffma2_rn(e[V_BL], w, c2[q]);
+        T[q] = Tn;
+        last[2 * q] = o0 ? pos1 : last[2 * q];
+        last[2 * q + 1] = o1 ? pos1 : last[2 * q + 1];
+      }
+      if (stop) {
+        bool d = true;
+#pragma unroll
+        for (int i = 0; i < 2 * NP; ++i) d = d && thr[i] == -kInf;
+        done = d;
+      }
     }
   }
   // a batch issued but not consumed must land before the block exits
@@ -365,21 +443,17 @@ __global__ void __launch_bounds__(kThreads) k_raster_fwd(
   float* img = image + (size_t)tp.view * 3 * hw;
   float* tf = final_T + (size_t)tp.view * hw;
   uint32_t* nc = n_contrib + (size_t)tp.view * hw;
-  if (tp.in0) {
-    const size_t pix = (size_t)tp.py * geo.g.width + tp.px;
-    img[pix] = fmaf(T.x, bg0, c0.x);
-    img[hw + pix] = fmaf(T.x, bg1, c1.x);
-    img[2 * hw + pix] = fmaf(T.x, bg2, c2.x);
-    tf[pix] = T.x;
-    nc[pix] = last0;
-  }
-  if (tp.in1) {
-    const size_t pix = (size_t)(tp.py + 4) * geo.g.width + tp.px;
-    img[pix] = fmaf(T.y, bg0, c0.y);
-    img[hw + pix] = fmaf(T.y, bg1, c1.y);
-    img[2 * hw + pix] = fmaf(T.y, bg2, c2.y);
-    tf[pix] = T.y;
-    nc[pix] = last1;
+#pragma unroll
+  for (int i = 0; i < 2 * NP; ++i) {
+    if (!tp.in[i]) continue;
+    const int q = i >> 1;
+    const float Ti = (i & 1) ? T[q].y : T[q].x;
+    const size_t pix = (size_t)(tp.py + 4 * i) * geo.g.width + tp.px;
+    img[pix] = fmaf(Ti, bg0, (i & 1) ? c0[q].y : c0[q].x);
+    img[hw + pix] = fmaf(Ti, bg1, (i & 1) ? c1[q].y : c1[q].x);
+    img[2 * hw + pix] = fmaf(Ti, bg2, (i & 1) ? c2[q].y : c2[q].x);
+    tf[pix] = Ti;
+    nc[pix] = last[i];
   }
 }
 
@@ -411,12 +485,16 @@ __device__ __forceinline__ void warp_sum10(const float (&v)[10], float& t0, floa
   t1 = c1;
 }
 
-__global__ void __launch_bounds__(kThreads) k_raster_bwd(
+template <int NP>
+__global__ void __launch_bounds__(Shape<NP>::kThreads) k_raster_bwd(
     const float* __restrict__ records, const uint32_t* __restrict__ ids,
     const int64_t* __restrict__ ranges, RasterGeom geo, float bg0, float bg1, float bg2,
     const float* __restrict__ dL_dimage, const float* __restrict__ final_T,
     const uint32_t* __restrict__ n_contrib, float* __restrict__ grad2d,
     uint32_t* __restrict__ status, WaitCfg wc) {
+  using Sh = Shape<NP>;
+  constexpr int kBatch = Sh::kBatch;
+  constexpr int kWarps = Sh::kWarps;
   __shared__ __align__(128) float s_rec[2][kBatch][GS_RECORD_FLOATS];
   __shared__ __align__(16) float s_acc[kBatch][GS_GRAD2D_FLOATS];
   __shared__ uint32_t s_id[2][kBatch];
@@ -426,10 +504,8 @@ __global__ void __launch_bounds__(kThreads) k_raster_bwd(
   __shared__ uint8_t s_list[kWarps][kBatch];
 
   const int tile = blockIdx.x;
-  const TilePix tp = tile_pixel(geo.g, tile);
+  const TilePix<NP> tp = tile_pixel<NP>(geo.g, tile);
   const size_t hw = (size_t)geo.g.width * geo.g.height;
-  const size_t pix0 = (size_t)tp.py * geo.g.width + tp.px;
-  const size_t pix1 = pix0 + 4 * (size_t)geo.g.width;
   int64_t start, end;
   tile_range(ranges, tile, geo.capacity, start, end, status);
   const float* rec_view = records + (size_t)tp.view * geo.n * GS_RECORD_FLOATS;
@@ -437,37 +513,48 @@ __global__ void __launch_bounds__(kThreads) k_raster_bwd(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool stalled = (int64_t)tile == wc.stall;  // test hook, see k_raster_fwd
 
-  // per-pixel state, pixel 0 in .x and pixel 1 in .y; an outside pixel has
-  // no contributors and zero upstream gradient
-  float2 Tfin = f2(1.f), g0 = f2(0.f), g1 = f2(0.f), g2 = f2(0.f);
-  uint32_t nc0 = 0, nc1 = 0;
+  // per-pixel state, by pixel pairs; an outside pixel has no contributors and
+  // zero upstream gradient
+  float2 Tfin[NP], g0[NP], g1[NP], g2[NP];
+  uint32_t nc[2 * NP];
   {
     const float* tf = final_T + (size_t)tp.view * hw;
-    const uint32_t* nc = n_contrib + (size_t)tp.view * hw;
+    const uint32_t* ncv = n_contrib + (size_t)tp.view * hw;
     const float* gi = dL_dimage + (size_t)tp.view * 3 * hw;
-    if (tp.in0) {
-      Tfin.x = tf[pix0];
-      nc0 = nc[pix0];
-      g0.x = gi[pix0];
-      g1.x = gi[hw + pix0];
-      g2.x = gi[2 * hw + pix0];
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+      Tfin[q] = f2(1.f);
+      g0[q] = g1[q] = g2[q] = f2(0.f);
     }
-    if (tp.in1) {
-      Tfin.y = tf[pix1];
-      nc1 = nc[pix1];
-      g0.y = gi[pix1];
-      g1.y = gi[hw + pix1];
-      g2.y = gi[2 * hw + pix1];
+#pragma unroll
+    for (int i = 0; i < 2 * NP; ++i) {
+      nc[i] = 0;
+      if (!tp.in[i]) continue;
+      const size_t pix = (size_t)(tp.py + 4 * i) * geo.g.width + tp.px;
+      const int q = i >> 1;
+      float* tq = (i & 1) ? &Tfin[q].y : &Tfin[q].x;
+      *tq = tf[pix];
+      nc[i] = ncv[pix];
+      ((i & 1) ? g0[q].y : g0[q].x) = gi[pix];
+      ((i & 1) ? g1[q].y : g1[q].x) = gi[hw + pix];
+      ((i & 1) ? g2[q].y : g2[q].x) = gi[2 * hw + pix];
     }
   }
   // T_final (bg . dL/dC): the background's share of dC/dalpha, before 1/(1-alpha)
-  const float2 tfbg =
-      __fmul2_rn(Tfin, __ffma2_rn(f2(bg2), g2, __ffma2_rn(f2(bg1), g1, __fmul2_rn(f2(bg0), g0))));
-  float2 T = Tfin;
-  float2 acc0 = f2(0.f), acc1 = f2(0.f), acc2 = f2(0.f);  // colour behind
+  float2 tfbg[NP], T[NP], acc0[NP], acc1[NP], acc2[NP];  // acc: colour behind
+#pragma unroll
+  for (int q = 0; q < NP; ++q) {
+    tfbg[q] = __fmul2_rn(Tfin[q], __ffma2_rn(f2(bg2), g2[q],
+                                             __ffma2_rn(f2(bg1), g1[q], __fmul2_rn(f2(bg0), g0[q]))));
+    T[q] = Tfin[q];
+    acc0[q] = acc1[q] = acc2[q] = f2(0.f);
+  }
 
-  // the longest prefix any pixel of the tile used
-  const uint32_t wm = __reduce_max_sync(0xffffffffu, max(nc0, nc1));
+  // the longest prefix any pixel of the warp, and of the tile, used
+  uint32_t mine = 0;
+#pragma unroll
+  for (int i = 0; i < 2 * NP; ++i) mine = max(mine, nc[i]);
+  const uint32_t wm = __reduce_max_sync(0xffffffffu, mine);
   if (lane == 0) s_wmax[warp] = wm;
   if (threadIdx.x == 0) {
     mbar_init(&s_bar[0], 1);
@@ -509,7 +596,10 @@ __global__ void __launch_bounds__(kThreads) k_raster_bwd(
   };
 
   const float pxc = (float)tp.px + 0.5f;
-  const float2 pyc = make_float2((float)tp.py + 0.5f, (float)tp.py + 4.5f);
+  float2 pyc[NP];
+#pragma unroll
+  for (int q = 0; q < NP; ++q)
+    pyc[q] = make_float2((float)(tp.py + 8 * q) + 0.5f, (float)(tp.py + 8 * q) + 4.5f);
   if (nb > 0) issue(0);
   for (int it = 0; it < nb; ++it) {
     const int b = nb - 1 - it;
@@ -524,8 +614,8 @@ __global__ void __launch_bounds__(kThreads) k_raster_bwd(
     pend[buf] = -1;
     if ((int)threadIdx.x < m) {
       float* r = &s_rec[buf][threadIdx.x][0];
-      const uint32_t mask = warp_block_mask_ellipse(
-          r, warp_block_mask(r[R_U], r[R_V], r[R_HX], r[R_HY], tp.x0, tp.y0), tp.x0, tp.y0);
+      const uint32_t mask = warp_block_mask_ellipse<NP>(
+          r, warp_block_mask<NP>(r[R_U], r[R_V], r[R_HX], r[R_HY], tp.x0, tp.y0), tp.x0, tp.y0);
       s_mask[threadIdx.x] = clipped[buf] ? 0u : (uint8_t)mask;
       r[R_OPAC] = 1.f / r[R_OPAC];  // d alpha / d opacity = alpha / o
     }
@@ -536,67 +626,82 @@ __global__ void __launch_bounds__(kThreads) k_raster_bwd(
     __syncthreads();
     // this warp's pixels use no entry at or past the longest prefix among them
     const int64_t wlim = (int64_t)wm - (int64_t)b * kBatch;
-    const int wc_n = warp_list(s_mask, s_list[warp], wlim < m ? (wlim > 0 ? (int)wlim : 0) : m);
+    const int wc_n =
+        warp_list<NP>(s_mask, s_list[warp], wlim < m ? (wlim > 0 ? (int)wlim : 0) : m);
     for (int k = wc_n - 1; k >= 0; --k) {
       const int j = s_list[warp][k];
       const uint32_t pos = (uint32_t)(b * kBatch + j);
       const float* r = &s_rec[buf][j][0];
-      float dx;
-      float2 dy, p1, p2;
-      const float2 zq = eval_zq_s(r, pxc, pyc, dx, dy, p1, p2);
-      const bool ok0 = pos < nc0 && zq.x <= 0.f;
-      const bool ok1 = pos < nc1 && zq.y <= 0.f;
-      const uint32_t bal = __ballot_sync(0xffffffffu, ok0 || ok1);
+      float dx, a1, a2;
+      eval_col_s(r, pxc, dx, a1, a2);
+      float2 dy[NP], p1[NP], p2[NP], zq[NP];
+      bool ok[2 * NP];
+      bool any = false;
+#pragma unroll
+      for (int q = 0; q < NP; ++q) {
+        zq[q] = eval_zq_s(r, a1, a2, pyc[q], dy[q], p1[q], p2[q]);
+        ok[2 * q] = pos < nc[2 * q] && zq[q].x <= 0.f;
+        ok[2 * q + 1] = pos < nc[2 * q + 1] && zq[q].y <= 0.f;
+        any = any || ok[2 * q] || ok[2 * q + 1];
+      }
+      const uint32_t bal = __ballot_sync(0xffffffffu, any);
       if (bal == 0u) continue;
-      // a pixel that does not blend this Gaussian takes alpha = 0, which
-      // leaves its T and colour-behind unchanged and adds nothing below
-      const float2 araw = make_float2(alpha_raw_of(zq.x), alpha_raw_of(zq.y));
-      const float2 a = make_float2(ok0 ? fminf(kAlphaMax, araw.x) : 0.f,
-                                   ok1 ? fminf(kAlphaMax, araw.y) : 0.f);
-      const float2 one_m = __fadd2_rn(f2(1.f), make_float2(-a.x, -a.y));
-      const float2 inv = make_float2(ok0 ? 1.f / one_m.x : 1.f, ok1 ? 1.f / one_m.y : 1.f);
-      T = __fmul2_rn(T, inv);  // transmittance in front of this Gaussian
-      const float2 w = __fmul2_rn(a, T);
-      const float2 d0 = __fadd2_rn(f2(r[R_R]), make_float2(-acc0.x, -acc0.y));
-      const float2 d1 = __fadd2_rn(f2(r[R_G]), make_float2(-acc1.x, -acc1.y));
-      const float2 d2 = __fadd2_rn(f2(r[R_B]), make_float2(-acc2.x, -acc2.y));
-      float2 s = __fmul2_rn(d0, g0);
-      s = __ffma2_rn(d1, g1, s);
-      s = __ffma2_rn(d2, g2, s);
-      const float2 bgt = __fmul2_rn(tfbg, inv);
-      const float2 dLda = __ffma2_rn(T, s, make_float2(-bgt.x, -bgt.y));
-      acc0 = __ffma2_rn(a, d0, acc0);
-      acc1 = __ffma2_rn(a, d1, acc1);
-      acc2 = __ffma2_rn(a, d2, acc2);
-      // d alpha / d(-q/2) = alpha below the clamp, 0 on it
-      float2 dpow = __fmul2_rn(a, dLda);
-      dpow.x = araw.x < kAlphaMax ? dpow.x : 0.f;
-      dpow.y = araw.y < kAlphaMax ? dpow.y : 0.f;
-      // d alpha / d mean = alpha conic d = alpha 2 ln2 W^T (p1, p2)
-      const float2 dpl = __fmul2_rn(dpow, f2(kTwoLn2));
-      const float2 du =
-          __fmul2_rn(dpl, __ffma2_rn(f2(r[R_W1X]), p1, __fmul2_rn(f2(r[R_W2X]), p2)));
-      const float2 dv =
-          __fmul2_rn(dpl, __ffma2_rn(f2(r[R_W1Y]), p1, __fmul2_rn(f2(r[R_W2Y]), p2)));
-      const float2 dyd = __fmul2_rn(dy, dpow);
-      const float2 dy2d = __fmul2_rn(dy, dyd);
-      const float2 wg0 = __fmul2_rn(w, g0), wg1 = __fmul2_rn(w, g1), wg2 = __fmul2_rn(w, g2);
-      const float2 n2 = __ffma2_rn(dv, dv, __fmul2_rn(du, du));
-      const float sd = dpow.x + dpow.y;
       float v[10];
-      v[0] = du.x + du.y;
-      v[1] = dv.x + dv.y;
-      // d alpha / d conic = -alpha/2 (dx^2, 2 dx dy, dy^2)
-      v[2] = -0.5f * dx * dx * sd;
-      v[3] = -dx * (dyd.x + dyd.y);
-      v[4] = -0.5f * (dy2d.x + dy2d.y);
-      v[5] = r[R_OPAC] * sd;  // d alpha / d opacity = alpha / o (slot holds 1/o)
-      v[6] = wg0.x + wg0.y;
-      v[7] = wg1.x + wg1.y;
-      v[8] = wg2.x + wg2.y;
-      v[9] = sqrtf(n2.x) + sqrtf(n2.y);
+#pragma unroll
+      for (int e = 0; e < 10; ++e) v[e] = 0.f;
+#pragma unroll
+      for (int q = 0; q < NP; ++q) {
+        const bool o0 = ok[2 * q], o1 = ok[2 * q + 1];
+        // a pixel that does not blend this Gaussian takes alpha = 0, which
+        // leaves its T and colour-behind unchanged and adds nothing below
+        const float2 araw = make_float2(alpha_raw_of(zq[q].x), alpha_raw_of(zq[q].y));
+        const float2 a = make_float2(o0 ? fminf(kAlphaMax, araw.x) : 0.f,
+                                     o1 ? fminf(kAlphaMax, araw.y) : 0.f);
+        const float2 one_m = __fadd2_rn(f2(1.f), make_float2(-a.x, -a.y));
+        const float2 inv = make_float2(o0 ? 1.f / one_m.x : 1.f, o1 ? 1.f / one_m.y : 1.f);
+        T[q] = __fmul2_rn(T[q], inv);  // transmittance in front of this Gaussian
+        const float2 w = __fmul2_rn(a, T[q]);
+        const float2 d0 = __fadd2_rn(f2(r[R_R]), make_float2(-acc0[q].x, -acc0[q].y));
+        const float2 d1 = __fadd2_rn(f2(r[R_G]), make_float2(-acc1[q].x, -acc1[q].y));
+        const float2 d2 = __fadd2_rn(f2(r[R_B]), make_float2(-acc2[q].x, -acc2[q].y));
+        float2 s = __fmul2_rn(d0, g0[q]);
+        s = __ffma2_rn(d1, g1[q], s);
+        s = __ffma2_rn(d2, g2[q], s);
+        const float2 bgt = __fmul2_rn(tfbg[q], inv);
+        const float2 dLda = __ffma2_rn(T[q], s, make_float2(-bgt.x, -bgt.y));
+        acc0[q] = __ffma2_rn(a, d0, acc0[q]);
+        acc1[q] = __ffma2_rn(a, d1, acc1[q]);
+        acc2[q] = __ffma2_rn(a, d2, acc2[q]);
+        // d alpha / d(-q/2) = alpha below the clamp, 0 on it
+        float2 dpow = __fmul2_rn(a, dLda);
+        dpow.x = araw.x < kAlphaMax ? dpow.x : 0.f;
+        dpow.y = araw.y < kAlphaMax ? dpow.y : 0.f;
+        // d alpha / d mean = alpha conic d = alpha 2 ln2 W^T (p1, p2)
+        const float2 dpl = __fmul2_rn(dpow, f2(kTwoLn2));
+        const float2 du = __fmul2_rn(
+            dpl, __ffma2_rn(f2(r[R_W1X]), p1[q], __fmul2_rn(f2(r[R_W2X]), p2[q])));
+        const float2 dv = __fmul2_rn(
+            dpl, __ffma2_rn(f2(r[R_W1Y]), p1[q], __fmul2_rn(f2(r[R_W2Y]), p2[q])));
+        const float2 dyd = __fmul2_rn(dy[q], dpow);
+        const float2 dy2d = __fmul2_rn(dy[q], dyd);
+        const float2 wg0 = __fmul2_rn(w, g0[q]), wg1 = __fmul2_rn(w, g1[q]);
+        const float2 wg2 = __fmul2_rn(w, g2[q]);
+        const float2 n2 = __ffma2_rn(dv, dv, __fmul2_rn(du, du));
+        const float sd = dpow.x + dpow.y;
+        v[0] += du.x + du.y;
+        v[1] += dv.x + dv.y;
+        // d alpha / d conic = -alpha/2 (dx^2, 2 dx dy, dy^2)
+        v[2] += -0.5f * dx * dx * sd;
+        v[3] += -dx * (dyd.x + dyd.y);
+        v[4] += -0.5f * (dy2d.x + dy2d.y);
+        v[5] += r[R_OPAC] * sd;  // d alpha / d opacity = alpha / o (slot holds 1/o)
+        v[6] += wg0.x + wg0.y;
+        v[7] += wg1.x + wg1.y;
+        v[8] += wg2.x + wg2.y;
+        v[9] += sqrtf(n2.x) + sqrtf(n2.y);
+      }
       if (__popc(bal) == 1) {
-        if (ok0 || ok1) {
+        if (any) {
 #pragma unroll
           for (int e = 0; e < 10; ++e) atomicAdd(&s_acc[j][e], v[e]);
         }
@@ -642,9 +747,8 @@ cudaError_t launch_raster_fwd(const float* records, const uint32_t* ids, const i
   const int64_t tiles = (int64_t)g.tiles_per_view * n_views;
   if (tiles == 0) return cudaSuccess;
   RasterGeom geo{g, n, n > 0 ? capacity : 0};
-  k_raster_fwd<<<(unsigned)tiles, kThreads, 0, stream>>>(records, ids, ranges, geo, bg[0], bg[1],
-                                                         bg[2], image, final_T, n_contrib, status,
-                                                         wc);
+  k_raster_fwd<kPairs><<<(unsigned)tiles, Shape<kPairs>::kThreads, 0, stream>>>(
+      records, ids, ranges, geo, bg[0], bg[1], bg[2], image, final_T, n_contrib, status, wc);
   return cudaGetLastError();
 }
 
@@ -656,9 +760,9 @@ cudaError_t launch_raster_bwd(const float* records, const uint32_t* ids, const i
   const int64_t tiles = (int64_t)g.tiles_per_view * n_views;
   if (tiles == 0) return cudaSuccess;
   RasterGeom geo{g, n, n > 0 ? capacity : 0};
-  k_raster_bwd<<<(unsigned)tiles, kThreads, 0, stream>>>(records, ids, ranges, geo, bg[0], bg[1],
-                                                         bg[2], dL_dimage, final_T, n_contrib,
-                                                         grad2d, status, wc);
+  k_raster_bwd<kPairs><<<(unsigned)tiles, Shape<kPairs>::kThreads, 0, stream>>>(
+      records, ids, ranges, geo, bg[0], bg[1], bg[2], dL_dimage, final_T, n_contrib, grad2d,
+      status, wc);
   return cudaGetLastError();
 }
 

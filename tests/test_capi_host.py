@@ -159,9 +159,10 @@ def test_densify_thresholds_convert_to_the_raw_parameter_units():
 
 def test_sort_plan_follows_the_grid_and_mode():
     """gs_bin_sort_plan (host only) names the emission path the workspace is
-    laid out for: tile placement while the (tiles + 1)^2 difference array
-    fits, emission by column up to 256 columns, by tile id beyond; radix pass
-    counts of 8-bit digits."""
+    laid out for: tile placement up to 16384 tiles per view while the
+    (tiles + 1)^2 difference array fits, emission by column up to 256
+    columns, by tile id beyond; radix pass counts of 8-bit digits; placement
+    blocks of about four per SM below a million Gaussians."""
     def plan(W, H, n, views, mode):
         cam = S.make_scene("fwd_1k_128").cameras[0]
         cam.width, cam.height, cam.cx, cam.cy = W, H, W / 2, H / 2
@@ -171,6 +172,12 @@ def test_sort_plan_follows_the_grid_and_mode():
     assert (p.gaussians_per_block, p.blocks_per_view) == (768, 1303)
     p = plan(1920, 1080, 3_000_000, 1, api.GS_SORT_PRESORT)       # larger blocks past 2M
     assert (p.gaussians_per_block, p.blocks_per_view) == (4096, 733)
+    p = plan(3840, 2160, 10_000_000, 1, api.GS_SORT_PRESORT)      # 4K: 240 x 135 tiles
+    assert (p.path, p.pair_passes) == (api.GS_PATH_COLUMNS, 1)
+    p = plan(128, 128, 1000, 1, api.GS_SORT_PRESORT)               # small scene: 32 per block
+    assert (p.path, p.gaussians_per_block, p.blocks_per_view) == (api.GS_PATH_TILES, 32, 32)
+    p = plan(800, 800, 100_000, 1, api.GS_SORT_PRESORT)
+    assert (p.gaussians_per_block, p.blocks_per_view) == (160, 625)
     p = plan(4096, 2576, 1000, 1, api.GS_SORT_PRESORT)            # 256 x 161 tiles
     assert (p.path, p.pair_passes) == (api.GS_PATH_COLUMNS, 1)
     p = plan(8192, 1296, 1000, 1, api.GS_SORT_PRESORT)            # 512 x 81 tiles
