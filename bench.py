@@ -12,7 +12,9 @@ step time). ``--workload`` selects one of the five workload shapes:
   fwd_100k_800      forward only
   train_1m_1080p    the full step above (default)
   train_6m_8x1080p  8 views, forward + backward + densify statistics summed
-                    over the views, 64-bit (tile << 32 | depth) sort keys
+                    over the views; the sort's keys are 64-bit ((view << 32 |
+                    depth) in the presort; the extras time the pages' own
+                    (tile << 32 | depth) pair-key sort too)
   train_10m_4k      the full step with the fused Adam update
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
@@ -52,7 +54,7 @@ STEPS = {
     "fwd_1k_128": dict(kind="fwd", sort="presort"),
     "fwd_100k_800": dict(kind="fwd", sort="presort"),
     "train_1m_1080p": dict(kind="train", sort="presort"),
-    "train_6m_8x1080p": dict(kind="fwdbwd", sort="full64"),
+    "train_6m_8x1080p": dict(kind="fwdbwd", sort="presort"),
     "train_10m_4k": dict(kind="train", sort="presort"),
 }
 DEFAULT_WORKLOAD = "train_1m_1080p"
@@ -66,7 +68,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(STEPS))
     ap.add_argument("--sort-mode", default=None, choices=["presort", "full64"],
-                    help="default: the workload's own (full64 for the 8-view workload)")
+                    help="default: presort (depth presort, pairs placed per tile)")
     ap.add_argument("--n", type=int, default=None, help="override the Gaussian count")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -747,11 +749,12 @@ def run_ours(args):
     # statistics the timed steps accumulated (it runs every few hundred
     # steps), the loss, the quantised-SH Adam step and the full-64 sort
     extras = {}
-    if world == 1 and not args.no_extras and args.workload == DEFAULT_WORKLOAD:
-        extras["gs_densify_and_prune"] = measure_densify(sp)
-        extras["gs_l1_dssim"] = measure_loss(sp)
-        extras["gs_adam_step_sh_quant"] = measure_quant_adam(sp)
-        if args.sort_mode != "full64":
+    if world == 1 and not args.no_extras:
+        if args.workload == DEFAULT_WORKLOAD:
+            extras["gs_densify_and_prune"] = measure_densify(sp)
+            extras["gs_l1_dssim"] = measure_loss(sp)
+            extras["gs_adam_step_sh_quant"] = measure_quant_adam(sp)
+        if args.sort_mode != "full64" and kind != "fwd":
             extras["gs_bin_sort_full64"] = measure_full64_sort(scene)
 
     if world > 1:

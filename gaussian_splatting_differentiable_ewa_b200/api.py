@@ -36,6 +36,7 @@ GS_STATUS_BIT_NONFINITE = 8
 
 # gs_debug_stall sites
 GS_STALL_NONE, GS_STALL_EMIT_LOOKBACK, GS_STALL_RASTER_FWD, GS_STALL_RASTER_BWD = 0, 1, 2, 3
+GS_STALL_SORT_LOOKBACK = 4
 
 GS_TILE = 16
 GS_MAX_VIEWS = 32
@@ -55,7 +56,7 @@ class GsCamera(_c.Structure):
 class GsParams(_c.Structure):
     _fields_ = [("means", _vp), ("log_scales", _vp), ("quats", _vp), ("opacity_logit", _vp),
                 ("sh", _vp), ("sh_degree", _c.c_int32), ("reserved", _c.c_int32),
-                ("n", _c.c_int64)]
+                ("n", _c.c_int64), ("sh_quant", _vp)]
 
 
 class GsGrads(_c.Structure):
@@ -126,6 +127,9 @@ SIGNATURES = [
     ("gs_adam_step_sh_quant", _c.c_int,
      [_c.c_void_p, _vp, _vp, _vp, _c.c_float, _c.c_float, _c.c_float, _c.c_float, _c.c_int64,
       _c.c_int32, _c.c_uint64, _vp]),
+    ("gs_densify_sh_quant_workspace_size", _c.c_size_t, [_c.c_int64, _c.c_int64]),
+    ("gs_densify_sh_quant", _c.c_int,
+     [_c.c_void_p, _vp, _vp, _vp, _c.c_void_p, _vp, _vp, _vp, _c.c_size_t, _vp]),
     ("gs_bin_sort_plan", _c.c_int,
      [_c.c_int64, _c.c_int32, _c.POINTER(GsCamera), _c.c_int32, _c.c_void_p]),
     ("gs_debug_stall", _c.c_int, [_c.c_int32, _c.c_int64, _c.c_double]),
@@ -200,9 +204,14 @@ def cameras(cams: Sequence) -> ctypes.Array:
     return arr
 
 
-def params(means, log_scales, quats, opacity_logit, sh, sh_degree: int) -> GsParams:
-    return GsParams(_ptr(means), _ptr(log_scales), _ptr(quats), _ptr(opacity_logit), _ptr(sh),
-                    int(sh_degree), 0, int(means.shape[0]))
+def params(means, log_scales, quats, opacity_logit, sh, sh_degree: int,
+           sh_quant=None) -> GsParams:
+    """sh_quant (a GsShQuant) replaces sh: pass sh=None with it."""
+    p = GsParams(_ptr(means), _ptr(log_scales), _ptr(quats), _ptr(opacity_logit), _ptr(sh),
+                 int(sh_degree), 0, int(means.shape[0]),
+                 _c.cast(_c.pointer(sh_quant), _vp) if sh_quant is not None else None)
+    p._sh_quant_ref = sh_quant  # the descriptor outlives the pointer to it
+    return p
 
 
 def grads(means, log_scales, quats, opacity_logit, sh) -> GsGrads:
@@ -339,15 +348,20 @@ def gs_l1_dssim(image, target, n_views: int, height: int, width: int, lam: float
 GS_QUANT_GROUP = 256
 
 
+GS_QUANT_PLANAR, GS_QUANT_PACKED = 0, 1
+
+
 class GsShQuant(_c.Structure):
     _fields_ = [("codes", _vp), ("bounds", _vp), ("n", _c.c_int64), ("k3", _c.c_int32),
-                ("bits", _c.c_int32)]
+                ("bits", _c.c_int32), ("layout", _c.c_int32), ("reserved", _c.c_int32)]
 
 
-def sh_quant(codes, bounds, n: int, k3: int, bits: int) -> GsShQuant:
-    """Descriptor of a quantised SH state: codes uint8/int16 [k3, n_pad],
-    bounds float32 [k3, n_pad // 256, 2]."""
-    return GsShQuant(_ptr(codes), _ptr(bounds), int(n), int(k3), int(bits))
+def sh_quant(codes, bounds, n: int, k3: int, bits: int, layout: int = GS_QUANT_PLANAR
+             ) -> GsShQuant:
+    """Descriptor of a quantised SH state: codes uint8/int16 [k3, n_pad]
+    (planar) or int16 [k3, n_pad // 32, 3, 32] (packed blocks of codes and
+    both moments), bounds float32 [k3, n_pad // 256, 2]."""
+    return GsShQuant(_ptr(codes), _ptr(bounds), int(n), int(k3), int(bits), int(layout), 0)
 
 
 def gs_sh_quantize(sh, q: GsShQuant, stream=None) -> None:
@@ -361,10 +375,25 @@ def gs_sh_dequantize(q: GsShQuant, sh, stream=None) -> None:
 def gs_adam_step_sh_quant(q: GsShQuant, grad_sh, exp_avg, exp_avg_sq, lr: float, beta1: float,
                           beta2: float, eps: float, step: int, rounding: int = 0, seed: int = 0,
                           stream=None) -> None:
+    """Planar state: exp_avg / exp_avg_sq int16 [k3, n_pad]; packed: None."""
     _check(lib().gs_adam_step_sh_quant(_c.byref(q), _ptr(grad_sh), _ptr(exp_avg),
                                        _ptr(exp_avg_sq), float(lr), float(beta1), float(beta2),
                                        float(eps), int(step), int(rounding), int(seed),
                                        _stream(stream)), "gs_adam_step_sh_quant")
+
+
+def gs_densify_sh_quant_workspace_size(n_in: int, n_out: int) -> int:
+    return int(lib().gs_densify_sh_quant_workspace_size(int(n_in), int(n_out)))
+
+
+def gs_densify_sh_quant(q_in: GsShQuant, m_in, v_in, decisions, q_out: GsShQuant, m_out, v_out,
+                        ws, stream=None) -> None:
+    """Quantised SH of densify_and_prune's output (planar moments as int16
+    [k3, n_pad] tensors, None for packed state)."""
+    _check(lib().gs_densify_sh_quant(_c.byref(q_in), _ptr(m_in), _ptr(v_in), _ptr(decisions),
+                                     _c.byref(q_out), _ptr(m_out), _ptr(v_out), _ptr(ws),
+                                     int(ws.numel() * ws.element_size()), _stream(stream)),
+           "gs_densify_sh_quant")
 
 
 GS_PATH_TILE_ID, GS_PATH_COLUMNS, GS_PATH_TILES = 0, 1, 2

@@ -25,20 +25,28 @@
 //                  append their pairs in depth order through shared-memory
 //                  buffers written out warp-wide. Keys are row << cbits |
 //                  column; the radix passes then sort by row alone.
+//  k_digit_hist / k_onesweep
+//                  the 64-bit sorts (depth presort; full-64 pair keys): a
+//                  stable least-significant-digit radix sort with 8-bit
+//                  digits, single-sweep. One read of the keys counts the
+//                  digits of every pass; each pass is then one kernel whose
+//                  partitions (taken in launch order by a ticket) rank their
+//                  keys stably in shared memory and find their global
+//                  offsets by decoupled look-back over the partitions before
+//                  them, one thread per digit.
 //  k_radix_count / k_radix_scan / k_radix_scatter
-//                  one stable least-significant-digit radix pass with digits
-//                  of up to 8 bits, reduce-then-scan: per-partition digit
+//                  the 32-bit sorts (row or tile bits after column or
+//                  tile-id emission), reduce-then-scan: per-partition digit
 //                  counts, a per-digit scan over partitions (with the digit
 //                  totals), then a scatter that ranks each partition's keys
 //                  stably (ballots over warp-striped steps), stages them in
-//                  shared memory and writes runs of equal digits. The tile
-//                  bits of the 32-bit pair keys are split evenly over the
-//                  fewest passes (13 bits: 7 + 6), so each key costs one
-//                  ballot per bit of its pass.
+//                  shared memory and writes runs of equal digits. The bits
+//                  are split evenly over the fewest passes (13 bits: 7 + 6),
+//                  so each key costs one ballot per bit of its pass.
 //  k_ranges        [start, end) of each tile in the sorted pairs.
-// The emission's look-back waits are bounded in time (WaitCfg) and report
-// through the status word instead of hanging; the radix passes never wait on
-// other blocks.
+// Look-back waits (emission and single-sweep passes) are bounded in time
+// (WaitCfg) and report through the status word instead of hanging; the
+// reduce-then-scan passes never wait on other blocks.
 
 #include <cuda_runtime.h>
 
@@ -55,7 +63,7 @@ constexpr int kSortThreads = 256;
 constexpr int kSortWarps = kSortThreads / 32;
 constexpr int kSortItems = 16;                        // pair passes
 constexpr int kSortTile = kSortThreads * kSortItems;  // keys per partition
-constexpr int kPresortItems = 8;                      // per-Gaussian depth passes
+constexpr int kPresortItems = 16;                     // per-Gaussian depth passes
 constexpr int kColItems = 256;     // Gaussians per column-emission block
 constexpr int kColBuf = 32;        // pairs a column stages before a warp-wide write
 constexpr int kMaxColumns = 256;   // widest tile grid the column emission takes
@@ -970,9 +978,14 @@ __device__ __forceinline__ uint32_t warp_peers(uint32_t d) {
   return peers;
 }
 
+// Scatter blocks per SM (reduce-then-scan scatter and single-sweep pass). The
+// passes are bound by latency at low occupancy (their DRAM traffic is the
+// keys' and values' bytes, read and written once): with 64-bit keys and 16
+// keys per thread, three blocks (80 registers, a few spilled) measured 6 %
+// faster than two on a 985M-key sort.
 template <typename K, int ITEMS>
 struct ScatterOcc {
-  static constexpr int kBlocks = sizeof(K) == 4 ? 3 : (ITEMS > 8 ? 2 : 4);
+  static constexpr int kBlocks = 3;
 };
 
 template <typename K, int BITS, int ITEMS>
@@ -1068,6 +1081,218 @@ __global__ void __launch_bounds__(kSortThreads, (ScatterOcc<K, ITEMS>::kBlocks))
   __syncthreads();
   const uint32_t remain = n - p * (uint32_t)TILE;
   const uint32_t valid = remain < (uint32_t)TILE ? remain : (uint32_t)TILE;
+  for (uint32_t j = tid; j < valid; j += kSortThreads) {
+    const K k = s_keys[j];
+    const uint32_t gpos = j + s_delta[(uint32_t)(k >> shift) & M];
+    if (gpos < n) {
+      keys_out[gpos] = k;
+      vals_out[gpos] = s_vals[j];
+    } else {
+      atomicOr(status, kStatusBounds);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Single-sweep radix passes (the full 64-bit key sort). One kernel counts
+// the digits of every pass over all keys at once; then each pass is one
+// kernel. A pass's partitions take their indices in launch order (an atomic
+// ticket), publish their digit counts, and find each digit's global offset
+// by decoupled look-back over the partitions before them: a partition
+// publishes its counts (an aggregate) before it waits on anything, and after
+// its look-back its inclusive prefix, so a waiting partition walks back only
+// to the nearest prefix, and every partition it waits on is already running.
+// Look-back words: [63:34] pass tag, [33:32] flag (1 aggregate, 2 inclusive
+// prefix), [31:0] count; the array is zeroed per call and each pass has its
+// own tag. A wait that runs out of time takes a zero prefix and reports.
+constexpr uint64_t kSwAgg = 1ull << 32;
+constexpr uint64_t kSwPre = 2ull << 32;
+constexpr uint64_t kSwFlags = 3ull << 32;
+constexpr int kSwBatch = 4;
+
+// Digit counts of every pass in one read of the keys. A thread takes 8
+// consecutive keys (vector loads) and adds each run of equal digits with one
+// shared atomic: a Gaussian's pairs are emitted together and share their
+// depth, so runs are long and the atomics few.
+template <typename K>
+__global__ void __launch_bounds__(256) k_digit_hist(const K* __restrict__ keys,
+                                                    const int64_t* __restrict__ n_ptr,
+                                                    int64_t capacity, RadixPlan plan,
+                                                    uint32_t* __restrict__ hist) {
+  __shared__ uint32_t s_h[8][256];
+  const int64_t n = *n_ptr;
+  if (n > capacity || n <= 0) return;
+  for (int k = threadIdx.x; k < 8 * 256; k += 256) (&s_h[0][0])[k] = 0u;
+  __syncthreads();
+  const int64_t chunks = (n + 7) / 8;
+  for (int64_t c = (int64_t)blockIdx.x * 256 + threadIdx.x; c < chunks;
+       c += (int64_t)gridDim.x * 256) {
+    const int64_t base = c * 8;
+    const int cnt = n - base < 8 ? (int)(n - base) : 8;
+    K k[8];
+    if (cnt == 8) {
+      uint4 raw[sizeof(K) / 2];
+      const uint4* src = reinterpret_cast<const uint4*>(keys + base);
+#pragma unroll
+      for (int r = 0; r < (int)(sizeof(K) / 2); ++r) raw[r] = src[r];
+      memcpy(k, raw, sizeof(k));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) k[j] = j < cnt ? keys[base + j] : (K)0;
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (q >= plan.passes) break;
+      const int sh = plan.shift[q];
+      uint32_t prev = (uint32_t)(k[0] >> sh) & 255u, run = 1;
+#pragma unroll
+      for (int j = 1; j < 8; ++j) {
+        if (j >= cnt) break;
+        const uint32_t d = (uint32_t)(k[j] >> sh) & 255u;
+        if (d == prev) {
+          ++run;
+        } else {
+          atomicAdd(&s_h[q][prev], run);
+          prev = d;
+          run = 1;
+        }
+      }
+      atomicAdd(&s_h[q][prev], run);
+    }
+  }
+  __syncthreads();
+  for (int k = threadIdx.x; k < plan.passes * 256; k += 256) {
+    const uint32_t c = (&s_h[0][0])[k];
+    if (c) atomicAdd(&hist[k], c);
+  }
+}
+
+template <typename K, int ITEMS>
+__global__ void __launch_bounds__(kSortThreads, (ScatterOcc<K, ITEMS>::kBlocks)) k_onesweep(
+    const K* __restrict__ keys_in, const uint32_t* __restrict__ vals_in,
+    K* __restrict__ keys_out, uint32_t* __restrict__ vals_out,
+    const int64_t* __restrict__ n_ptr, int64_t capacity, int shift, int pass,
+    const uint32_t* __restrict__ hist, uint64_t* __restrict__ lookback,
+    uint32_t* __restrict__ ticket, WaitCfg wc, uint32_t* __restrict__ status) {
+  constexpr int R = 256;
+  constexpr uint32_t M = R - 1;
+  constexpr int TILE = SortTile<ITEMS>::kItems;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  K* s_keys = reinterpret_cast<K*>(smem_raw);                          // [TILE]
+  uint32_t* s_vals = reinterpret_cast<uint32_t*>(s_keys + TILE);       // [TILE]
+  uint32_t* s_whist = s_vals + TILE;                                   // [warps][R]
+  uint32_t* s_delta = s_whist + kSortWarps * R;                        // [R]
+  __shared__ uint32_t s_scan[9];
+  __shared__ uint32_t s_p;
+
+  const int64_t n64 = *n_ptr;
+  if (n64 > capacity || n64 <= 0) return;
+  const uint32_t n = (uint32_t)n64;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) s_p = atomicAdd(ticket, 1u);
+  for (int k = tid; k < kSortWarps * R; k += kSortThreads) s_whist[k] = 0u;
+  __syncthreads();
+  const uint32_t p = s_p;
+  if ((uint64_t)p * TILE >= n) return;  // the whole block: no partition left
+  const uint32_t first = p * (uint32_t)TILE + (uint32_t)warp * (ITEMS * 32) + lane;
+  K key[ITEMS];
+  uint32_t val[ITEMS];
+#pragma unroll
+  for (int it = 0; it < ITEMS; ++it) {
+    const uint32_t idx = first + it * 32;
+    key[it] = idx < n ? keys_in[idx] : (K)0;
+    val[it] = idx < n ? vals_in[idx] : 0u;
+  }
+  const uint32_t hcount = hist[tid];
+  uint32_t* wh = s_whist + warp * R;
+#pragma unroll
+  for (int it = 0; it < ITEMS; ++it) {
+    const uint32_t idx = first + it * 32;
+    const uint32_t d = idx < n ? ((uint32_t)(key[it] >> shift) & M) : M;
+    atomicAdd(&wh[d], 1u);
+  }
+  __syncthreads();
+  // per digit: warp offsets and the partition's count (keys past the end sit
+  // in the largest digit and are not counted)
+  uint32_t count = 0;
+  {
+#pragma unroll
+    for (int w = 0; w < kSortWarps; ++w) {
+      const uint32_t c = s_whist[w * R + tid];
+      s_whist[w * R + tid] = count;
+      count += c;
+    }
+  }
+  const uint32_t remain = n - p * (uint32_t)TILE;
+  const uint32_t valid = remain < (uint32_t)TILE ? remain : (uint32_t)TILE;
+  const uint32_t real = tid == (int)M ? count - ((uint32_t)TILE - valid) : count;
+  const uint64_t tag = (uint64_t)(pass + 1) << 34;
+  uint64_t* row = lookback + (uint64_t)p * R;
+  const bool publish = (int64_t)p != wc.stall;  // test hook: a silent partition
+  if (publish) st_relaxed_u64(row + tid, tag | (p == 0 ? kSwPre : kSwAgg) | real);
+  uint32_t tot;
+  const uint32_t lstart = block_exclusive_scan_256(count, s_scan, tot);  // syncs the block
+#pragma unroll
+  for (int w = 0; w < kSortWarps; ++w) s_whist[w * R + tid] += lstart;
+  __syncthreads();
+  // stable rank within the warp -> position within the partition
+  const uint32_t lt = lanemask_lt();
+#pragma unroll
+  for (int it = 0; it < ITEMS; ++it) {
+    const uint32_t idx = first + it * 32;
+    const uint32_t d = idx < n ? ((uint32_t)(key[it] >> shift) & M) : M;
+    const uint32_t peers = warp_peers<8>(d);
+    const uint32_t before = wh[d];
+    __syncwarp();
+    if ((peers & lt) == 0) wh[d] = before + __popc(peers);
+    __syncwarp();
+    const uint32_t pos = before + __popc(peers & lt);
+    s_keys[pos] = key[it];
+    s_vals[pos] = val[it];
+  }
+  // the pass's digit starts, then this partition's global offsets; ranking
+  // first gives the partitions before this one time to publish prefixes
+  uint32_t all;
+  const uint32_t dbase = block_exclusive_scan_256(hcount, s_scan, all);  // syncs the block
+  // decoupled look-back for this thread's digit
+  // (kSwBatch predecessors' words are loaded at once, so a long walk costs
+  // one load latency per batch rather than per partition)
+  uint32_t excl = 0;
+  if (p > 0) {
+    int64_t j = (int64_t)p - 1;
+    bool done = false;
+    while (!done && j >= 0) {
+      uint64_t w[kSwBatch];
+#pragma unroll
+      for (int b = 0; b < kSwBatch; ++b)
+        w[b] = j - b >= 0 ? ld_relaxed_u64(lookback + (uint64_t)(j - b) * R + tid) : 0ull;
+#pragma unroll
+      for (int b = 0; b < kSwBatch; ++b) {
+        if (done || j - b < 0) break;
+        uint64_t v = w[b];
+        if ((v & ~((1ull << 34) - 1)) != tag || (v & kSwFlags) == 0) {
+          const uint64_t* src = lookback + (uint64_t)(j - b) * R + tid;
+          const uint64_t t0 = globaltimer_ns();
+          while (true) {
+            __nanosleep(32);
+            v = ld_relaxed_u64(src);
+            if ((v & ~((1ull << 34) - 1)) == tag && (v & kSwFlags) != 0) break;
+            if (globaltimer_ns() - t0 > wc.limit_ns) {
+              atomicOr(status, kStatusTimeout);
+              v = tag | kSwPre;  // give up: a zero prefix ends the walk
+              break;
+            }
+          }
+        }
+        excl += (uint32_t)v;
+        if ((v & kSwFlags) == kSwPre) done = true;
+      }
+      j -= kSwBatch;
+    }
+    if (publish) st_relaxed_u64(row + tid, tag | kSwPre | (excl + real));
+  }
+  s_delta[tid] = dbase + excl - lstart;  // local slot -> global position
+  __syncthreads();
   for (uint32_t j = tid; j < valid; j += kSortThreads) {
     const K k = s_keys[j];
     const uint32_t gpos = j + s_delta[(uint32_t)(k >> shift) & M];
@@ -1205,6 +1430,42 @@ cudaError_t run_radix_passes(K* keys_a, uint32_t* vals_a, K* keys_b, uint32_t* v
   return cudaSuccess;
 }
 
+// The plan's passes (8-bit digits) as single-sweep passes, ping-ponging like
+// run_radix_passes. hist: [8][256] digit counts, zeroed by the caller;
+// lookback: [parts][256] words, zeroed by the caller; tickets: one zeroed
+// counter per pass.
+template <typename K, int ITEMS>
+cudaError_t run_onesweep_passes(K* keys_a, uint32_t* vals_a, K* keys_b, uint32_t* vals_b,
+                                const int64_t* n_ptr, int64_t capacity, int64_t max_items,
+                                const RadixPlan& plan, uint32_t* hist, uint64_t* lookback,
+                                uint32_t* tickets, const WaitCfg& wc, uint32_t* status,
+                                int sms, cudaStream_t stream) {
+  const int64_t parts = (max_items + SortTile<ITEMS>::kItems - 1) / SortTile<ITEMS>::kItems;
+  if (parts == 0) return cudaSuccess;
+  for (int q = 0; q < plan.passes; ++q)
+    if (plan.bits[q] != 8) return cudaErrorInvalidValue;
+  k_digit_hist<K><<<sms * 4, 256, 0, stream>>>(keys_a, n_ptr, capacity, plan, hist);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = scatter_smem_bytes<K, 8, ITEMS>();
+  e = cudaFuncSetAttribute(k_onesweep<K, ITEMS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+  if (e != cudaSuccess) return e;
+  K* kin = keys_a;
+  uint32_t* vin = vals_a;
+  K* kout = keys_b;
+  uint32_t* vout = vals_b;
+  for (int q = 0; q < plan.passes; ++q) {
+    k_onesweep<K, ITEMS><<<(unsigned)parts, kSortThreads, smem, stream>>>(
+        kin, vin, kout, vout, n_ptr, capacity, plan.shift[q], q, hist + 256 * q, lookback,
+        tickets + q, wc, status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    K* tk = kin; kin = kout; kout = tk;
+    uint32_t* tv = vin; vin = vout; vout = tv;
+  }
+  return cudaSuccess;
+}
+
 int num_sms() {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -1274,10 +1535,10 @@ cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
     k_depth_keys<<<(int)blocks, 256, 0, stream>>>(bins4, a.n, a.n_views, a.pkeys[0], a.pvals[0],
                                                   a.n_items_dev, a.n_visible, a.status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    e = run_radix_passes<uint64_t, kPresortItems>(a.pkeys[0], a.pvals[0], a.pkeys[1], a.pvals[1],
-                                                  a.n_items_dev, n_items, n_items, a.presort,
-                                                  a.counts, a.counts_stride, a.totals, a.status,
-                                                  stream);
+    e = run_onesweep_passes<uint64_t, kPresortItems>(
+        a.pkeys[0], a.pvals[0], a.pkeys[1], a.pvals[1], a.n_items_dev, n_items, n_items,
+        a.presort, a.digit_hist, a.sweep_lookback, a.counters + 1, a.sort_wait, a.status, sms,
+        stream);
     if (e != cudaSuccess) return e;
     const int fin = a.presort.passes & 1;
     if (a.tile_emit) {
@@ -1352,10 +1613,11 @@ cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
       bins4, nullptr, nullptr, a.n, a.n_views, a.grid, a.keys[a.emit_buf], a.vals[a.emit_buf],
       a.capacity, a.n_pairs, a.emit_lookback, a.counters + 0, a.status, a.wait);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  e = run_radix_passes<uint64_t, kSortItems>(a.keys[a.emit_buf], a.vals[a.emit_buf],
-                                             a.keys[a.emit_buf ^ 1], a.vals[a.emit_buf ^ 1],
-                                             a.n_pairs, a.capacity, a.capacity, a.pairs, a.counts,
-                                             a.counts_stride, a.totals, a.status, stream);
+  e = run_onesweep_passes<uint64_t, kSortItems>(a.keys[a.emit_buf], a.vals[a.emit_buf],
+                                                a.keys[a.emit_buf ^ 1], a.vals[a.emit_buf ^ 1],
+                                                a.n_pairs, a.capacity, a.capacity, a.pairs,
+                                                a.digit_hist, a.sweep_lookback, a.counters + 1,
+                                                a.sort_wait, a.status, sms, stream);
   if (e != cudaSuccess) return e;
   const int out = a.emit_buf ^ (a.pairs.passes & 1);
   k_ranges<uint64_t><<<sms * 4, 256, 0, stream>>>(a.keys[out], a.n_pairs, a.capacity, a.n_tiles,

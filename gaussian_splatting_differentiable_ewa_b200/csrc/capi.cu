@@ -47,7 +47,9 @@ struct Layout {
   int64_t counts_stride = 0;
   size_t off_hist = 0, off_emit_lb = 0, off_counts = 0, off_keys0 = 0, off_keys1 = 0,
          off_vals1 = 0, off_pkeys0 = 0, off_pkeys1 = 0, off_pvals0 = 0, off_pvals1 = 0,
-         off_crect = 0, off_tile_totals = 0, off_tile_base = 0;
+         off_crect = 0, off_tile_totals = 0, off_tile_base = 0, off_digit_hist = 0,
+         off_sweep_lb = 0;
+  size_t sweep_lb_bytes = 0;
   size_t total = 0;
 };
 
@@ -116,6 +118,14 @@ bool make_layout(int64_t n, int32_t n_views, const gs_camera* cams, int64_t capa
   L.off_keys0 = off; off = align_up(off + (size_t)kcap * L.key_bytes);
   L.off_keys1 = off; off = align_up(off + (size_t)kcap * L.key_bytes);
   L.off_vals1 = off; off = align_up(off + (size_t)kcap * 4);
+  // single-sweep passes (the pair keys in full-64 mode, the depth keys in
+  // presort mode): every pass's digit counts, one look-back word per
+  // (partition, digit)
+  L.off_digit_hist = off; off = align_up(off + 8 * 256 * sizeof(uint32_t));
+  L.sweep_lb_bytes = (size_t)(mode == GS_SORT_FULL64 ? pair_partitions(capacity)
+                                                     : presort_partitions(items)) *
+                     256 * sizeof(uint64_t);
+  L.off_sweep_lb = off; off = align_up(off + L.sweep_lb_bytes);
   if (mode == GS_SORT_PRESORT) {
     L.off_pkeys0 = off; off = align_up(off + (size_t)items * 8);
     L.off_pkeys1 = off; off = align_up(off + (size_t)items * 8);
@@ -162,6 +172,25 @@ uint32_t* status_word(void* ws) {
   return reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(ws) + kStatusOffset);
 }
 
+bool quant_ok(const gs_sh_quant* q) {
+  if (!q || q->n < 0 || q->n >= (1ll << 31)) return false;
+  if (q->bits != 8 && q->bits != 16) return false;
+  if (q->k3 != 3 && q->k3 != 12 && q->k3 != 27 && q->k3 != 48) return false;
+  if (q->layout != GS_QUANT_PLANAR && q->layout != GS_QUANT_PACKED) return false;
+  if (q->n == 0) return true;
+  // codes (and packed moments) move four at a time
+  const size_t a = q->layout == GS_QUANT_PACKED ? 8 : (size_t)(q->bits / 2);
+  return q->codes && q->bounds && aligned(q->codes, a) && aligned(q->bounds, 8);
+}
+
+// The SH source of a parameter set: exactly one of sh and sh_quant, the
+// codes matching n and the degree.
+bool params_sh_ok(const gs_params& p) {
+  if (!p.sh_quant) return p.sh != nullptr;
+  if (p.sh || !quant_ok(p.sh_quant)) return false;
+  return p.sh_quant->n == p.n && p.sh_quant->k3 == 3 * (p.sh_degree + 1) * (p.sh_degree + 1);
+}
+
 }  // namespace
 
 extern "C" {
@@ -197,8 +226,8 @@ gs_status gs_project(const gs_params* params, const gs_camera* cams, int32_t n_v
   if (p.n >= (1ll << 31) || p.n * n_views >= (1ll << 40)) return GS_ERR_OVERFLOW;
   if (p.sh_degree < 0 || p.sh_degree > 3) return GS_ERR_INVALID_ARG;
   if (p.n == 0) return GS_OK;
-  if (!p.means || !p.log_scales || !p.quats || !p.opacity_logit || !p.sh || !out->records ||
-      !out->bins || !out->radii)
+  if (!p.means || !p.log_scales || !p.quats || !p.opacity_logit || !params_sh_ok(p) ||
+      !out->records || !out->bins || !out->radii)
     return GS_ERR_INVALID_ARG;
   if (!aligned(p.means, 16) || !aligned(p.log_scales, 16) || !aligned(p.quats, 16) ||
       !aligned(out->records, 16) || !aligned(out->bins, 16))
@@ -231,6 +260,10 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
       cudaMemsetAsync(w + L.off_emit_lb, 0, (size_t)emit_blocks(items) * 8, st) != cudaSuccess ||
       cudaMemsetAsync(out->ranges, 0, (size_t)tiles * 2 * sizeof(int64_t), st) != cudaSuccess)
     return GS_ERR_CUDA;
+  if (cudaMemsetAsync(w + L.off_digit_hist, 0, 8 * 256 * sizeof(uint32_t), st) != cudaSuccess ||
+      (L.sweep_lb_bytes &&
+       cudaMemsetAsync(w + L.off_sweep_lb, 0, L.sweep_lb_bytes, st) != cudaSuccess))
+    return GS_ERR_CUDA;
 
   BinSortArgs a{};
   a.bins = proj->bins;
@@ -261,9 +294,12 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
   a.counts = reinterpret_cast<uint32_t*>(w + L.off_counts);
   a.counts_stride = L.counts_stride;
   a.emit_lookback = reinterpret_cast<uint64_t*>(w + L.off_emit_lb);
+  a.digit_hist = reinterpret_cast<uint32_t*>(w + L.off_digit_hist);
+  a.sweep_lookback = reinterpret_cast<uint64_t*>(w + L.off_sweep_lb);
   a.counters = reinterpret_cast<uint32_t*>(w + kCountersOffset);
   a.status = reinterpret_cast<uint32_t*>(w + kStatusOffset);
   a.wait = wait_cfg(GS_STALL_EMIT_LOOKBACK);
+  a.sort_wait = wait_cfg(GS_STALL_SORT_LOOKBACK);
   a.n_pairs = out->n_pairs;
   a.n_items_dev = reinterpret_cast<int64_t*>(w + kNItemsOffset);
   a.pair_total = reinterpret_cast<unsigned long long*>(w + kPairTotalOffset);
@@ -300,8 +336,8 @@ namespace {
 
 gs_status check_grads_args(const gs_params& p, const gs_grads* grads, bool need) {
   if (!grads) return need ? GS_ERR_INVALID_ARG : GS_OK;
-  if (p.n > 0 && (!p.means || !p.log_scales || !p.quats || !p.opacity_logit || !p.sh ||
-                  !grads->means || !grads->log_scales || !grads->quats ||
+  if (p.n > 0 && (!p.means || !p.log_scales || !p.quats || !p.opacity_logit ||
+                  !params_sh_ok(p) || !grads->means || !grads->log_scales || !grads->quats ||
                   !grads->opacity_logit || !grads->sh))
     return GS_ERR_INVALID_ARG;
   if (!aligned(p.means, 16) || !aligned(p.log_scales, 16) || !aligned(p.quats, 16) ||
@@ -462,11 +498,15 @@ size_t gs_densify_workspace_size(int64_t n) {
 }
 
 namespace {
-bool dp_tensors(const gs_grads* g, bool need, gsb::DpTensorPtrs& t) {
+// with_sh false: the SH block is not touched (quantised SH), its pointer is
+// not needed
+bool dp_tensors(const gs_grads* g, bool need, bool with_sh, gsb::DpTensorPtrs& t) {
   if (!g) return !need;
-  t = gsb::DpTensorPtrs{g->means, g->log_scales, g->quats, g->opacity_logit, g->sh};
-  return t.means && t.log_scales && t.quats && t.logit && t.sh && aligned(t.means, 16) &&
-         aligned(t.log_scales, 16) && aligned(t.quats, 16) && aligned(t.sh, 16);
+  t = gsb::DpTensorPtrs{g->means, g->log_scales, g->quats, g->opacity_logit,
+                        with_sh ? g->sh : nullptr};
+  return t.means && t.log_scales && t.quats && t.logit && (!with_sh || t.sh) &&
+         aligned(t.means, 16) && aligned(t.log_scales, 16) && aligned(t.quats, 16) &&
+         aligned(t.sh, 16);
 }
 }  // namespace
 
@@ -488,9 +528,13 @@ gs_status gs_densify_and_prune(const gs_params* in, const gs_grads* m_in, const 
   gs_grads pin{const_cast<float*>(in->means), const_cast<float*>(in->log_scales),
                const_cast<float*>(in->quats), const_cast<float*>(in->opacity_logit),
                const_cast<float*>(in->sh)};
+  // quantised SH: the SH blocks are gs_densify_sh_quant's, which needs the codes
+  const bool with_sh = in->sh_quant == nullptr;
+  if (!params_sh_ok(*in) || (!with_sh && !codes)) return GS_ERR_INVALID_ARG;
   gsb::DpTensorPtrs tp, tm, tv, op, om, ov;
-  if (!dp_tensors(&pin, true, tp) || !dp_tensors(m_in, true, tm) || !dp_tensors(v_in, true, tv) ||
-      !dp_tensors(out, true, op) || !dp_tensors(m_out, true, om) || !dp_tensors(v_out, true, ov))
+  if (!dp_tensors(&pin, true, with_sh, tp) || !dp_tensors(m_in, true, with_sh, tm) ||
+      !dp_tensors(v_in, true, with_sh, tv) || !dp_tensors(out, true, with_sh, op) ||
+      !dp_tensors(m_out, true, with_sh, om) || !dp_tensors(v_out, true, with_sh, ov))
     return GS_ERR_INVALID_ARG;
   if (!accum || !denom || !z) return GS_ERR_INVALID_ARG;
   unsigned char* w = static_cast<unsigned char*>(ws);
@@ -500,7 +544,7 @@ gs_status gs_densify_and_prune(const gs_params* in, const gs_grads* m_in, const 
                                  w + align_up(kControlBytes + (size_t)densify_blocks(n) * 4));
   gsb::DensifyArgs a{dp->grad_threshold, dp->log_scale_split, dp->logit_min_opacity,
                      dp->log_max_scale, dp->log_split_shrink};
-  const int k3 = 3 * (in->sh_degree + 1) * (in->sh_degree + 1);
+  const int k3 = with_sh ? 3 * (in->sh_degree + 1) * (in->sh_degree + 1) : 0;
   return cuda_status(gsb::launch_densify_and_prune(
       tp, tm, tv, accum, denom, z, n, k3, a, code_buf, block_counts, out_capacity, n_out,
       reinterpret_cast<uint32_t*>(w + kStatusOffset), op, om, ov, st));
@@ -530,33 +574,18 @@ gs_status gs_l1_dssim(const float* image, const float* target, int32_t n_views, 
                                           static_cast<cudaStream_t>(stream)));
 }
 
-namespace {
-bool quant_ok(const gs_sh_quant* q) {
-  if (!q || q->n < 0 || q->n >= (1ll << 31)) return false;
-  if (q->bits != 8 && q->bits != 16) return false;
-  if (q->k3 != 3 && q->k3 != 12 && q->k3 != 27 && q->k3 != 48) return false;
-  if (q->n == 0) return true;
-  // codes move four at a time
-  return q->codes && q->bounds && aligned(q->codes, q->bits / 2) && aligned(q->bounds, 8);
-}
-}  // namespace
-
 gs_status gs_sh_quantize(const float* sh, const gs_sh_quant* q, void* stream) {
   if (!quant_ok(q)) return GS_ERR_INVALID_ARG;
   if (q->n == 0) return GS_OK;
   if (!sh || !aligned(sh, 4)) return GS_ERR_INVALID_ARG;
-  return cuda_status(gsb::launch_sh_quantize(sh, q->n, q->k3, q->bits, q->codes,
-                                             reinterpret_cast<float2*>(q->bounds),
-                                             static_cast<cudaStream_t>(stream)));
+  return cuda_status(gsb::launch_sh_quantize(sh, *q, static_cast<cudaStream_t>(stream)));
 }
 
 gs_status gs_sh_dequantize(const gs_sh_quant* q, float* sh, void* stream) {
   if (!quant_ok(q)) return GS_ERR_INVALID_ARG;
   if (q->n == 0) return GS_OK;
   if (!sh || !aligned(sh, 4)) return GS_ERR_INVALID_ARG;
-  return cuda_status(gsb::launch_sh_dequantize(q->codes, reinterpret_cast<const float2*>(q->bounds),
-                                               q->n, q->k3, q->bits, sh,
-                                               static_cast<cudaStream_t>(stream)));
+  return cuda_status(gsb::launch_sh_dequantize(*q, sh, static_cast<cudaStream_t>(stream)));
 }
 
 gs_status gs_adam_step_sh_quant(const gs_sh_quant* q, const float* grad_sh, uint16_t* exp_avg,
@@ -566,13 +595,53 @@ gs_status gs_adam_step_sh_quant(const gs_sh_quant* q, const float* grad_sh, uint
   if (!quant_ok(q) || step < 1 || (rounding != 0 && rounding != 1)) return GS_ERR_INVALID_ARG;
   if (!(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f) || !(eps >= 0.f))
     return GS_ERR_INVALID_ARG;
-  if (q->n == 0) return GS_OK;
-  if (!grad_sh || !exp_avg || !exp_avg_sq || !aligned(grad_sh, 4) || !aligned(exp_avg, 8) ||
-      !aligned(exp_avg_sq, 8))
+  // packed blocks carry their moments; planar moments come beside the state
+  const bool packed = q->layout == GS_QUANT_PACKED;
+  if (packed ? (exp_avg || exp_avg_sq) : (q->n > 0 && (!exp_avg || !exp_avg_sq)))
     return GS_ERR_INVALID_ARG;
-  return cuda_status(gsb::launch_adam_sh_quant(
-      q->codes, reinterpret_cast<float2*>(q->bounds), grad_sh, exp_avg, exp_avg_sq, q->n, q->k3,
-      q->bits, lr, beta1, beta2, eps, step, rounding, seed, static_cast<cudaStream_t>(stream)));
+  if (q->n == 0) return GS_OK;
+  if (!grad_sh || !aligned(grad_sh, 4) || !aligned(exp_avg, 8) || !aligned(exp_avg_sq, 8))
+    return GS_ERR_INVALID_ARG;
+  return cuda_status(gsb::launch_adam_sh_quant(*q, grad_sh, exp_avg, exp_avg_sq, lr, beta1, beta2,
+                                               eps, step, rounding, seed,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+size_t gs_densify_sh_quant_workspace_size(int64_t n_in, int64_t n_out) {
+  if (n_in < 0 || n_in >= (1ll << 31) || n_out < 0 || n_out >= (1ll << 31)) return 0;
+  size_t off = kControlBytes;
+  off = align_up(off + (size_t)densify_blocks(n_in) * sizeof(uint32_t));  // block counts
+  off = align_up(off + sizeof(int64_t));                                  // the map's count
+  off = align_up(off + (size_t)n_out * sizeof(uint32_t));                 // output -> input
+  return off;
+}
+
+gs_status gs_densify_sh_quant(const gs_sh_quant* in, const uint16_t* m_in, const uint16_t* v_in,
+                              const int8_t* decisions, const gs_sh_quant* out, uint16_t* m_out,
+                              uint16_t* v_out, void* ws, size_t ws_bytes, void* stream) {
+  if (!quant_ok(in) || !quant_ok(out) || !ws || !aligned(ws, kAlign)) return GS_ERR_INVALID_ARG;
+  if (in->k3 != out->k3 || in->bits != out->bits || in->layout != out->layout)
+    return GS_ERR_INVALID_ARG;
+  if (out->n > 2 * in->n) return GS_ERR_INVALID_ARG;
+  const bool packed = in->layout == GS_QUANT_PACKED;
+  if (packed ? (m_in || v_in || m_out || v_out)
+             : (!m_in || !v_in || !m_out || !v_out || !aligned(m_in, 8) || !aligned(v_in, 8) ||
+                !aligned(m_out, 8) || !aligned(v_out, 8)))
+    return GS_ERR_INVALID_ARG;
+  if (in->n > 0 && !decisions) return GS_ERR_INVALID_ARG;
+  if (ws_bytes < gs_densify_sh_quant_workspace_size(in->n, out->n)) return GS_ERR_INVALID_ARG;
+  if (in->n == 0) return out->n == 0 ? GS_OK : GS_ERR_INVALID_ARG;
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  size_t off = kControlBytes;
+  uint32_t* block_counts = reinterpret_cast<uint32_t*>(w + off);
+  off = align_up(off + (size_t)densify_blocks(in->n) * sizeof(uint32_t));
+  int64_t* n_out_dev = reinterpret_cast<int64_t*>(w + off);
+  off = align_up(off + sizeof(int64_t));
+  uint32_t* src = reinterpret_cast<uint32_t*>(w + off);
+  return cuda_status(gsb::launch_densify_sh_quant(*in, m_in, v_in, decisions, *out, m_out, v_out,
+                                                  block_counts, n_out_dev, src,
+                                                  reinterpret_cast<uint32_t*>(w + kStatusOffset),
+                                                  static_cast<cudaStream_t>(stream)));
 }
 
 gs_status gs_bin_sort_plan(int64_t n, int32_t n_views, const gs_camera* cams,
@@ -588,7 +657,7 @@ gs_status gs_bin_sort_plan(int64_t n, int32_t n_views, const gs_camera* cams,
 }
 
 gs_status gs_debug_stall(int32_t site, int64_t index, double wait_limit_s) {
-  if (site < GS_STALL_NONE || site > GS_STALL_RASTER_BWD) return GS_ERR_INVALID_ARG;
+  if (site < GS_STALL_NONE || site > GS_STALL_SORT_LOOKBACK) return GS_ERR_INVALID_ARG;
   if (!(wait_limit_s >= 0.0) || wait_limit_s > 60.0) return GS_ERR_INVALID_ARG;
   if (site != GS_STALL_NONE && index < 0) return GS_ERR_INVALID_ARG;
   g_stall_site.store(GS_STALL_NONE);

@@ -21,6 +21,9 @@
 //               fields; the SH blocks (most of the bytes) are moved by the
 //               whole warp in contiguous runs; six blocks per SM (40
 //               registers) keep more of those runs in flight.
+//  k_dsq_count / k_dsq_map  the same positions from given decisions, as an
+//               output -> input map for quantised SH (quant.cu re-encodes
+//               the output groups from it).
 
 #include <cuda_runtime.h>
 
@@ -259,6 +262,62 @@ __global__ void __launch_bounds__(kDpThreads, 6) k_dp_emit(
     copy_sh_warp<float>(p_in, m_in, v_in, p_out, m_out, v_out, k3, c, pos, i - lane);
 }
 
+// Output counts of each block of decisions (the quantised-SH map).
+__global__ void __launch_bounds__(kDpThreads) k_dsq_count(const int8_t* __restrict__ codes, int n,
+                                                          uint32_t* __restrict__ block_counts) {
+  __shared__ uint32_t s_w[kDpThreads / 32];
+  const int i = blockIdx.x * kDpThreads + threadIdx.x;
+  uint32_t s = i < n ? (uint32_t)dp_count(codes[i]) : 0u;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t t = 0;
+#pragma unroll
+    for (int w = 0; w < kDpThreads / 32; ++w) t += s_w[w];
+    block_counts[blockIdx.x] = t;
+  }
+}
+
+// src[o] for every output o of input i (positions as k_dp_emit takes them):
+// i, with bit 31 set for a clone's copy and both split children (their
+// moments start at zero).
+__global__ void __launch_bounds__(kDpThreads) k_dsq_map(const int8_t* __restrict__ codes, int n,
+                                                        const uint32_t* __restrict__ block_offsets,
+                                                        const int64_t* __restrict__ n_out,
+                                                        int64_t capacity,
+                                                        uint32_t* __restrict__ src) {
+  __shared__ uint32_t s_w[kDpThreads / 32];
+  if (*n_out > capacity) return;  // nothing is written
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t i = (int64_t)blockIdx.x * kDpThreads + threadIdx.x;
+  const int8_t c = i < n ? codes[i] : kPrune;
+  const uint32_t cnt = (uint32_t)dp_count(c);
+  uint32_t incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) s_w[warp] = incl;
+  __syncthreads();
+  uint32_t before = 0;
+#pragma unroll
+  for (int w = 0; w < kDpThreads / 32; ++w) before += w < warp ? s_w[w] : 0u;
+  const int64_t pos = (int64_t)block_offsets[blockIdx.x] + before + incl - cnt;
+  const uint32_t id = (uint32_t)i, zero = 0x80000000u;
+  if (c == kKeep) {
+    src[pos] = id;
+  } else if (c == kClone) {
+    src[pos] = id;
+    src[pos + 1] = id | zero;
+  } else if (c == kSplit) {
+    src[pos] = id | zero;
+    src[pos + 1] = id | zero;
+  }
+}
+
 
 DpConst to_const(const DpTensorPtrs& t) {
   return DpConst{reinterpret_cast<const float4*>(t.means), reinterpret_cast<const float4*>(t.log_scales),
@@ -290,6 +349,17 @@ cudaError_t launch_densify_and_prune(const DpTensorPtrs& p_in, const DpTensorPtr
   k_dp_emit<<<nb, kDpThreads, 0, stream>>>(to_const(p_in), to_const(m_in), to_const(v_in), z, n,
                                            k3, args.log_split_shrink, codes, block_counts, n_out,
                                            capacity, to_mut(p_out), to_mut(m_out), to_mut(v_out));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_densify_map(const int8_t* decisions, int n, uint32_t* block_counts,
+                               int64_t capacity, int64_t* n_out, uint32_t* src,
+                               uint32_t* status, cudaStream_t stream) {
+  const int nb = (int)densify_blocks(n);
+  if (nb == 0) return cudaMemsetAsync(n_out, 0, sizeof(int64_t), stream);
+  k_dsq_count<<<nb, kDpThreads, 0, stream>>>(decisions, n, block_counts);
+  k_dp_scan<<<1, 1024, 0, stream>>>(block_counts, nb, capacity, n_out, status);
+  k_dsq_map<<<nb, kDpThreads, 0, stream>>>(decisions, n, block_counts, n_out, capacity, src);
   return cudaGetLastError();
 }
 

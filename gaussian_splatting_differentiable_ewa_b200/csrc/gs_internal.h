@@ -44,9 +44,12 @@ struct BinSortArgs {
   uint32_t* counts;                  // [256][counts_stride] radix digit counts / offsets
   int64_t counts_stride;             // partitions of the largest pass, a multiple of 4
   uint64_t* emit_lookback;           // [emit blocks]
+  uint32_t* digit_hist;              // [8][256] digit counts of every single-sweep pass
+  uint64_t* sweep_lookback;          // [partitions][256] single-sweep look-back words
   uint32_t* counters;                // [16] dynamic block counters
   uint32_t* status;
-  WaitCfg wait;                      // look-back wait limit (and test stall)
+  WaitCfg wait;                      // emission look-back wait limit (and test stall)
+  WaitCfg sort_wait;                 // single-sweep look-back wait limit (and test stall)
   int64_t* n_pairs;
   int64_t* n_items_dev;
   unsigned long long* pair_total;  // column emission: exact pair count
@@ -58,6 +61,30 @@ struct BinSortArgs {
   int64_t* ranges;
   int64_t n_tiles;     // n_views * tiles per view
 };
+
+// Quantised SH as the kernels read it: the codes of value j of Gaussian i at
+// j * n_pad + i (planar, 8 or 16 bits) or in word 32 + ... of block
+// (j, i / 32) of the packed layout; bounds (min, max) per (j, i / 256).
+enum { kShqPlanar8 = 0, kShqPlanar16 = 1, kShqPacked = 2 };
+struct ShQuant {
+  const void* codes;
+  const float2* bounds;
+  int64_t n_pad;
+  int64_t n_groups;
+  float qmax;
+  int kind;
+};
+inline ShQuant shq_of(const gs_sh_quant* q) {
+  ShQuant r{};
+  if (!q) return r;
+  r.codes = q->codes;
+  r.bounds = reinterpret_cast<const float2*>(q->bounds);
+  r.n_pad = (q->n + GS_QUANT_GROUP - 1) / GS_QUANT_GROUP * GS_QUANT_GROUP;
+  r.n_groups = r.n_pad / GS_QUANT_GROUP;
+  r.qmax = (float)((1 << q->bits) - 1);
+  r.kind = q->layout == GS_QUANT_PACKED ? kShqPacked : (q->bits == 8 ? kShqPlanar8 : kShqPlanar16);
+  return r;
+}
 
 cudaError_t launch_project(const gs_params& p, const CamSet& cams, int n_views, float* records,
                            float* bins, int* radii, uint32_t* status, const WaitCfg& wc,
@@ -122,14 +149,26 @@ cudaError_t launch_l1_dssim(const float* image, const float* target, int n_views
                             float lambda, double* terms, float* grad, double* sums,
                             unsigned* done, cudaStream_t stream);
 
-// Quantised SH state: codes [k3][n_pad], bounds [k3][n_pad / 256].
-cudaError_t launch_sh_quantize(const float* sh, int64_t n, int k3, int bits, void* codes,
-                               float2* bounds, cudaStream_t stream);
-cudaError_t launch_sh_dequantize(const void* codes, const float2* bounds, int64_t n, int k3,
-                                 int bits, float* sh, cudaStream_t stream);
-cudaError_t launch_adam_sh_quant(void* codes, float2* bounds, const float* grad, uint16_t* m,
-                                 uint16_t* v, int64_t n, int k3, int bits, float lr, float beta1,
-                                 float beta2, float eps, int64_t step, int rounding,
-                                 uint64_t seed, cudaStream_t stream);
+// Quantised SH state (gs_sh_quant, either layout; bounds [k3][n_pad / 256]).
+cudaError_t launch_sh_quantize(const float* sh, const gs_sh_quant& q, cudaStream_t stream);
+cudaError_t launch_sh_dequantize(const gs_sh_quant& q, float* sh, cudaStream_t stream);
+cudaError_t launch_adam_sh_quant(const gs_sh_quant& q, const float* grad, uint16_t* m,
+                                 uint16_t* v, float lr, float beta1, float beta2, float eps,
+                                 int64_t step, int rounding, uint64_t seed, cudaStream_t stream);
+// Output positions of densify_and_prune from its decisions: per-block output
+// counts, their scan (checked against capacity, the count to *n_out), and the
+// map src[o] = input of output o, bit 31 set where its moments start at zero.
+cudaError_t launch_densify_map(const int8_t* decisions, int n, uint32_t* block_counts,
+                               int64_t capacity, int64_t* n_out, uint32_t* src,
+                               uint32_t* status, cudaStream_t stream);
+// densify_and_prune of quantised SH: output positions from the decisions
+// (block counts, their scan, the output -> input map src [n_out], bit 31 set
+// where the moments start at zero), then every output group decoded from its
+// inputs and encoded anew.
+cudaError_t launch_densify_sh_quant(const gs_sh_quant& in, const uint16_t* m_in,
+                                    const uint16_t* v_in, const int8_t* decisions,
+                                    const gs_sh_quant& out, uint16_t* m_out, uint16_t* v_out,
+                                    uint32_t* block_counts, int64_t* n_out_dev, uint32_t* src,
+                                    uint32_t* status, cudaStream_t stream);
 
 }  // namespace gsb

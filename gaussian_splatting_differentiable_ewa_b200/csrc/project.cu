@@ -14,8 +14,16 @@
 // summing the views in registers before one write of every gradient; the
 // block's SH coefficients stream into shared memory (cp.async) while the
 // parameters load and the view-independent part is computed.
+//
+// Quantised SH (the Spirula page's codes with per-256 bounds): both kernels
+// read the codes where they use them and decode each one as the decoder
+// does, fma(q, (max - min) / (2^b - 1), min), so colour and gradients equal
+// those of the float path on the decoded coefficients bit for bit. A forward
+// block of 256 Gaussians is one group of the codes.
 
 #include <cuda_runtime.h>
+
+#include <type_traits>
 
 #include "gs_internal.h"
 
@@ -118,6 +126,7 @@ constexpr double kLog2_255 = 7.9943534368588578;    // log2(255)
 constexpr int kProjThreads = 128;     // projection backward block
 constexpr int kProjFwdThreads = 256;  // projection forward block
 constexpr int kShStride = kProjThreads + 1;  // padded row: conflict-free banks
+constexpr int kFwdQStride = kProjFwdThreads + 1;  // forward, decoded codes
 
 // Stage the SH coefficients of Gaussians [i0, i0 + cnt) in shared memory,
 // coefficient-major with a padded row (s[c * kShStride + local i]), by
@@ -215,7 +224,63 @@ __device__ __forceinline__ bool sh_colour_smem(const float* __restrict__ shi, fl
   return isfinite(acc[0] + acc[1] + acc[2]);  // before the clamp, which drops a NaN
 }
 
-template <int DEG>
+// (min, step) of value j in group g, the step rounded as the decoder rounds it.
+__device__ __forceinline__ float2 shq_scale(const ShQuant& q, int j, int64_t g) {
+  const float2 b = __ldg(q.bounds + (int64_t)j * q.n_groups + g);
+  return make_float2(b.x, __fdiv_rn(__fsub_rn(b.y, b.x), q.qmax));
+}
+
+// Colour from coefficients staged coefficient-major in shared memory
+// (shi[idx * STRIDE]), same arithmetic as sh_colour_smem.
+template <int DEG, int STRIDE>
+__device__ __forceinline__ bool sh_colour_strided(const float* __restrict__ shi, float x, float y,
+                                                  float z, float rgb[3]) {
+  constexpr int K = (DEG + 1) * (DEG + 1);
+  float Y[16];
+  sh_basis<DEG>(x, y, z, Y);
+  float acc[3] = {0.5f, 0.5f, 0.5f};
+#pragma unroll
+  for (int idx = 0; idx < K * 3; ++idx)
+    acc[idx % 3] = fmaf(Y[idx / 3], shi[idx * STRIDE], acc[idx % 3]);
+#pragma unroll
+  for (int ch = 0; ch < 3; ++ch) rgb[ch] = fmaxf(acc[ch], 0.f);
+  return isfinite(acc[0] + acc[1] + acc[2]);  // before the clamp, which drops a NaN
+}
+
+// The K3 decoded coefficients of Gaussian i into dst[c * STRIDE]: each
+// thread its own Gaussian, so a warp's loads of one coefficient are
+// consecutive codes, twelve loads in flight at a time.
+template <int K3, int KIND, int STRIDE>
+__device__ __forceinline__ void decode_codes(const ShQuant& q, const float2* s_qs, int64_t i,
+                                             float* dst) {
+  using T = typename std::conditional<KIND == kShqPlanar8, uint8_t, unsigned short>::type;
+  const int64_t base = KIND == kShqPacked ? (i >> 5) * 96 + (i & 31) : i;
+  const int64_t stride = KIND == kShqPacked ? (q.n_pad >> 5) * 96 : q.n_pad;
+  const T* p = static_cast<const T*>(q.codes) + base;
+  constexpr int kChunk = K3 < 12 ? K3 : 12;
+#pragma unroll
+  for (int c0 = 0; c0 < K3; c0 += kChunk) {
+    float cv[kChunk];
+#pragma unroll
+    for (int k = 0; k < kChunk; ++k) {
+      if (c0 + k < K3) cv[k] = (float)__ldg(p);
+      p += stride;
+    }
+#pragma unroll
+    for (int k = 0; k < kChunk; ++k) {
+      const int c = c0 + k;
+      if (c >= K3) break;
+      const float2 sc = s_qs[c];
+      dst[c * STRIDE] = __fmaf_rn(cv[k], sc.y, sc.x);
+    }
+  }
+}
+
+static_assert(kProjFwdThreads == GS_QUANT_GROUP, "a forward block is one group of the codes");
+
+// QK: -1 float SH, else the kind of quantised codes (compile-time, so the
+// decode carries no layout branches).
+template <int DEG, int QK>
 __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __restrict__ means,
                                                           const float4* __restrict__ log_scales,
                                                           const float4* __restrict__ quats,
@@ -226,15 +291,26 @@ __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __
                                                           float4* __restrict__ bins,
                                                           int* __restrict__ radii,
                                                           uint32_t* __restrict__ status,
-                                                          uint64_t wait_ns) {
+                                                          uint64_t wait_ns, ShQuant shq) {
   constexpr int K = (DEG + 1) * (DEG + 1);
+  constexpr bool QUANT = QK >= 0;
   // the block's SH coefficients are one contiguous range: a full block with a
   // 16-byte-aligned array fetches them with one bulk copy that lands while
   // the geometry is computed
-  extern __shared__ __align__(16) float s_sh[];  // [kProjFwdThreads][K * 3]
+  extern __shared__ __align__(16) float s_sh[];  // [kProjFwdThreads][K * 3] (codes: [K * 3][257])
   __shared__ __align__(8) uint64_t s_bar;
+  __shared__ float2 s_qs[QUANT ? 48 : 1];       // quantised: (min, step) per value
   const int64_t i0 = (int64_t)blockIdx.x * kProjFwdThreads;
-  const bool staged = ((reinterpret_cast<uintptr_t>(sh) & 15) == 0) &&
+  if constexpr (QUANT) {
+    // the block's codes decoded at once into s_sh [K * 3][kFwdQStride], each
+    // thread its own Gaussian's column (read back only by that thread)
+    if (threadIdx.x < K * 3) s_qs[threadIdx.x] = shq_scale(shq, threadIdx.x, blockIdx.x);
+    __syncthreads();
+    if (i0 + threadIdx.x < (int64_t)n)
+      decode_codes<K * 3, (QK < 0 ? 0 : QK), kFwdQStride>(shq, s_qs, i0 + threadIdx.x,
+                                                         s_sh + threadIdx.x);
+  }
+  const bool staged = !QUANT && ((reinterpret_cast<uintptr_t>(sh) & 15) == 0) &&
                       i0 + kProjFwdThreads <= (int64_t)n;
   if (staged) {
     if (threadIdx.x == 0) {
@@ -275,7 +351,7 @@ __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __
   const double opac_d = 1.0 / (1.0 + exp(-(double)lg));
   // alpha >= 1/255 needs q <= Q = 2 ln(255 o); Q <= 0: the splat never counts
   const double Qa = 2.0 * log(255.0 * opac_d);
-  const float* shi = sh + (size_t)i * K * 3;
+  const float* shi = QUANT ? nullptr : sh + (size_t)i * K * 3;
 
   const Grid g = grid_of(cams.c[0]);
   for (int v = 0; v < n_views; ++v) {
@@ -389,7 +465,10 @@ __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __
           float rgb[3];
           bool colour_finite;
           if (staged && !sh_ready) sh_ready = mbar_wait_bounded(&s_bar, 0u, wait_ns, status);
-          if (sh_ready && staged) {
+          if constexpr (QUANT) {
+            colour_finite = sh_colour_strided<DEG, kFwdQStride>(s_sh + threadIdx.x, dxv * inv,
+                                                                 dyv * inv, dzv * inv, rgb);
+          } else if (sh_ready && staged) {
             colour_finite = sh_colour_smem<DEG>(s_sh + (size_t)threadIdx.x * K * 3, dxv * inv,
                                                 dyv * inv, dzv * inv, rgb);
           } else {  // not staged, or the staging copy did not land in time
@@ -435,14 +514,14 @@ __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __
 // (coefficient-major, coalesced global traffic); the SH gradients are summed
 // over views in shared memory rather than in registers. With ALIAS (one view)
 // the gradients overwrite the staged coefficients slot by slot.
-template <int DEG, bool ALIAS>
+template <int DEG, bool ALIAS, bool QUANT>
 __global__ void __launch_bounds__(kProjThreads, 6) k_project_bwd(
     const float4* __restrict__ means, const float4* __restrict__ log_scales,
     const float4* __restrict__ quats, const float* __restrict__ logit,
     const float* __restrict__ sh, const float4* __restrict__ grad2d,
     const int* __restrict__ radii, int n, int n_views, CamSet cams, float4* __restrict__ g_means,
     float4* __restrict__ g_log_scales, float4* __restrict__ g_quats, float* __restrict__ g_logit,
-    float* __restrict__ g_sh) {
+    float* __restrict__ g_sh, ShQuant shq) {
   constexpr int K = (DEG + 1) * (DEG + 1);
   constexpr int K3 = K * 3;
   extern __shared__ float s_pb[];
@@ -450,9 +529,26 @@ __global__ void __launch_bounds__(kProjThreads, 6) k_project_bwd(
   float* s_dsh = ALIAS ? s_pb : s_pb + K3 * kShStride;  // [K3][kShStride]
   const int64_t i0 = (int64_t)blockIdx.x * kProjThreads;
   const int cnt = (int)min((int64_t)kProjThreads, (int64_t)n - i0);
-  // the coefficients stream into shared memory while the parameters load and
-  // the view-independent part is computed
-  stage_sh_async<K3>(sh, i0, cnt, s_coef);
+  if constexpr (QUANT) {
+    // decoded into the same coefficient-major slots (coalesced code reads)
+    __shared__ float2 s_qs[K3];
+    if (threadIdx.x < K3) s_qs[threadIdx.x] = shq_scale(shq, threadIdx.x, i0 / GS_QUANT_GROUP);
+    __syncthreads();
+    if ((int)threadIdx.x < cnt) {
+      const int64_t i = i0 + threadIdx.x;
+      float* dst = s_coef + threadIdx.x;
+      if (shq.kind == kShqPlanar8)
+        decode_codes<K3, kShqPlanar8, kShStride>(shq, s_qs, i, dst);
+      else if (shq.kind == kShqPlanar16)
+        decode_codes<K3, kShqPlanar16, kShStride>(shq, s_qs, i, dst);
+      else
+        decode_codes<K3, kShqPacked, kShStride>(shq, s_qs, i, dst);
+    }
+  } else {
+    // the coefficients stream into shared memory while the parameters load
+    // and the view-independent part is computed
+    stage_sh_async<K3>(sh, i0, cnt, s_coef);
+  }
   if (!ALIAS) {
 #pragma unroll
     for (int c = 0; c < K3; ++c) s_dsh[c * kShStride + threadIdx.x] = 0.f;
@@ -650,12 +746,24 @@ cudaError_t launch_project(const gs_params& p, const CamSet& cams, int n_views, 
   auto q = reinterpret_cast<const float4*>(p.quats);
   auto r = reinterpret_cast<float4*>(records);
   auto b = reinterpret_cast<float4*>(bins);
-#define GS_PFWD(D)                                                                          \
-  {                                                                                         \
-    const int smem = threads * 3 * (D + 1) * (D + 1) * (int)sizeof(float);                  \
-    cudaFuncSetAttribute(k_project<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);   \
-    k_project<D><<<blocks, threads, smem, stream>>>(m, s, q, p.opacity_logit, p.sh, n, n_views, \
-                                                    cams, r, b, radii, status, wc.limit_ns); \
+  const ShQuant shq = shq_of(p.sh_quant);
+#define GS_PFWD1(D, Q)                                                                       \
+  {                                                                                          \
+    const int smem = (Q >= 0 ? kFwdQStride : threads) * 3 * (D + 1) * (D + 1) * (int)sizeof(float); \
+    cudaFuncSetAttribute(k_project<D, Q>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); \
+    k_project<D, Q><<<blocks, threads, smem, stream>>>(m, s, q, p.opacity_logit, p.sh, n,     \
+                                                       n_views, cams, r, b, radii, status,    \
+                                                       wc.limit_ns, shq);                     \
+  }
+#define GS_PFWD(D)                                 \
+  if (!p.sh_quant) {                               \
+    GS_PFWD1(D, -1);                               \
+  } else if (shq.kind == kShqPlanar8) {            \
+    GS_PFWD1(D, kShqPlanar8);                      \
+  } else if (shq.kind == kShqPlanar16) {           \
+    GS_PFWD1(D, kShqPlanar16);                     \
+  } else {                                         \
+    GS_PFWD1(D, kShqPacked);                       \
   }
   switch (p.sh_degree) {
     case 0: GS_PFWD(0); break;
@@ -664,6 +772,7 @@ cudaError_t launch_project(const gs_params& p, const CamSet& cams, int n_views, 
     default: GS_PFWD(3); break;
   }
 #undef GS_PFWD
+#undef GS_PFWD1
   return cudaGetLastError();
 }
 
@@ -677,6 +786,7 @@ cudaError_t launch_project_bwd(const gs_params& p, const CamSet& cams, int n_vie
   const int K3 = 3 * (p.sh_degree + 1) * (p.sh_degree + 1);
   const bool alias = n_views == 1;
   const size_t smem = (size_t)(alias ? 1 : 2) * K3 * kShStride * sizeof(float);
+  const ShQuant shq = shq_of(p.sh_quant);
   auto m = reinterpret_cast<const float4*>(p.means);
   auto s = reinterpret_cast<const float4*>(p.log_scales);
   auto q = reinterpret_cast<const float4*>(p.quats);
@@ -684,12 +794,18 @@ cudaError_t launch_project_bwd(const gs_params& p, const CamSet& cams, int n_vie
   auto gm = reinterpret_cast<float4*>(g.means);
   auto gs = reinterpret_cast<float4*>(g.log_scales);
   auto gq = reinterpret_cast<float4*>(g.quats);
-#define GS_PBWD1(D, AL)                                                                      \
-  cudaFuncSetAttribute(k_project_bwd<D, AL>, cudaFuncAttributeMaxDynamicSharedMemorySize,      \
+#define GS_PBWD2(D, AL, Q)                                                                   \
+  cudaFuncSetAttribute(k_project_bwd<D, AL, Q>, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
                        (int)smem);                                                              \
-  k_project_bwd<D, AL><<<blocks, threads, smem, stream>>>(m, s, q, p.opacity_logit, p.sh, g2,   \
-                                                          radii, n, n_views, cams, gm, gs, gq,  \
-                                                          g.opacity_logit, g.sh)
+  k_project_bwd<D, AL, Q><<<blocks, threads, smem, stream>>>(                                   \
+      m, s, q, p.opacity_logit, p.sh, g2, radii, n, n_views, cams, gm, gs, gq, g.opacity_logit, \
+      g.sh, shq)
+#define GS_PBWD1(D, AL)       \
+  if (p.sh_quant) {           \
+    GS_PBWD2(D, AL, true);    \
+  } else {                    \
+    GS_PBWD2(D, AL, false);   \
+  }
 #define GS_PBWD(D)            \
   if (alias) {                \
     GS_PBWD1(D, true);        \
@@ -704,6 +820,7 @@ cudaError_t launch_project_bwd(const gs_params& p, const CamSet& cams, int n_vie
   }
 #undef GS_PBWD
 #undef GS_PBWD1
+#undef GS_PBWD2
   return cudaGetLastError();
 }
 

@@ -1,22 +1,27 @@
-// quant.cu -- quantised SH state: encode, decode, and Adam on the codes.
+// quant.cu -- quantised SH state: encode, decode, Adam on the codes, and
+// densify_and_prune of the codes.
 //
 // The Spirula VRAM page (sec. 魔法一, quantised training) keeps the SH
 // coefficients as 8- or 16-bit fixed point, every 256 units sharing one
-// (min, max) pair, gradients in float32 and the Adam moments in 16-bit words
-// in a transposed layout. Here a unit is one SH value and the layout is
-// coefficient-major: codes [3K][n_pad], one group = one coefficient of 256
-// consecutive Gaussians, bounds float2 [3K][n_pad / 256]; the moments are
-// bfloat16 [3K][n_pad] beside them. A code q decodes to
-// min + q (max - min) / (2^b - 1).
+// (min, max) pair, gradients in float32 and the Adam state in 16-bit words,
+// parameter and moments transposed and packed together. Here a unit is one SH
+// value and both layouts are coefficient-major, one group = one coefficient of
+// 256 consecutive Gaussians, bounds float2 [3K][n_pad / 256]:
+//   planar  codes [3K][n_pad] (8 or 16 bits), bfloat16 moments [3K][n_pad]
+//           in two arrays beside them;
+//   packed  uint16 blocks [3K][n_pad / 32][3][32]: the codes of 32
+//           consecutive Gaussians, then their two moments, 192 bytes.
+// A code q decodes to min + q (max - min) / (2^b - 1).
 //
 // One 256-thread block owns one group of Gaussians for every coefficient.
 // The float32 SH (or its gradient) of those Gaussians, [256][3K] in the
 // parameter layout, is staged through shared memory transposed, so that a
 // warp then works on whole coefficients: lane l holds the four consecutive
-// Gaussians 4 l .. 4 l + 3 of each half of the group, moves their codes and
-// moments with one vector access per array and half, and takes the group's
-// min and max with warp shuffles. Loads are issued for both halves before
-// any arithmetic, so each warp keeps six vector loads in flight.
+// Gaussians 4 l .. 4 l + 3 of each half of the group (always inside one
+// packed block), moves their codes and moments with one vector access per
+// array and half, and takes the group's min and max with warp shuffles.
+// Loads are issued for both halves before any arithmetic, so each warp keeps
+// six vector loads in flight.
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -62,6 +67,33 @@ struct CodeT<16> {
   __device__ static Vec pack(const int (&c)[4]) {
     return make_uint2((uint32_t)c[0] | ((uint32_t)c[1] << 16),
                       (uint32_t)c[2] | ((uint32_t)c[3] << 16));
+  }
+};
+
+// Where the four values (j, i .. i + 3) of a layout live (i a multiple of 4).
+// S is the stored code type (packed blocks hold 16-bit words for 8-bit codes
+// too); the moments follow the codes of a packed block at +32 and +64 words.
+template <int BITS, int LAYOUT>
+struct QL;
+template <int BITS>
+struct QL<BITS, GS_QUANT_PLANAR> {
+  using S = CodeT<BITS>;
+  __device__ static typename S::T* code(void* codes, int j, int64_t i, int64_t n_pad) {
+    return static_cast<typename S::T*>(codes) + (int64_t)j * n_pad + i;
+  }
+  __device__ static uint16_t* mom(void*, uint16_t* arr, int, int j, int64_t i, int64_t n_pad) {
+    return arr + (int64_t)j * n_pad + i;
+  }
+};
+template <int BITS>
+struct QL<BITS, GS_QUANT_PACKED> {
+  using S = CodeT<16>;
+  __device__ static uint16_t* code(void* codes, int j, int64_t i, int64_t n_pad) {
+    return static_cast<uint16_t*>(codes) + (((int64_t)j * (n_pad >> 5) + (i >> 5)) * 96 + (i & 31));
+  }
+  __device__ static uint16_t* mom(void* codes, uint16_t*, int which, int j, int64_t i,
+                                  int64_t n_pad) {
+    return code(codes, j, i, n_pad) + 32 * which;
   }
 };
 
@@ -131,30 +163,35 @@ __device__ __forceinline__ void stage_transposed(const float* __restrict__ src, 
   }
 }
 
-// Store four consecutive values at row[base ..]: one vector store when all
-// four are real Gaussians, element stores for the ragged end of the last group.
+// Store four consecutive values at p: one vector store when all four are
+// real Gaussians (avail >= 4), element stores for the ragged end of the last
+// group.
 template <typename T, typename Vec>
-__device__ __forceinline__ void store4(T* row, int base, int cnt, Vec packed,
-                                       const T (&each)[4]) {
-  if (base + 4 <= cnt) {
-    *reinterpret_cast<Vec*>(row + base) = packed;
+__device__ __forceinline__ void store4(T* p, int avail, Vec packed, const T (&each)[4]) {
+  if (avail >= 4) {
+    *reinterpret_cast<Vec*>(p) = packed;
   } else {
 #pragma unroll
     for (int k = 0; k < 4; ++k)
-      if (base + k < cnt) row[base + k] = each[k];
+      if (k < avail) p[k] = each[k];
   }
+}
+
+__device__ __forceinline__ uint2 pack_bf16x4(const uint16_t (&b)[4]) {
+  return make_uint2(b[0] | ((uint32_t)b[1] << 16), b[2] | ((uint32_t)b[3] << 16));
 }
 
 // Encode the lane's values x[e] (group positions lane_pos(e) of coefficient
 // j) with the group's min and max, in float32 exactly as stated above:
 // t = (x - min) * ((2^b - 1) / (max - min)), then rint(t) or floor(t + u).
-template <int BITS>
+template <int BITS, int LAYOUT>
 __device__ __forceinline__ void encode_group(const float (&x)[kPerLane], int cnt, int j, int g,
                                              int64_t i0, int64_t n_pad, int n_groups,
-                                             typename CodeT<BITS>::T* __restrict__ codes,
+                                             void* __restrict__ codes,
                                              float2* __restrict__ bounds, int rounding,
                                              uint64_t seed, uint64_t ctr_base) {
-  using C = CodeT<BITS>;
+  using L = QL<BITS, LAYOUT>;
+  using C = typename L::S;
   float lo = INFINITY, hi = -INFINITY;
 #pragma unroll
   for (int e = 0; e < kPerLane; ++e)
@@ -168,7 +205,6 @@ __device__ __forceinline__ void encode_group(const float (&x)[kPerLane], int cnt
   constexpr int qmax = (1 << BITS) - 1;
   const float range = __fsub_rn(hi, lo);
   const float inv = range > 0.f ? __fdiv_rn((float)qmax, range) : 0.f;
-  typename C::T* row = codes + (int64_t)j * n_pad + i0;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     int c[4];
@@ -189,14 +225,13 @@ __device__ __forceinline__ void encode_group(const float (&x)[kPerLane], int cnt
       each[k] = (typename C::T)c[k];
     }
     const int base = lane_pos(4 * h);
-    if (base < cnt) store4(row, base, cnt, C::pack(c), each);
+    if (base < cnt) store4(L::code(codes, j, i0 + base, n_pad), cnt - base, C::pack(c), each);
   }
 }
 
-template <int BITS, int K3>
+template <int BITS, int K3, int LAYOUT>
 __global__ void __launch_bounds__(kQG) k_sh_quantize(const float* __restrict__ sh, int64_t n,
-                                                     int64_t n_pad,
-                                                     typename CodeT<BITS>::T* __restrict__ codes,
+                                                     int64_t n_pad, void* __restrict__ codes,
                                                      float2* __restrict__ bounds) {
   extern __shared__ float4 s_q4[];
   float* s_q = reinterpret_cast<float*>(s_q4);
@@ -218,16 +253,16 @@ __global__ void __launch_bounds__(kQG) k_sh_quantize(const float* __restrict__ s
       x[4 * h + 2] = v.z;
       x[4 * h + 3] = v.w;
     }
-    encode_group<BITS>(x, cnt, j, g, i0, n_pad, n_groups, codes, bounds, 0, 0, 0);
+    encode_group<BITS, LAYOUT>(x, cnt, j, g, i0, n_pad, n_groups, codes, bounds, 0, 0, 0);
   }
 }
 
-template <int BITS, int K3>
+template <int BITS, int K3, int LAYOUT>
 __global__ void __launch_bounds__(kQG)
-    k_sh_dequantize(const typename CodeT<BITS>::T* __restrict__ codes,
-                    const float2* __restrict__ bounds, int64_t n, int64_t n_pad,
-                    float* __restrict__ sh) {
-  using C = CodeT<BITS>;
+    k_sh_dequantize(const void* __restrict__ codes, const float2* __restrict__ bounds, int64_t n,
+                    int64_t n_pad, float* __restrict__ sh) {
+  using L = QL<BITS, LAYOUT>;
+  using C = typename L::S;
   extern __shared__ float4 s_q4[];
   float* s_q = reinterpret_cast<float*>(s_q4);
   const int g = blockIdx.x;
@@ -236,14 +271,15 @@ __global__ void __launch_bounds__(kQG)
   const int n_groups = (int)(n_pad / kQG);
   const int warp = threadIdx.x >> 5;
   constexpr float qmax = (float)((1 << BITS) - 1);
+  void* cw = const_cast<void*>(codes);
   for (int j = warp; j < K3; j += kQG / 32) {
     const float2 b = __ldg(bounds + (int64_t)j * n_groups + g);
     const float step = __fdiv_rn(__fsub_rn(b.y, b.x), qmax);
-    const typename C::T* row = codes + (int64_t)j * n_pad + i0;
     typename C::Vec w[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h)
-      w[h] = __ldg(reinterpret_cast<const typename C::Vec*>(row + lane_pos(4 * h)));
+      w[h] = __ldg(reinterpret_cast<const typename C::Vec*>(
+          L::code(cw, j, i0 + lane_pos(4 * h), n_pad)));
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       float c[4];
@@ -265,14 +301,15 @@ __global__ void __launch_bounds__(kQG)
   }
 }
 
-template <int BITS, int K3>
+template <int BITS, int K3, int LAYOUT>
 __global__ void __launch_bounds__(kQG)
-    k_adam_sh_quant(typename CodeT<BITS>::T* __restrict__ codes, float2* __restrict__ bounds,
+    k_adam_sh_quant(void* __restrict__ codes, float2* __restrict__ bounds,
                     const float* __restrict__ grad, uint16_t* __restrict__ m_buf,
                     uint16_t* __restrict__ v_buf, int64_t n, int64_t n_pad, float lr,
                     float beta1, float beta2, float eps, float ibc1, float ibc2, int rounding,
                     uint64_t seed, uint64_t ctr_base) {
-  using C = CodeT<BITS>;
+  using L = QL<BITS, LAYOUT>;
+  using C = typename L::S;
   extern __shared__ float4 s_q4[];
   float* s_q = reinterpret_cast<float*>(s_q4);
   const int g = blockIdx.x;
@@ -286,20 +323,18 @@ __global__ void __launch_bounds__(kQG)
   typename C::Vec w[2];
   uint2 mw[2], vw[2];
   auto load_coef = [&](int j) {
-    const int64_t off = (int64_t)j * n_pad + i0;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int base = lane_pos(4 * h);
-      w[h] = *reinterpret_cast<const typename C::Vec*>(codes + off + base);
-      mw[h] = *reinterpret_cast<const uint2*>(m_buf + off + base);
-      vw[h] = *reinterpret_cast<const uint2*>(v_buf + off + base);
+      const int64_t i = i0 + lane_pos(4 * h);
+      w[h] = *reinterpret_cast<const typename C::Vec*>(L::code(codes, j, i, n_pad));
+      mw[h] = *reinterpret_cast<const uint2*>(L::mom(codes, m_buf, 1, j, i, n_pad));
+      vw[h] = *reinterpret_cast<const uint2*>(L::mom(codes, v_buf, 2, j, i, n_pad));
     }
   };
   if (warp < K3) load_coef(warp);
   stage_transposed<K3>(grad + i0 * K3, cnt, s_q, (reinterpret_cast<uintptr_t>(grad) & 15) == 0);
   __syncthreads();
   for (int j = warp; j < K3; j += kQG / 32) {
-    const int64_t off = (int64_t)j * n_pad + i0;
     const float2 b = bounds[(int64_t)j * n_groups + g];
     if (j != warp) load_coef(j);   // the padding past n is in bounds
     const float step = __fdiv_rn(__fsub_rn(b.y, b.x), qmax);
@@ -324,18 +359,78 @@ __global__ void __launch_bounds__(kQG)
         vb[k] = bf16_bits(v[k]);
       }
       if (base < cnt) {
-        store4(m_buf + off, base, cnt,
-               make_uint2(mb[0] | ((uint32_t)mb[1] << 16), mb[2] | ((uint32_t)mb[3] << 16)),
-               mb);
-        store4(v_buf + off, base, cnt,
-               make_uint2(vb[0] | ((uint32_t)vb[1] << 16), vb[2] | ((uint32_t)vb[3] << 16)),
-               vb);
+        const int64_t i = i0 + base;
+        store4(L::mom(codes, m_buf, 1, j, i, n_pad), cnt - base, pack_bf16x4(mb), mb);
+        store4(L::mom(codes, v_buf, 2, j, i, n_pad), cnt - base, pack_bf16x4(vb), vb);
       }
     }
     // every lane has read the group's old bounds before lane 0 rewrites them
     __syncwarp();
-    encode_group<BITS>(x, cnt, j, g, i0, n_pad, n_groups, codes, bounds, rounding, seed,
-                       ctr_base);
+    encode_group<BITS, LAYOUT>(x, cnt, j, g, i0, n_pad, n_groups, codes, bounds, rounding, seed,
+                               ctr_base);
+  }
+}
+
+// densify_and_prune of the codes: output group g (256 outputs) takes, for
+// every coefficient, the decoded values of the inputs src[o] & 0x7fffffff
+// it comes from, writes their moments (zero where bit 31 of src[o] is set)
+// and encodes the group anew with nearest rounding. A count that differs
+// from the map's (*n_out_dev) writes nothing and reports.
+template <int BITS, int K3, int LAYOUT>
+__global__ void __launch_bounds__(kQG)
+    k_dsq_emit(const void* __restrict__ in_codes, const float2* __restrict__ in_bounds,
+               const uint16_t* __restrict__ m_in, const uint16_t* __restrict__ v_in,
+               int64_t n_pad_in, const uint32_t* __restrict__ src,
+               const int64_t* __restrict__ n_out_dev, int64_t n_out, int64_t n_pad_out,
+               void* __restrict__ out_codes, float2* __restrict__ out_bounds,
+               uint16_t* __restrict__ m_out, uint16_t* __restrict__ v_out,
+               uint32_t* __restrict__ status) {
+  using L = QL<BITS, LAYOUT>;
+  using C = typename L::S;
+  if (*n_out_dev != n_out) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, kStatusCapacity);
+    return;
+  }
+  const int g = blockIdx.x;
+  const int64_t i0 = (int64_t)g * kQG;
+  const int cnt = (int)(n_out - i0 < kQG ? n_out - i0 : kQG);
+  const int n_groups_in = (int)(n_pad_in / kQG), n_groups_out = (int)(n_pad_out / kQG);
+  const int warp = threadIdx.x >> 5;
+  constexpr float qmax = (float)((1 << BITS) - 1);
+  void* icw = const_cast<void*>(in_codes);
+  uint16_t* mi = const_cast<uint16_t*>(m_in);
+  uint16_t* vi = const_cast<uint16_t*>(v_in);
+  uint32_t sv[kPerLane];
+#pragma unroll
+  for (int e = 0; e < kPerLane; ++e) sv[e] = lane_pos(e) < cnt ? __ldg(&src[i0 + lane_pos(e)]) : 0u;
+  for (int j = warp; j < K3; j += kQG / 32) {
+    float x[kPerLane];
+    uint16_t mb[kPerLane], vb[kPerLane];
+#pragma unroll
+    for (int e = 0; e < kPerLane; ++e) {
+      const int64_t i = sv[e] & 0x7fffffffu;
+      const bool zero = (sv[e] >> 31) != 0u;
+      const float2 b = __ldg(in_bounds + (int64_t)j * n_groups_in + (i >> 8));
+      const float step = __fdiv_rn(__fsub_rn(b.y, b.x), qmax);
+      const float q = (float)*L::code(icw, j, i, n_pad_in);
+      x[e] = __fmaf_rn(q, step, b.x);
+      mb[e] = zero ? (uint16_t)0 : *L::mom(icw, mi, 1, j, i, n_pad_in);
+      vb[e] = zero ? (uint16_t)0 : *L::mom(icw, vi, 2, j, i, n_pad_in);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int base = lane_pos(4 * h);
+      if (base < cnt) {
+        const uint16_t m4[4] = {mb[4 * h], mb[4 * h + 1], mb[4 * h + 2], mb[4 * h + 3]};
+        const uint16_t v4[4] = {vb[4 * h], vb[4 * h + 1], vb[4 * h + 2], vb[4 * h + 3]};
+        store4(L::mom(out_codes, m_out, 1, j, i0 + base, n_pad_out), cnt - base, pack_bf16x4(m4),
+               m4);
+        store4(L::mom(out_codes, v_out, 2, j, i0 + base, n_pad_out), cnt - base, pack_bf16x4(v4),
+               v4);
+      }
+    }
+    encode_group<BITS, LAYOUT>(x, cnt, j, g, i0, n_pad_out, n_groups_out, out_codes, out_bounds,
+                               0, 0, 0);
   }
 }
 
@@ -356,75 +451,98 @@ cudaError_t with_k3(int k3, F&& f) {
   }
 }
 
+// Calls f(integral_constant BITS, integral_constant LAYOUT) for the state's
+// code width and layout.
+template <typename F>
+cudaError_t with_bits_layout(const gs_sh_quant& q, F&& f) {
+  const bool packed = q.layout == GS_QUANT_PACKED;
+  if (q.bits == 8)
+    return packed ? f(std::integral_constant<int, 8>(), std::integral_constant<int, 1>())
+                  : f(std::integral_constant<int, 8>(), std::integral_constant<int, 0>());
+  return packed ? f(std::integral_constant<int, 16>(), std::integral_constant<int, 1>())
+                : f(std::integral_constant<int, 16>(), std::integral_constant<int, 0>());
+}
+
+int64_t padded(int64_t n) { return (n + kQG - 1) / kQG * kQG; }
+
 }  // namespace
 
-cudaError_t launch_sh_quantize(const float* sh, int64_t n, int k3, int bits, void* codes,
-                               float2* bounds, cudaStream_t stream) {
-  const int64_t n_pad = (n + kQG - 1) / kQG * kQG;
+cudaError_t launch_sh_quantize(const float* sh, const gs_sh_quant& q, cudaStream_t stream) {
+  const int64_t n_pad = padded(q.n);
   const unsigned grid = (unsigned)(n_pad / kQG);
-  const size_t smem = sizeof(float) * k3 * kQPitch;
-  return with_k3(k3, [&](auto K) -> cudaError_t {
-    constexpr int K3 = decltype(K)::value;
-    cudaError_t e;
-    if (bits == 8) {
-      if ((e = set_smem(k_sh_quantize<8, K3>, smem)) != cudaSuccess) return e;
-      k_sh_quantize<8, K3><<<grid, kQG, smem, stream>>>(sh, n, n_pad,
-                                                         static_cast<uint8_t*>(codes), bounds);
-    } else {
-      if ((e = set_smem(k_sh_quantize<16, K3>, smem)) != cudaSuccess) return e;
-      k_sh_quantize<16, K3><<<grid, kQG, smem, stream>>>(sh, n, n_pad,
-                                                          static_cast<uint16_t*>(codes), bounds);
-    }
-    return cudaGetLastError();
+  const size_t smem = sizeof(float) * q.k3 * kQPitch;
+  auto bounds = reinterpret_cast<float2*>(q.bounds);
+  return with_k3(q.k3, [&](auto K) -> cudaError_t {
+    return with_bits_layout(q, [&](auto B, auto LY) -> cudaError_t {
+      constexpr int K3 = decltype(K)::value, BITS = decltype(B)::value, LAY = decltype(LY)::value;
+      cudaError_t e = set_smem(k_sh_quantize<BITS, K3, LAY>, smem);
+      if (e != cudaSuccess) return e;
+      k_sh_quantize<BITS, K3, LAY><<<grid, kQG, smem, stream>>>(sh, q.n, n_pad, q.codes, bounds);
+      return cudaGetLastError();
+    });
   });
 }
 
-cudaError_t launch_sh_dequantize(const void* codes, const float2* bounds, int64_t n, int k3,
-                                 int bits, float* sh, cudaStream_t stream) {
-  const int64_t n_pad = (n + kQG - 1) / kQG * kQG;
+cudaError_t launch_sh_dequantize(const gs_sh_quant& q, float* sh, cudaStream_t stream) {
+  const int64_t n_pad = padded(q.n);
   const unsigned grid = (unsigned)(n_pad / kQG);
-  const size_t smem = sizeof(float) * k3 * kQPitch;
-  return with_k3(k3, [&](auto K) -> cudaError_t {
-    constexpr int K3 = decltype(K)::value;
-    cudaError_t e;
-    if (bits == 8) {
-      if ((e = set_smem(k_sh_dequantize<8, K3>, smem)) != cudaSuccess) return e;
-      k_sh_dequantize<8, K3><<<grid, kQG, smem, stream>>>(static_cast<const uint8_t*>(codes),
-                                                           bounds, n, n_pad, sh);
-    } else {
-      if ((e = set_smem(k_sh_dequantize<16, K3>, smem)) != cudaSuccess) return e;
-      k_sh_dequantize<16, K3><<<grid, kQG, smem, stream>>>(static_cast<const uint16_t*>(codes),
-                                                            bounds, n, n_pad, sh);
-    }
-    return cudaGetLastError();
+  const size_t smem = sizeof(float) * q.k3 * kQPitch;
+  auto bounds = reinterpret_cast<const float2*>(q.bounds);
+  return with_k3(q.k3, [&](auto K) -> cudaError_t {
+    return with_bits_layout(q, [&](auto B, auto LY) -> cudaError_t {
+      constexpr int K3 = decltype(K)::value, BITS = decltype(B)::value, LAY = decltype(LY)::value;
+      cudaError_t e = set_smem(k_sh_dequantize<BITS, K3, LAY>, smem);
+      if (e != cudaSuccess) return e;
+      k_sh_dequantize<BITS, K3, LAY><<<grid, kQG, smem, stream>>>(q.codes, bounds, q.n, n_pad,
+                                                                  sh);
+      return cudaGetLastError();
+    });
   });
 }
 
-cudaError_t launch_adam_sh_quant(void* codes, float2* bounds, const float* grad, uint16_t* m,
-                                 uint16_t* v, int64_t n, int k3, int bits, float lr, float beta1,
-                                 float beta2, float eps, int64_t step, int rounding,
-                                 uint64_t seed, cudaStream_t stream) {
-  const int64_t n_pad = (n + kQG - 1) / kQG * kQG;
+cudaError_t launch_adam_sh_quant(const gs_sh_quant& q, const float* grad, uint16_t* m,
+                                 uint16_t* v, float lr, float beta1, float beta2, float eps,
+                                 int64_t step, int rounding, uint64_t seed, cudaStream_t stream) {
+  const int64_t n_pad = padded(q.n);
   const unsigned grid = (unsigned)(n_pad / kQG);
-  const size_t smem = sizeof(float) * k3 * kQPitch;
+  const size_t smem = sizeof(float) * q.k3 * kQPitch;
   const float ibc1 = (float)(1.0 / (1.0 - pow((double)beta1, (double)step)));
   const float ibc2 = (float)(1.0 / (1.0 - pow((double)beta2, (double)step)));
   const uint64_t ctr_base = (uint64_t)step << 37;
-  return with_k3(k3, [&](auto K) -> cudaError_t {
-    constexpr int K3 = decltype(K)::value;
-    cudaError_t e;
-    if (bits == 8) {
-      if ((e = set_smem(k_adam_sh_quant<8, K3>, smem)) != cudaSuccess) return e;
-      k_adam_sh_quant<8, K3><<<grid, kQG, smem, stream>>>(
-          static_cast<uint8_t*>(codes), bounds, grad, m, v, n, n_pad, lr, beta1, beta2, eps,
-          ibc1, ibc2, rounding, seed, ctr_base);
-    } else {
-      if ((e = set_smem(k_adam_sh_quant<16, K3>, smem)) != cudaSuccess) return e;
-      k_adam_sh_quant<16, K3><<<grid, kQG, smem, stream>>>(
-          static_cast<uint16_t*>(codes), bounds, grad, m, v, n, n_pad, lr, beta1, beta2, eps,
-          ibc1, ibc2, rounding, seed, ctr_base);
-    }
-    return cudaGetLastError();
+  auto bounds = reinterpret_cast<float2*>(q.bounds);
+  return with_k3(q.k3, [&](auto K) -> cudaError_t {
+    return with_bits_layout(q, [&](auto B, auto LY) -> cudaError_t {
+      constexpr int K3 = decltype(K)::value, BITS = decltype(B)::value, LAY = decltype(LY)::value;
+      cudaError_t e = set_smem(k_adam_sh_quant<BITS, K3, LAY>, smem);
+      if (e != cudaSuccess) return e;
+      k_adam_sh_quant<BITS, K3, LAY><<<grid, kQG, smem, stream>>>(
+          q.codes, bounds, grad, m, v, q.n, n_pad, lr, beta1, beta2, eps, ibc1, ibc2, rounding,
+          seed, ctr_base);
+      return cudaGetLastError();
+    });
+  });
+}
+
+cudaError_t launch_densify_sh_quant(const gs_sh_quant& in, const uint16_t* m_in,
+                                    const uint16_t* v_in, const int8_t* decisions,
+                                    const gs_sh_quant& out, uint16_t* m_out, uint16_t* v_out,
+                                    uint32_t* block_counts, int64_t* n_out_dev, uint32_t* src,
+                                    uint32_t* status, cudaStream_t stream) {
+  cudaError_t e = launch_densify_map(decisions, (int)in.n, block_counts, out.n, n_out_dev, src,
+                                     status, stream);
+  if (e != cudaSuccess || out.n == 0) return e;
+  const int64_t n_pad_in = padded(in.n), n_pad_out = padded(out.n);
+  const unsigned grid = (unsigned)(n_pad_out / kQG);
+  auto ib = reinterpret_cast<const float2*>(in.bounds);
+  auto ob = reinterpret_cast<float2*>(out.bounds);
+  return with_k3(in.k3, [&](auto K) -> cudaError_t {
+    return with_bits_layout(in, [&](auto B, auto LY) -> cudaError_t {
+      constexpr int K3 = decltype(K)::value, BITS = decltype(B)::value, LAY = decltype(LY)::value;
+      k_dsq_emit<BITS, K3, LAY><<<grid, kQG, 0, stream>>>(in.codes, ib, m_in, v_in, n_pad_in,
+                                                          src, n_out_dev, out.n, n_pad_out,
+                                                          out.codes, ob, m_out, v_out, status);
+      return cudaGetLastError();
+    });
   });
 }
 

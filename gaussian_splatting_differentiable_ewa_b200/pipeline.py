@@ -78,9 +78,11 @@ class Splatter:
 
     # ------------------------------------------------------------ buffers
     def _alloc_gaussians(self, means, log_scales, quats, opacity_logit, sh, exp_avg=None,
-                         exp_avg_sq=None) -> None:
+                         exp_avg_sq=None, sh_state=None) -> None:
         """Adopt the given parameter values (and Adam moments, zero if None) and
-        (re)allocate every buffer whose size follows the Gaussian count.
+        (re)allocate every buffer whose size follows the Gaussian count. With
+        quantised SH, sh_state = (codes, bounds, exp_avg16, exp_avg_sq16) is
+        adopted as the SH state (else sh is quantised afresh).
 
         Parameters, gradients and both moments each live in one flat buffer,
         every group at a 16-byte aligned offset (the same offsets in all four)
@@ -130,12 +132,15 @@ class Splatter:
         if self.sh_bits is not None:
             self.exp_avg["sh"] = self.exp_avg_sq["sh"] = None
         if self.sh_bits is not None:
-            self._quantise_sh()
+            self._quantise_sh(sh_state)
         self.accum_plain = torch.zeros(n, dtype=f32, device=dev)
         self.accum_abs = torch.zeros(n, dtype=f32, device=dev)
         self.denom = torch.zeros(n, dtype=torch.int32, device=dev)
+        # with quantised SH the kernels read the codes themselves
+        quant = self.sh_bits is not None
         self.c_params = api.params(self.means, self.log_scales, self.quats, self.opacity_logit,
-                                   self.sh, self.deg)
+                                   None if quant else self.sh, self.deg,
+                                   sh_quant=self.sh_q if quant else None)
         self.c_grads = api.grads(*[self.grads[k] for k, _ in self.param_list])
         self.c_proj = api.projected(self.records, self.bins, self.radii)
         if getattr(self, "_shard", None) is not None:
@@ -143,22 +148,31 @@ class Splatter:
         if getattr(self, "ws", None) is not None:
             self._alloc_pairs(self.capacity)  # the workspace follows the count too
 
-    def _quantise_sh(self) -> None:
+    def _quantise_sh(self, state=None) -> None:
         """Quantised SH state: the SH live as codes with per-256 bounds and
-        bfloat16 Adam moments; ``self.sh`` becomes the float32 decode target
-        that the projection reads, refreshed before every forward."""
+        bfloat16 Adam moments, which the projection and its backward decode
+        where they use them; ``self.sh`` holds the decoded float32 values
+        for inspection (refresh_sh_float)."""
         if self.sh_bits not in (8, 16):
             raise ValueError("sh_bits must be 8 or 16")
         n, k3, dev = self.n, 3 * self.K, self.device
         n_pad = -(-n // api.GS_QUANT_GROUP) * api.GS_QUANT_GROUP
-        self.sh_codes = torch.zeros((k3, n_pad), device=dev,
-                                    dtype=torch.uint8 if self.sh_bits == 8 else torch.int16)
-        self.sh_bounds = torch.zeros((k3, n_pad // api.GS_QUANT_GROUP, 2), dtype=torch.float32,
-                                     device=dev)
+        if state is None:
+            self.sh_codes = torch.zeros((k3, n_pad), device=dev,
+                                        dtype=torch.uint8 if self.sh_bits == 8 else torch.int16)
+            self.sh_bounds = torch.zeros((k3, n_pad // api.GS_QUANT_GROUP, 2),
+                                         dtype=torch.float32, device=dev)
+            self.sh_m16 = torch.zeros((k3, n_pad), dtype=torch.int16, device=dev)
+            self.sh_v16 = torch.zeros((k3, n_pad), dtype=torch.int16, device=dev)
+        else:
+            self.sh_codes, self.sh_bounds, self.sh_m16, self.sh_v16 = state
         self.sh_q = api.sh_quant(self.sh_codes, self.sh_bounds, n, k3, self.sh_bits)
-        self.sh_m16 = torch.zeros((k3, n_pad), dtype=torch.int16, device=dev)
-        self.sh_v16 = torch.zeros((k3, n_pad), dtype=torch.int16, device=dev)
-        api.gs_sh_quantize(self.sh, self.sh_q, self.stream)
+        if state is None:
+            api.gs_sh_quantize(self.sh, self.sh_q, self.stream)
+        self.refresh_sh_float()
+
+    def refresh_sh_float(self) -> None:
+        """Quantised SH: decode the codes into ``self.sh``."""
         api.gs_sh_dequantize(self.sh_q, self.sh, self.stream)
 
     def _alloc_pairs(self, capacity: int) -> None:
@@ -189,8 +203,6 @@ class Splatter:
 
     # ------------------------------------------------------------ the calls
     def project(self):
-        if self.sh_bits is not None:
-            api.gs_sh_dequantize(self.sh_q, self.sh, self.stream)
         api.gs_project(self.c_params, self.cams, self.V, self.c_proj, self.ws, self.stream)
 
     def bin_sort(self):
@@ -464,9 +476,10 @@ class Splatter:
         per-Gaussian buffer is reallocated and the statistics restart from
         zero. z: standard normal draws float32 [n][2][3] for the split
         children (drawn on the device from `seed` when None). Returns the
-        per-Gaussian codes (0 pruned, 1 kept, 2 cloned, 3 split)."""
-        if self.sh_bits is not None:
-            raise NotImplementedError("densify_and_prune with quantised SH state")
+        per-Gaussian codes (0 pruned, 1 kept, 2 cloned, 3 split). With
+        quantised SH, gs_densify_sh_quant builds the new SH state from the
+        codes (decoded values gathered, groups encoded anew)."""
+        quant = self.sh_bits is not None
         self._gather_for_densify()
         n, dev = self.n, self.device
         if z is None:
@@ -480,29 +493,44 @@ class Splatter:
             return torch.empty((cap,) + tuple(t.shape[1:]), dtype=t.dtype, device=dev)
 
         out = {k: like(t) for k, t in self.param_list}
-        m_out = {k: like(t) for k, t in self.param_list}
-        v_out = {k: like(t) for k, t in self.param_list}
+        m_out = {k: like(t) for k, t in self.param_list if not (quant and k == "sh")}
+        v_out = {k: like(t) for k, t in self.param_list if not (quant and k == "sh")}
+        grads_of = lambda d: api.grads(*[d.get(k) for k in names])  # noqa: E731
         n_out = torch.zeros(1, dtype=torch.int64, device=dev)
         codes = torch.empty(max(n, 1), dtype=torch.int8, device=dev)
         ws = torch.zeros((api.gs_densify_workspace_size(n) + 255) // 256 * 256 // 8,
                          dtype=torch.int64, device=dev)
         dp = api.densify_params(grad_threshold, scale_split, min_opacity, max_scale, split_shrink)
-        api.gs_densify_and_prune(self.c_params,
-                                 api.grads(*[self.exp_avg[k] for k in names]),
-                                 api.grads(*[self.exp_avg_sq[k] for k in names]),
+        api.gs_densify_and_prune(self.c_params, grads_of(self.exp_avg), grads_of(self.exp_avg_sq),
                                  self.accum_abs if use_abs else self.accum_plain, self.denom,
-                                 z, dp, api.grads(*[out[k] for k in names]),
-                                 api.grads(*[m_out[k] for k in names]),
-                                 api.grads(*[v_out[k] for k in names]), cap, n_out, codes, ws,
-                                 self.stream)
+                                 z, dp, grads_of(out), grads_of(m_out), grads_of(v_out), cap,
+                                 n_out, codes, ws, self.stream)
         st = api.gs_get_status(ws, self.stream)
         if st != api.GS_OK:
             raise api.GsError(st, "gs_densify_and_prune")
         m = int(n_out.item())
-        keep = lambda d: {k: d[k][:m] for k in names}  # noqa: E731
+        keep = lambda d: {k: d[k][:m] for k in d}  # noqa: E731
         o, mo, vo = keep(out), keep(m_out), keep(v_out)
+        sh_state = None
+        if quant:
+            k3 = 3 * self.K
+            m_pad = -(-m // api.GS_QUANT_GROUP) * api.GS_QUANT_GROUP
+            state = (torch.zeros((k3, m_pad), device=dev, dtype=self.sh_codes.dtype),
+                     torch.zeros((k3, m_pad // api.GS_QUANT_GROUP, 2), dtype=torch.float32,
+                                 device=dev),
+                     torch.zeros((k3, m_pad), dtype=torch.int16, device=dev),
+                     torch.zeros((k3, m_pad), dtype=torch.int16, device=dev))
+            q_out = api.sh_quant(state[0], state[1], m, k3, self.sh_bits)
+            ws2 = torch.zeros((api.gs_densify_sh_quant_workspace_size(n, m) + 255) // 256 * 256
+                              // 8, dtype=torch.int64, device=dev)
+            api.gs_densify_sh_quant(self.sh_q, self.sh_m16, self.sh_v16, codes, q_out, state[2],
+                                    state[3], ws2, self.stream)
+            st = api.gs_get_status(ws2, self.stream)
+            if st != api.GS_OK:
+                raise api.GsError(st, "gs_densify_sh_quant")
+            sh_state = state  # o["sh"] is not written: the decode of the new codes fills it
         self._alloc_gaussians(o["means"], o["log_scales"], o["quats"], o["opacity_logit"],
-                              o["sh"], mo, vo)
+                              o["sh"], mo, vo, sh_state=sh_state)
         return codes[:n]
 
     def status(self) -> int:

@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define GS_ABI_VERSION 2
+#define GS_ABI_VERSION 3
 #define GS_TILE 16            /* tile edge in pixels */
 #define GS_MAX_VIEWS 32       /* views per call */
 #define GS_RECORD_FLOATS 16   /* floats per projected record */
@@ -100,7 +100,16 @@ typedef struct gs_camera {
  *                                inside; need not be unit)
  *   opacity_logit  float [n]     opacity = sigmoid(logit)
  *   sh             float [n][(sh_degree+1)^2][3]  real SH colour coefficients
+ *   sh_quant       the same coefficients as quantised codes (gs_sh_quant,
+ *                  below) instead: exactly one of sh and sh_quant is
+ *                  non-NULL. The calls that read the coefficients
+ *                  (gs_project, gs_project_bwd, gs_rasterize_bwd with
+ *                  gradients) then decode each code where they use it, to the
+ *                  float gs_sh_dequantize would give, so their results equal
+ *                  those of the float path on the decoded SH bit for bit;
+ *                  sh_quant->n must equal n and sh_quant->k3 3 (sh_degree+1)^2.
  * The float4 arrays must be 16-byte aligned. */
+struct gs_sh_quant;
 typedef struct gs_params {
   const float* means;
   const float* log_scales;
@@ -110,6 +119,7 @@ typedef struct gs_params {
   int32_t sh_degree;  /* 0..3 */
   int32_t reserved;
   int64_t n;          /* number of Gaussians, 0 <= n < 2^31 */
+  const struct gs_sh_quant* sh_quant;
 } gs_params;
 
 /* Gradients of the raw parameters: same layouts as gs_params (pad lanes are
@@ -416,7 +426,10 @@ size_t gs_densify_workspace_size(int64_t n);
  * exceeds out_capacity nothing is written and GS_ERR_CAPACITY is raised in
  * the status word. accum is the view-space gradient accumulator of
  * gs_densify_stats (plain or absolute), denom its visibility count. codes, if
- * not NULL, receives int8 [n]: 0 pruned, 1 kept, 2 cloned, 3 split. Outputs
+ * not NULL, receives int8 [n]: 0 pruned, 1 kept, 2 cloned, 3 split. With
+ * quantised SH (in->sh_quant set) the SH blocks are not touched here (the sh
+ * fields of out, m_out, v_out may be NULL) and codes must not be NULL:
+ * gs_densify_sh_quant then builds the output's SH state from them. Outputs
  * must not overlap the inputs. */
 gs_status gs_densify_and_prune(const gs_params* in, const gs_grads* m_in, const gs_grads* v_in,
                                const float* accum, const int32_t* denom, const float* z,
@@ -452,51 +465,87 @@ gs_status gs_l1_dssim(const float* image, const float* target, int32_t n_views, 
 /* ---- quantised SH state (Spirula VRAM page, sec. 魔法一) ----------------
  * SH coefficients kept as 8- or 16-bit codes, every 256 Gaussians of one
  * coefficient sharing a (min, max) pair; the Adam moments of those values are
- * bfloat16 in the same coefficient-major layout. With n_pad = n rounded up to
- * a multiple of GS_QUANT_GROUP and k3 = 3 (degree + 1)^2:
- *   codes   uint8 (bits 8) or uint16 (bits 16) [k3][n_pad]; value j of
- *           Gaussian i (j = 3 coefficient + channel) at j * n_pad + i;
+ * bfloat16. With n_pad = n rounded up to a multiple of GS_QUANT_GROUP and
+ * k3 = 3 (degree + 1)^2, value j of Gaussian i (j = 3 coefficient + channel)
+ * lives, by layout:
+ *   GS_QUANT_PLANAR  codes uint8 (bits 8) or uint16 (bits 16) [k3][n_pad],
+ *       the code at j * n_pad + i; the moments are two separate uint16
+ *       (bfloat16) arrays [k3][n_pad] passed beside the state;
+ *   GS_QUANT_PACKED  the page's packed optimiser block: codes is uint16
+ *       [k3][n_pad / 32][3][32]; the block (j, i / 32) holds the 32 codes of
+ *       Gaussians 32 (i / 32) .. + 31 (a 16-bit word each, also for 8-bit
+ *       codes), then their 32 first moments, then their 32 second moments
+ *       (bfloat16): 192 bytes, so the 32 lanes of a warp that update 32
+ *       consecutive values touch two cache lines.
  *   bounds  float [k3][n_pad / 256][2]: the (min, max) of group (j, i / 256);
- *   a code q decodes to min + q (max - min) / (2^bits - 1).
+ *   a code q decodes to min + q (max - min) / (2^bits - 1), in float32 as
+ *   fma(q, (max - min) / (2^bits - 1), min) with each operation rounded.
  * Encoding takes each group's min and max over its real Gaussians and rounds
  * t = (x - min) * ((2^bits - 1) / (max - min)) in float32 to nearest-even
  * (rounding 0) or to floor(t + u) (rounding 1, u in [0, 1) from SplitMix64
  * output number step * 2^37 + j * 2^31 + i + 1 of `seed`, top 24 bits);
  * a group with max == min gets code 0. Padding lanes are never written. */
 #define GS_QUANT_GROUP 256
+enum { GS_QUANT_PLANAR = 0, GS_QUANT_PACKED = 1 };
 
 typedef struct gs_sh_quant {
   void* codes;      /* see above; device memory, caller-owned, 4-byte (8-bit
-                       codes) or 8-byte (16-bit codes) aligned */
+                       planar codes) or 8-byte aligned */
   float* bounds;    /* see above; device memory, caller-owned */
   int64_t n;        /* Gaussians, 0 <= n < 2^31 */
   int32_t k3;       /* values per Gaussian: 3, 12, 27 or 48 */
   int32_t bits;     /* 8 or 16 */
+  int32_t layout;   /* GS_QUANT_PLANAR or GS_QUANT_PACKED */
+  int32_t reserved;
 } gs_sh_quant;
 
-/* Encode float SH [n][k3] (the gs_params layout) into q (nearest rounding). */
+/* Encode float SH [n][k3] (the gs_params layout) into q (nearest rounding).
+ * Only codes and bounds are written (packed blocks keep their moments). */
 gs_status gs_sh_quantize(const float* sh, const gs_sh_quant* q, void* stream);
 
 /* Decode q into float SH [n][k3] (float32: fma(q, (max - min) / (2^bits - 1), min)). */
 gs_status gs_sh_dequantize(const gs_sh_quant* q, float* sh, void* stream);
 
 /* One Adam step on the quantised SH, fused: decode each value, update its
- * bfloat16 moments exp_avg / exp_avg_sq ([k3][n_pad], round to nearest-even)
- * with the float32 gradient grad_sh ([n][k3], the gs_grads layout), take the
- * step of gs_adam_step (lr, beta1, beta2, eps, bias corrections of `step`),
- * then re-encode the group with its new min and max (rounding as above).
- * The moments must be 8-byte aligned. Argument errors as gs_adam_step, plus
- * rounding not 0/1, bits not 8/16, k3 not 3/12/27/48. */
+ * bfloat16 moments (round to nearest-even) with the float32 gradient grad_sh
+ * ([n][k3], the gs_grads layout), take the step of gs_adam_step (lr, beta1,
+ * beta2, eps, bias corrections of `step`), then re-encode the group with its
+ * new min and max (rounding as above). Planar: the moments are exp_avg /
+ * exp_avg_sq ([k3][n_pad], 8-byte aligned). Packed: they are in the blocks
+ * and exp_avg / exp_avg_sq must be NULL. Both layouts give the same codes,
+ * bounds and moments. Argument errors as gs_adam_step, plus rounding not
+ * 0/1, bits not 8/16, k3 not 3/12/27/48, an unknown layout. */
 gs_status gs_adam_step_sh_quant(const gs_sh_quant* q, const float* grad_sh, uint16_t* exp_avg,
                                 uint16_t* exp_avg_sq, float lr, float beta1, float beta2,
                                 float eps, int64_t step, int32_t rounding, uint64_t seed,
                                 void* stream);
 
+/* densify_and_prune for quantised SH (jsqmd.com sec. 1 and 3.3, with the
+ * Spirula page's quantised state). `decisions` are the int8 codes
+ * gs_densify_and_prune wrote for the same n Gaussians (0 pruned, 1 kept,
+ * 2 cloned, 3 split); out->n must be their output count (1 per kept, 2 per
+ * cloned or split Gaussian). Output Gaussian o takes the SH values of the
+ * input it comes from (decoded), in gs_densify_and_prune's order, and its
+ * groups are encoded anew with nearest rounding, so out equals gs_sh_quantize
+ * of the decoded input SH gathered in that order. Moments: a kept Gaussian
+ * and a clone's first copy keep theirs; a clone's copy and split children
+ * get zeros. in and out have the same k3, bits and layout; planar moments
+ * are m_in / v_in -> m_out / v_out ([k3][n_pad] each), packed ones travel
+ * in the blocks (the four pointers NULL). ws: device workspace of
+ * gs_densify_sh_quant_workspace_size(in->n, out->n) bytes, 256-byte aligned
+ * (the first 256 bytes hold the status word). The output must not overlap
+ * the input. Four launches on `stream`. */
+size_t gs_densify_sh_quant_workspace_size(int64_t n_in, int64_t n_out);
+gs_status gs_densify_sh_quant(const gs_sh_quant* in, const uint16_t* m_in, const uint16_t* v_in,
+                              const int8_t* decisions, const gs_sh_quant* out, uint16_t* m_out,
+                              uint16_t* v_out, void* ws, size_t ws_bytes, void* stream);
+
 /* Test hook for the timeout path (the pages have no counterpart). Every
  * device-side wait of the library (an mbarrier phase in gs_project and the
- * rasteriser, a look-back flag in gs_bin_sort's emission) gives up after a
- * time limit, sets GS_STATUS_BIT_TIMEOUT and lets its kernel finish. This
- * call makes one such wait run out on purpose, without faulting anything:
+ * rasteriser, a look-back flag in gs_bin_sort's emission and radix passes)
+ * gives up after a time limit, sets GS_STATUS_BIT_TIMEOUT and lets its kernel
+ * finish. This call makes one such wait run out on purpose, without faulting
+ * anything:
  *   GS_STALL_RASTER_FWD / GS_STALL_RASTER_BWD  global tile `index` of the
  *     next rasteriser calls issues no record copies and waits in vain for
  *     its first batch (its pixels keep the background / add no gradient);
@@ -504,12 +553,16 @@ gs_status gs_adam_step_sh_quant(const gs_sh_quant* q, const float* grad_sh, uint
  *     look-back scan (GS_SORT_FULL64, and GS_SORT_PRESORT on grids that
  *     sort by tile id) never publishes its prefix, so its successors' waits
  *     run out;
+ *   GS_STALL_SORT_LOOKBACK  partition `index` (of 4096 keys) of gs_bin_sort's
+ *     single-sweep radix passes (the depth keys of GS_SORT_PRESORT, the pair
+ *     keys of GS_SORT_FULL64) publishes neither its digit counts nor its
+ *     prefix in any pass, so the waits of the partitions after it run out;
  *   GS_STALL_NONE  back to normal.
  * wait_limit_s (> 0) replaces the default limit of 2 s for every wait while
  * the setting holds; 0 keeps the default. Process-wide, not thread-safe
  * against concurrent calls of the library; meant for tests only. */
 enum { GS_STALL_NONE = 0, GS_STALL_EMIT_LOOKBACK = 1, GS_STALL_RASTER_FWD = 2,
-       GS_STALL_RASTER_BWD = 3 };
+       GS_STALL_RASTER_BWD = 3, GS_STALL_SORT_LOOKBACK = 4 };
 gs_status gs_debug_stall(int32_t site, int64_t index, double wait_limit_s);
 
 /* Synchronise `stream`, return the status word accumulated in workspace `ws`

@@ -71,6 +71,18 @@ int main(void) {
   CHECK(gs_sh_quantize(NULL, &q, NULL) == GS_OK); /* no Gaussians: nothing to do */
   q.bits = 12;
   CHECK(gs_sh_quantize(NULL, &q, NULL) == GS_ERR_INVALID_ARG);
+  q.bits = 16;
+  q.layout = 2; /* neither planar nor packed */
+  CHECK(gs_sh_quantize(NULL, &q, NULL) == GS_ERR_INVALID_ARG);
+  q.layout = GS_QUANT_PACKED;
+  CHECK(gs_sh_quantize(NULL, &q, NULL) == GS_OK);
+  CHECK(gs_densify_sh_quant_workspace_size(1000, 1500) > 0);
+  CHECK(gs_densify_sh_quant_workspace_size(-1, 0) == 0);
+  /* quantised SH and float SH together are refused */
+  p.n = 10;
+  p.sh = (const float*)(uintptr_t)4096;
+  p.sh_quant = &q;
+  CHECK(gs_project(&p, &cam, 1, &out, ws, NULL) == GS_ERR_INVALID_ARG);
 
   CHECK(gs_adam_step(NULL, 1, 0.9f, 0.999f, 1e-15f, 1, NULL) == GS_ERR_INVALID_ARG);
   CHECK(gs_densify_workspace_size(1000) > 0 && gs_densify_workspace_size(-1) == 0);

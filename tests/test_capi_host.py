@@ -31,7 +31,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_status_strings():
-    assert api.gs_abi_version() == 2
+    assert api.gs_abi_version() == 3
     for s in range(7):
         assert api.status_string(s) not in ("", "unknown status")
 
@@ -97,6 +97,8 @@ def test_bad_arguments_are_rejected_before_any_cuda_call():
 def test_debug_stall_arguments():
     assert api.lib().gs_debug_stall(api.GS_STALL_RASTER_FWD, -1, 0.0) == api.GS_ERR_INVALID_ARG
     assert api.lib().gs_debug_stall(9, 0, 0.0) == api.GS_ERR_INVALID_ARG
+    assert api.lib().gs_debug_stall(api.GS_STALL_SORT_LOOKBACK + 1, 0, 0.0) == api.GS_ERR_INVALID_ARG
+    api.gs_debug_stall(api.GS_STALL_SORT_LOOKBACK, 1, 0.05)
     assert api.lib().gs_debug_stall(api.GS_STALL_NONE, 0, -1.0) == api.GS_ERR_INVALID_ARG
     assert api.lib().gs_debug_stall(api.GS_STALL_NONE, 0, 61.0) == api.GS_ERR_INVALID_ARG
     api.gs_debug_stall(api.GS_STALL_RASTER_BWD, 3, 0.05)

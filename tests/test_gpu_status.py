@@ -2,8 +2,8 @@
 
 Each bounded wait of the library gives up after a time limit, sets the timeout
 bit and lets its kernel finish; gs_debug_stall makes one such wait run out on
-purpose (a tile or an emission block waits for a copy or a flag that nothing
-provides), with a short limit. Malformed list entries and ranges are clipped by
+purpose (a tile, an emission block or a radix partition waits for a copy or
+a flag that nothing provides), with a short limit. Malformed list entries and ranges are clipped by
 the rasteriser's own bounds checks and reported. Nothing here faults: every
 access stays inside its buffer.
 """
@@ -101,6 +101,36 @@ def test_emission_lookback_wait_that_runs_out_is_reported():
     ids = sp.ids.clone()
     ranges = sp.ranges.clone()
     api.gs_debug_stall(api.GS_STALL_EMIT_LOOKBACK, 1, LIMIT_S)
+    sp.bin_sort()
+    torch.cuda.synchronize()
+    api.gs_debug_stall(api.GS_STALL_NONE)
+    st = sp.status()
+    assert st == api.GS_ERR_DEVICE_TIMEOUT, api.status_string(st)
+    sp.bin_sort()
+    torch.cuda.synchronize()
+    assert sp.status() == api.GS_OK
+    assert torch.equal(sp.ranges, ranges)
+    n = int(sp.n_pairs.item())
+    assert torch.equal(sp.ids[:n], ids[:n])
+
+
+@pytest.mark.parametrize("mode", [api.GS_SORT_PRESORT, api.GS_SORT_FULL64])
+def test_sort_lookback_wait_that_runs_out_is_reported(mode):
+    # the 64-bit radix passes (depth keys in presort mode, pair keys in
+    # full-64 mode) are single-sweep: partition 1 never publishes its counts,
+    # so partition 2 waits for it in every pass until the limit
+    sc = S.make_scene("fwd_100k_800", n=12000, width=200, height=152)
+    sp = Splatter(sc, sort_mode=mode)
+    sp.ensure_capacity()
+    sp.project()
+    sp.bin_sort()
+    torch.cuda.synchronize()
+    assert sp.status() == api.GS_OK
+    keys = 12000 if mode == api.GS_SORT_PRESORT else int(sp.n_pairs.item())
+    assert keys > 2 * 4096   # at least three partitions
+    ids = sp.ids.clone()
+    ranges = sp.ranges.clone()
+    api.gs_debug_stall(api.GS_STALL_SORT_LOOKBACK, 1, LIMIT_S)
     sp.bin_sort()
     torch.cuda.synchronize()
     api.gs_debug_stall(api.GS_STALL_NONE)
