@@ -92,9 +92,11 @@ def peaks():
         with open(path) as f:
             d = json.load(f)
         return dict(hbm_gbs=float(d["hbm_gbs"]), sm_max_mhz=float(d.get("sm_max_mhz", 1965.0)),
-                    source="measured")
+                    source="measured: MEASURED_PEAKS.json hbm_gbs (copy bandwidth)")
     except Exception:
-        return dict(hbm_gbs=6650.0, sm_max_mhz=1965.0, source="fallback")
+        # no measured file: an earlier copy-bandwidth measurement on this GPU model
+        return dict(hbm_gbs=6650.0, sm_max_mhz=1965.0,
+                    source="fallback: 6650 GB/s copy bandwidth (no MEASURED_PEAKS.json)")
 
 
 class ClockSampler:
@@ -176,7 +178,8 @@ def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float) -> dict:
                     pair, 8 B per pair for the ranges; the presort paths
                     (depth presort, pairs placed per tile) move far fewer
                     bytes and are counted by their own model: every id written
-                    once, the per-Gaussian depth keys sorted (passes x 24 B),
+                    once, the per-Gaussian depth keys counted (8 B) and sorted
+                    (passes x 24 B),
                     the packed rectangles and the (tile, Gaussian block) count
                     table read and written once;
       raster fwd    4 B id + 40 B record per pair + 20 B written per pixel;
@@ -198,10 +201,10 @@ def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float) -> dict:
         sort_bytes = V * n * 24 + n_pairs * (12 + pair * 24 + 8 + 8)
     elif plan["path"] == "tiles":
         table = plan["tiles"] * plan["bpv"] * 4
-        sort_bytes = (n_pairs * 4 + V * n * (16 + 12 + pre * 24 + 12 + 16 + 16)
+        sort_bytes = (n_pairs * 4 + V * n * (16 + 12 + 8 + pre * 24 + 12 + 16 + 16)
                       + 3 * table + plan["tiles"] * 24)
     else:
-        sort_bytes = n_pairs * (8 + pair * 16 + 4) + V * n * (16 + pre * 24 + 12)
+        sort_bytes = n_pairs * (8 + pair * 16 + 4) + V * n * (16 + 8 + pre * 24 + 12)
     return {
         "gs_project": dict(bytes=n * pbytes + V * n * 48, exps=0.0),
         "gs_bin_sort": dict(bytes=sort_bytes, exps=0.0),
@@ -217,14 +220,16 @@ def launches_per_step(sp, sort_mode: str, kind: str = "train") -> int:
     """Library kernels launched by one step (memsets excluded)."""
     plan = sort_plan(sp, sort_mode)
     pre, pair = plan["pre"], plan["pair"]
+    # the 64-bit sorts are single-sweep (a digit-count read + one kernel per
+    # pass); the 32-bit row / tile passes are count, scan, scatter
     if sort_mode == "full64":
-        sort = 1 + 3 * pair + 1                 # emit, passes, ranges
+        sort = 1 + 1 + pair + 1                 # emit, digit counts, passes, ranges
     elif plan["path"] == "tiles":
-        sort = 1 + 3 * pre + 4                  # keys, presort, count, scan, base, place
+        sort = 1 + 1 + pre + 4                  # keys, presort, count, scan, base, place
     elif plan["path"] == "columns":
-        sort = 1 + 3 * pre + 3 + 3 * pair + 1   # ..., count, scan, emit, row passes, ranges
+        sort = 1 + 1 + pre + 3 + 3 * pair + 1   # ..., count, scan, emit, row passes, ranges
     else:
-        sort = 1 + 3 * pre + 1 + 3 * pair + 1
+        sort = 1 + 1 + pre + 1 + 3 * pair + 1
     # project, sort, raster fwd (+ raster bwd, project bwd, densify (+ adam))
     return 1 + sort + 1 + {"fwd": 0, "fwdbwd": 3, "train": 4}[kind]
 
@@ -806,7 +811,7 @@ def run_ours(args):
         roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"],
                 "unit": "GB/s", "frac": ach / pk["hbm_gbs"],
                 "traffic": profiled_traffic(dk, args.workload),
-                "peak_source": pk["source"] + " (MEASURED_PEAKS.json copy bandwidth)"}
+                "peak_source": pk["source"]}
     # step roofline: sum over calls of max(bytes / HBM, exps / SFU)
     bound_ms = sum(k["bound_ms"] for k in kernels.values())
     n_launch = launches_per_step(sp, args.sort_mode, kind)

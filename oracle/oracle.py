@@ -558,6 +558,41 @@ def dequantize_groups(codes: np.ndarray, bounds: np.ndarray, n: int, bits: int) 
     return lo + c * (hi - lo) / qmax
 
 
+def fma_f32(a, b, c) -> np.ndarray:
+    """float32 fused multiply-add, correctly rounded (round to nearest-even),
+    elementwise on float32 arrays: a*b is exact in float64 (24 + 24
+    significant bits), p + c is taken with its exact error (Knuth's TwoSum),
+    and the float64 sum is rounded to float32, except where it sits exactly
+    halfway between two float32 values: there the error's sign decides."""
+    f64 = np.float64
+    a, b, c = (np.asarray(x, np.float32).astype(f64) for x in (a, b, c))
+    p = a * b
+    s = p + c
+    bv = s - p
+    e = (p - (s - bv)) + (c - bv)
+    r = s.astype(np.float32)
+    rd = r.astype(f64)
+    up = np.nextafter(r, np.float32(np.inf))
+    dn = np.nextafter(r, np.float32(-np.inf))
+    tie_up = (s - rd) * 2 == up.astype(f64) - rd
+    tie_dn = (rd - s) * 2 == rd - dn.astype(f64)
+    r = np.where(tie_up & (e > 0), up, r)
+    r = np.where(tie_dn & (e < 0), dn, r)
+    return np.asarray(r, np.float32)
+
+
+def dequantize_groups_f32(codes: np.ndarray, bounds: np.ndarray, n: int, bits: int) -> np.ndarray:
+    """The float32 decoding of the codes, as the state's definition fixes
+    it: step = (max - min) / (2^b - 1) with each operation rounded to
+    float32, then x = fma(q, step, min) rounded once -> float32 [3K][n]."""
+    f = np.float32
+    g = np.arange(n) // Q_GROUP
+    lo = np.asarray(bounds, f)[:, g, 0]
+    hi = np.asarray(bounds, f)[:, g, 1]
+    step = ((hi - lo).astype(f) / f((1 << bits) - 1)).astype(f)
+    return fma_f32(np.asarray(codes)[:, :n].astype(f), step, lo)
+
+
 def sh_quantize(sh: np.ndarray, bits: int):
     """Quantised SH state of float32 SH [N][K][3]: (codes [3K][n_pad], bounds
     [3K][n_pad / 256][2]) with round-to-nearest."""

@@ -310,16 +310,18 @@ def test_densify_of_quantised_sh_equals_encoding_the_gathered_values(bits, layou
         ocodes, obounds, _ = _state(n_out, k3, bits)
     q_in = api.sh_quant(codes, bounds, n, k3, bits, layout)
     q_out = api.sh_quant(ocodes, obounds, n_out, k3, bits, layout)
-    api.gs_sh_quantize(torch.from_numpy(sh).cuda(), q_in)
+    # the input state comes from the oracle's encoder
+    c0, b0 = O.sh_quantize(sh, bits)
+    c0_t = torch.from_numpy(c0.view(np.int16) if bits == 16 else c0).cuda()
+    bounds.copy_(torch.from_numpy(b0))
     m_in = torch.from_numpy(m_np.copy()).cuda()
     v_in = torch.from_numpy(v_np.copy()).cuda()
     m_out = torch.zeros((k3, m_pad), dtype=torch.int16, device="cuda")
     v_out = torch.zeros_like(m_out)
     if packed:
-        codes[:, :, 1, :] = m_in.view(k3, n_pad // 32, 32)
-        codes[:, :, 2, :] = v_in.view(k3, n_pad // 32, 32)
-    decoded = torch.empty((n, K, 3), device="cuda")
-    api.gs_sh_dequantize(q_in, decoded)
+        codes.copy_(_pack(c0_t, m_in, v_in, bits))
+    else:
+        codes.copy_(c0_t)
     ws = torch.zeros((api.gs_densify_sh_quant_workspace_size(n, n_out) + 255) // 256 * 32,
                      dtype=torch.int64, device="cuda")
     decisions = torch.from_numpy(dec).cuda()
@@ -328,7 +330,7 @@ def test_densify_of_quantised_sh_equals_encoding_the_gathered_values(bits, layou
     else:
         api.gs_densify_sh_quant(q_in, m_in, v_in, decisions, q_out, m_out, v_out, ws)
     assert api.gs_get_status(ws, None) == api.GS_OK
-    # expected, from the decoded input
+    # expected, from the oracle's float32 decoding of the input codes
     src, zero = [], []
     for i, c in enumerate(dec):
         if c == 1:
@@ -338,8 +340,8 @@ def test_densify_of_quantised_sh_equals_encoding_the_gathered_values(bits, layou
         elif c == 3:
             src += [i, i]; zero += [True, True]
     src, zero = np.array(src), np.array(zero)
-    gathered = decoded.cpu().numpy()[src]
-    want_c, want_b = O.sh_quantize(gathered, bits)
+    decoded = O.dequantize_groups_f32(c0, b0, n, bits).T.reshape(n, K, 3)
+    want_c, want_b = O.sh_quantize(decoded[src], bits)
     want_m = np.where(zero[None, :], 0, m_np[:, src])
     want_v = np.where(zero[None, :], 0, v_np[:, src])
     if packed:

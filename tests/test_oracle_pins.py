@@ -845,6 +845,64 @@ def test_bf16_rounding_closed_forms():
     assert np.all(np.abs(back - x) <= np.abs(x) * 2.0 ** -8)
 
 
+def _round_f32_exact(x) -> np.float32:
+    """float32 nearest to the rational x (ties to even), by brute force over
+    the candidates around float(x)."""
+    from fractions import Fraction
+    r0 = np.float32(float(x))
+    cands = [r0, np.nextafter(r0, np.float32(np.inf)), np.nextafter(r0, np.float32(-np.inf))]
+    best = min(abs(Fraction(float(c)) - x) for c in cands)
+    ties = [c for c in cands if abs(Fraction(float(c)) - x) == best]
+    if len(ties) > 1:
+        ties = [c for c in ties if int(np.float32(c).view(np.uint32)) % 2 == 0]
+    return np.float32(ties[0])
+
+
+def test_fma_f32_is_the_correctly_rounded_fused_multiply_add():
+    """Against exact rational arithmetic: random triples (with cancellation),
+    and sums that sit on a float32 halfway point in float64 while the exact
+    value does not (97 * 257 * 673 = 2^24 + 1, so 24929 * (673 * 2^-24) is
+    the midpoint 1 + 2^-24 exactly)."""
+    from fractions import Fraction
+    rng = np.random.default_rng(11)
+    a = rng.normal(0, 1, 400).astype(np.float32)
+    b = rng.normal(0, 1, 400).astype(np.float32) * np.float32(2.0) ** rng.integers(-30, 30, 400)
+    c = (-(a.astype(np.float64) * b) * (1 + rng.normal(0, 1e-6, 400))).astype(np.float32)
+    c[::3] = rng.normal(0, 1, 134).astype(np.float32)
+    mid_a, mid_b = np.float32(24929.0), np.float32(673.0 * 2.0 ** -24)
+    tiny = np.float32(2.0 ** -80)
+    a = np.concatenate([a, [mid_a] * 3])
+    b = np.concatenate([b, [mid_b] * 3])
+    c = np.concatenate([c, [tiny, np.float32(0), -tiny]])
+    got = O.fma_f32(a, b, c)
+    for k in range(len(a)):
+        exact = Fraction(float(a[k])) * Fraction(float(b[k])) + Fraction(float(c[k]))
+        assert got[k] == _round_f32_exact(exact), k
+    assert got[-3] == np.float32(1 + 2.0 ** -23)      # just above the midpoint: up
+    assert got[-2] == np.float32(1.0) and got[-1] == np.float32(1.0)  # tie to even; below
+
+
+def test_float32_decoding_of_the_codes():
+    """Code 0 decodes to the group's min exactly, a constant group to its
+    value, and every value within float32 rounding of the float64 decoding."""
+    rng = np.random.default_rng(12)
+    n, K = 600, 4
+    sh = rng.normal(0, 1, (n, K, 3)).astype(np.float32)
+    sh[256:512, 1, 2] = -0.75
+    for bits in (8, 16):
+        codes, bounds = O.sh_quantize(sh, bits)
+        x32 = O.dequantize_groups_f32(codes, bounds, n, bits)
+        x64 = O.dequantize_groups(codes, bounds, n, bits)
+        assert x32.dtype == np.float32 and x32.shape == (12, n)
+        g = np.arange(n) // 256
+        lo, hi = bounds[:, g, 0], bounds[:, g, 1]
+        zero = codes[:, :n] == 0
+        assert np.array_equal(x32[zero], lo[zero])
+        assert np.all(x32[5, 256:512] == np.float32(-0.75))
+        mag = np.maximum(np.abs(lo), np.abs(hi)).astype(np.float64)
+        assert np.all(np.abs(x32 - x64) <= 2.0 ** -22 * mag + 1e-30)
+
+
 def test_quantize_groups_structure_and_error_bound():
     """Groups are one coefficient of 256 consecutive Gaussians; the group's
     min and max are exact codes 0 and 2^b - 1; nearest rounding is off by at
