@@ -199,5 +199,9 @@ def test_bench_work_model_uses_the_library_plan():
     sp = types.SimpleNamespace(n=1_000_000, V=1, W=1920, H=1080, cams=cams)
     plan = bench.sort_plan(sp, "presort")
     assert plan == dict(path="tiles", pre=4, pair=0, bpv=1303, tiles=8160)
-    assert bench.launches_per_step(sp, "presort") == 23
+    # project; depth keys, digit counts, 4 single-sweep passes, count, scan, base,
+    # place; raster fwd, raster bwd, project bwd, densify stats, Adam
+    assert bench.launches_per_step(sp, "presort") == 1 + (1 + 1 + 4 + 4) + 5
     assert bench.sort_plan(sp, "full64")["pair"] == 6
+    # emit, digit counts, 6 passes, ranges
+    assert bench.launches_per_step(sp, "full64") == 1 + (1 + 1 + 6 + 1) + 5
