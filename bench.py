@@ -4,8 +4,10 @@
 One step of the default workload (train_1m_1080p: 1,000,000 SH3 Gaussians,
 1920x1080, fx = fy = 1200, upstream image gradient N(0, 1e-2), synthetic and
 seeded) is gs_project -> gs_bin_sort -> gs_rasterize_fwd -> gs_rasterize_bwd
-(screen space) -> gs_project_bwd -> gs_densify_stats -> gs_adam_step. The
-metric is the step time and its pixel throughput (Mpix/s = rendered pixels /
+(screen space) -> gs_project_bwd_adam (projection backward, densification
+statistics and the Adam step in one launch; with N > 1 GPUs the gradients are
+exchanged, so the tail is gs_project_bwd -> gs_densify_stats -> the sharded
+Adam step). The metric is the step time and its pixel throughput (Mpix/s = rendered pixels /
 step time). ``--workload`` selects one of the five workload shapes:
 
   fwd_1k_128        forward only (project, bin_sort, rasterize_fwd)
@@ -15,7 +17,7 @@ step time). ``--workload`` selects one of the five workload shapes:
                     over the views; the sort's keys are 64-bit ((view << 32 |
                     depth) in the presort; the extras time the pages' own
                     (tile << 32 | depth) pair-key sort too)
-  train_10m_4k      the full step with the fused Adam update
+  train_10m_4k      the full step
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl ours|reference]
@@ -188,7 +190,11 @@ def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float) -> dict:
       project bwd   parameters read and gradients written once, 36 B of
                     screen-space gradients per Gaussian and view;
       densify       16 B per Gaussian and view + 24 B per Gaussian;
-      adam          28 B per parameter (p, g, m, v read; p, m, v written).
+      adam          28 B per parameter (p, g, m, v read; p, m, v written);
+      fused tail    (projection backward + statistics + Adam in one launch)
+                    the parameters and both moments read and written once,
+                    36 B of screen-space gradients per Gaussian and view,
+                    24 B of statistics per Gaussian.
 
     Exps: the (pixel, Gaussian) evaluations with alpha >= 1/255 reached
     before the pixel stops (counted by the oracle on a pixel sample)."""
@@ -213,11 +219,16 @@ def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float) -> dict:
         "gs_project_bwd": dict(bytes=n * 2 * pbytes + V * n * 36, exps=0.0),
         "gs_densify_stats": dict(bytes=V * n * 16 + n * 24, exps=0.0),
         "gs_adam_step": dict(bytes=n * (pbytes // 4) * 28, exps=0.0),
+        # fused tail: parameters read and written, both moments read and
+        # written, the screen-space gradients, the statistics read and written
+        "gs_project_bwd_adam": dict(bytes=n * 6 * pbytes + V * n * 36 + n * 24, exps=0.0),
     }
 
 
-def launches_per_step(sp, sort_mode: str, kind: str = "train") -> int:
-    """Library kernels launched by one step (memsets excluded)."""
+def launches_per_step(sp, sort_mode: str, kind: str = "train", fused: bool = False) -> int:
+    """Library kernels launched by one step (memsets excluded); fused: the
+    training step ends with the one-launch projection backward + statistics
+    + Adam."""
     plan = sort_plan(sp, sort_mode)
     pre, pair = plan["pre"], plan["pair"]
     # the 64-bit sorts are single-sweep (a digit-count read + one kernel per
@@ -230,8 +241,10 @@ def launches_per_step(sp, sort_mode: str, kind: str = "train") -> int:
         sort = 1 + 1 + pre + 3 + 3 * pair + 1   # ..., count, scan, emit, row passes, ranges
     else:
         sort = 1 + 1 + pre + 1 + 3 * pair + 1
-    # project, sort, raster fwd (+ raster bwd, project bwd, densify (+ adam))
-    return 1 + sort + 1 + {"fwd": 0, "fwdbwd": 3, "train": 4}[kind]
+    # project, sort, raster fwd (+ raster bwd, project bwd, densify (+ adam)),
+    # or raster bwd + the fused tail
+    tail = 2 if (kind == "train" and fused) else {"fwd": 0, "fwdbwd": 3, "train": 4}[kind]
+    return 1 + sort + 1 + tail
 
 
 # C call -> (kernel, source file) for the ncu traffic lookup
@@ -612,10 +625,15 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
     pixels = V * c.width * c.height
 
+    # a one-GPU training step ends with the fused tail (projection backward,
+    # densification statistics and Adam in one launch); with N > 1 the
+    # gradients are exchanged, so the tail stays three calls
+    fused = kind == "train" and sp.fused_tail_ok()
     names = ["gs_project", "gs_bin_sort", "gs_rasterize_fwd"]
     if kind != "fwd":
-        names += ["gs_rasterize_bwd", "gs_project_bwd", "gs_densify_stats"]
-    if kind == "train":
+        names += ["gs_rasterize_bwd"]
+        names += ["gs_project_bwd_adam"] if fused else ["gs_project_bwd", "gs_densify_stats"]
+    if kind == "train" and not fused:
         names += ["gs_adam_step" if world == 1 else "reduce_scatter+gs_adam_step+all_gather"]
 
     # one CUDA graph per call (not Adam, whose bias corrections follow the
@@ -644,6 +662,10 @@ def run_ours(args):
             return
         call("rasterize_bwd", lambda: sp.rasterize_bwd(dL, with_params=False))
         mark(4)
+        if fused:
+            sp.project_bwd_adam()  # not in a graph: the bias corrections follow the step
+            mark(5)
+            return
         call("project_bwd", sp.project_bwd)
         mark(5)
         call("densify_stats", sp.densify_stats)
@@ -814,7 +836,7 @@ def run_ours(args):
                 "peak_source": pk["source"]}
     # step roofline: sum over calls of max(bytes / HBM, exps / SFU)
     bound_ms = sum(k["bound_ms"] for k in kernels.values())
-    n_launch = launches_per_step(sp, args.sort_mode, kind)
+    n_launch = launches_per_step(sp, args.sort_mode, kind, fused)
     line = {
         "metric": METRIC, "value": value, "unit": "Mpix/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,

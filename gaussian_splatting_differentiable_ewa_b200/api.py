@@ -105,6 +105,10 @@ SIGNATURES = [
     ("gs_project_bwd", _c.c_int,
      [_c.POINTER(GsParams), _c.POINTER(GsCamera), _c.c_int32, _vp, _vp, _c.POINTER(GsGrads),
       _vp]),
+    ("gs_project_bwd_adam", _c.c_int,
+     [_c.POINTER(GsParams), _c.POINTER(GsCamera), _c.c_int32, _vp, _vp, _c.POINTER(GsGrads),
+      _c.POINTER(GsGrads), _c.POINTER(_c.c_float), _c.c_float, _c.c_float, _c.c_float,
+      _c.c_int64, _vp, _vp, _vp, _vp]),
     ("gs_densify_stats", _c.c_int,
      [_vp, _vp, _c.c_int32, _c.c_int64, _vp, _vp, _vp, _vp]),
     ("gs_adam_step", _c.c_int,
@@ -281,6 +285,20 @@ def gs_project_bwd(p: GsParams, cams_arr, n_views: int, radii, grad2d, g: GsGrad
                    stream=None) -> None:
     _check(lib().gs_project_bwd(_c.byref(p), cams_arr, int(n_views), _ptr(radii), _ptr(grad2d),
                                 _c.byref(g), _stream(stream)), "gs_project_bwd")
+
+
+def gs_project_bwd_adam(p: GsParams, cams_arr, n_views: int, radii, grad2d, exp_avg: GsGrads,
+                        exp_avg_sq: GsGrads, lr, beta1: float, beta2: float, eps: float,
+                        step: int, accum_plain=None, accum_abs=None, denom=None,
+                        stream=None) -> None:
+    """lr: the five group learning rates (means, log_scales, quats,
+    opacity_logit, sh); the parameters of p are updated in place."""
+    lr5 = (_c.c_float * 5)(*[float(x) for x in lr])
+    _check(lib().gs_project_bwd_adam(_c.byref(p), cams_arr, int(n_views), _ptr(radii),
+                                     _ptr(grad2d), _c.byref(exp_avg), _c.byref(exp_avg_sq), lr5,
+                                     float(beta1), float(beta2), float(eps), int(step),
+                                     _ptr(accum_plain), _ptr(accum_abs), _ptr(denom),
+                                     _stream(stream)), "gs_project_bwd_adam")
 
 
 def gs_densify_stats(grad2d, radii, n_views: int, n: int, accum_plain, accum_abs, denom,

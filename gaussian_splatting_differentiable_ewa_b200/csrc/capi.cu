@@ -365,6 +365,60 @@ gs_status gs_project_bwd(const gs_params* params, const gs_camera* cams, int32_t
                                         static_cast<cudaStream_t>(stream)));
 }
 
+gs_status gs_project_bwd_adam(const gs_params* params, const gs_camera* cams, int32_t n_views,
+                              const int32_t* radii, const float* grad2d, gs_grads* exp_avg,
+                              gs_grads* exp_avg_sq, const float* lr, float beta1, float beta2,
+                              float eps, int64_t step, float* accum_plain, float* accum_abs,
+                              int32_t* denom, void* stream) {
+  if (!params || !check_cams(cams, n_views) || !exp_avg || !exp_avg_sq || !lr)
+    return GS_ERR_INVALID_ARG;
+  const gs_params& p = *params;
+  if (p.n < 0 || p.sh_degree < 0 || p.sh_degree > 3 || p.sh_quant) return GS_ERR_INVALID_ARG;
+  if (p.n >= (1ll << 31)) return GS_ERR_OVERFLOW;
+  if (step < 1 || !(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f) ||
+      !(eps >= 0.f))
+    return GS_ERR_INVALID_ARG;
+  const bool stats = accum_plain || accum_abs || denom;
+  if (stats && !(accum_plain && accum_abs && denom)) return GS_ERR_INVALID_ARG;
+  // the moments take the gradients' place: same layouts and alignment checks
+  if (check_grads_args(p, exp_avg, true) != GS_OK || check_grads_args(p, exp_avg_sq, true) != GS_OK)
+    return GS_ERR_INVALID_ARG;
+  if (p.n == 0) return GS_OK;
+  if (!radii || !grad2d || !aligned(grad2d, 16)) return GS_ERR_INVALID_ARG;
+  // the SH blocks move as float4
+  if (!aligned(p.sh, 16) || !aligned(exp_avg->sh, 16) || !aligned(exp_avg_sq->sh, 16))
+    return GS_ERR_INVALID_ARG;
+  AdamTail t{};
+  t.p_means = reinterpret_cast<float4*>(const_cast<float*>(p.means));
+  t.p_log_scales = reinterpret_cast<float4*>(const_cast<float*>(p.log_scales));
+  t.p_quats = reinterpret_cast<float4*>(const_cast<float*>(p.quats));
+  t.p_logit = const_cast<float*>(p.opacity_logit);
+  t.p_sh = const_cast<float*>(p.sh);
+  t.m_means = reinterpret_cast<float4*>(exp_avg->means);
+  t.m_log_scales = reinterpret_cast<float4*>(exp_avg->log_scales);
+  t.m_quats = reinterpret_cast<float4*>(exp_avg->quats);
+  t.m_logit = exp_avg->opacity_logit;
+  t.m_sh = exp_avg->sh;
+  t.v_means = reinterpret_cast<float4*>(exp_avg_sq->means);
+  t.v_log_scales = reinterpret_cast<float4*>(exp_avg_sq->log_scales);
+  t.v_quats = reinterpret_cast<float4*>(exp_avg_sq->quats);
+  t.v_logit = exp_avg_sq->opacity_logit;
+  t.v_sh = exp_avg_sq->sh;
+  for (int k = 0; k < 5; ++k) t.lr[k] = lr[k];
+  t.b1 = beta1;
+  t.b2 = beta2;
+  t.eps = eps;
+  // the bias corrections exactly as gs_adam_step takes them
+  t.ibc1 = (float)(1.0 / (1.0 - pow((double)beta1, (double)step)));
+  t.ibc2 = (float)(1.0 / (1.0 - pow((double)beta2, (double)step)));
+  t.accum_plain = accum_plain;
+  t.accum_abs = accum_abs;
+  t.denom = denom;
+  const CamSet cs = pack_cams(cams, n_views);
+  return cuda_status(launch_project_bwd_adam(p, cs, n_views, grad2d, radii, t,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
 gs_status gs_rasterize_bwd(const gs_params* params, const gs_projected* proj,
                            const gs_binned* bins, const gs_camera* cams, int32_t n_views,
                            const float* bg, const float* dL_dimage, const float* final_T,

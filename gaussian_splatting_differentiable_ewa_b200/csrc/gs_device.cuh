@@ -190,4 +190,24 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
+// One Adam update (lshu.cn sec. 3.3; Kingma and Ba with bias correction,
+// eps outside the square root); ibc1 = 1 / (1 - b1^t), ibc2 = 1 / (1 - b2^t).
+// The square root and the division use the SFU (a few ulp on the step, far
+// inside the update's own scale), which keeps the callers on HBM rather than
+// on the multi-instruction IEEE sequences. Shared by the Adam kernel and the
+// fused projection backward, so the two give identical parameters.
+__device__ __forceinline__ void adam_one(float& p, float g, float& m, float& v, float lr, float b1,
+                                         float b2, float eps, float ibc1, float ibc2) {
+  m = fmaf(b1, m, (1.f - b1) * g);
+  v = fmaf(b2, v, (1.f - b2) * g * g);
+  const float denom = sqrtf(v * ibc2) + eps;
+  p -= __fdividef(lr * (m * ibc1), denom);
+}
+
+// ||(gx, gy)|| of a view's screen-space mean gradient (the plain
+// densification statistic), one fixed operation sequence for every caller.
+__device__ __forceinline__ float densify_norm(float gx, float gy) {
+  return sqrtf(fmaf(gx, gx, gy * gy));
+}
+
 }  // namespace gsb

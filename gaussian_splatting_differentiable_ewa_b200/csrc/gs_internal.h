@@ -86,12 +86,33 @@ inline ShQuant shq_of(const gs_sh_quant* q) {
   return r;
 }
 
+// The training step's tail fused into the projection backward: parameters
+// (updated in place), both Adam moments, per-group learning rates (means,
+// log-scales, quaternions, opacity logits, SH), the bias corrections, and the
+// densification statistics (null accumulators: none).
+struct AdamTail {
+  float4 *p_means, *p_log_scales, *p_quats;
+  float *p_logit, *p_sh;
+  float4 *m_means, *m_log_scales, *m_quats;
+  float *m_logit, *m_sh;
+  float4 *v_means, *v_log_scales, *v_quats;
+  float *v_logit, *v_sh;
+  float lr[5];
+  float b1, b2, eps, ibc1, ibc2;
+  float* accum_plain;
+  float* accum_abs;
+  int* denom;
+};
+
 cudaError_t launch_project(const gs_params& p, const CamSet& cams, int n_views, float* records,
                            float* bins, int* radii, uint32_t* status, const WaitCfg& wc,
                            cudaStream_t stream);
 cudaError_t launch_project_bwd(const gs_params& p, const CamSet& cams, int n_views,
                                const float* grad2d, const int* radii, const gs_grads& g,
                                cudaStream_t stream);
+cudaError_t launch_project_bwd_adam(const gs_params& p, const CamSet& cams, int n_views,
+                                    const float* grad2d, const int* radii, const AdamTail& t,
+                                    cudaStream_t stream);
 cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream);
 cudaError_t launch_raster_fwd(const float* records, const uint32_t* ids, const int64_t* ranges,
                               int64_t capacity, const Grid& g, int n_views, int n,

@@ -31,7 +31,7 @@ __global__ void __launch_bounds__(256) k_densify(const float4* __restrict__ grad
     if (radii[r] <= 0) continue;
     const float4 a = grad2d[r * 3 + 0];
     const float4 c = grad2d[r * 3 + 2];
-    pl += sqrtf(a.x * a.x + a.y * a.y);
+    pl += densify_norm(a.x, a.y);
     ab += c.y;
     ++cnt;
   }
@@ -56,18 +56,6 @@ struct AdamTable {
 constexpr int kAdamThreads = 256;
 constexpr int kAdamVecPerThread = 4;
 constexpr int64_t kAdamFloatsPerBlock = (int64_t)kAdamThreads * kAdamVecPerThread * 4;
-
-// One Adam update; ibc1 = 1 / (1 - b1^t), ibc2 = 1 / (1 - b2^t). The square
-// root and the division use the SFU (a few ulp on the step, far inside the
-// update's own scale), which keeps the kernel on HBM rather than on the
-// multi-instruction IEEE sequences.
-__device__ __forceinline__ void adam_one(float& p, float g, float& m, float& v, float lr, float b1,
-                                         float b2, float eps, float ibc1, float ibc2) {
-  m = fmaf(b1, m, (1.f - b1) * g);
-  v = fmaf(b2, v, (1.f - b2) * g * g);
-  const float denom = sqrtf(v * ibc2) + eps;
-  p -= __fdividef(lr * (m * ibc1), denom);
-}
 
 __global__ void __launch_bounds__(kAdamThreads) k_adam(AdamTable t, float b1, float b2, float eps,
                                                        float ibc1, float ibc2) {

@@ -514,14 +514,19 @@ __global__ void __launch_bounds__(kProjFwdThreads, 3) k_project(const float4* __
 // (coefficient-major, coalesced global traffic); the SH gradients are summed
 // over views in shared memory rather than in registers. With ALIAS (one view)
 // the gradients overwrite the staged coefficients slot by slot.
-template <int DEG, bool ALIAS, bool QUANT>
+// With FUSE the gradients are not written: the Adam step (adam_one, the
+// update of the Adam kernel) is applied to the parameters in place and the
+// densification statistics are accumulated from the same screen-space
+// gradients (densify_norm, as the statistics kernel), so the fused tail gives
+// what the three separate calls give, bit for bit.
+template <int DEG, bool ALIAS, bool QUANT, bool FUSE>
 __global__ void __launch_bounds__(kProjThreads, 6) k_project_bwd(
     const float4* __restrict__ means, const float4* __restrict__ log_scales,
     const float4* __restrict__ quats, const float* __restrict__ logit,
     const float* __restrict__ sh, const float4* __restrict__ grad2d,
     const int* __restrict__ radii, int n, int n_views, CamSet cams, float4* __restrict__ g_means,
     float4* __restrict__ g_log_scales, float4* __restrict__ g_quats, float* __restrict__ g_logit,
-    float* __restrict__ g_sh, ShQuant shq) {
+    float* __restrict__ g_sh, ShQuant shq, AdamTail tail) {
   constexpr int K = (DEG + 1) * (DEG + 1);
   constexpr int K3 = K * 3;
   extern __shared__ float s_pb[];
@@ -556,10 +561,11 @@ __global__ void __launch_bounds__(kProjThreads, 6) k_project_bwd(
   const int i = (int)i0 + threadIdx.x;
   const bool live = i < n;
   const int il = live ? i : (int)i0;  // a dead thread computes on a valid index, writes nothing
-  const float4 m = __ldg(&means[il]);
-  const float4 ls = __ldg(&log_scales[il]);
-  const float4 q = __ldg(&quats[il]);
-  const float lg = __ldg(&logit[il]);
+  // fused: the parameters are read where this thread later writes them
+  const float4 m = FUSE ? tail.p_means[il] : __ldg(&means[il]);
+  const float4 ls = FUSE ? tail.p_log_scales[il] : __ldg(&log_scales[il]);
+  const float4 q = FUSE ? tail.p_quats[il] : __ldg(&quats[il]);
+  const float lg = FUSE ? tail.p_logit[il] : __ldg(&logit[il]);
 
   const float qn2 = q.x * q.x + q.y * q.y + q.z * q.z + q.w * q.w;
   const float qinv = rsqrtf(qn2);
@@ -581,6 +587,8 @@ __global__ void __launch_bounds__(kProjThreads, 6) k_project_bwd(
   float* dsh_t = s_dsh + threadIdx.x;
   cp_async_wait_all();
   __syncthreads();
+  float st_plain = 0.f, st_abs = 0.f;  // fused densification statistics
+  int st_cnt = 0;
   if (live) {
   bool touched = false;
   for (int v = 0; v < n_views; ++v) {
@@ -589,6 +597,11 @@ __global__ void __launch_bounds__(kProjThreads, 6) k_project_bwd(
     const float4* G4 = grad2d + ((size_t)v * n + i) * 3;
     const float4 ga = G4[0], gb = G4[1], gc = G4[2];
     const float G[9] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w, gc.x};
+    if (FUSE) {
+      st_plain += densify_norm(ga.x, ga.y);
+      st_abs += gc.y;
+      ++st_cnt;
+    }
     const gs_camera& c = cams.c[v];
     const float W[3][3] = {{c.viewmat[0], c.viewmat[1], c.viewmat[2]},
                            {c.viewmat[4], c.viewmat[5], c.viewmat[6]},
@@ -723,13 +736,83 @@ __global__ void __launch_bounds__(kProjThreads, 6) k_project_bwd(
   dqy = (dqy - qy * proj) * qinv;
   dqz = (dqz - qz * proj) * qinv;
 
-  g_means[i] = make_float4(dmu[0], dmu[1], dmu[2], 0.f);
-  g_log_scales[i] = make_float4(dls[0], dls[1], dls[2], 0.f);
-  g_quats[i] = make_float4(dqw, dqx, dqy, dqz);
-  g_logit[i] = dopac * opac * (1.f - opac);
+  if constexpr (FUSE) {
+    const float b1 = tail.b1, b2 = tail.b2, eps = tail.eps, c1 = tail.ibc1, c2 = tail.ibc2;
+    auto step4 = [&](float4 p, float4 g, float4* P, float4* Mv, float4* Vv, float lr) {
+      float4 mm = __ldcs(Mv + i), vv = __ldcs(Vv + i);
+      adam_one(p.x, g.x, mm.x, vv.x, lr, b1, b2, eps, c1, c2);
+      adam_one(p.y, g.y, mm.y, vv.y, lr, b1, b2, eps, c1, c2);
+      adam_one(p.z, g.z, mm.z, vv.z, lr, b1, b2, eps, c1, c2);
+      adam_one(p.w, g.w, mm.w, vv.w, lr, b1, b2, eps, c1, c2);
+      __stcs(P + i, p);
+      __stcs(Mv + i, mm);
+      __stcs(Vv + i, vv);
+    };
+    step4(m, make_float4(dmu[0], dmu[1], dmu[2], 0.f), tail.p_means, tail.m_means, tail.v_means,
+          tail.lr[0]);
+    step4(ls, make_float4(dls[0], dls[1], dls[2], 0.f), tail.p_log_scales, tail.m_log_scales,
+          tail.v_log_scales, tail.lr[1]);
+    step4(q, make_float4(dqw, dqx, dqy, dqz), tail.p_quats, tail.m_quats, tail.v_quats,
+          tail.lr[2]);
+    float pl = lg, ml = tail.m_logit[i], vl = tail.v_logit[i];
+    adam_one(pl, dopac * opac * (1.f - opac), ml, vl, tail.lr[3], b1, b2, eps, c1, c2);
+    tail.p_logit[i] = pl;
+    tail.m_logit[i] = ml;
+    tail.v_logit[i] = vl;
+    if (tail.accum_plain && st_cnt) {
+      tail.accum_plain[i] += st_plain;
+      tail.accum_abs[i] += st_abs;
+      tail.denom[i] += st_cnt;
+    }
+  } else {
+    g_means[i] = make_float4(dmu[0], dmu[1], dmu[2], 0.f);
+    g_log_scales[i] = make_float4(dls[0], dls[1], dls[2], 0.f);
+    g_quats[i] = make_float4(dqw, dqx, dqy, dqz);
+    g_logit[i] = dopac * opac * (1.f - opac);
+  }
   }
   __syncthreads();
-  unstage_sh<K3>(g_sh, i0, cnt, s_dsh);
+  if constexpr (FUSE) {
+    // the block's SH coefficients and their moments: one contiguous range,
+    // moved as float4 (16-byte aligned: the block starts at a multiple of
+    // 128 Gaussians) with four vectors of each array in flight per thread;
+    // every float is read and written once, so the accesses stream past L2
+    const int64_t base = i0 * K3;
+    const int total = cnt * K3;
+    const int total4 = total >> 2;
+    const float lr = tail.lr[4];
+    float4* P4 = reinterpret_cast<float4*>(tail.p_sh + base);
+    float4* M4 = reinterpret_cast<float4*>(tail.m_sh + base);
+    float4* V4 = reinterpret_cast<float4*>(tail.v_sh + base);
+    auto grad_at = [&](int e) {
+      const int t = e / K3, c = e - t * K3;
+      return s_dsh[c * kShStride + t];
+    };
+#pragma unroll 4
+    for (int e4 = threadIdx.x; e4 < total4; e4 += kProjThreads) {
+      float4 p = __ldcs(P4 + e4), mm = __ldcs(M4 + e4), vv = __ldcs(V4 + e4);
+      const int e = 4 * e4;
+      adam_one(p.x, grad_at(e), mm.x, vv.x, lr, tail.b1, tail.b2, tail.eps, tail.ibc1, tail.ibc2);
+      adam_one(p.y, grad_at(e + 1), mm.y, vv.y, lr, tail.b1, tail.b2, tail.eps, tail.ibc1,
+               tail.ibc2);
+      adam_one(p.z, grad_at(e + 2), mm.z, vv.z, lr, tail.b1, tail.b2, tail.eps, tail.ibc1,
+               tail.ibc2);
+      adam_one(p.w, grad_at(e + 3), mm.w, vv.w, lr, tail.b1, tail.b2, tail.eps, tail.ibc1,
+               tail.ibc2);
+      __stcs(P4 + e4, p);
+      __stcs(M4 + e4, mm);
+      __stcs(V4 + e4, vv);
+    }
+    for (int e = 4 * total4 + threadIdx.x; e < total; e += kProjThreads) {  // ragged end
+      float p = tail.p_sh[base + e], mm = tail.m_sh[base + e], vv = tail.v_sh[base + e];
+      adam_one(p, grad_at(e), mm, vv, lr, tail.b1, tail.b2, tail.eps, tail.ibc1, tail.ibc2);
+      tail.p_sh[base + e] = p;
+      tail.m_sh[base + e] = mm;
+      tail.v_sh[base + e] = vv;
+    }
+  } else {
+    unstage_sh<K3>(g_sh, i0, cnt, s_dsh);
+  }
 }
 
 }  // namespace
@@ -794,12 +877,12 @@ cudaError_t launch_project_bwd(const gs_params& p, const CamSet& cams, int n_vie
   auto gm = reinterpret_cast<float4*>(g.means);
   auto gs = reinterpret_cast<float4*>(g.log_scales);
   auto gq = reinterpret_cast<float4*>(g.quats);
-#define GS_PBWD2(D, AL, Q)                                                                   \
-  cudaFuncSetAttribute(k_project_bwd<D, AL, Q>, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
-                       (int)smem);                                                              \
-  k_project_bwd<D, AL, Q><<<blocks, threads, smem, stream>>>(                                   \
-      m, s, q, p.opacity_logit, p.sh, g2, radii, n, n_views, cams, gm, gs, gq, g.opacity_logit, \
-      g.sh, shq)
+#define GS_PBWD2(D, AL, Q)                                                                    \
+  cudaFuncSetAttribute(k_project_bwd<D, AL, Q, false>,                                           \
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                  \
+  k_project_bwd<D, AL, Q, false><<<blocks, threads, smem, stream>>>(                             \
+      m, s, q, p.opacity_logit, p.sh, g2, radii, n, n_views, cams, gm, gs, gq, g.opacity_logit,  \
+      g.sh, shq, AdamTail{})
 #define GS_PBWD1(D, AL)       \
   if (p.sh_quant) {           \
     GS_PBWD2(D, AL, true);    \
@@ -821,6 +904,41 @@ cudaError_t launch_project_bwd(const gs_params& p, const CamSet& cams, int n_vie
 #undef GS_PBWD
 #undef GS_PBWD1
 #undef GS_PBWD2
+  return cudaGetLastError();
+}
+
+cudaError_t launch_project_bwd_adam(const gs_params& p, const CamSet& cams, int n_views,
+                                    const float* grad2d, const int* radii, const AdamTail& t,
+                                    cudaStream_t stream) {
+  const int n = (int)p.n;
+  if (n == 0) return cudaSuccess;
+  const int threads = kProjThreads;
+  const int blocks = (n + threads - 1) / threads;
+  const int K3 = 3 * (p.sh_degree + 1) * (p.sh_degree + 1);
+  const bool alias = n_views == 1;
+  const size_t smem = (size_t)(alias ? 1 : 2) * K3 * kShStride * sizeof(float);
+  auto g2 = reinterpret_cast<const float4*>(grad2d);
+  // the parameters are read through the tail's pointers (they are updated in place)
+#define GS_PBWDF1(D, AL)                                                                        \
+  cudaFuncSetAttribute(k_project_bwd<D, AL, false, true>,                                         \
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                   \
+  k_project_bwd<D, AL, false, true><<<blocks, threads, smem, stream>>>(                           \
+      t.p_means, t.p_log_scales, t.p_quats, t.p_logit, t.p_sh, g2, radii, n, n_views, cams,      \
+      nullptr, nullptr, nullptr, nullptr, nullptr, ShQuant{}, t)
+#define GS_PBWDF(D)           \
+  if (alias) {                \
+    GS_PBWDF1(D, true);       \
+  } else {                    \
+    GS_PBWDF1(D, false);      \
+  }
+  switch (p.sh_degree) {
+    case 0: GS_PBWDF(0); break;
+    case 1: GS_PBWDF(1); break;
+    case 2: GS_PBWDF(2); break;
+    default: GS_PBWDF(3); break;
+  }
+#undef GS_PBWDF
+#undef GS_PBWDF1
   return cudaGetLastError();
 }
 

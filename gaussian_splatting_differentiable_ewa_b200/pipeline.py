@@ -142,6 +142,8 @@ class Splatter:
                                    None if quant else self.sh, self.deg,
                                    sh_quant=self.sh_q if quant else None)
         self.c_grads = api.grads(*[self.grads[k] for k, _ in self.param_list])
+        self.c_m = api.grads(*[self.exp_avg[k] for k, _ in self.param_list])
+        self.c_v = api.grads(*[self.exp_avg_sq[k] for k, _ in self.param_list])
         self.c_proj = api.projected(self.records, self.bins, self.radii)
         if getattr(self, "_shard", None) is not None:
             self._plan_shard()  # the slices follow the buffer size
@@ -221,6 +223,26 @@ class Splatter:
     def project_bwd(self):
         api.gs_project_bwd(self.c_params, self.cams, self.V, self.radii, self.grad2d,
                            self.c_grads, self.stream)
+
+    def fused_tail_ok(self) -> bool:
+        """Whether project_bwd_adam can end a step: one GPU's optimiser over
+        float32 SH."""
+        return self._shard is None and self.sh_bits is None
+
+    def project_bwd_adam(self, beta1=0.9, beta2=0.999, eps=1e-15, stats: bool = True):
+        """The step's tail in one launch (gs_project_bwd_adam): projection
+        backward from ``self.grad2d``, densification statistics (unless
+        stats is False) and the Adam step, the parameters updated in place;
+        the gradients are not materialised."""
+        if not self.fused_tail_ok():
+            raise ValueError("the fused tail needs an unsharded optimiser and float32 SH")
+        self.step_count += 1
+        names = [k for k, _ in self.param_list]
+        api.gs_project_bwd_adam(self.c_params, self.cams, self.V, self.radii, self.grad2d,
+                                self.c_m, self.c_v, [self.lr[k] for k in names], beta1, beta2,
+                                eps, self.step_count, self.accum_plain if stats else None,
+                                self.accum_abs if stats else None,
+                                self.denom if stats else None, self.stream)
 
     def densify_stats(self):
         api.gs_densify_stats(self.grad2d, self.radii, self.V, self.n, self.accum_plain,
@@ -341,12 +363,24 @@ class Splatter:
         self.bin_sort()
         self.rasterize_fwd()
 
-    def train_step(self, dL_dimage: torch.Tensor, adam: bool = True):
-        self.forward()
+    def _backward_tail(self, dL_dimage: torch.Tensor, adam: bool) -> None:
+        # with Adam on one GPU and float SH: screen-space backward, then the
+        # fused projection backward + statistics + Adam (no gradient arrays)
+        if adam and self.fused_tail_ok():
+            self.rasterize_bwd(dL_dimage, with_params=False)
+            self.project_bwd_adam()
+            return
         self.rasterize_bwd(dL_dimage)
         self.densify_stats()
         if adam:
             self.adam_step()
+
+    def train_step(self, dL_dimage: torch.Tensor, adam: bool = True):
+        """Render, backward, densification statistics and (with adam) the
+        Adam step; ``self.grads`` is written only on the unfused path
+        (adam False, a sharded optimiser or quantised SH)."""
+        self.forward()
+        self._backward_tail(dL_dimage, adam)
 
     def loss(self, target: torch.Tensor, lam: float = 0.2, grad: bool = True) -> torch.Tensor:
         """(1 - lam) L1 + lam (1 - SSIM) of the rendered image against
@@ -370,10 +404,7 @@ class Splatter:
         and its image gradient, then the backward, statistics and Adam."""
         self.forward()
         self.loss(target, lam)
-        self.rasterize_bwd(self.dL_loss)
-        self.densify_stats()
-        if adam:
-            self.adam_step()
+        self._backward_tail(self.dL_loss, adam)
 
     def train_from_host(self, dL_host, image_host, adam: bool = True, grad_hook=None) -> None:
         """Training steps fed from host memory, copies overlapped with compute.
@@ -427,8 +458,13 @@ class Splatter:
                     self._dL_dev[buf ^ 1].copy_(dL_host[k + 1], non_blocking=True)
                     uploaded[buf ^ 1].record(cs)
             comp.wait_event(uploaded[buf])
-            self.rasterize_bwd(self._dL_dev[buf])
+            # without a hook on the gradients the tail is the fused one
+            fused = adam and grad_hook is None and self.fused_tail_ok()
+            self.rasterize_bwd(self._dL_dev[buf], with_params=not fused)
             consumed[buf].record(comp)
+            if fused:
+                self.project_bwd_adam()
+                continue
             if grad_hook is not None:
                 with torch.cuda.stream(comp):
                     grad_hook()

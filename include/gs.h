@@ -360,6 +360,28 @@ gs_status gs_project_bwd(const gs_params* params, const gs_camera* cams, int32_t
                          const int32_t* radii, const float* grad2d, gs_grads* grads,
                          void* stream);
 
+/* The single-GPU training step's tail in one pass (lshu.cn sec. 3.3 Adam with
+ * per-group learning rates; jsqmd.com sec. 2 densification statistics): the
+ * projection backward of gs_project_bwd, then, instead of writing gradients,
+ * the Adam step of gs_adam_step applied to every parameter of every Gaussian
+ * (padding lanes included, with gradient 0) and the statistics of
+ * gs_densify_stats, all from the values in registers. The parameters of
+ * *params are updated IN PLACE (its arrays must be writable device memory);
+ * exp_avg / exp_avg_sq are the moments in the gs_params layouts (updated);
+ * lr[5] the learning rates of means, log-scales, quaternions, opacity logits
+ * and SH; beta1, beta2, eps, step as gs_adam_step. accum_plain, accum_abs
+ * (float [n]) and denom (int32 [n]) receive the statistics as
+ * gs_densify_stats adds them; all three NULL skips them. Parameters, moments
+ * and statistics equal those of gs_project_bwd + gs_densify_stats +
+ * gs_adam_step over the same groups, bit for bit. Float SH only
+ * (params->sh_quant NULL); the SH arrays of params, exp_avg and exp_avg_sq
+ * 16-byte aligned. Argument errors as those calls. One launch. */
+gs_status gs_project_bwd_adam(const gs_params* params, const gs_camera* cams, int32_t n_views,
+                              const int32_t* radii, const float* grad2d, gs_grads* exp_avg,
+                              gs_grads* exp_avg_sq, const float* lr, float beta1, float beta2,
+                              float eps, int64_t step, float* accum_plain, float* accum_abs,
+                              int32_t* denom, void* stream);
+
 /* Densification statistics (jsqmd.com sec. 2 table and sec. 3.1
  * `add_densification_stats`): for each view v and Gaussian i with
  * radii[v][i] > 0, accumulate

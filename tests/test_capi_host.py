@@ -205,3 +205,5 @@ def test_bench_work_model_uses_the_library_plan():
     assert bench.sort_plan(sp, "full64")["pair"] == 6
     # emit, digit counts, 6 passes, ranges
     assert bench.launches_per_step(sp, "full64") == 1 + (1 + 1 + 6 + 1) + 5
+    # the fused tail: raster fwd, raster bwd, projection backward + statistics + Adam
+    assert bench.launches_per_step(sp, "presort", fused=True) == 1 + (1 + 1 + 4 + 4) + 3

@@ -611,3 +611,48 @@ def test_sharded_optimizer_on_one_rank_matches_the_plain_step():
     assert torch.equal(a.param_flat, b.param_flat)
     assert torch.equal(a.m_flat, b.m_flat) and torch.equal(a.v_flat, b.v_flat)
     assert not torch.equal(a.param_flat, Splatter(sc).param_flat)   # the steps moved them
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("train_1m_1080p", dict(n=20000, width=320, height=192)),
+    ("train_6m_8x1080p", dict(n=6000, width=256, height=144, n_views=3)),
+    ("fwd_1k_128", dict()),
+])
+def test_fused_tail_equals_the_three_calls(name, kw):
+    """gs_project_bwd_adam (projection backward, densification statistics and
+    Adam in one launch, parameters updated in place) against gs_project_bwd +
+    gs_densify_stats + gs_adam_step from the same screen-space gradients and
+    state: parameters, moments and statistics bit for bit (SH degree 3 with
+    one view and with three, and degree 0)."""
+    sc = S.make_scene(name, **kw)
+    sp = Splatter(sc)
+    sp.ensure_capacity()
+    c = sc.cameras[0]
+    dL = torch.as_tensor(S.make_upstream_grad(sp.V, c.height, c.width, seed=3)).cuda()
+    sp.forward()
+    sp.rasterize_bwd(dL, with_params=False)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    sp.m_flat.copy_(torch.randn(sp.m_flat.shape, generator=g, device="cuda") * 1e-3)
+    sp.v_flat.copy_(torch.rand(sp.v_flat.shape, generator=g, device="cuda") * 1e-6)
+    sp.accum_plain.fill_(0.25)
+    sp.accum_abs.fill_(0.5)
+    sp.denom.fill_(2)
+    bufs = lambda: (sp.param_flat, sp.m_flat, sp.v_flat, sp.accum_plain, sp.accum_abs,  # noqa
+                    sp.denom)
+    state0 = [t.clone() for t in bufs()]
+    sp.step_count = 4
+    sp.project_bwd()
+    sp.densify_stats()
+    sp.adam_step()
+    torch.cuda.synchronize()
+    want = [t.clone() for t in bufs()]
+    for t, t0 in zip(bufs(), state0):
+        t.copy_(t0)
+    sp.step_count = 4
+    sp.project_bwd_adam()
+    torch.cuda.synchronize()
+    assert sp.status() == api.GS_OK
+    for got, w, label in zip(bufs(), want, ("params", "m", "v", "plain", "abs", "denom")):
+        assert torch.equal(got, w), label
+    assert not torch.equal(want[0], state0[0])   # the step moved the parameters
