@@ -204,6 +204,13 @@ __device__ __forceinline__ void adam_one(float& p, float g, float& m, float& v, 
   p -= __fdividef(lr * (m * ibc1), denom);
 }
 
+// Start moving the 128-byte line holding p towards L2 (no register result).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+__device__ __forceinline__ int lane_of_thread() { return (int)(threadIdx.x & 31); }
+
 // ||(gx, gy)|| of a view's screen-space mean gradient (the plain
 // densification statistic), one fixed operation sequence for every caller.
 __device__ __forceinline__ float densify_norm(float gx, float gy) {

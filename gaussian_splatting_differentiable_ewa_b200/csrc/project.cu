@@ -589,6 +589,31 @@ __global__ void __launch_bounds__(kProjThreads, 6) k_project_bwd(
   __syncthreads();
   float st_plain = 0.f, st_abs = 0.f;  // fused densification statistics
   int st_cnt = 0;
+  if constexpr (FUSE) {
+    // the moments this block updates at the end start towards L2 now, so
+    // their loads there overlap the chain rule below
+    // (one request per 128-byte line: every 8th lane for the float4 arrays,
+    // the first lane for the float ones)
+    if (live && (lane_of_thread() & 7) == 0) {
+      prefetch_l2(tail.m_means + i);
+      prefetch_l2(tail.v_means + i);
+      prefetch_l2(tail.m_log_scales + i);
+      prefetch_l2(tail.v_log_scales + i);
+      prefetch_l2(tail.m_quats + i);
+      prefetch_l2(tail.v_quats + i);
+      if (lane_of_thread() == 0) {
+        prefetch_l2(tail.m_logit + i);
+        prefetch_l2(tail.v_logit + i);
+      }
+    }
+    const int64_t sb = i0 * K3;
+    const int lines = (cnt * K3 + 31) / 32;  // 128-byte lines of the block's SH range
+    for (int l = threadIdx.x; l < lines; l += kProjThreads) {
+      prefetch_l2(tail.m_sh + sb + 32 * l);
+      prefetch_l2(tail.v_sh + sb + 32 * l);
+      prefetch_l2(tail.p_sh + sb + 32 * l);
+    }
+  }
   if (live) {
   bool touched = false;
   for (int v = 0; v < n_views; ++v) {
