@@ -253,6 +253,7 @@ KERNEL_OF = {
     "gs_rasterize_fwd": ("k_raster_fwd", "raster.cu"),
     "gs_rasterize_bwd": ("k_raster_bwd", "raster.cu"),
     "gs_project_bwd": ("k_project_bwd", "project.cu"),
+    "gs_project_bwd_adam": ("k_project_bwd_fused", "project.cu"),
     "gs_adam_step": ("k_adam", "optim.cu"),
 }
 

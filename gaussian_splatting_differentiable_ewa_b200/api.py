@@ -97,10 +97,10 @@ SIGNATURES = [
       _c.POINTER(GsBinned), _vp, _c.c_size_t, _vp]),
     ("gs_rasterize_fwd", _c.c_int,
      [_c.POINTER(GsProjected), _c.POINTER(GsBinned), _c.POINTER(GsCamera), _c.c_int32,
-      _c.c_int64, _c.POINTER(_c.c_float), _vp, _vp, _vp, _vp, _vp]),
+      _c.c_int64, _c.POINTER(_c.c_float), _vp, _vp, _vp, _vp, _vp, _vp]),
     ("gs_rasterize_bwd", _c.c_int,
      [_c.POINTER(GsParams), _c.POINTER(GsProjected), _c.POINTER(GsBinned),
-      _c.POINTER(GsCamera), _c.c_int32, _c.POINTER(_c.c_float), _vp, _vp, _vp, _vp,
+      _c.POINTER(GsCamera), _c.c_int32, _c.POINTER(_c.c_float), _vp, _vp, _vp, _vp, _vp,
       _c.POINTER(GsGrads), _vp, _vp]),
     ("gs_project_bwd", _c.c_int,
      [_c.POINTER(GsParams), _c.POINTER(GsCamera), _c.c_int32, _vp, _vp, _c.POINTER(GsGrads),
@@ -260,18 +260,21 @@ def gs_bin_sort(proj: GsProjected, cams_arr, n_views: int, n: int, sort_mode: in
 
 
 def gs_rasterize_fwd(proj: GsProjected, bins: GsBinned, cams_arr, n_views: int, n: int, bg,
-                     image, final_T, n_contrib, ws, stream=None) -> None:
+                     image, final_T, n_contrib, ws, stream=None, warp_masks=None) -> None:
+    """warp_masks: optional uint8 [pair_capacity] the backward can reuse."""
     _check(lib().gs_rasterize_fwd(_c.byref(proj), _c.byref(bins), cams_arr, int(n_views), int(n),
                                   _floats3(bg), _ptr(image), _ptr(final_T), _ptr(n_contrib),
-                                  _ptr(ws), _stream(stream)), "gs_rasterize_fwd")
+                                  _ptr(warp_masks), _ptr(ws), _stream(stream)),
+           "gs_rasterize_fwd")
 
 
 def gs_rasterize_bwd(p: GsParams, proj: GsProjected, bins: GsBinned, cams_arr, n_views: int, bg,
                      dL_dimage, final_T, n_contrib, grad2d, g: Optional[GsGrads], ws,
-                     stream=None) -> None:
+                     stream=None, warp_masks=None) -> None:
+    """warp_masks: the forward's (same lists), or None to test every entry again."""
     _check(lib().gs_rasterize_bwd(_c.byref(p), _c.byref(proj), _c.byref(bins), cams_arr,
                                   int(n_views), _floats3(bg), _ptr(dL_dimage), _ptr(final_T),
-                                  _ptr(n_contrib), _ptr(grad2d),
+                                  _ptr(n_contrib), _ptr(warp_masks), _ptr(grad2d),
                                   None if g is None else _c.byref(g), _ptr(ws), _stream(stream)),
            "gs_rasterize_bwd")
 

@@ -317,7 +317,8 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
 
 gs_status gs_rasterize_fwd(const gs_projected* proj, const gs_binned* bins, const gs_camera* cams,
                            int32_t n_views, int64_t n, const float* bg, float* image,
-                           float* final_T, uint32_t* n_contrib, void* ws, void* stream) {
+                           float* final_T, uint32_t* n_contrib, uint8_t* warp_masks, void* ws,
+                           void* stream) {
   if (!proj || !bins || !bg || !check_cams(cams, n_views) || !status_ws_ok(ws))
     return GS_ERR_INVALID_ARG;
   if (n < 0) return GS_ERR_INVALID_ARG;
@@ -327,7 +328,7 @@ gs_status gs_rasterize_fwd(const gs_projected* proj, const gs_binned* bins, cons
   const Grid g = grid_of(cams[0]);
   return cuda_status(launch_raster_fwd(proj->records, bins->ids, bins->ranges, bins->pair_capacity,
                                        g, n_views, (int)n, bg, image, final_T, n_contrib,
-                                       status_word(ws),
+                                       warp_masks, status_word(ws),
                                        wait_cfg(GS_STALL_RASTER_FWD),
                                        static_cast<cudaStream_t>(stream)));
 }
@@ -422,8 +423,8 @@ gs_status gs_project_bwd_adam(const gs_params* params, const gs_camera* cams, in
 gs_status gs_rasterize_bwd(const gs_params* params, const gs_projected* proj,
                            const gs_binned* bins, const gs_camera* cams, int32_t n_views,
                            const float* bg, const float* dL_dimage, const float* final_T,
-                           const uint32_t* n_contrib, float* grad2d, gs_grads* grads,
-                           void* ws, void* stream) {
+                           const uint32_t* n_contrib, const uint8_t* warp_masks,
+                           float* grad2d, gs_grads* grads, void* ws, void* stream) {
   if (!params || !proj || !bins || !bg || !check_cams(cams, n_views) || !status_ws_ok(ws))
     return GS_ERR_INVALID_ARG;
   const gs_params& p = *params;
@@ -441,7 +442,8 @@ gs_status gs_rasterize_bwd(const gs_params* params, const gs_projected* proj,
       cudaSuccess)
     return GS_ERR_CUDA;
   cudaError_t e = launch_raster_bwd(proj->records, bins->ids, bins->ranges, bins->pair_capacity, g,
-                                    n_views, (int)p.n, bg, dL_dimage, final_T, n_contrib, grad2d,
+                                    n_views, (int)p.n, bg, dL_dimage, final_T, n_contrib,
+                                    warp_masks, grad2d,
                                     status_word(ws),
                                     wait_cfg(GS_STALL_RASTER_BWD), st);
   if (e != cudaSuccess) return GS_ERR_CUDA;

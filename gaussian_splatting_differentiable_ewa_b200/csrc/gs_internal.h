@@ -117,14 +117,15 @@ cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream);
 cudaError_t launch_raster_fwd(const float* records, const uint32_t* ids, const int64_t* ranges,
                               int64_t capacity, const Grid& g, int n_views, int n,
                               const float bg[3], float* image,
-                              float* final_T, uint32_t* n_contrib, uint32_t* status,
-                              const WaitCfg& wc, cudaStream_t stream);
+                              float* final_T, uint32_t* n_contrib, uint8_t* warp_masks,
+                              uint32_t* status, const WaitCfg& wc, cudaStream_t stream);
 cudaError_t launch_raster_bwd(const float* records, const uint32_t* ids, const int64_t* ranges,
                               int64_t capacity, const Grid& g, int n_views, int n,
                               const float bg[3],
                               const float* dL_dimage, const float* final_T,
-                              const uint32_t* n_contrib, float* grad2d, uint32_t* status,
-                              const WaitCfg& wc, cudaStream_t stream);
+                              const uint32_t* n_contrib, const uint8_t* warp_masks,
+                              float* grad2d, uint32_t* status, const WaitCfg& wc,
+                              cudaStream_t stream);
 cudaError_t launch_densify(const float* grad2d, const int* radii, int n_views, int n,
                            float* accum_plain, float* accum_abs, int* denom, cudaStream_t stream);
 cudaError_t launch_adam(const gs_adam_group* groups, int n_groups, float b1, float b2, float eps,

@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(Shape<NP>::kThreads) k_raster_fwd(
     const float* __restrict__ records, const uint32_t* __restrict__ ids,
     const int64_t* __restrict__ ranges, RasterGeom geo, float bg0, float bg1, float bg2,
     float* __restrict__ image, float* __restrict__ final_T, uint32_t* __restrict__ n_contrib,
-    uint32_t* __restrict__ status, WaitCfg wc) {
+    uint8_t* __restrict__ wmask_out, uint32_t* __restrict__ status, WaitCfg wc) {
   using Sh = Shape<NP>;
   constexpr int kBatch = Sh::kBatch;
   __shared__ __align__(128) float s_rec[kBatch][GS_RECORD_FLOATS];
@@ -371,7 +371,9 @@ __global__ void __launch_bounds__(Shape<NP>::kThreads) k_raster_fwd(
     if ((int)threadIdx.x < m) {
       const uint32_t mask = prepare_record<NP>(&s_rec[threadIdx.x][0], &s_ev[threadIdx.x][0],
                                                tp.x0, tp.y0);
-      s_mask[threadIdx.x] = clipped ? 0u : (uint8_t)mask;
+      const uint8_t mk = clipped ? 0u : (uint8_t)mask;
+      s_mask[threadIdx.x] = mk;
+      if (wmask_out) wmask_out[start + (int64_t)b * kBatch + threadIdx.x] = mk;
     }
     __syncthreads();  // s_rec is free again
     if (b + 1 < nb) {
@@ -490,8 +492,8 @@ __global__ void __launch_bounds__(Shape<NP>::kThreads) k_raster_bwd(
     const float* __restrict__ records, const uint32_t* __restrict__ ids,
     const int64_t* __restrict__ ranges, RasterGeom geo, float bg0, float bg1, float bg2,
     const float* __restrict__ dL_dimage, const float* __restrict__ final_T,
-    const uint32_t* __restrict__ n_contrib, float* __restrict__ grad2d,
-    uint32_t* __restrict__ status, WaitCfg wc) {
+    const uint32_t* __restrict__ n_contrib, const uint8_t* __restrict__ wmask_in,
+    float* __restrict__ grad2d, uint32_t* __restrict__ status, WaitCfg wc) {
   using Sh = Shape<NP>;
   constexpr int kBatch = Sh::kBatch;
   constexpr int kWarps = Sh::kWarps;
@@ -614,8 +616,12 @@ __global__ void __launch_bounds__(Shape<NP>::kThreads) k_raster_bwd(
     pend[buf] = -1;
     if ((int)threadIdx.x < m) {
       float* r = &s_rec[buf][threadIdx.x][0];
-      const uint32_t mask = warp_block_mask_ellipse<NP>(
-          r, warp_block_mask<NP>(r[R_U], r[R_V], r[R_HX], r[R_HY], tp.x0, tp.y0), tp.x0, tp.y0);
+      // the forward's mask of this entry, or the same test again
+      const uint32_t mask =
+          wmask_in ? (uint32_t)wmask_in[start + (int64_t)b * kBatch + threadIdx.x]
+                   : warp_block_mask_ellipse<NP>(
+                         r, warp_block_mask<NP>(r[R_U], r[R_V], r[R_HX], r[R_HY], tp.x0, tp.y0),
+                         tp.x0, tp.y0);
       s_mask[threadIdx.x] = clipped[buf] ? 0u : (uint8_t)mask;
       r[R_OPAC] = 1.f / r[R_OPAC];  // d alpha / d opacity = alpha / o
     }
@@ -742,26 +748,30 @@ __global__ void __launch_bounds__(Shape<NP>::kThreads) k_raster_bwd(
 cudaError_t launch_raster_fwd(const float* records, const uint32_t* ids, const int64_t* ranges,
                               int64_t capacity, const Grid& g, int n_views, int n,
                               const float bg[3], float* image, float* final_T,
-                              uint32_t* n_contrib, uint32_t* status, const WaitCfg& wc,
+                              uint32_t* n_contrib, uint8_t* warp_masks, uint32_t* status,
+                              const WaitCfg& wc,
                               cudaStream_t stream) {
   const int64_t tiles = (int64_t)g.tiles_per_view * n_views;
   if (tiles == 0) return cudaSuccess;
   RasterGeom geo{g, n, n > 0 ? capacity : 0};
   k_raster_fwd<kPairs><<<(unsigned)tiles, Shape<kPairs>::kThreads, 0, stream>>>(
-      records, ids, ranges, geo, bg[0], bg[1], bg[2], image, final_T, n_contrib, status, wc);
+      records, ids, ranges, geo, bg[0], bg[1], bg[2], image, final_T, n_contrib, warp_masks, status,
+      wc);
   return cudaGetLastError();
 }
 
 cudaError_t launch_raster_bwd(const float* records, const uint32_t* ids, const int64_t* ranges,
                               int64_t capacity, const Grid& g, int n_views, int n,
                               const float bg[3], const float* dL_dimage, const float* final_T,
-                              const uint32_t* n_contrib, float* grad2d, uint32_t* status,
+                              const uint32_t* n_contrib, const uint8_t* warp_masks,
+                              float* grad2d, uint32_t* status,
                               const WaitCfg& wc, cudaStream_t stream) {
   const int64_t tiles = (int64_t)g.tiles_per_view * n_views;
   if (tiles == 0) return cudaSuccess;
   RasterGeom geo{g, n, n > 0 ? capacity : 0};
   k_raster_bwd<kPairs><<<(unsigned)tiles, Shape<kPairs>::kThreads, 0, stream>>>(
-      records, ids, ranges, geo, bg[0], bg[1], bg[2], dL_dimage, final_T, n_contrib, grad2d,
+      records, ids, ranges, geo, bg[0], bg[1], bg[2], dL_dimage, final_T, n_contrib, warp_masks,
+      grad2d,
       status, wc);
   return cudaGetLastError();
 }

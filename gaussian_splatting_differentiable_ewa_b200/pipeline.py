@@ -180,6 +180,8 @@ class Splatter:
     def _alloc_pairs(self, capacity: int) -> None:
         self.capacity = int(capacity)
         self.ids = torch.empty(max(self.capacity, 1), dtype=torch.int32, device=self.device)
+        # the forward's per-entry warp masks, reused by the backward
+        self.warp_masks = torch.empty(max(self.capacity, 1), dtype=torch.uint8, device=self.device)
         nbytes = api.gs_workspace_size(self.n, self.cams, self.V, self.capacity, self.sort_mode)
         if nbytes == 0:
             raise ValueError("invalid workspace request")
@@ -213,12 +215,14 @@ class Splatter:
 
     def rasterize_fwd(self):
         api.gs_rasterize_fwd(self.c_proj, self.c_bins, self.cams, self.V, self.n, self.bg,
-                             self.image, self.final_T, self.n_contrib, self.ws, self.stream)
+                             self.image, self.final_T, self.n_contrib, self.ws, self.stream,
+                             warp_masks=self.warp_masks)
 
     def rasterize_bwd(self, dL_dimage: torch.Tensor, with_params: bool = True):
         api.gs_rasterize_bwd(self.c_params, self.c_proj, self.c_bins, self.cams, self.V, self.bg,
                              dL_dimage, self.final_T, self.n_contrib, self.grad2d,
-                             self.c_grads if with_params else None, self.ws, self.stream)
+                             self.c_grads if with_params else None, self.ws, self.stream,
+                             warp_masks=self.warp_masks)
 
     def project_bwd(self):
         api.gs_project_bwd(self.c_params, self.cams, self.V, self.radii, self.grad2d,

@@ -314,6 +314,12 @@ gs_status gs_bin_sort_noalloc(const gs_projected* proj, const gs_camera* cams, i
  *   final_T   float [n_views][H][W]  transmittance after the last contributor
  *   n_contrib uint32 [n_views][H][W] 1 + position in the tile's list of the
  *             last contributing Gaussian (0 if none)
+ *   warp_masks (optional, NULL skips it) uint8 [pair_capacity], by pair
+ *             position: for every list entry the forward examined, bit w
+ *             (0..3) set if the entry's alpha >= 1/255 ellipse reaches the
+ *             tile's 8x8 pixel block w (blocks in row-major order within the
+ *             tile); entries past a tile's early stop are not written.
+ *             gs_rasterize_bwd reads it instead of testing every entry again.
  * `bg` is a host pointer to 3 floats. The test alpha_raw >= 1/255 is taken as
  * zq <= 0 on the record's evaluation form (see gs_projected) and alpha_raw
  * as 2^-zq / 255 with the SFU exp2. `ws` (device, 256-byte aligned, its
@@ -326,7 +332,7 @@ gs_status gs_bin_sort_noalloc(const gs_projected* proj, const gs_camera* cams, i
 gs_status gs_rasterize_fwd(const gs_projected* proj, const gs_binned* bins,
                            const gs_camera* cams, int32_t n_views, int64_t n,
                            const float* bg, float* image, float* final_T,
-                           uint32_t* n_contrib, void* ws, void* stream);
+                           uint32_t* n_contrib, uint8_t* warp_masks, void* ws, void* stream);
 
 /* Backward of gs_rasterize_fwd and gs_project (lshu.cn sec. 1
  * "differentiable rasterisation"). Given dL/dimage [n_views][3][H][W] and the
@@ -339,14 +345,16 @@ gs_status gs_rasterize_fwd(const gs_projected* proj, const gs_binned* bins,
  * (0 and 1 together are the view's plain view-space gradient), then the
  * gradients of the raw parameters summed over views into *grads
  * (overwritten; see gs_project_bwd). grad2d is overwritten. With
- * grads == NULL only grad2d is computed. `ws` as for gs_rasterize_fwd (the
- * same conditions are reported; a tile whose batch copy timed out adds
- * nothing further to grad2d). */
+ * grads == NULL only grad2d is computed. warp_masks: NULL, or the forward's
+ * (same binned lists and records): the backward then takes each entry's
+ * block mask from it (the entries it replays all lie before the forward's
+ * stop). `ws` as for gs_rasterize_fwd (the same conditions are reported; a
+ * tile whose batch copy timed out adds nothing further to grad2d). */
 gs_status gs_rasterize_bwd(const gs_params* params, const gs_projected* proj,
                            const gs_binned* bins, const gs_camera* cams, int32_t n_views,
                            const float* bg, const float* dL_dimage, const float* final_T,
-                           const uint32_t* n_contrib, float* grad2d, gs_grads* grads,
-                           void* ws, void* stream);
+                           const uint32_t* n_contrib, const uint8_t* warp_masks,
+                           float* grad2d, gs_grads* grads, void* ws, void* stream);
 
 /* Projection backward alone (the second half of gs_rasterize_bwd): the
  * gradients of the raw parameters from the screen-space gradients grad2d

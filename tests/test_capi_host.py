@@ -80,9 +80,10 @@ def test_bad_arguments_are_rejected_before_any_cuda_call():
     bn = api.GsBinned(None, None, None, 10)
     bg = (ctypes.c_float * 3)()
     assert L.gs_rasterize_fwd(ctypes.byref(out), ctypes.byref(bn), cams, 1, 10, bg, None, None,
-                              None, None, None) == api.GS_ERR_INVALID_ARG
+                              None, None, None, None) == api.GS_ERR_INVALID_ARG
     assert L.gs_rasterize_bwd(ctypes.byref(p), ctypes.byref(out), ctypes.byref(bn), cams, 1, bg,
-                              None, None, None, None, None, None, None) == api.GS_ERR_INVALID_ARG
+                              None, None, None, None, None, None, None, None) == \
+        api.GS_ERR_INVALID_ARG
     b = api.GsBinned(None, None, None, 10)
     assert L.gs_bin_sort(ctypes.byref(out), cams, 1, 10, 0, ctypes.byref(b), None, 0, None) == \
         api.GS_ERR_INVALID_ARG

@@ -656,3 +656,27 @@ def test_fused_tail_equals_the_three_calls(name, kw):
     for got, w, label in zip(bufs(), want, ("params", "m", "v", "plain", "abs", "denom")):
         assert torch.equal(got, w), label
     assert not torch.equal(want[0], state0[0])   # the step moved the parameters
+
+
+def test_backward_with_the_forwards_warp_masks_equals_testing_again():
+    """gs_rasterize_bwd taking each entry's 8x8-block mask from the forward
+    (warp_masks) against recomputing it: the same entries are replayed, so
+    grad2d agrees up to the order of its float atomic sums; the masks of a
+    1080p view cover only the entries before each tile's stop."""
+    sc = S.make_scene("train_1m_1080p", n=30000, width=640, height=384)
+    sp = Splatter(sc)
+    sp.ensure_capacity()
+    c = sc.cameras[0]
+    dL = torch.as_tensor(S.make_upstream_grad(1, c.height, c.width, seed=2)).cuda()
+    sp.forward()
+    sp.rasterize_bwd(dL, with_params=False)
+    torch.cuda.synchronize()
+    with_masks = sp.grad2d.clone()
+    api.gs_rasterize_bwd(sp.c_params, sp.c_proj, sp.c_bins, sp.cams, sp.V, sp.bg, dL,
+                         sp.final_T, sp.n_contrib, sp.grad2d, None, sp.ws, None,
+                         warp_masks=None)
+    torch.cuda.synchronize()
+    assert sp.status() == api.GS_OK
+    a, b = with_masks.cpu().numpy(), sp.grad2d.cpu().numpy()
+    assert np.count_nonzero(a) == np.count_nonzero(b)
+    assert np.abs(a - b).max() <= 1e-6 * np.abs(b).max()
