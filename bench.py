@@ -166,7 +166,7 @@ def sort_plan(sp, sort_mode: str) -> dict:
     path = {api.GS_PATH_TILES: "tiles", api.GS_PATH_COLUMNS: "columns",
             api.GS_PATH_TILE_ID: "tile_id"}[p.path]
     return dict(path=path, pre=p.presort_passes, pair=p.pair_passes, bpv=p.blocks_per_view,
-                tiles=tiles)
+                tiles=tiles, pair_sweep=bool(p.pair_single_sweep))
 
 
 def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float) -> dict:
@@ -237,10 +237,14 @@ def launches_per_step(sp, sort_mode: str, kind: str = "train", fused: bool = Fal
         sort = 1 + 1 + pair + 1                 # emit, digit counts, passes, ranges
     elif plan["path"] == "tiles":
         sort = 1 + 1 + pre + 4                  # keys, presort, count, scan, base, place
-    elif plan["path"] == "columns":
-        sort = 1 + 1 + pre + 3 + 3 * pair + 1   # ..., count, scan, emit, row passes, ranges
     else:
-        sort = 1 + 1 + pre + 1 + 3 * pair + 1
+        # row (columns) or tile-id passes: digit counts + one kernel each when
+        # single-sweep, count + scan + scatter each otherwise
+        passes = (1 + pair) if plan["pair_sweep"] else 3 * pair
+        if plan["path"] == "columns":
+            sort = 1 + 1 + pre + 3 + passes + 1   # ..., count, scan, emit, row passes, ranges
+        else:
+            sort = 1 + 1 + pre + 1 + passes + 1
     # project, sort, raster fwd (+ raster bwd, project bwd, densify (+ adam)),
     # or raster bwd + the fused tail
     tail = 2 if (kind == "train" and fused) else {"fwd": 0, "fwdbwd": 3, "train": 4}[kind]

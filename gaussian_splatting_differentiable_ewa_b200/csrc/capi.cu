@@ -708,6 +708,8 @@ gs_status gs_bin_sort_plan(int64_t n, int32_t n_views, const gs_camera* cams,
   plan->presort_passes = sort_mode == GS_SORT_PRESORT ? L.presort.passes : 0;
   plan->pair_passes = L.tile_emit ? 0 : L.pairs.passes;
   plan->gaussians_per_block = L.tile_emit ? L.gsize : 0;
+  plan->pair_single_sweep = pair_passes_single_sweep(L.pairs, sort_mode) ? 1 : 0;
+  plan->reserved = 0;
   plan->blocks_per_view = L.tile_emit ? L.tile_bpv : 0;
   return GS_OK;
 }

@@ -20,6 +20,9 @@ struct RadixPlan {
 // `key_bits` significant bits in the fewest passes of at most 8 bits; with
 // `balanced` the bits are split evenly (13 -> 7 + 6), else 8 per pass.
 RadixPlan make_radix_plan(int key_bits, bool balanced);
+// Whether a plan's pair passes run single-sweep (the 64-bit keys of full-64
+// mode; the 32-bit keys of the other paths take reduce-then-scan passes).
+bool pair_passes_single_sweep(const RadixPlan& pairs, int sort_mode);
 
 struct BinSortArgs {
   const float* bins;    // [n_views][n][4] binning records

@@ -220,6 +220,10 @@ size_t gs_workspace_size(int64_t n, int32_t n_views, const gs_camera* cams,
  *   presort_passes   radix passes over the per-Gaussian depth keys (0 in
  *                    full-64 mode);
  *   pair_passes      radix passes over the pair keys (0 on GS_PATH_TILES);
+ *   pair_single_sweep  1 if those passes are single-sweep (one digit-count
+ *                    kernel, then one kernel per pass: the 64-bit keys of
+ *                    full-64 mode), 0 if reduce-then-scan (three kernels per
+ *                    pass: the 32-bit keys of the other paths);
  *   gaussians_per_block, blocks_per_view  the Gaussian blocks of
  *                    GS_PATH_TILES (0 otherwise).
  * Returns GS_ERR_INVALID_ARG for a request gs_workspace_size rejects. */
@@ -229,6 +233,8 @@ typedef struct gs_sort_plan {
   int32_t presort_passes;
   int32_t pair_passes;
   int32_t gaussians_per_block;
+  int32_t pair_single_sweep;
+  int32_t reserved;
   int64_t blocks_per_view;
 } gs_sort_plan;
 gs_status gs_bin_sort_plan(int64_t n, int32_t n_views, const gs_camera* cams,

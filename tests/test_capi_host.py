@@ -177,6 +177,7 @@ def test_sort_plan_follows_the_grid_and_mode():
     assert (p.gaussians_per_block, p.blocks_per_view) == (4096, 733)
     p = plan(3840, 2160, 10_000_000, 1, api.GS_SORT_PRESORT)      # 4K: 240 x 135 tiles
     assert (p.path, p.pair_passes) == (api.GS_PATH_COLUMNS, 1)
+    assert p.pair_single_sweep == 0                                 # 32-bit row keys
     p = plan(128, 128, 1000, 1, api.GS_SORT_PRESORT)               # small scene: 32 per block
     assert (p.path, p.gaussians_per_block, p.blocks_per_view) == (api.GS_PATH_TILES, 32, 32)
     p = plan(800, 800, 100_000, 1, api.GS_SORT_PRESORT)
@@ -185,10 +186,14 @@ def test_sort_plan_follows_the_grid_and_mode():
     assert (p.path, p.pair_passes) == (api.GS_PATH_COLUMNS, 1)
     p = plan(8192, 1296, 1000, 1, api.GS_SORT_PRESORT)            # 512 x 81 tiles
     assert (p.path, p.pair_passes) == (api.GS_PATH_TILE_ID, 2)
+    assert p.pair_single_sweep == 0
+    p = plan(8192, 1296, 1000, 2, api.GS_SORT_PRESORT)            # 82944 tiles: 17 bits, 6 + 6 + 5
+    assert (p.pair_passes, p.pair_single_sweep) == (3, 0)       # 82944 tiles: 17 bits
     p = plan(1920, 1080, 1000, 8, api.GS_SORT_PRESORT)            # 3 view bits in the key
     assert p.presort_passes == 5
     p = plan(1920, 1080, 1000, 1, api.GS_SORT_FULL64)             # 13 tile bits + 32
     assert (p.path, p.presort_passes, p.pair_passes) == (api.GS_PATH_TILE_ID, 0, 6)
+    assert p.pair_single_sweep == 1
     with pytest.raises(api.GsError):
         plan(1920, 1080, -1, 1, api.GS_SORT_PRESORT)
 
@@ -199,7 +204,7 @@ def test_bench_work_model_uses_the_library_plan():
     cams = api.cameras(S.make_scene("train_1m_1080p", n=10).cameras)
     sp = types.SimpleNamespace(n=1_000_000, V=1, W=1920, H=1080, cams=cams)
     plan = bench.sort_plan(sp, "presort")
-    assert plan == dict(path="tiles", pre=4, pair=0, bpv=1303, tiles=8160)
+    assert plan == dict(path="tiles", pre=4, pair=0, bpv=1303, tiles=8160, pair_sweep=False)
     # project; depth keys, digit counts, 4 single-sweep passes, count, scan, base,
     # place; raster fwd, raster bwd, project bwd, densify stats, Adam
     assert bench.launches_per_step(sp, "presort") == 1 + (1 + 1 + 4 + 4) + 5
