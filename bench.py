@@ -43,6 +43,7 @@ import subprocess
 import sys
 import tempfile
 import time
+from typing import Optional
 
 import numpy as np
 
@@ -169,7 +170,20 @@ def sort_plan(sp, sort_mode: str) -> dict:
                 tiles=tiles, pair_sweep=bool(p.pair_single_sweep))
 
 
-def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float) -> dict:
+# FP32 operations of the blend kernels (an FMA is one operation): per (pixel,
+# list entry) evaluation, the evaluation form -- dx, dy, p1 and p2 (two FMAs
+# each), zq (two FMAs) and the test zq <= 0; per contributing pixel in the
+# forward, alpha = min(0.99, 2^-zq / 255) (multiply, min; the exp2 is an SFU
+# op), T (1 - alpha) (FMA, multiply), w = alpha T and the three colour FMAs;
+# in the backward, alpha, 1 - alpha and its reciprocal, T, w, the colour
+# behind (3 differences, 3 FMAs), dL/dalpha (3 + 2), the clamp, dalpha/dmean
+# through both eigen rows (6), the conic terms (5), opacity (1), colour (3),
+# the absolute-gradient norm (3) and the ten per-pixel sums.
+OPS_EVAL, OPS_FWD_CONTRIB, OPS_BWD_CONTRIB = 9, 8, 48
+
+
+def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float,
+                     examined: Optional[int] = None, evals: Optional[float] = None) -> dict:
     """Algorithmic bytes (and exp evaluations) per launch of each call, from
     the per-unit figures of the hot-path scope table (its measurement part):
 
@@ -184,9 +198,16 @@ def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float) -> dict:
                     (passes x 24 B),
                     the packed rectangles and the (tile, Gaussian block) count
                     table read and written once;
-      raster fwd    4 B id + 40 B record per pair + 20 B written per pixel;
-      raster bwd    the same list + 40 B of gradient atomics per pair + 12 B
-                    of dL/dpixel per pixel;
+      raster fwd    4 B id + 40 B record per pair read + 20 B written per
+                    pixel; the pairs read are the list entries the forward
+                    examined (`examined`: a tile stops walking its list once
+                    all its pixels have saturated), all pairs when not given;
+      raster bwd    the same entries + 40 B of gradient atomics each + 12 B
+                    of dL/dpixel per pixel; both blend kernels also count
+                    FP32 operations (OPS_*): `evals` (pixel, entry)
+                    evaluations -- 64 pixels for every 8x8 block an
+                    examined entry's mask names -- and `exps` contributing
+                    ones;
       project bwd   parameters read and gradients written once, 36 B of
                     screen-space gradients per Gaussian and view;
       densify       16 B per Gaussian and view + 24 B per Gaussian;
@@ -200,6 +221,8 @@ def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float) -> dict:
     before the pixel stops (counted by the oracle on a pixel sample)."""
     n, V = sp.n, sp.V
     P = V * sp.W * sp.H
+    walked = n_pairs if examined is None else examined
+    ev = 0.0 if evals is None else float(evals)
     pbytes = (11 + 3 * sp.K) * 4
     plan = sort_plan(sp, sort_mode)
     pre, pair = plan["pre"], plan["pair"]
@@ -214,8 +237,10 @@ def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float) -> dict:
     return {
         "gs_project": dict(bytes=n * pbytes + V * n * 48, exps=0.0),
         "gs_bin_sort": dict(bytes=sort_bytes, exps=0.0),
-        "gs_rasterize_fwd": dict(bytes=n_pairs * 44 + P * 20, exps=exps),
-        "gs_rasterize_bwd": dict(bytes=n_pairs * (44 + 40) + P * 12, exps=exps),
+        "gs_rasterize_fwd": dict(bytes=walked * 44 + P * 20, exps=exps,
+                                 ops=ev * OPS_EVAL + exps * OPS_FWD_CONTRIB),
+        "gs_rasterize_bwd": dict(bytes=walked * (44 + 40) + P * 12, exps=exps,
+                                 ops=ev * OPS_EVAL + exps * OPS_BWD_CONTRIB),
         "gs_project_bwd": dict(bytes=n * 2 * pbytes + V * n * 36, exps=0.0),
         "gs_densify_stats": dict(bytes=V * n * 16 + n * 24, exps=0.0),
         "gs_adam_step": dict(bytes=n * (pbytes // 4) * 28, exps=0.0),
@@ -300,6 +325,12 @@ def working_set_bytes(sp) -> int:
 def sfu_peak_gexps(sm_mhz: float, sms: int = 148) -> float:
     # MUFU.EX2: 16 results per SM per clock (4 per SM sub-partition)
     return sms * 16 * sm_mhz * 1e6 / 1e9
+
+
+def alu_peak_gops(sm_mhz: float, sms: int = 148) -> float:
+    # FP32: 128 lanes per SM, one operation (an FMA counting as one) per lane
+    # per clock
+    return sms * 128 * sm_mhz * 1e6 / 1e9
 
 
 # ----------------------------------------------------------------- CPU oracle
@@ -622,6 +653,19 @@ def run_ours(args):
         sp.shard_optimizer(rank, world)
     sp.ensure_capacity()
     V = sp.V
+    # the list entries a forward examines (the work model's raster units):
+    # entry masks are 4-bit, so entries still holding 0xFF after one forward
+    # were never reached (their tile had stopped)
+    sp.project()
+    sp.bin_sort()
+    sp.warp_masks.fill_(0xFF)
+    sp.rasterize_fwd()
+    torch.cuda.synchronize()
+    wm = sp.warp_masks[:int(sp.n_pairs.item())]
+    wm = wm[wm != 0xFF].to(torch.int32)
+    examined = int(wm.numel())
+    # (pixel, entry) evaluations: 64 pixels per 8x8 block an entry's mask names
+    evals = 64 * int(sum(((wm >> b) & 1).sum().item() for b in range(4)))
     # the parameters and moments the timed steps start from (Adam moves them;
     # the protocol run below starts from the same state)
     start_state = [t.clone() for t in (sp.param_flat, sp.m_flat, sp.v_flat)]
@@ -802,11 +846,12 @@ def run_ours(args):
         cpu, nexp_mean = cpu_baseline(scene, kind)
         exps = nexp_mean * pixels
     pk = peaks()
-    work = algorithmic_work(sp, n_pairs, args.sort_mode, exps or 0.0)
+    work = algorithmic_work(sp, n_pairs, args.sort_mode, exps or 0.0, examined, evals)
     if world > 1 and kind == "train":
         work["gs_adam_step"]["bytes"] /= world  # each rank updates its slice only
     kernels = {}
     sfu = sfu_peak_gexps(pk["sm_max_mhz"])
+    alu = alu_peak_gops(pk["sm_max_mhz"])
     for nm in names:
         key = nm if nm in work else "gs_adam_step"
         if key not in work:
@@ -820,6 +865,10 @@ def run_ours(args):
             k["gexps"] = w["exps"] / t / 1e9
             k["sfu_frac"] = k["gexps"] / sfu
             bound_s = max(bound_s, w["exps"] / (sfu * 1e9))
+        if w.get("ops"):
+            k["gops"] = w["ops"] / t / 1e9
+            k["alu_frac"] = k["gops"] / alu
+            bound_s = max(bound_s, w["ops"] / (alu * 1e9))
         k["bound_ms"] = bound_s * 1000.0
         k["roofline_frac"] = bound_s / t
         kernels[nm] = k
@@ -827,7 +876,14 @@ def run_ours(args):
     dk = "gs_adam_step" if dom not in work else dom
     t_hbm = work[dk]["bytes"] / (pk["hbm_gbs"] * 1e9)
     t_sfu = (work[dk]["exps"] / (sfu * 1e9)) if exps else 0.0
-    if t_sfu > t_hbm:
+    t_alu = work[dk].get("ops", 0.0) / (alu * 1e9)
+    if t_alu > max(t_hbm, t_sfu):
+        ach = work[dk]["ops"] / (per_call[dom] / 1000.0) / 1e9
+        roof = {"kernel": dom, "bound": "alu", "achieved": ach, "peak": alu, "unit": "Gop/s",
+                "frac": ach / alu, "traffic": profiled_traffic(dk, args.workload),
+                "peak_source": "148 SM x 128 FP32 lanes x %.0f MHz (max SM clock), FP32 "
+                               "operations of the evaluation form" % pk["sm_max_mhz"]}
+    elif t_sfu > t_hbm:
         ach = work[dk]["exps"] / (per_call[dom] / 1000.0) / 1e9
         roof = {"kernel": dom, "bound": "alu", "achieved": ach, "peak": sfu, "unit": "Gexp/s",
                 "frac": ach / sfu, "traffic": profiled_traffic(dk, args.workload),
@@ -839,7 +895,7 @@ def run_ours(args):
                 "unit": "GB/s", "frac": ach / pk["hbm_gbs"],
                 "traffic": profiled_traffic(dk, args.workload),
                 "peak_source": pk["source"]}
-    # step roofline: sum over calls of max(bytes / HBM, exps / SFU)
+    # step roofline: sum over calls of max(bytes / HBM, exps / SFU, ops / FP32)
     bound_ms = sum(k["bound_ms"] for k in kernels.values())
     n_launch = launches_per_step(sp, args.sort_mode, kind, fused)
     line = {
@@ -849,10 +905,12 @@ def run_ours(args):
         "data": "synthetic",
         "config": {"workload": args.workload, "step": kind, "gaussians": sp.n,
                    "width": c.width, "height": c.height, "views_per_gpu": V,
-                   "sh_degree": sp.deg, "pairs": n_pairs, "sort_mode": args.sort_mode,
+                   "sh_degree": sp.deg, "pairs": n_pairs, "pairs_examined": examined,
+                   "sort_mode": args.sort_mode,
                    "sort_path": sort_plan(sp, args.sort_mode)["path"],
                    "launch": "host launches" if graphs is None else
-                             "one CUDA graph per call (Adam launched from the host)",
+                             "one CUDA graph per call (the step's Adam, fused or not, launched "
+                             "from the host: its bias corrections follow the step)",
                    "l2": ("working set %.0f MB inside the 126 MB L2: flushed (256 MB write) "
                           "before every step, outside the step's own timing"
                           % (working_set_bytes(sp) / 1e6)) if flush_l2 else
