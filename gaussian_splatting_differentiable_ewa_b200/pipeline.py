@@ -90,6 +90,7 @@ class Splatter:
         collective moves a whole buffer and equal 16-byte aligned slices of
         it can be handed to ranks."""
         dev, f32 = self.device, torch.float32
+        self._gen = getattr(self, "_gen", 0) + 1
         src = [("means", means), ("log_scales", log_scales), ("quats", quats),
                ("opacity_logit", opacity_logit), ("sh", sh)]
         self.n = n = int(means.shape[0])
@@ -178,6 +179,7 @@ class Splatter:
         api.gs_sh_dequantize(self.sh_q, self.sh, self.stream)
 
     def _alloc_pairs(self, capacity: int) -> None:
+        self._gen = getattr(self, "_gen", 0) + 1  # captured graphs name the old buffers
         self.capacity = int(capacity)
         self.ids = torch.empty(max(self.capacity, 1), dtype=torch.int32, device=self.device)
         # the forward's per-entry warp masks, reused by the backward
@@ -213,10 +215,11 @@ class Splatter:
         api.gs_bin_sort(self.c_proj, self.cams, self.V, self.n, self.sort_mode, self.c_bins,
                         self.ws, self.stream)
 
-    def rasterize_fwd(self):
+    def rasterize_fwd(self, image: Optional[torch.Tensor] = None):
+        """Render into ``self.image`` (or `image`, a tensor of its shape)."""
         api.gs_rasterize_fwd(self.c_proj, self.c_bins, self.cams, self.V, self.n, self.bg,
-                             self.image, self.final_T, self.n_contrib, self.ws, self.stream,
-                             warp_masks=self.warp_masks)
+                             self.image if image is None else image, self.final_T,
+                             self.n_contrib, self.ws, self.stream, warp_masks=self.warp_masks)
 
     def rasterize_bwd(self, dL_dimage: torch.Tensor, with_params: bool = True):
         api.gs_rasterize_bwd(self.c_params, self.c_proj, self.c_bins, self.cams, self.V, self.bg,
@@ -325,6 +328,30 @@ class Splatter:
                 None if sh is None else (sh["lo"], sh["hi"]),
                 None if sh is None else sh["group"])
 
+    def _graph_of(self, fn) -> "torch.cuda.CUDAGraph":
+        """A CUDA graph of one fixed-shape call: run once outside capture (on
+        a capture stream ordered after the current one), then captured."""
+        saved = self.stream
+        cap = torch.cuda.Stream(device=self.device)
+        cap.wait_stream(torch.cuda.current_stream(self.device))
+        if saved is not None:
+            cap.wait_stream(saved)
+        try:
+            with torch.cuda.stream(cap):
+                self.stream = cap
+                fn()
+            cap.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                self.stream = cap
+                fn()
+        finally:
+            self.stream = saved
+        torch.cuda.current_stream(self.device).wait_stream(cap)
+        if saved is not None:
+            saved.wait_stream(cap)
+        return g
+
     def capture_calls(self, dL_dimage: Optional[torch.Tensor] = None) -> dict:
         """CUDA graphs of this Splatter's fixed-shape calls: 'project',
         'bin_sort', 'rasterize_fwd' and, given an upstream gradient,
@@ -332,35 +359,17 @@ class Splatter:
         Every size and pointer of those calls is fixed once ensure_capacity has
         sized the buffers, so a graph replays the call's kernels with no host
         launch gaps between them (gs_bin_sort alone is up to 17 launches).
-        Replays run on the current stream. The Adam step is not captured: its
-        bias corrections follow the step count, a host value of the call. The
-        graphs stay valid until a buffer is reallocated (ensure_capacity growing
-        the pairs, densify_and_prune)."""
+        Replays run on the current stream. The Adam step (fused or not) is not
+        captured: its bias corrections follow the step count, a host value of
+        the call. The graphs stay valid until a buffer is reallocated
+        (ensure_capacity growing the pairs, densify_and_prune)."""
         calls = {"project": self.project, "bin_sort": self.bin_sort,
                  "rasterize_fwd": self.rasterize_fwd}
         if dL_dimage is not None:
             calls["rasterize_bwd"] = lambda: self.rasterize_bwd(dL_dimage, with_params=False)
             calls["project_bwd"] = self.project_bwd
             calls["densify_stats"] = self.densify_stats
-        saved = self.stream
-        cap = torch.cuda.Stream(device=self.device)
-        cap.wait_stream(torch.cuda.current_stream(self.device))
-        graphs = {}
-        try:
-            for name, fn in calls.items():
-                with torch.cuda.stream(cap):
-                    self.stream = cap
-                    fn()  # the call once outside capture, on the capture stream
-                cap.synchronize()
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=cap):
-                    self.stream = cap
-                    fn()
-                graphs[name] = g
-        finally:
-            self.stream = saved
-        torch.cuda.current_stream(self.device).wait_stream(cap)
-        return graphs
+        return {name: self._graph_of(fn) for name, fn in calls.items()}
 
     def forward(self):
         self.project()
@@ -415,56 +424,81 @@ class Splatter:
 
         Step k uploads ``dL_host[k]`` (pinned, [V][3][H][W] float32), runs one
         training step and downloads the rendered image into ``image_host[k]``
-        (pinned). The copies run on a second stream: step k + 1's gradient
-        uploads (into the other of two device buffers) while step k computes,
-        and step k's image downloads while its backward runs; events order the
-        next forward after that download and each upload after the backward
-        that last read its buffer. Everything is enqueued; the caller
-        synchronises. ``self.stream`` must be a stream other than the legacy
-        default stream (which would serialise the two). ``grad_hook()``, if
-        given, runs on the compute stream between the backward and the
-        statistics (e.g. a gradient clip; the multi-GPU exchange is part of
-        adam_step once shard_optimizer was called)."""
+        (pinned). The copies run on two streams of their own, one per
+        direction, so that an upload and a download proceed together: step
+        k + 1's gradient uploads (into the other of two device buffers) as
+        soon as step k - 1's backward is done with that buffer, and step k's
+        image downloads while its backward runs; events order the next
+        forward after that download and each backward after its upload.
+        Everything is enqueued; the caller synchronises. ``self.stream`` must
+        be a stream other than the legacy default stream (which would
+        serialise them). ``grad_hook()``, if given, runs on the compute
+        stream between the backward and the statistics (e.g. a gradient clip;
+        the multi-GPU exchange is part of adam_step once shard_optimizer was
+        called)."""
         comp = self.stream
         if comp is None:
             raise ValueError("train_from_host needs Splatter(stream=...) on a created stream")
         n = len(dL_host)
         if n != len(image_host):
             raise ValueError("one image buffer per gradient")
-        if getattr(self, "_copy_stream", None) is None:
-            self._copy_stream = torch.cuda.Stream(device=self.device)
+        if getattr(self, "_copy_streams", None) is None:
+            self._copy_streams = (torch.cuda.Stream(device=self.device),
+                                  torch.cuda.Stream(device=self.device))
             self._dL_dev = [torch.empty((self.V, 3, self.H, self.W), dtype=torch.float32,
                                         device=self.device) for _ in range(2)]
-        cs = self._copy_stream
+        up, down = self._copy_streams
+        # one CUDA graph per fixed-shape call (two for the backward, one per
+        # gradient buffer), kept until a buffer is reallocated
+        hg = getattr(self, "_host_graphs", None)
+        if hg is None or hg[0] != self._gen:
+            gr = {"project": self._graph_of(self.project),
+                  "bin_sort": self._graph_of(self.bin_sort),
+                  "rasterize_fwd": self._graph_of(self.rasterize_fwd)}
+            for b in range(2):
+                gr["bwd%d" % b] = self._graph_of(
+                    lambda b=b: self.rasterize_bwd(self._dL_dev[b], with_params=False))
+            self._host_graphs = hg = (self._gen, gr)
+        gr = hg[1]
+
+        def run(name, fn):
+            with torch.cuda.stream(comp):
+                gr[name].replay() if name in gr else fn()
+
         uploaded = [torch.cuda.Event(), torch.cuda.Event()]
         consumed = [torch.cuda.Event(), torch.cuda.Event()]
         rendered = torch.cuda.Event()
         downloaded = torch.cuda.Event()
-        cs.wait_stream(comp)  # nothing earlier on the compute stream is overtaken
-        with torch.cuda.stream(cs):
+        up.wait_stream(comp)  # nothing earlier on the compute stream is overtaken
+        down.wait_stream(comp)
+        with torch.cuda.stream(up):
             self._dL_dev[0].copy_(dL_host[0], non_blocking=True)
-            uploaded[0].record(cs)
+            uploaded[0].record(up)
         for k in range(n):
             buf = k & 1
-            self.project()
-            self.bin_sort()
+            if k + 1 < n:  # the next step's gradient, once its buffer is free
+                if k >= 1:
+                    up.wait_event(consumed[buf ^ 1])  # step k - 1's backward is done with it
+                with torch.cuda.stream(up):
+                    self._dL_dev[buf ^ 1].copy_(dL_host[k + 1], non_blocking=True)
+                    uploaded[buf ^ 1].record(up)
+            run("project", self.project)
+            run("bin_sort", self.bin_sort)
             if k > 0:
                 comp.wait_event(downloaded)  # the previous image has left
-            self.rasterize_fwd()
+            run("rasterize_fwd", self.rasterize_fwd)
             rendered.record(comp)
-            cs.wait_event(rendered)
-            with torch.cuda.stream(cs):
+            down.wait_event(rendered)
+            with torch.cuda.stream(down):
                 image_host[k].copy_(self.image, non_blocking=True)
-                downloaded.record(cs)
-                if k + 1 < n:
-                    if k >= 1:
-                        cs.wait_event(consumed[buf ^ 1])  # step k - 1's backward is done with it
-                    self._dL_dev[buf ^ 1].copy_(dL_host[k + 1], non_blocking=True)
-                    uploaded[buf ^ 1].record(cs)
+                downloaded.record(down)
             comp.wait_event(uploaded[buf])
             # without a hook on the gradients the tail is the fused one
             fused = adam and grad_hook is None and self.fused_tail_ok()
-            self.rasterize_bwd(self._dL_dev[buf], with_params=not fused)
+            if fused:
+                run("bwd%d" % buf, None)
+            else:
+                self.rasterize_bwd(self._dL_dev[buf])
             consumed[buf].record(comp)
             if fused:
                 self.project_bwd_adam()
@@ -479,32 +513,50 @@ class Splatter:
 
     def render_to_host(self, image_host) -> None:
         """Forward renders delivered to host memory, copies overlapped with
-        compute: step k renders and downloads the image into ``image_host[k]``
-        (pinned, [V][3][H][W] float32) on a second stream while step k + 1
-        projects and sorts; step k + 1's rasterisation waits for that download.
-        Everything is enqueued; the caller synchronises. ``self.stream`` must
-        be a created stream (see train_from_host)."""
+        compute: step k renders into one of two device image buffers and
+        downloads it into ``image_host[k]`` (pinned, [V][3][H][W] float32) on a
+        second stream while step k + 1 projects, sorts and renders into the
+        other buffer; a render waits only for the download of the buffer it
+        reuses (step k - 1's). The calls replay as CUDA graphs, kept until a
+        buffer is reallocated. Everything is enqueued; the caller
+        synchronises; ``self.image`` ends up holding the last image.
+        ``self.stream`` must be a created stream (see train_from_host)."""
         comp = self.stream
         if comp is None:
             raise ValueError("render_to_host needs Splatter(stream=...) on a created stream")
         if getattr(self, "_copy_stream", None) is None:
             self._copy_stream = torch.cuda.Stream(device=self.device)
         cs = self._copy_stream
+        rg = getattr(self, "_render_graphs", None)
+        if rg is None or rg[0] != self._gen:
+            imgs = [self.image, torch.empty_like(self.image)]
+            gr = {"project": self._graph_of(self.project),
+                  "bin_sort": self._graph_of(self.bin_sort)}
+            for b in range(2):
+                gr["fwd%d" % b] = self._graph_of(lambda b=b: self.rasterize_fwd(imgs[b]))
+            self._render_graphs = rg = (self._gen, gr, imgs)
+        gr, imgs = rg[1], rg[2]
         rendered = torch.cuda.Event()
-        downloaded = torch.cuda.Event()
+        downloaded = [torch.cuda.Event(), torch.cuda.Event()]
         cs.wait_stream(comp)
-        for k in range(len(image_host)):
-            self.project()
-            self.bin_sort()
-            if k > 0:
-                comp.wait_event(downloaded)
-            self.rasterize_fwd()
-            rendered.record(comp)
-            cs.wait_event(rendered)
-            with torch.cuda.stream(cs):
-                image_host[k].copy_(self.image, non_blocking=True)
-                downloaded.record(cs)
-        comp.wait_event(downloaded)
+        n = len(image_host)
+        with torch.cuda.stream(comp):
+            for k in range(n):
+                b = k & 1
+                gr["project"].replay()
+                gr["bin_sort"].replay()
+                if k > 1:
+                    comp.wait_event(downloaded[b])  # step k - 2's image has left this buffer
+                gr["fwd%d" % b].replay()
+                rendered.record(comp)
+                cs.wait_event(rendered)
+                with torch.cuda.stream(cs):
+                    image_host[k].copy_(imgs[b], non_blocking=True)
+                    downloaded[b].record(cs)
+            if n > 0:
+                if (n - 1) & 1:
+                    self.image.copy_(imgs[1])
+                comp.wait_event(downloaded[(n - 1) & 1])
 
     def densify_and_prune(self, grad_threshold: float = 0.0002, scale_split: float = 0.05,
                           min_opacity: float = 0.005, max_scale: float = 1.0,

@@ -683,3 +683,25 @@ def test_backward_with_the_forwards_warp_masks_equals_testing_again():
     a, b = with_masks.cpu().numpy(), sp.grad2d.cpu().numpy()
     assert np.count_nonzero(a) == np.count_nonzero(b)
     assert np.abs(a - b).max() <= 1e-6 * np.abs(b).max()
+
+
+def test_render_to_host_matches_device_renders():
+    # forward-only host delivery: double-buffered device images, graphs,
+    # downloads on a second stream; every host image equals the device render
+    sc = S.make_scene("fwd_100k_800", n=20000, width=400, height=304)
+    ref = Splatter(sc)
+    ref.ensure_capacity()
+    ref.forward()
+    torch.cuda.synchronize()
+    want = ref.image.cpu().numpy()
+    sp = Splatter(sc, stream=torch.cuda.Stream())
+    sp.ensure_capacity()
+    for steps in (3, 2):   # an odd and an even count (the last image in either buffer)
+        h_out = [torch.empty(sp.image.shape, dtype=torch.float32).pin_memory()
+                 for _ in range(steps)]
+        sp.render_to_host(h_out)
+        torch.cuda.synchronize()
+        assert sp.status() == api.GS_OK
+        for h in h_out:
+            assert np.array_equal(h.numpy(), want)
+        assert np.array_equal(sp.image.cpu().numpy(), want)
