@@ -792,7 +792,8 @@ def run_ours(args):
 
     # end to end through the library's host-fed calls: every step uploads its
     # upstream gradient from pinned host memory (training) and downloads the
-    # rendered image to it, on a copy stream overlapping the compute stream
+    # rendered image to it, on copy streams (one per direction) overlapping
+    # the compute stream
     e2e = None
     if not args.no_e2e:
         h_out = torch.empty(sp.image.shape, dtype=torch.float32).pin_memory()
