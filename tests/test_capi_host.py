@@ -213,3 +213,17 @@ def test_bench_work_model_uses_the_library_plan():
     assert bench.launches_per_step(sp, "full64") == 1 + (1 + 1 + 6 + 1) + 5
     # the fused tail: raster fwd, raster bwd, projection backward + statistics + Adam
     assert bench.launches_per_step(sp, "presort", fused=True) == 1 + (1 + 1 + 4 + 4) + 3
+    # blend kernels: bytes on the examined entries, FP32 operations on the
+    # evaluations and the contributing pixels
+    sp.K = 16
+    P = 1920 * 1080
+    w = bench.algorithmic_work(sp, 26_000_000, "presort", 1.0e8, 2_000_000, 3.0e8)
+    assert w["gs_rasterize_fwd"]["bytes"] == 2_000_000 * 44 + P * 20
+    assert w["gs_rasterize_bwd"]["bytes"] == 2_000_000 * 84 + P * 12
+    assert w["gs_rasterize_fwd"]["ops"] == 3.0e8 * bench.OPS_EVAL + 1.0e8 * bench.OPS_FWD_CONTRIB
+    assert w["gs_rasterize_bwd"]["ops"] == 3.0e8 * bench.OPS_EVAL + 1.0e8 * bench.OPS_BWD_CONTRIB
+    assert w["gs_project_bwd_adam"]["bytes"] == 1_000_000 * (6 * 236 + 36 + 24)
+    # without the examined count every pair is charged (the scope table's ceiling)
+    w0 = bench.algorithmic_work(sp, 26_000_000, "presort", 1.0e8)
+    assert w0["gs_rasterize_fwd"]["bytes"] == 26_000_000 * 44 + P * 20
+    assert bench.alu_peak_gops(1965.0) == pytest.approx(148 * 128 * 1.965)
