@@ -295,8 +295,15 @@ def test_adam_matches_oracle_on_generated_inputs():
         assert P.rel_l2(p.cpu().numpy(), rp) < 1e-6
 
 
-def test_train_step_adam_state_matches_oracle():
-    sc, sp = _setup("fwd_1k_128", dict(n=800), api.GS_SORT_FULL64)
+@pytest.mark.parametrize("name,kw,mode", [
+    ("fwd_1k_128", dict(n=800), api.GS_SORT_FULL64),
+    ("fwd_100k_800", dict(n=1500, width=160, height=120), api.GS_SORT_PRESORT),
+])
+def test_train_step_adam_state_matches_oracle(name, kw, mode):
+    # one training step on one GPU runs the fused tail (projection backward,
+    # statistics and Adam in one launch): SH degree 0 and 3 against the
+    # oracle's gradients through its Adam step
+    sc, sp = _setup(name, kw, mode)
     p0 = {k: t.clone() for k, t in sp.param_list}
     c = sc.cameras[0]
     dL = S.make_upstream_grad(1, c.height, c.width, seed=1)
