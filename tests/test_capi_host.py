@@ -130,6 +130,47 @@ def test_loss_and_quant_arguments_are_rejected_before_any_cuda_call():
                                    None) == api.GS_ERR_INVALID_ARG   # beta1 1
     q = api.GsShQuant(None, None, 0, 12, 8)
     assert L.gs_sh_quantize(None, ctypes.byref(q), None) == api.GS_OK
+    # packed state: moments travel in the blocks, so separate moment arrays are refused
+    qp = api.GsShQuant(16, 16, 100, 12, 16, api.GS_QUANT_PACKED, 0)
+    assert L.gs_adam_step_sh_quant(ctypes.byref(qp), p, p, p, 1e-3, 0.9, 0.999, 1e-15, 1, 0, 0,
+                                   None) == api.GS_ERR_INVALID_ARG
+    qx = api.GsShQuant(16, 16, 100, 12, 16, 7, 0)        # no such layout
+    assert L.gs_sh_quantize(p, ctypes.byref(qx), None) == api.GS_ERR_INVALID_ARG
+    # densify of the codes: mismatched widths or layouts, a count above 2 n,
+    # planar moments missing, a workspace too small
+    a = api.GsShQuant(16, 16, 100, 12, 8, api.GS_QUANT_PLANAR, 0)
+    b16 = api.GsShQuant(16, 16, 150, 12, 16, api.GS_QUANT_PLANAR, 0)
+    big = api.GsShQuant(16, 16, 201, 12, 8, api.GS_QUANT_PLANAR, 0)
+    ok = api.GsShQuant(16, 16, 150, 12, 8, api.GS_QUANT_PLANAR, 0)
+    ws = ctypes.c_void_p(4096)
+    nws = api.gs_densify_sh_quant_workspace_size(100, 150)
+    assert nws > 0 and api.gs_densify_sh_quant_workspace_size(-1, 0) == 0
+    f = L.gs_densify_sh_quant
+    assert f(ctypes.byref(a), p, p, p, ctypes.byref(b16), p, p, ws, nws, None) == \
+        api.GS_ERR_INVALID_ARG
+    assert f(ctypes.byref(a), p, p, p, ctypes.byref(big), p, p, ws, nws, None) == \
+        api.GS_ERR_INVALID_ARG
+    assert f(ctypes.byref(a), None, p, p, ctypes.byref(ok), p, p, ws, nws, None) == \
+        api.GS_ERR_INVALID_ARG
+    assert f(ctypes.byref(a), p, p, p, ctypes.byref(ok), p, p, ws, 8, None) == \
+        api.GS_ERR_INVALID_ARG
+    # the fused step tail: quantised SH, step 0, beta1 = 1, half the statistics
+    cams = api.cameras(S.make_scene("fwd_1k_128", n=10).cameras)
+    pr = api.GsParams(16, 16, 16, 16, 16, 0, 0, 10, None)
+    g = api.GsGrads(16, 16, 16, 16, 16)
+    lr5 = (ctypes.c_float * 5)(1e-3, 1e-3, 1e-3, 1e-3, 1e-3)
+    fa = L.gs_project_bwd_adam
+    assert fa(ctypes.byref(pr), cams, 1, p, p, ctypes.byref(g), ctypes.byref(g), lr5, 0.9,
+              0.999, 1e-15, 0, None, None, None, None) == api.GS_ERR_INVALID_ARG
+    assert fa(ctypes.byref(pr), cams, 1, p, p, ctypes.byref(g), ctypes.byref(g), lr5, 1.0,
+              0.999, 1e-15, 1, None, None, None, None) == api.GS_ERR_INVALID_ARG
+    assert fa(ctypes.byref(pr), cams, 1, p, p, ctypes.byref(g), ctypes.byref(g), lr5, 0.9,
+              0.999, 1e-15, 1, p, None, None, None) == api.GS_ERR_INVALID_ARG
+    qs = api.GsShQuant(16, 16, 10, 3, 8, api.GS_QUANT_PLANAR, 0)
+    prq = api.GsParams(16, 16, 16, 16, None, 0, 0, 10,
+                       ctypes.cast(ctypes.pointer(qs), ctypes.c_void_p))
+    assert fa(ctypes.byref(prq), cams, 1, p, p, ctypes.byref(g), ctypes.byref(g), lr5, 0.9,
+              0.999, 1e-15, 1, None, None, None, None) == api.GS_ERR_INVALID_ARG
 
 
 def test_densify_thresholds_convert_to_the_raw_parameter_units():
