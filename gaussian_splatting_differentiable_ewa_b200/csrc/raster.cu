@@ -204,6 +204,16 @@ __device__ __forceinline__ uint32_t warp_block_mask_ellipse(const float* r, uint
   return mask;
 }
 
+// Both tests on a record in its stored form, out of line: the backward runs
+// it only when no forward masks are given, and inlined there its registers
+// counted against the whole walk (70 registers, 7 blocks per SM, against 64
+// and 8 out of line: 0.550 against 0.573 ms on the 1M-splat 1080p frame).
+template <int NP>
+__device__ __noinline__ uint32_t record_block_mask(const float* r, int x0, int y0) {
+  return warp_block_mask_ellipse<NP>(
+      r, warp_block_mask<NP>(r[R_U], r[R_V], r[R_HX], r[R_HY], x0, y0), x0, y0);
+}
+
 // The pixel-independent part of the evaluation at column pxc: dx = pxc - uh
 // and a_i = fma(w_ix, dx, c_i), as (x, x) pairs.
 struct EvCol {
@@ -619,9 +629,7 @@ __global__ void __launch_bounds__(Shape<NP>::kThreads) k_raster_bwd(
       // the forward's mask of this entry, or the same test again
       const uint32_t mask =
           wmask_in ? (uint32_t)wmask_in[start + (int64_t)b * kBatch + threadIdx.x]
-                   : warp_block_mask_ellipse<NP>(
-                         r, warp_block_mask<NP>(r[R_U], r[R_V], r[R_HX], r[R_HY], tp.x0, tp.y0),
-                         tp.x0, tp.y0);
+                   : record_block_mask<NP>(r, tp.x0, tp.y0);
       s_mask[threadIdx.x] = clipped[buf] ? 0u : (uint8_t)mask;
       r[R_OPAC] = 1.f / r[R_OPAC];  // d alpha / d opacity = alpha / o
     }

@@ -349,6 +349,36 @@ def test_capacity_exceeded_reports_and_empties():
 
 
 @pytest.mark.parametrize("mode", MODES)
+def test_pair_count_beyond_32_bits_reports_and_empties(mode):
+    """140,000 Gaussians that each cover all 240 x 135 tiles of a 3840x2160
+    view need 4,536,000,000 pairs, more than a 32-bit count holds: the count
+    comes back exact (the oracle's rectangles summed in int64), the capacity
+    error is raised, every range stays empty, the image is the background and
+    the backward writes zero gradients."""
+    sc = S.make_scene("train_10m_4k", n=140_000)
+    sc.log_scales[:] = np.log(30.0)
+    sc.opacity_logit[:] = 4.0
+    sc.background = np.array([0.25, 0.5, 0.75], np.float32)
+    projs = O.project_views(sc)
+    r = projs[0]["rect"].astype(np.int64)
+    need = int(((r[:, 1] - r[:, 0] + 1) * (r[:, 3] - r[:, 2] + 1))[projs[0]["valid"] != 0].sum())
+    assert need > 1 << 32
+    sp = Splatter(sc, sort_mode=mode, pair_capacity=1 << 16)
+    sp.forward()
+    assert sp.status() == api.GS_ERR_CAPACITY
+    assert int(sp.n_pairs.item()) == need
+    assert int(sp.ranges.abs().sum().item()) == 0
+    assert torch.all(sp.final_T == 1.0)
+    img = sp.image.cpu().numpy()
+    for ch in range(3):
+        assert np.all(img[0, ch] == sc.background[ch])
+    sp.rasterize_bwd(torch.ones((1, 3, 2160, 3840), device="cuda"))
+    torch.cuda.synchronize()
+    for t in sp.grads.values():
+        assert torch.all(t == 0)
+
+
+@pytest.mark.parametrize("mode", MODES)
 def test_empty_and_all_culled(mode):
     for n, behind in ((0, False), (50, True)):
         sc = S.make_scene("fwd_1k_128", n=max(n, 1))
