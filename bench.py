@@ -167,7 +167,8 @@ def sort_plan(sp, sort_mode: str) -> dict:
     path = {api.GS_PATH_TILES: "tiles", api.GS_PATH_COLUMNS: "columns",
             api.GS_PATH_TILE_ID: "tile_id"}[p.path]
     return dict(path=path, pre=p.presort_passes, pair=p.pair_passes, bpv=p.blocks_per_view,
-                tiles=tiles, pair_sweep=bool(p.pair_single_sweep))
+                tiles=tiles, pair_sweep=bool(p.pair_single_sweep),
+                count_ranges=bool(p.ranges_from_counts))
 
 
 # FP32 operations of the blend kernels (an FMA is one operation): per (pixel,
@@ -197,7 +198,12 @@ def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float,
                     once, the per-Gaussian depth keys counted (8 B) and sorted
                     (passes x 24 B),
                     the packed rectangles and the (tile, Gaussian block) count
-                    table read and written once;
+                    table read and written once. Where the ranges come from
+                    the tile counts (plan count_ranges), the last pass writes
+                    ids only (8 B of keys less per pair in full-64 mode, 4 B
+                    on the column path), nothing reads the keys for the
+                    ranges, and the rectangles are read once more (16 B per
+                    Gaussian and view);
       raster fwd    4 B id + 40 B record per pair read + 20 B written per
                     pixel; the pairs read are the list entries the forward
                     examined (`examined`: a tile stops walking its list once
@@ -226,14 +232,17 @@ def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float,
     pbytes = (11 + 3 * sp.K) * 4
     plan = sort_plan(sp, sort_mode)
     pre, pair = plan["pre"], plan["pair"]
+    cr = plan["count_ranges"]
     if sort_mode == "full64":
-        sort_bytes = V * n * 24 + n_pairs * (12 + pair * 24 + 8 + 8)
+        sort_bytes = (V * n * (24 + (16 if cr else 0))
+                      + n_pairs * (12 + pair * 24 + 8 + (-8 if cr else 8)))
     elif plan["path"] == "tiles":
         table = plan["tiles"] * plan["bpv"] * 4
         sort_bytes = (n_pairs * 4 + V * n * (16 + 12 + 8 + pre * 24 + 12 + 16 + 16)
                       + 3 * table + plan["tiles"] * 24)
     else:
-        sort_bytes = n_pairs * (8 + pair * 16 + 4) + V * n * (16 + 8 + pre * 24 + 12)
+        sort_bytes = (n_pairs * (8 + pair * 16 + (-4 if cr else 4))
+                      + V * n * (16 + 8 + pre * 24 + 12 + (16 if cr else 0)))
     return {
         "gs_project": dict(bytes=n * pbytes + V * n * 48, exps=0.0),
         "gs_bin_sort": dict(bytes=sort_bytes, exps=0.0),
@@ -259,7 +268,9 @@ def launches_per_step(sp, sort_mode: str, kind: str = "train", fused: bool = Fal
     # the 64-bit sorts are single-sweep (a digit-count read + one kernel per
     # pass); the 32-bit row / tile passes are count, scan, scatter
     if sort_mode == "full64":
-        sort = 1 + 1 + pair + 1                 # emit, digit counts, passes, ranges
+        # emit, digit counts, passes, ranges (from the keys, or the tile-count
+        # histogram and its scan)
+        sort = 1 + 1 + pair + (2 if plan["count_ranges"] else 1)
     elif plan["path"] == "tiles":
         sort = 1 + 1 + pre + 4                  # keys, presort, count, scan, base, place
     else:
@@ -267,7 +278,9 @@ def launches_per_step(sp, sort_mode: str, kind: str = "train", fused: bool = Fal
         # single-sweep, count + scan + scatter each otherwise
         passes = (1 + pair) if plan["pair_sweep"] else 3 * pair
         if plan["path"] == "columns":
-            sort = 1 + 1 + pre + 3 + passes + 1   # ..., count, scan, emit, row passes, ranges
+            # ..., count, scan, emit, row passes, ranges (from the keys, or the
+            # tile-count histogram and its scan)
+            sort = 1 + 1 + pre + 3 + passes + (2 if plan["count_ranges"] else 1)
         else:
             sort = 1 + 1 + pre + 1 + passes + 1
     # project, sort, raster fwd (+ raster bwd, project bwd, densify (+ adam)),

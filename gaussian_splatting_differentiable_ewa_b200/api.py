@@ -423,7 +423,7 @@ GS_PATH_TILE_ID, GS_PATH_COLUMNS, GS_PATH_TILES = 0, 1, 2
 class GsSortPlan(_c.Structure):
     _fields_ = [("path", _c.c_int32), ("presort_passes", _c.c_int32),
                 ("pair_passes", _c.c_int32), ("gaussians_per_block", _c.c_int32),
-                ("pair_single_sweep", _c.c_int32), ("reserved", _c.c_int32),
+                ("pair_single_sweep", _c.c_int32), ("ranges_from_counts", _c.c_int32),
                 ("blocks_per_view", _c.c_int64)]
 
 

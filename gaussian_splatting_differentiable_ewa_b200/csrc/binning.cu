@@ -724,6 +724,155 @@ __global__ void __launch_bounds__(32) k_emit_cols(
                  __shfl_sync(0xffffffffu, fill, L), status);
   }
 }
+// (4) the ranges, from the tile counts instead of the sorted keys (grids
+// whose difference array fits a block's shared memory). The pairs end up
+// ordered by global tile, view-major and row-major within a view, so tile
+// t's slice starts after every pair of the views before it and of the tiles
+// before it in its view; a tile's pair count is the number of rectangles
+// covering it. The rows pass then needs no keys written: nothing reads them.
+
+// (4a) per view: a 2-D difference array of the rectangles' corners (+1 at
+// (y0, x0) and (y1 + 1, x1 + 1), -1 at (y0, x1 + 1) and (y1 + 1, x0)),
+// summed per block in shared memory and added into the view's array in
+// global memory, and the view's pair total. Grid (blocks per view, views):
+// block b takes a contiguous share of the view's rectangles -- its presorted
+// visible ones (kBins false, from the packed rectangles of the column
+// emission), or all n of its binning records (kBins true, full-64 mode).
+template <bool kBins>
+__global__ void __launch_bounds__(1024) k_tile_hist(const uint4* __restrict__ crect,
+                                                    const float4* __restrict__ bins, int n,
+                                                    const uint32_t* __restrict__ n_visible,
+                                                    Grid g, int* __restrict__ diff,
+                                                    unsigned long long* __restrict__ view_pairs) {
+  extern __shared__ int s_d[];  // [tiles_y + 1][tiles_x + 1]
+  __shared__ unsigned long long s_tot[32];
+  const int v = blockIdx.y;
+  const int W = g.tiles_x + 1, H = g.tiles_y + 1;
+  for (int k = threadIdx.x; k < W * H; k += blockDim.x) s_d[k] = 0;
+  __syncthreads();
+  int64_t vs, nv;
+  if (kBins) {
+    vs = (int64_t)v * n;
+    nv = n;
+  } else {
+    view_span(n_visible, v, vs, nv);
+  }
+  const int64_t share = (nv + gridDim.x - 1) / gridDim.x;
+  const int64_t first = vs + (int64_t)blockIdx.x * share;
+  const int64_t last = min(vs + nv, first + share);
+  uint64_t mine = 0;
+  for (int64_t i = first + threadIdx.x; i < last; i += blockDim.x) {
+    uint32_t rx, ry;
+    if (kBins) {
+      const float4 b = __ldg(&bins[i]);
+      rx = __float_as_uint(b.y);
+      ry = __float_as_uint(b.z);
+    } else {
+      const uint4 r = crect[i];
+      rx = r.x;
+      ry = r.y;
+    }
+    const int x0 = rx & 0xffffu, x1 = rx >> 16, y0 = ry & 0xffffu, y1 = ry >> 16;
+    if (x0 <= x1 && y0 <= y1) {
+      atomicAdd(&s_d[y0 * W + x0], 1);
+      atomicAdd(&s_d[y0 * W + x1 + 1], -1);
+      atomicAdd(&s_d[(y1 + 1) * W + x0], -1);
+      atomicAdd(&s_d[(y1 + 1) * W + x1 + 1], 1);
+      mine += (uint64_t)(x1 - x0 + 1) * (uint64_t)(y1 - y0 + 1);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
+  if ((threadIdx.x & 31) == 0) s_tot[threadIdx.x >> 5] = mine;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long t = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += s_tot[w];
+    if (t) atomicAdd(&view_pairs[v], t);
+  }
+  int* gd = diff + (int64_t)v * W * H;
+  for (int k = threadIdx.x; k < W * H; k += blockDim.x) {
+    const int x = s_d[k];
+    if (x) atomicAdd(&gd[k], x);
+  }
+}
+
+// (4b) per view (one block of 1024 threads each): the difference array summed
+// along rows then columns gives each tile's count; thread i takes a run of
+// consecutive tiles, a block scan of the runs' sums gives every tile's start
+// within the view, after the pairs of the views before it. Nothing is written
+// when the pairs of all views exceed the capacity (every range stays empty,
+// as zeroed).
+__global__ void __launch_bounds__(1024) k_tile_ranges(
+    const int* __restrict__ diff, const unsigned long long* __restrict__ view_pairs,
+    int n_views, Grid g, int64_t capacity, int64_t* __restrict__ ranges) {
+  extern __shared__ int s_d[];  // [tiles_y + 1][tiles_x + 1]
+  __shared__ uint32_t s_warp[33];
+  unsigned long long total = 0;
+  for (int u = 0; u < n_views; ++u) total += view_pairs[u];
+  if ((int64_t)total > capacity) return;
+  const int v = blockIdx.x;
+  const int W = g.tiles_x + 1, H = g.tiles_y + 1;
+  const int* gd = diff + (int64_t)v * W * H;
+  for (int k = threadIdx.x; k < W * H; k += blockDim.x) s_d[k] = gd[k];
+  __syncthreads();
+  for (int r = threadIdx.x; r < H - 1; r += blockDim.x) {
+    int acc = 0;
+    for (int c = 0; c < W - 1; ++c) {
+      acc += s_d[r * W + c];
+      s_d[r * W + c] = acc;
+    }
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < W - 1; c += blockDim.x) {
+    int acc = 0;
+    for (int r = 0; r < H - 1; ++r) {
+      acc += s_d[r * W + c];
+      s_d[r * W + c] = acc;
+    }
+  }
+  __syncthreads();
+  int64_t base = 0;
+  for (int u = 0; u < v; ++u) base += (int64_t)view_pairs[u];
+  const int tpv = g.tiles_per_view;
+  const int run = (tpv + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int t0 = (int)threadIdx.x * run;
+  // a view's pairs are at most the capacity (checked above): 32 bits hold them
+  uint32_t sum = 0;
+  for (int t = t0; t < min(t0 + run, tpv); ++t) {
+    const int r = t / g.tiles_x;
+    sum += (uint32_t)s_d[r * W + (t - r * g.tiles_x)];
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t w = lane < (int)(blockDim.x >> 5) ? s_warp[lane] : 0u;
+    uint32_t wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
+    }
+    s_warp[lane] = wi - w;
+  }
+  __syncthreads();
+  int64_t pos = base + (int64_t)(s_warp[warp] + incl - sum);
+  int64_t* rv = ranges + 2 * (int64_t)v * tpv;
+  for (int t = t0; t < min(t0 + run, tpv); ++t) {
+    const int r = t / g.tiles_x;
+    const int64_t c = s_d[r * W + (t - r * g.tiles_x)];
+    rv[2 * (int64_t)t] = pos;
+    rv[2 * (int64_t)t + 1] = pos + c;
+    pos += c;
+  }
+}
 
 // Fused pair count + scan + emission.
 // MODE 0 (full 64-bit keys): items are the n_views * n Gaussians in index
@@ -1009,7 +1158,8 @@ size_t scatter_smem_bytes() {
 // counts, block-local digit starts, ranking by ballots, staging in shared
 // memory in sorted order, then runs of equal digits written at their global
 // offsets. Keys past the end take the largest digit: they rank after every
-// real key of the partition and are never written.
+// real key of the partition and are never written. keys_out may be null (a
+// last pass whose keys nothing reads): then only the values are written.
 template <typename K, int BITS, int ITEMS>
 __global__ void __launch_bounds__(kSortThreads, (ScatterOcc<K, ITEMS>::kBlocks)) k_radix_scatter(
     const K* __restrict__ keys_in, const uint32_t* __restrict__ vals_in,
@@ -1096,7 +1246,7 @@ __global__ void __launch_bounds__(kSortThreads, (ScatterOcc<K, ITEMS>::kBlocks))
     const K k = s_keys[j];
     const uint32_t gpos = j + s_delta[(uint32_t)(k >> shift) & M];
     if (gpos < n) {
-      keys_out[gpos] = k;
+      if (keys_out) keys_out[gpos] = k;
       vals_out[gpos] = s_vals[j];
     } else {
       atomicOr(status, kStatusBounds);
@@ -1308,7 +1458,7 @@ __global__ void __launch_bounds__(kSortThreads, (ScatterOcc<K, ITEMS>::kBlocks))
     const K k = s_keys[j];
     const uint32_t gpos = j + s_delta[(uint32_t)(k >> shift) & M];
     if (gpos < n) {
-      keys_out[gpos] = k;
+      if (keys_out) keys_out[gpos] = k;
       vals_out[gpos] = s_vals[j];
     } else {
       atomicOr(status, kStatusBounds);
@@ -1407,11 +1557,13 @@ cudaError_t radix_pass(const K* kin, const uint32_t* vin, K* kout, uint32_t* vou
 
 // The plan's passes, ping-ponging between (keys_a, vals_a) and (keys_b,
 // vals_b); grids sized for `max_items`, the device count read from n_ptr.
+// last_keys false: the last pass writes the values only.
 template <typename K, int ITEMS>
 cudaError_t run_radix_passes(K* keys_a, uint32_t* vals_a, K* keys_b, uint32_t* vals_b,
                              const int64_t* n_ptr, int64_t capacity, int64_t max_items,
                              const RadixPlan& plan, uint32_t* counts, int64_t stride,
-                             uint32_t* totals, uint32_t* status, cudaStream_t stream) {
+                             uint32_t* totals, uint32_t* status, cudaStream_t stream,
+                             bool last_keys = true) {
   const int64_t parts = (max_items + SortTile<ITEMS>::kItems - 1) / SortTile<ITEMS>::kItems;
   if (parts == 0) return cudaSuccess;
   K* kin = keys_a;
@@ -1420,19 +1572,20 @@ cudaError_t run_radix_passes(K* keys_a, uint32_t* vals_a, K* keys_b, uint32_t* v
   uint32_t* vout = vals_b;
   for (int p = 0; p < plan.passes; ++p) {
     const int sh = plan.shift[p];
+    K* kout_p = (p + 1 == plan.passes && !last_keys) ? nullptr : kout;
     cudaError_t e = cudaErrorInvalidValue;
     if constexpr (sizeof(K) == 4) {
       switch (plan.bits[p]) {
-        case 4: e = radix_pass<K, 4, ITEMS>(kin, vin, kout, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream); break;
-        case 5: e = radix_pass<K, 5, ITEMS>(kin, vin, kout, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream); break;
-        case 6: e = radix_pass<K, 6, ITEMS>(kin, vin, kout, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream); break;
-        case 7: e = radix_pass<K, 7, ITEMS>(kin, vin, kout, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream); break;
-        case 8: e = radix_pass<K, 8, ITEMS>(kin, vin, kout, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream); break;
+        case 4: e = radix_pass<K, 4, ITEMS>(kin, vin, kout_p, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream); break;
+        case 5: e = radix_pass<K, 5, ITEMS>(kin, vin, kout_p, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream); break;
+        case 6: e = radix_pass<K, 6, ITEMS>(kin, vin, kout_p, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream); break;
+        case 7: e = radix_pass<K, 7, ITEMS>(kin, vin, kout_p, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream); break;
+        case 8: e = radix_pass<K, 8, ITEMS>(kin, vin, kout_p, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream); break;
         default: break;
       }
     } else {
       if (plan.bits[p] == 8)
-        e = radix_pass<K, 8, ITEMS>(kin, vin, kout, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream);
+        e = radix_pass<K, 8, ITEMS>(kin, vin, kout_p, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream);
     }
     if (e != cudaSuccess) return e;
     K* tk = kin; kin = kout; kout = tk;
@@ -1450,7 +1603,7 @@ cudaError_t run_onesweep_passes(K* keys_a, uint32_t* vals_a, K* keys_b, uint32_t
                                 const int64_t* n_ptr, int64_t capacity, int64_t max_items,
                                 const RadixPlan& plan, uint32_t* hist, uint64_t* lookback,
                                 uint32_t* tickets, const WaitCfg& wc, uint32_t* status,
-                                int sms, cudaStream_t stream) {
+                                int sms, cudaStream_t stream, bool last_keys = true) {
   const int64_t parts = (max_items + SortTile<ITEMS>::kItems - 1) / SortTile<ITEMS>::kItems;
   if (parts == 0) return cudaSuccess;
   for (int q = 0; q < plan.passes; ++q)
@@ -1468,8 +1621,8 @@ cudaError_t run_onesweep_passes(K* keys_a, uint32_t* vals_a, K* keys_b, uint32_t
   uint32_t* vout = vals_b;
   for (int q = 0; q < plan.passes; ++q) {
     k_onesweep<K, ITEMS><<<(unsigned)parts, kSortThreads, smem, stream>>>(
-        kin, vin, kout, vout, n_ptr, capacity, plan.shift[q], q, hist + 256 * q, lookback,
-        tickets + q, wc, status);
+        kin, vin, (q + 1 == plan.passes && !last_keys) ? nullptr : kout, vout, n_ptr, capacity,
+        plan.shift[q], q, hist + 256 * q, lookback, tickets + q, wc, status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     K* tk = kin; kin = kout; kout = tk;
     uint32_t* tv = vin; vin = vout; vout = tv;
@@ -1519,6 +1672,9 @@ bool column_emission(const Grid& g) { return g.tiles_x <= kMaxColumns; }
 // block 72 regions to scan, and the emission by column (then one radix pass
 // over the rows) measured 1.7x faster there (12.0 against 20.5 ms for 849M
 // pairs).
+bool count_ranges_fit(const Grid& g) {
+  return (int64_t)(g.tiles_x + 1) * (g.tiles_y + 1) * (int64_t)sizeof(int) <= kTileDiffBytes;
+}
 bool tile_emission(const Grid& g) {
   return g.tiles_per_view <= 16384 &&
          (int64_t)(g.tiles_x + 1) * (g.tiles_y + 1) * (int64_t)sizeof(int) <= kTileDiffBytes;
@@ -1542,7 +1698,8 @@ cudaError_t sort_pairs32(const BinSortArgs& a, cudaStream_t stream) {
   return run_radix_passes<uint32_t, kSortItems>(
       reinterpret_cast<uint32_t*>(a.keys[a.emit_buf]), a.vals[a.emit_buf],
       reinterpret_cast<uint32_t*>(a.keys[a.emit_buf ^ 1]), a.vals[a.emit_buf ^ 1], a.n_pairs,
-      a.capacity, a.capacity, a.pairs, a.counts, a.counts_stride, a.totals, a.status, stream);
+      a.capacity, a.capacity, a.pairs, a.counts, a.counts_stride, a.totals, a.status, stream,
+      !a.count_ranges);
 }
 
 cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
@@ -1602,6 +1759,23 @@ cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
       k_col_count<<<(unsigned)cb, kColItems, 0, stream>>>(bins4, a.pkeys[fin], a.pvals[fin], a.n,
                                                           a.n_views, a.grid, a.counts,
                                                           a.counts_stride, a.pair_total, a.crect);
+      if (a.count_ranges) {
+        // the ranges from the tile counts, before the pairs exist
+        const Grid& g = a.grid;
+        const size_t dsmem = (size_t)(g.tiles_x + 1) * (g.tiles_y + 1) * sizeof(int);
+        if ((e = cudaFuncSetAttribute(k_tile_hist<false>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsmem)) !=
+                cudaSuccess ||
+            (e = cudaFuncSetAttribute(k_tile_ranges, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)dsmem)) != cudaSuccess)
+          return e;
+        // about one 1024-thread block per SM over all views
+        const int bpv = sms / a.n_views > 0 ? sms / a.n_views : 1;
+        k_tile_hist<false><<<dim3((unsigned)bpv, (unsigned)a.n_views), 1024, dsmem, stream>>>(
+            a.crect, nullptr, a.n, a.n_visible, g, a.tile_diff, a.view_pairs);
+        k_tile_ranges<<<(unsigned)a.n_views, 1024, dsmem, stream>>>(
+            a.tile_diff, a.view_pairs, a.n_views, g, a.capacity, a.ranges);
+      }
       k_radix_scan<<<(unsigned)a.grid.tiles_x, 256, 0, stream>>>(
           a.counts, a.counts_stride, a.n_items_dev, n_items, kColItems, a.totals);
       const dim3 grid((unsigned)cb, (unsigned)((a.grid.tiles_x + 31) / 32));
@@ -1613,6 +1787,7 @@ cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
       // 3) stable sort by row
       e = sort_pairs32(a, stream);
       if (e != cudaSuccess) return e;
+      if (a.count_ranges) return cudaSuccess;
       const int out = a.emit_buf ^ (a.pairs.passes & 1);
       k_ranges<uint32_t><<<sms * 4, 256, 0, stream>>>(
           reinterpret_cast<uint32_t*>(a.keys[out]), a.n_pairs, a.capacity, a.n_tiles, a.cbits,
@@ -1639,12 +1814,31 @@ cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
       bins4, nullptr, nullptr, a.n, a.n_views, a.grid, a.keys[a.emit_buf], a.vals[a.emit_buf],
       a.capacity, a.n_pairs, a.emit_lookback, a.counters + 0, a.status, a.wait);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (a.count_ranges) {
+    // the ranges from the tile counts of the binning records; the last pass
+    // then writes no keys
+    const Grid& g = a.grid;
+    const size_t dsmem = (size_t)(g.tiles_x + 1) * (g.tiles_y + 1) * sizeof(int);
+    if ((e = cudaFuncSetAttribute(k_tile_hist<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)dsmem)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(k_tile_ranges, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)dsmem)) != cudaSuccess)
+      return e;
+    const int bpv = sms / a.n_views > 0 ? sms / a.n_views : 1;
+    k_tile_hist<true><<<dim3((unsigned)bpv, (unsigned)a.n_views), 1024, dsmem, stream>>>(
+        nullptr, bins4, a.n, nullptr, g, a.tile_diff, a.view_pairs);
+    k_tile_ranges<<<(unsigned)a.n_views, 1024, dsmem, stream>>>(
+        a.tile_diff, a.view_pairs, a.n_views, g, a.capacity, a.ranges);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   e = run_onesweep_passes<uint64_t, kSortItems>(a.keys[a.emit_buf], a.vals[a.emit_buf],
                                                 a.keys[a.emit_buf ^ 1], a.vals[a.emit_buf ^ 1],
                                                 a.n_pairs, a.capacity, a.capacity, a.pairs,
                                                 a.digit_hist, a.sweep_lookback, a.counters + 1,
-                                                a.sort_wait, a.status, sms, stream);
+                                                a.sort_wait, a.status, sms, stream,
+                                                !a.count_ranges);
   if (e != cudaSuccess) return e;
+  if (a.count_ranges) return cudaSuccess;
   const int out = a.emit_buf ^ (a.pairs.passes & 1);
   k_ranges<uint64_t><<<sms * 4, 256, 0, stream>>>(a.keys[out], a.n_pairs, a.capacity, a.n_tiles,
                                                   0, 0u, a.ranges, a.status);

@@ -42,14 +42,15 @@ struct Layout {
   bool tile_emit = false;
   int gsize = 0, tile_bpv = 0;
   bool column_emit = false;
+  bool count_ranges = false;
   int cbits = 0;
   int key_bytes = 8;
   int64_t counts_stride = 0;
   size_t off_hist = 0, off_emit_lb = 0, off_counts = 0, off_keys0 = 0, off_keys1 = 0,
          off_vals1 = 0, off_pkeys0 = 0, off_pkeys1 = 0, off_pvals0 = 0, off_pvals1 = 0,
          off_crect = 0, off_tile_totals = 0, off_tile_base = 0, off_digit_hist = 0,
-         off_sweep_lb = 0;
-  size_t sweep_lb_bytes = 0;
+         off_sweep_lb = 0, off_tdiff = 0, off_view_pairs = 0;
+  size_t sweep_lb_bytes = 0, tdiff_bytes = 0;
   size_t total = 0;
 };
 
@@ -78,6 +79,7 @@ bool make_layout(int64_t n, int32_t n_views, const gs_camera* cams, int64_t capa
   if (mode == GS_SORT_FULL64) {
     L.key_bytes = 8;
     L.pairs = make_radix_plan(32 + tile_bits, false);
+    L.count_ranges = count_ranges_fit(g);
   } else {
     L.key_bytes = 4;
     L.presort = make_radix_plan(32 + bits_for((uint64_t)n_views - 1), false);
@@ -90,6 +92,7 @@ bool make_layout(int64_t n, int32_t n_views, const gs_camera* cams, int64_t capa
       // keys row << cbits | column; the radix passes sort the row bits
       L.cbits = bits_for((uint64_t)g.tiles_x - 1);
       if (L.cbits == 0) L.cbits = 1;
+      L.count_ranges = count_ranges_fit(g);
       L.pairs = make_radix_plan(bits_for((uint64_t)g.tiles_y * n_views - 1), true);
       for (int i = 0; i < L.pairs.passes; ++i) L.pairs.shift[i] += L.cbits;
     } else {
@@ -138,6 +141,12 @@ bool make_layout(int64_t n, int32_t n_views, const gs_camera* cams, int64_t capa
       L.off_tile_totals = off; off = align_up(off + (size_t)tiles * 4);
       L.off_tile_base = off; off = align_up(off + (size_t)tiles * 4);
     }
+  }
+  if (L.count_ranges) {
+    // per view: the tile-count difference array, and the view's pair total
+    L.tdiff_bytes = (size_t)n_views * (g.tiles_x + 1) * (g.tiles_y + 1) * sizeof(int);
+    L.off_tdiff = off; off = align_up(off + L.tdiff_bytes);
+    L.off_view_pairs = off; off = align_up(off + GS_MAX_VIEWS * sizeof(uint64_t));
   }
   L.total = off;
   return true;
@@ -264,6 +273,11 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
       (L.sweep_lb_bytes &&
        cudaMemsetAsync(w + L.off_sweep_lb, 0, L.sweep_lb_bytes, st) != cudaSuccess))
     return GS_ERR_CUDA;
+  if (L.count_ranges &&
+      (cudaMemsetAsync(w + L.off_tdiff, 0, L.tdiff_bytes, st) != cudaSuccess ||
+       cudaMemsetAsync(w + L.off_view_pairs, 0, GS_MAX_VIEWS * sizeof(uint64_t), st) !=
+           cudaSuccess))
+    return GS_ERR_CUDA;
 
   BinSortArgs a{};
   a.bins = proj->bins;
@@ -277,6 +291,11 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
   a.tile_bpv = L.tile_bpv;
   a.column_emit = L.column_emit;
   a.cbits = L.cbits;
+  a.count_ranges = L.count_ranges;
+  if (L.count_ranges) {
+    a.tile_diff = reinterpret_cast<int*>(w + L.off_tdiff);
+    a.view_pairs = reinterpret_cast<unsigned long long*>(w + L.off_view_pairs);
+  }
   a.pairs = L.pairs;
   a.presort = L.presort;
   a.emit_buf = L.pairs.passes & 1;
@@ -709,7 +728,7 @@ gs_status gs_bin_sort_plan(int64_t n, int32_t n_views, const gs_camera* cams,
   plan->pair_passes = L.tile_emit ? 0 : L.pairs.passes;
   plan->gaussians_per_block = L.tile_emit ? L.gsize : 0;
   plan->pair_single_sweep = pair_passes_single_sweep(L.pairs, sort_mode) ? 1 : 0;
-  plan->reserved = 0;
+  plan->ranges_from_counts = L.count_ranges ? 1 : 0;
   plan->blocks_per_view = L.tile_emit ? L.tile_bpv : 0;
   return GS_OK;
 }

@@ -61,6 +61,9 @@ struct BinSortArgs {
   uint32_t* tile_totals;             // tile emission: pairs per tile [n_tiles]
   uint32_t* tile_base;               // tile emission: first position of each tile [n_tiles]
   int64_t* scan_n;                   // tile emission: blocks per view, for the scan
+  bool count_ranges;                 // column emission: ranges from the tile counts
+  int* tile_diff;                    // count_ranges: [n_views][tiles_y + 1][tiles_x + 1]
+  unsigned long long* view_pairs;    // count_ranges: pairs per view [GS_MAX_VIEWS]
   int64_t* ranges;
   int64_t n_tiles;     // n_views * tiles per view
 };
@@ -139,6 +142,7 @@ int64_t presort_partitions(int64_t items);  // radix partitions over depth keys
 int64_t column_blocks(int64_t items);       // column-emission blocks
 bool column_emission(const Grid& g);        // presort mode emits by column on this grid
 bool tile_emission(const Grid& g);          // presort mode places pairs directly on this grid
+bool count_ranges_fit(const Grid& g);       // a view's tile-count difference array fits a block
 int tile_gsize(int64_t n);                  // tile emission: Gaussians per block
 int64_t emit_blocks(int64_t items);
 

@@ -224,6 +224,12 @@ size_t gs_workspace_size(int64_t n, int32_t n_views, const gs_camera* cams,
  *                    kernel, then one kernel per pass: the 64-bit keys of
  *                    full-64 mode), 0 if reduce-then-scan (three kernels per
  *                    pass: the 32-bit keys of the other paths);
+ *   ranges_from_counts  1 if the tile ranges come from per-tile pair counts
+ *                    (a difference array of the rectangles' corners per
+ *                    view, two kernels) rather than from a read of the
+ *                    sorted keys, whose last pass then writes no keys:
+ *                    GS_PATH_COLUMNS and full-64 mode on grids whose
+ *                    (tiles_x + 1) (tiles_y + 1) counters fit 160 KiB;
  *   gaussians_per_block, blocks_per_view  the Gaussian blocks of
  *                    GS_PATH_TILES (0 otherwise).
  * Returns GS_ERR_INVALID_ARG for a request gs_workspace_size rejects. */
@@ -234,7 +240,7 @@ typedef struct gs_sort_plan {
   int32_t pair_passes;
   int32_t gaussians_per_block;
   int32_t pair_single_sweep;
-  int32_t reserved;
+  int32_t ranges_from_counts;
   int64_t blocks_per_view;
 } gs_sort_plan;
 gs_status gs_bin_sort_plan(int64_t n, int32_t n_views, const gs_camera* cams,

@@ -219,12 +219,14 @@ def test_sort_plan_follows_the_grid_and_mode():
     p = plan(3840, 2160, 10_000_000, 1, api.GS_SORT_PRESORT)      # 4K: 240 x 135 tiles
     assert (p.path, p.pair_passes) == (api.GS_PATH_COLUMNS, 1)
     assert p.pair_single_sweep == 0                                 # 32-bit row keys
+    assert p.ranges_from_counts == 1                                # 241 x 136 ints fit
     p = plan(128, 128, 1000, 1, api.GS_SORT_PRESORT)               # small scene: 32 per block
     assert (p.path, p.gaussians_per_block, p.blocks_per_view) == (api.GS_PATH_TILES, 32, 32)
     p = plan(800, 800, 100_000, 1, api.GS_SORT_PRESORT)
     assert (p.gaussians_per_block, p.blocks_per_view) == (160, 625)
     p = plan(4096, 2576, 1000, 1, api.GS_SORT_PRESORT)            # 256 x 161 tiles
     assert (p.path, p.pair_passes) == (api.GS_PATH_COLUMNS, 1)
+    assert p.ranges_from_counts == 0                                # 257 x 162 ints do not
     p = plan(8192, 1296, 1000, 1, api.GS_SORT_PRESORT)            # 512 x 81 tiles
     assert (p.path, p.pair_passes) == (api.GS_PATH_TILE_ID, 2)
     assert p.pair_single_sweep == 0
@@ -234,7 +236,9 @@ def test_sort_plan_follows_the_grid_and_mode():
     assert p.presort_passes == 5
     p = plan(1920, 1080, 1000, 1, api.GS_SORT_FULL64)             # 13 tile bits + 32
     assert (p.path, p.presort_passes, p.pair_passes) == (api.GS_PATH_TILE_ID, 0, 6)
-    assert p.pair_single_sweep == 1
+    assert p.pair_single_sweep == 1 and p.ranges_from_counts == 1
+    p = plan(8192, 1296, 1000, 1, api.GS_SORT_FULL64)             # 513 x 82 counters: too many
+    assert p.ranges_from_counts == 0
     with pytest.raises(api.GsError):
         plan(1920, 1080, -1, 1, api.GS_SORT_PRESORT)
 
@@ -245,15 +249,24 @@ def test_bench_work_model_uses_the_library_plan():
     cams = api.cameras(S.make_scene("train_1m_1080p", n=10).cameras)
     sp = types.SimpleNamespace(n=1_000_000, V=1, W=1920, H=1080, cams=cams)
     plan = bench.sort_plan(sp, "presort")
-    assert plan == dict(path="tiles", pre=4, pair=0, bpv=1303, tiles=8160, pair_sweep=False)
+    assert plan == dict(path="tiles", pre=4, pair=0, bpv=1303, tiles=8160, pair_sweep=False,
+                        count_ranges=False)
     # project; depth keys, digit counts, 4 single-sweep passes, count, scan, base,
     # place; raster fwd, raster bwd, project bwd, densify stats, Adam
     assert bench.launches_per_step(sp, "presort") == 1 + (1 + 1 + 4 + 4) + 5
     assert bench.sort_plan(sp, "full64")["pair"] == 6
-    # emit, digit counts, 6 passes, ranges
-    assert bench.launches_per_step(sp, "full64") == 1 + (1 + 1 + 6 + 1) + 5
+    # emit, digit counts, 6 passes, tile histogram, ranges from it
+    assert bench.sort_plan(sp, "full64")["count_ranges"]
+    assert bench.launches_per_step(sp, "full64") == 1 + (1 + 1 + 6 + 2) + 5
     # the fused tail: raster fwd, raster bwd, projection backward + statistics + Adam
     assert bench.launches_per_step(sp, "presort", fused=True) == 1 + (1 + 1 + 4 + 4) + 3
+    # a 4K view: depth keys, digit counts, 4 passes, column count, tile histogram,
+    # ranges from it, column scan, emission, one row pass (count, scan, scatter)
+    sp4 = types.SimpleNamespace(n=10_000_000, V=1, W=3840, H=2160,
+                                cams=api.cameras(S.make_scene("train_10m_4k", n=10).cameras))
+    assert bench.sort_plan(sp4, "presort")["count_ranges"]
+    assert bench.launches_per_step(sp4, "presort", fused=True) == \
+        1 + (1 + 1 + 4 + 1 + 2 + 2 + 3) + 3
     # blend kernels: bytes on the examined entries, FP32 operations on the
     # evaluations and the contributing pixels
     sp.K = 16
