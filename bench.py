@@ -168,7 +168,7 @@ def sort_plan(sp, sort_mode: str) -> dict:
             api.GS_PATH_TILE_ID: "tile_id"}[p.path]
     return dict(path=path, pre=p.presort_passes, pair=p.pair_passes, bpv=p.blocks_per_view,
                 tiles=tiles, pair_sweep=bool(p.pair_single_sweep),
-                count_ranges=bool(p.ranges_from_counts))
+                count_ranges=bool(p.ranges_from_counts), key_bytes=int(p.pair_key_bytes))
 
 
 # FP32 operations of the blend kernels (an FMA is one operation): per (pixel,
@@ -198,12 +198,14 @@ def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float,
                     once, the per-Gaussian depth keys counted (8 B) and sorted
                     (passes x 24 B),
                     the packed rectangles and the (tile, Gaussian block) count
-                    table read and written once. Where the ranges come from
-                    the tile counts (plan count_ranges), the last pass writes
-                    ids only (8 B of keys less per pair in full-64 mode, 4 B
-                    on the column path), nothing reads the keys for the
-                    ranges, and the rectangles are read once more (16 B per
-                    Gaussian and view);
+                    table read and written once; the column path emits
+                    key + id per pair and each rows pass reads and writes
+                    them, with keys of the plan's width (4 B, or the row
+                    alone in 1 or 2 B). Where the ranges come from the tile
+                    counts (plan count_ranges), the last pass writes ids only
+                    and nothing reads the keys for the ranges (a key's bytes
+                    less twice per pair), and the rectangles are read once
+                    more (16 B per Gaussian and view);
       raster fwd    4 B id + 40 B record per pair read + 20 B written per
                     pixel; the pairs read are the list entries the forward
                     examined (`examined`: a tile stops walking its list once
@@ -241,7 +243,8 @@ def algorithmic_work(sp, n_pairs: int, sort_mode: str, exps: float,
         sort_bytes = (n_pairs * 4 + V * n * (16 + 12 + 8 + pre * 24 + 12 + 16 + 16)
                       + 3 * table + plan["tiles"] * 24)
     else:
-        sort_bytes = (n_pairs * (8 + pair * 16 + (-4 if cr else 4))
+        kb = plan["key_bytes"]
+        sort_bytes = (n_pairs * ((kb + 4) + pair * 2 * (kb + 4) + (-kb if cr else kb))
                       + V * n * (16 + 8 + pre * 24 + 12 + (16 if cr else 0)))
     return {
         "gs_project": dict(bytes=n * pbytes + V * n * 48, exps=0.0),

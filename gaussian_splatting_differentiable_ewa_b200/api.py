@@ -424,7 +424,8 @@ class GsSortPlan(_c.Structure):
     _fields_ = [("path", _c.c_int32), ("presort_passes", _c.c_int32),
                 ("pair_passes", _c.c_int32), ("gaussians_per_block", _c.c_int32),
                 ("pair_single_sweep", _c.c_int32), ("ranges_from_counts", _c.c_int32),
-                ("blocks_per_view", _c.c_int64)]
+                ("blocks_per_view", _c.c_int64), ("pair_key_bytes", _c.c_int32),
+                ("reserved", _c.c_int32)]
 
 
 def gs_bin_sort_plan(n: int, cams_arr, n_views: int, sort_mode: int) -> GsSortPlan:

@@ -66,6 +66,7 @@ constexpr int kSortTile = kSortThreads * kSortItems;  // keys per partition
 constexpr int kPresortItems = 16;                     // per-Gaussian depth passes
 constexpr int kColItems = 256;     // Gaussians per column-emission block
 constexpr int kColBuf = 32;        // pairs a column stages before a warp-wide write
+constexpr int kColStage = 128;     // rectangles a column-emission warp compacts at a time
 constexpr int kMaxColumns = 256;   // widest tile grid the column emission takes
 constexpr int kColPitch = 33;      // buffer row: conflict-free along and across columns
 constexpr int kRegionCols = 32;    // tile-emission region: kRegionCols x kRegionRows tiles
@@ -602,9 +603,10 @@ __global__ void __launch_bounds__(kColItems) k_col_count(
 
 // Warp-wide write of the first `count` (<= 32) pairs of buffer column `bc`
 // to global positions base, base + 1, ...
-__device__ __forceinline__ void flush_column(uint32_t* __restrict__ keys_out,
+template <typename KT>
+__device__ __forceinline__ void flush_column(KT* __restrict__ keys_out,
                                              uint32_t* __restrict__ ids_out, int64_t capacity,
-                                             const uint32_t* s_bk, const uint32_t* s_bi, int bc,
+                                             const KT* s_bk, const uint32_t* s_bi, int bc,
                                              uint32_t base, uint32_t count,
                                              uint32_t* __restrict__ status) {
   const uint32_t lane = threadIdx.x & 31;
@@ -619,14 +621,21 @@ __device__ __forceinline__ void flush_column(uint32_t* __restrict__ keys_out,
   }
 }
 
+// KT: the key type. 32 bits: row << cbits | column (the ranges are then read
+// off the sorted keys); 8 or 16 bits: the row alone, when the ranges come
+// from the tile counts and only the rows pass reads the keys.
+template <typename KT>
 __global__ void __launch_bounds__(32) k_emit_cols(
     const uint4* __restrict__ crect, int64_t items, Grid g, int cbits,
     const uint32_t* __restrict__ offsets, int64_t stride, const uint32_t* __restrict__ totals,
-    const unsigned long long* __restrict__ pair_total, uint32_t* __restrict__ keys_out,
+    const unsigned long long* __restrict__ pair_total, KT* __restrict__ keys_out,
     uint32_t* __restrict__ ids_out, int64_t capacity, int64_t* __restrict__ n_pairs,
     uint32_t* __restrict__ status) {
-  __shared__ uint32_t s_bk[kColBuf * kColPitch], s_bi[kColBuf * kColPitch];
-  __shared__ uint4 s_rect[kColItems];  // this warp's rectangles, compacted
+  // keys buffered at their own width: narrow keys leave room for more blocks
+  // per SM (one-byte keys: 9.4 KB a block against 12.5 KB)
+  __shared__ KT s_bk[kColBuf * kColPitch];
+  __shared__ uint32_t s_bi[kColBuf * kColPitch];
+  __shared__ uint4 s_rect[kColStage];  // this warp's rectangles, compacted
   const int lane = threadIdx.x;
   const unsigned long long total = *pair_total;
   if (blockIdx.x == 0 && blockIdx.y == 0 && lane == 0) {
@@ -650,68 +659,76 @@ __global__ void __launch_bounds__(32) k_emit_cols(
   }
   uint32_t gofs = below + incl - tot_c;
   if (col < (uint32_t)g.tiles_x) gofs += offsets[(int64_t)col * stride + blockIdx.x];
-  // compact the block's rectangles that reach columns wlo .. wlo + 31
   const uint32_t lt = lanemask_lt();
-  int cnt = 0;
   const int64_t first = (int64_t)blockIdx.x * kColItems;
-#pragma unroll 2
-  for (int c = 0; c < kColItems / 32; ++c) {
-    const int64_t item = first + c * 32 + lane;
-    uint4 r = make_uint4(1u, 0u, 0u, 0u);
-    if (item < items) r = crect[item];
-    const uint32_t x0 = r.x & 0xffffu, x1 = r.x >> 16;
-    const bool hit = x0 <= x1 && x1 >= wlo && x0 <= wlo + 31u;
-    const uint32_t bal = __ballot_sync(0xffffffffu, hit);
-    if (hit) s_rect[cnt + __popc(bal & lt)] = r;
-    cnt += __popc(bal);
-  }
-  __syncwarp();
   uint32_t fill = 0;
-  for (int k = 0; k < cnt; ++k) {
-    const uint4 r = s_rect[k];
-    // this warp's columns of the rectangle
-    const uint32_t cx0 = max(r.x & 0xffffu, wlo);
-    const uint32_t cx1 = min(r.x >> 16, wlo + 31u);
-    const uint32_t wp = cx1 - cx0 + 1;
-    const float inv_wp = 1.f / (float)wp;
-    const bool owner = col >= cx0 && col <= cx1;
-    const uint32_t y0 = r.y & 0xffffu, h = (r.y >> 16) - y0 + 1;
-    const uint32_t row0 = r.z + y0;
-    for (uint32_t r0 = 0; r0 < h; r0 += kColBuf) {  // row chunks, uniform across the warp
-      const uint32_t hc = min(h - r0, (uint32_t)kColBuf);
-      // make room: columns that cannot take hc more pairs are written out
-      uint32_t need = __ballot_sync(0xffffffffu, owner && fill + hc > kColBuf);
-      if (need) {
-        __syncwarp();
-        do {
-          const int L = __ffs(need) - 1;
-          need &= need - 1;
-          flush_column(keys_out, ids_out, capacity, s_bk, s_bi, L,
-                       __shfl_sync(0xffffffffu, gofs, L), __shfl_sync(0xffffffffu, fill, L),
-                       status);
-          if (lane == L) {
-            gofs += fill;
-            fill = 0;
-          }
-        } while (need);
-        __syncwarp();
-      }
-      // the chunk's wp * hc pairs, 32 at a time: pair p is row p / wp, column
-      // cx0 + p % wp, written after that column's fill pairs
-      const uint32_t np = wp * hc;
-      for (uint32_t p0 = 0; p0 < np; p0 += 32) {
-        const uint32_t p = p0 + (uint32_t)lane;
-        const uint32_t rr = min((uint32_t)(((float)p + 0.5f) * inv_wp), hc - 1);
-        const uint32_t cc = min(p - rr * wp, wp - 1);
-        const uint32_t bc = cx0 + cc - wlo;  // buffer column = owning lane
-        const uint32_t f = __shfl_sync(0xffffffffu, fill, (int)bc);
-        if (p < np) {
-          const int at = (int)(f + rr) * kColPitch + (int)bc;
-          s_bk[at] = ((row0 + r0 + rr) << cbits) | (wlo + bc);
-          s_bi[at] = r.w;
+  // the block's rectangles kColStage at a time (a smaller staging buffer, more
+  // blocks per SM): compact those that reach columns wlo .. wlo + 31, in
+  // depth order, then place their pairs
+  for (int stage = 0; stage < kColItems; stage += kColStage) {
+    int cnt = 0;
+    __syncwarp();  // the previous stage's rectangles are read
+#pragma unroll 2
+    for (int c = 0; c < kColStage / 32; ++c) {
+      const int64_t item = first + stage + c * 32 + lane;
+      uint4 r = make_uint4(1u, 0u, 0u, 0u);
+      if (item < items) r = crect[item];
+      const uint32_t x0 = r.x & 0xffffu, x1 = r.x >> 16;
+      const bool hit = x0 <= x1 && x1 >= wlo && x0 <= wlo + 31u;
+      const uint32_t bal = __ballot_sync(0xffffffffu, hit);
+      if (hit) s_rect[cnt + __popc(bal & lt)] = r;
+      cnt += __popc(bal);
+    }
+    __syncwarp();
+    for (int k = 0; k < cnt; ++k) {
+      const uint4 r = s_rect[k];
+      // this warp's columns of the rectangle
+      const uint32_t cx0 = max(r.x & 0xffffu, wlo);
+      const uint32_t cx1 = min(r.x >> 16, wlo + 31u);
+      const uint32_t wp = cx1 - cx0 + 1;
+      const float inv_wp = 1.f / (float)wp;
+      const bool owner = col >= cx0 && col <= cx1;
+      const uint32_t y0 = r.y & 0xffffu, h = (r.y >> 16) - y0 + 1;
+      const uint32_t row0 = r.z + y0;
+      for (uint32_t r0 = 0; r0 < h; r0 += kColBuf) {  // row chunks, uniform across the warp
+        const uint32_t hc = min(h - r0, (uint32_t)kColBuf);
+        // make room: columns that cannot take hc more pairs are written out
+        uint32_t need = __ballot_sync(0xffffffffu, owner && fill + hc > kColBuf);
+        if (need) {
+          __syncwarp();
+          do {
+            const int L = __ffs(need) - 1;
+            need &= need - 1;
+            flush_column(keys_out, ids_out, capacity, s_bk, s_bi, L,
+                         __shfl_sync(0xffffffffu, gofs, L), __shfl_sync(0xffffffffu, fill, L),
+                         status);
+            if (lane == L) {
+              gofs += fill;
+              fill = 0;
+            }
+          } while (need);
+          __syncwarp();
         }
+        // the chunk's wp * hc pairs, 32 at a time: pair p is row p / wp, column
+        // cx0 + p % wp, written after that column's fill pairs
+        const uint32_t np = wp * hc;
+        for (uint32_t p0 = 0; p0 < np; p0 += 32) {
+          const uint32_t p = p0 + (uint32_t)lane;
+          const uint32_t rr = min((uint32_t)(((float)p + 0.5f) * inv_wp), hc - 1);
+          const uint32_t cc = min(p - rr * wp, wp - 1);
+          const uint32_t bc = cx0 + cc - wlo;  // buffer column = owning lane
+          const uint32_t f = __shfl_sync(0xffffffffu, fill, (int)bc);
+          if (p < np) {
+            const int at = (int)(f + rr) * kColPitch + (int)bc;
+            if constexpr (sizeof(KT) == 4)
+              s_bk[at] = ((row0 + r0 + rr) << cbits) | (wlo + bc);
+            else
+              s_bk[at] = (KT)(row0 + r0 + rr);
+            s_bi[at] = r.w;
+          }
+        }
+        if (owner) fill += hc;
       }
-      if (owner) fill += hc;
     }
   }
   // what is left in each column's buffer
@@ -1056,20 +1073,28 @@ __global__ void __launch_bounds__(kSortThreads) k_radix_count(
   const uint32_t n = (uint32_t)n64;
   const uint32_t p = blockIdx.x;
   if (p * (uint32_t)TILE >= n) return;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5;
   for (int k = tid; k < kSortWarps * R; k += kSortThreads) (&s_h[0][0])[k] = 0u;
-  const uint32_t first = p * (uint32_t)TILE + (uint32_t)warp * (ITEMS * 32) + lane;
+  // a histogram needs no order: each thread takes ITEMS consecutive keys,
+  // with 16-byte loads when they are all there
+  static_assert((ITEMS * sizeof(K)) % 16 == 0, "whole 16-byte loads");
+  constexpr int kVec = (int)(ITEMS * sizeof(K) / 16);
+  const uint32_t first = p * (uint32_t)TILE + (uint32_t)tid * ITEMS;
   K key[ITEMS];
+  if (first + ITEMS <= n) {
+    uint4 v[kVec];
+    const uint4* src = reinterpret_cast<const uint4*>(keys + first);
 #pragma unroll
-  for (int it = 0; it < ITEMS; ++it) {
-    const uint32_t idx = first + it * 32;
-    key[it] = idx < n ? keys[idx] : (K)0;
+    for (int q = 0; q < kVec; ++q) v[q] = src[q];
+    memcpy(key, v, sizeof(key));
+  } else {
+#pragma unroll
+    for (int it = 0; it < ITEMS; ++it) key[it] = first + it < n ? keys[first + it] : (K)0;
   }
   __syncthreads();
 #pragma unroll
   for (int it = 0; it < ITEMS; ++it) {
-    const uint32_t idx = first + it * 32;
-    if (idx < n) atomicAdd(&s_h[warp][(uint32_t)(key[it] >> shift) & M], 1u);
+    if (first + it < n) atomicAdd(&s_h[warp][(uint32_t)(key[it] >> shift) & M], 1u);
   }
   __syncthreads();
   for (int d = tid; d < R; d += kSortThreads) {
@@ -1146,6 +1171,15 @@ __device__ __forceinline__ uint32_t warp_peers(uint32_t d) {
 template <typename K, int ITEMS>
 struct ScatterOcc {
   static constexpr int kBlocks = 3;
+};
+// Narrow keys (the rows of the column path) hold few registers: four blocks.
+template <int ITEMS>
+struct ScatterOcc<uint8_t, ITEMS> {
+  static constexpr int kBlocks = 4;
+};
+template <int ITEMS>
+struct ScatterOcc<uint16_t, ITEMS> {
+  static constexpr int kBlocks = 4;
 };
 
 template <typename K, int BITS, int ITEMS>
@@ -1574,7 +1608,7 @@ cudaError_t run_radix_passes(K* keys_a, uint32_t* vals_a, K* keys_b, uint32_t* v
     const int sh = plan.shift[p];
     K* kout_p = (p + 1 == plan.passes && !last_keys) ? nullptr : kout;
     cudaError_t e = cudaErrorInvalidValue;
-    if constexpr (sizeof(K) == 4) {
+    if constexpr (sizeof(K) <= 4) {
       switch (plan.bits[p]) {
         case 4: e = radix_pass<K, 4, ITEMS>(kin, vin, kout_p, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream); break;
         case 5: e = radix_pass<K, 5, ITEMS>(kin, vin, kout_p, vout, n_ptr, capacity, parts, sh, counts, stride, totals, status, stream); break;
@@ -1694,12 +1728,38 @@ int tile_gsize(int64_t n) {
 // passes over their evenly split digits. (Single-sweep passes were measured
 // slower on these keys: a 4K view's one 8-bit row pass over 849M pairs took
 // the whole binning from 11.9 to 13.0 ms.)
-cudaError_t sort_pairs32(const BinSortArgs& a, cudaStream_t stream) {
-  return run_radix_passes<uint32_t, kSortItems>(
-      reinterpret_cast<uint32_t*>(a.keys[a.emit_buf]), a.vals[a.emit_buf],
-      reinterpret_cast<uint32_t*>(a.keys[a.emit_buf ^ 1]), a.vals[a.emit_buf ^ 1], a.n_pairs,
+template <typename KT>
+cudaError_t sort_pairs(const BinSortArgs& a, cudaStream_t stream) {
+  return run_radix_passes<KT, kSortItems>(
+      reinterpret_cast<KT*>(a.keys[a.emit_buf]), a.vals[a.emit_buf],
+      reinterpret_cast<KT*>(a.keys[a.emit_buf ^ 1]), a.vals[a.emit_buf ^ 1], a.n_pairs,
       a.capacity, a.capacity, a.pairs, a.counts, a.counts_stride, a.totals, a.status, stream,
       !a.count_ranges);
+}
+
+// The column path from the emission on, with KT keys: emission, the rows
+// passes, the ranges off the keys unless they came from the counts.
+template <typename KT>
+cudaError_t emit_and_sort_columns(const BinSortArgs& a, int64_t n_items, int64_t cb, int sms,
+                                  cudaStream_t stream) {
+  const dim3 grid((unsigned)cb, (unsigned)((a.grid.tiles_x + 31) / 32));
+  k_emit_cols<KT><<<grid, 32, 0, stream>>>(
+      a.crect, n_items, a.grid, a.cbits, a.counts, a.counts_stride, a.totals, a.pair_total,
+      reinterpret_cast<KT*>(a.keys[a.emit_buf]), a.vals[a.emit_buf], a.capacity, a.n_pairs,
+      a.status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // 3) stable sort by row
+  if ((e = sort_pairs<KT>(a, stream)) != cudaSuccess) return e;
+  if (a.count_ranges) return cudaSuccess;
+  if constexpr (sizeof(KT) == 4) {
+    const int out = a.emit_buf ^ (a.pairs.passes & 1);
+    k_ranges<uint32_t><<<sms * 4, 256, 0, stream>>>(
+        reinterpret_cast<uint32_t*>(a.keys[out]), a.n_pairs, a.capacity, a.n_tiles, a.cbits,
+        (uint32_t)a.grid.tiles_x, a.ranges, a.status);
+    return cudaGetLastError();
+  }
+  return cudaErrorInvalidValue;  // narrow keys carry no column: ranges come from the counts
 }
 
 cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
@@ -1778,21 +1838,10 @@ cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
       }
       k_radix_scan<<<(unsigned)a.grid.tiles_x, 256, 0, stream>>>(
           a.counts, a.counts_stride, a.n_items_dev, n_items, kColItems, a.totals);
-      const dim3 grid((unsigned)cb, (unsigned)((a.grid.tiles_x + 31) / 32));
-      k_emit_cols<<<grid, 32, 0, stream>>>(
-          a.crect, n_items, a.grid, a.cbits, a.counts, a.counts_stride, a.totals, a.pair_total,
-          reinterpret_cast<uint32_t*>(a.keys[a.emit_buf]), a.vals[a.emit_buf], a.capacity,
-          a.n_pairs, a.status);
-      if ((e = cudaGetLastError()) != cudaSuccess) return e;
-      // 3) stable sort by row
-      e = sort_pairs32(a, stream);
-      if (e != cudaSuccess) return e;
-      if (a.count_ranges) return cudaSuccess;
-      const int out = a.emit_buf ^ (a.pairs.passes & 1);
-      k_ranges<uint32_t><<<sms * 4, 256, 0, stream>>>(
-          reinterpret_cast<uint32_t*>(a.keys[out]), a.n_pairs, a.capacity, a.n_tiles, a.cbits,
-          (uint32_t)a.grid.tiles_x, a.ranges, a.status);
-      return cudaGetLastError();
+      if (a.row_key_bytes == 1) return emit_and_sort_columns<uint8_t>(a, n_items, cb, sms, stream);
+      if (a.row_key_bytes == 2)
+        return emit_and_sort_columns<uint16_t>(a, n_items, cb, sms, stream);
+      return emit_and_sort_columns<uint32_t>(a, n_items, cb, sms, stream);
     }
     // 2) emission in depth order, 32-bit tile keys
     k_emit<1, uint32_t><<<(unsigned)eb, kEmitThreads, 0, stream>>>(
@@ -1801,7 +1850,7 @@ cudaError_t launch_bin_sort(const BinSortArgs& a, cudaStream_t stream) {
         a.n_pairs, a.emit_lookback, a.counters + 0, a.status, a.wait);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // 3) stable sort by tile
-    e = sort_pairs32(a, stream);
+    e = sort_pairs<uint32_t>(a, stream);
     if (e != cudaSuccess) return e;
     const int out = a.emit_buf ^ (a.pairs.passes & 1);
     k_ranges<uint32_t><<<sms * 4, 256, 0, stream>>>(reinterpret_cast<uint32_t*>(a.keys[out]),

@@ -43,6 +43,7 @@ struct Layout {
   int gsize = 0, tile_bpv = 0;
   bool column_emit = false;
   bool count_ranges = false;
+  int row_key_bytes = 4;
   int cbits = 0;
   int key_bytes = 8;
   int64_t counts_stride = 0;
@@ -93,8 +94,15 @@ bool make_layout(int64_t n, int32_t n_views, const gs_camera* cams, int64_t capa
       L.cbits = bits_for((uint64_t)g.tiles_x - 1);
       if (L.cbits == 0) L.cbits = 1;
       L.count_ranges = count_ranges_fit(g);
-      L.pairs = make_radix_plan(bits_for((uint64_t)g.tiles_y * n_views - 1), true);
-      for (int i = 0; i < L.pairs.passes; ++i) L.pairs.shift[i] += L.cbits;
+      const uint64_t rows = (uint64_t)g.tiles_y * n_views;
+      L.pairs = make_radix_plan(bits_for(rows - 1), true);
+      if (L.count_ranges && rows <= 65536) {
+        // the ranges come from the tile counts: the keys are the rows alone
+        L.row_key_bytes = rows <= 256 ? 1 : 2;
+        L.key_bytes = L.row_key_bytes;
+      } else {
+        for (int i = 0; i < L.pairs.passes; ++i) L.pairs.shift[i] += L.cbits;
+      }
     } else {
       L.pairs = make_radix_plan(tile_bits, true);
     }
@@ -292,6 +300,7 @@ gs_status gs_bin_sort(const gs_projected* proj, const gs_camera* cams, int32_t n
   a.column_emit = L.column_emit;
   a.cbits = L.cbits;
   a.count_ranges = L.count_ranges;
+  a.row_key_bytes = L.row_key_bytes;
   if (L.count_ranges) {
     a.tile_diff = reinterpret_cast<int*>(w + L.off_tdiff);
     a.view_pairs = reinterpret_cast<unsigned long long*>(w + L.off_view_pairs);
@@ -729,6 +738,8 @@ gs_status gs_bin_sort_plan(int64_t n, int32_t n_views, const gs_camera* cams,
   plan->gaussians_per_block = L.tile_emit ? L.gsize : 0;
   plan->pair_single_sweep = pair_passes_single_sweep(L.pairs, sort_mode) ? 1 : 0;
   plan->ranges_from_counts = L.count_ranges ? 1 : 0;
+  plan->pair_key_bytes = L.tile_emit ? 0 : L.key_bytes;
+  plan->reserved = 0;
   plan->blocks_per_view = L.tile_emit ? L.tile_bpv : 0;
   return GS_OK;
 }

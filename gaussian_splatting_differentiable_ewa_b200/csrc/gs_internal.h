@@ -62,6 +62,7 @@ struct BinSortArgs {
   uint32_t* tile_base;               // tile emission: first position of each tile [n_tiles]
   int64_t* scan_n;                   // tile emission: blocks per view, for the scan
   bool count_ranges;                 // column emission: ranges from the tile counts
+  int row_key_bytes;                 // column emission: 1, 2 (rows alone) or 4 bytes per key
   int* tile_diff;                    // count_ranges: [n_views][tiles_y + 1][tiles_x + 1]
   unsigned long long* view_pairs;    // count_ranges: pairs per view [GS_MAX_VIEWS]
   int64_t* ranges;

@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define GS_ABI_VERSION 3
+#define GS_ABI_VERSION 4
 #define GS_TILE 16            /* tile edge in pixels */
 #define GS_MAX_VIEWS 32       /* views per call */
 #define GS_RECORD_FLOATS 16   /* floats per projected record */
@@ -230,6 +230,12 @@ size_t gs_workspace_size(int64_t n, int32_t n_views, const gs_camera* cams,
  *                    sorted keys, whose last pass then writes no keys:
  *                    GS_PATH_COLUMNS and full-64 mode on grids whose
  *                    (tiles_x + 1) (tiles_y + 1) counters fit 160 KiB;
+ *   pair_key_bytes   bytes per pair key: 8 in full-64 mode, 4 on
+ *                    GS_PATH_TILE_ID and on GS_PATH_COLUMNS when the ranges
+ *                    are read off the keys (row << column bits | column);
+ *                    on GS_PATH_COLUMNS with ranges_from_counts the keys are
+ *                    the rows alone: 1 byte up to 256 rows (views x tile
+ *                    rows), 2 up to 65536; 0 on GS_PATH_TILES (no keys);
  *   gaussians_per_block, blocks_per_view  the Gaussian blocks of
  *                    GS_PATH_TILES (0 otherwise).
  * Returns GS_ERR_INVALID_ARG for a request gs_workspace_size rejects. */
@@ -242,6 +248,8 @@ typedef struct gs_sort_plan {
   int32_t pair_single_sweep;
   int32_t ranges_from_counts;
   int64_t blocks_per_view;
+  int32_t pair_key_bytes;
+  int32_t reserved;
 } gs_sort_plan;
 gs_status gs_bin_sort_plan(int64_t n, int32_t n_views, const gs_camera* cams,
                            int32_t sort_mode, gs_sort_plan* plan);

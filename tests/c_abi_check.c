@@ -37,6 +37,22 @@ int main(void) {
   CHECK(gs_workspace_size(-1, 1, &cam, 10, GS_SORT_FULL64) == 0);
   CHECK(gs_workspace_size(10, 0, &cam, 10, GS_SORT_FULL64) == 0);
 
+  /* the sort plan of a 3840 x 2160 view: pairs by tile column, ranges from
+   * the tile counts, the 135 rows as one-byte keys */
+  {
+    gs_camera c4 = cam;
+    c4.width = 3840;
+    c4.height = 2160;
+    gs_sort_plan pl;
+    memset(&pl, 0xff, sizeof pl);
+    CHECK(sizeof(gs_sort_plan) == 40);
+    CHECK(gs_bin_sort_plan(1000, 1, &c4, GS_SORT_PRESORT, &pl) == GS_OK);
+    CHECK(pl.path == GS_PATH_COLUMNS && pl.ranges_from_counts == 1 && pl.pair_key_bytes == 1);
+    CHECK(pl.pair_passes == 1 && pl.reserved == 0);
+    CHECK(gs_bin_sort_plan(1000, 1, &c4, GS_SORT_FULL64, &pl) == GS_OK);
+    CHECK(pl.pair_key_bytes == 8 && pl.ranges_from_counts == 1);
+  }
+
   gs_params p;
   memset(&p, 0, sizeof p);
   p.n = 10;

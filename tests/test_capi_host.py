@@ -31,7 +31,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_status_strings():
-    assert api.gs_abi_version() == 3
+    assert api.gs_abi_version() == 4
     for s in range(7):
         assert api.status_string(s) not in ("", "unknown status")
 
@@ -220,6 +220,10 @@ def test_sort_plan_follows_the_grid_and_mode():
     assert (p.path, p.pair_passes) == (api.GS_PATH_COLUMNS, 1)
     assert p.pair_single_sweep == 0                                 # 32-bit row keys
     assert p.ranges_from_counts == 1                                # 241 x 136 ints fit
+    assert p.pair_key_bytes == 1                                    # 135 rows: the row alone
+    p = plan(3840, 2160, 1000, 2, api.GS_SORT_PRESORT)            # 270 rows: two bytes
+    assert (p.pair_key_bytes, p.pair_passes, p.ranges_from_counts) == (2, 2, 1)
+    assert ctypes.sizeof(api.GsSortPlan) == 40
     p = plan(128, 128, 1000, 1, api.GS_SORT_PRESORT)               # small scene: 32 per block
     assert (p.path, p.gaussians_per_block, p.blocks_per_view) == (api.GS_PATH_TILES, 32, 32)
     p = plan(800, 800, 100_000, 1, api.GS_SORT_PRESORT)
@@ -227,6 +231,7 @@ def test_sort_plan_follows_the_grid_and_mode():
     p = plan(4096, 2576, 1000, 1, api.GS_SORT_PRESORT)            # 256 x 161 tiles
     assert (p.path, p.pair_passes) == (api.GS_PATH_COLUMNS, 1)
     assert p.ranges_from_counts == 0                                # 257 x 162 ints do not
+    assert p.pair_key_bytes == 4                                    # row << 8 | column
     p = plan(8192, 1296, 1000, 1, api.GS_SORT_PRESORT)            # 512 x 81 tiles
     assert (p.path, p.pair_passes) == (api.GS_PATH_TILE_ID, 2)
     assert p.pair_single_sweep == 0
@@ -250,7 +255,7 @@ def test_bench_work_model_uses_the_library_plan():
     sp = types.SimpleNamespace(n=1_000_000, V=1, W=1920, H=1080, cams=cams)
     plan = bench.sort_plan(sp, "presort")
     assert plan == dict(path="tiles", pre=4, pair=0, bpv=1303, tiles=8160, pair_sweep=False,
-                        count_ranges=False)
+                        count_ranges=False, key_bytes=0)
     # project; depth keys, digit counts, 4 single-sweep passes, count, scan, base,
     # place; raster fwd, raster bwd, project bwd, densify stats, Adam
     assert bench.launches_per_step(sp, "presort") == 1 + (1 + 1 + 4 + 4) + 5

@@ -116,15 +116,18 @@ def test_binning_bit_exact(name, kw, how, mode):
 
 @pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("W,H", [(200, 136), (4300, 40), (4096, 2576), (8192, 1296),
-                                 (4096, 1600), (8192, 640)])
+                                 (4096, 1600), (8192, 640), (3840, 2160)])
 def test_binning_isolated_with_ties_and_ragged_tail(mode, W, H):
     # screen-space inputs straight from the generator: many equal depth keys
     # (ties broken by index), culled entries, rectangles clipped by the image.
     # Grids in presort mode: 13 x 9 and 269 x 3 tiles place pairs straight at
-    # their positions; 256 x 161 (too many tiles for that) emits by column;
-    # 512 x 81 (too wide for columns too) emits by tile id. With two views,
-    # 256 x 100 sorts its 200 rows in one 8-bit pass and 512 x 40 its 40960
-    # tile ids in two; the others split their digits evenly.
+    # their positions; 256 x 161 (too many tiles for that) emits by column
+    # with row << 8 | column keys and reads the ranges off them (its tile
+    # counters do not fit a block); 512 x 81 (too wide for columns too) emits
+    # by tile id. With two views, 256 x 100 sorts its 200 rows as one-byte
+    # keys in one 8-bit pass, 240 x 135 its 270 rows as two-byte keys in two
+    # passes (5 + 4 bits), both with ranges from the tile counts, and 512 x 40
+    # its 40960 tile ids in two; the others split their digits evenly.
     n, V = 3000, 2
     d = S.make_projected_2d(n, W, H, seed=3, n_views=V)
     tx, ty = (W + 15) // 16, (H + 15) // 16
