@@ -285,4 +285,16 @@ def test_bench_work_model_uses_the_library_plan():
     # without the examined count every pair is charged (the scope table's ceiling)
     w0 = bench.algorithmic_work(sp, 26_000_000, "presort", 1.0e8)
     assert w0["gs_rasterize_fwd"]["bytes"] == 26_000_000 * 44 + P * 20
+    # full-64 mode, ranges from the tile counts: per pair 12 B emitted, 24 B a pass,
+    # 8 B of digit counts, the last pass's 8 B of keys not written; per Gaussian
+    # and view 24 B read for the keys and 16 B for the tile histogram
+    wf = bench.algorithmic_work(sp, 26_000_000, "full64", 0.0)
+    assert wf["gs_bin_sort"]["bytes"] == 26_000_000 * (12 + 6 * 24 + 8 - 8) + 1_000_000 * 40
+    # the 4K column path: one-byte row keys emitted with the ids, one rows pass
+    # (read and written), the last write without keys; per Gaussian the depth
+    # keys' 4 passes and the rectangles read for the histogram
+    sp4.K = 16
+    w4 = bench.algorithmic_work(sp4, 849_000_000, "presort", 0.0)
+    assert w4["gs_bin_sort"]["bytes"] == (849_000_000 * ((1 + 4) + 2 * (1 + 4) - 1)
+                                          + 10_000_000 * (16 + 8 + 4 * 24 + 12 + 16))
     assert bench.alu_peak_gops(1965.0) == pytest.approx(148 * 128 * 1.965)
