@@ -23,8 +23,16 @@
 //                  ordered by tile column: per-block column counts from a
 //                  difference array, their scan, then lanes owning columns
 //                  append their pairs in depth order through shared-memory
-//                  buffers written out warp-wide. Keys are row << cbits |
-//                  column; the radix passes then sort by row alone.
+//                  buffers written out warp-wide. The radix passes then sort
+//                  by row alone; the keys are the row in one or two bytes
+//                  when the ranges come from the tile counts, else
+//                  row << cbits | column.
+//  k_tile_hist / k_tile_ranges
+//                  (column path and full-64 mode, grids whose per-view tile
+//                  counters fit a block) every tile's pair count from a
+//                  per-view 2-D difference array of the rectangles' corners,
+//                  and a scan of the counts per view: the ranges before the
+//                  pairs exist, so nothing reads the sorted keys.
 //  k_digit_hist / k_onesweep
 //                  the 64-bit sorts (depth presort; full-64 pair keys): a
 //                  stable least-significant-digit radix sort with 8-bit
@@ -35,15 +43,16 @@
 //                  offsets by decoupled look-back over the partitions before
 //                  them, one thread per digit.
 //  k_radix_count / k_radix_scan / k_radix_scatter
-//                  the 32-bit sorts (row or tile bits after column or
-//                  tile-id emission), reduce-then-scan: per-partition digit
+//                  the 8-, 16- and 32-bit sorts (row or tile bits after
+//                  column or tile-id emission), reduce-then-scan: per-partition digit
 //                  counts, a per-digit scan over partitions (with the digit
 //                  totals), then a scatter that ranks each partition's keys
 //                  stably (ballots over warp-striped steps), stages them in
 //                  shared memory and writes runs of equal digits. The bits
 //                  are split evenly over the fewest passes (13 bits: 7 + 6),
 //                  so each key costs one ballot per bit of its pass.
-//  k_ranges        [start, end) of each tile in the sorted pairs.
+//  k_ranges        [start, end) of each tile in the sorted pairs (where the
+//                  tile counts do not give them).
 // Look-back waits (emission and single-sweep passes) are bounded in time
 // (WaitCfg) and report through the status word instead of hanging; the
 // reduce-then-scan passes never wait on other blocks.
